@@ -1,0 +1,240 @@
+/*
+ * lowram.h — C ABI of a B200 (sm_100a) library for decode-time attention over a
+ * LowRAM-compressed KV cache.
+ *
+ * What the library computes (one "unit" = one sequence b, one layer l, one KV head):
+ *
+ *   1. Chunk scoring.  The N prefill tokens of a unit are split into chunks of C tokens.
+ *      Each live chunk c is scored against the step's queries:
+ *          s_c = sum_{j in group} q_j . kbar_{l,c} / sqrt(d_h),  kbar_{l,c} = abar_c . B_l
+ *      where abar_c is the chunk's mean coefficient row (the chunk key summary).
+ *      Sources: "LowRAM: Low-Rank Keys and Amortised Values for Composable KV Cache
+ *      Compression at Test-Time" (arXiv 2611.07025 abstract: only a selected subset of KV
+ *      pairs is reconstructed per step); rit.work "lowram-kv-cache-compression", section
+ *      "Значения предсказывают, ключи раскладывают по общему базису" (the context is split
+ *      into fragments and the ones that fit the current query are chosen).  The pages do not
+ *      define the summary or the score; the mean-key reading is this library's.
+ *   2. Top-k selection of the k highest-scoring live chunks (ties go to the lower chunk id).
+ *   3. Key rebuild from the cross-layer low-rank form, for the selected chunks only:
+ *          khat_t = sigma_t * a_t . B_l
+ *      a_t is the token's coefficient row, shared by the G layers of a layer group; B_l is the
+ *      layer's slice of the group basis ("LowRAM Compresses KV Cache Asymmetrically",
+ *      section "Cross-Layer Low-Rank Key Compression"; rit.work post: keys via xKV with a
+ *      common basis for adjacent layers).  sigma_t is the per-token int8 scale, else 1.
+ *   4. Value rebuild with the per-head predictor and the stored residuals:
+ *          vhat_t = W2 . silu(W1 . khat_t) (+ rho_t * delta_t if token t is flagged)
+ *      ("LowRAM Compresses KV Cache Asymmetrically", section "Core Mechanism: Predict
+ *      Values and Keep Difficult Residuals": Vhat = f(K), delta = V - Vhat kept for the
+ *      worst-predicted tokens).  rho_t is the residual's int8 scale, else 1.
+ *   5. GQA attention of each query head j of the unit over the rebuilt tokens of the
+ *      selected chunks plus the uncompressed tail of tokens generated after prefill:
+ *          o_j = softmax_t(q_j . k_t / sqrt(d_h)) . v_t
+ *      ("OjaKV", section 3 "预备知识：低秩注意力", the attention equations; the raw tail:
+ *      rit.work post, same section as in step 1).
+ *
+ * Layouts: all arrays are row-major, last index contiguous.  Symbols: B batch, L layers,
+ * G layers per group, Hkv KV heads, Hq query heads (g = Hq/Hkv per KV head), d head dim,
+ * r rank, h predictor hidden width, N compressed tokens, C chunk size, nC = N/C chunks,
+ * nL live chunks per (b, group, KV head) (nL = nC without eviction), T tail capacity.
+ * Query head j belongs to KV head j / g.
+ *
+ * Error behaviour: every entry point returns a lowram_status.  Argument and shape checks
+ * run on the host before anything is launched and return LOWRAM_EINVAL with no side
+ * effect.  A CUDA error becomes LOWRAM_ECUDA; lowram_last_error_string() gives the CUDA
+ * runtime's text for the calling thread.  Kernels never trap: a device-side check that
+ * fails records an error word that lowram_cache_validate() turns into LOWRAM_ECORRUPT.
+ */
+#ifndef LOWRAM_H
+#define LOWRAM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* lowram_stream; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  LOWRAM_OK = 0,
+  LOWRAM_EINVAL = 1,        /* bad argument, shape or pointer; nothing was launched */
+  LOWRAM_ENOMEM = 2,        /* a device allocation failed (create only) */
+  LOWRAM_ECUDA = 3,         /* a CUDA runtime call or launch failed */
+  LOWRAM_EUNSUPPORTED = 4,  /* the shapes are valid but no kernel in this build handles them */
+  LOWRAM_ECORRUPT = 5,      /* lowram_cache_validate found an inconsistent index table */
+  LOWRAM_ETIMEOUT = 6       /* a kernel gave up a bounded wait and returned early */
+} lowram_status;
+
+typedef enum {
+  LOWRAM_F32 = 0,  /* fp32 storage and fp32 arithmetic everywhere */
+  LOWRAM_BF16 = 1  /* bf16 storage; tensor-core products with fp32 accumulation */
+} lowram_dtype;
+
+typedef enum {
+  LOWRAM_STORE_NATIVE = 0, /* coefficients and residuals stored in the config dtype */
+  LOWRAM_STORE_INT8 = 1    /* int8 coefficients and residuals with one fp16 scale per row
+                              ("LowRAM Compresses KV Cache Asymmetrically", section
+                              "Composition with Quantization and Eviction").  Needs BF16. */
+} lowram_store;
+
+/* Shapes of one compressed cache.  Constraints checked by lowram_cache_create:
+ * n_layers % group == 0, n_q_heads % n_kv_heads == 0, n_ctx % chunk == 0,
+ * 1 <= top_k <= n_live <= n_ctx/chunk, rank <= group*head_dim, chunk <= 32767,
+ * n_q_heads/n_kv_heads <= 16, head_dim <= 256, rank <= 512, mlp_hidden <= 1024,
+ * n_ctx/chunk <= 8192, tail_cap <= 4096. */
+typedef struct {
+  int32_t batch;       /* B */
+  int32_t n_layers;    /* L */
+  int32_t group;       /* G: layers sharing one coefficient matrix */
+  int32_t n_kv_heads;  /* Hkv */
+  int32_t n_q_heads;   /* Hq */
+  int32_t head_dim;    /* d */
+  int32_t rank;        /* r */
+  int32_t mlp_hidden;  /* h */
+  int32_t n_ctx;       /* N compressed (prefill) tokens per sequence */
+  int32_t chunk;       /* C */
+  int32_t top_k;       /* k chunks selected per unit and step */
+  int32_t tail_cap;    /* T: capacity of the raw tail per (b, l, KV head) */
+  int32_t n_live;      /* nL: live chunks per (b, group, KV head) */
+  int32_t dtype;       /* lowram_dtype */
+  int32_t store;       /* lowram_store */
+} lowram_config;
+
+/* Source arrays of a compressed cache, all DEVICE pointers, read by lowram_cache_create
+ * (which copies them; the caller keeps ownership and may free them once the create
+ * stream has reached the copy).  "dt" is fp32 (LOWRAM_F32) or bf16 (LOWRAM_BF16).
+ *
+ *   coeff      [B][L/G][Hkv][nL*C][r]  dt, or int8 with STORE_INT8.  Rows of live chunks
+ *                                      only, chunk after chunk in ascending chunk id.
+ *   coeff_scale[B][L/G][Hkv][nL*C]     fp16 per-row scale (STORE_INT8), else NULL.
+ *   basis      [L][Hkv][r][d]          dt.  B_l, the layer's slice of the group basis.
+ *   w1         [L][Hkv][h][d]          dt.  Predictor first layer (out x in), no bias.
+ *   w2         [L][Hkv][d][h]          dt.  Predictor second layer (out x in), no bias.
+ *   summary    [B][L/G][Hkv][nL][r]    dt (bf16 with STORE_INT8).  abar: the mean of the
+ *                                      chunk's (dequantised) coefficient rows.
+ *   slot       [B][L/G][Hkv][nC]       int16: storage slot of chunk c, or -1 if evicted.
+ *                                      NULL means no eviction (slot[c] = c, nL = nC).
+ *                                      Live slots are 0..nL-1 in ascending chunk id.
+ *   res_ptr    [B][L][Hkv][nL+1]       int32 global record offsets: records of slot s of a
+ *                                      unit are [res_ptr[s], res_ptr[s+1]).  Non-decreasing.
+ *   res_pos    [R]                     uint16 token offset of the record inside its chunk,
+ *                                      strictly increasing within a chunk, < C.
+ *   res_val    [R][d]                  dt, or int8 with STORE_INT8.  delta rows.
+ *   res_scale  [R]                     fp16 per-record scale (STORE_INT8), else NULL.
+ *   tail_k     [B][L][Hkv][T][d]       dt (bf16 with STORE_INT8).  Raw tail keys.
+ *   tail_v     [B][L][Hkv][T][d]       dt (bf16 with STORE_INT8).  Raw tail values.
+ *   tail_len   [B]                     int32, 0 <= tail_len[b] <= T.
+ * Every pointer must be 16-byte aligned. */
+typedef struct {
+  const void* coeff;
+  const void* coeff_scale;
+  const void* basis;
+  const void* w1;
+  const void* w2;
+  const void* summary;
+  const int16_t* slot;
+  const int32_t* res_ptr;
+  const uint16_t* res_pos;
+  const void* res_val;
+  const void* res_scale;
+  const void* tail_k;
+  const void* tail_v;
+  const int32_t* tail_len;
+  int64_t n_records; /* R: total residual records (length of res_pos/res_val/res_scale) */
+} lowram_cache_src;
+
+typedef struct lowram_cache lowram_cache; /* opaque; owns its device memory */
+
+/* Byte accounting of a cache (host only). */
+typedef struct {
+  uint64_t coeff;       /* coefficient rows (+ their scales) */
+  uint64_t basis;       /* per-layer bases */
+  uint64_t predictor;   /* W1 and W2 */
+  uint64_t summary;     /* chunk key summaries */
+  uint64_t residual;    /* residual rows, positions, scales and CSR offsets */
+  uint64_t index;       /* eviction slot map */
+  uint64_t tail;        /* raw tail keys and values (+ lengths) */
+  uint64_t total;       /* sum of the above: the compressed cache */
+  uint64_t dense_equiv; /* M_KV * B for the same N (at 2 bytes per scalar for BF16 and
+                           int8 stores, 4 for F32) plus the same raw tail */
+} lowram_bytes;
+
+/* Execution path chosen by lowram_decode_attn. */
+typedef enum {
+  LOWRAM_PATH_AUTO = 0,  /* tensor-core path when the shapes allow it, else CUDA cores */
+  LOWRAM_PATH_SIMT = 1,  /* CUDA-core path (any shapes; the only path for LOWRAM_F32) */
+  LOWRAM_PATH_TC = 2     /* tcgen05 tensor-core path; LOWRAM_EUNSUPPORTED if shapes don't fit */
+} lowram_path;
+
+/* Dense KV-cache bytes M_KV * B = 2 * L * Hkv * d * N * s * B ("LowRAM Compresses KV Cache
+ * Asymmetrically", section "Core Mechanism", the M_KV formula).  Host only; returns 0 if an
+ * argument is negative. */
+uint64_t lowram_dense_kv_bytes(int32_t n_layers, int32_t n_kv_heads, int32_t head_dim,
+                               int64_t n_ctx, int32_t bytes_per_scalar, int32_t batch);
+
+/* Copy a compressed cache into memory the cache object owns, derive the folded predictor
+ * weights W1' = W1 . B_l^T per (layer, KV head) (an exact rewrite: W1 . khat = W1' . a), and
+ * allocate the per-call scratch for up to cfg->batch sequences and all layers.
+ * Stream-ordered on `stream`; the object is usable on that stream immediately.
+ * Returns EINVAL for bad shapes or NULL/unaligned pointers, ENOMEM if allocation fails. */
+lowram_status lowram_cache_create(const lowram_config* cfg, const lowram_cache_src* src,
+                                  lowram_cache** out, lowram_stream stream);
+
+/* Free everything the cache owns (synchronises the device first).  NULL is a no-op. */
+void lowram_cache_destroy(lowram_cache* cache);
+
+/* Decode-time attention for layers [layer0, layer0 + n_layers) of every sequence.
+ *   q   [n_layers][B][Hq][d]  dt, DEVICE.  One decode query per sequence per layer.
+ *   out [n_layers][B][Hq][d]  dt, DEVICE.  o_j of step 5.
+ *   sel [n_layers][B][Hkv][k] int32, DEVICE, may be NULL: the selected chunk ids of each
+ *                             unit in ascending order.
+ * Runs steps 1-5 on `stream`: no host synchronisation and no allocation.  One cache must
+ * not be used by two streams at the same time (the scratch is shared).  Returns EINVAL
+ * for a bad layer range or NULL q/out, EUNSUPPORTED if `path` cannot serve the shapes. */
+lowram_status lowram_decode_attn(lowram_cache* cache, int32_t layer0, int32_t n_layers,
+                                 const void* q, void* out, int32_t* sel, int32_t path,
+                                 lowram_stream stream);
+
+/* Steps 1-2 alone: chunk scores and the top-k selection.
+ *   scores [n_layers][B][Hkv][nC] fp32, DEVICE, may be NULL: s_c, -inf for evicted chunks.
+ *   sel    [n_layers][B][Hkv][k]  int32, DEVICE, may be NULL (ids ascending). */
+lowram_status lowram_select_chunks(lowram_cache* cache, int32_t layer0, int32_t n_layers,
+                                   const void* q, float* scores, int32_t* sel,
+                                   lowram_stream stream);
+
+/* Same as lowram_decode_attn with HOST buffers q_host/out_host/sel_host (sel may be NULL):
+ * copies q to the device, decodes, copies the results back and synchronises `stream`.
+ * Pinned host memory makes the copies asynchronous; pageable memory works too. */
+lowram_status lowram_decode_attn_host(lowram_cache* cache, int32_t layer0, int32_t n_layers,
+                                      const void* q_host, void* out_host, int32_t* sel_host,
+                                      lowram_stream stream);
+
+/* Byte accounting (host only, no device access). */
+lowram_status lowram_cache_bytes(const lowram_cache* cache, lowram_bytes* out);
+
+/* Device-side consistency check of the index tables (slot map, CSR offsets, record
+ * positions, tail lengths) and of the error word left by earlier kernels.  Synchronises
+ * `stream`.  Returns ECORRUPT if a table is inconsistent, ETIMEOUT if an earlier kernel
+ * reported a bounded wait that ran out, OK otherwise; the error word is cleared. */
+lowram_status lowram_cache_validate(lowram_cache* cache, lowram_stream stream);
+
+/* Optional timing hook: when events != NULL, lowram_decode_attn records events[0] before
+ * its first kernel, events[1] after steps 1-2 and the tail, events[2] after the chunk
+ * attention kernel and events[3] after the combine, all on the call's stream.  The events
+ * are cudaEvent_t handles owned by the caller; pass NULL to switch the hook off. */
+lowram_status lowram_cache_set_stage_events(lowram_cache* cache, void* const* events);
+
+/* Number of kernels the last lowram_decode_attn call on this cache launched. */
+int32_t lowram_cache_last_launches(const lowram_cache* cache);
+
+/* Which path the last lowram_decode_attn call on this cache ran (a lowram_path value). */
+int32_t lowram_cache_last_path(const lowram_cache* cache);
+
+const char* lowram_status_string(lowram_status status);
+const char* lowram_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LOWRAM_H */
