@@ -1,0 +1,398 @@
+"""Benchmark: decode-time attention over a LowRAM-compressed KV cache on B200.
+
+One step = one all-layer decode call (steps 1-5 for every layer and sequence) of the
+32K-context Llama-3.1-8B-shaped workload (batch 4, bf16), inputs resident in HBM.  The
+metric is queries/s, one query = one (sequence, layer) decode-attention evaluation over all
+32 query heads.  Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lowram|reference]
+                  [--config NAME] [--path auto|simt|tc] [--sweep]
+
+Multi-GPU: one process per GPU (torchrun); every rank holds its own replica of the
+workload (different seeds) and no collective runs on the data path ("weak" scaling);
+the reported time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import lowram_synth as S  # noqa: E402
+
+METRIC = "decode-attn queries/s over compressed KV at 32K ctx; achieved % of HBM roofline"
+DEFAULT_CONFIG = "llama8b_32k_bf16"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="lowram", choices=["lowram", "reference"])
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--sweep", action="store_true",
+                    help="also run the batch sweep 1,4,16,32,64 (extra JSON lines)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------------ environment
+
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except FileNotFoundError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.f.name)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        seen = set()
+        for _, _, flags in rows:
+            for n, v in zip(names, flags):
+                if v.lower() == "active":
+                    seen.add(n)
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1],
+                "reasons": sorted(seen), "samples": len(rows)}
+
+
+# ------------------------------------------------------------------- byte accounting
+
+def algorithmic_bytes(cfg, cache_host: dict, sel: np.ndarray, layer0: int, n_layers: int) -> dict:
+    """Bytes the method must move for one decode call, from the call's actual selection.
+
+    Per unit: the coefficient rows (+ int8 scales) of its selected chunks, the residual
+    records of those chunks (values, positions, int8 scales) and their CSR offsets, the raw
+    tail (actual lengths), q and out.  Once per (sequence, layer group, KV head): the chunk
+    summaries and the slot map; coefficient rows of a chunk selected by several layers of
+    one group are counted once.  Once per (layer, KV head): basis, folded W1' and W2.
+    """
+    B, Hkv, g, d, r, h = cfg.batch, cfg.n_kv_heads, cfg.q_per_kv, cfg.head_dim, cfg.rank, cfg.mlp_hidden
+    C, k, T = cfg.chunk, cfg.top_k, cfg.tail_cap
+    s = 4 if cfg.dtype == "f32" else 2
+    i8 = cfg.store == "int8"
+    sa = 1 if i8 else s
+    res_ptr = cache_host["res_ptr"]
+    slot = cache_host["slot"]
+    tail_len = cache_host["tail_len"]
+    coeff = 0
+    resid = 0
+    ptrs = 0
+    groups_seen = {}
+    for li in range(n_layers):
+        l = layer0 + li
+        grp = l // cfg.group
+        for b in range(B):
+            for hk in range(Hkv):
+                key = (b, grp, hk)
+                chosen = groups_seen.setdefault(key, set())
+                for c in sel[li, b, hk]:
+                    sl = int(slot[b, grp, hk, c])
+                    chosen.add(sl)
+                    n = int(res_ptr[b, l, hk, sl + 1] - res_ptr[b, l, hk, sl])
+                    resid += n * (d * sa + 2 + (2 if i8 else 0))
+                ptrs += (k + 1) * 4
+    for key, chosen in groups_seen.items():
+        coeff += len(chosen) * C * (r * sa + (2 if i8 else 0))
+    n_units = n_layers * B * Hkv
+    summaries = len(groups_seen) * cfg.n_live * r * s
+    slotmap = len(groups_seen) * cfg.n_chunks * 2 if cfg.n_live < cfg.n_chunks else 0
+    tail = sum(2 * int(tail_len[b]) * d * (2 if i8 else s) for b in range(B)) * n_layers * Hkv
+    qo = 2 * n_units * g * d * s
+    weights = n_layers * Hkv * (r * d * s + h * r * (2 if s == 2 else 4) + d * h * s)
+    w1f = n_layers * Hkv * h * r * (2 if s == 2 else 4)
+    total = coeff + resid + ptrs + summaries + slotmap + tail + qo + weights
+    attend = coeff + resid + ptrs + w1f
+    return {"total": total, "attend": attend, "coeff": coeff, "residual": resid,
+            "summary": summaries, "tail": tail, "weights": weights}
+
+
+# ---------------------------------------------------------------------- CPU oracle leg
+
+def oracle_rate(cfg, cache, q, budget_s: float = 15.0, seed: int = 0):
+    """Time the fp64 oracle on a bounded sample of units; returns (queries/s, sample desc,
+    threads used)."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = 1
+    npc = S.cache_to_numpy(cache)
+    oc = O.OracleCache(npc)
+    qf = q.detach().cpu().double().numpy()
+    rng = np.random.default_rng(seed)
+    units = [(li, b, h) for li in range(q.shape[0]) for b in range(cfg.batch)
+             for h in range(cfg.n_kv_heads)]
+    order = rng.permutation(len(units))
+    done = 0
+    t0 = time.perf_counter()
+    for i in order:
+        li, b, h = units[i]
+        O.decode_unit(oc, b, li, h, qf[li, b, h * cfg.q_per_kv:(h + 1) * cfg.q_per_kv])
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    queries = done / cfg.n_kv_heads
+    return queries / dt, f"{done} of {len(units)} units (seeded), {dt:.1f} s", threads
+
+
+# --------------------------------------------------------------------------- lowram
+
+def run_lowram(args, ws, rank, local):
+    import kv_cache_compression_lowram_b200 as K
+    cfg = S.CONFIGS[args.config]
+    if rank > 0:
+        cfg = cfg.replace(seed=cfg.seed + 7919 * rank)
+    dev = torch.device("cuda", local)
+    torch.manual_seed(0)
+    cache = S.make_cache(cfg, device=dev)
+    q = S.make_queries(cache)
+    lc = K.LowramCache.from_synth(cache)
+    path = {"auto": K.PATH_AUTO, "simt": K.PATH_SIMT, "tc": K.PATH_TC}[args.path]
+    out = torch.empty_like(q)
+    sel = torch.empty(cfg.n_layers, cfg.batch, cfg.n_kv_heads, cfg.top_k, dtype=torch.int32,
+                      device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        K.lowram_decode_attn(lc.handle, 0, cfg.n_layers, q, out, sel, path)
+    torch.cuda.synchronize()
+    launches_per_step = lc.last_launches
+    used_path = {1: "simt", 2: "tc"}.get(lc.last_path, "?")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(ws)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        K.lowram_cache_set_stage_events(lc.handle, evs[i])
+        K.lowram_decode_attn(lc.handle, 0, cfg.n_layers, q, out, sel, path)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop()
+    K.lowram_cache_set_stage_events(lc.handle, None)
+    ms_total = start.elapsed_time(end)
+    ms_total = max_over_ranks(ms_total, ws)
+    ms_step = ms_total / args.steps
+    stage_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(3)]
+
+    # end to end through the host entry point: pinned q in, pinned out back, every step
+    q_h = q.cpu().pin_memory()
+    out_h = torch.empty_like(q_h).pin_memory()
+    for _ in range(2):
+        K.lowram_decode_attn_host(lc.handle, 0, cfg.n_layers, q_h, out_h)
+    barrier(ws)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    e2e_steps = max(3, args.steps // 2)
+    for _ in range(e2e_steps):
+        K.lowram_decode_attn_host(lc.handle, 0, cfg.n_layers, q_h, out_h)
+    e2e_ms = (time.perf_counter() - t0) * 1e3 / e2e_steps
+    e2e_ms = max_over_ranks(e2e_ms, ws)
+
+    queries_step = cfg.batch * cfg.n_layers
+    value = queries_step * ws / (ms_step / 1e3)
+    host = {"res_ptr": cache.res_ptr.cpu().numpy(), "slot": cache.slot.cpu().numpy().astype(np.int64),
+            "tail_len": cache.tail_len.cpu().numpy()}
+    ab = algorithmic_bytes(cfg, host, sel.cpu().numpy(), 0, cfg.n_layers)
+    peak, peak_kind = peaks()
+    attend_ms = stage_ms[1]
+    achieved = ab["attend"] / (attend_ms / 1e3) / 1e9
+    call_gbs = ab["total"] / (ms_step / 1e3) / 1e9
+    qbytes = q.numel() * q.element_size()
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "queries/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": cfg.dtype if cfg.store == "native" else "int8+bf16",
+        "data": "synthetic (seeded generator; shapes of the named workload, no weights or datasets)",
+        "config": {"workload": cfg.name, "batch": cfg.batch, "n_layers": cfg.n_layers,
+                   "n_ctx": cfg.n_ctx, "chunk": cfg.chunk, "top_k": cfg.top_k, "rank": cfg.rank,
+                   "kv_heads": cfg.n_kv_heads, "q_heads": cfg.n_q_heads, "head_dim": cfg.head_dim,
+                   "mlp_hidden": cfg.mlp_hidden, "tail": cfg.tail_cap, "resid_frac": cfg.resid_frac,
+                   "store": cfg.store, "evict_frac": cfg.evict_frac, "path": used_path,
+                   "parallelism": f"replicas x{ws}",
+                   "l2": "inputs larger than L2 (%.2f GB of algorithmic bytes per step)" % (ab["total"] / 1e9)},
+        "roofline": {"bound": "hbm", "kernel": "attend_" + used_path,
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": ab["attend"],
+                     "launch_ms": round(attend_ms, 4)},
+        "call_roofline": {"algorithmic_bytes": ab["total"], "achieved_gbs": round(call_gbs, 1),
+                          "frac": round(call_gbs / peak, 4),
+                          "stage_ms": {"select_tail": round(stage_ms[0], 4),
+                                       "attend": round(stage_ms[1], 4),
+                                       "combine": round(stage_ms[2], 4)}},
+        "e2e": {"value": round(queries_step * ws / (e2e_ms / 1e3), 1), "unit": "queries/s",
+                "h2d_bytes_per_step": qbytes, "d2h_bytes_per_step": qbytes},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        rate, sample, threads = oracle_rate(cfg, cache, q)
+        line["cpu_baseline"] = {"value": round(rate, 3), "unit": "queries/s", "cores": threads,
+                                "kind": "oracle", "sample": sample}
+    lc.close()
+    return line
+
+
+def run_reference(args, ws, rank):
+    """The oracle (fp64 numpy, host cores) on the same workload, bounded samples per step."""
+    if rank != 0:
+        return None
+    cfg = S.CONFIGS[args.config]
+    cache = S.make_cache(cfg, device="cuda" if torch.cuda.is_available() else "cpu")
+    q = S.make_queries(cache)
+    budget = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_rate(cfg, cache, q, budget_s=budget)
+    rates = []
+    samples = []
+    threads = 1
+    for i in range(args.steps):
+        rate, sample, threads = oracle_rate(cfg, cache, q, budget_s=budget, seed=i + 1)
+        rates.append(rate)
+        samples.append(sample)
+    value = statistics.mean(rates)
+    ms_step = cfg.batch * cfg.n_layers / value * 1e3
+    return {
+        "metric": METRIC, "value": round(value, 3), "unit": "queries/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": cfg.name, "batch": cfg.batch, "n_layers": cfg.n_layers,
+                   "n_ctx": cfg.n_ctx},
+        "cpu_baseline": {"value": round(value, 3), "unit": "queries/s", "cores": threads,
+                         "kind": "oracle", "sample": samples[0] + f" per step, {args.steps} steps"},
+        "e2e": {"value": round(value, 3), "unit": "queries/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    ws, rank, local = dist_init()
+    if args.impl == "reference":
+        line = run_reference(args, ws, rank)
+    else:
+        line = run_lowram(args, ws, rank, local)
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+    if args.sweep and args.impl == "lowram":
+        for b in (1, 4, 16, 32, 64):
+            args.config = f"llama8b_32k_bf16_b{b}"
+            args.no_cpu_baseline = True
+            torch.cuda.empty_cache()
+            line = run_lowram(args, ws, rank, local)
+            if rank == 0:
+                print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -172,6 +172,12 @@ typedef enum {
 uint64_t lowram_dense_kv_bytes(int32_t n_layers, int32_t n_kv_heads, int32_t head_dim,
                                int64_t n_ctx, int32_t bytes_per_scalar, int32_t batch);
 
+/* Byte accounting of a cache with these shapes and n_records residual records, without
+ * creating it (host only; for capacity planning).  has_slot says whether an eviction slot
+ * map is stored (only when n_live < n_ctx/chunk).  Returns EINVAL for a bad config. */
+lowram_status lowram_config_bytes(const lowram_config* cfg, int64_t n_records, int32_t has_slot,
+                                  lowram_bytes* out);
+
 /* Copy a compressed cache into memory the cache object owns, derive the folded predictor
  * weights W1' = W1 . B_l^T per (layer, KV head) (an exact rewrite: W1 . khat = W1' . a), and
  * allocate the per-call scratch for up to cfg->batch sequences and all layers.
@@ -209,7 +215,7 @@ lowram_status lowram_decode_attn_host(lowram_cache* cache, int32_t layer0, int32
                                       const void* q_host, void* out_host, int32_t* sel_host,
                                       lowram_stream stream);
 
-/* Byte accounting (host only, no device access). */
+/* Byte accounting of a created cache (host only, no device access). */
 lowram_status lowram_cache_bytes(const lowram_cache* cache, lowram_bytes* out);
 
 /* Device-side consistency check of the index tables (slot map, CSR offsets, record

@@ -1,0 +1,317 @@
+"""Python binding of liblowram.so: decode-time attention over a LowRAM-compressed KV cache.
+
+This module only marshals arguments (torch tensors -> device pointers, config objects ->
+C structs) for the C ABI declared in ``include/lowram.h``; every step of the computation
+runs in the library's CUDA kernels.  The library must be built first
+(``python -m kv_cache_compression_lowram_b200.build``); if it is missing, every call raises.
+
+Entry points keep the C names: ``lowram_cache_create``, ``lowram_decode_attn``,
+``lowram_select_chunks``, ``lowram_decode_attn_host``, ``lowram_cache_bytes``,
+``lowram_config_bytes``, ``lowram_cache_validate``, ``lowram_cache_destroy``,
+``lowram_dense_kv_bytes``, ``lowram_cache_set_stage_events``,
+``lowram_cache_last_launches``, ``lowram_cache_last_path``.  ``LowramCache`` wraps a handle.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+__all__ = [
+    "LowramError", "LIB_PATH", "PATH_AUTO", "PATH_SIMT", "PATH_TC", "lib",
+    "lowram_dense_kv_bytes", "lowram_config_bytes", "lowram_cache_create",
+    "lowram_cache_destroy", "lowram_decode_attn", "lowram_select_chunks",
+    "lowram_decode_attn_host", "lowram_cache_bytes", "lowram_cache_validate",
+    "lowram_cache_set_stage_events", "lowram_cache_last_launches", "lowram_cache_last_path",
+    "LowramCache", "config_struct",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblowram.so")
+PATH_AUTO, PATH_SIMT, PATH_TC = 0, 1, 2
+STATUS = {0: "LOWRAM_OK", 1: "LOWRAM_EINVAL", 2: "LOWRAM_ENOMEM", 3: "LOWRAM_ECUDA",
+          4: "LOWRAM_EUNSUPPORTED", 5: "LOWRAM_ECORRUPT", 6: "LOWRAM_ETIMEOUT"}
+
+
+class LowramError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}: {detail}")
+        self.status = status
+
+
+class LowramConfigC(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "batch", "n_layers", "group", "n_kv_heads", "n_q_heads", "head_dim", "rank",
+        "mlp_hidden", "n_ctx", "chunk", "top_k", "tail_cap", "n_live", "dtype", "store")]
+
+
+class LowramSrcC(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "coeff", "coeff_scale", "basis", "w1", "w2", "summary", "slot", "res_ptr", "res_pos",
+        "res_val", "res_scale", "tail_k", "tail_v", "tail_len")] + [("n_records", ctypes.c_int64)]
+
+
+class LowramBytesC(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_uint64) for n in (
+        "coeff", "basis", "predictor", "summary", "residual", "index", "tail", "total",
+        "dense_equiv")]
+
+
+_LIB = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (raises if liblowram.so was not built)."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m kv_cache_compression_lowram_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, U64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64
+    sig = {
+        "lowram_dense_kv_bytes": (U64, [I32, I32, I32, I64, I32, I32]),
+        "lowram_config_bytes": (I32, [ctypes.POINTER(LowramConfigC), I64, I32,
+                                      ctypes.POINTER(LowramBytesC)]),
+        "lowram_cache_create": (I32, [ctypes.POINTER(LowramConfigC), ctypes.POINTER(LowramSrcC),
+                                      ctypes.POINTER(P), P]),
+        "lowram_cache_destroy": (None, [P]),
+        "lowram_decode_attn": (I32, [P, I32, I32, P, P, P, I32, P]),
+        "lowram_select_chunks": (I32, [P, I32, I32, P, P, P, P]),
+        "lowram_decode_attn_host": (I32, [P, I32, I32, P, P, P, P]),
+        "lowram_cache_bytes": (I32, [P, ctypes.POINTER(LowramBytesC)]),
+        "lowram_cache_validate": (I32, [P, P]),
+        "lowram_cache_set_stage_events": (I32, [P, P]),
+        "lowram_cache_last_launches": (I32, [P]),
+        "lowram_cache_last_path": (I32, [P]),
+        "lowram_status_string": (ctypes.c_char_p, [I32]),
+        "lowram_last_error_string": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _LIB = L
+    return L
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise LowramError(status, where, lib().lowram_last_error_string().decode())
+
+
+# --------------------------------------------------------------------------- marshalling
+
+def _get(cfg, name):
+    return cfg[name] if isinstance(cfg, dict) else getattr(cfg, name)
+
+
+def config_struct(cfg) -> LowramConfigC:
+    """C config from an object or dict with the ``lowram.h`` field names.
+
+    ``dtype`` may be "f32"/"bf16" or 0/1, ``store`` "native"/"int8" or 0/1.  ``n_live``
+    defaults to n_ctx // chunk (no eviction).
+    """
+    c = LowramConfigC()
+    for n in ("batch", "n_layers", "group", "n_kv_heads", "n_q_heads", "head_dim", "rank",
+              "mlp_hidden", "n_ctx", "chunk", "top_k", "tail_cap"):
+        setattr(c, n, int(_get(cfg, n)))
+    try:
+        n_live = int(_get(cfg, "n_live"))
+    except (AttributeError, KeyError):
+        n_live = c.n_ctx // c.chunk
+    c.n_live = n_live
+    dt = _get(cfg, "dtype")
+    c.dtype = {"f32": 0, "bf16": 1}.get(dt, dt) if isinstance(dt, str) else int(dt)
+    stv = _get(cfg, "store")
+    c.store = {"native": 0, "int8": 1}.get(stv, stv) if isinstance(stv, str) else int(stv)
+    return c
+
+
+def _ptr(t) -> int:
+    if t is None:
+        return 0
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to liblowram must be contiguous")
+    return int(t.data_ptr())
+
+
+def _stream(stream) -> int:
+    if stream is not None:
+        return int(stream) if isinstance(stream, int) else int(stream.cuda_stream)
+    import torch
+    if torch.cuda.is_available():
+        return int(torch.cuda.current_stream().cuda_stream)
+    return 0
+
+
+def _bytes_dict(b: LowramBytesC) -> dict:
+    return {n: int(getattr(b, n)) for n, _ in LowramBytesC._fields_}
+
+
+def lowram_dense_kv_bytes(n_layers: int, n_kv_heads: int, head_dim: int, n_ctx: int,
+                          bytes_per_scalar: int, batch: int) -> int:
+    return int(lib().lowram_dense_kv_bytes(n_layers, n_kv_heads, head_dim, n_ctx,
+                                           bytes_per_scalar, batch))
+
+
+def lowram_config_bytes(cfg, n_records: int, has_slot: bool = True) -> dict:
+    out = LowramBytesC()
+    c = config_struct(cfg)
+    _check(lib().lowram_config_bytes(ctypes.byref(c), int(n_records), int(has_slot),
+                                     ctypes.byref(out)), "lowram_config_bytes")
+    return _bytes_dict(out)
+
+
+def lowram_cache_create(cfg, arrays, stream=None) -> int:
+    """Create a cache from device tensors.  ``arrays`` is a mapping (or an object with
+    attributes) holding coeff, coeff_scale, basis, w1, w2, summary, slot, res_ptr, res_pos,
+    res_val, res_scale, tail_k, tail_v, tail_len (layouts of ``lowram.h``)."""
+    src = LowramSrcC()
+    names = ("coeff", "coeff_scale", "basis", "w1", "w2", "summary", "slot", "res_ptr",
+             "res_pos", "res_val", "res_scale", "tail_k", "tail_v", "tail_len")
+    keep = []
+    for n in names:
+        try:
+            t = _get(arrays, n)
+        except (AttributeError, KeyError):
+            t = None
+        if t is not None and not t.is_cuda:
+            raise ValueError(f"{n} must be a CUDA tensor")
+        keep.append(t)
+        setattr(src, n, _ptr(t))
+    rp = _get(arrays, "res_pos")
+    src.n_records = int(rp.shape[0]) if rp is not None else 0
+    c = config_struct(cfg)
+    h = ctypes.c_void_p()
+    _check(lib().lowram_cache_create(ctypes.byref(c), ctypes.byref(src), ctypes.byref(h),
+                                     _stream(stream)), "lowram_cache_create")
+    return int(h.value)
+
+
+def lowram_cache_destroy(handle: int) -> None:
+    if handle:
+        lib().lowram_cache_destroy(handle)
+
+
+def lowram_decode_attn(handle: int, layer0: int, n_layers: int, q, out, sel=None,
+                       path: int = PATH_AUTO, stream=None) -> None:
+    _check(lib().lowram_decode_attn(handle, layer0, n_layers, _ptr(q), _ptr(out), _ptr(sel),
+                                    path, _stream(stream)), "lowram_decode_attn")
+
+
+def lowram_select_chunks(handle: int, layer0: int, n_layers: int, q, scores=None, sel=None,
+                         stream=None) -> None:
+    _check(lib().lowram_select_chunks(handle, layer0, n_layers, _ptr(q), _ptr(scores), _ptr(sel),
+                                      _stream(stream)), "lowram_select_chunks")
+
+
+def lowram_decode_attn_host(handle: int, layer0: int, n_layers: int, q_host, out_host,
+                            sel_host=None, stream=None) -> None:
+    _check(lib().lowram_decode_attn_host(handle, layer0, n_layers, _ptr(q_host), _ptr(out_host),
+                                         _ptr(sel_host), _stream(stream)),
+           "lowram_decode_attn_host")
+
+
+def lowram_cache_bytes(handle: int) -> dict:
+    out = LowramBytesC()
+    _check(lib().lowram_cache_bytes(handle, ctypes.byref(out)), "lowram_cache_bytes")
+    return _bytes_dict(out)
+
+
+def lowram_cache_validate(handle: int, stream=None) -> int:
+    """Returns the lowram_status (0 = consistent, 5 = corrupt tables, 6 = a wait timed out)."""
+    st = int(lib().lowram_cache_validate(handle, _stream(stream)))
+    if st not in (0, 5, 6):
+        _check(st, "lowram_cache_validate")
+    return st
+
+
+def lowram_cache_set_stage_events(handle: int, events=None) -> None:
+    if events is None:
+        _check(lib().lowram_cache_set_stage_events(handle, None), "set_stage_events")
+        return
+    arr = (ctypes.c_void_p * 4)(*[int(e.cuda_event) for e in events])
+    _check(lib().lowram_cache_set_stage_events(handle, ctypes.cast(arr, ctypes.c_void_p)),
+           "set_stage_events")
+
+
+def lowram_cache_last_launches(handle: int) -> int:
+    return int(lib().lowram_cache_last_launches(handle))
+
+
+def lowram_cache_last_path(handle: int) -> int:
+    return int(lib().lowram_cache_last_path(handle))
+
+
+class LowramCache:
+    """Owning wrapper of a cache handle (destroys it on ``close``/garbage collection)."""
+
+    def __init__(self, cfg, arrays, stream=None):
+        self.cfg = cfg
+        self.handle = lowram_cache_create(cfg, arrays, stream)
+
+    @classmethod
+    def from_synth(cls, cache, stream=None):
+        """From an object with ``.cfg`` and the storage tensors as attributes."""
+        cfg = cache.cfg
+        cs = config_struct(cfg)
+        try:
+            cs.n_live = int(cfg.n_live)
+        except AttributeError:
+            pass
+        return cls({n: getattr(cs, n) for n, _ in LowramConfigC._fields_}, cache, stream)
+
+    def decode(self, q, out=None, sel: bool = False, layer0: int = 0,
+               n_layers: Optional[int] = None, path: int = PATH_AUTO, stream=None):
+        import torch
+        if n_layers is None:
+            n_layers = int(q.shape[0])
+        if out is None:
+            out = torch.empty_like(q)
+        s = None
+        if sel:
+            c = self.cfg
+            s = torch.empty(n_layers, _get(c, "batch"), _get(c, "n_kv_heads"), _get(c, "top_k"),
+                            dtype=torch.int32, device=q.device)
+        lowram_decode_attn(self.handle, layer0, n_layers, q, out, s, path, stream)
+        return (out, s) if sel else out
+
+    def select(self, q, layer0: int = 0, n_layers: Optional[int] = None, stream=None):
+        import torch
+        c = self.cfg
+        if n_layers is None:
+            n_layers = int(q.shape[0])
+        nC = _get(c, "n_ctx") // _get(c, "chunk")
+        scores = torch.empty(n_layers, _get(c, "batch"), _get(c, "n_kv_heads"), nC,
+                             dtype=torch.float32, device=q.device)
+        sel = torch.empty(n_layers, _get(c, "batch"), _get(c, "n_kv_heads"), _get(c, "top_k"),
+                          dtype=torch.int32, device=q.device)
+        lowram_select_chunks(self.handle, layer0, n_layers, q, scores, sel, stream)
+        return scores, sel
+
+    def bytes(self) -> dict:
+        return lowram_cache_bytes(self.handle)
+
+    def validate(self, stream=None) -> int:
+        return lowram_cache_validate(self.handle, stream)
+
+    @property
+    def last_path(self) -> int:
+        return lowram_cache_last_path(self.handle)
+
+    @property
+    def last_launches(self) -> int:
+        return lowram_cache_last_launches(self.handle)
+
+    def close(self) -> None:
+        if getattr(self, "handle", 0):
+            lowram_cache_destroy(self.handle)
+            self.handle = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

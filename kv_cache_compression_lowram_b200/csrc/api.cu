@@ -1,0 +1,425 @@
+// C ABI of the LowRAM decode library: cache object, argument checks, launches.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "lowram_internal.cuh"
+
+using namespace lowram;
+
+struct lowram_cache {
+  lowram_config cfg;
+  int nC, nL, NG, g, device, n_sm;
+  size_t s_dt;                 // bytes of one dt element
+  void* owned[24];
+  int n_owned;
+  CacheBuffers cb;
+  float* w1f_t;                // [L][Hkv][r][h] fp32 fold for the CUDA-core path
+  void* w1f_tc;                // [L][Hkv][h][r] 16-bit fold / 2 for the tensor-core path
+  Scratch sc;
+  size_t part_floats;          // capacity of sc.part
+  void* q_stage;               // host entry point staging
+  void* out_stage;
+  int32_t* sel_stage;
+  cudaEvent_t ev[4];
+  bool ev_on;
+  int last_launches, last_path;
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+lowram_status cuda_fail(cudaError_t e, const char* where) {
+  g_last_error = std::string(where) + ": " + cudaGetErrorString(e);
+  return LOWRAM_ECUDA;
+}
+
+lowram_status inval(const char* why) {
+  g_last_error = why;
+  return LOWRAM_EINVAL;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+lowram_status check_config(const lowram_config* c) {
+  if (!c) return inval("config is NULL");
+  if (c->batch < 1 || c->n_layers < 1 || c->group < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1 ||
+      c->head_dim < 1 || c->rank < 1 || c->mlp_hidden < 1 || c->n_ctx < 1 || c->chunk < 1 ||
+      c->top_k < 1 || c->tail_cap < 0 || c->n_live < 1)
+    return inval("config sizes must be positive");
+  if (c->n_layers % c->group) return inval("n_layers must be a multiple of group");
+  if (c->n_q_heads % c->n_kv_heads) return inval("n_q_heads must be a multiple of n_kv_heads");
+  if (c->n_ctx % c->chunk) return inval("n_ctx must be a multiple of chunk");
+  const int nC = c->n_ctx / c->chunk;
+  if (c->n_live > nC) return inval("n_live exceeds the number of chunks");
+  if (c->top_k > c->n_live) return inval("top_k exceeds the live chunks");
+  if (c->rank > c->group * c->head_dim) return inval("rank exceeds group * head_dim");
+  if (c->chunk > 32767) return inval("chunk exceeds 32767");
+  if (c->n_q_heads / c->n_kv_heads > kMaxG) return inval("more than 16 query heads per KV head");
+  if (c->head_dim > kMaxD || c->rank > kMaxR || c->mlp_hidden > kMaxH)
+    return inval("head_dim/rank/mlp_hidden above the supported maximum (256/512/1024)");
+  if (nC > kMaxChunks) return inval("more than 8192 chunks");
+  if (c->tail_cap > kMaxTail) return inval("tail_cap exceeds 4096");
+  if (c->dtype != LOWRAM_F32 && c->dtype != LOWRAM_BF16) return inval("unknown dtype");
+  if (c->store != LOWRAM_STORE_NATIVE && c->store != LOWRAM_STORE_INT8) return inval("unknown store");
+  if (c->store == LOWRAM_STORE_INT8 && c->dtype != LOWRAM_BF16) return inval("int8 store needs BF16");
+  return LOWRAM_OK;
+}
+
+void fill_bytes(const lowram_config* c, int64_t n_records, bool has_slot, lowram_bytes* b) {
+  const uint64_t B = c->batch, L = c->n_layers, G = c->group, H = c->n_kv_heads;
+  const uint64_t d = c->head_dim, r = c->rank, h = c->mlp_hidden, N = c->n_ctx, C = c->chunk;
+  const uint64_t T = c->tail_cap, nC = N / C, nL = c->n_live, NG = L / G;
+  const uint64_t s = c->dtype == LOWRAM_F32 ? 4 : 2;
+  const bool i8 = c->store == LOWRAM_STORE_INT8;
+  const uint64_t sa = i8 ? 1 : s;
+  const uint64_t R = (uint64_t)n_records;
+  b->coeff = B * NG * H * nL * C * (r * sa + (i8 ? 2 : 0));
+  b->basis = L * H * r * d * s;
+  b->predictor = 2 * L * H * h * d * s;
+  b->summary = B * NG * H * nL * r * s;
+  b->residual = R * (d * sa + 2 + (i8 ? 2 : 0)) + B * L * H * (nL + 1) * 4;
+  b->index = has_slot ? B * NG * H * nC * 2 : 0;
+  const uint64_t st = i8 ? 2 : s;
+  b->tail = 2 * B * L * H * T * d * st + 4 * B;
+  b->total = b->coeff + b->basis + b->predictor + b->summary + b->residual + b->index + b->tail;
+  b->dense_equiv = lowram_dense_kv_bytes(c->n_layers, c->n_kv_heads, c->head_dim, c->n_ctx,
+                                         (int32_t)s, c->batch) +
+                   2 * B * L * H * T * d * s;
+}
+
+Geom make_geom(const lowram_cache* c, int layer0, int n_layers, bool tc) {
+  Geom g;
+  const lowram_config& f = c->cfg;
+  g.B = f.batch; g.L = f.n_layers; g.G = f.group; g.Hkv = f.n_kv_heads; g.Hq = f.n_q_heads;
+  g.g = f.n_q_heads / f.n_kv_heads; g.d = f.head_dim; g.r = f.rank; g.h = f.mlp_hidden;
+  g.N = f.n_ctx; g.C = f.chunk; g.nC = c->nC; g.nL = c->nL; g.k = f.top_k; g.T = f.tail_cap;
+  g.layer0 = layer0; g.n_layers = n_layers;
+  g.U = n_layers * g.Hkv * g.B;
+  const long long total = (long long)g.U * g.k;
+  const long long pmax = tc ? c->n_sm : 4LL * c->n_sm;
+  g.P = (int)(total < pmax ? total : pmax);
+  g.rec_stride = (2 * g.g + g.g * g.h + g.g * g.d + 3) & ~3;
+  g.tail_stride = (2 * g.g + g.g * g.d + 3) & ~3;
+  g.max_rec = max_records_per_unit(total, g.P, g.k);
+  g.qk_scale_log2 = 1.4426950408889634f / sqrtf((float)g.d);
+  return g;
+}
+
+template <typename P>
+lowram_status alloc(lowram_cache* c, P** out, size_t bytes) {
+  void* p = nullptr;
+  if (bytes == 0) bytes = 16;
+  cudaError_t e = cudaMalloc(&p, bytes);
+  if (e != cudaSuccess) {
+    g_last_error = std::string("cudaMalloc: ") + cudaGetErrorString(e);
+    return LOWRAM_ENOMEM;
+  }
+  c->owned[c->n_owned++] = p;
+  *out = static_cast<P*>(p);
+  return LOWRAM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+uint64_t lowram_dense_kv_bytes(int32_t n_layers, int32_t n_kv_heads, int32_t head_dim,
+                               int64_t n_ctx, int32_t bytes_per_scalar, int32_t batch) {
+  if (n_layers < 0 || n_kv_heads < 0 || head_dim < 0 || n_ctx < 0 || bytes_per_scalar < 0 ||
+      batch < 0)
+    return 0;
+  return 2ull * (uint64_t)n_layers * (uint64_t)n_kv_heads * (uint64_t)head_dim *
+         (uint64_t)n_ctx * (uint64_t)bytes_per_scalar * (uint64_t)batch;
+}
+
+lowram_status lowram_config_bytes(const lowram_config* cfg, int64_t n_records, int32_t has_slot,
+                                  lowram_bytes* out) {
+  lowram_status st = check_config(cfg);
+  if (st != LOWRAM_OK) return st;
+  if (!out || n_records < 0) return inval("bad n_records or NULL output");
+  fill_bytes(cfg, n_records, has_slot != 0 && cfg->n_live < cfg->n_ctx / cfg->chunk, out);
+  return LOWRAM_OK;
+}
+
+const char* lowram_status_string(lowram_status s) {
+  switch (s) {
+    case LOWRAM_OK: return "ok";
+    case LOWRAM_EINVAL: return "invalid argument";
+    case LOWRAM_ENOMEM: return "out of device memory";
+    case LOWRAM_ECUDA: return "CUDA error";
+    case LOWRAM_EUNSUPPORTED: return "unsupported shapes for the requested path";
+    case LOWRAM_ECORRUPT: return "inconsistent cache tables";
+    case LOWRAM_ETIMEOUT: return "a kernel gave up a bounded wait";
+  }
+  return "unknown status";
+}
+
+const char* lowram_last_error_string(void) { return g_last_error.c_str(); }
+
+lowram_status lowram_cache_create(const lowram_config* cfg, const lowram_cache_src* src,
+                                  lowram_cache** out, lowram_stream stream) {
+  lowram_status st = check_config(cfg);
+  if (st != LOWRAM_OK) return st;
+  if (!src || !out) return inval("NULL src or out");
+  *out = nullptr;
+  const bool i8 = cfg->store == LOWRAM_STORE_INT8;
+  const int nC = cfg->n_ctx / cfg->chunk;
+  const bool evict = cfg->n_live < nC;
+  const void* need[] = {src->coeff, src->basis, src->w1, src->w2, src->summary, src->res_ptr,
+                        src->tail_k, src->tail_v, src->tail_len};
+  for (const void* p : need)
+    if (!p || !aligned16(p)) return inval("a required source pointer is NULL or not 16-byte aligned");
+  if (src->n_records < 0 || src->n_records >= (1LL << 31)) return inval("n_records out of range");
+  if (src->n_records > 0 && (!src->res_pos || !src->res_val || !aligned16(src->res_val) ||
+                             !aligned16(src->res_pos)))
+    return inval("residual arrays missing or misaligned");
+  if (i8 && (!src->coeff_scale || !aligned16(src->coeff_scale) ||
+             (src->n_records > 0 && (!src->res_scale || !aligned16(src->res_scale)))))
+    return inval("int8 store needs coeff_scale and res_scale");
+  if (evict && (!src->slot || !aligned16(src->slot))) return inval("eviction needs a slot map");
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  int n_sm = 0;
+  e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+
+  lowram_cache* c = new lowram_cache();
+  std::memset(c, 0, sizeof(*c));
+  c->cfg = *cfg;
+  c->nC = nC; c->nL = cfg->n_live; c->NG = cfg->n_layers / cfg->group;
+  c->g = cfg->n_q_heads / cfg->n_kv_heads;
+  c->device = dev; c->n_sm = n_sm;
+  c->s_dt = cfg->dtype == LOWRAM_F32 ? 4 : 2;
+
+  const size_t B = cfg->batch, L = cfg->n_layers, H = cfg->n_kv_heads, d = cfg->head_dim;
+  const size_t r = cfg->rank, h = cfg->mlp_hidden, C = cfg->chunk, T = cfg->tail_cap;
+  const size_t nL = cfg->n_live, NG = c->NG, R = (size_t)src->n_records, s = c->s_dt;
+  const size_t sa = i8 ? 1 : s, st16 = i8 ? 2 : s;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  struct Item { const void* from; void** to; size_t bytes; };
+  void* p_coeff = nullptr; void* p_cscale = nullptr; void* p_basis = nullptr; void* p_w1 = nullptr;
+  void* p_w2 = nullptr; void* p_summ = nullptr; void* p_slot = nullptr; void* p_rptr = nullptr;
+  void* p_rpos = nullptr; void* p_rval = nullptr; void* p_rscale = nullptr; void* p_tk = nullptr;
+  void* p_tv = nullptr; void* p_tl = nullptr;
+  Item items[] = {
+      {src->coeff, &p_coeff, B * NG * H * nL * C * r * sa},
+      {i8 ? src->coeff_scale : nullptr, &p_cscale, i8 ? B * NG * H * nL * C * 2 : 0},
+      {src->basis, &p_basis, L * H * r * d * s},
+      {src->w1, &p_w1, L * H * h * d * s},
+      {src->w2, &p_w2, L * H * d * h * s},
+      {src->summary, &p_summ, B * NG * H * nL * r * s},
+      {evict ? src->slot : nullptr, &p_slot, evict ? B * NG * H * nC * 2 : 0},
+      {src->res_ptr, &p_rptr, B * L * H * (nL + 1) * 4},
+      {R ? src->res_pos : nullptr, &p_rpos, R * 2},
+      {R ? src->res_val : nullptr, &p_rval, R * d * sa},
+      {(i8 && R) ? src->res_scale : nullptr, &p_rscale, (i8 && R) ? R * 2 : 0},
+      {src->tail_k, &p_tk, B * L * H * T * d * st16},
+      {src->tail_v, &p_tv, B * L * H * T * d * st16},
+      {src->tail_len, &p_tl, B * 4},
+  };
+  for (Item& it : items) {
+    if (!it.from) continue;
+    st = alloc(c, it.to, it.bytes);
+    if (st != LOWRAM_OK) { lowram_cache_destroy(c); return st; }
+    if (it.bytes) {
+      e = cudaMemcpyAsync(*it.to, it.from, it.bytes, cudaMemcpyDeviceToDevice, cs);
+      if (e != cudaSuccess) { lowram_cache_destroy(c); return cuda_fail(e, "cudaMemcpyAsync"); }
+    }
+  }
+  c->cb.coeff = p_coeff; c->cb.coeff_scale = static_cast<const __half*>(p_cscale);
+  c->cb.basis = p_basis; c->cb.w1 = p_w1; c->cb.w2 = p_w2; c->cb.summary = p_summ;
+  c->cb.slot = static_cast<const int16_t*>(p_slot);
+  c->cb.res_ptr = static_cast<const int32_t*>(p_rptr);
+  c->cb.res_pos = static_cast<const uint16_t*>(p_rpos);
+  c->cb.res_val = p_rval; c->cb.res_scale = static_cast<const __half*>(p_rscale);
+  c->cb.tail_k = p_tk; c->cb.tail_v = p_tv; c->cb.tail_len = static_cast<const int32_t*>(p_tl);
+  c->cb.n_records = src->n_records;
+
+  // folded predictor weights
+  Geom gall = make_geom(c, 0, cfg->n_layers, false);
+  if ((st = alloc(c, &c->w1f_t, L * H * r * h * 4)) != LOWRAM_OK) { lowram_cache_destroy(c); return st; }
+  if (cfg->dtype == LOWRAM_BF16) {
+    if ((st = alloc(c, &c->w1f_tc, L * H * h * r * 2)) != LOWRAM_OK) { lowram_cache_destroy(c); return st; }
+  }
+  e = launch_fold(gall, c->cb, cfg->dtype, cfg->store, c->w1f_t, c->w1f_tc, cs);
+  if (e != cudaSuccess) { lowram_cache_destroy(c); return cuda_fail(e, "fold"); }
+
+  // scratch for an all-layer call
+  const size_t Umax = L * H * B;
+  const size_t g = c->g, k = cfg->top_k;
+  const size_t rec_stride = (2 * g + g * h + g * d + 3) & ~size_t(3);
+  const size_t tail_stride = (2 * g + g * d + 3) & ~size_t(3);
+  c->part_floats = (Umax + 4 * (size_t)n_sm + 1) * rec_stride;
+  if ((st = alloc(c, &c->sc.qt, Umax * g * r * 4)) != LOWRAM_OK ||
+      (st = alloc(c, &c->sc.qt_tc, Umax * 16 * r * 2)) != LOWRAM_OK ||
+      (st = alloc(c, &c->sc.sel_slot, Umax * k * 4)) != LOWRAM_OK ||
+      (st = alloc(c, &c->sc.sel_id, Umax * k * 4)) != LOWRAM_OK ||
+      (st = alloc(c, &c->sc.part, c->part_floats * 4)) != LOWRAM_OK ||
+      (st = alloc(c, &c->sc.tail_part, Umax * tail_stride * 4)) != LOWRAM_OK ||
+      (st = alloc(c, &c->sc.err, 16)) != LOWRAM_OK ||
+      (st = alloc(c, &c->q_stage, L * B * cfg->n_q_heads * d * s)) != LOWRAM_OK ||
+      (st = alloc(c, &c->out_stage, L * B * cfg->n_q_heads * d * s)) != LOWRAM_OK ||
+      (st = alloc(c, &c->sel_stage, Umax * k * 4)) != LOWRAM_OK) {
+    lowram_cache_destroy(c);
+    return st;
+  }
+  e = cudaMemsetAsync(c->sc.err, 0, 16, cs);
+  if (e != cudaSuccess) { lowram_cache_destroy(c); return cuda_fail(e, "cudaMemsetAsync"); }
+  e = cudaMemsetAsync(c->sc.qt_tc, 0, Umax * 16 * r * 2, cs);
+  if (e != cudaSuccess) { lowram_cache_destroy(c); return cuda_fail(e, "cudaMemsetAsync"); }
+  c->last_path = -1;
+  *out = c;
+  return LOWRAM_OK;
+}
+
+void lowram_cache_destroy(lowram_cache* c) {
+  if (!c) return;
+  cudaDeviceSynchronize();
+  for (int i = 0; i < c->n_owned; ++i) cudaFree(c->owned[i]);
+  delete c;
+}
+
+lowram_status lowram_cache_bytes(const lowram_cache* c, lowram_bytes* out) {
+  if (!c || !out) return inval("NULL cache or output");
+  fill_bytes(&c->cfg, c->cb.n_records, c->cb.slot != nullptr, out);
+  return LOWRAM_OK;
+}
+
+lowram_status lowram_cache_set_stage_events(lowram_cache* c, void* const* events) {
+  if (!c) return inval("NULL cache");
+  if (!events) {
+    c->ev_on = false;
+    return LOWRAM_OK;
+  }
+  for (int i = 0; i < 4; ++i) {
+    if (!events[i]) return inval("NULL event");
+    c->ev[i] = static_cast<cudaEvent_t>(events[i]);
+  }
+  c->ev_on = true;
+  return LOWRAM_OK;
+}
+
+int32_t lowram_cache_last_launches(const lowram_cache* c) { return c ? c->last_launches : 0; }
+int32_t lowram_cache_last_path(const lowram_cache* c) { return c ? c->last_path : -1; }
+
+static lowram_status check_layers(const lowram_cache* c, int32_t layer0, int32_t n_layers) {
+  if (!c) return inval("NULL cache");
+  if (layer0 < 0 || n_layers < 1 || layer0 + n_layers > c->cfg.n_layers)
+    return inval("layer range outside the cache");
+  return LOWRAM_OK;
+}
+
+lowram_status lowram_select_chunks(lowram_cache* c, int32_t layer0, int32_t n_layers,
+                                   const void* q, float* scores, int32_t* sel,
+                                   lowram_stream stream) {
+  lowram_status st = check_layers(c, layer0, n_layers);
+  if (st != LOWRAM_OK) return st;
+  if (!q) return inval("NULL q");
+  Geom g = make_geom(c, layer0, n_layers, false);
+  cudaError_t e = launch_select(g, c->cb, c->sc, c->cfg.dtype, q, scores, sel, 0, false,
+                                reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "select kernel");
+  return LOWRAM_OK;
+}
+
+lowram_status lowram_decode_attn(lowram_cache* c, int32_t layer0, int32_t n_layers,
+                                 const void* q, void* out, int32_t* sel, int32_t path,
+                                 lowram_stream stream) {
+  lowram_status st = check_layers(c, layer0, n_layers);
+  if (st != LOWRAM_OK) return st;
+  if (!q || !out) return inval("NULL q or out");
+  if (path < LOWRAM_PATH_AUTO || path > LOWRAM_PATH_TC) return inval("unknown path");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const bool tc_able = attend_tc_supported(make_geom(c, layer0, n_layers, true), c->cfg.dtype,
+                                           c->cfg.store);
+  bool tc = false;
+  if (path == LOWRAM_PATH_TC) {
+    if (!tc_able) {
+      g_last_error = "the tensor-core path does not handle these shapes";
+      return LOWRAM_EUNSUPPORTED;
+    }
+    tc = true;
+  } else if (path == LOWRAM_PATH_AUTO) {
+    tc = tc_able;
+  }
+  Geom g = make_geom(c, layer0, n_layers, tc);
+  cudaError_t e;
+  if (c->ev_on && (e = cudaEventRecord(c->ev[0], s)) != cudaSuccess) return cuda_fail(e, "event");
+  const int tc_q_mode = tc ? (c->cfg.store == LOWRAM_STORE_INT8 ? 2 : 1) : 0;
+  e = launch_select(g, c->cb, c->sc, c->cfg.dtype, q, nullptr, sel, tc_q_mode, true, s);
+  if (e != cudaSuccess) return cuda_fail(e, "select kernel");
+  if (c->ev_on && (e = cudaEventRecord(c->ev[1], s)) != cudaSuccess) return cuda_fail(e, "event");
+  if (tc)
+    e = launch_attend_tc(g, c->cb, c->sc, c->cfg.store, c->w1f_tc, c->n_sm, s);
+  else
+    e = launch_attend_simt(g, c->cb, c->sc, c->cfg.dtype, c->cfg.store, c->w1f_t, s);
+  if (e != cudaSuccess) return cuda_fail(e, "chunk attention kernel");
+  if (c->ev_on && (e = cudaEventRecord(c->ev[2], s)) != cudaSuccess) return cuda_fail(e, "event");
+  e = launch_combine(g, c->cb, c->sc, c->cfg.dtype, out, s);
+  if (e != cudaSuccess) return cuda_fail(e, "combine kernel");
+  if (c->ev_on && (e = cudaEventRecord(c->ev[3], s)) != cudaSuccess) return cuda_fail(e, "event");
+  c->last_launches = 3;
+  c->last_path = tc ? LOWRAM_PATH_TC : LOWRAM_PATH_SIMT;
+  return LOWRAM_OK;
+}
+
+lowram_status lowram_decode_attn_host(lowram_cache* c, int32_t layer0, int32_t n_layers,
+                                      const void* q_host, void* out_host, int32_t* sel_host,
+                                      lowram_stream stream) {
+  lowram_status st = check_layers(c, layer0, n_layers);
+  if (st != LOWRAM_OK) return st;
+  if (!q_host || !out_host) return inval("NULL q or out");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t qbytes = (size_t)n_layers * c->cfg.batch * c->cfg.n_q_heads * c->cfg.head_dim * c->s_dt;
+  const size_t sbytes = (size_t)n_layers * c->cfg.batch * c->cfg.n_kv_heads * c->cfg.top_k * 4;
+  cudaError_t e = cudaMemcpyAsync(c->q_stage, q_host, qbytes, cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return cuda_fail(e, "copy q to the device");
+  st = lowram_decode_attn(c, layer0, n_layers, c->q_stage, c->out_stage,
+                          sel_host ? c->sel_stage : nullptr, LOWRAM_PATH_AUTO, stream);
+  if (st != LOWRAM_OK) return st;
+  e = cudaMemcpyAsync(out_host, c->out_stage, qbytes, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "copy out to the host");
+  if (sel_host) {
+    e = cudaMemcpyAsync(sel_host, c->sel_stage, sbytes, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_fail(e, "copy sel to the host");
+  }
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  return LOWRAM_OK;
+}
+
+lowram_status lowram_cache_validate(lowram_cache* c, lowram_stream stream) {
+  if (!c) return inval("NULL cache");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Geom g = make_geom(c, 0, c->cfg.n_layers, false);
+  cudaError_t e = launch_validate(g, c->cb, c->sc.err, s);
+  if (e != cudaSuccess) return cuda_fail(e, "validate kernel");
+  uint32_t word = 0;
+  e = cudaMemcpyAsync(&word, c->sc.err, 4, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "read error word");
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  e = cudaMemsetAsync(c->sc.err, 0, 4, s);
+  if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  if (word & (ERR_SLOT | ERR_RES_PTR | ERR_RES_POS | ERR_TAIL_LEN | ERR_SELECT)) {
+    char buf[96];
+    std::snprintf(buf, sizeof buf, "cache tables inconsistent (error word 0x%x)", word);
+    g_last_error = buf;
+    return LOWRAM_ECORRUPT;
+  }
+  if (word & ERR_TIMEOUT) {
+    g_last_error = "a kernel gave up a bounded wait";
+    return LOWRAM_ETIMEOUT;
+  }
+  return LOWRAM_OK;
+}
+
+}  // extern "C"

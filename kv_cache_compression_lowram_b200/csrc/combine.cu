@@ -1,0 +1,210 @@
+// Final step: merge the softmax partials of a unit (raw tail + every chunk piece),
+// apply the predictor's second layer once to the softmax-weighted hidden sum and
+// normalise:
+//     o_j = (W2 . sum_t p_jt h_t + sum_t p_jt delta_t + sum_tail p_jt v_t) / sum_t p_jt
+// This is the exact regrouping of sum_t p_jt (W2 h_t + delta_t) for the rebuilt values of
+// "LowRAM Compresses KV Cache Asymmetrically", section "Core Mechanism" (Vhat = f(K) plus
+// delta for the worst tokens), inside the attention of "OjaKV", section 3.
+// Also: the create-time fold W1' = W1 B_l^T and the device-side table check.
+#include "lowram_internal.cuh"
+
+namespace lowram {
+namespace {
+
+constexpr int kThreads = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+combine_kernel(Geom g, CacheBuffers cb, Scratch sc, T* __restrict__ out) {
+  extern __shared__ __align__(16) float sm[];
+  const int u = blockIdx.x;
+  const Unit un = unit_of(g, u);
+  const int l = g.layer0 + un.li;
+  const long long total = (long long)g.U * g.k;
+  const int c0 = cta_of_tile(total, g.P, (long long)u * g.k);
+  const int c1 = cta_of_tile(total, g.P, (long long)(u + 1) * g.k - 1);
+  const int nrec = c1 - c0 + 1;
+  if (nrec > g.max_rec) {  // cannot happen with a consistent tile partition
+    if (threadIdx.x == 0) atomicOr(sc.err, ERR_SELECT);
+    return;
+  }
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarp = blockDim.x >> 5;
+
+  float* accH = sm;                   // [g][h]
+  float* accD = accH + g.g * g.h;     // [g][d]
+  float* lsum = accD + g.g * g.d;     // [g]
+  float* wts = lsum + g.g;            // [nrec + 1][g]  (last row: tail)
+
+  const float* trec = sc.tail_part + (size_t)u * g.tail_stride;
+  for (int j = tid; j < g.g; j += blockDim.x) {
+    float M = trec[j];
+    for (int r = 0; r < nrec; ++r) M = fmaxf(M, sc.part[(size_t)(u + c0 + r) * g.rec_stride + j]);
+    float L = 0.f;
+    for (int r = 0; r < nrec; ++r) {
+      const float* rec = sc.part + (size_t)(u + c0 + r) * g.rec_stride;
+      const float w = rec[j] == -INFINITY ? 0.f : exp2f(rec[j] - M);
+      wts[r * g.g + j] = w;
+      L += w * rec[g.g + j];
+    }
+    const float wt = trec[j] == -INFINITY ? 0.f : exp2f(trec[j] - M);
+    wts[nrec * g.g + j] = wt;
+    L += wt * trec[g.g + j];
+    lsum[j] = L;
+  }
+  __syncthreads();
+  for (int i = tid; i < g.g * g.h; i += blockDim.x) {
+    const int j = i / g.h;
+    float a = 0.f;
+    for (int r = 0; r < nrec; ++r)
+      a = fmaf(wts[r * g.g + j], sc.part[(size_t)(u + c0 + r) * g.rec_stride + 2 * g.g + i], a);
+    accH[i] = a;
+  }
+  for (int i = tid; i < g.g * g.d; i += blockDim.x) {
+    const int j = i / g.d;
+    float a = wts[nrec * g.g + j] * trec[2 * g.g + i];
+    for (int r = 0; r < nrec; ++r)
+      a = fmaf(wts[r * g.g + j],
+               sc.part[(size_t)(u + c0 + r) * g.rec_stride + 2 * g.g + g.g * g.h + i], a);
+    accD[i] = a;
+  }
+  __syncthreads();
+  // second predictor layer on the weighted hidden sums: one warp per output row dd
+  const T* W2 = reinterpret_cast<const T*>(cb.w2) + ((size_t)l * g.Hkv + un.hkv) * g.d * g.h;
+  T* o = out + ((size_t)(un.li * g.B + un.b) * g.Hq + (size_t)un.hkv * g.g) * g.d;
+  for (int dd = warp; dd < g.d; dd += nwarp) {
+    const T* row = W2 + (size_t)dd * g.h;
+    float a[kMaxG];
+#pragma unroll
+    for (int j = 0; j < kMaxG; ++j) a[j] = 0.f;
+    for (int i = lane; i < g.h; i += 32) {
+      const float w = to_f(row[i]);
+#pragma unroll
+      for (int j = 0; j < kMaxG; ++j)
+        if (j < g.g) a[j] = fmaf(w, accH[j * g.h + i], a[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxG; ++j) {
+      if (j < g.g) {
+        const float s = warp_sum(a[j]);
+        if (lane == 0) o[(size_t)j * g.d + dd] = from_f<T>((s + accD[j * g.d + dd]) / lsum[j]);
+      }
+    }
+  }
+}
+
+// W1'[i][rr] = sum_dd W1[i][dd] * B_l[rr][dd] for every (layer, KV head).
+template <typename T>
+__global__ void fold_kernel(Geom g, const T* __restrict__ w1, const T* __restrict__ basis,
+                            float* __restrict__ w1f_t, __nv_bfloat16* __restrict__ w1f_bf16,
+                            __half* __restrict__ w1f_f16) {
+  const size_t n = (size_t)g.L * g.Hkv * g.h * g.r;
+  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < n;
+       idx += (size_t)gridDim.x * blockDim.x) {
+    const int rr = (int)(idx % g.r);
+    const int i = (int)((idx / g.r) % g.h);
+    const size_t lh = idx / ((size_t)g.r * g.h);
+    const T* wr = w1 + (lh * g.h + i) * g.d;
+    const T* br = basis + (lh * g.r + rr) * g.d;
+    float a = 0.f;
+    for (int dd = 0; dd < g.d; ++dd) a = fmaf(to_f(wr[dd]), to_f(br[dd]), a);
+    if (w1f_t) w1f_t[(lh * g.r + rr) * g.h + i] = a;
+    // tensor-core copy holds W1'/2: the MMA then yields u = x/2 and silu(x) = u + u*tanh(u)
+    if (w1f_bf16) w1f_bf16[idx] = __float2bfloat16_rn(0.5f * a);
+    if (w1f_f16) w1f_f16[idx] = __float2half_rn(0.5f * a);
+  }
+}
+
+__global__ void validate_kernel(Geom g, CacheBuffers cb, uint32_t* err) {
+  const int NG = g.L / g.G;
+  const int n_slot_rows = g.B * NG * g.Hkv;
+  const int n_units = g.B * g.L * g.Hkv;
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx < n_slot_rows && cb.slot) {
+    const int16_t* s = cb.slot + (size_t)idx * g.nC;
+    int next = 0;
+    bool bad = false;
+    for (int c = 0; c < g.nC; ++c) {
+      const int v = s[c];
+      if (v == -1) continue;
+      if (v != next) bad = true;
+      ++next;
+    }
+    if (next != g.nL) bad = true;
+    if (bad) atomicOr(err, ERR_SLOT);
+  }
+  if (idx < n_units) {
+    const int32_t* p = cb.res_ptr + (size_t)idx * (g.nL + 1);
+    bool bad_ptr = false, bad_pos = false;
+    for (int s = 0; s <= g.nL; ++s) {
+      if (p[s] < 0 || p[s] > cb.n_records) bad_ptr = true;
+      if (s < g.nL && p[s + 1] < p[s]) bad_ptr = true;
+    }
+    if (!bad_ptr) {
+      for (int s = 0; s < g.nL; ++s) {
+        int prev = -1;
+        for (int r = p[s]; r < p[s + 1]; ++r) {
+          const int pos = cb.res_pos[r];
+          if (pos >= g.C || pos <= prev) bad_pos = true;
+          prev = pos;
+        }
+      }
+    }
+    if (bad_ptr) atomicOr(err, ERR_RES_PTR);
+    if (bad_pos) atomicOr(err, ERR_RES_POS);
+  }
+  if (idx < g.B) {
+    const int tl = cb.tail_len[idx];
+    if (tl < 0 || tl > g.T) atomicOr(err, ERR_TAIL_LEN);
+  }
+}
+
+}  // namespace
+
+size_t combine_smem_bytes(const Geom& g) {
+  return sizeof(float) * ((size_t)g.g * g.h + (size_t)g.g * g.d + g.g + (size_t)(g.max_rec + 1) * g.g);
+}
+
+cudaError_t launch_combine(const Geom& g, const CacheBuffers& cb, const Scratch& sc, int dtype,
+                           void* out, cudaStream_t s) {
+  const size_t smem = combine_smem_bytes(g);
+  if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
+  cudaError_t e;
+  if (dtype == LOWRAM_F32) {
+    auto k = combine_kernel<float>;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<g.U, kThreads, smem, s>>>(g, cb, sc, static_cast<float*>(out));
+  } else {
+    auto k = combine_kernel<__nv_bfloat16>;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<g.U, kThreads, smem, s>>>(g, cb, sc, static_cast<__nv_bfloat16*>(out));
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fold(const Geom& g, const CacheBuffers& cb, int dtype, int store,
+                        float* w1f_t, void* w1f_tc, cudaStream_t s) {
+  const size_t n = (size_t)g.L * g.Hkv * g.h * g.r;
+  const int blocks = (int)((n + 255) / 256 < 65535 * 8 ? (n + 255) / 256 : 65535 * 8);
+  if (dtype == LOWRAM_F32) {
+    fold_kernel<float><<<blocks, 256, 0, s>>>(g, static_cast<const float*>(cb.w1),
+                                              static_cast<const float*>(cb.basis), w1f_t,
+                                              nullptr, nullptr);
+  } else {
+    __nv_bfloat16* bf = store == LOWRAM_STORE_INT8 ? nullptr : static_cast<__nv_bfloat16*>(w1f_tc);
+    __half* hf = store == LOWRAM_STORE_INT8 ? static_cast<__half*>(w1f_tc) : nullptr;
+    fold_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+        g, static_cast<const __nv_bfloat16*>(cb.w1), static_cast<const __nv_bfloat16*>(cb.basis),
+        w1f_t, bf, hf);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_validate(const Geom& g, const CacheBuffers& cb, uint32_t* err, cudaStream_t s) {
+  const int n = g.B * g.L * g.Hkv;
+  validate_kernel<<<(n + 127) / 128, 128, 0, s>>>(g, cb, err);
+  return cudaGetLastError();
+}
+
+}  // namespace lowram

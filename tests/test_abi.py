@@ -1,0 +1,93 @@
+"""The C-ABI library loads, exports every declared symbol and validates on the host.
+
+No compute call here needs a GPU: only host-only entry points and argument checks that
+return before any CUDA call.
+"""
+
+import ctypes
+import dataclasses
+import glob
+import os
+import re
+
+import pytest
+
+import kv_cache_compression_lowram_b200 as K
+import lowram_synth as S
+import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for hdr in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(hdr).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b(lowram_[a-z0-9_]+)\s*\(", text):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = K.lib()
+    names = _declared_functions()
+    assert len(names) >= 14
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_dense_kv_bytes_worked_example():
+    # Llama-3.1-8B, 32K prompt, batch 4, fp16: 16 GiB ("OjaKV" abstract; M_KV formula of
+    # "LowRAM Compresses KV Cache Asymmetrically", section "Core Mechanism")
+    assert K.lowram_dense_kv_bytes(32, 8, 128, 32768, 2, 4) == 17179869184
+    assert K.lowram_dense_kv_bytes(32, 8, 128, 32768, 2, 4) == O.dense_kv_bytes(32, 8, 128, 32768, 2, 4)
+    assert K.lowram_dense_kv_bytes(-1, 8, 128, 32768, 2, 4) == 0
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "mistral7b_group_bf16", "llama8b_32k_bf16",
+                                  "llama8b_64k_int8_evict", "llama8b_32k_bf16_b64"])
+def test_config_bytes_match_oracle_closed_form(name):
+    cfg = S.CONFIGS[name]
+    n_rec = cfg.batch * cfg.n_layers * cfg.n_kv_heads * cfg.n_resid // 3
+    got = K.lowram_config_bytes(cfg, n_rec, has_slot=True)
+    want = O.compressed_bytes(dataclasses.asdict(cfg), n_rec)
+    assert got == want
+
+
+def test_bad_configs_rejected_on_host():
+    bad = [
+        dict(top_k=10_000),
+        dict(n_ctx=1000),            # not a multiple of chunk
+        dict(n_q_heads=30),          # not a multiple of n_kv_heads
+        dict(n_layers=30),           # not a multiple of group
+        dict(rank=10_000),
+        dict(dtype="f32", store="int8"),
+        dict(batch=0),
+    ]
+    for kw in bad:
+        cfg = S.LLAMA_32K.replace(**kw)
+        with pytest.raises(K.LowramError) as ei:
+            K.lowram_config_bytes(cfg, 0)
+        assert ei.value.status == 1
+
+
+def test_create_rejects_null_sources_without_touching_cuda():
+    lib = K.lib()
+    c = K.config_struct(S.TINY_F32)
+    src = K.LowramSrcC()
+    h = ctypes.c_void_p()
+    st = lib.lowram_cache_create(ctypes.byref(c), ctypes.byref(src), ctypes.byref(h), None)
+    assert st == 1 and not h.value
+    assert b"NULL" in lib.lowram_last_error_string()
+    # NULL cache handles are rejected, not dereferenced
+    assert lib.lowram_decode_attn(None, 0, 1, None, None, None, 0, None) == 1
+    assert lib.lowram_cache_validate(None, None) == 1
+    assert lib.lowram_cache_last_launches(None) == 0
+    lib.lowram_cache_destroy(None)
+
+
+def test_status_strings():
+    lib = K.lib()
+    for s in range(7):
+        assert lib.lowram_status_string(s)
