@@ -232,6 +232,9 @@ def lowram_cache_set_stage_events(handle: int, events=None) -> None:
     if events is None:
         _check(lib().lowram_cache_set_stage_events(handle, None), "set_stage_events")
         return
+    for e in events:
+        if int(e.cuda_event) == 0:   # torch creates the CUDA event on its first record
+            e.record()
     arr = (ctypes.c_void_p * 4)(*[int(e.cuda_event) for e in events])
     _check(lib().lowram_cache_set_stage_events(handle, ctypes.cast(arr, ctypes.c_void_p)),
            "set_stage_events")

@@ -12,7 +12,7 @@ struct lowram_cache {
   lowram_config cfg;
   int nC, nL, NG, g, device, n_sm;
   size_t s_dt;                 // bytes of one dt element
-  void* owned[24];
+  void* owned[48];             // every device allocation the cache owns
   int n_owned;
   CacheBuffers cb;
   float* w1f_t;                // [L][Hkv][r][h] fp32 fold for the CUDA-core path
@@ -112,6 +112,10 @@ template <typename P>
 lowram_status alloc(lowram_cache* c, P** out, size_t bytes) {
   void* p = nullptr;
   if (bytes == 0) bytes = 16;
+  if (c->n_owned >= (int)(sizeof(c->owned) / sizeof(c->owned[0]))) {
+    g_last_error = "internal: too many owned allocations";
+    return LOWRAM_ENOMEM;
+  }
   cudaError_t e = cudaMalloc(&p, bytes);
   if (e != cudaSuccess) {
     g_last_error = std::string("cudaMalloc: ") + cudaGetErrorString(e);

@@ -1,12 +1,600 @@
-// Steps 3-5 on tcgen05 tensor cores (placeholder until the kernel lands).
+// Steps 3-5 on tcgen05 tensor cores (sm_100a): rebuild the selected chunks on chip and
+// attend over them, fused in one persistent kernel.
+//
+// Per selected chunk of C tokens (coefficient rows A_c, C x r, bf16) of a unit:
+//   S  = A_c . Qt^T                 scores q_j . khat_t / sqrt(d) * log2(e) in the low-rank
+//                                   form (Qt_j = B_l q_j, "OjaKV" 3.1 projects queries into
+//                                   the key basis); M=128 tokens, N=16 heads (g used)
+//   D1 = W1'/2 . A_sub^T            pre-activations / 2 of the predictor's hidden layer,
+//                                   W1' = W1 B_l^T (exact fold of W1 khat_t); M=128 hidden
+//                                   rows per half, N=64 tokens per sub-tile, A from TMEM
+//   H  = silu(2 * D1) = u + u tanh(u), written back to TMEM as fp16 (MUFU tanh)
+//   D3 = H . P                      softmax-weighted hidden sums per head (A = H from TMEM,
+//                                   B = P, the chunk's probabilities, fp16 in SMEM)
+// while a softmax warpgroup keeps the online max/sum per head and accumulates the
+// residual rows delta_t of the flagged tokens (CUDA cores).  The predictor's second layer
+// is applied once per unit in the combine kernel: sum_t p_t (W2 h_t + delta_t) =
+// W2 (sum_t p_t h_t) + sum_t p_t delta_t.  Key rebuild: "LowRAM Compresses KV Cache
+// Asymmetrically", section "Cross-Layer Low-Rank Key Compression"; values: same page,
+// "Core Mechanism" (Vhat = f(K), delta kept for the worst tokens); attention: "OjaKV", 3.
+//
+// Warp roles (14 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-5 and 6-9 the
+// two hidden-row halves (silu epilogue, D3 accumulation), 10-13 softmax + residuals.
+// A warp reaches TMEM lanes 32*(warp%4) .. +31, so each warpgroup of four consecutive
+// warps covers all 128 lanes.
+// TMEM (512 columns): W1' halves [0,128), D1 double buffer x 2 halves [128,384),
+// S double buffer [384,416), D3 double buffer x 2 halves [416,480).
+// Every wait is bounded: on timeout the kernel raises the error word, drains its own
+// copies and MMAs, frees TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "lowram_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace lowram {
+namespace {
 
-bool attend_tc_supported(const Geom&, int, int) { return false; }
+using namespace tc;
 
-cudaError_t launch_attend_tc(const Geom&, const CacheBuffers&, const Scratch&, int, const void*,
-                             int, cudaStream_t) {
+constexpr int kThreadsTC = 448;   // 14 warps
+constexpr int kHid = 256;
+constexpr int kDh = 128;
+
+template <int R, int C>
+struct TcLayout {
+  static constexpr int NT = 64;
+  static constexpr int SUBS = C / NT;
+  static constexpr int STAGES = 4;
+  static constexpr int RES_CAP = 32;
+  static constexpr int KSLABS = R / 64;
+  static constexpr int A_STAGE = KSLABS * 16384;     // 128 rows x 128 B per 64-wide K slab
+  static constexpr int Q_BUF = KSLABS * 2048;        // 16 rows x 128 B per slab
+  static constexpr int P_BUF = 16 * C * 2;
+  static constexpr int P_SBO = (C / 8) * 128;
+  static constexpr int RES_BUF = RES_CAP * kDh * 2;
+  static constexpr int P32_BUF = 16 * C * 4;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_Q = OFF_A + STAGES * A_STAGE;
+  static constexpr int OFF_P = OFF_Q + 2 * Q_BUF;
+  static constexpr int OFF_RES = OFF_P + 2 * P_BUF;
+  static constexpr int OFF_P32 = OFF_RES + STAGES * RES_BUF;
+  static constexpr int OFF_MISC = OFF_P32 + 2 * P32_BUF;
+  static constexpr int MISC_BYTES = 2048;
+  static constexpr int SMEM = OFF_MISC + MISC_BYTES + 1024;   // + alignment slack
+  // TMEM columns
+  static constexpr uint32_t T_W1 = 0;
+  static constexpr uint32_t T_D1 = 128;
+  static constexpr uint32_t T_S = 384;
+  static constexpr uint32_t T_D3 = 416;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(R / 2 <= 64, "W1' half must fit 64 TMEM columns");
+};
+
+struct Bars {
+  uint64_t a_full[4], a_empty[4];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t s_full[2], s_free[2];
+  uint64_t d1_full[2], h_ready[2];
+  uint64_t p_ready[2];
+  uint64_t d3_full[2], d3_free[2];
+  uint64_t w1_ready;
+  uint64_t drain;
+};
+
+struct Misc {
+  Bars bars;
+  float alpha[4][16];   // per-chunk rescale factors, ring of 4 (see the softmax warpgroup)
+  float red_max[4][16];
+  float red_sum[4][16];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ float bf16_bits_to_f(uint16_t b) {
+  return __uint_as_float(((uint32_t)b) << 16);
+}
+
+template <int R, int C, int GQ>
+__global__ void __maxnreg__(144)
+attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __restrict__ w1f,
+                 const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmQ) {
+  using Lay = TcLayout<R, C>;
+  constexpr int SUBS = Lay::SUBS, STAGES = Lay::STAGES, KSLABS = Lay::KSLABS;
+  extern __shared__ unsigned char smem_dyn[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  Misc* misc = reinterpret_cast<Misc*>(smem + Lay::OFF_MISC);
+  Bars& bar = misc->bars;
+  volatile int* abort_flag = &misc->abort_flag;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long total = (long long)g.U * g.k;
+  const long long x0 = tile_begin(total, g.P, blockIdx.x);
+  const long long x1 = tile_begin(total, g.P, blockIdx.x + 1);
+  const int NCH = (int)(x1 - x0);
+  const int NS = NCH * SUBS;
+  const int NG = g.L / g.G;
+  uint32_t* err = sc.err;
+
+  // ------------------------------------------------------------------ set-up
+  if (tid == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&bar.a_full[i], 1);
+      mbar_init(&bar.a_empty[i], 2);      // MMA commit + softmax warpgroup
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar.q_full[i], 1);
+      mbar_init(&bar.q_empty[i], 1);
+      mbar_init(&bar.s_full[i], 1);
+      mbar_init(&bar.s_free[i], 4);       // 4 softmax warps
+      mbar_init(&bar.d1_full[i], 1);
+      mbar_init(&bar.h_ready[i], 8);      // 8 epilogue warps
+      mbar_init(&bar.p_ready[i], 1);
+      mbar_init(&bar.d3_full[i], 1);
+      mbar_init(&bar.d3_free[i], 8);
+    }
+    mbar_init(&bar.w1_ready, 8);
+    mbar_init(&bar.drain, 1);
+    misc->abort_flag = 0;
+    mbar_init_fence();
+  }
+  // zero both P tiles (rows >= g stay zero for the whole kernel)
+  for (int i = tid; i < 2 * Lay::P_BUF / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(smem + Lay::OFF_P)[i] = make_uint4(0, 0, 0, 0);
+  fence_proxy_async_smem();
+  if (warp == 1) {
+    tmem_alloc(&misc->tmem_base, Lay::TMEM_COLS);
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc->tmem_base;
+
+  const uint32_t sA = smem_u32(smem + Lay::OFF_A);
+  const uint32_t sQ = smem_u32(smem + Lay::OFF_Q);
+  const uint32_t sP = smem_u32(smem + Lay::OFF_P);
+  constexpr uint32_t IDESC_S = idesc_f16(128, 16, 1, 1);    // bf16 x bf16
+  constexpr uint32_t IDESC_1 = idesc_f16(128, 64, 1, 1);    // bf16 (TMEM) x bf16
+  constexpr uint32_t IDESC_3 = idesc_f16(128, 16, 0, 0);    // f16 (TMEM) x f16
+
+  if (warp == 0) {
+    // ============================================================ TMA producer
+    if (lane == 0 && NCH > 0) {
+      int unit_i = -1, prev_u = -1, issued = 0, q_issued = 0;
+      for (int ci = 0; ci < NCH; ++ci) {
+        const long long x = x0 + ci;
+        const int u = (int)(x / g.k);
+        if (u != prev_u) {
+          ++unit_i;
+          prev_u = u;
+          const int qb = unit_i & 1;
+          if (unit_i >= 2 && !mbar_wait(&bar.q_empty[qb], ((unit_i >> 1) - 1) & 1, abort_flag, err, ERR_TIMEOUT))
+            break;
+          mbar_expect_tx(&bar.q_full[qb], 16 * R * 2);
+          for (int ks = 0; ks < KSLABS; ++ks)
+            tma_load_2d(smem + Lay::OFF_Q + qb * Lay::Q_BUF + ks * 2048, &tmQ, &bar.q_full[qb], ks * 64, u * 16);
+          q_issued = unit_i + 1;
+        }
+        const int st = ci % STAGES;
+        if (ci >= STAGES && !mbar_wait(&bar.a_empty[st], ((ci / STAGES) - 1) & 1, abort_flag, err, ERR_TIMEOUT))
+          break;
+        const Unit un = unit_of(g, u);
+        const int l = g.layer0 + un.li;
+        const int grp = l / g.G;
+        const int slot = sc.sel_slot[x];
+        const int row0 = (int)(((((long long)un.b * NG + grp) * g.Hkv + un.hkv) * g.nL + slot) * C);
+        const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nL + 1);
+        const int r0 = rptr[slot], r1 = rptr[slot + 1];
+        const int nres = min(r1 - r0, Lay::RES_CAP);
+        mbar_expect_tx(&bar.a_full[st], (uint32_t)(C * R * 2 + nres * kDh * 2));
+        for (int ks = 0; ks < KSLABS; ++ks)
+          tma_load_2d(smem + Lay::OFF_A + st * Lay::A_STAGE + ks * 16384, &tmA, &bar.a_full[st], ks * 64, row0);
+        if (nres > 0)
+          bulk_load(smem + Lay::OFF_RES + st * Lay::RES_BUF,
+                    reinterpret_cast<const unsigned char*>(cb.res_val) + (size_t)r0 * kDh * 2,
+                    (uint32_t)(nres * kDh * 2), &bar.a_full[st]);
+        issued = ci + 1;
+      }
+      if (*abort_flag) {
+        // let every copy this thread started land before the CTA's shared memory goes away
+        volatile int never = 0;
+        for (int ci = max(0, issued - STAGES); ci < issued; ++ci)
+          mbar_wait(&bar.a_full[ci % STAGES], (ci / STAGES) & 1, &never, err, ERR_TIMEOUT);
+        for (int ui = max(0, q_issued - 2); ui < q_issued; ++ui)
+          mbar_wait(&bar.q_full[ui & 1], (ui >> 1) & 1, &never, err, ERR_TIMEOUT);
+      }
+    }
+  } else if (warp == 1) {
+    // ============================================================ MMA issuer
+    if (lane == 0 && NS > 0) {
+      int m_unit_i = -1, m_cur_u = -1, m_seg_i = -1, m_cur_seg = -1;
+      auto a_slab = [&](int st, int kk) -> uint32_t {
+        return sA + st * Lay::A_STAGE + (kk >> 2) * 16384 + (kk & 3) * 32;
+      };
+      auto issue_mma1 = [&](int n) -> bool {
+        const int ci = n / SUBS, sub = n % SUBS;
+        const long long x = x0 + ci;
+        const int u = (int)(x / g.k);
+        const int st = ci % STAGES;
+        if (sub == 0) {
+          if (!mbar_wait(&bar.a_full[st], (ci / STAGES) & 1, abort_flag, err, ERR_TIMEOUT)) return false;
+          if (u != m_cur_u) {
+            if (m_cur_u >= 0) mma_commit(&bar.q_empty[m_unit_i & 1]);
+            ++m_unit_i;
+            m_cur_u = u;
+            if (!mbar_wait(&bar.q_full[m_unit_i & 1], (m_unit_i >> 1) & 1, abort_flag, err, ERR_TIMEOUT))
+              return false;
+            const int seg = u / g.B;
+            if (seg != m_cur_seg) {
+              ++m_seg_i;
+              m_cur_seg = seg;
+              if (!mbar_wait(&bar.w1_ready, m_seg_i & 1, abort_flag, err, ERR_TIMEOUT)) return false;
+            }
+          }
+          const int sb = ci & 1;
+          if (ci >= 2 && !mbar_wait(&bar.s_free[sb], ((ci >> 1) - 1) & 1, abort_flag, err, ERR_TIMEOUT))
+            return false;
+          tc_fence_after();
+          const uint32_t qbase = sQ + (m_unit_i & 1) * Lay::Q_BUF;
+#pragma unroll
+          for (int kk = 0; kk < R / 16; ++kk) {
+            const uint64_t ad = smem_desc(a_slab(st, kk), 16, 1024, 2);
+            const uint64_t bd = smem_desc(qbase + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, 2);
+            mma_ss(tmem + Lay::T_S + sb * 16, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bar.s_full[sb]);
+        } else {
+          tc_fence_after();
+        }
+        const int b = n & 1;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+          for (int kk = 0; kk < R / 16; ++kk) {
+            const uint64_t bd = smem_desc(a_slab(st, kk) + sub * 8192, 16, 1024, 2);
+            mma_ts(tmem + Lay::T_D1 + (b * 2 + hh) * 64, tmem + Lay::T_W1 + hh * (R / 2) + kk * 8, bd,
+                   IDESC_1, kk > 0 ? 1u : 0u);
+          }
+        }
+        mma_commit(&bar.d1_full[b]);
+        if (sub == SUBS - 1) mma_commit(&bar.a_empty[st]);
+        return true;
+      };
+
+      bool ok = issue_mma1(0);
+      if (ok && NS > 1) ok = issue_mma1(1);
+      for (int n = 0; ok && n < NS; ++n) {
+        const int ci = n / SUBS, sub = n % SUBS, b = n & 1, pb = ci & 1;
+        if (!mbar_wait(&bar.h_ready[b], (n >> 1) & 1, abort_flag, err, ERR_TIMEOUT)) break;
+        if (sub == 0) {
+          if (!mbar_wait(&bar.p_ready[pb], (ci >> 1) & 1, abort_flag, err, ERR_TIMEOUT)) break;
+          if (ci >= 2 && !mbar_wait(&bar.d3_free[pb], ((ci >> 1) - 1) & 1, abort_flag, err, ERR_TIMEOUT)) break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = smem_desc(sP + pb * Lay::P_BUF + sub * 1024 + kk * 256, 128, Lay::P_SBO, 0);
+            mma_ts(tmem + Lay::T_D3 + (pb * 2 + hh) * 16, tmem + Lay::T_D1 + (b * 2 + hh) * 64 + kk * 8, bd,
+                   IDESC_3, (sub > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        if (sub == SUBS - 1) mma_commit(&bar.d3_full[pb]);
+        if (n + 2 < NS) ok = issue_mma1(n + 2);
+      }
+      // every MMA this thread issued must finish before TMEM is released
+      mma_commit(&bar.drain);
+      volatile int never = 0;
+      mbar_wait(&bar.drain, 0, &never, err, ERR_TIMEOUT);
+    }
+  } else if (warp >= 2 && warp < 10) {
+    // ============================================================ hidden-row epilogue
+    const int hh = (warp - 2) >> 2;
+    const int wl = warp & 3;
+    const int row = wl * 32 + lane;              // hidden unit inside the half
+    const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
+    float accH[GQ];
+#pragma unroll
+    for (int j = 0; j < GQ; ++j) accH[j] = 0.f;
+    int cur_u = -1, cur_seg = -1, pending_c = -1;
+    bool ok = true;
+
+    auto process_d3 = [&](int c) -> bool {
+      const int pb = c & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.d3_full[pb], (c >> 1) & 1, abort_flag, err, ERR_TIMEOUT)))
+        return false;
+      tc_fence_after();
+      uint32_t v[16];
+      tmem_ld16(tmem + lane_off + Lay::T_D3 + (pb * 2 + hh) * 16, v);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.d3_free[pb]);
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) accH[j] = fmaf(accH[j], misc->alpha[c & 3][j], __uint_as_float(v[j]));
+      return true;
+    };
+    auto write_partial = [&](int u) {
+      float* rec = sc.part + (size_t)(u + blockIdx.x) * g.rec_stride + 2 * GQ;
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) {
+        rec[j * kHid + hh * 128 + row] = accH[j];
+        accH[j] = 0.f;
+      }
+    };
+
+    for (int n = 0; ok && n < NS; ++n) {
+      const int ci = n / SUBS, sub = n % SUBS;
+      const long long x = x0 + ci;
+      const int u = (int)(x / g.k);
+      if (sub == 0 && u != cur_u) {
+        const int seg = u / g.B;
+        if (seg != cur_seg) {
+          // the previous segment's MMAs are complete (its last D1 was observed): swap W1'
+          const Unit un = unit_of(g, u);
+          const int l = g.layer0 + un.li;
+          const uint4* src = reinterpret_cast<const uint4*>(
+              w1f + (((size_t)l * g.Hkv + un.hkv) * kHid + hh * 128 + row) * R);
+#pragma unroll
+          for (int half = 0; half < R / 64; ++half) {
+            uint32_t w[32];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint4 q = __ldg(src + half * 8 + i);
+              w[4 * i] = q.x; w[4 * i + 1] = q.y; w[4 * i + 2] = q.z; w[4 * i + 3] = q.w;
+            }
+            tmem_st32(tmem + lane_off + Lay::T_W1 + hh * (R / 2) + half * 32, w);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar.w1_ready);
+          cur_seg = seg;
+        }
+        if (cur_u >= 0) {
+          if (pending_c >= 0) {
+            if (!process_d3(pending_c)) { ok = false; break; }
+            pending_c = -1;
+          }
+          write_partial(cur_u);
+        }
+        cur_u = u;
+      }
+      const int b = n & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.d1_full[b], (n >> 1) & 1, abort_flag, err, ERR_TIMEOUT))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t dcol = tmem + lane_off + Lay::T_D1 + (b * 2 + hh) * 64;
+      uint32_t h[32];
+      {
+        uint32_t v[32];
+        tmem_ld32(dcol, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          h[c] = silu_half2_of_halfx(pack_f16x2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])));
+        tmem_ld32(dcol + 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          h[16 + c] = silu_half2_of_halfx(pack_f16x2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])));
+      }
+      tmem_st32(dcol, h);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.h_ready[b]);
+      if (sub == 0 && pending_c >= 0) {
+        if (!process_d3(pending_c)) { ok = false; break; }
+        pending_c = -1;
+      }
+      if (sub == SUBS - 1) pending_c = ci;
+    }
+    if (ok && pending_c >= 0) ok = process_d3(pending_c);
+    if (ok && cur_u >= 0) write_partial(cur_u);
+  } else if (warp >= 10) {
+    // ============================================================ softmax + residuals
+    const int w = warp & 3;
+    const int t = w * 32 + lane;                 // token (scores) and head-dim index (residuals)
+    const uint32_t lane_off = (uint32_t)(w * 32) << 16;
+    float m_run[GQ], l_run[GQ], accD[GQ];
+#pragma unroll
+    for (int j = 0; j < GQ; ++j) { m_run[j] = -INFINITY; l_run[j] = 0.f; accD[j] = 0.f; }
+    float* p32_base = reinterpret_cast<float*>(smem + Lay::OFF_P32);
+    unsigned char* pbase = smem + Lay::OFF_P;
+    int cur_u = -1;
+    auto write_partial = [&](int u) {
+      float* rec = sc.part + (size_t)(u + blockIdx.x) * g.rec_stride;
+      if (t == 0) {
+#pragma unroll
+        for (int j = 0; j < GQ; ++j) { rec[j] = m_run[j]; rec[GQ + j] = l_run[j]; }
+      }
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) {
+        rec[2 * GQ + GQ * kHid + j * kDh + t] = accD[j];
+        m_run[j] = -INFINITY; l_run[j] = 0.f; accD[j] = 0.f;
+      }
+    };
+    // After a failed wait a warp stops working ("live" false) but keeps passing the named
+    // barriers of every remaining chunk, so the other warps of the group never block on it;
+    // once the abort flag is up every wait returns at once.
+    bool live = true;
+    for (int ci = 0; ci < NCH; ++ci) {
+      const long long x = x0 + ci;
+      const int u = (int)(x / g.k);
+      if (u != cur_u) {
+        if (cur_u >= 0 && live) write_partial(cur_u);
+        cur_u = u;
+      }
+      const int st = ci % STAGES, sb = ci & 1, pb = ci & 1;
+      live = __all_sync(0xffffffffu, live && mbar_wait(&bar.a_full[st], (ci / STAGES) & 1, abort_flag, err, ERR_TIMEOUT) &&
+                                         mbar_wait(&bar.s_full[sb], (ci >> 1) & 1, abort_flag, err, ERR_TIMEOUT));
+      uint32_t sv[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) sv[j] = 0u;
+      if (live) {
+        tc_fence_after();
+        tmem_ld16(tmem + lane_off + Lay::T_S + sb * 16, sv);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar.s_free[sb]);
+      }
+      const bool valid = t < C;
+      float p[GQ], al[GQ];
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) {
+        const float s = valid ? __uint_as_float(sv[j]) : -INFINITY;
+        const float m = warp_max(s);
+        if (lane == 0) misc->red_max[w][j] = m;
+        p[j] = s;
+      }
+      named_bar_sync(1, 128);
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) {
+        const float mc = fmaxf(fmaxf(misc->red_max[0][j], misc->red_max[1][j]),
+                               fmaxf(misc->red_max[2][j], misc->red_max[3][j]));
+        const float mn = fmaxf(m_run[j], mc);
+        al[j] = exp2f(m_run[j] - mn);
+        p[j] = exp2f(p[j] - mn);
+        m_run[j] = mn;
+      }
+      // the P buffer is free once the MMAs of chunk ci-2 that read it are done
+      live = __all_sync(0xffffffffu,
+                        live && (ci < 2 || mbar_wait(&bar.d3_full[pb], ((ci - 2) >> 1) & 1, abort_flag, err, ERR_TIMEOUT)));
+      float* p32 = p32_base + pb * 16 * C;
+      if (valid && live) {
+#pragma unroll
+        for (int j = 0; j < GQ; ++j) {
+          const uint32_t off = (j >> 3) * Lay::P_SBO + (t >> 3) * 128 + (j & 7) * 16 + (t & 7) * 2;
+          *reinterpret_cast<__half*>(pbase + pb * Lay::P_BUF + off) = __float2half_rn(p[j]);
+          p32[j * C + t] = p[j];
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) {
+        const float s = warp_sum(p[j]);
+        if (lane == 0) misc->red_sum[w][j] = s;
+      }
+      // alpha of chunk ci is read by the epilogue warps after D3(ci) completes, which is
+      // before this warpgroup reaches chunk ci+4 (it waits for D3(ci+2) there): a ring of 4
+      if (t == 0) {
+#pragma unroll
+        for (int j = 0; j < GQ; ++j) misc->alpha[ci & 3][j] = al[j];
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (t == 0 && live) mbar_arrive(&bar.p_ready[pb]);
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) {
+        l_run[j] = l_run[j] * al[j] + misc->red_sum[0][j] + misc->red_sum[1][j] +
+                   misc->red_sum[2][j] + misc->red_sum[3][j];
+        accD[j] *= al[j];
+      }
+      // residual rows of the chunk's flagged tokens: thread t owns head-dim element t
+      if (live) {
+        const Unit un = unit_of(g, u);
+        const int l = g.layer0 + un.li;
+        const int slot = sc.sel_slot[x];
+        const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nL + 1);
+        const int r0 = rptr[slot], r1 = rptr[slot + 1];
+        const uint16_t* rs = reinterpret_cast<const uint16_t*>(smem + Lay::OFF_RES + st * Lay::RES_BUF);
+        const uint16_t* rg = reinterpret_cast<const uint16_t*>(cb.res_val);
+        for (int rec = r0; rec < r1; ++rec) {
+          const int pos = cb.res_pos[rec];
+          const int i = rec - r0;
+          const float dv = i < Lay::RES_CAP ? bf16_bits_to_f(rs[i * kDh + t])
+                                            : bf16_bits_to_f(rg[(size_t)rec * kDh + t]);
+#pragma unroll
+          for (int j = 0; j < GQ; ++j) accD[j] = fmaf(p32[j * C + pos], dv, accD[j]);
+        }
+      }
+      named_bar_sync(1, 128);
+      if (t == 0 && live) mbar_arrive(&bar.a_empty[st]);
+    }
+    if (live && !*abort_flag && cur_u >= 0) write_partial(cur_u);
+  }
+
+  // ------------------------------------------------------------------ teardown
+  __syncwarp();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, Lay::TMEM_COLS);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int R, int C, int GQ>
+cudaError_t launch_tc(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const void* w1f,
+                      cudaStream_t s) {
+  using Lay = TcLayout<R, C>;
+  const int NG = g.L / g.G;
+  const uint64_t rows = (uint64_t)g.B * NG * g.Hkv * g.nL * C;
+  CUtensorMap tmA, tmQ;
+  if (!make_map(&tmA, cb.coeff, R, rows, C)) return cudaErrorInvalidValue;
+  if (!make_map(&tmQ, sc.qt_tc, R, (uint64_t)g.U * 16, 16)) return cudaErrorInvalidValue;
+  auto k = attend_tc_kernel<R, C, GQ>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
+  if (e != cudaSuccess) return e;
+  k<<<g.P, kThreadsTC, Lay::SMEM, s>>>(g, cb, sc, static_cast<const __nv_bfloat16*>(w1f), tmA, tmQ);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attend_tc_supported(const Geom& g, int dtype, int store) {
+  if (dtype != LOWRAM_BF16 || store != LOWRAM_STORE_NATIVE) return false;
+  if (g.d != kDh || g.h != kHid || !(g.g == 4 || g.g == 8)) return false;
+  if (!(g.r == 64 || g.r == 128) || !(g.C == 64 || g.C == 128)) return false;
+  const uint64_t rows = (uint64_t)g.B * (g.L / g.G) * g.Hkv * g.nL * g.C;
+  if (rows >= (1ull << 31) || (uint64_t)g.U * 16 >= (1ull << 31)) return false;
+  return encode_fn() != nullptr;
+}
+
+cudaError_t launch_attend_tc(const Geom& g, const CacheBuffers& cb, const Scratch& sc, int store,
+                             const void* w1f_tc, int n_sm, cudaStream_t s) {
+  (void)n_sm;
+  if (store != LOWRAM_STORE_NATIVE) return cudaErrorNotSupported;
+#define LOWRAM_TC_CASE(RR, CC, GG) \
+  if (g.r == RR && g.C == CC && g.g == GG) return launch_tc<RR, CC, GG>(g, cb, sc, w1f_tc, s);
+  LOWRAM_TC_CASE(128, 128, 4)
+  LOWRAM_TC_CASE(128, 64, 4)
+  LOWRAM_TC_CASE(64, 128, 4)
+  LOWRAM_TC_CASE(64, 64, 4)
+  LOWRAM_TC_CASE(128, 128, 8)
+  LOWRAM_TC_CASE(128, 64, 8)
+  LOWRAM_TC_CASE(64, 128, 8)
+  LOWRAM_TC_CASE(64, 64, 8)
+#undef LOWRAM_TC_CASE
   return cudaErrorNotSupported;
 }
 

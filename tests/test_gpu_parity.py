@@ -50,7 +50,10 @@ def test_tiny_f32_every_unit(path):
     check(cfg, _oracle(cache), q, out, sel, scores=scores)
 
 
-@pytest.mark.parametrize("path", [K.PATH_AUTO, K.PATH_SIMT])
+ALL_PATHS = [K.PATH_AUTO, K.PATH_SIMT, K.PATH_TC]
+
+
+@pytest.mark.parametrize("path", ALL_PATHS)
 def test_mistral_group_bf16_every_unit(path):
     cfg = S.MISTRAL_GROUP
     cache = S.make_cache(cfg)
@@ -59,7 +62,7 @@ def test_mistral_group_bf16_every_unit(path):
     check(cfg, _oracle(cache), q, out, sel, scores=scores)
 
 
-@pytest.mark.parametrize("path", [K.PATH_AUTO, K.PATH_SIMT])
+@pytest.mark.parametrize("path", ALL_PATHS)
 def test_sharp_queries_strict_selection(path):
     """Peaky softmax and well-separated chunk scores: the exact-selection rule applies."""
     cfg = S.MISTRAL_GROUP
@@ -70,7 +73,7 @@ def test_sharp_queries_strict_selection(path):
     assert res["strict_selection_units"] >= res["units"] // 2
 
 
-@pytest.mark.parametrize("path", [K.PATH_AUTO, K.PATH_SIMT])
+@pytest.mark.parametrize("path", ALL_PATHS)
 def test_ragged_tail_select_all_full_residuals(path):
     cfg = _small("mistral7b_group_bf16", batch=3, n_ctx=1024, top_k=16, resid_frac=1.0,
                  tail_cap=64)
@@ -81,13 +84,33 @@ def test_ragged_tail_select_all_full_residuals(path):
     assert (sel.cpu() == torch.arange(16, dtype=torch.int32)).all()
 
 
-@pytest.mark.parametrize("path", [K.PATH_AUTO, K.PATH_SIMT])
+@pytest.mark.parametrize("path", ALL_PATHS)
 def test_top1_and_no_residuals(path):
     cfg = _small("mistral7b_group_bf16", n_ctx=2048, top_k=1, resid_frac=0.0)
     cache = S.make_cache(cfg)
     q = S.make_queries(cache)
     out, sel, scores, _ = _run(cache, q, path)
     check(cfg, _oracle(cache), q, out, sel, scores=scores)
+
+
+@pytest.mark.parametrize("path", ALL_PATHS)
+def test_tail_longer_than_block_and_many_units(path):
+    """Four sequences with the 32K shape cut to 8K context: 64 units x 32 chunks spread over
+    every SM, units straddling CTA ranges, tails of 128, 0, 1 and 77 tokens."""
+    cfg = S.LLAMA_32K.replace(name="llama_8k", n_ctx=8192, n_layers=4, top_k=32)
+    cache = S.make_cache(cfg, tail_len=[128, 0, 1, 77])
+    q = S.make_queries(cache)
+    out, sel, scores, p = _run(cache, q, path)
+    if path == K.PATH_TC:
+        assert p == K.PATH_TC
+    check(cfg, _oracle(cache), q, out, sel, scores=scores)
+
+
+def test_auto_picks_tensor_cores_for_bf16():
+    cache = S.make_cache(S.MISTRAL_GROUP)
+    q = S.make_queries(cache)
+    _, _, _, p = _run(cache, q, K.PATH_AUTO)
+    assert p == K.PATH_TC
 
 
 def test_odd_shapes_f32():
@@ -159,7 +182,7 @@ def llama32k():
     return cfg, cache
 
 
-@pytest.mark.parametrize("path", [K.PATH_AUTO, K.PATH_SIMT])
+@pytest.mark.parametrize("path", ALL_PATHS)
 def test_llama_32k_all_layers_sampled(llama32k, path):
     cfg, cache = llama32k
     q = S.make_queries(cache)
