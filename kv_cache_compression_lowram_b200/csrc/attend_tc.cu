@@ -18,8 +18,8 @@
 // Asymmetrically", section "Cross-Layer Low-Rank Key Compression"; values: same page,
 // "Core Mechanism" (Vhat = f(K), delta kept for the worst tokens); attention: "OjaKV", 3.
 //
-// Warp roles (14 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-5 and 6-9 the
-// two hidden-row halves (silu epilogue, D3 accumulation), 10-13 softmax + residuals.
+// Warp roles (16 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-3 idle, 4-7 and 8-11
+// the two hidden-row halves (silu epilogue, D3 accumulation), 12-15 softmax + residuals.
 // A warp reaches TMEM lanes 32*(warp%4) .. +31, so each warpgroup of four consecutive
 // warps covers all 128 lanes.
 // TMEM (512 columns): W1' halves [0,128), D1 double buffer x 2 halves [128,384),
@@ -37,7 +37,9 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreadsTC = 448;   // 14 warps
+constexpr int kThreadsTC = 512;   // 16 warps: register allocation rounds to whole warpgroups
+constexpr int kEpiWarp0 = 4;      // first hidden-row epilogue warp
+constexpr int kSoftWarp0 = 12;    // first softmax warp
 constexpr int kHid = 256;
 constexpr int kDh = 128;
 
@@ -96,7 +98,7 @@ __device__ __forceinline__ float bf16_bits_to_f(uint16_t b) {
 }
 
 template <int R, int C, int GQ>
-__global__ void __maxnreg__(144)
+__global__ void __launch_bounds__(kThreadsTC, 1)
 attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __restrict__ w1f,
                  const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmQ) {
   using Lay = TcLayout<R, C>;
@@ -289,9 +291,9 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       volatile int never = 0;
       mbar_wait(&bar.drain, 0, &never, err, ERR_TIMEOUT);
     }
-  } else if (warp >= 2 && warp < 10) {
+  } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 8) {
     // ============================================================ hidden-row epilogue
-    const int hh = (warp - 2) >> 2;
+    const int hh = (warp - kEpiWarp0) >> 2;
     const int wl = warp & 3;
     const int row = wl * 32 + lane;              // hidden unit inside the half
     const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
@@ -396,7 +398,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
     }
     if (ok && pending_c >= 0) ok = process_d3(pending_c);
     if (ok && cur_u >= 0) write_partial(cur_u);
-  } else if (warp >= 10) {
+  } else if (warp >= kSoftWarp0) {
     // ============================================================ softmax + residuals
     const int w = warp & 3;
     const int t = w * 32 + lane;                 // token (scores) and head-dim index (residuals)
