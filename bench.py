@@ -74,13 +74,31 @@ def barrier(ws):
         dist.barrier()
 
 
-def max_over_ranks(x: float, ws: int) -> float:
+def _reduce(x: float, ws: int, op: str) -> float:
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    """The slowest rank's time (every multi-GPU number is timed as the max over ranks)."""
+    return _reduce(x, ws, "max")
+
+
+def replica_config(cfg, rank: int):
+    """Each rank decodes its own replica of the workload (own seed): no data-path exchange."""
+    return cfg if rank == 0 else cfg.replace(seed=cfg.seed + 7919 * rank)
+
+
+def aggregate_rate(queries_per_rank: float, ms_total: float, ws: int):
+    """Whole-job throughput: all ranks' queries over the slowest rank's time."""
+    ms = max_over_ranks(ms_total, ws)
+    total_q = _reduce(queries_per_rank, ws, "sum")
+    return total_q / (ms / 1e3), ms
 
 
 def peaks():
@@ -230,9 +248,7 @@ def oracle_rate(cfg, cache, q, budget_s: float = 15.0, seed: int = 0):
 
 def run_lowram(args, ws, rank, local):
     import kv_cache_compression_lowram_b200 as K
-    cfg = S.CONFIGS[args.config]
-    if rank > 0:
-        cfg = cfg.replace(seed=cfg.seed + 7919 * rank)
+    cfg = replica_config(S.CONFIGS[args.config], rank)
     dev = torch.device("cuda", local)
     torch.manual_seed(0)
     cache = S.make_cache(cfg, device=dev)
@@ -266,8 +282,8 @@ def run_lowram(args, ws, rank, local):
     barrier(ws)
     clk = clocks.stop()
     K.lowram_cache_set_stage_events(lc.handle, None)
-    ms_total = start.elapsed_time(end)
-    ms_total = max_over_ranks(ms_total, ws)
+    queries_step = cfg.batch * cfg.n_layers
+    value, ms_total = aggregate_rate(queries_step * args.steps, start.elapsed_time(end), ws)
     ms_step = ms_total / args.steps
     stage_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(3)]
 
@@ -285,8 +301,6 @@ def run_lowram(args, ws, rank, local):
     e2e_ms = (time.perf_counter() - t0) * 1e3 / e2e_steps
     e2e_ms = max_over_ranks(e2e_ms, ws)
 
-    queries_step = cfg.batch * cfg.n_layers
-    value = queries_step * ws / (ms_step / 1e3)
     host = {"res_ptr": cache.res_ptr.cpu().numpy(), "slot": cache.slot.cpu().numpy().astype(np.int64),
             "tail_len": cache.tail_len.cpu().numpy()}
     ab = algorithmic_bytes(cfg, host, sel.cpu().numpy(), 0, cfg.n_layers)
