@@ -236,6 +236,36 @@ int32_t lowram_cache_last_launches(const lowram_cache* cache);
 /* Which path the last lowram_decode_attn call on this cache ran (a lowram_path value). */
 int32_t lowram_cache_last_path(const lowram_cache* cache);
 
+/* Decode-time attention with no device allocation at all, for callers that cannot call
+ * cudaMalloc on their decode path (an engine that reserves all device memory for its own
+ * pool, a runtime that forbids allocation after start-up, a thread capturing a CUDA graph
+ * in a mode that rejects allocation calls).  The pages have no counterpart of this entry
+ * point; it is a deployment variant of lowram_decode_attn.
+ *
+ * It reads the compressed cache straight from the caller's DEVICE arrays `src` (layouts of
+ * lowram_cache_src, no copy, no cache object), runs the CUDA-core decode kernels for layers
+ * [layer0, layer0 + n_layers) and writes out / sel exactly like lowram_decode_attn (q, out,
+ * sel: DEVICE, layouts as there).  All scratch -- the folded W1' of the requested layers,
+ * the projected queries, the selection, the split partials and an error word -- lives in
+ * one static device array of 16 MiB inside the library, which every GPU that loads the
+ * library holds until the process exits.
+ *
+ * Limits and behaviour:
+ *  - A call whose scratch exceeds 16 MiB is rejected with LOWRAM_EINVAL and a message giving
+ *    the bytes needed (for the 32K Llama-shaped cache: one to three layers per call fit).
+ *  - It calls no cudaMalloc, cudaFree or allocating library routine.
+ *  - The first call on a device looks up the array's device address with
+ *    cudaGetSymbolAddress (once per device, with that device current); make that first call
+ *    before any stream capture.
+ *  - Every call shares the array, which keeps the last call's contents (the error word is
+ *    cleared at the start of each call): calls that overlap on the GPU -- on two streams,
+ *    or on the same device from two threads -- race and must be serialised by the caller.
+ *  - Stream-ordered on `stream`, no host synchronisation; same error codes as
+ *    lowram_decode_attn. */
+lowram_status lowram_decode_attn_static(const lowram_config* cfg, const lowram_cache_src* src,
+                                        int32_t layer0, int32_t n_layers, const void* q,
+                                        void* out, int32_t* sel, lowram_stream stream);
+
 const char* lowram_status_string(lowram_status status);
 const char* lowram_last_error_string(void);
 

@@ -24,7 +24,7 @@ __all__ = [
     "lowram_cache_destroy", "lowram_decode_attn", "lowram_select_chunks",
     "lowram_decode_attn_host", "lowram_cache_bytes", "lowram_cache_validate",
     "lowram_cache_set_stage_events", "lowram_cache_last_launches", "lowram_cache_last_path",
-    "LowramCache", "config_struct",
+    "LowramCache", "config_struct", "lowram_decode_attn_static",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblowram.so")
@@ -85,6 +85,8 @@ def lib() -> ctypes.CDLL:
         "lowram_cache_set_stage_events": (I32, [P, P]),
         "lowram_cache_last_launches": (I32, [P]),
         "lowram_cache_last_path": (I32, [P]),
+        "lowram_decode_attn_static": (I32, [ctypes.POINTER(LowramConfigC), ctypes.POINTER(LowramSrcC),
+                                            I32, I32, P, P, P, P]),
         "lowram_status_string": (ctypes.c_char_p, [I32]),
         "lowram_last_error_string": (ctypes.c_char_p, []),
     }
@@ -164,10 +166,7 @@ def lowram_config_bytes(cfg, n_records: int, has_slot: bool = True) -> dict:
     return _bytes_dict(out)
 
 
-def lowram_cache_create(cfg, arrays, stream=None) -> int:
-    """Create a cache from device tensors.  ``arrays`` is a mapping (or an object with
-    attributes) holding coeff, coeff_scale, basis, w1, w2, summary, slot, res_ptr, res_pos,
-    res_val, res_scale, tail_k, tail_v, tail_len (layouts of ``lowram.h``)."""
+def _src_struct(arrays):
     src = LowramSrcC()
     names = ("coeff", "coeff_scale", "basis", "w1", "w2", "summary", "slot", "res_ptr",
              "res_pos", "res_val", "res_scale", "tail_k", "tail_v", "tail_len")
@@ -183,6 +182,14 @@ def lowram_cache_create(cfg, arrays, stream=None) -> int:
         setattr(src, n, _ptr(t))
     rp = _get(arrays, "res_pos")
     src.n_records = int(rp.shape[0]) if rp is not None else 0
+    return src, keep
+
+
+def lowram_cache_create(cfg, arrays, stream=None) -> int:
+    """Create a cache from device tensors.  ``arrays`` is a mapping (or an object with
+    attributes) holding coeff, coeff_scale, basis, w1, w2, summary, slot, res_ptr, res_pos,
+    res_val, res_scale, tail_k, tail_v, tail_len (layouts of ``lowram.h``)."""
+    src, keep = _src_struct(arrays)
     c = config_struct(cfg)
     h = ctypes.c_void_p()
     _check(lib().lowram_cache_create(ctypes.byref(c), ctypes.byref(src), ctypes.byref(h),
@@ -212,6 +219,17 @@ def lowram_decode_attn_host(handle: int, layer0: int, n_layers: int, q_host, out
     _check(lib().lowram_decode_attn_host(handle, layer0, n_layers, _ptr(q_host), _ptr(out_host),
                                          _ptr(sel_host), _stream(stream)),
            "lowram_decode_attn_host")
+
+
+def lowram_decode_attn_static(cfg, arrays, layer0: int, n_layers: int, q, out, sel=None,
+                              stream=None) -> None:
+    """Decode straight from the caller's device arrays with no device allocation (the
+    library's static scratch; see ``lowram.h``)."""
+    src, keep = _src_struct(arrays)
+    c = config_struct(cfg)
+    _check(lib().lowram_decode_attn_static(ctypes.byref(c), ctypes.byref(src), layer0, n_layers,
+                                           _ptr(q), _ptr(out), _ptr(sel), _stream(stream)),
+           "lowram_decode_attn_static")
 
 
 def lowram_cache_bytes(handle: int) -> dict:

@@ -128,6 +128,11 @@ lowram_status alloc(lowram_cache* c, P** out, size_t bytes) {
 
 }  // namespace
 
+namespace lowram {
+// Sets the calling thread's text returned by lowram_last_error_string (for other files).
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace lowram
+
 extern "C" {
 
 uint64_t lowram_dense_kv_bytes(int32_t n_layers, int32_t n_kv_heads, int32_t head_dim,
