@@ -71,6 +71,7 @@ struct TcLayout {
   static constexpr uint32_t T_D3 = 416;
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(R / 2 <= 64, "W1' half must fit 64 TMEM columns");
+  static_assert(STAGES == 4 && RES_CAP <= 32, "Misc holds 4 stages of at most 32 positions");
 };
 
 struct Bars {
@@ -86,12 +87,17 @@ struct Bars {
 
 struct Misc {
   Bars bars;
+  int stage_rec[4][2];               // residual record range [r0, r1) of the chunk in a stage
+  uint16_t stage_pos[4][32];         // token offsets of its first RES_CAP records
   float alpha[4][16];   // per-chunk rescale factors, ring of 4 (see the softmax warpgroup)
   float red_max[4][16];
   float red_sum[4][16];
   uint32_t tmem_base;
   int abort_flag;
 };
+
+static_assert(sizeof(Misc) <= 2048, "Misc must fit its shared-memory slot");
+static_assert(sizeof(((Misc*)0)->stage_rec) / sizeof(int[2]) == 4, "one record range per stage");
 
 __device__ __forceinline__ float bf16_bits_to_f(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);
@@ -189,6 +195,10 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
         const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nL + 1);
         const int r0 = rptr[slot], r1 = rptr[slot + 1];
         const int nres = min(r1 - r0, Lay::RES_CAP);
+        // record range and positions for the softmax warpgroup (published by the arrive below)
+        misc->stage_rec[st][0] = r0;
+        misc->stage_rec[st][1] = r1;
+        for (int i = 0; i < nres; ++i) misc->stage_pos[st][i] = cb.res_pos[r0 + i];
         mbar_expect_tx(&bar.a_full[st], (uint32_t)(C * R * 2 + nres * kDh * 2));
         for (int ks = 0; ks < KSLABS; ++ks)
           tma_load_2d(smem + Lay::OFF_A + st * Lay::A_STAGE + ks * 16384, &tmA, &bar.a_full[st], ks * 64, row0);
@@ -497,20 +507,24 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
                    misc->red_sum[2][j] + misc->red_sum[3][j];
         accD[j] *= al[j];
       }
-      // residual rows of the chunk's flagged tokens: thread t owns head-dim element t
+      // residual rows of the chunk's flagged tokens: thread t owns head-dim element t.
+      // The producer left the record range and positions in shared memory with the rows.
       if (live) {
-        const Unit un = unit_of(g, u);
-        const int l = g.layer0 + un.li;
-        const int slot = sc.sel_slot[x];
-        const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nL + 1);
-        const int r0 = rptr[slot], r1 = rptr[slot + 1];
+        const int r0 = misc->stage_rec[st][0], r1 = misc->stage_rec[st][1];
+        const int n = r1 - r0, nfast = min(n, Lay::RES_CAP);
         const uint16_t* rs = reinterpret_cast<const uint16_t*>(smem + Lay::OFF_RES + st * Lay::RES_BUF);
+        const uint16_t* sp = misc->stage_pos[st];
+#pragma unroll 4
+        for (int i = 0; i < nfast; ++i) {
+          const int pos = sp[i];
+          const float dv = bf16_bits_to_f(rs[i * kDh + t]);
+#pragma unroll
+          for (int j = 0; j < GQ; ++j) accD[j] = fmaf(p32[j * C + pos], dv, accD[j]);
+        }
         const uint16_t* rg = reinterpret_cast<const uint16_t*>(cb.res_val);
-        for (int rec = r0; rec < r1; ++rec) {
-          const int pos = cb.res_pos[rec];
-          const int i = rec - r0;
-          const float dv = i < Lay::RES_CAP ? bf16_bits_to_f(rs[i * kDh + t])
-                                            : bf16_bits_to_f(rg[(size_t)rec * kDh + t]);
+        for (int i = nfast; i < n; ++i) {   // records beyond the staged ones (rare)
+          const int pos = cb.res_pos[r0 + i];
+          const float dv = bf16_bits_to_f(rg[(size_t)(r0 + i) * kDh + t]);
 #pragma unroll
           for (int j = 0; j < GQ; ++j) accD[j] = fmaf(p32[j * C + pos], dv, accD[j]);
         }

@@ -13,6 +13,22 @@ namespace {
 
 constexpr int kThreads = 256;
 
+// 8 consecutive row elements as floats (one 16-byte load for bf16, two for fp32).
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+__device__ __forceinline__ void load8(const float* p, float (&v)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(Geom g, CacheBuffers cb, Scratch sc, T* __restrict__ out) {
@@ -28,7 +44,7 @@ combine_kernel(Geom g, CacheBuffers cb, Scratch sc, T* __restrict__ out) {
     if (threadIdx.x == 0) atomicOr(sc.err, ERR_SELECT);
     return;
   }
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarp = blockDim.x >> 5;
+  const int tid = threadIdx.x;
 
   float* accH = sm;                   // [g][h]
   float* accD = accH + g.g * g.h;     // [g][d]
@@ -68,26 +84,40 @@ combine_kernel(Geom g, CacheBuffers cb, Scratch sc, T* __restrict__ out) {
     accD[i] = a;
   }
   __syncthreads();
-  // second predictor layer on the weighted hidden sums: one warp per output row dd
+  // second predictor layer on the weighted hidden sums: one thread per (output row dd,
+  // group of up to 4 heads), W2 rows read with 16-byte loads, accH broadcast from smem
   const T* W2 = reinterpret_cast<const T*>(cb.w2) + ((size_t)l * g.Hkv + un.hkv) * g.d * g.h;
   T* o = out + ((size_t)(un.li * g.B + un.b) * g.Hq + (size_t)un.hkv * g.g) * g.d;
-  for (int dd = warp; dd < g.d; dd += nwarp) {
+  const int jgroups = (g.g + 3) / 4;
+  for (int item = tid; item < g.d * jgroups; item += blockDim.x) {
+    const int dd = item % g.d, j0 = (item / g.d) * 4;
     const T* row = W2 + (size_t)dd * g.h;
-    float a[kMaxG];
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    if ((g.h & 7) == 0) {
+      for (int i = 0; i < g.h; i += 8) {
+        float v[8];
+        load8(row + i, v);
 #pragma unroll
-    for (int j = 0; j < kMaxG; ++j) a[j] = 0.f;
-    for (int i = lane; i < g.h; i += 32) {
-      const float w = to_f(row[i]);
+        for (int jj = 0; jj < 4; ++jj) {
+          if (j0 + jj < g.g) {
+            const float* hsum = accH + (j0 + jj) * g.h + i;
 #pragma unroll
-      for (int j = 0; j < kMaxG; ++j)
-        if (j < g.g) a[j] = fmaf(w, accH[j * g.h + i], a[j]);
+            for (int x = 0; x < 8; ++x) a[jj] = fmaf(v[x], hsum[x], a[jj]);
+          }
+        }
+      }
+    } else {
+      for (int i = 0; i < g.h; ++i) {
+        const float v = to_f(row[i]);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+          if (j0 + jj < g.g) a[jj] = fmaf(v, accH[(j0 + jj) * g.h + i], a[jj]);
+      }
     }
 #pragma unroll
-    for (int j = 0; j < kMaxG; ++j) {
-      if (j < g.g) {
-        const float s = warp_sum(a[j]);
-        if (lane == 0) o[(size_t)j * g.d + dd] = from_f<T>((s + accD[j * g.d + dd]) / lsum[j]);
-      }
+    for (int jj = 0; jj < 4; ++jj) {
+      const int j = j0 + jj;
+      if (j < g.g) o[(size_t)j * g.d + dd] = from_f<T>((a[jj] + accD[j * g.d + dd]) / lsum[j]);
     }
   }
 }

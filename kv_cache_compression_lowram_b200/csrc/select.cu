@@ -10,20 +10,25 @@
 // selected subset is reconstructed per step); rit.work "lowram-kv-cache-compression",
 // section "Значения предсказывают, ключи раскладывают по общему базису" (fragments chosen
 // by the current query; new tokens kept uncompressed).  Ties go to the lower chunk id.
+//
+// Work is spread so that no thread waits on a chain of shuffles: every projection, score
+// and tail logit is one thread's dot product over 16-byte loads; top-k of up to 1024 chunks
+// is a rank count over the keys in shared memory (bitonic sort above that).
 #include "lowram_internal.cuh"
 
 namespace lowram {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kTailBlock = 128;
+constexpr int kTailBlock = 256;
+constexpr int kRankMax = 1024;   // rank-count top-k up to this many chunks
 
 __device__ __forceinline__ uint32_t float_order(float x) {
   uint32_t u = __float_as_uint(x);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__device__ __forceinline__ int next_pow2(int n) {
+__host__ __device__ __forceinline__ int next_pow2(int n) {
   int p = 1;
   while (p < n) p <<= 1;
   return p;
@@ -48,6 +53,44 @@ __device__ void bitonic_sort(unsigned long long* keys, int n) {
   }
 }
 
+// 8 consecutive elements of a row as floats (16-byte load for bf16, two for fp32).
+template <typename T> struct Vec8;
+template <> struct Vec8<__nv_bfloat16> {
+  static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+};
+template <> struct Vec8<float> {
+  static __device__ __forceinline__ void load(const float* p, float (&v)[8]) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+};
+
+// dot(row[0:n], x[0:n]) with x in shared memory; n % 8 == 0 uses vector loads.
+template <typename T>
+__device__ __forceinline__ float row_dot(const T* row, const float* x, int n) {
+  float a = 0.f;
+  if ((n & 7) == 0) {
+    for (int e = 0; e < n; e += 8) {
+      float v[8];
+      Vec8<T>::load(row + e, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a = fmaf(v[i], x[e + i], a);
+    }
+  } else {
+    for (int e = 0; e < n; ++e) a = fmaf(to_f(row[e]), x[e], a);
+  }
+  return a;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
@@ -60,7 +103,8 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
   const int grp = l / g.G;
   const int NG = g.L / g.G;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarp = blockDim.x >> 5;
-  const int nCp = next_pow2(g.nC);
+  const bool rank_topk = g.nC <= kRankMax;
+  const int nCp = rank_topk ? g.nC : next_pow2(g.nC);
   const int kp = next_pow2(g.k);
 
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(smem_raw);  // [nCp]
@@ -68,8 +112,8 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
   float* qt = qs + g.g * g.d;                                                   // [g][r]
   float* qsum = qt + g.g * g.r;                                                 // [r]
   float* sc_s = qsum + g.r;                                                     // [nC]
-  int* selv = reinterpret_cast<int*>(sc_s + g.nC);                              // [kp]
-  float* lg = reinterpret_cast<float*>(selv + kp);                              // [g][128]
+  int* selv = reinterpret_cast<int*>(sc_s + g.nC);                              // [max(kp, nC)]
+  float* lg = reinterpret_cast<float*>(selv + max(kp, g.nC));                   // [g][kTailBlock]
   float* acc = lg + g.g * kTailBlock;                                           // [g][d]
   float* mrun = acc + g.g * g.d;                                                // [g]
   float* lrun = mrun + g.g;                                                     // [g]
@@ -80,16 +124,37 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
   for (int i = tid; i < g.g * g.d; i += blockDim.x) qs[i] = to_f(q[qoff + i]);
   __syncthreads();
 
-  // --- qt_j = B_l q_j (coefficient space), one warp per basis row
+  // --- qt_j = B_l q_j: one thread per (basis row, group of up to 4 heads)
   const T* Bl = reinterpret_cast<const T*>(cb.basis) + ((size_t)l * g.Hkv + un.hkv) * g.r * g.d;
-  for (int i = warp; i < g.r; i += nwarp) {
+  const int jgroups = (g.g + 3) / 4;
+  for (int item = tid; item < g.r * jgroups; item += blockDim.x) {
+    const int i = item % g.r, j0 = (item / g.r) * 4;
     const T* row = Bl + (size_t)i * g.d;
-    for (int j = 0; j < g.g; ++j) {
-      float a = 0.f;
-      for (int dd = lane; dd < g.d; dd += 32) a = fmaf(to_f(row[dd]), qs[j * g.d + dd], a);
-      a = warp_sum(a);
-      if (lane == 0) qt[j * g.r + i] = a;
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    if ((g.d & 7) == 0) {
+      for (int e = 0; e < g.d; e += 8) {
+        float v[8];
+        Vec8<T>::load(row + e, v);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          if (j0 + jj < g.g) {
+            const float* qq = qs + (j0 + jj) * g.d + e;
+#pragma unroll
+            for (int x = 0; x < 8; ++x) a[jj] = fmaf(v[x], qq[x], a[jj]);
+          }
+        }
+      }
+    } else {
+      for (int e = 0; e < g.d; ++e) {
+        const float v = to_f(row[e]);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+          if (j0 + jj < g.g) a[jj] = fmaf(v, qs[(j0 + jj) * g.d + e], a[jj]);
+      }
     }
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj)
+      if (j0 + jj < g.g) qt[(j0 + jj) * g.r + i] = a[jj];
   }
   __syncthreads();
   for (int i = tid; i < g.r; i += blockDim.x) {
@@ -112,58 +177,79 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
   }
   __syncthreads();
 
-  // --- chunk scores over live chunks
+  // --- chunk scores over live chunks: one thread per chunk
   const int16_t* slot = cb.slot ? cb.slot + (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * g.nC : nullptr;
   const T* summ = reinterpret_cast<const T*>(cb.summary) +
                   (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * (size_t)g.nL * g.r;
   const float inv_sqrt_d = rsqrtf((float)g.d);
-  for (int c = warp; c < g.nC; c += nwarp) {
-    int sl = slot ? (int)slot[c] : c;
+  for (int c = tid; c < g.nC; c += blockDim.x) {
+    const int sl = slot ? (int)slot[c] : c;
     float s = -INFINITY;
     if (sl >= 0 && sl < g.nL) {
-      const T* row = summ + (size_t)sl * g.r;
-      float a = 0.f;
-      for (int i = lane; i < g.r; i += 32) a = fmaf(qsum[i], to_f(row[i]), a);
-      a = warp_sum(a);
-      s = a * inv_sqrt_d;
-    } else if (sl >= g.nL && lane == 0) {
+      s = row_dot(summ + (size_t)sl * g.r, qsum, g.r) * inv_sqrt_d;
+    } else if (sl >= g.nL) {
       atomicOr(sc.err, ERR_SLOT);
     }
-    if (lane == 0) sc_s[c] = s;
+    sc_s[c] = s;
+    keys[c] = ((unsigned long long)(~float_order(s)) << 32) | (unsigned)c;
   }
+  for (int c = g.nC + tid; c < nCp; c += blockDim.x) keys[c] = ~0ull;
   __syncthreads();
   if (scores_out) {
     float* so = scores_out + ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * g.nC;
     for (int c = tid; c < g.nC; c += blockDim.x) so[c] = sc_s[c];
   }
 
-  // --- top-k: sort (descending score, ascending id), keep k, sort the ids ascending
-  for (int c = tid; c < nCp; c += blockDim.x) {
-    keys[c] = c < g.nC ? ((unsigned long long)(~float_order(sc_s[c])) << 32) | (unsigned)c
-                       : ~0ull;
-  }
-  __syncthreads();
-  bitonic_sort(keys, nCp);
-  for (int i = tid; i < kp; i += blockDim.x) selv[i] = i < g.k ? (int)(keys[i] & 0xffffffffu) : 0x7fffffff;
-  __syncthreads();
-  // ascending ids (kp <= nCp, reuse the key buffer)
-  for (int i = tid; i < kp; i += blockDim.x) keys[i] = (unsigned long long)(unsigned)selv[i];
-  __syncthreads();
-  bitonic_sort(keys, kp);
-  for (int i = tid; i < g.k; i += blockDim.x) {
-    int id = (int)keys[i];
-    int sl = slot ? (int)slot[id] : id;
-    if (sl < 0 || sl >= g.nL) {
-      atomicOr(sc.err, ERR_SELECT);
-      sl = 0;
+  // --- top-k: order by (descending score, ascending id); keep k; ids ascending
+  int32_t* sel_slot = sc.sel_slot + (size_t)u * g.k;
+  int32_t* sel_id = sc.sel_id + (size_t)u * g.k;
+  int32_t* sel_user = sel_out ? sel_out + ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * g.k : nullptr;
+  if (rank_topk) {
+    // rank of each key among all keys (keys are distinct: the id is in the low bits)
+    for (int c = tid; c < g.nC; c += blockDim.x) {
+      const unsigned long long kc = keys[c];
+      int rank = 0;
+#pragma unroll 8
+      for (int c2 = 0; c2 < g.nC; ++c2) rank += keys[c2] < kc ? 1 : 0;
+      selv[c] = rank < g.k ? 1 : 0;
     }
-    sc.sel_slot[(size_t)u * g.k + i] = sl;
-    sc.sel_id[(size_t)u * g.k + i] = id;
-    if (sel_out) sel_out[((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * g.k + i] = id;
+    __syncthreads();
+    // position among the selected ids = number of selected ids below it
+    for (int c = tid; c < g.nC; c += blockDim.x) {
+      if (!selv[c]) continue;
+      int pos = 0;
+      for (int c2 = 0; c2 < c; ++c2) pos += selv[c2];
+      int sl = slot ? (int)slot[c] : c;
+      if (sl < 0 || sl >= g.nL) {
+        atomicOr(sc.err, ERR_SELECT);
+        sl = 0;
+      }
+      sel_slot[pos] = sl;
+      sel_id[pos] = c;
+      if (sel_user) sel_user[pos] = c;
+    }
+  } else {
+    bitonic_sort(keys, nCp);
+    for (int i = tid; i < kp; i += blockDim.x) selv[i] = i < g.k ? (int)(keys[i] & 0xffffffffu) : 0x7fffffff;
+    __syncthreads();
+    for (int i = tid; i < kp; i += blockDim.x) keys[i] = (unsigned long long)(unsigned)selv[i];
+    __syncthreads();
+    bitonic_sort(keys, kp);
+    for (int i = tid; i < g.k; i += blockDim.x) {
+      const int id = (int)keys[i];
+      int sl = slot ? (int)slot[id] : id;
+      if (sl < 0 || sl >= g.nL) {
+        atomicOr(sc.err, ERR_SELECT);
+        sl = 0;
+      }
+      sel_slot[i] = sl;
+      sel_id[i] = id;
+      if (sel_user) sel_user[i] = id;
+    }
   }
   if (!do_tail) return;
 
-  // --- raw tail: partial softmax over its tokens (online, blocks of 128 tokens)
+  // --- raw tail: partial softmax over its tokens (online, blocks of kTailBlock tokens)
   int tl = cb.tail_len[un.b];
   if (tl < 0 || tl > g.T) {
     if (tid == 0) atomicOr(sc.err, ERR_TAIL_LEN);
@@ -180,14 +266,10 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
   const T* tv = reinterpret_cast<const T*>(cb.tail_v) + toff;
   for (int t0 = 0; t0 < tl; t0 += kTailBlock) {
     const int nb = min(kTailBlock, tl - t0);
-    for (int t = warp; t < nb; t += nwarp) {
+    // logits: one thread per token, all query heads of the unit
+    for (int t = tid; t < nb; t += blockDim.x) {
       const T* row = tk + (size_t)(t0 + t) * g.d;
-      for (int j = 0; j < g.g; ++j) {
-        float a = 0.f;
-        for (int dd = lane; dd < g.d; dd += 32) a = fmaf(to_f(row[dd]), qs[j * g.d + dd], a);
-        a = warp_sum(a);
-        if (lane == 0) lg[j * kTailBlock + t] = a * g.qk_scale_log2;
-      }
+      for (int j = 0; j < g.g; ++j) lg[j * kTailBlock + t] = row_dot(row, qs + j * g.d, g.d) * g.qk_scale_log2;
     }
     __syncthreads();
     for (int j = warp; j < g.g; j += nwarp) {
@@ -197,7 +279,7 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
       const float mnew = fmaxf(mrun[j], m);
       float s = 0.f;
       for (int t = lane; t < nb; t += 32) {
-        float p = exp2f(lg[j * kTailBlock + t] - mnew);
+        const float p = exp2f(lg[j * kTailBlock + t] - mnew);
         lg[j * kTailBlock + t] = p;
         s += p;
       }
@@ -212,9 +294,18 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
     __syncthreads();
     for (int i = tid; i < g.g * g.d; i += blockDim.x) {
       const int j = i / g.d, dd = i % g.d;
-      float a = acc[i] * alpha[j];
-      for (int t = 0; t < nb; ++t) a = fmaf(lg[j * kTailBlock + t], to_f(tv[(size_t)(t0 + t) * g.d + dd]), a);
-      acc[i] = a;
+      const float* p = lg + j * kTailBlock;
+      const T* col = tv + (size_t)t0 * g.d + dd;
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      int t = 0;
+      for (; t + 4 <= nb; t += 4) {
+        a0 = fmaf(p[t], to_f(col[(size_t)t * g.d]), a0);
+        a1 = fmaf(p[t + 1], to_f(col[(size_t)(t + 1) * g.d]), a1);
+        a2 = fmaf(p[t + 2], to_f(col[(size_t)(t + 2) * g.d]), a2);
+        a3 = fmaf(p[t + 3], to_f(col[(size_t)(t + 3) * g.d]), a3);
+      }
+      for (; t < nb; ++t) a0 = fmaf(p[t], to_f(col[(size_t)t * g.d]), a0);
+      acc[i] = acc[i] * alpha[j] + ((a0 + a1) + (a2 + a3));
     }
     __syncthreads();
   }
@@ -227,12 +318,12 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
 }
 
 size_t select_smem_bytes(const Geom& g) {
-  int nCp = 1;
-  while (nCp < g.nC) nCp <<= 1;
+  const int nCp = g.nC <= kRankMax ? g.nC : next_pow2(g.nC);
   int kp = 1;
   while (kp < g.k) kp <<= 1;
-  size_t floats = (size_t)g.g * g.d + (size_t)g.g * g.r + g.r + g.nC + kp +
-                  (size_t)g.g * kTailBlock + (size_t)g.g * g.d + 3 * g.g;
+  const size_t floats = (size_t)g.g * g.d + (size_t)g.g * g.r + g.r + g.nC +
+                        (size_t)(kp > g.nC ? kp : g.nC) + (size_t)g.g * kTailBlock +
+                        (size_t)g.g * g.d + 3 * g.g;
   return (size_t)nCp * 8 + floats * 4;
 }
 
