@@ -19,7 +19,8 @@
 // "Core Mechanism" (Vhat = f(K), delta kept for the worst tokens); attention: "OjaKV", 3.
 //
 // Warp roles (16 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-3 idle, 4-7 and 8-11
-// the two hidden-row halves (silu epilogue, D3 accumulation), 12-15 softmax + residuals.
+// two silu epilogue groups taking alternate sub-tiles (both hidden halves each), 12-15
+// softmax + residuals + accumulation of the chunks' D3.
 // A warp reaches TMEM lanes 32*(warp%4) .. +31, so each warpgroup of four consecutive
 // warps covers all 128 lanes.
 // TMEM (512 columns): W1' halves [0,128), D1 double buffer x 2 halves [128,384),
@@ -81,7 +82,8 @@ struct Bars {
   uint64_t d1_full[2], h_ready[2];
   uint64_t p_ready[2];
   uint64_t d3_full[2], d3_free[2];
-  uint64_t w1_ready;
+  uint64_t w1_ready;   // W1' of the next (layer, KV head) is in TMEM
+  uint64_t seg_done;   // every MMA that read the previous W1' is complete
   uint64_t drain;
 };
 
@@ -89,7 +91,6 @@ struct Misc {
   Bars bars;
   int stage_rec[4][2];               // residual record range [r0, r1) of the chunk in a stage
   uint16_t stage_pos[4][32];         // token offsets of its first RES_CAP records
-  float alpha[4][16];   // per-chunk rescale factors, ring of 4 (see the softmax warpgroup)
   float red_max[4][16];
   float red_sum[4][16];
   uint32_t tmem_base;
@@ -137,12 +138,13 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       mbar_init(&bar.s_full[i], 1);
       mbar_init(&bar.s_free[i], 4);       // 4 softmax warps
       mbar_init(&bar.d1_full[i], 1);
-      mbar_init(&bar.h_ready[i], 8);      // 8 epilogue warps
+      mbar_init(&bar.h_ready[i], 4);      // the 4 warps of the sub-tile's epilogue group
       mbar_init(&bar.p_ready[i], 1);
       mbar_init(&bar.d3_full[i], 1);
-      mbar_init(&bar.d3_free[i], 8);
+      mbar_init(&bar.d3_free[i], 4);      // 4 softmax warps
     }
-    mbar_init(&bar.w1_ready, 8);
+    mbar_init(&bar.w1_ready, 4);          // epilogue group A
+    mbar_init(&bar.seg_done, 1);
     mbar_init(&bar.drain, 1);
     misc->abort_flag = 0;
     mbar_init_fence();
@@ -271,6 +273,10 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
         }
         mma_commit(&bar.d1_full[b]);
         if (sub == SUBS - 1) mma_commit(&bar.a_empty[st]);
+        if (n + 1 < NS) {
+          const int u1 = (int)((x0 + (n + 1) / SUBS) / g.k);
+          if (u1 / g.B != m_cur_seg) mma_commit(&bar.seg_done);   // last read of this W1'
+        }
         return true;
       };
 
@@ -302,62 +308,48 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       mbar_wait(&bar.drain, 0, &never, err, ERR_TIMEOUT);
     }
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 8) {
-    // ============================================================ hidden-row epilogue
-    const int hh = (warp - kEpiWarp0) >> 2;
+    // ============================================================ silu epilogue
+    // Warpgroup A (warps 4-7) takes the even sub-tiles, B (8-11) the odd ones, each doing
+    // both hidden halves, so one group's MUFU work overlaps the other's TMEM round trips.
+    // Group A also swaps W1' in TMEM when the (layer, KV head) changes.
+    const int grp_ab = (warp - kEpiWarp0) >> 2;  // 0 = A (even), 1 = B (odd)
     const int wl = warp & 3;
-    const int row = wl * 32 + lane;              // hidden unit inside the half
+    const int row = wl * 32 + lane;              // hidden unit inside a half
     const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
-    float accH[GQ];
-#pragma unroll
-    for (int j = 0; j < GQ; ++j) accH[j] = 0.f;
-    int cur_u = -1, cur_seg = -1, pending_c = -1;
+    const int b = grp_ab;                        // D1 buffer of this group's sub-tiles
+    int cur_seg = -1, seg_i = -1;
     bool ok = true;
-
-    auto process_d3 = [&](int c) -> bool {
-      const int pb = c & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.d3_full[pb], (c >> 1) & 1, abort_flag, err, ERR_TIMEOUT)))
-        return false;
-      tc_fence_after();
-      uint32_t v[16];
-      tmem_ld16(tmem + lane_off + Lay::T_D3 + (pb * 2 + hh) * 16, v);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar.d3_free[pb]);
-#pragma unroll
-      for (int j = 0; j < GQ; ++j) accH[j] = fmaf(accH[j], misc->alpha[c & 3][j], __uint_as_float(v[j]));
-      return true;
-    };
-    auto write_partial = [&](int u) {
-      float* rec = sc.part + (size_t)(u + blockIdx.x) * g.rec_stride + 2 * GQ;
-#pragma unroll
-      for (int j = 0; j < GQ; ++j) {
-        rec[j * kHid + hh * 128 + row] = accH[j];
-        accH[j] = 0.f;
-      }
-    };
-
-    for (int n = 0; ok && n < NS; ++n) {
-      const int ci = n / SUBS, sub = n % SUBS;
-      const long long x = x0 + ci;
-      const int u = (int)(x / g.k);
-      if (sub == 0 && u != cur_u) {
+    for (int n = grp_ab; ok && n < NS; n += 2) {
+      if (grp_ab == 0) {
+        // perform every W1' swap that falls at or before sub-tile n
+        const int ci = n / SUBS;
+        const long long x = x0 + ci;
+        const int u = (int)(x / g.k);
         const int seg = u / g.B;
         if (seg != cur_seg) {
-          // the previous segment's MMAs are complete (its last D1 was observed): swap W1'
+          ++seg_i;
+          if (seg_i > 0) {
+            // the previous segment's last MMA reading W1' must be complete
+            ok = __all_sync(0xffffffffu, mbar_wait(&bar.seg_done, (seg_i - 1) & 1, abort_flag, err, ERR_TIMEOUT));
+            if (!ok) break;
+            tc_fence_after();
+          }
           const Unit un = unit_of(g, u);
           const int l = g.layer0 + un.li;
-          const uint4* src = reinterpret_cast<const uint4*>(
-              w1f + (((size_t)l * g.Hkv + un.hkv) * kHid + hh * 128 + row) * R);
 #pragma unroll
-          for (int half = 0; half < R / 64; ++half) {
-            uint32_t w[32];
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint4* src = reinterpret_cast<const uint4*>(
+                w1f + (((size_t)l * g.Hkv + un.hkv) * kHid + hh * 128 + row) * R);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const uint4 q = __ldg(src + half * 8 + i);
-              w[4 * i] = q.x; w[4 * i + 1] = q.y; w[4 * i + 2] = q.z; w[4 * i + 3] = q.w;
+            for (int half = 0; half < R / 64; ++half) {
+              uint32_t w[32];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const uint4 q = __ldg(src + half * 8 + i);
+                w[4 * i] = q.x; w[4 * i + 1] = q.y; w[4 * i + 2] = q.z; w[4 * i + 3] = q.w;
+              }
+              tmem_st32(tmem + lane_off + Lay::T_W1 + hh * (R / 2) + half * 32, w);
             }
-            tmem_st32(tmem + lane_off + Lay::T_W1 + hh * (R / 2) + half * 32, w);
           }
           tmem_wait_st();
           tc_fence_before();
@@ -365,60 +357,111 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
           if (lane == 0) mbar_arrive(&bar.w1_ready);
           cur_seg = seg;
         }
-        if (cur_u >= 0) {
-          if (pending_c >= 0) {
-            if (!process_d3(pending_c)) { ok = false; break; }
-            pending_c = -1;
-          }
-          write_partial(cur_u);
-        }
-        cur_u = u;
       }
-      const int b = n & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(&bar.d1_full[b], (n >> 1) & 1, abort_flag, err, ERR_TIMEOUT))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t dcol = tmem + lane_off + Lay::T_D1 + (b * 2 + hh) * 64;
-      uint32_t h[32];
-      {
-        uint32_t v[32];
-        tmem_ld32(dcol, v);
-        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-          h[c] = silu_half2_of_halfx(pack_f16x2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])));
-        tmem_ld32(dcol + 32, v);
-        tmem_wait_ld();
+      for (int hh = 0; hh < 2; ++hh) {
+        const uint32_t dcol = tmem + lane_off + Lay::T_D1 + (b * 2 + hh) * 64;
+        uint32_t h[32];
+        {
+          uint32_t v[32];
+          tmem_ld32(dcol, v);
+          tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
-          h[16 + c] = silu_half2_of_halfx(pack_f16x2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])));
+          for (int c = 0; c < 16; ++c)
+            h[c] = silu_half2_of_halfx(pack_f16x2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])));
+          tmem_ld32(dcol + 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            h[16 + c] = silu_half2_of_halfx(pack_f16x2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])));
+        }
+        tmem_st32(dcol, h);
       }
-      tmem_st32(dcol, h);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.h_ready[b]);
-      if (sub == 0 && pending_c >= 0) {
-        if (!process_d3(pending_c)) { ok = false; break; }
-        pending_c = -1;
+      if (grp_ab == 0 && n + 1 < NS) {
+        // a segment that starts at group B's sub-tile n+1 needs W1' before B can go on
+        const int ci1 = (n + 1) / SUBS;
+        const int u1 = (int)((x0 + ci1) / g.k);
+        const int seg1 = u1 / g.B;
+        if (seg1 != cur_seg) {
+          ++seg_i;
+          ok = __all_sync(0xffffffffu, mbar_wait(&bar.seg_done, (seg_i - 1) & 1, abort_flag, err, ERR_TIMEOUT));
+          if (!ok) break;
+          tc_fence_after();
+          const Unit un = unit_of(g, u1);
+          const int l = g.layer0 + un.li;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint4* src = reinterpret_cast<const uint4*>(
+                w1f + (((size_t)l * g.Hkv + un.hkv) * kHid + hh * 128 + row) * R);
+#pragma unroll
+            for (int half = 0; half < R / 64; ++half) {
+              uint32_t w[32];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const uint4 q = __ldg(src + half * 8 + i);
+                w[4 * i] = q.x; w[4 * i + 1] = q.y; w[4 * i + 2] = q.z; w[4 * i + 3] = q.w;
+              }
+              tmem_st32(tmem + lane_off + Lay::T_W1 + hh * (R / 2) + half * 32, w);
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar.w1_ready);
+          cur_seg = seg1;
+        }
       }
-      if (sub == SUBS - 1) pending_c = ci;
     }
-    if (ok && pending_c >= 0) ok = process_d3(pending_c);
-    if (ok && cur_u >= 0) write_partial(cur_u);
   } else if (warp >= kSoftWarp0) {
     // ============================================================ softmax + residuals
+    // Per chunk: online max/sum per head, the fp16 P tile for the D3 MMA, the residual rows
+    // of the flagged tokens, and (one chunk later) the chunk's D3 = H . P folded into the
+    // softmax-weighted hidden sums.  Thread t is token t for the scores, head-dim element t
+    // for the residuals and hidden row t of both halves for D3.
     const int w = warp & 3;
-    const int t = w * 32 + lane;                 // token (scores) and head-dim index (residuals)
+    const int t = w * 32 + lane;
     const uint32_t lane_off = (uint32_t)(w * 32) << 16;
-    float m_run[GQ], l_run[GQ], accD[GQ];
+    float m_run[GQ], l_run[GQ], accD[GQ], accH0[GQ], accH1[GQ], al_prev[GQ];
 #pragma unroll
-    for (int j = 0; j < GQ; ++j) { m_run[j] = -INFINITY; l_run[j] = 0.f; accD[j] = 0.f; }
+    for (int j = 0; j < GQ; ++j) {
+      m_run[j] = -INFINITY; l_run[j] = 0.f; accD[j] = 0.f; accH0[j] = 0.f; accH1[j] = 0.f;
+      al_prev[j] = 1.f;
+    }
     float* p32_base = reinterpret_cast<float*>(smem + Lay::OFF_P32);
     unsigned char* pbase = smem + Lay::OFF_P;
     int cur_u = -1;
+    // After a failed wait a warp stops working ("live" false) but keeps passing the named
+    // barriers of every remaining chunk, so the other warps of the group never block on it;
+    // once the abort flag is up every wait returns at once.
+    bool live = true;
+    // fold D3 of chunk c (rescaled chunk sums H.P of both halves) into accH
+    auto fold_d3 = [&](int c) {
+      const int pb = c & 1;
+      live = __all_sync(0xffffffffu, live && mbar_wait(&bar.d3_full[pb], (c >> 1) & 1, abort_flag, err, ERR_TIMEOUT));
+      if (!live) return;
+      tc_fence_after();
+      uint32_t v0[16], v1[16];
+      tmem_ld16(tmem + lane_off + Lay::T_D3 + (pb * 2 + 0) * 16, v0);
+      tmem_ld16(tmem + lane_off + Lay::T_D3 + (pb * 2 + 1) * 16, v1);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar.d3_free[pb]);
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) {
+        accH0[j] = fmaf(accH0[j], al_prev[j], __uint_as_float(v0[j]));
+        accH1[j] = fmaf(accH1[j], al_prev[j], __uint_as_float(v1[j]));
+      }
+    };
     auto write_partial = [&](int u) {
       float* rec = sc.part + (size_t)(u + blockIdx.x) * g.rec_stride;
       if (t == 0) {
@@ -427,19 +470,20 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       }
 #pragma unroll
       for (int j = 0; j < GQ; ++j) {
+        rec[2 * GQ + j * kHid + t] = accH0[j];
+        rec[2 * GQ + j * kHid + 128 + t] = accH1[j];
         rec[2 * GQ + GQ * kHid + j * kDh + t] = accD[j];
-        m_run[j] = -INFINITY; l_run[j] = 0.f; accD[j] = 0.f;
+        m_run[j] = -INFINITY; l_run[j] = 0.f; accD[j] = 0.f; accH0[j] = 0.f; accH1[j] = 0.f;
       }
     };
-    // After a failed wait a warp stops working ("live" false) but keeps passing the named
-    // barriers of every remaining chunk, so the other warps of the group never block on it;
-    // once the abort flag is up every wait returns at once.
-    bool live = true;
     for (int ci = 0; ci < NCH; ++ci) {
       const long long x = x0 + ci;
       const int u = (int)(x / g.k);
       if (u != cur_u) {
-        if (cur_u >= 0 && live) write_partial(cur_u);
+        if (cur_u >= 0) {
+          fold_d3(ci - 1);                 // the previous unit's last chunk
+          if (live) write_partial(cur_u);
+        }
         cur_u = u;
       }
       const int st = ci % STAGES, sb = ci & 1, pb = ci & 1;
@@ -475,9 +519,8 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
         p[j] = exp2f(p[j] - mn);
         m_run[j] = mn;
       }
-      // the P buffer is free once the MMAs of chunk ci-2 that read it are done
-      live = __all_sync(0xffffffffu,
-                        live && (ci < 2 || mbar_wait(&bar.d3_full[pb], ((ci - 2) >> 1) & 1, abort_flag, err, ERR_TIMEOUT)));
+      // P buffer pb was last read by the MMAs of chunk ci-2, whose D3 this group has
+      // already folded (so they are complete)
       float* p32 = p32_base + pb * 16 * C;
       if (valid && live) {
 #pragma unroll
@@ -491,12 +534,6 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       for (int j = 0; j < GQ; ++j) {
         const float s = warp_sum(p[j]);
         if (lane == 0) misc->red_sum[w][j] = s;
-      }
-      // alpha of chunk ci is read by the epilogue warps after D3(ci) completes, which is
-      // before this warpgroup reaches chunk ci+4 (it waits for D3(ci+2) there): a ring of 4
-      if (t == 0) {
-#pragma unroll
-        for (int j = 0; j < GQ; ++j) misc->alpha[ci & 3][j] = al[j];
       }
       fence_proxy_async_smem();
       named_bar_sync(1, 128);
@@ -531,8 +568,22 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       }
       named_bar_sync(1, 128);
       if (t == 0 && live) mbar_arrive(&bar.a_empty[st]);
+      // fold the previous chunk's D3 when it belongs to this unit (its MMAs ran meanwhile);
+      // the chunk sums of ci-1 are relative to m after ci-1, so rescale by al of ci-1 first
+      if (ci >= 1 && (int)((x0 + ci - 1) / g.k) == u) {
+        fold_d3(ci - 1);
+      }
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) {
+        // accH is kept relative to the running max after the last folded chunk; the next
+        // fold multiplies by the rescale factor of the chunk being folded
+        al_prev[j] = al[j];
+      }
     }
-    if (live && !*abort_flag && cur_u >= 0) write_partial(cur_u);
+    if (NCH > 0) {
+      fold_d3(NCH - 1);
+      if (live && !*abort_flag && cur_u >= 0) write_partial(cur_u);
+    }
   }
 
   // ------------------------------------------------------------------ teardown
