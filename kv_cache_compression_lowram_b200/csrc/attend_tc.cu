@@ -100,6 +100,35 @@ struct Misc {
 static_assert(sizeof(Misc) <= 2048, "Misc must fit its shared-memory slot");
 static_assert(sizeof(((Misc*)0)->stage_rec) / sizeof(int[2]) == 4, "one record range per stage");
 
+// Sequential walk over a CTA's chunk tiles: the unit of each chunk, the chunk's index in its
+// unit and the unit's (layer, KV head) segment, updated by counters (no division per step).
+struct TileWalk {
+  int ci, u, rem, seg, ub, k, B;
+  __device__ __forceinline__ void init(long long x0, int k_, int B_) {
+    k = k_;
+    B = B_;
+    ci = 0;
+    u = (int)(x0 / k);
+    rem = (int)(x0 - (long long)u * k);
+    seg = u / B;
+    ub = u - seg * B;
+  }
+  __device__ __forceinline__ void advance_to(int target) {
+    while (ci < target) {
+      ++ci;
+      if (++rem == k) {
+        rem = 0;
+        ++u;
+        if (++ub == B) {
+          ub = 0;
+          ++seg;
+        }
+      }
+    }
+  }
+  __device__ __forceinline__ bool next_starts_segment() const { return rem + 1 == k && ub + 1 == B; }
+};
+
 __device__ __forceinline__ float bf16_bits_to_f(uint16_t b) {
   return __uint_as_float(((uint32_t)b) << 16);
 }
@@ -172,9 +201,12 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
     // ============================================================ TMA producer
     if (lane == 0 && NCH > 0) {
       int unit_i = -1, prev_u = -1, issued = 0, q_issued = 0;
+      TileWalk wk;
+      wk.init(x0, g.k, g.B);
       for (int ci = 0; ci < NCH; ++ci) {
         const long long x = x0 + ci;
-        const int u = (int)(x / g.k);
+        wk.advance_to(ci);
+        const int u = wk.u;
         if (u != prev_u) {
           ++unit_i;
           prev_u = u;
@@ -223,13 +255,20 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
     // ============================================================ MMA issuer
     if (lane == 0 && NS > 0) {
       int m_unit_i = -1, m_cur_u = -1, m_seg_i = -1, m_cur_seg = -1;
-      auto a_slab = [&](int st, int kk) -> uint32_t {
-        return sA + st * Lay::A_STAGE + (kk >> 2) * 16384 + (kk & 3) * 32;
-      };
+      // Descriptors are built once; a K step, stage, buffer or sub-tile only moves the
+      // start address, i.e. adds (byte offset >> 4) to the low field (no carry: every
+      // shared address here is below 256 KiB).
+      const uint64_t dA0 = smem_desc(sA, 16, 1024, 2);              // coefficient tiles
+      const uint64_t dQ0 = smem_desc(sQ, 16, 1024, 2);              // projected queries
+      const uint64_t dP0 = smem_desc(sP, 128, Lay::P_SBO, 0);       // probabilities
+      const uint32_t t_w1 = tmem + Lay::T_W1, t_d1 = tmem + Lay::T_D1;
+      const uint32_t t_s = tmem + Lay::T_S, t_d3 = tmem + Lay::T_D3;
+      TileWalk wk;
+      wk.init(x0, g.k, g.B);
       auto issue_mma1 = [&](int n) -> bool {
         const int ci = n / SUBS, sub = n % SUBS;
-        const long long x = x0 + ci;
-        const int u = (int)(x / g.k);
+        wk.advance_to(ci);
+        const int u = wk.u;
         const int st = ci % STAGES;
         if (sub == 0) {
           if (!mbar_wait(&bar.a_full[st], (ci / STAGES) & 1, abort_flag, err, ERR_TIMEOUT)) return false;
@@ -239,7 +278,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
             m_cur_u = u;
             if (!mbar_wait(&bar.q_full[m_unit_i & 1], (m_unit_i >> 1) & 1, abort_flag, err, ERR_TIMEOUT))
               return false;
-            const int seg = u / g.B;
+            const int seg = wk.seg;
             if (seg != m_cur_seg) {
               ++m_seg_i;
               m_cur_seg = seg;
@@ -250,33 +289,31 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
           if (ci >= 2 && !mbar_wait(&bar.s_free[sb], ((ci >> 1) - 1) & 1, abort_flag, err, ERR_TIMEOUT))
             return false;
           tc_fence_after();
-          const uint32_t qbase = sQ + (m_unit_i & 1) * Lay::Q_BUF;
+          const uint64_t dA = dA0 + (uint64_t)((st * Lay::A_STAGE) >> 4);
+          const uint64_t dQ = dQ0 + (uint64_t)(((m_unit_i & 1) * Lay::Q_BUF) >> 4);
+          const uint32_t ts = t_s + sb * 16;
 #pragma unroll
-          for (int kk = 0; kk < R / 16; ++kk) {
-            const uint64_t ad = smem_desc(a_slab(st, kk), 16, 1024, 2);
-            const uint64_t bd = smem_desc(qbase + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024, 2);
-            mma_ss(tmem + Lay::T_S + sb * 16, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < R / 16; ++kk)
+            mma_ss(ts, dA + (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2),
+                   dQ + (uint64_t)((kk >> 2) * 128 + (kk & 3) * 2), IDESC_S, kk > 0 ? 1u : 0u);
           mma_commit(&bar.s_full[sb]);
         } else {
           tc_fence_after();
         }
         const int b = n & 1;
+        const uint64_t dB = dA0 + (uint64_t)((st * Lay::A_STAGE + sub * 8192) >> 4);
+        const uint32_t td = t_d1 + b * 128;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
-          for (int kk = 0; kk < R / 16; ++kk) {
-            const uint64_t bd = smem_desc(a_slab(st, kk) + sub * 8192, 16, 1024, 2);
-            mma_ts(tmem + Lay::T_D1 + (b * 2 + hh) * 64, tmem + Lay::T_W1 + hh * (R / 2) + kk * 8, bd,
-                   IDESC_1, kk > 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < R / 16; ++kk)
+            mma_ts(td + hh * 64, t_w1 + hh * (R / 2) + kk * 8,
+                   dB + (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2), IDESC_1, kk > 0 ? 1u : 0u);
         }
         mma_commit(&bar.d1_full[b]);
         if (sub == SUBS - 1) mma_commit(&bar.a_empty[st]);
-        if (n + 1 < NS) {
-          const int u1 = (int)((x0 + (n + 1) / SUBS) / g.k);
-          if (u1 / g.B != m_cur_seg) mma_commit(&bar.seg_done);   // last read of this W1'
-        }
+        if (n + 1 < NS && sub == SUBS - 1 && wk.next_starts_segment())
+          mma_commit(&bar.seg_done);   // the last MMA that reads this W1' has been issued
         return true;
       };
 
@@ -290,14 +327,14 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
           if (ci >= 2 && !mbar_wait(&bar.d3_free[pb], ((ci >> 1) - 1) & 1, abort_flag, err, ERR_TIMEOUT)) break;
         }
         tc_fence_after();
+        const uint64_t dP = dP0 + (uint64_t)((pb * Lay::P_BUF + sub * 1024) >> 4);
+        const uint32_t acc0 = sub > 0 ? 1u : 0u;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bd = smem_desc(sP + pb * Lay::P_BUF + sub * 1024 + kk * 256, 128, Lay::P_SBO, 0);
-            mma_ts(tmem + Lay::T_D3 + (pb * 2 + hh) * 16, tmem + Lay::T_D1 + (b * 2 + hh) * 64 + kk * 8, bd,
-                   IDESC_3, (sub > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(t_d3 + pb * 32 + hh * 16, t_d1 + b * 128 + hh * 64 + kk * 8, dP + (uint64_t)(kk * 16),
+                   IDESC_3, kk > 0 ? 1u : acc0);
         }
         if (sub == SUBS - 1) mma_commit(&bar.d3_full[pb]);
         if (n + 2 < NS) ok = issue_mma1(n + 2);
@@ -319,13 +356,14 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
     const int b = grp_ab;                        // D1 buffer of this group's sub-tiles
     int cur_seg = -1, seg_i = -1;
     bool ok = true;
+    TileWalk wk;
+    wk.init(x0, g.k, g.B);
     for (int n = grp_ab; ok && n < NS; n += 2) {
+      wk.advance_to(n / SUBS);
       if (grp_ab == 0) {
         // perform every W1' swap that falls at or before sub-tile n
-        const int ci = n / SUBS;
-        const long long x = x0 + ci;
-        const int u = (int)(x / g.k);
-        const int seg = u / g.B;
+        const int u = wk.u;
+        const int seg = wk.seg;
         if (seg != cur_seg) {
           ++seg_i;
           if (seg_i > 0) {
@@ -386,12 +424,11 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar.h_ready[b]);
-      if (grp_ab == 0 && n + 1 < NS) {
+      if (grp_ab == 0 && n + 1 < NS && (n + 1) % SUBS == 0 && wk.next_starts_segment()) {
         // a segment that starts at group B's sub-tile n+1 needs W1' before B can go on
-        const int ci1 = (n + 1) / SUBS;
-        const int u1 = (int)((x0 + ci1) / g.k);
-        const int seg1 = u1 / g.B;
-        if (seg1 != cur_seg) {
+        const int u1 = wk.u + 1;
+        const int seg1 = wk.seg + 1;
+        {
           ++seg_i;
           ok = __all_sync(0xffffffffu, mbar_wait(&bar.seg_done, (seg_i - 1) & 1, abort_flag, err, ERR_TIMEOUT));
           if (!ok) break;
@@ -476,9 +513,11 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
         m_run[j] = -INFINITY; l_run[j] = 0.f; accD[j] = 0.f; accH0[j] = 0.f; accH1[j] = 0.f;
       }
     };
+    TileWalk wk;
+    wk.init(x0, g.k, g.B);
     for (int ci = 0; ci < NCH; ++ci) {
-      const long long x = x0 + ci;
-      const int u = (int)(x / g.k);
+      wk.advance_to(ci);
+      const int u = wk.u;
       if (u != cur_u) {
         if (cur_u >= 0) {
           fold_d3(ci - 1);                 // the previous unit's last chunk
@@ -570,7 +609,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       if (t == 0 && live) mbar_arrive(&bar.a_empty[st]);
       // fold the previous chunk's D3 when it belongs to this unit (its MMAs ran meanwhile);
       // the chunk sums of ci-1 are relative to m after ci-1, so rescale by al of ci-1 first
-      if (ci >= 1 && (int)((x0 + ci - 1) / g.k) == u) {
+      if (ci >= 1 && wk.rem != 0) {        // chunk ci-1 belongs to this unit too
         fold_d3(ci - 1);
       }
 #pragma unroll
