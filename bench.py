@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--sweep", action="store_true",
                     help="also run the batch sweep 1,4,16,32,64 (extra JSON lines)")
+    ap.add_argument("--dense", action="store_true",
+                    help="only the uncompressed bf16 dense-KV baseline at its largest batch")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -353,6 +355,66 @@ def run_lowram(args, ws, rank, local):
     return line
 
 
+def run_dense(args, ws, rank, local, cfg_name=DEFAULT_CONFIG):
+    """Uncompressed bf16 decode attention over the same context (N + T tokens) at the largest
+    batch whose dense cache fits in device memory: the baseline of the batch sweep."""
+    import kv_cache_compression_lowram_b200 as K
+    cfg = S.CONFIGS[cfg_name]
+    dev = torch.device("cuda", local)
+    S_ = cfg.n_ctx + cfg.tail_cap
+    per_seq = 2 * cfg.n_layers * cfg.n_kv_heads * S_ * cfg.head_dim * 2
+    free, _ = torch.cuda.mem_get_info(dev)
+    B = max(1, int((free - 6e9) // per_seq))
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(cfg.seed + 17 + rank)
+    k = torch.empty(B, cfg.n_layers, cfg.n_kv_heads, S_, cfg.head_dim, dtype=torch.bfloat16, device=dev)
+    v = torch.empty_like(k)
+    for b in range(B):   # per sequence, to keep the fp32 temporaries small
+        k[b] = torch.randn(k.shape[1:], generator=gen, device=dev).to(torch.bfloat16)
+        v[b] = (0.1 * torch.randn(v.shape[1:], generator=gen, device=dev)).to(torch.bfloat16)
+    q = (torch.randn(cfg.n_layers, B, cfg.n_q_heads, cfg.head_dim, generator=gen, device=dev)
+         / math.sqrt(cfg.head_dim)).to(torch.bfloat16)
+    out = torch.empty_like(q)
+    for _ in range(args.warmup):
+        K.lowram_dense_decode_attn(k, v, q, out)
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 10))
+    clocks = ClockSampler(local)
+    barrier(ws)
+    clocks.start()
+    time.sleep(0.3)
+    stream = torch.cuda.current_stream()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        K.lowram_dense_decode_attn(k, v, q, out)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    value, ms_total = aggregate_rate(B * cfg.n_layers * steps, start.elapsed_time(end), ws)
+    ms_step = ms_total / steps
+    bytes_step = k.numel() * 2 * 2 + q.numel() * 2 * 2
+    peak, peak_kind = peaks()
+    achieved = bytes_step / (ms_step / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "queries/s", "n_gpus": ws, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "impl": "dense_baseline",
+        "config": {"workload": f"dense_bf16_{cfg.name}_b{B}", "batch": B, "n_layers": cfg.n_layers,
+                   "tokens": S_, "kv_heads": cfg.n_kv_heads, "q_heads": cfg.n_q_heads,
+                   "head_dim": cfg.head_dim, "dense_cache_gb": round(k.numel() * 4 / 1e9, 2)},
+        "roofline": {"bound": "hbm", "kernel": "dense_kernel", "achieved": round(achieved, 1),
+                     "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "peak_kind": peak_kind},
+        "gpu_launches": steps, "clocks": clk,
+    }
+    del k, v
+    torch.cuda.empty_cache()
+    return line
+
+
 def run_reference(args, ws, rank):
     """The oracle (fp64 numpy, host cores) on the same workload, bounded samples per step."""
     if rank != 0:
@@ -391,18 +453,27 @@ def main():
     ws, rank, local = dist_init()
     if args.impl == "reference":
         line = run_reference(args, ws, rank)
+    elif args.dense:
+        line = run_dense(args, ws, rank, local)
     else:
         line = run_lowram(args, ws, rank, local)
     if rank == 0 and line is not None:
         print(json.dumps(line), flush=True)
-    if args.sweep and args.impl == "lowram":
+    if args.sweep and args.impl == "lowram" and not args.dense:
+        import gc
         for b in (1, 4, 16, 32, 64):
             args.config = f"llama8b_32k_bf16_b{b}"
             args.no_cpu_baseline = True
+            gc.collect()
             torch.cuda.empty_cache()
             line = run_lowram(args, ws, rank, local)
             if rank == 0:
                 print(json.dumps(line), flush=True)
+        gc.collect()
+        torch.cuda.empty_cache()
+        line = run_dense(args, ws, rank, local)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist
         dist.destroy_process_group()

@@ -236,6 +236,18 @@ int32_t lowram_cache_last_launches(const lowram_cache* cache);
 /* Which path the last lowram_decode_attn call on this cache ran (a lowram_path value). */
 int32_t lowram_cache_last_path(const lowram_cache* cache);
 
+/* Dense decode attention over an UNCOMPRESSED bf16 KV cache, the baseline a compressed cache
+ * is compared with: every cached token is attended, o_j = softmax_t(q_j . k_t / sqrt(d)) v_t
+ * ("OjaKV", section 3, attention), and the cache holds M_KV = 2 L Hkv d N s bytes per
+ * sequence ("LowRAM Compresses KV Cache Asymmetrically", section "Core Mechanism").
+ *   k, v [B][L][Hkv][S][d] bf16, DEVICE, 16-byte aligned;
+ *   q, out [L][B][Hq][d] bf16, DEVICE.  All L layers in one call, stream-ordered.
+ * Needs head_dim % 8 == 0, head_dim <= 256, Hq/Hkv <= 16; returns EINVAL otherwise. */
+lowram_status lowram_dense_decode_attn(int32_t batch, int32_t n_layers, int32_t n_kv_heads,
+                                       int32_t n_q_heads, int32_t head_dim, int64_t seq_len,
+                                       const void* k, const void* v, const void* q, void* out,
+                                       lowram_stream stream);
+
 /* Decode-time attention with no device allocation at all, for callers that cannot call
  * cudaMalloc on their decode path (an engine that reserves all device memory for its own
  * pool, a runtime that forbids allocation after start-up, a thread capturing a CUDA graph

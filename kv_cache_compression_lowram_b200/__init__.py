@@ -24,7 +24,7 @@ __all__ = [
     "lowram_cache_destroy", "lowram_decode_attn", "lowram_select_chunks",
     "lowram_decode_attn_host", "lowram_cache_bytes", "lowram_cache_validate",
     "lowram_cache_set_stage_events", "lowram_cache_last_launches", "lowram_cache_last_path",
-    "LowramCache", "config_struct", "lowram_decode_attn_static",
+    "LowramCache", "config_struct", "lowram_decode_attn_static", "lowram_dense_decode_attn",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblowram.so")
@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
         "lowram_cache_last_path": (I32, [P]),
         "lowram_decode_attn_static": (I32, [ctypes.POINTER(LowramConfigC), ctypes.POINTER(LowramSrcC),
                                             I32, I32, P, P, P, P]),
+        "lowram_dense_decode_attn": (I32, [I32, I32, I32, I32, I32, I64, P, P, P, P, P]),
         "lowram_status_string": (ctypes.c_char_p, [I32]),
         "lowram_last_error_string": (ctypes.c_char_p, []),
     }
@@ -230,6 +231,14 @@ def lowram_decode_attn_static(cfg, arrays, layer0: int, n_layers: int, q, out, s
     _check(lib().lowram_decode_attn_static(ctypes.byref(c), ctypes.byref(src), layer0, n_layers,
                                            _ptr(q), _ptr(out), _ptr(sel), _stream(stream)),
            "lowram_decode_attn_static")
+
+
+def lowram_dense_decode_attn(k, v, q, out, stream=None) -> None:
+    """Dense baseline: k, v [B][L][Hkv][S][d] bf16, q/out [L][B][Hq][d] bf16 (device)."""
+    B, L, Hkv, S_, d = (int(x) for x in k.shape)
+    Hq = int(q.shape[2])
+    _check(lib().lowram_dense_decode_attn(B, L, Hkv, Hq, d, S_, _ptr(k), _ptr(v), _ptr(q), _ptr(out),
+                                          _stream(stream)), "lowram_dense_decode_attn")
 
 
 def lowram_cache_bytes(handle: int) -> dict:

@@ -199,7 +199,10 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
 
   if (warp == 0) {
     // ============================================================ TMA producer
-    if (lane == 0 && NCH > 0) {
+    // The whole warp walks the tiles (waits and bookkeeping are warp-uniform); one elected
+    // lane issues the copies.
+    const bool leader = elect_one();
+    if (NCH > 0) {
       int unit_i = -1, prev_u = -1, issued = 0, q_issued = 0;
       TileWalk wk;
       wk.init(x0, g.k, g.B);
@@ -211,15 +214,21 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
           ++unit_i;
           prev_u = u;
           const int qb = unit_i & 1;
-          if (unit_i >= 2 && !mbar_wait(&bar.q_empty[qb], ((unit_i >> 1) - 1) & 1, abort_flag, err, ERR_TIMEOUT))
+          if (unit_i >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar.q_empty[qb], ((unit_i >> 1) - 1) & 1,
+                                                                abort_flag, err, ERR_TIMEOUT)))
             break;
-          mbar_expect_tx(&bar.q_full[qb], 16 * R * 2);
-          for (int ks = 0; ks < KSLABS; ++ks)
-            tma_load_2d(smem + Lay::OFF_Q + qb * Lay::Q_BUF + ks * 2048, &tmQ, &bar.q_full[qb], ks * 64, u * 16);
+          if (leader) {
+            mbar_expect_tx(&bar.q_full[qb], 16 * R * 2);
+#pragma unroll
+            for (int ks = 0; ks < KSLABS; ++ks)
+              tma_load_2d(smem + Lay::OFF_Q + qb * Lay::Q_BUF + ks * 2048, &tmQ, &bar.q_full[qb], ks * 64, u * 16);
+          }
+          __syncwarp();
           q_issued = unit_i + 1;
         }
         const int st = ci % STAGES;
-        if (ci >= STAGES && !mbar_wait(&bar.a_empty[st], ((ci / STAGES) - 1) & 1, abort_flag, err, ERR_TIMEOUT))
+        if (ci >= STAGES && !__all_sync(0xffffffffu, mbar_wait(&bar.a_empty[st], ((ci / STAGES) - 1) & 1,
+                                                               abort_flag, err, ERR_TIMEOUT)))
           break;
         const Unit un = unit_of(g, u);
         const int l = g.layer0 + un.li;
@@ -230,20 +239,27 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
         const int r0 = rptr[slot], r1 = rptr[slot + 1];
         const int nres = min(r1 - r0, Lay::RES_CAP);
         // record range and positions for the softmax warpgroup (published by the arrive below)
-        misc->stage_rec[st][0] = r0;
-        misc->stage_rec[st][1] = r1;
-        for (int i = 0; i < nres; ++i) misc->stage_pos[st][i] = cb.res_pos[r0 + i];
-        mbar_expect_tx(&bar.a_full[st], (uint32_t)(C * R * 2 + nres * kDh * 2));
-        for (int ks = 0; ks < KSLABS; ++ks)
-          tma_load_2d(smem + Lay::OFF_A + st * Lay::A_STAGE + ks * 16384, &tmA, &bar.a_full[st], ks * 64, row0);
-        if (nres > 0)
-          bulk_load(smem + Lay::OFF_RES + st * Lay::RES_BUF,
-                    reinterpret_cast<const unsigned char*>(cb.res_val) + (size_t)r0 * kDh * 2,
-                    (uint32_t)(nres * kDh * 2), &bar.a_full[st]);
+        if (lane == 0) {
+          misc->stage_rec[st][0] = r0;
+          misc->stage_rec[st][1] = r1;
+        }
+        if (lane < nres) misc->stage_pos[st][lane] = cb.res_pos[r0 + lane];
+        __syncwarp();
+        if (leader) {
+          mbar_expect_tx(&bar.a_full[st], (uint32_t)(C * R * 2 + nres * kDh * 2));
+#pragma unroll
+          for (int ks = 0; ks < KSLABS; ++ks)
+            tma_load_2d(smem + Lay::OFF_A + st * Lay::A_STAGE + ks * 16384, &tmA, &bar.a_full[st], ks * 64, row0);
+          if (nres > 0)
+            bulk_load(smem + Lay::OFF_RES + st * Lay::RES_BUF,
+                      reinterpret_cast<const unsigned char*>(cb.res_val) + (size_t)r0 * kDh * 2,
+                      (uint32_t)(nres * kDh * 2), &bar.a_full[st]);
+        }
+        __syncwarp();
         issued = ci + 1;
       }
-      if (*abort_flag) {
-        // let every copy this thread started land before the CTA's shared memory goes away
+      if (*abort_flag && leader) {
+        // let every copy this warp started land before the CTA's shared memory goes away
         volatile int never = 0;
         for (int ci = max(0, issued - STAGES); ci < issued; ++ci)
           mbar_wait(&bar.a_full[ci % STAGES], (ci / STAGES) & 1, &never, err, ERR_TIMEOUT);
@@ -253,7 +269,10 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
     }
   } else if (warp == 1) {
     // ============================================================ MMA issuer
-    if (lane == 0 && NS > 0) {
+    // The whole warp runs the schedule and waits; one elected lane issues every MMA and
+    // commit, so descriptors and TMEM addresses stay warp-uniform.
+    const bool leader = elect_one();
+    if (NS > 0) {
       int m_unit_i = -1, m_cur_u = -1, m_seg_i = -1, m_cur_seg = -1;
       // Descriptors are built once; a K step, stage, buffer or sub-tile only moves the
       // start address, i.e. adds (byte offset >> 4) to the low field (no carry: every
@@ -265,55 +284,61 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       const uint32_t t_s = tmem + Lay::T_S, t_d3 = tmem + Lay::T_D3;
       TileWalk wk;
       wk.init(x0, g.k, g.B);
+      auto wait_all = [&](uint64_t* b, uint32_t par) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(b, par, abort_flag, err, ERR_TIMEOUT));
+      };
       auto issue_mma1 = [&](int n) -> bool {
         const int ci = n / SUBS, sub = n % SUBS;
         wk.advance_to(ci);
         const int u = wk.u;
         const int st = ci % STAGES;
         if (sub == 0) {
-          if (!mbar_wait(&bar.a_full[st], (ci / STAGES) & 1, abort_flag, err, ERR_TIMEOUT)) return false;
+          if (!wait_all(&bar.a_full[st], (ci / STAGES) & 1)) return false;
           if (u != m_cur_u) {
-            if (m_cur_u >= 0) mma_commit(&bar.q_empty[m_unit_i & 1]);
+            if (m_cur_u >= 0 && leader) mma_commit(&bar.q_empty[m_unit_i & 1]);
             ++m_unit_i;
             m_cur_u = u;
-            if (!mbar_wait(&bar.q_full[m_unit_i & 1], (m_unit_i >> 1) & 1, abort_flag, err, ERR_TIMEOUT))
-              return false;
+            if (!wait_all(&bar.q_full[m_unit_i & 1], (m_unit_i >> 1) & 1)) return false;
             const int seg = wk.seg;
             if (seg != m_cur_seg) {
               ++m_seg_i;
               m_cur_seg = seg;
-              if (!mbar_wait(&bar.w1_ready, m_seg_i & 1, abort_flag, err, ERR_TIMEOUT)) return false;
+              if (!wait_all(&bar.w1_ready, m_seg_i & 1)) return false;
             }
           }
           const int sb = ci & 1;
-          if (ci >= 2 && !mbar_wait(&bar.s_free[sb], ((ci >> 1) - 1) & 1, abort_flag, err, ERR_TIMEOUT))
-            return false;
+          if (ci >= 2 && !wait_all(&bar.s_free[sb], ((ci >> 1) - 1) & 1)) return false;
           tc_fence_after();
           const uint64_t dA = dA0 + (uint64_t)((st * Lay::A_STAGE) >> 4);
           const uint64_t dQ = dQ0 + (uint64_t)(((m_unit_i & 1) * Lay::Q_BUF) >> 4);
           const uint32_t ts = t_s + sb * 16;
+          if (leader) {
 #pragma unroll
-          for (int kk = 0; kk < R / 16; ++kk)
-            mma_ss(ts, dA + (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2),
-                   dQ + (uint64_t)((kk >> 2) * 128 + (kk & 3) * 2), IDESC_S, kk > 0 ? 1u : 0u);
-          mma_commit(&bar.s_full[sb]);
+            for (int kk = 0; kk < R / 16; ++kk)
+              mma_ss(ts, dA + (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2),
+                     dQ + (uint64_t)((kk >> 2) * 128 + (kk & 3) * 2), IDESC_S, kk > 0 ? 1u : 0u);
+            mma_commit(&bar.s_full[sb]);
+          }
         } else {
           tc_fence_after();
         }
         const int b = n & 1;
         const uint64_t dB = dA0 + (uint64_t)((st * Lay::A_STAGE + sub * 8192) >> 4);
         const uint32_t td = t_d1 + b * 128;
+        if (leader) {
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
+          for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
-          for (int kk = 0; kk < R / 16; ++kk)
-            mma_ts(td + hh * 64, t_w1 + hh * (R / 2) + kk * 8,
-                   dB + (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2), IDESC_1, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < R / 16; ++kk)
+              mma_ts(td + hh * 64, t_w1 + hh * (R / 2) + kk * 8,
+                     dB + (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2), IDESC_1, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(&bar.d1_full[b]);
+          if (sub == SUBS - 1) mma_commit(&bar.a_empty[st]);
+          if (n + 1 < NS && sub == SUBS - 1 && wk.next_starts_segment())
+            mma_commit(&bar.seg_done);   // the last MMA that reads this W1' has been issued
         }
-        mma_commit(&bar.d1_full[b]);
-        if (sub == SUBS - 1) mma_commit(&bar.a_empty[st]);
-        if (n + 1 < NS && sub == SUBS - 1 && wk.next_starts_segment())
-          mma_commit(&bar.seg_done);   // the last MMA that reads this W1' has been issued
+        __syncwarp();
         return true;
       };
 
@@ -321,28 +346,34 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       if (ok && NS > 1) ok = issue_mma1(1);
       for (int n = 0; ok && n < NS; ++n) {
         const int ci = n / SUBS, sub = n % SUBS, b = n & 1, pb = ci & 1;
-        if (!mbar_wait(&bar.h_ready[b], (n >> 1) & 1, abort_flag, err, ERR_TIMEOUT)) break;
+        if (!wait_all(&bar.h_ready[b], (n >> 1) & 1)) break;
         if (sub == 0) {
-          if (!mbar_wait(&bar.p_ready[pb], (ci >> 1) & 1, abort_flag, err, ERR_TIMEOUT)) break;
-          if (ci >= 2 && !mbar_wait(&bar.d3_free[pb], ((ci >> 1) - 1) & 1, abort_flag, err, ERR_TIMEOUT)) break;
+          if (!wait_all(&bar.p_ready[pb], (ci >> 1) & 1)) break;
+          if (ci >= 2 && !wait_all(&bar.d3_free[pb], ((ci >> 1) - 1) & 1)) break;
         }
         tc_fence_after();
         const uint64_t dP = dP0 + (uint64_t)((pb * Lay::P_BUF + sub * 1024) >> 4);
         const uint32_t acc0 = sub > 0 ? 1u : 0u;
+        if (leader) {
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
+          for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ts(t_d3 + pb * 32 + hh * 16, t_d1 + b * 128 + hh * 64 + kk * 8, dP + (uint64_t)(kk * 16),
-                   IDESC_3, kk > 0 ? 1u : acc0);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ts(t_d3 + pb * 32 + hh * 16, t_d1 + b * 128 + hh * 64 + kk * 8, dP + (uint64_t)(kk * 16),
+                     IDESC_3, kk > 0 ? 1u : acc0);
+          }
+          if (sub == SUBS - 1) mma_commit(&bar.d3_full[pb]);
         }
-        if (sub == SUBS - 1) mma_commit(&bar.d3_full[pb]);
+        __syncwarp();
         if (n + 2 < NS) ok = issue_mma1(n + 2);
       }
-      // every MMA this thread issued must finish before TMEM is released
-      mma_commit(&bar.drain);
-      volatile int never = 0;
-      mbar_wait(&bar.drain, 0, &never, err, ERR_TIMEOUT);
+      // every MMA this warp issued must finish before TMEM is released
+      if (leader) {
+        mma_commit(&bar.drain);
+        volatile int never = 0;
+        mbar_wait(&bar.drain, 0, &never, err, ERR_TIMEOUT);
+      }
+      __syncwarp();
     }
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 8) {
     // ============================================================ silu epilogue

@@ -201,6 +201,18 @@ __device__ __forceinline__ uint32_t silu_half2_of_halfx(uint32_t u) {
   return r;
 }
 
+// One lane of a converged warp (the lowest), chosen with elect.sync.  Issuing tcgen05/TMA
+// work from an elected lane of a converged warp keeps the operands warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t is = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(is));
+  return is != 0;
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

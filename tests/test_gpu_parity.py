@@ -303,3 +303,24 @@ def test_bad_layer_range_rejected():
         lc.decode(q, layer0=1)          # 2 layers from layer 1 exceeds the cache
     assert ei.value.status == 1
     lc.close()
+
+
+def test_dense_baseline_matches_textbook_attention():
+    """The uncompressed baseline kernel against the oracle's textbook attention."""
+    g = torch.Generator().manual_seed(11)
+    B, L, Hkv, Hq, S_, d = 2, 2, 2, 8, 1000, 128       # 1000 tokens: ragged last block
+    k = torch.randn(B, L, Hkv, S_, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, L, Hkv, S_, d, generator=g).to(torch.bfloat16)
+    q = (torch.randn(L, B, Hq, d, generator=g) * 0.3).to(torch.bfloat16)
+    out = torch.empty(L, B, Hq, d, dtype=torch.bfloat16, device=DEV)
+    K.lowram_dense_decode_attn(k.to(DEV), v.to(DEV), q.to(DEV), out)
+    torch.cuda.synchronize()
+    gq = Hq // Hkv
+    for l in range(L):
+        for b in range(B):
+            for h in range(Hkv):
+                ref = O.attend(q[l, b, h * gq:(h + 1) * gq].double().numpy(),
+                               k[b, l, h].double().numpy(), v[b, l, h].double().numpy())
+                got = out[l, b, h * gq:(h + 1) * gq].cpu().double().numpy()
+                err = np.abs(got - ref).max(axis=1) / np.linalg.norm(ref, axis=1)
+                assert err.max() <= 2e-2
