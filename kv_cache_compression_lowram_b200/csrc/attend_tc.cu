@@ -312,13 +312,28 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
           const uint64_t dA = dA0 + (uint64_t)((st * Lay::A_STAGE) >> 4);
           const uint64_t dQ = dQ0 + (uint64_t)(((m_unit_i & 1) * Lay::Q_BUF) >> 4);
           const uint32_t ts = t_s + sb * 16;
+          const int b0 = n & 1;
+          const uint64_t dB = dA0 + (uint64_t)((st * Lay::A_STAGE + sub * 8192) >> 4);
+          const uint32_t td = t_d1 + b0 * 128;
           if (leader) {
+            // three independent accumulation chains (scores, hidden half 0, hidden half 1)
+            // interleaved step by step, so one chain's accumulator latency hides behind the
+            // others
 #pragma unroll
-            for (int kk = 0; kk < R / 16; ++kk)
-              mma_ss(ts, dA + (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2),
-                     dQ + (uint64_t)((kk >> 2) * 128 + (kk & 3) * 2), IDESC_S, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < R / 16; ++kk) {
+              const uint64_t ko = (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2);
+              const uint32_t acc = kk > 0 ? 1u : 0u;
+              mma_ss(ts, dA + ko, dQ + (uint64_t)((kk >> 2) * 128 + (kk & 3) * 2), IDESC_S, acc);
+              mma_ts(td, t_w1 + kk * 8, dB + ko, IDESC_1, acc);
+              mma_ts(td + 64, t_w1 + (R / 2) + kk * 8, dB + ko, IDESC_1, acc);
+            }
             mma_commit(&bar.s_full[sb]);
+            mma_commit(&bar.d1_full[b0]);
+            if (sub == SUBS - 1) mma_commit(&bar.a_empty[st]);
+            if (n + 1 < NS && sub == SUBS - 1 && wk.next_starts_segment()) mma_commit(&bar.seg_done);
           }
+          __syncwarp();
+          return true;
         } else {
           tc_fence_after();
         }
@@ -327,11 +342,11 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
         const uint32_t td = t_d1 + b * 128;
         if (leader) {
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-#pragma unroll
-            for (int kk = 0; kk < R / 16; ++kk)
-              mma_ts(td + hh * 64, t_w1 + hh * (R / 2) + kk * 8,
-                     dB + (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2), IDESC_1, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < R / 16; ++kk) {   // the two hidden halves interleaved
+            const uint64_t ko = (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2);
+            const uint32_t acc = kk > 0 ? 1u : 0u;
+            mma_ts(td, t_w1 + kk * 8, dB + ko, IDESC_1, acc);
+            mma_ts(td + 64, t_w1 + (R / 2) + kk * 8, dB + ko, IDESC_1, acc);
           }
           mma_commit(&bar.d1_full[b]);
           if (sub == SUBS - 1) mma_commit(&bar.a_empty[st]);
@@ -356,9 +371,9 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
         const uint32_t acc0 = sub > 0 ? 1u : 0u;
         if (leader) {
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
+          for (int kk = 0; kk < 4; ++kk) {          // the two hidden halves interleaved
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
+            for (int hh = 0; hh < 2; ++hh)
               mma_ts(t_d3 + pb * 32 + hh * 16, t_d1 + b * 128 + hh * 64 + kk * 8, dP + (uint64_t)(kk * 16),
                      IDESC_3, kk > 0 ? 1u : acc0);
           }
