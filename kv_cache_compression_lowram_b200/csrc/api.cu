@@ -226,7 +226,6 @@ lowram_status lowram_cache_create(const lowram_config* cfg, const lowram_cache_s
       {evict ? src->slot : nullptr, &p_slot, evict ? B * NG * H * nC * 2 : 0},
       {src->res_ptr, &p_rptr, B * L * H * (nL + 1) * 4},
       {R ? src->res_pos : nullptr, &p_rpos, R * 2},
-      {R ? src->res_val : nullptr, &p_rval, R * d * sa},
       {(i8 && R) ? src->res_scale : nullptr, &p_rscale, (i8 && R) ? R * 2 : 0},
       {src->tail_k, &p_tk, B * L * H * T * d * st16},
       {src->tail_v, &p_tv, B * L * H * T * d * st16},
@@ -241,6 +240,15 @@ lowram_status lowram_cache_create(const lowram_config* cfg, const lowram_cache_s
       if (e != cudaSuccess) { lowram_cache_destroy(c); return cuda_fail(e, "cudaMemcpyAsync"); }
     }
   }
+  // residual rows, followed by kResPad zero rows: the tensor-core kernel loads a fixed box
+  // of kResPad rows from each chunk's first record, so the box never leaves the array
+  if ((st = alloc(c, &p_rval, (R + kResPad) * d * sa)) != LOWRAM_OK) { lowram_cache_destroy(c); return st; }
+  if (R) {
+    e = cudaMemcpyAsync(p_rval, src->res_val, R * d * sa, cudaMemcpyDeviceToDevice, cs);
+    if (e != cudaSuccess) { lowram_cache_destroy(c); return cuda_fail(e, "cudaMemcpyAsync"); }
+  }
+  e = cudaMemsetAsync(static_cast<unsigned char*>(p_rval) + R * d * sa, 0, kResPad * d * sa, cs);
+  if (e != cudaSuccess) { lowram_cache_destroy(c); return cuda_fail(e, "cudaMemsetAsync"); }
   c->cb.coeff = p_coeff; c->cb.coeff_scale = static_cast<const __half*>(p_cscale);
   c->cb.basis = p_basis; c->cb.w1 = p_w1; c->cb.w2 = p_w2; c->cb.summary = p_summ;
   c->cb.slot = static_cast<const int16_t*>(p_slot);

@@ -11,20 +11,23 @@
 //   H  = silu(2 * D1) = u + u tanh(u), written back to TMEM as fp16 (MUFU tanh)
 //   D3 = H . P                      softmax-weighted hidden sums per head (A = H from TMEM,
 //                                   B = P, the chunk's probabilities, fp16 in SMEM)
-// while a softmax warpgroup keeps the online max/sum per head and accumulates the
-// residual rows delta_t of the flagged tokens (CUDA cores).  The predictor's second layer
-// is applied once per unit in the combine kernel: sum_t p_t (W2 h_t + delta_t) =
+//   D4 = Delta^T . P_res            softmax-weighted residual rows delta_t of the flagged
+//                                   tokens (A = the rows as TMA loads them, MN-major; B = the
+//                                   probabilities at those tokens, bf16)
+// while a softmax warpgroup keeps the online max/sum per head.  The predictor's second
+// layer is applied once per unit in the combine kernel: sum_t p_t (W2 h_t + delta_t) =
 // W2 (sum_t p_t h_t) + sum_t p_t delta_t.  Key rebuild: "LowRAM Compresses KV Cache
 // Asymmetrically", section "Cross-Layer Low-Rank Key Compression"; values: same page,
 // "Core Mechanism" (Vhat = f(K), delta kept for the worst tokens); attention: "OjaKV", 3.
 //
 // Warp roles (16 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-3 idle, 4-7 and 8-11
 // two silu epilogue groups taking alternate sub-tiles (both hidden halves each), 12-15
-// softmax + residuals + accumulation of the chunks' D3.
+// softmax, the P / P_res tiles and the accumulation of the chunks' D3 / D4.
 // A warp reaches TMEM lanes 32*(warp%4) .. +31, so each warpgroup of four consecutive
 // warps covers all 128 lanes.
 // TMEM (512 columns): W1' halves [0,128), D1 double buffer x 2 halves [128,384),
-// S double buffer [384,416), D3 double buffer x 2 halves [416,480).
+// S double buffer [384,416), D3 double buffer x 2 halves [416,480), D4 double buffer
+// [480,512).
 // Every wait is bounded: on timeout the kernel raises the error word, drains its own
 // copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -43,26 +46,29 @@ constexpr int kEpiWarp0 = 4;      // first hidden-row epilogue warp
 constexpr int kSoftWarp0 = 12;    // first softmax warp
 constexpr int kHid = 256;
 constexpr int kDh = 128;
+constexpr int kResCap = kResPad;  // residual records per chunk handled by the tensor cores
+static_assert(kResCap == 32, "the P_res tile and the D4 MMAs assume 32 records");
 
 template <int R, int C>
 struct TcLayout {
   static constexpr int NT = 64;
   static constexpr int SUBS = C / NT;
   static constexpr int STAGES = 4;
-  static constexpr int RES_CAP = 32;
   static constexpr int KSLABS = R / 64;
   static constexpr int A_STAGE = KSLABS * 16384;     // 128 rows x 128 B per 64-wide K slab
   static constexpr int Q_BUF = KSLABS * 2048;        // 16 rows x 128 B per slab
   static constexpr int P_BUF = 16 * C * 2;
   static constexpr int P_SBO = (C / 8) * 128;
-  static constexpr int RES_BUF = RES_CAP * kDh * 2;
-  static constexpr int P32_BUF = 16 * C * 4;
+  static constexpr int RES_SLAB = kResCap * 128;     // 32 records x 64 dims (128 B)
+  static constexpr int RES_BUF = 2 * RES_SLAB;
+  static constexpr int PR_BUF = 16 * kResCap * 2;
+  static constexpr int PR_SBO = (kResCap / 8) * 128;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_Q = OFF_A + STAGES * A_STAGE;
-  static constexpr int OFF_P = OFF_Q + 2 * Q_BUF;
-  static constexpr int OFF_RES = OFF_P + 2 * P_BUF;
-  static constexpr int OFF_P32 = OFF_RES + STAGES * RES_BUF;
-  static constexpr int OFF_MISC = OFF_P32 + 2 * P32_BUF;
+  static constexpr int OFF_RES = OFF_Q + 2 * Q_BUF;
+  static constexpr int OFF_P = OFF_RES + STAGES * RES_BUF;
+  static constexpr int OFF_PR = OFF_P + 2 * P_BUF;
+  static constexpr int OFF_MISC = OFF_PR + 2 * PR_BUF;
   static constexpr int MISC_BYTES = 2048;
   static constexpr int SMEM = OFF_MISC + MISC_BYTES + 1024;   // + alignment slack
   // TMEM columns
@@ -70,13 +76,16 @@ struct TcLayout {
   static constexpr uint32_t T_D1 = 128;
   static constexpr uint32_t T_S = 384;
   static constexpr uint32_t T_D3 = 416;
+  static constexpr uint32_t T_D4 = 480;
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(R / 2 <= 64, "W1' half must fit 64 TMEM columns");
-  static_assert(STAGES == 4 && RES_CAP <= 32, "Misc holds 4 stages of at most 32 positions");
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(OFF_Q % 1024 == 0 && OFF_RES % 1024 == 0, "128-byte-swizzled operands need 1024-byte alignment");
 };
 
 struct Bars {
-  uint64_t a_full[4], a_empty[4];
+  uint64_t a_full[4], a_empty[4];     // coefficient tiles
+  uint64_t r_full[4], r_empty[4];     // residual rows (+ their record range and token map)
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[2], s_free[2];
   uint64_t d1_full[2], h_ready[2];
@@ -90,7 +99,7 @@ struct Bars {
 struct Misc {
   Bars bars;
   int stage_rec[4][2];               // residual record range [r0, r1) of the chunk in a stage
-  uint16_t stage_pos[4][32];         // token offsets of its first RES_CAP records
+  int8_t stage_idx[4][128];          // token -> its record index if below kResCap, else -1
   float red_max[4][16];
   float red_sum[4][16];
   uint32_t tmem_base;
@@ -98,7 +107,6 @@ struct Misc {
 };
 
 static_assert(sizeof(Misc) <= 2048, "Misc must fit its shared-memory slot");
-static_assert(sizeof(((Misc*)0)->stage_rec) / sizeof(int[2]) == 4, "one record range per stage");
 
 // Sequential walk over a CTA's chunk tiles: the unit of each chunk, the chunk's index in its
 // unit and the unit's (layer, KV head) segment, updated by counters (no division per step).
@@ -129,14 +137,17 @@ struct TileWalk {
   __device__ __forceinline__ bool next_starts_segment() const { return rem + 1 == k && ub + 1 == B; }
 };
 
-__device__ __forceinline__ float bf16_bits_to_f(uint16_t b) {
-  return __uint_as_float(((uint32_t)b) << 16);
+// Offset of element (row j, column k) in a K-major operand tile without swizzle: 8 x 16-byte
+// core matrices, K-adjacent ones 128 bytes apart, 8-row groups sbo bytes apart.
+__device__ __forceinline__ uint32_t kmajor_off(int j, int k, int sbo) {
+  return (uint32_t)((j >> 3) * sbo + (k >> 3) * 128 + (j & 7) * 16 + (k & 7) * 2);
 }
 
 template <int R, int C, int GQ>
 __global__ void __launch_bounds__(kThreadsTC, 1)
 attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __restrict__ w1f,
-                 const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmQ) {
+                 const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmQ,
+                 const __grid_constant__ CUtensorMap tmRes) {
   using Lay = TcLayout<R, C>;
   constexpr int SUBS = Lay::SUBS, STAGES = Lay::STAGES, KSLABS = Lay::KSLABS;
   extern __shared__ unsigned char smem_dyn[];
@@ -159,7 +170,9 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
   if (tid == 0) {
     for (int i = 0; i < STAGES; ++i) {
       mbar_init(&bar.a_full[i], 1);
-      mbar_init(&bar.a_empty[i], 2);      // MMA commit + softmax warpgroup
+      mbar_init(&bar.a_empty[i], 1);
+      mbar_init(&bar.r_full[i], 1);
+      mbar_init(&bar.r_empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar.q_full[i], 1);
@@ -178,8 +191,8 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
     misc->abort_flag = 0;
     mbar_init_fence();
   }
-  // zero both P tiles (rows >= g stay zero for the whole kernel)
-  for (int i = tid; i < 2 * Lay::P_BUF / 16; i += blockDim.x)
+  // zero the P and P_res tiles (rows >= g stay zero for the whole kernel)
+  for (int i = tid; i < (2 * Lay::P_BUF + 2 * Lay::PR_BUF) / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(smem + Lay::OFF_P)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
   if (warp == 1) {
@@ -193,9 +206,12 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
   const uint32_t sA = smem_u32(smem + Lay::OFF_A);
   const uint32_t sQ = smem_u32(smem + Lay::OFF_Q);
   const uint32_t sP = smem_u32(smem + Lay::OFF_P);
-  constexpr uint32_t IDESC_S = idesc_f16(128, 16, 1, 1);    // bf16 x bf16
-  constexpr uint32_t IDESC_1 = idesc_f16(128, 64, 1, 1);    // bf16 (TMEM) x bf16
-  constexpr uint32_t IDESC_3 = idesc_f16(128, 16, 0, 0);    // f16 (TMEM) x f16
+  const uint32_t sRes = smem_u32(smem + Lay::OFF_RES);
+  const uint32_t sPR = smem_u32(smem + Lay::OFF_PR);
+  constexpr uint32_t IDESC_S = idesc_f16(128, 16, 1, 1);        // bf16 x bf16
+  constexpr uint32_t IDESC_1 = idesc_f16(128, 64, 1, 1);        // bf16 (TMEM) x bf16
+  constexpr uint32_t IDESC_3 = idesc_f16(128, 16, 0, 0);        // f16 (TMEM) x f16
+  constexpr uint32_t IDESC_4 = idesc_f16(128, 16, 1, 1, 1, 0);  // bf16 (MN-major) x bf16
 
   if (warp == 0) {
     // ============================================================ TMA producer
@@ -203,7 +219,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
     // lane issues the copies.
     const bool leader = elect_one();
     if (NCH > 0) {
-      int unit_i = -1, prev_u = -1, issued = 0, q_issued = 0;
+      int unit_i = -1, prev_u = -1, issued_a = 0, issued_r = 0, q_issued = 0;
       TileWalk wk;
       wk.init(x0, g.k, g.B);
       for (int ci = 0; ci < NCH; ++ci) {
@@ -227,42 +243,55 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
           q_issued = unit_i + 1;
         }
         const int st = ci % STAGES;
-        if (ci >= STAGES && !__all_sync(0xffffffffu, mbar_wait(&bar.a_empty[st], ((ci / STAGES) - 1) & 1,
-                                                               abort_flag, err, ERR_TIMEOUT)))
+        const uint32_t par = ((ci / STAGES) - 1) & 1;
+        if (ci >= STAGES && !__all_sync(0xffffffffu, mbar_wait(&bar.a_empty[st], par, abort_flag, err, ERR_TIMEOUT)))
           break;
         const Unit un = unit_of(g, u);
         const int l = g.layer0 + un.li;
         const int grp = l / g.G;
         const int slot = sc.sel_slot[x];
         const int row0 = (int)(((((long long)un.b * NG + grp) * g.Hkv + un.hkv) * g.nL + slot) * C);
+        if (leader) {
+          mbar_expect_tx(&bar.a_full[st], (uint32_t)(C * R * 2));
+#pragma unroll
+          for (int ks = 0; ks < KSLABS; ++ks)
+            tma_load_2d(smem + Lay::OFF_A + st * Lay::A_STAGE + ks * 16384, &tmA, &bar.a_full[st], ks * 64, row0);
+        }
+        __syncwarp();
+        issued_a = ci + 1;
         const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nL + 1);
         const int r0 = rptr[slot], r1 = rptr[slot + 1];
-        const int nres = min(r1 - r0, Lay::RES_CAP);
-        // record range and positions for the softmax warpgroup (published by the arrive below)
+        const int nres = min(r1 - r0, kResCap);
+        const int my_pos = lane < nres ? (int)cb.res_pos[r0 + lane] : C;
+        if (ci >= STAGES && !__all_sync(0xffffffffu, mbar_wait(&bar.r_empty[st], par, abort_flag, err, ERR_TIMEOUT)))
+          break;
+        // record range and token -> record map for the softmax warps (published by the
+        // arrive below); a position outside the chunk is left out of the map
         if (lane == 0) {
           misc->stage_rec[st][0] = r0;
           misc->stage_rec[st][1] = r1;
         }
-        if (lane < nres) misc->stage_pos[st][lane] = cb.res_pos[r0 + lane];
+        for (int w4 = lane; w4 < C / 4; w4 += 32) reinterpret_cast<uint32_t*>(misc->stage_idx[st])[w4] = 0xffffffffu;
+        __syncwarp();
+        if (my_pos < C) misc->stage_idx[st][my_pos] = (int8_t)lane;
         __syncwarp();
         if (leader) {
-          mbar_expect_tx(&bar.a_full[st], (uint32_t)(C * R * 2 + nres * kDh * 2));
-#pragma unroll
-          for (int ks = 0; ks < KSLABS; ++ks)
-            tma_load_2d(smem + Lay::OFF_A + st * Lay::A_STAGE + ks * 16384, &tmA, &bar.a_full[st], ks * 64, row0);
-          if (nres > 0)
-            bulk_load(smem + Lay::OFF_RES + st * Lay::RES_BUF,
-                      reinterpret_cast<const unsigned char*>(cb.res_val) + (size_t)r0 * kDh * 2,
-                      (uint32_t)(nres * kDh * 2), &bar.a_full[st]);
+          // records r0 .. r0+31 in two 64-dim slabs; rows past the chunk's own records meet
+          // zero probabilities, and the cache keeps 32 zero rows after its last record
+          mbar_expect_tx(&bar.r_full[st], (uint32_t)Lay::RES_BUF);
+          tma_load_2d(smem + Lay::OFF_RES + st * Lay::RES_BUF, &tmRes, &bar.r_full[st], 0, r0);
+          tma_load_2d(smem + Lay::OFF_RES + st * Lay::RES_BUF + Lay::RES_SLAB, &tmRes, &bar.r_full[st], 64, r0);
         }
         __syncwarp();
-        issued = ci + 1;
+        issued_r = ci + 1;
       }
       if (*abort_flag && leader) {
         // let every copy this warp started land before the CTA's shared memory goes away
         volatile int never = 0;
-        for (int ci = max(0, issued - STAGES); ci < issued; ++ci)
+        for (int ci = max(0, issued_a - STAGES); ci < issued_a; ++ci)
           mbar_wait(&bar.a_full[ci % STAGES], (ci / STAGES) & 1, &never, err, ERR_TIMEOUT);
+        for (int ci = max(0, issued_r - STAGES); ci < issued_r; ++ci)
+          mbar_wait(&bar.r_full[ci % STAGES], (ci / STAGES) & 1, &never, err, ERR_TIMEOUT);
         for (int ui = max(0, q_issued - 2); ui < q_issued; ++ui)
           mbar_wait(&bar.q_full[ui & 1], (ui >> 1) & 1, &never, err, ERR_TIMEOUT);
       }
@@ -280,8 +309,10 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       const uint64_t dA0 = smem_desc(sA, 16, 1024, 2);              // coefficient tiles
       const uint64_t dQ0 = smem_desc(sQ, 16, 1024, 2);              // projected queries
       const uint64_t dP0 = smem_desc(sP, 128, Lay::P_SBO, 0);       // probabilities
+      const uint64_t dR0 = smem_desc(sRes, Lay::RES_SLAB, 1024, 2); // residual rows, MN-major
+      const uint64_t dPR0 = smem_desc(sPR, 128, Lay::PR_SBO, 0);    // probabilities at records
       const uint32_t t_w1 = tmem + Lay::T_W1, t_d1 = tmem + Lay::T_D1;
-      const uint32_t t_s = tmem + Lay::T_S, t_d3 = tmem + Lay::T_D3;
+      const uint32_t t_s = tmem + Lay::T_S, t_d3 = tmem + Lay::T_D3, t_d4 = tmem + Lay::T_D4;
       TileWalk wk;
       wk.init(x0, g.k, g.B);
       auto wait_all = [&](uint64_t* b, uint32_t par) -> bool {
@@ -362,12 +393,16 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       for (int n = 0; ok && n < NS; ++n) {
         const int ci = n / SUBS, sub = n % SUBS, b = n & 1, pb = ci & 1;
         if (!wait_all(&bar.h_ready[b], (n >> 1) & 1)) break;
+        const int st = ci % STAGES;
         if (sub == 0) {
           if (!wait_all(&bar.p_ready[pb], (ci >> 1) & 1)) break;
+          if (!wait_all(&bar.r_full[st], (ci / STAGES) & 1)) break;
           if (ci >= 2 && !wait_all(&bar.d3_free[pb], ((ci >> 1) - 1) & 1)) break;
         }
         tc_fence_after();
         const uint64_t dP = dP0 + (uint64_t)((pb * Lay::P_BUF + sub * 1024) >> 4);
+        const uint64_t dPR = dPR0 + (uint64_t)((pb * Lay::PR_BUF) >> 4);
+        const uint64_t dR = dR0 + (uint64_t)((st * Lay::RES_BUF) >> 4);
         const uint32_t acc0 = sub > 0 ? 1u : 0u;
         if (leader) {
 #pragma unroll
@@ -376,7 +411,13 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
             for (int hh = 0; hh < 2; ++hh)
               mma_ts(t_d3 + pb * 32 + hh * 16, t_d1 + b * 128 + hh * 64 + kk * 8, dP + (uint64_t)(kk * 16),
                      IDESC_3, kk > 0 ? 1u : acc0);
+            // residual rows with the chunk's first sub-tile: 16 records = two 8-row groups
+            // of the MN-major tile
+            if (sub == 0 && kk < kResCap / 16)
+              mma_ss(t_d4 + pb * 16, dR + (uint64_t)(kk * (2048 >> 4)), dPR + (uint64_t)(kk * 16), IDESC_4,
+                     kk > 0 ? 1u : 0u);
           }
+          if (sub == 0) mma_commit(&bar.r_empty[st]);
           if (sub == SUBS - 1) mma_commit(&bar.d3_full[pb]);
         }
         __syncwarp();
@@ -505,36 +546,38 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       }
     }
   } else if (warp >= kSoftWarp0) {
-    // ============================================================ softmax + residuals
-    // Per chunk: online max/sum per head, the fp16 P tile for the D3 MMA, the residual rows
-    // of the flagged tokens, and (one chunk later) the chunk's D3 = H . P folded into the
-    // softmax-weighted hidden sums.  Thread t is token t for the scores, head-dim element t
-    // for the residuals and hidden row t of both halves for D3.
+    // ============================================================ softmax + accumulation
+    // Per chunk: online max/sum per head, the fp16 P tile and the bf16 P_res tile (the
+    // probabilities at the flagged tokens) for the MMAs, residual records beyond the first
+    // 32 on CUDA cores, and (one chunk later) the chunk's D3 / D4 folded into the running
+    // sums.  Thread t is token t for the scores, hidden row t of both halves for D3 and
+    // head-dim element t for D4 and the extra records.
     const int w = warp & 3;
     const int t = w * 32 + lane;
     const uint32_t lane_off = (uint32_t)(w * 32) << 16;
-    float m_run[GQ], l_run[GQ], accD[GQ], accH0[GQ], accH1[GQ], al_prev[GQ];
+    float m_run[GQ], l_run[GQ], accD[GQ], accD4[GQ], accH0[GQ], accH1[GQ], al_prev[GQ];
 #pragma unroll
     for (int j = 0; j < GQ; ++j) {
-      m_run[j] = -INFINITY; l_run[j] = 0.f; accD[j] = 0.f; accH0[j] = 0.f; accH1[j] = 0.f;
-      al_prev[j] = 1.f;
+      m_run[j] = -INFINITY; l_run[j] = 0.f; accD[j] = 0.f; accD4[j] = 0.f; accH0[j] = 0.f;
+      accH1[j] = 0.f; al_prev[j] = 1.f;
     }
-    float* p32_base = reinterpret_cast<float*>(smem + Lay::OFF_P32);
     unsigned char* pbase = smem + Lay::OFF_P;
+    unsigned char* prbase = smem + Lay::OFF_PR;
     int cur_u = -1;
     // After a failed wait a warp stops working ("live" false) but keeps passing the named
     // barriers of every remaining chunk, so the other warps of the group never block on it;
     // once the abort flag is up every wait returns at once.
     bool live = true;
-    // fold D3 of chunk c (rescaled chunk sums H.P of both halves) into accH
-    auto fold_d3 = [&](int c) {
+    // fold D3 / D4 of chunk c (sums relative to the running max after c) into the totals
+    auto fold = [&](int c) {
       const int pb = c & 1;
       live = __all_sync(0xffffffffu, live && mbar_wait(&bar.d3_full[pb], (c >> 1) & 1, abort_flag, err, ERR_TIMEOUT));
       if (!live) return;
       tc_fence_after();
-      uint32_t v0[16], v1[16];
-      tmem_ld16(tmem + lane_off + Lay::T_D3 + (pb * 2 + 0) * 16, v0);
-      tmem_ld16(tmem + lane_off + Lay::T_D3 + (pb * 2 + 1) * 16, v1);
+      uint32_t v0[16], v1[16], v4[16];
+      tmem_ld16(tmem + lane_off + Lay::T_D3 + pb * 32, v0);
+      tmem_ld16(tmem + lane_off + Lay::T_D3 + pb * 32 + 16, v1);
+      tmem_ld16(tmem + lane_off + Lay::T_D4 + pb * 16, v4);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -543,6 +586,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       for (int j = 0; j < GQ; ++j) {
         accH0[j] = fmaf(accH0[j], al_prev[j], __uint_as_float(v0[j]));
         accH1[j] = fmaf(accH1[j], al_prev[j], __uint_as_float(v1[j]));
+        accD4[j] = fmaf(accD4[j], al_prev[j], __uint_as_float(v4[j]));
       }
     };
     auto write_partial = [&](int u) {
@@ -555,8 +599,9 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       for (int j = 0; j < GQ; ++j) {
         rec[2 * GQ + j * kHid + t] = accH0[j];
         rec[2 * GQ + j * kHid + 128 + t] = accH1[j];
-        rec[2 * GQ + GQ * kHid + j * kDh + t] = accD[j];
-        m_run[j] = -INFINITY; l_run[j] = 0.f; accD[j] = 0.f; accH0[j] = 0.f; accH1[j] = 0.f;
+        rec[2 * GQ + GQ * kHid + j * kDh + t] = accD[j] + accD4[j];
+        m_run[j] = -INFINITY; l_run[j] = 0.f; accD[j] = 0.f; accD4[j] = 0.f; accH0[j] = 0.f;
+        accH1[j] = 0.f;
       }
     };
     TileWalk wk;
@@ -566,13 +611,13 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       const int u = wk.u;
       if (u != cur_u) {
         if (cur_u >= 0) {
-          fold_d3(ci - 1);                 // the previous unit's last chunk
+          fold(ci - 1);                    // the previous unit's last chunk
           if (live) write_partial(cur_u);
         }
         cur_u = u;
       }
       const int st = ci % STAGES, sb = ci & 1, pb = ci & 1;
-      live = __all_sync(0xffffffffu, live && mbar_wait(&bar.a_full[st], (ci / STAGES) & 1, abort_flag, err, ERR_TIMEOUT) &&
+      live = __all_sync(0xffffffffu, live && mbar_wait(&bar.r_full[st], (ci / STAGES) & 1, abort_flag, err, ERR_TIMEOUT) &&
                                          mbar_wait(&bar.s_full[sb], (ci >> 1) & 1, abort_flag, err, ERR_TIMEOUT));
       uint32_t sv[16];
 #pragma unroll
@@ -590,8 +635,8 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
 #pragma unroll
       for (int j = 0; j < GQ; ++j) {
         const float s = valid ? __uint_as_float(sv[j]) : -INFINITY;
-        const float m = warp_max(s);
-        if (lane == 0) misc->red_max[w][j] = m;
+        const float mx = warp_max(s);
+        if (lane == 0) misc->red_max[w][j] = mx;
         p[j] = s;
       }
       named_bar_sync(1, 128);
@@ -604,16 +649,26 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
         p[j] = exp2f(p[j] - mn);
         m_run[j] = mn;
       }
-      // P buffer pb was last read by the MMAs of chunk ci-2, whose D3 this group has
-      // already folded (so they are complete)
-      float* p32 = p32_base + pb * 16 * C;
+      // the P and P_res buffers pb were last read by the MMAs of chunk ci-2, whose D3 / D4
+      // this group has already folded (so they are complete)
+      const int r0 = misc->stage_rec[st][0], r1 = misc->stage_rec[st][1];
+      const int nrec = r1 - r0;
+      unsigned char* pt = pbase + pb * Lay::P_BUF;
+      unsigned char* pr = prbase + pb * Lay::PR_BUF;
       if (valid && live) {
+        const int idx = misc->stage_idx[st][t];
 #pragma unroll
         for (int j = 0; j < GQ; ++j) {
-          const uint32_t off = (j >> 3) * Lay::P_SBO + (t >> 3) * 128 + (j & 7) * 16 + (t & 7) * 2;
-          *reinterpret_cast<__half*>(pbase + pb * Lay::P_BUF + off) = __float2half_rn(p[j]);
-          p32[j * C + t] = p[j];
+          *reinterpret_cast<__half*>(pt + kmajor_off(j, t, Lay::P_SBO)) = __float2half_rn(p[j]);
+          // P_res: row j, column i = probability of head j at the chunk's i-th flagged token
+          if (idx >= 0)
+            *reinterpret_cast<__nv_bfloat16*>(pr + kmajor_off(j, idx, Lay::PR_SBO)) = __float2bfloat16_rn(p[j]);
         }
+      }
+      if (live && t < kResCap && t >= nrec) {   // columns past the chunk's records
+#pragma unroll
+        for (int j = 0; j < GQ; ++j)
+          *reinterpret_cast<__nv_bfloat16*>(pr + kmajor_off(j, t, Lay::PR_SBO)) = __float2bfloat16_rn(0.f);
       }
 #pragma unroll
       for (int j = 0; j < GQ; ++j) {
@@ -629,44 +684,29 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
                    misc->red_sum[2][j] + misc->red_sum[3][j];
         accD[j] *= al[j];
       }
-      // residual rows of the chunk's flagged tokens: thread t owns head-dim element t.
-      // The producer left the record range and positions in shared memory with the rows.
-      if (live) {
-        const int r0 = misc->stage_rec[st][0], r1 = misc->stage_rec[st][1];
-        const int n = r1 - r0, nfast = min(n, Lay::RES_CAP);
-        const uint16_t* rs = reinterpret_cast<const uint16_t*>(smem + Lay::OFF_RES + st * Lay::RES_BUF);
-        const uint16_t* sp = misc->stage_pos[st];
-#pragma unroll 4
-        for (int i = 0; i < nfast; ++i) {
-          const int pos = sp[i];
-          const float dv = bf16_bits_to_f(rs[i * kDh + t]);
-#pragma unroll
-          for (int j = 0; j < GQ; ++j) accD[j] = fmaf(p32[j * C + pos], dv, accD[j]);
-        }
+      // records beyond the first kResCap (rare): CUDA cores, with the rows straight from
+      // global memory and the probabilities from the fp16 P tile
+      if (live && nrec > kResCap) {
         const uint16_t* rg = reinterpret_cast<const uint16_t*>(cb.res_val);
-        for (int i = nfast; i < n; ++i) {   // records beyond the staged ones (rare)
+        for (int i = kResCap; i < nrec; ++i) {
           const int pos = cb.res_pos[r0 + i];
-          const float dv = bf16_bits_to_f(rg[(size_t)(r0 + i) * kDh + t]);
+          if (pos >= C) continue;
+          const float dv = __uint_as_float(((uint32_t)rg[(size_t)(r0 + i) * kDh + t]) << 16);
 #pragma unroll
-          for (int j = 0; j < GQ; ++j) accD[j] = fmaf(p32[j * C + pos], dv, accD[j]);
+          for (int j = 0; j < GQ; ++j)
+            accD[j] = fmaf(__half2float(*reinterpret_cast<const __half*>(pt + kmajor_off(j, pos, Lay::P_SBO))), dv,
+                           accD[j]);
         }
       }
-      named_bar_sync(1, 128);
-      if (t == 0 && live) mbar_arrive(&bar.a_empty[st]);
-      // fold the previous chunk's D3 when it belongs to this unit (its MMAs ran meanwhile);
-      // the chunk sums of ci-1 are relative to m after ci-1, so rescale by al of ci-1 first
-      if (ci >= 1 && wk.rem != 0) {        // chunk ci-1 belongs to this unit too
-        fold_d3(ci - 1);
-      }
+      // fold the previous chunk's D3 / D4 when it belongs to this unit (its MMAs ran
+      // meanwhile); it is relative to the max after chunk ci-1, so the running sums are
+      // rescaled by that chunk's factor first
+      if (ci >= 1 && wk.rem != 0) fold(ci - 1);
 #pragma unroll
-      for (int j = 0; j < GQ; ++j) {
-        // accH is kept relative to the running max after the last folded chunk; the next
-        // fold multiplies by the rescale factor of the chunk being folded
-        al_prev[j] = al[j];
-      }
+      for (int j = 0; j < GQ; ++j) al_prev[j] = al[j];
     }
     if (NCH > 0) {
-      fold_d3(NCH - 1);
+      fold(NCH - 1);
       if (live && !*abort_flag && cur_u >= 0) write_partial(cur_u);
     }
   }
@@ -692,6 +732,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// 2-D bf16 tensor map over a row-major [rows][inner] array, boxes of 64 x box_rows elements
+// delivered in the 128-byte swizzle layout.
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
   auto enc = encode_fn();
   if (!enc) return false;
@@ -711,18 +753,24 @@ cudaError_t launch_tc(const Geom& g, const CacheBuffers& cb, const Scratch& sc, 
   using Lay = TcLayout<R, C>;
   const int NG = g.L / g.G;
   const uint64_t rows = (uint64_t)g.B * NG * g.Hkv * g.nL * C;
-  CUtensorMap tmA, tmQ;
+  CUtensorMap tmA, tmQ, tmRes;
   if (!make_map(&tmA, cb.coeff, R, rows, C)) return cudaErrorInvalidValue;
   if (!make_map(&tmQ, sc.qt_tc, R, (uint64_t)g.U * 16, 16)) return cudaErrorInvalidValue;
+  // the cache keeps kResPad zero rows after its residual rows, so every box is in bounds
+  if (!make_map(&tmRes, cb.res_val, kDh, (uint64_t)cb.n_records + kResPad, kResCap))
+    return cudaErrorInvalidValue;
   auto k = attend_tc_kernel<R, C, GQ>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
   if (e != cudaSuccess) return e;
-  k<<<g.P, kThreadsTC, Lay::SMEM, s>>>(g, cb, sc, static_cast<const __nv_bfloat16*>(w1f), tmA, tmQ);
+  k<<<g.P, kThreadsTC, Lay::SMEM, s>>>(g, cb, sc, static_cast<const __nv_bfloat16*>(w1f), tmA, tmQ,
+                                        tmRes);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+// The cache object pads its residual array by kResPad zero rows; callers that pass their
+// own arrays (the allocation-free entry point) use the CUDA-core kernels.
 bool attend_tc_supported(const Geom& g, int dtype, int store) {
   if (dtype != LOWRAM_BF16 || store != LOWRAM_STORE_NATIVE) return false;
   if (g.d != kDh || g.h != kHid || !(g.g == 4 || g.g == 8)) return false;
@@ -736,6 +784,7 @@ cudaError_t launch_attend_tc(const Geom& g, const CacheBuffers& cb, const Scratc
                              const void* w1f_tc, int n_sm, cudaStream_t s) {
   (void)n_sm;
   if (store != LOWRAM_STORE_NATIVE) return cudaErrorNotSupported;
+  if (cb.n_records + kResPad >= (1ll << 31)) return cudaErrorNotSupported;
 #define LOWRAM_TC_CASE(RR, CC, GG) \
   if (g.r == RR && g.C == CC && g.g == GG) return launch_tc<RR, CC, GG>(g, cb, sc, w1f_tc, s);
   LOWRAM_TC_CASE(128, 128, 4)

@@ -26,6 +26,7 @@ constexpr int kMaxR = 512;         // rank
 constexpr int kMaxH = 1024;        // predictor hidden width
 constexpr int kMaxChunks = 8192;   // chunks per unit
 constexpr int kMaxTail = 4096;
+constexpr int kResPad = 32;        // zero rows kept after a cache's residual rows
 
 // Geometry shared by every kernel of one decode call.
 struct Geom {
