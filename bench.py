@@ -103,6 +103,33 @@ def aggregate_rate(queries_per_rank: float, ms_total: float, ws: int):
     return total_q / (ms / 1e3), ms
 
 
+# DRAM traffic of the tensor-core attend kernel per launch (dram__bytes_read.sum +
+# dram__bytes_write.sum from one ncu capture:
+#   ncu --set full --clock-control none -k regex:attend_tc -s 1 -c 1 -o prof \
+#       python bench.py --config llama8b_32k_bf16_b1 --steps 1 --warmup 1 --no-cpu-baseline
+# 344.21 MB on that 256-unit case, scaled by the units of the named workload: 1024, x4).
+# The figure stands only while the kernel's sources are the captured ones, so it carries
+# their hash.
+ATTEND_TC_SOURCES = ("attend_tc.cu", "tc_ptx.cuh", "lowram_internal.cuh")
+MEASURED_TRAFFIC = {
+    "llama8b_32k_bf16": {"bytes": 1376841728, "sources_sha1": "1ff65992c4b3b80667a73168da76f69f757d9e0d"},
+}
+
+
+def measured_traffic(workload: str, path: str):
+    """ncu DRAM bytes per attend launch, or None (other path, workload or kernel version)."""
+    rec = MEASURED_TRAFFIC.get(workload)
+    if rec is None or path != "tc":
+        return None
+    import hashlib
+    h = hashlib.sha1()
+    csrc = os.path.join(os.path.dirname(os.path.abspath(__file__)), "kv_cache_compression_lowram_b200", "csrc")
+    for f in ATTEND_TC_SOURCES:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return rec["bytes"] if h.hexdigest() == rec["sources_sha1"] else None
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -333,7 +360,8 @@ def run_lowram(args, ws, rank, local):
                    "l2": "inputs larger than L2 (%.2f GB of algorithmic bytes per step)" % (ab["total"] / 1e9)},
         "roofline": {"bound": "hbm", "kernel": "attend_" + used_path,
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
+                     "frac": round(achieved / peak, 4),
+                     "traffic": measured_traffic(cfg.name, used_path),
                      "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": ab["attend"],
                      "launch_ms": round(attend_ms, 4)},
