@@ -317,6 +317,345 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
   for (int i = tid; i < g.g * g.d; i += blockDim.x) rec[2 * g.g + i] = acc[i];
 }
 
+// ---------------------------------------------------------------------------- fast path
+// The same computation for the common shapes (bf16, d = 128, r in {64, 128}, g in {4, 8},
+// at most kRankMax chunks), arranged so that every thread issues all of its global loads
+// before it uses any of them: the kernel above spends most of its time waiting on one
+// 16-byte load after another.  Basis and summary rows are split across threads, the raw
+// tail is staged block by block in shared memory with cooperative 16-byte loads (rows
+// padded by 16 bytes against bank conflicts), and the selected ids are placed with a
+// ballot scan instead of a serial count.
+constexpr int kFastTB = 64;               // tail tokens per staged block
+constexpr int kRowPad = 8;                // bf16 elements of padding per staged tail row
+
+template <int R, int GQ>
+struct FastSmem {
+  static constexpr int D = 128;
+  static constexpr int KROW = D + kRowPad;
+  static constexpr size_t bytes(int nC) {
+    return (size_t)nC * 8                      // keys
+           + (size_t)GQ * D * 4                // qs
+           + (size_t)GQ * R * 4                // qt
+           + (size_t)R * 4                     // qsum
+           + (size_t)nC * 4                    // scores
+           + (size_t)nC * 4                    // selected flags
+           + (size_t)kFastTB * KROW * 2        // tail K block
+           + (size_t)kFastTB * D * 2           // tail V block
+           + (size_t)GQ * kFastTB * 4          // logits / probabilities
+           + (size_t)4 * GQ * D * 4            // P.V partial sums of the 4 token quarters
+           + (size_t)3 * GQ * 4 + 64;          // mrun, lrun, alpha, warp totals
+  }
+};
+
+template <int R, int GQ>
+__global__ void __launch_bounds__(kThreads)
+select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __restrict__ q,
+                   float* __restrict__ scores_out, int32_t* __restrict__ sel_out, int tc_q_mode,
+                   int do_tail) {
+  constexpr int D = 128;
+  using SM = FastSmem<R, GQ>;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int u = blockIdx.x;
+  const Unit un = unit_of(g, u);
+  const int l = g.layer0 + un.li;
+  const int grp = l / g.G;
+  const int NG = g.L / g.G;
+  const int nC = g.nC;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(smem_raw);   // [nC]
+  float* qs = reinterpret_cast<float*>(keys + nC);                               // [GQ][D]
+  float* qt = qs + GQ * D;                                                       // [GQ][R]
+  float* qsum = qt + GQ * R;                                                     // [R]
+  float* sc_s = qsum + R;                                                        // [nC]
+  int* selv = reinterpret_cast<int*>(sc_s + nC);                                 // [nC]
+  __nv_bfloat16* kblk = reinterpret_cast<__nv_bfloat16*>(selv + nC);            // [TB][KROW]
+  __nv_bfloat16* vblk = kblk + kFastTB * SM::KROW;                               // [TB][D]
+  float* lg = reinterpret_cast<float*>(vblk + kFastTB * D);                      // [GQ][TB]
+  float* pv = lg + GQ * kFastTB;                                                 // [4][GQ][D]
+  float* mrun = pv + 4 * GQ * D;                                                 // [GQ]
+  float* lrun = mrun + GQ;
+  float* alpha = lrun + GQ;
+  int* wtot = reinterpret_cast<int*>(alpha + GQ);                                // [8]
+
+  // --- the unit's queries (GQ x 128 bf16: one 16-byte load per thread for GQ <= 16)
+  const size_t qoff = ((size_t)(un.li * g.B + un.b) * g.Hq + (size_t)un.hkv * GQ) * D;
+  if (tid < GQ * D / 8) {
+    float v[8];
+    Vec8<__nv_bfloat16>::load(q + qoff + tid * 8, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) qs[tid * 8 + i] = v[i];
+  }
+  __syncthreads();
+
+  // --- qt_j = B_l q_j: each basis row split over PARTS threads, all loads issued first
+  {
+    constexpr int PARTS = kThreads / R;          // 2 for r = 128, 4 for r = 64
+    constexpr int SEG = D / PARTS;               // elements per thread
+    const int i = tid / PARTS, part = tid % PARTS;
+    const __nv_bfloat16* row = reinterpret_cast<const __nv_bfloat16*>(cb.basis) +
+                               (((size_t)l * g.Hkv + un.hkv) * R + i) * D + part * SEG;
+    uint4 w[SEG / 8];
+#pragma unroll
+    for (int e = 0; e < SEG / 8; ++e) w[e] = __ldg(reinterpret_cast<const uint4*>(row) + e);
+    float a[GQ];
+#pragma unroll
+    for (int j = 0; j < GQ; ++j) a[j] = 0.f;
+#pragma unroll
+    for (int e = 0; e < SEG / 8; ++e) {
+      const uint32_t ww[4] = {w[e].x, w[e].y, w[e].z, w[e].w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float v0 = __uint_as_float(ww[h] << 16), v1 = __uint_as_float(ww[h] & 0xffff0000u);
+        const int col = part * SEG + e * 8 + 2 * h;
+#pragma unroll
+        for (int j = 0; j < GQ; ++j) a[j] = fmaf(v1, qs[j * D + col + 1], fmaf(v0, qs[j * D + col], a[j]));
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < GQ; ++j) {
+#pragma unroll
+      for (int o = 1; o < PARTS; o <<= 1) a[j] += __shfl_xor_sync(0xffffffffu, a[j], o);
+    }
+    if (part == 0) {
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) qt[j * R + i] = a[j];
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < R; i += kThreads) {
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < GQ; ++j) s += qt[j * R + i];
+    qsum[i] = s;
+  }
+  for (int i = tid; i < GQ * R; i += kThreads) sc.qt[(size_t)u * GQ * R + i] = qt[i] * g.qk_scale_log2;
+  if (tc_q_mode) {
+    for (int i = tid; i < 16 * R; i += kThreads) {
+      const int j = i / R;
+      const float v = j < GQ ? qt[i] * g.qk_scale_log2 : 0.f;
+      if (tc_q_mode == 1)
+        reinterpret_cast<__nv_bfloat16*>(sc.qt_tc)[(size_t)u * 16 * R + i] = __float2bfloat16_rn(v);
+      else
+        reinterpret_cast<__half*>(sc.qt_tc)[(size_t)u * 16 * R + i] = __float2half_rn(v);
+    }
+  }
+  __syncthreads();
+
+  // --- chunk scores: one thread per chunk, the whole summary row loaded at once
+  const int16_t* slot = cb.slot ? cb.slot + (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * nC : nullptr;
+  const __nv_bfloat16* summ = reinterpret_cast<const __nv_bfloat16*>(cb.summary) +
+                              (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * (size_t)g.nL * R;
+  const float inv_sqrt_d = rsqrtf((float)D);
+  for (int c = tid; c < nC; c += kThreads) {
+    const int sl = slot ? (int)slot[c] : c;
+    float s = -INFINITY;
+    if (sl >= 0 && sl < g.nL) {
+      const uint4* row = reinterpret_cast<const uint4*>(summ + (size_t)sl * R);
+      uint4 w[R / 8];
+#pragma unroll
+      for (int e = 0; e < R / 8; ++e) w[e] = __ldg(row + e);
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int e = 0; e < R / 8; ++e) {
+        const uint32_t ww[4] = {w[e].x, w[e].y, w[e].z, w[e].w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          a0 = fmaf(__uint_as_float(ww[h] << 16), qsum[e * 8 + 2 * h], a0);
+          a1 = fmaf(__uint_as_float(ww[h] & 0xffff0000u), qsum[e * 8 + 2 * h + 1], a1);
+        }
+      }
+      s = (a0 + a1) * inv_sqrt_d;
+    } else if (sl >= g.nL) {
+      atomicOr(sc.err, ERR_SLOT);
+    }
+    sc_s[c] = s;
+    keys[c] = ((unsigned long long)(~float_order(s)) << 32) | (unsigned)c;
+  }
+  __syncthreads();
+  if (scores_out) {
+    float* so = scores_out + ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * nC;
+    for (int c = tid; c < nC; c += kThreads) so[c] = sc_s[c];
+  }
+
+  // --- top-k by rank count (keys are distinct: the id is in the low bits), then the
+  // selected ids in ascending order by a ballot scan
+  for (int c = tid; c < nC; c += kThreads) {
+    const unsigned long long kc = keys[c];
+    int rank = 0;
+#pragma unroll 8
+    for (int c2 = 0; c2 < nC; ++c2) rank += keys[c2] < kc ? 1 : 0;
+    selv[c] = rank < g.k ? 1 : 0;
+  }
+  __syncthreads();
+  int32_t* sel_slot = sc.sel_slot + (size_t)u * g.k;
+  int32_t* sel_id = sc.sel_id + (size_t)u * g.k;
+  int32_t* sel_user = sel_out ? sel_out + ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * g.k : nullptr;
+  int run = 0;
+  for (int base = 0; base < nC; base += kThreads) {
+    const int c = base + tid;
+    const int f = c < nC ? selv[c] : 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, f);
+    if (lane == 0) wtot[warp] = __popc(bal);
+    __syncthreads();
+    int woff = 0, btot = 0;
+#pragma unroll
+    for (int w2 = 0; w2 < kThreads / 32; ++w2) {
+      const int t2 = wtot[w2];
+      woff += w2 < warp ? t2 : 0;
+      btot += t2;
+    }
+    if (f) {
+      const int pos = run + woff + __popc(bal & ((1u << lane) - 1u));
+      int sl = slot ? (int)slot[c] : c;
+      if (sl < 0 || sl >= g.nL) {
+        atomicOr(sc.err, ERR_SELECT);
+        sl = 0;
+      }
+      if (pos < g.k) {
+        sel_slot[pos] = sl;
+        sel_id[pos] = c;
+        if (sel_user) sel_user[pos] = c;
+      }
+    }
+    run += btot;
+    __syncthreads();   // wtot is rewritten by the next round
+  }
+  if (!do_tail) return;
+
+  // --- raw tail: partial softmax over its tokens, staged in blocks of kFastTB tokens
+  int tl = cb.tail_len[un.b];
+  if (tl < 0 || tl > g.T) {
+    if (tid == 0) atomicOr(sc.err, ERR_TAIL_LEN);
+    tl = tl < 0 ? 0 : g.T;
+  }
+  constexpr int NACC = GQ * D / 2 / kThreads;   // (head, dim pair) sums per thread
+  float accr[NACC][2];
+#pragma unroll
+  for (int n = 0; n < NACC; ++n) accr[n][0] = accr[n][1] = 0.f;
+  if (tid < GQ) {
+    mrun[tid] = -INFINITY;
+    lrun[tid] = 0.f;
+  }
+  __syncthreads();
+  const size_t toff = (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (size_t)g.T * D;
+  const __nv_bfloat16* tk = reinterpret_cast<const __nv_bfloat16*>(cb.tail_k) + toff;
+  const __nv_bfloat16* tv = reinterpret_cast<const __nv_bfloat16*>(cb.tail_v) + toff;
+  for (int t0 = 0; t0 < tl; t0 += kFastTB) {
+    const int nb = min(kFastTB, tl - t0);
+    // stage the block's key and value rows: 16 x 16 bytes per row, 4 + 4 loads per thread
+    {
+      uint4 kv[8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int it = tid + k * kThreads, t = it >> 4, e = it & 15;
+        const bool in = t < nb;
+        kv[k] = in ? __ldg(reinterpret_cast<const uint4*>(tk + (size_t)(t0 + t) * D) + e) : make_uint4(0, 0, 0, 0);
+        kv[4 + k] = in ? __ldg(reinterpret_cast<const uint4*>(tv + (size_t)(t0 + t) * D) + e) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int it = tid + k * kThreads, t = it >> 4, e = it & 15;
+        *reinterpret_cast<uint4*>(kblk + t * SM::KROW + e * 8) = kv[k];
+        *reinterpret_cast<uint4*>(vblk + t * D + e * 8) = kv[4 + k];
+      }
+    }
+    __syncthreads();
+    // logits: thread (token, GQ/4 heads)
+    {
+      constexpr int JPT = GQ / 4;
+      const int t = tid & (kFastTB - 1), jb = tid / kFastTB;
+      float a[JPT];
+#pragma unroll
+      for (int jj = 0; jj < JPT; ++jj) a[jj] = 0.f;
+      const uint4* krow = reinterpret_cast<const uint4*>(kblk + t * SM::KROW);
+#pragma unroll 4
+      for (int e = 0; e < D / 8; ++e) {
+        const uint4 w = krow[e];
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float v0 = __uint_as_float(ww[h] << 16), v1 = __uint_as_float(ww[h] & 0xffff0000u);
+#pragma unroll
+          for (int jj = 0; jj < JPT; ++jj) {
+            const float* qq = qs + (jb * JPT + jj) * D + e * 8 + 2 * h;
+            a[jj] = fmaf(v1, qq[1], fmaf(v0, qq[0], a[jj]));
+          }
+        }
+      }
+#pragma unroll
+      for (int jj = 0; jj < JPT; ++jj)
+        lg[(jb * JPT + jj) * kFastTB + t] = t < nb ? a[jj] * g.qk_scale_log2 : -INFINITY;
+    }
+    __syncthreads();
+    // online softmax update: one warp per head
+    if (warp < GQ) {
+      const int j = warp;
+      const float x0 = lg[j * kFastTB + lane], x1 = lg[j * kFastTB + 32 + lane];
+      const float mnew = fmaxf(mrun[j], warp_max(fmaxf(x0, x1)));
+      const float p0 = exp2f(x0 - mnew), p1 = exp2f(x1 - mnew);
+      lg[j * kFastTB + lane] = p0;
+      lg[j * kFastTB + 32 + lane] = p1;
+      const float ssum = warp_sum(p0 + p1);
+      if (lane == 0) {
+        const float a = exp2f(mrun[j] - mnew);   // 0 while mrun = -inf
+        alpha[j] = a;
+        lrun[j] = lrun[j] * a + ssum;
+        mrun[j] = mnew;
+      }
+    }
+    __syncthreads();
+    // P.V over the block: thread (dim pair, quarter of the tokens), all heads
+    {
+      const int dp = tid & 63, tq = tid >> 6;
+      float sacc[GQ][2];
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) sacc[j][0] = sacc[j][1] = 0.f;
+      const int tb = tq * (kFastTB / 4), te = min(tb + kFastTB / 4, nb);
+      for (int t = tb; t < te; ++t) {
+        const uint32_t w = reinterpret_cast<const uint32_t*>(vblk + t * D)[dp];
+        const float v0 = __uint_as_float(w << 16), v1 = __uint_as_float(w & 0xffff0000u);
+#pragma unroll
+        for (int j = 0; j < GQ; ++j) {
+          const float pj = lg[j * kFastTB + t];
+          sacc[j][0] = fmaf(pj, v0, sacc[j][0]);
+          sacc[j][1] = fmaf(pj, v1, sacc[j][1]);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) {
+        pv[(tq * GQ + j) * D + 2 * dp] = sacc[j][0];
+        pv[(tq * GQ + j) * D + 2 * dp + 1] = sacc[j][1];
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int n = 0; n < NACC; ++n) {
+      const int it = tid + n * kThreads, j = it >> 6, dp = it & 63;
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        s0 += pv[(q4 * GQ + j) * D + 2 * dp];
+        s1 += pv[(q4 * GQ + j) * D + 2 * dp + 1];
+      }
+      accr[n][0] = accr[n][0] * alpha[j] + s0;
+      accr[n][1] = accr[n][1] * alpha[j] + s1;
+    }
+    __syncthreads();   // the next block reuses the staging buffers
+  }
+  float* rec = sc.tail_part + (size_t)u * g.tail_stride;
+  if (tid < GQ) {
+    rec[tid] = mrun[tid];
+    rec[GQ + tid] = lrun[tid];
+  }
+#pragma unroll
+  for (int n = 0; n < NACC; ++n) {
+    const int it = tid + n * kThreads, j = it >> 6, dp = it & 63;
+    rec[2 * GQ + j * D + 2 * dp] = accr[n][0];
+    rec[2 * GQ + j * D + 2 * dp + 1] = accr[n][1];
+  }
+}
+
 size_t select_smem_bytes(const Geom& g) {
   const int nCp = g.nC <= kRankMax ? g.nC : next_pow2(g.nC);
   int kp = 1;
@@ -329,9 +668,35 @@ size_t select_smem_bytes(const Geom& g) {
 
 }  // namespace
 
+namespace {
+
+template <int R, int GQ>
+cudaError_t launch_select_fast(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const void* q,
+                               float* scores_out, int32_t* sel_out, int tc_q_mode, bool tail,
+                               cudaStream_t s) {
+  const size_t smem = FastSmem<R, GQ>::bytes(g.nC);
+  auto k = select_fast_kernel<R, GQ>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  k<<<g.U, kThreads, smem, s>>>(g, cb, sc, static_cast<const __nv_bfloat16*>(q), scores_out, sel_out,
+                                tc_q_mode, tail ? 1 : 0);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t launch_select(const Geom& g, const CacheBuffers& cb, const Scratch& sc, int dtype,
                           const void* q, float* scores_out, int32_t* sel_out, int tc_q_mode,
                           bool tail, cudaStream_t s) {
+  if (dtype == LOWRAM_BF16 && g.d == 128 && g.nC <= kRankMax && (reinterpret_cast<uintptr_t>(q) & 15) == 0) {
+#define LOWRAM_SELECT_FAST(RR, GG) \
+    if (g.r == RR && g.g == GG) return launch_select_fast<RR, GG>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s);
+    LOWRAM_SELECT_FAST(128, 4)
+    LOWRAM_SELECT_FAST(128, 8)
+    LOWRAM_SELECT_FAST(64, 4)
+    LOWRAM_SELECT_FAST(64, 8)
+#undef LOWRAM_SELECT_FAST
+  }
   const size_t smem = select_smem_bytes(g);
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   if (dtype == LOWRAM_F32) {
