@@ -122,6 +122,105 @@ combine_kernel(Geom g, CacheBuffers cb, Scratch sc, T* __restrict__ out) {
   }
 }
 
+// The same merge for bf16 with d = 128, h = 256, g in {4, 8}, arranged so that no thread
+// waits on one load after another: each W2 row is split over two threads whose 16 x 16-byte
+// loads are all issued on entry (they land while the partials are merged), and the
+// partial records are read as float4.
+template <int GQ>
+__global__ void __launch_bounds__(kThreads)
+combine_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, __nv_bfloat16* __restrict__ out) {
+  constexpr int D = 128, H = 256;
+  extern __shared__ __align__(16) float sm[];
+  const int u = blockIdx.x;
+  const Unit un = unit_of(g, u);
+  const int l = g.layer0 + un.li;
+  const int tid = threadIdx.x;
+  // this thread's half of W2 row dd, requested before anything else
+  const int dd = tid >> 1, half = tid & 1;
+  const uint4* wrow = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(cb.w2) +
+                                                     (((size_t)l * g.Hkv + un.hkv) * D + dd) * H + half * (H / 2));
+  uint4 w[H / 16];
+#pragma unroll
+  for (int e = 0; e < H / 16; ++e) w[e] = __ldg(wrow + e);
+
+  const long long total = (long long)g.U * g.k;
+  const int c0 = cta_of_tile(total, g.P, (long long)u * g.k);
+  const int c1 = cta_of_tile(total, g.P, (long long)(u + 1) * g.k - 1);
+  const int nrec = c1 - c0 + 1;
+  if (nrec > g.max_rec) {  // cannot happen with a consistent tile partition
+    if (tid == 0) atomicOr(sc.err, ERR_SELECT);
+    return;
+  }
+  float* accH = sm;                 // [GQ][H]
+  float* accD = accH + GQ * H;      // [GQ][D]
+  float* lsum = accD + GQ * D;      // [GQ]
+  float* wts = lsum + GQ;           // [nrec + 1][GQ]  (last row: tail)
+  const float* trec = sc.tail_part + (size_t)u * g.tail_stride;
+  const float* rec0 = sc.part + (size_t)(u + c0) * g.rec_stride;
+  if (tid < GQ) {
+    const int j = tid;
+    float M = trec[j];
+    for (int r = 0; r < nrec; ++r) M = fmaxf(M, rec0[(size_t)r * g.rec_stride + j]);
+    float L = 0.f;
+    for (int r = 0; r < nrec; ++r) {
+      const float* rec = rec0 + (size_t)r * g.rec_stride;
+      const float wr = rec[j] == -INFINITY ? 0.f : exp2f(rec[j] - M);
+      wts[r * GQ + j] = wr;
+      L += wr * rec[GQ + j];
+    }
+    const float wt = trec[j] == -INFINITY ? 0.f : exp2f(trec[j] - M);
+    wts[nrec * GQ + j] = wt;
+    lsum[j] = L + wt * trec[GQ + j];
+  }
+  __syncthreads();
+  // weighted hidden sums and residual/tail sums, four floats per thread and record
+  for (int i4 = tid; i4 < GQ * H / 4; i4 += kThreads) {
+    const int j = (i4 * 4) / H;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r = 0; r < nrec; ++r) {
+      const float4 v = *reinterpret_cast<const float4*>(rec0 + (size_t)r * g.rec_stride + 2 * GQ + i4 * 4);
+      const float wr = wts[r * GQ + j];
+      a.x = fmaf(wr, v.x, a.x); a.y = fmaf(wr, v.y, a.y); a.z = fmaf(wr, v.z, a.z); a.w = fmaf(wr, v.w, a.w);
+    }
+    *reinterpret_cast<float4*>(accH + i4 * 4) = a;
+  }
+  for (int i4 = tid; i4 < GQ * D / 4; i4 += kThreads) {
+    const int j = (i4 * 4) / D;
+    const float wt = wts[nrec * GQ + j];
+    const float4 tv = *reinterpret_cast<const float4*>(trec + 2 * GQ + i4 * 4);
+    float4 a = make_float4(wt * tv.x, wt * tv.y, wt * tv.z, wt * tv.w);
+    for (int r = 0; r < nrec; ++r) {
+      const float4 v = *reinterpret_cast<const float4*>(rec0 + (size_t)r * g.rec_stride + 2 * GQ + GQ * H + i4 * 4);
+      const float wr = wts[r * GQ + j];
+      a.x = fmaf(wr, v.x, a.x); a.y = fmaf(wr, v.y, a.y); a.z = fmaf(wr, v.z, a.z); a.w = fmaf(wr, v.w, a.w);
+    }
+    *reinterpret_cast<float4*>(accD + i4 * 4) = a;
+  }
+  __syncthreads();
+  // second predictor layer: this thread's half row against every head's hidden sums
+  float a[GQ];
+#pragma unroll
+  for (int j = 0; j < GQ; ++j) a[j] = 0.f;
+#pragma unroll
+  for (int e = 0; e < H / 16; ++e) {
+    const uint32_t ww[4] = {w[e].x, w[e].y, w[e].z, w[e].w};
+#pragma unroll
+    for (int h2 = 0; h2 < 4; ++h2) {
+      const float v0 = __uint_as_float(ww[h2] << 16), v1 = __uint_as_float(ww[h2] & 0xffff0000u);
+      const int m = half * (H / 2) + e * 8 + 2 * h2;
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) a[j] = fmaf(v1, accH[j * H + m + 1], fmaf(v0, accH[j * H + m], a[j]));
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < GQ; ++j) a[j] += __shfl_xor_sync(0xffffffffu, a[j], 1);
+  if (half == 0) {
+    __nv_bfloat16* o = out + ((size_t)(un.li * g.B + un.b) * g.Hq + (size_t)un.hkv * GQ) * D;
+#pragma unroll
+    for (int j = 0; j < GQ; ++j) o[(size_t)j * D + dd] = __float2bfloat16_rn((a[j] + accD[j * D + dd]) / lsum[j]);
+  }
+}
+
 // W1'[i][rr] = sum_dd W1[i][dd] * B_l[rr][dd] for every (layer, KV head).
 template <typename T>
 __global__ void fold_kernel(Geom g, const T* __restrict__ w1, const T* __restrict__ basis,
@@ -204,6 +303,11 @@ cudaError_t launch_combine(const Geom& g, const CacheBuffers& cb, const Scratch&
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<g.U, kThreads, smem, s>>>(g, cb, sc, static_cast<float*>(out));
+  } else if (g.d == 128 && g.h == 256 && (g.g == 4 || g.g == 8)) {
+    auto k = g.g == 4 ? combine_fast_kernel<4> : combine_fast_kernel<8>;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k<<<g.U, kThreads, smem, s>>>(g, cb, sc, static_cast<__nv_bfloat16*>(out));
   } else {
     auto k = combine_kernel<__nv_bfloat16>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
