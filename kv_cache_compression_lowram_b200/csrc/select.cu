@@ -326,6 +326,16 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
 // padded by 16 bytes against bank conflicts), and the selected ids are placed with a
 // ballot scan instead of a serial count.
 constexpr int kFastTB = 64;               // tail tokens per staged block
+
+// 16-byte asynchronous copy global -> shared (zero-filled when !valid); completes at the
+// next cp.async.wait_group.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, bool valid) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gsrc), "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 constexpr int kRowPad = 8;                // bf16 elements of padding per staged tail row
 
 template <int R, int GQ>
@@ -377,6 +387,29 @@ select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
   float* lrun = mrun + GQ;
   float* alpha = lrun + GQ;
   int* wtot = reinterpret_cast<int*>(alpha + GQ);                                // [8]
+  __shared__ int radix_state[2];
+
+  // the raw tail's first block goes to shared memory asynchronously right away; it lands
+  // while the queries are projected and the chunks scored and selected
+  int tl = do_tail ? cb.tail_len[un.b] : 0;
+  if (tl < 0 || tl > g.T) {
+    if (tid == 0) atomicOr(sc.err, ERR_TAIL_LEN);
+    tl = tl < 0 ? 0 : g.T;
+  }
+  const size_t toff = (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (size_t)g.T * D;
+  const __nv_bfloat16* tk = reinterpret_cast<const __nv_bfloat16*>(cb.tail_k) + toff;
+  const __nv_bfloat16* tv = reinterpret_cast<const __nv_bfloat16*>(cb.tail_v) + toff;
+  if (do_tail) {
+    const int nb0 = min(kFastTB, tl);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int it = tid + k * kThreads, t = it >> 4, e = it & 15;
+      const bool in = t < nb0;
+      cp_async16(kblk + t * SM::KROW + e * 8, in ? tk + (size_t)t * D + e * 8 : tk, in);
+      cp_async16(vblk + t * D + e * 8, in ? tv + (size_t)t * D + e * 8 : tv, in);
+    }
+    cp_async_commit();
+  }
 
   // --- the unit's queries (GQ x 128 bf16: one 16-byte load per thread for GQ <= 16)
   const size_t qoff = ((size_t)(un.li * g.B + un.b) * g.Hq + (size_t)un.hkv * GQ) * D;
@@ -478,16 +511,66 @@ select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
     for (int c = tid; c < nC; c += kThreads) so[c] = sc_s[c];
   }
 
-  // --- top-k by rank count (keys are distinct: the id is in the low bits), then the
-  // selected ids in ascending order by a ballot scan
-  for (int c = tid; c < nC; c += kThreads) {
-    const unsigned long long kc = keys[c];
-    int rank = 0;
-#pragma unroll 8
-    for (int c2 = 0; c2 < nC; ++c2) rank += keys[c2] < kc ? 1 : 0;
-    selv[c] = rank < g.k ? 1 : 0;
+  // --- top-k: radix select on the 32-bit order key (ascending = descending score), 8 bits
+  // a pass, finds the k-th smallest key T and how many keys equal to T are still to take;
+  // those go to the lowest ids.  hist reuses the logit buffer (free until the tail).
+  int* hist = reinterpret_cast<int*>(lg);
+  uint32_t prefix = 0;
+  int kk = g.k;
+#pragma unroll 1
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    hist[tid] = 0;
+    __syncthreads();
+    for (int c = tid; c < nC; c += kThreads) {
+      const uint32_t k32 = (uint32_t)(keys[c] >> 32);
+      if (shift == 24 || (k32 >> (shift + 8)) == (prefix >> (shift + 8))) atomicAdd(&hist[(k32 >> shift) & 255], 1);
+    }
+    __syncthreads();
+    const int hv = hist[tid];
+    int v = hv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int nv = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += nv;
+    }
+    if (lane == 31) wtot[warp] = v;
+    __syncthreads();
+    int woff = 0;
+#pragma unroll
+    for (int w2 = 0; w2 < kThreads / 32; ++w2) woff += w2 < warp ? wtot[w2] : 0;
+    const int incl = v + woff, excl = incl - hv;
+    if (excl < kk && incl >= kk) {
+      radix_state[0] = tid;
+      radix_state[1] = excl;
+    }
+    __syncthreads();
+    prefix |= (uint32_t)radix_state[0] << shift;
+    kk -= radix_state[1];
+    __syncthreads();   // hist and wtot are rewritten by the next pass
   }
-  __syncthreads();
+  // selected: key below T, or equal to T and among the kk lowest such ids
+  {
+    int eqrun = 0;
+    for (int base = 0; base < nC; base += kThreads) {
+      const int c = base + tid;
+      const uint32_t k32 = c < nC ? (uint32_t)(keys[c] >> 32) : 0xffffffffu;
+      const bool feq = c < nC && k32 == prefix;
+      const unsigned beq = __ballot_sync(0xffffffffu, feq);
+      if (lane == 0) wtot[warp] = __popc(beq);
+      __syncthreads();
+      int woff = 0, btot = 0;
+#pragma unroll
+      for (int w2 = 0; w2 < kThreads / 32; ++w2) {
+        const int t2 = wtot[w2];
+        woff += w2 < warp ? t2 : 0;
+        btot += t2;
+      }
+      const int eqrank = eqrun + woff + __popc(beq & ((1u << lane) - 1u));
+      if (c < nC) selv[c] = (k32 < prefix || (feq && eqrank < kk)) ? 1 : 0;
+      eqrun += btot;
+      __syncthreads();
+    }
+  }
   int32_t* sel_slot = sc.sel_slot + (size_t)u * g.k;
   int32_t* sel_id = sc.sel_id + (size_t)u * g.k;
   int32_t* sel_user = sel_out ? sel_out + ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * g.k : nullptr;
@@ -524,11 +607,6 @@ select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
   if (!do_tail) return;
 
   // --- raw tail: partial softmax over its tokens, staged in blocks of kFastTB tokens
-  int tl = cb.tail_len[un.b];
-  if (tl < 0 || tl > g.T) {
-    if (tid == 0) atomicOr(sc.err, ERR_TAIL_LEN);
-    tl = tl < 0 ? 0 : g.T;
-  }
   constexpr int NACC = GQ * D / 2 / kThreads;   // (head, dim pair) sums per thread
   float accr[NACC][2];
 #pragma unroll
@@ -538,13 +616,12 @@ select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
     lrun[tid] = 0.f;
   }
   __syncthreads();
-  const size_t toff = (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (size_t)g.T * D;
-  const __nv_bfloat16* tk = reinterpret_cast<const __nv_bfloat16*>(cb.tail_k) + toff;
-  const __nv_bfloat16* tv = reinterpret_cast<const __nv_bfloat16*>(cb.tail_v) + toff;
+  cp_async_wait_all();   // the first block (zero rows past the tail when it is short)
   for (int t0 = 0; t0 < tl; t0 += kFastTB) {
     const int nb = min(kFastTB, tl - t0);
     // stage the block's key and value rows: 16 x 16 bytes per row, 4 + 4 loads per thread
-    {
+    // (the first block is already in place)
+    if (t0 > 0) {
       uint4 kv[8];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
