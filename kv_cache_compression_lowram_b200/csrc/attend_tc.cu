@@ -1,7 +1,8 @@
 // Steps 3-5 on tcgen05 tensor cores (sm_100a): rebuild the selected chunks on chip and
 // attend over them, fused in one persistent kernel.
 //
-// Per selected chunk of C tokens (coefficient rows A_c, C x r, bf16) of a unit:
+// Per selected chunk of C tokens (coefficient rows A_c, C x r, bf16; fp16 when the cache
+// stores int8 rows, see below) of a unit:
 //   S  = A_c . Qt^T                 scores q_j . khat_t / sqrt(d) * log2(e) in the low-rank
 //                                   form (Qt_j = B_l q_j, "OjaKV" 3.1 projects queries into
 //                                   the key basis); M=128 tokens, N=16 heads (g used)
@@ -13,14 +14,15 @@
 //                                   B = P, the chunk's probabilities, fp16 in SMEM)
 //   D4 = Delta^T . P_res            softmax-weighted residual rows delta_t of the flagged
 //                                   tokens (A = the rows as TMA loads them, MN-major; B = the
-//                                   probabilities at those tokens, bf16)
+//                                   probabilities at those tokens, bf16 / fp16)
 // while a softmax warpgroup keeps the online max/sum per head.  The predictor's second
 // layer is applied once per unit in the combine kernel: sum_t p_t (W2 h_t + delta_t) =
 // W2 (sum_t p_t h_t) + sum_t p_t delta_t.  Key rebuild: "LowRAM Compresses KV Cache
 // Asymmetrically", section "Cross-Layer Low-Rank Key Compression"; values: same page,
 // "Core Mechanism" (Vhat = f(K), delta kept for the worst tokens); attention: "OjaKV", 3.
 //
-// Warp roles (16 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-3 idle, 4-7 and 8-11
+// Warp roles (16 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-3 int8 converters
+// (idle for a native store), 4-7 and 8-11
 // two silu epilogue groups taking alternate sub-tiles (both hidden halves each), 12-15
 // softmax, the P / P_res tiles and the accumulation of the chunks' D3 / D4.
 // A warp reaches TMEM lanes 32*(warp%4) .. +31, so each warpgroup of four consecutive
@@ -49,11 +51,18 @@ constexpr int kDh = 128;
 constexpr int kResCap = kResPad;  // residual records per chunk handled by the tensor cores
 static_assert(kResCap == 32, "the P_res tile and the D4 MMAs assume 32 records");
 
-template <int R, int C>
+// I8: the cache stores coefficients and residual rows as int8 with an fp16 scale per row
+// ("LowRAM Compresses KV Cache Asymmetrically", composition with quantisation); they arrive
+// in an int8 staging ring and warps 2-3 write the scaled tiles as fp16 (every integer of
+// |x| <= 127 and its product with the scale fit fp16 with 11 significant bits, and the
+// conversion needs no int-to-float instructions, which share a unit with the epilogue's
+// tanh).  The operands that meet them in an MMA (W1', the projected queries, P_res) are fp16
+// too.
+template <int R, int C, bool I8>
 struct TcLayout {
   static constexpr int NT = 64;
   static constexpr int SUBS = C / NT;
-  static constexpr int STAGES = 4;
+  static constexpr int STAGES = I8 ? 3 : 4;
   static constexpr int KSLABS = R / 64;
   static constexpr int A_STAGE = KSLABS * 16384;     // 128 rows x 128 B per 64-wide K slab
   static constexpr int Q_BUF = KSLABS * 2048;        // 16 rows x 128 B per slab
@@ -68,8 +77,12 @@ struct TcLayout {
   static constexpr int OFF_RES = OFF_Q + 2 * Q_BUF;
   static constexpr int OFF_P = OFF_RES + STAGES * RES_BUF;
   static constexpr int OFF_PR = OFF_P + 2 * P_BUF;
-  static constexpr int OFF_MISC = OFF_PR + 2 * PR_BUF;
-  static constexpr int MISC_BYTES = 2048;
+  static constexpr int SA_SLOT = C * R + C * 2;           // int8 tile + fp16 row scales
+  static constexpr int SR_SLOT = kResCap * kDh;            // int8 residual rows
+  static constexpr int OFF_SA = OFF_PR + 2 * PR_BUF;
+  static constexpr int OFF_SR = OFF_SA + (I8 ? 2 * SA_SLOT : 0);
+  static constexpr int OFF_MISC = OFF_SR + (I8 ? 2 * SR_SLOT : 0);
+  static constexpr int MISC_BYTES = 3072;
   static constexpr int SMEM = OFF_MISC + MISC_BYTES + 1024;   // + alignment slack
   // TMEM columns
   static constexpr uint32_t T_W1 = 0;
@@ -80,6 +93,7 @@ struct TcLayout {
   static constexpr uint32_t TMEM_COLS = 512;
   static_assert(R / 2 <= 64, "W1' half must fit 64 TMEM columns");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static_assert(SA_SLOT % 16 == 0 && OFF_SA % 16 == 0, "bulk copies need 16-byte alignment");
   static_assert(OFF_Q % 1024 == 0 && OFF_RES % 1024 == 0, "128-byte-swizzled operands need 1024-byte alignment");
 };
 
@@ -91,6 +105,8 @@ struct Bars {
   uint64_t d1_full[2], h_ready[2];
   uint64_t p_ready[2];
   uint64_t d3_full[2], d3_free[2];
+  uint64_t stg_full[2], stg_empty[2];   // int8 coefficient staging (int8 store)
+  uint64_t rstg_full[2], rstg_empty[2]; // int8 residual staging (int8 store)
   uint64_t w1_ready;   // W1' of the next (layer, KV head) is in TMEM
   uint64_t seg_done;   // every MMA that read the previous W1' is complete
   uint64_t drain;
@@ -100,13 +116,14 @@ struct Misc {
   Bars bars;
   int stage_rec[4][2];               // residual record range [r0, r1) of the chunk in a stage
   int8_t stage_idx[4][128];          // token -> its record index if below kResCap, else -1
+  __half stage_rs[4][32];            // int8 store: scales of the first kResCap records (0 past)
   float red_max[4][16];
   float red_sum[4][16];
   uint32_t tmem_base;
   int abort_flag;
 };
 
-static_assert(sizeof(Misc) <= 2048, "Misc must fit its shared-memory slot");
+static_assert(sizeof(Misc) <= 3072, "Misc must fit its shared-memory slot");
 
 // Sequential walk over a CTA's chunk tiles: the unit of each chunk, the chunk's index in its
 // unit and the unit's (layer, KV head) segment, updated by counters (no division per step).
@@ -143,12 +160,36 @@ __device__ __forceinline__ uint32_t kmajor_off(int j, int k, int sbo) {
   return (uint32_t)((j >> 3) * sbo + (k >> 3) * 128 + (j & 7) * 16 + (k & 7) * 2);
 }
 
-template <int R, int C, int GQ>
+// One 16-bit MMA operand element: fp16 for the int8 variant, bf16 otherwise.
+template <bool F16>
+__device__ __forceinline__ void st_op16(unsigned char* p, float v) {
+  if (F16)
+    *reinterpret_cast<__half*>(p) = __float2half_rn(v);
+  else
+    *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(v);
+}
+
+// Four int8 values (one 32-bit word, lowest byte first) times a scale, as two fp16 pairs.
+// Flipping the sign bit gives x + 128 as an unsigned byte u; the fp16 with bit pattern
+// 0x6400 | u is 1024 + u exactly, so subtracting 1152 gives x exactly, and the product with
+// the scale is rounded once (to nearest).
+__device__ __forceinline__ void i8x4_scaled_f16(uint32_t w, __half2 scale, uint32_t& lo, uint32_t& hi) {
+  const uint32_t u = w ^ 0x80808080u;
+  const uint32_t m01 = __byte_perm(u, 0x64646464u, 0x4140);   // (1024 + u0, 1024 + u1)
+  const uint32_t m23 = __byte_perm(u, 0x64646464u, 0x4342);   // (1024 + u2, 1024 + u3)
+  const __half2 bias = __halves2half2(__ushort_as_half((unsigned short)0x6480), __ushort_as_half((unsigned short)0x6480));
+  const __half2 x01 = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&m01), bias), scale);
+  const __half2 x23 = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&m23), bias), scale);
+  lo = *reinterpret_cast<const uint32_t*>(&x01);
+  hi = *reinterpret_cast<const uint32_t*>(&x23);
+}
+
+template <int R, int C, int GQ, bool I8>
 __global__ void __launch_bounds__(kThreadsTC, 1)
 attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __restrict__ w1f,
                  const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmQ,
                  const __grid_constant__ CUtensorMap tmRes) {
-  using Lay = TcLayout<R, C>;
+  using Lay = TcLayout<R, C, I8>;
   constexpr int SUBS = Lay::SUBS, STAGES = Lay::STAGES, KSLABS = Lay::KSLABS;
   extern __shared__ unsigned char smem_dyn[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -169,10 +210,16 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
   // ------------------------------------------------------------------ set-up
   if (tid == 0) {
     for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&bar.a_full[i], 1);
+      mbar_init(&bar.a_full[i], I8 ? 2 : 1);   // the two converter warps, or the TMA arrive
       mbar_init(&bar.a_empty[i], 1);
-      mbar_init(&bar.r_full[i], 1);
+      mbar_init(&bar.r_full[i], I8 ? 2 : 1);
       mbar_init(&bar.r_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar.stg_full[i], 1);
+      mbar_init(&bar.stg_empty[i], 2);
+      mbar_init(&bar.rstg_full[i], 1);
+      mbar_init(&bar.rstg_empty[i], 2);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar.q_full[i], 1);
@@ -208,10 +255,11 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
   const uint32_t sP = smem_u32(smem + Lay::OFF_P);
   const uint32_t sRes = smem_u32(smem + Lay::OFF_RES);
   const uint32_t sPR = smem_u32(smem + Lay::OFF_PR);
-  constexpr uint32_t IDESC_S = idesc_f16(128, 16, 1, 1);        // bf16 x bf16
-  constexpr uint32_t IDESC_1 = idesc_f16(128, 64, 1, 1);        // bf16 (TMEM) x bf16
-  constexpr uint32_t IDESC_3 = idesc_f16(128, 16, 0, 0);        // f16 (TMEM) x f16
-  constexpr uint32_t IDESC_4 = idesc_f16(128, 16, 1, 1, 1, 0);  // bf16 (MN-major) x bf16
+  constexpr int F16B = I8 ? 0 : 1;   // operand format of the tile MMAs: 1 = bf16, 0 = fp16
+  constexpr uint32_t IDESC_S = idesc_f16(128, 16, F16B, F16B);        // tile x queries
+  constexpr uint32_t IDESC_1 = idesc_f16(128, 64, F16B, F16B);        // W1' (TMEM) x tile
+  constexpr uint32_t IDESC_3 = idesc_f16(128, 16, 0, 0);              // H (TMEM, fp16) x P (fp16)
+  constexpr uint32_t IDESC_4 = idesc_f16(128, 16, F16B, F16B, 1, 0);  // residual rows (MN-major) x P_res
 
   if (warp == 0) {
     // ============================================================ TMA producer
@@ -242,20 +290,34 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
           __syncwarp();
           q_issued = unit_i + 1;
         }
-        const int st = ci % STAGES;
+        const int st = ci % STAGES, s2 = ci & 1;
         const uint32_t par = ((ci / STAGES) - 1) & 1;
-        if (ci >= STAGES && !__all_sync(0xffffffffu, mbar_wait(&bar.a_empty[st], par, abort_flag, err, ERR_TIMEOUT)))
+        if (I8) {   // the int8 tile goes to the staging ring; the converters fill stage st
+          if (ci >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar.stg_empty[s2], ((ci >> 1) - 1) & 1, abort_flag,
+                                                            err, ERR_TIMEOUT)))
+            break;
+        } else if (ci >= STAGES &&
+                   !__all_sync(0xffffffffu, mbar_wait(&bar.a_empty[st], par, abort_flag, err, ERR_TIMEOUT))) {
           break;
+        }
         const Unit un = unit_of(g, u);
         const int l = g.layer0 + un.li;
         const int grp = l / g.G;
         const int slot = sc.sel_slot[x];
         const int row0 = (int)(((((long long)un.b * NG + grp) * g.Hkv + un.hkv) * g.nL + slot) * C);
         if (leader) {
-          mbar_expect_tx(&bar.a_full[st], (uint32_t)(C * R * 2));
+          if (I8) {
+            unsigned char* dst = smem + Lay::OFF_SA + s2 * Lay::SA_SLOT;
+            mbar_expect_tx(&bar.stg_full[s2], (uint32_t)Lay::SA_SLOT);
+            bulk_load(dst, static_cast<const unsigned char*>(cb.coeff) + (size_t)row0 * R, (uint32_t)(C * R),
+                      &bar.stg_full[s2]);
+            bulk_load(dst + C * R, cb.coeff_scale + row0, (uint32_t)(C * 2), &bar.stg_full[s2]);
+          } else {
+            mbar_expect_tx(&bar.a_full[st], (uint32_t)(C * R * 2));
 #pragma unroll
-          for (int ks = 0; ks < KSLABS; ++ks)
-            tma_load_2d(smem + Lay::OFF_A + st * Lay::A_STAGE + ks * 16384, &tmA, &bar.a_full[st], ks * 64, row0);
+            for (int ks = 0; ks < KSLABS; ++ks)
+              tma_load_2d(smem + Lay::OFF_A + st * Lay::A_STAGE + ks * 16384, &tmA, &bar.a_full[st], ks * 64, row0);
+          }
         }
         __syncwarp();
         issued_a = ci + 1;
@@ -263,8 +325,13 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
         const int r0 = rptr[slot], r1 = rptr[slot + 1];
         const int nres = min(r1 - r0, kResCap);
         const int my_pos = lane < nres ? (int)cb.res_pos[r0 + lane] : C;
+        const __half my_rs = (I8 && lane < nres) ? cb.res_scale[r0 + lane] : __ushort_as_half((unsigned short)0);
         if (ci >= STAGES && !__all_sync(0xffffffffu, mbar_wait(&bar.r_empty[st], par, abort_flag, err, ERR_TIMEOUT)))
           break;
+        if (I8 && ci >= 2 &&
+            !__all_sync(0xffffffffu, mbar_wait(&bar.rstg_empty[s2], ((ci >> 1) - 1) & 1, abort_flag, err, ERR_TIMEOUT)))
+          break;
+        if (I8) misc->stage_rs[st][lane] = my_rs;
         // record range and token -> record map for the softmax warps (published by the
         // arrive below); a position outside the chunk is left out of the map
         if (lane == 0) {
@@ -276,11 +343,19 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
         if (my_pos < C) misc->stage_idx[st][my_pos] = (int8_t)lane;
         __syncwarp();
         if (leader) {
-          // records r0 .. r0+31 in two 64-dim slabs; rows past the chunk's own records meet
-          // zero probabilities, and the cache keeps 32 zero rows after its last record
-          mbar_expect_tx(&bar.r_full[st], (uint32_t)Lay::RES_BUF);
-          tma_load_2d(smem + Lay::OFF_RES + st * Lay::RES_BUF, &tmRes, &bar.r_full[st], 0, r0);
-          tma_load_2d(smem + Lay::OFF_RES + st * Lay::RES_BUF + Lay::RES_SLAB, &tmRes, &bar.r_full[st], 64, r0);
+          // records r0 .. r0+31 (rows past the chunk's own records meet zero probabilities,
+          // and the cache keeps 32 zero rows after its last record): two 64-dim slabs by
+          // TMA, or 32 int8 rows into the staging ring
+          if (I8) {
+            mbar_expect_tx(&bar.rstg_full[s2], (uint32_t)Lay::SR_SLOT);
+            bulk_load(smem + Lay::OFF_SR + s2 * Lay::SR_SLOT,
+                      static_cast<const unsigned char*>(cb.res_val) + (size_t)r0 * kDh, (uint32_t)Lay::SR_SLOT,
+                      &bar.rstg_full[s2]);
+          } else {
+            mbar_expect_tx(&bar.r_full[st], (uint32_t)Lay::RES_BUF);
+            tma_load_2d(smem + Lay::OFF_RES + st * Lay::RES_BUF, &tmRes, &bar.r_full[st], 0, r0);
+            tma_load_2d(smem + Lay::OFF_RES + st * Lay::RES_BUF + Lay::RES_SLAB, &tmRes, &bar.r_full[st], 64, r0);
+          }
         }
         __syncwarp();
         issued_r = ci + 1;
@@ -288,10 +363,17 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       if (*abort_flag && leader) {
         // let every copy this warp started land before the CTA's shared memory goes away
         volatile int never = 0;
-        for (int ci = max(0, issued_a - STAGES); ci < issued_a; ++ci)
-          mbar_wait(&bar.a_full[ci % STAGES], (ci / STAGES) & 1, &never, err, ERR_TIMEOUT);
-        for (int ci = max(0, issued_r - STAGES); ci < issued_r; ++ci)
-          mbar_wait(&bar.r_full[ci % STAGES], (ci / STAGES) & 1, &never, err, ERR_TIMEOUT);
+        if (I8) {
+          for (int ci = max(0, issued_a - 2); ci < issued_a; ++ci)
+            mbar_wait(&bar.stg_full[ci & 1], (ci >> 1) & 1, &never, err, ERR_TIMEOUT);
+          for (int ci = max(0, issued_r - 2); ci < issued_r; ++ci)
+            mbar_wait(&bar.rstg_full[ci & 1], (ci >> 1) & 1, &never, err, ERR_TIMEOUT);
+        } else {
+          for (int ci = max(0, issued_a - STAGES); ci < issued_a; ++ci)
+            mbar_wait(&bar.a_full[ci % STAGES], (ci / STAGES) & 1, &never, err, ERR_TIMEOUT);
+          for (int ci = max(0, issued_r - STAGES); ci < issued_r; ++ci)
+            mbar_wait(&bar.r_full[ci % STAGES], (ci / STAGES) & 1, &never, err, ERR_TIMEOUT);
+        }
         for (int ui = max(0, q_issued - 2); ui < q_issued; ++ui)
           mbar_wait(&bar.q_full[ui & 1], (ui >> 1) & 1, &never, err, ERR_TIMEOUT);
       }
@@ -431,6 +513,76 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       }
       __syncwarp();
     }
+  } else if (I8 && (warp == 2 || warp == 3)) {
+    // ============================================================ int8 converters
+    // Per chunk: the staged int8 coefficient rows times their fp16 scales become the fp16
+    // tile of stage st in the 128-byte-swizzle K-major layout the MMAs read (16-byte piece
+    // j of row t at j ^ (t % 8) inside its 64-column slab), and the staged int8 residual
+    // rows times their scales become the fp16 MN-major tile of the D4 MMA (same swizzle,
+    // rows = records, 64-dim slabs).
+    const int ct = tid - 64;   // 0..63
+    bool ok = true;
+    for (int ci = 0; ok && ci < NCH; ++ci) {
+      const int st = ci % STAGES, s2 = ci & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar.stg_full[s2], (ci >> 1) & 1, abort_flag, err, ERR_TIMEOUT));
+      if (ok && ci >= STAGES)
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar.a_empty[st], ((ci / STAGES) - 1) & 1, abort_flag, err, ERR_TIMEOUT));
+      if (!ok) break;
+      {
+        const unsigned char* src = smem + Lay::OFF_SA + s2 * Lay::SA_SLOT;
+        const __half* scl = reinterpret_cast<const __half*>(src + C * R);
+        unsigned char* dst = smem + Lay::OFF_A + st * Lay::A_STAGE;
+        constexpr int P16 = R / 16;   // 16-element pieces per row
+        for (int it = ct; it < C * P16; it += 64) {
+          const int t = it / P16, c16 = it % P16;
+          const uint4 q = *reinterpret_cast<const uint4*>(src + t * R + c16 * 16);
+          const __half2 sg = __half2half2(scl[t]);
+          uint32_t o[8];
+          i8x4_scaled_f16(q.x, sg, o[0], o[1]);
+          i8x4_scaled_f16(q.y, sg, o[2], o[3]);
+          i8x4_scaled_f16(q.z, sg, o[4], o[5]);
+          i8x4_scaled_f16(q.w, sg, o[6], o[7]);
+          const int col = c16 * 16, ks = col >> 6, j = (col & 63) >> 3;
+          unsigned char* row = dst + ks * 16384 + t * 128;
+          *reinterpret_cast<uint4*>(row + ((j ^ (t & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(row + (((j + 1) ^ (t & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bar.stg_empty[s2]);
+        mbar_arrive(&bar.a_full[st]);
+      }
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar.rstg_full[s2], (ci >> 1) & 1, abort_flag, err, ERR_TIMEOUT));
+      if (ok && ci >= STAGES)
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar.r_empty[st], ((ci / STAGES) - 1) & 1, abort_flag, err, ERR_TIMEOUT));
+      if (!ok) break;
+      {
+        const unsigned char* src = smem + Lay::OFF_SR + s2 * Lay::SR_SLOT;
+        unsigned char* dst = smem + Lay::OFF_RES + st * Lay::RES_BUF;
+        for (int it = ct; it < kResCap * (kDh / 16); it += 64) {
+          const int i = it / (kDh / 16), c16 = it % (kDh / 16);
+          const uint4 q = *reinterpret_cast<const uint4*>(src + i * kDh + c16 * 16);
+          const __half2 sg = __half2half2(misc->stage_rs[st][i]);
+          uint32_t o[8];
+          i8x4_scaled_f16(q.x, sg, o[0], o[1]);
+          i8x4_scaled_f16(q.y, sg, o[2], o[3]);
+          i8x4_scaled_f16(q.z, sg, o[4], o[5]);
+          i8x4_scaled_f16(q.w, sg, o[6], o[7]);
+          const int dim = c16 * 16, slab = dim >> 6, j = (dim & 63) >> 3;
+          unsigned char* row = dst + slab * Lay::RES_SLAB + i * 128;
+          *reinterpret_cast<uint4*>(row + ((j ^ (i & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(row + (((j + 1) ^ (i & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bar.rstg_empty[s2]);
+        mbar_arrive(&bar.r_full[st]);
+      }
+    }
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 8) {
     // ============================================================ silu epilogue
     // Warpgroup A (warps 4-7) takes the even sub-tiles, B (8-11) the odd ones, each doing
@@ -547,7 +699,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
     }
   } else if (warp >= kSoftWarp0) {
     // ============================================================ softmax + accumulation
-    // Per chunk: online max/sum per head, the fp16 P tile and the bf16 P_res tile (the
+    // Per chunk: online max/sum per head, the fp16 P tile and the P_res tile (the
     // probabilities at the flagged tokens) for the MMAs, residual records beyond the first
     // 32 on CUDA cores, and (one chunk later) the chunk's D3 / D4 folded into the running
     // sums.  Thread t is token t for the scores, hidden row t of both halves for D3 and
@@ -661,14 +813,13 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
         for (int j = 0; j < GQ; ++j) {
           *reinterpret_cast<__half*>(pt + kmajor_off(j, t, Lay::P_SBO)) = __float2half_rn(p[j]);
           // P_res: row j, column i = probability of head j at the chunk's i-th flagged token
-          if (idx >= 0)
-            *reinterpret_cast<__nv_bfloat16*>(pr + kmajor_off(j, idx, Lay::PR_SBO)) = __float2bfloat16_rn(p[j]);
+          if (idx >= 0) st_op16<I8>(pr + kmajor_off(j, idx, Lay::PR_SBO), p[j]);
         }
       }
       if (live && t < kResCap && t >= nrec) {   // columns past the chunk's records
 #pragma unroll
         for (int j = 0; j < GQ; ++j)
-          *reinterpret_cast<__nv_bfloat16*>(pr + kmajor_off(j, t, Lay::PR_SBO)) = __float2bfloat16_rn(0.f);
+          st_op16<I8>(pr + kmajor_off(j, t, Lay::PR_SBO), 0.f);
       }
 #pragma unroll
       for (int j = 0; j < GQ; ++j) {
@@ -688,10 +839,12 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       // global memory and the probabilities from the fp16 P tile
       if (live && nrec > kResCap) {
         const uint16_t* rg = reinterpret_cast<const uint16_t*>(cb.res_val);
+        const int8_t* rg8 = reinterpret_cast<const int8_t*>(cb.res_val);
         for (int i = kResCap; i < nrec; ++i) {
           const int pos = cb.res_pos[r0 + i];
           if (pos >= C) continue;
-          const float dv = __uint_as_float(((uint32_t)rg[(size_t)(r0 + i) * kDh + t]) << 16);
+          const float dv = I8 ? (float)rg8[(size_t)(r0 + i) * kDh + t] * __half2float(cb.res_scale[r0 + i])
+                              : __uint_as_float(((uint32_t)rg[(size_t)(r0 + i) * kDh + t]) << 16);
 #pragma unroll
           for (int j = 0; j < GQ; ++j)
             accD[j] = fmaf(__half2float(*reinterpret_cast<const __half*>(pt + kmajor_off(j, pos, Lay::P_SBO))), dv,
@@ -747,19 +900,24 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
   return r == CUDA_SUCCESS;
 }
 
-template <int R, int C, int GQ>
+template <int R, int C, int GQ, bool I8>
 cudaError_t launch_tc(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const void* w1f,
                       cudaStream_t s) {
-  using Lay = TcLayout<R, C>;
+  using Lay = TcLayout<R, C, I8>;
   const int NG = g.L / g.G;
   const uint64_t rows = (uint64_t)g.B * NG * g.Hkv * g.nL * C;
   CUtensorMap tmA, tmQ, tmRes;
-  if (!make_map(&tmA, cb.coeff, R, rows, C)) return cudaErrorInvalidValue;
   if (!make_map(&tmQ, sc.qt_tc, R, (uint64_t)g.U * 16, 16)) return cudaErrorInvalidValue;
-  // the cache keeps kResPad zero rows after its residual rows, so every box is in bounds
-  if (!make_map(&tmRes, cb.res_val, kDh, (uint64_t)cb.n_records + kResPad, kResCap))
-    return cudaErrorInvalidValue;
-  auto k = attend_tc_kernel<R, C, GQ>;
+  if (I8) {   // int8 rows arrive by plain bulk copies; the tile maps are not used
+    tmA = tmQ;
+    tmRes = tmQ;
+  } else {
+    if (!make_map(&tmA, cb.coeff, R, rows, C)) return cudaErrorInvalidValue;
+    // the cache keeps kResPad zero rows after its residual rows, so every box is in bounds
+    if (!make_map(&tmRes, cb.res_val, kDh, (uint64_t)cb.n_records + kResPad, kResCap))
+      return cudaErrorInvalidValue;
+  }
+  auto k = attend_tc_kernel<R, C, GQ, I8>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
   if (e != cudaSuccess) return e;
   k<<<g.P, kThreadsTC, Lay::SMEM, s>>>(g, cb, sc, static_cast<const __nv_bfloat16*>(w1f), tmA, tmQ,
@@ -770,9 +928,11 @@ cudaError_t launch_tc(const Geom& g, const CacheBuffers& cb, const Scratch& sc, 
 }  // namespace
 
 // The cache object pads its residual array by kResPad zero rows; callers that pass their
-// own arrays (the allocation-free entry point) use the CUDA-core kernels.
+// own arrays (the allocation-free entry point) use the CUDA-core kernels.  The int8 store is
+// taken for 128-token chunks.
 bool attend_tc_supported(const Geom& g, int dtype, int store) {
-  if (dtype != LOWRAM_BF16 || store != LOWRAM_STORE_NATIVE) return false;
+  if (dtype != LOWRAM_BF16) return false;
+  if (store != LOWRAM_STORE_NATIVE && !(store == LOWRAM_STORE_INT8 && g.C == 128)) return false;
   if (g.d != kDh || g.h != kHid || !(g.g == 4 || g.g == 8)) return false;
   if (!(g.r == 64 || g.r == 128) || !(g.C == 64 || g.C == 128)) return false;
   const uint64_t rows = (uint64_t)g.B * (g.L / g.G) * g.Hkv * g.nL * g.C;
@@ -783,10 +943,20 @@ bool attend_tc_supported(const Geom& g, int dtype, int store) {
 cudaError_t launch_attend_tc(const Geom& g, const CacheBuffers& cb, const Scratch& sc, int store,
                              const void* w1f_tc, int n_sm, cudaStream_t s) {
   (void)n_sm;
-  if (store != LOWRAM_STORE_NATIVE) return cudaErrorNotSupported;
   if (cb.n_records + kResPad >= (1ll << 31)) return cudaErrorNotSupported;
+  if (store == LOWRAM_STORE_INT8) {
+#define LOWRAM_TC_CASE8(RR, GG) \
+    if (g.r == RR && g.C == 128 && g.g == GG) return launch_tc<RR, 128, GG, true>(g, cb, sc, w1f_tc, s);
+    LOWRAM_TC_CASE8(128, 4)
+    LOWRAM_TC_CASE8(64, 4)
+    LOWRAM_TC_CASE8(128, 8)
+    LOWRAM_TC_CASE8(64, 8)
+#undef LOWRAM_TC_CASE8
+    return cudaErrorNotSupported;
+  }
+  if (store != LOWRAM_STORE_NATIVE) return cudaErrorNotSupported;
 #define LOWRAM_TC_CASE(RR, CC, GG) \
-  if (g.r == RR && g.C == CC && g.g == GG) return launch_tc<RR, CC, GG>(g, cb, sc, w1f_tc, s);
+  if (g.r == RR && g.C == CC && g.g == GG) return launch_tc<RR, CC, GG, false>(g, cb, sc, w1f_tc, s);
   LOWRAM_TC_CASE(128, 128, 4)
   LOWRAM_TC_CASE(128, 64, 4)
   LOWRAM_TC_CASE(64, 128, 4)

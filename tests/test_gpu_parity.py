@@ -133,6 +133,19 @@ def test_int8_eviction_small_every_unit(path):
     check(cfg, _oracle(cache), q, out, sel, scores=scores)
 
 
+@pytest.mark.parametrize("rank,resid_frac", [(64, 0.125), (128, 0.4)])
+def test_int8_rank_and_residual_overflow(rank, resid_frac):
+    """int8 rows at both ranks; at 40 % flagged tokens most chunks hold more residual
+    records than one residual tile, so the records past it take the overflow route."""
+    cfg = S.LLAMA_64K_INT8.replace(name=f"int8_r{rank}", batch=1, n_layers=4, n_kv_heads=2,
+                                   n_q_heads=8, n_ctx=8192, rank=rank, resid_frac=resid_frac,
+                                   top_k=16)
+    cache = S.make_cache(cfg, tail_len=[33])
+    q = S.make_queries(cache)
+    out, sel, scores, _ = _run(cache, q)
+    check(cfg, _oracle(cache), q, out, sel, scores=scores)
+
+
 def test_int8_eviction_select_all_live():
     cfg = S.LLAMA_64K_INT8.replace(name="int8_all", batch=1, n_layers=4, n_kv_heads=2,
                                    n_q_heads=8, n_ctx=4096, top_k=16)
