@@ -101,10 +101,10 @@ struct Bars {
   uint64_t a_full[4], a_empty[4];     // coefficient tiles
   uint64_t r_full[4], r_empty[4];     // residual rows (+ their record range and token map)
   uint64_t q_full[2], q_empty[2];
-  uint64_t s_full[2], s_free[2];
+  uint64_t s_full[2];
   uint64_t d1_full[2], h_ready[2];
   uint64_t p_ready[2];
-  uint64_t d3_full[2], d3_free[2];
+  uint64_t d3_full[2];
   uint64_t stg_full[2], stg_empty[2];   // int8 coefficient staging (int8 store)
   uint64_t rstg_full[2], rstg_empty[2]; // int8 residual staging (int8 store)
   uint64_t w1_ready;   // W1' of the next (layer, KV head) is in TMEM
@@ -225,12 +225,10 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       mbar_init(&bar.q_full[i], 1);
       mbar_init(&bar.q_empty[i], 1);
       mbar_init(&bar.s_full[i], 1);
-      mbar_init(&bar.s_free[i], 4);       // 4 softmax warps
       mbar_init(&bar.d1_full[i], 1);
       mbar_init(&bar.h_ready[i], 4);      // the 4 warps of the sub-tile's epilogue group
       mbar_init(&bar.p_ready[i], 1);
       mbar_init(&bar.d3_full[i], 1);
-      mbar_init(&bar.d3_free[i], 4);      // 4 softmax warps
     }
     mbar_init(&bar.w1_ready, 4);          // epilogue group A
     mbar_init(&bar.seg_done, 1);
@@ -419,8 +417,9 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
               if (!wait_all(&bar.w1_ready, m_seg_i & 1)) return false;
             }
           }
+          // The S buffer of chunk ci was last read by the softmax for chunk ci-2, before it
+          // published that chunk's probabilities, which this warp has waited for already.
           const int sb = ci & 1;
-          if (ci >= 2 && !wait_all(&bar.s_free[sb], ((ci >> 1) - 1) & 1)) return false;
           tc_fence_after();
           const uint64_t dA = dA0 + (uint64_t)((st * Lay::A_STAGE) >> 4);
           const uint64_t dQ = dQ0 + (uint64_t)(((m_unit_i & 1) * Lay::Q_BUF) >> 4);
@@ -476,11 +475,11 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
         const int ci = n / SUBS, sub = n % SUBS, b = n & 1, pb = ci & 1;
         if (!wait_all(&bar.h_ready[b], (n >> 1) & 1)) break;
         const int st = ci % STAGES;
-        if (sub == 0) {
-          if (!wait_all(&bar.p_ready[pb], (ci >> 1) & 1)) break;
-          if (!wait_all(&bar.r_full[st], (ci / STAGES) & 1)) break;
-          if (ci >= 2 && !wait_all(&bar.d3_free[pb], ((ci >> 1) - 1) & 1)) break;
-        }
+        // One acquire covers the softmax's hand-offs: before it publishes the probabilities
+        // of chunk ci it has waited for the chunk's residual rows and read out the D3 / D4
+        // buffer of chunk ci-2.  Each wait costs this warp far more than a satisfied test
+        // suggests (it shares its issue slots with busy epilogue and softmax warps).
+        if (sub == 0 && !wait_all(&bar.p_ready[pb], (ci >> 1) & 1)) break;
         tc_fence_after();
         const uint64_t dP = dP0 + (uint64_t)((pb * Lay::P_BUF + sub * 1024) >> 4);
         const uint64_t dPR = dPR0 + (uint64_t)((pb * Lay::PR_BUF) >> 4);
@@ -733,7 +732,6 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar.d3_free[pb]);
 #pragma unroll
       for (int j = 0; j < GQ; ++j) {
         accH0[j] = fmaf(accH0[j], al_prev[j], __uint_as_float(v0[j]));
@@ -780,7 +778,6 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar.s_free[sb]);
       }
       const bool valid = t < C;
       float p[GQ], al[GQ];
