@@ -6,9 +6,10 @@
 //   S  = A_c . Qt^T                 scores q_j . khat_t / sqrt(d) * log2(e) in the low-rank
 //                                   form (Qt_j = B_l q_j, "OjaKV" 3.1 projects queries into
 //                                   the key basis); M=128 tokens, N=16 heads (g used)
-//   D1 = W1'/2 . A_sub^T            pre-activations / 2 of the predictor's hidden layer,
-//                                   W1' = W1 B_l^T (exact fold of W1 khat_t); M=128 hidden
-//                                   rows per half, N=64 tokens per sub-tile, A from TMEM
+//   D1 = W1'_hh/2 . A_c^T           pre-activations / 2 of the predictor's hidden layer,
+//                                   W1' = W1 B_l^T (exact fold of W1 khat_t); a sub-tile is
+//                                   one half hh of the 256 hidden units: M=128 hidden rows,
+//                                   N=C tokens, both operands in shared memory
 //   H  = silu(2 * D1) = u + u tanh(u), written back to TMEM as fp16 (MUFU tanh)
 //   D3 = H . P                      softmax-weighted hidden sums per head (A = H from TMEM,
 //                                   B = P, the chunk's probabilities, fp16 in SMEM)
@@ -21,15 +22,19 @@
 // Asymmetrically", section "Cross-Layer Low-Rank Key Compression"; values: same page,
 // "Core Mechanism" (Vhat = f(K), delta kept for the worst tokens); attention: "OjaKV", 3.
 //
-// Warp roles (16 warps): 0 TMA producer, 1 MMA issuer + TMEM owner, 2-3 int8 converters
-// (idle for a native store), 4-7 and 8-11
-// two silu epilogue groups taking alternate sub-tiles (both hidden halves each), 12-15
-// softmax, the P / P_res tiles and the accumulation of the chunks' D3 / D4.
+// Warp roles (16 warps): 0 TMA producer (tiles, queries, residual rows, W1' halves), 1 MMA
+// issuer + TMEM owner, 2-3 int8 converters (idle for a native store), 4-7 and 8-11 the silu
+// epilogue groups of hidden halves 0 and 1, 12-15 softmax, the P / P_res tiles and the
+// accumulation of the chunks' D3 / D4.
 // A warp reaches TMEM lanes 32*(warp%4) .. +31, so each warpgroup of four consecutive
 // warps covers all 128 lanes.
-// TMEM (512 columns): W1' halves [0,128), D1 double buffer x 2 halves [128,384),
-// S double buffer [384,416), D3 double buffer x 2 halves [416,480), D4 double buffer
-// [480,512).
+// Sub-tile n (hidden half n % 2 of chunk n / 2) has D1 buffer n % 3: with three buffers for
+// two epilogue groups the pre-activations of sub-tile n+3 are computed while the epilogue
+// still works on n+1 and n+2, so neither the tensor core nor the epilogue waits for the
+// other's round trip.  W1' lives in shared memory (the SS form costs no more tensor time at
+// N=128 than the TS form, and frees the 128 TMEM columns the third buffer needs).
+// TMEM (512 columns): D1 buffers [0,384), S double buffer [384,416), D3 double buffer x 2
+// halves [416,480), D4 double buffer [480,512).
 // Every wait is bounded: on timeout the kernel raises the error word, drains its own
 // copies and MMAs, frees TMEM and returns.
 #include <cuda.h>
@@ -60,11 +65,12 @@ static_assert(kResCap == 32, "the P_res tile and the D4 MMAs assume 32 records")
 // too.
 template <int R, int C, bool I8>
 struct TcLayout {
-  static constexpr int NT = 64;
-  static constexpr int SUBS = C / NT;
-  static constexpr int STAGES = I8 ? 3 : 4;
+  static constexpr int SUBS = 2;                     // sub-tiles per chunk = hidden halves
+  static constexpr int NBUF = 3;                     // D1 buffers
+  static constexpr int STAGES = I8 ? 2 : 3;
   static constexpr int KSLABS = R / 64;
   static constexpr int A_STAGE = KSLABS * 16384;     // 128 rows x 128 B per 64-wide K slab
+  static constexpr int W_HALF = KSLABS * 16384;      // 128 hidden rows x R of W1'/2, same layout
   static constexpr int Q_BUF = KSLABS * 2048;        // 16 rows x 128 B per slab
   static constexpr int P_BUF = 16 * C * 2;
   static constexpr int P_SBO = (C / 8) * 128;
@@ -72,7 +78,8 @@ struct TcLayout {
   static constexpr int RES_BUF = 2 * RES_SLAB;
   static constexpr int PR_BUF = 16 * kResCap * 2;
   static constexpr int PR_SBO = (kResCap / 8) * 128;
-  static constexpr int OFF_A = 0;
+  static constexpr int OFF_W = 0;
+  static constexpr int OFF_A = OFF_W + 2 * W_HALF;
   static constexpr int OFF_Q = OFF_A + STAGES * A_STAGE;
   static constexpr int OFF_RES = OFF_Q + 2 * Q_BUF;
   static constexpr int OFF_P = OFF_RES + STAGES * RES_BUF;
@@ -85,16 +92,15 @@ struct TcLayout {
   static constexpr int MISC_BYTES = 3072;
   static constexpr int SMEM = OFF_MISC + MISC_BYTES + 1024;   // + alignment slack
   // TMEM columns
-  static constexpr uint32_t T_W1 = 0;
-  static constexpr uint32_t T_D1 = 128;
+  static constexpr uint32_t T_D1 = 0;
   static constexpr uint32_t T_S = 384;
   static constexpr uint32_t T_D3 = 416;
   static constexpr uint32_t T_D4 = 480;
   static constexpr uint32_t TMEM_COLS = 512;
-  static_assert(R / 2 <= 64, "W1' half must fit 64 TMEM columns");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static_assert(SA_SLOT % 16 == 0 && OFF_SA % 16 == 0, "bulk copies need 16-byte alignment");
-  static_assert(OFF_Q % 1024 == 0 && OFF_RES % 1024 == 0, "128-byte-swizzled operands need 1024-byte alignment");
+  static_assert(OFF_A % 1024 == 0 && OFF_Q % 1024 == 0 && OFF_RES % 1024 == 0,
+                "128-byte-swizzled operands need 1024-byte alignment");
 };
 
 struct Bars {
@@ -102,12 +108,12 @@ struct Bars {
   uint64_t r_full[4], r_empty[4];     // residual rows (+ their record range and token map)
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full[2];
-  uint64_t d1_full[2], h_ready[2];
+  uint64_t d1_full[3], h_ready[3];   // per D1 buffer
   uint64_t p_ready[2];
   uint64_t d3_full[2];
   uint64_t stg_full[2], stg_empty[2];   // int8 coefficient staging (int8 store)
   uint64_t rstg_full[2], rstg_empty[2]; // int8 residual staging (int8 store)
-  uint64_t w1_ready;   // W1' of the next (layer, KV head) is in TMEM
+  uint64_t w1_ready;   // W1' of the next (layer, KV head) is in shared memory
   uint64_t seg_done;   // every MMA that read the previous W1' is complete
   uint64_t drain;
 };
@@ -186,11 +192,11 @@ __device__ __forceinline__ void i8x4_scaled_f16(uint32_t w, __half2 scale, uint3
 
 template <int R, int C, int GQ, bool I8>
 __global__ void __launch_bounds__(kThreadsTC, 1)
-attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __restrict__ w1f,
+attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CUtensorMap tmW,
                  const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmQ,
                  const __grid_constant__ CUtensorMap tmRes) {
   using Lay = TcLayout<R, C, I8>;
-  constexpr int SUBS = Lay::SUBS, STAGES = Lay::STAGES, KSLABS = Lay::KSLABS;
+  constexpr int SUBS = Lay::SUBS, STAGES = Lay::STAGES, KSLABS = Lay::KSLABS, NBUF = Lay::NBUF;
   extern __shared__ unsigned char smem_dyn[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
@@ -225,12 +231,14 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       mbar_init(&bar.q_full[i], 1);
       mbar_init(&bar.q_empty[i], 1);
       mbar_init(&bar.s_full[i], 1);
-      mbar_init(&bar.d1_full[i], 1);
-      mbar_init(&bar.h_ready[i], 4);      // the 4 warps of the sub-tile's epilogue group
       mbar_init(&bar.p_ready[i], 1);
       mbar_init(&bar.d3_full[i], 1);
     }
-    mbar_init(&bar.w1_ready, 4);          // epilogue group A
+    for (int i = 0; i < NBUF; ++i) {
+      mbar_init(&bar.d1_full[i], 1);
+      mbar_init(&bar.h_ready[i], 4);      // the 4 warps of the sub-tile's epilogue group
+    }
+    mbar_init(&bar.w1_ready, 1);          // TMA
     mbar_init(&bar.seg_done, 1);
     mbar_init(&bar.drain, 1);
     misc->abort_flag = 0;
@@ -248,6 +256,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
   tc_fence_after();
   const uint32_t tmem = misc->tmem_base;
 
+  const uint32_t sW = smem_u32(smem + Lay::OFF_W);
   const uint32_t sA = smem_u32(smem + Lay::OFF_A);
   const uint32_t sQ = smem_u32(smem + Lay::OFF_Q);
   const uint32_t sP = smem_u32(smem + Lay::OFF_P);
@@ -255,7 +264,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
   const uint32_t sPR = smem_u32(smem + Lay::OFF_PR);
   constexpr int F16B = I8 ? 0 : 1;   // operand format of the tile MMAs: 1 = bf16, 0 = fp16
   constexpr uint32_t IDESC_S = idesc_f16(128, 16, F16B, F16B);        // tile x queries
-  constexpr uint32_t IDESC_1 = idesc_f16(128, 64, F16B, F16B);        // W1' (TMEM) x tile
+  constexpr uint32_t IDESC_1 = idesc_f16(128, C, F16B, F16B);         // W1' half x tile
   constexpr uint32_t IDESC_3 = idesc_f16(128, 16, 0, 0);              // H (TMEM, fp16) x P (fp16)
   constexpr uint32_t IDESC_4 = idesc_f16(128, 16, F16B, F16B, 1, 0);  // residual rows (MN-major) x P_res
 
@@ -266,6 +275,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
     const bool leader = elect_one();
     if (NCH > 0) {
       int unit_i = -1, prev_u = -1, issued_a = 0, issued_r = 0, q_issued = 0;
+      int seg_i = -1, prev_seg = -1, w1_issued = 0;
       TileWalk wk;
       wk.init(x0, g.k, g.B);
       for (int ci = 0; ci < NCH; ++ci) {
@@ -319,6 +329,27 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
         }
         __syncwarp();
         issued_a = ci + 1;
+        if (wk.seg != prev_seg) {
+          // the first chunk of a (layer, KV head): its W1' halves, once every MMA that read
+          // the previous pair's has completed
+          ++seg_i;
+          prev_seg = wk.seg;
+          if (seg_i > 0 && !__all_sync(0xffffffffu, mbar_wait(&bar.seg_done, (seg_i - 1) & 1, abort_flag, err,
+                                                              ERR_TIMEOUT)))
+            break;
+          if (leader) {
+            mbar_expect_tx(&bar.w1_ready, (uint32_t)(2 * Lay::W_HALF));
+            const int wrow = (l * g.Hkv + un.hkv) * kHid;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+              for (int ks = 0; ks < KSLABS; ++ks)
+                tma_load_2d(smem + Lay::OFF_W + hh * Lay::W_HALF + ks * 16384, &tmW, &bar.w1_ready, ks * 64,
+                            wrow + hh * 128);
+          }
+          __syncwarp();
+          w1_issued = seg_i + 1;
+        }
         const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nL + 1);
         const int r0 = rptr[slot], r1 = rptr[slot + 1];
         const int nres = min(r1 - r0, kResCap);
@@ -374,6 +405,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
         }
         for (int ui = max(0, q_issued - 2); ui < q_issued; ++ui)
           mbar_wait(&bar.q_full[ui & 1], (ui >> 1) & 1, &never, err, ERR_TIMEOUT);
+        if (w1_issued > 0) mbar_wait(&bar.w1_ready, (w1_issued - 1) & 1, &never, err, ERR_TIMEOUT);
       }
     }
   } else if (warp == 1) {
@@ -386,25 +418,34 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
       // Descriptors are built once; a K step, stage, buffer or sub-tile only moves the
       // start address, i.e. adds (byte offset >> 4) to the low field (no carry: every
       // shared address here is below 256 KiB).
+      const uint64_t dW0 = smem_desc(sW, 16, 1024, 2);              // W1' halves
       const uint64_t dA0 = smem_desc(sA, 16, 1024, 2);              // coefficient tiles
       const uint64_t dQ0 = smem_desc(sQ, 16, 1024, 2);              // projected queries
       const uint64_t dP0 = smem_desc(sP, 128, Lay::P_SBO, 0);       // probabilities
       const uint64_t dR0 = smem_desc(sRes, Lay::RES_SLAB, 1024, 2); // residual rows, MN-major
       const uint64_t dPR0 = smem_desc(sPR, 128, Lay::PR_SBO, 0);    // probabilities at records
-      const uint32_t t_w1 = tmem + Lay::T_W1, t_d1 = tmem + Lay::T_D1;
+      const uint32_t t_d1 = tmem + Lay::T_D1;
       const uint32_t t_s = tmem + Lay::T_S, t_d3 = tmem + Lay::T_D3, t_d4 = tmem + Lay::T_D4;
       TileWalk wk;
       wk.init(x0, g.k, g.B);
       auto wait_all = [&](uint64_t* b, uint32_t par) -> bool {
         return __all_sync(0xffffffffu, mbar_wait(b, par, abort_flag, err, ERR_TIMEOUT));
       };
+      // Pre-activations of sub-tile n (hidden half hh = n % 2 of chunk n / 2) into D1 buffer
+      // n % 3; hidden half 0 also carries the chunk's scores (two accumulation chains
+      // interleaved).  Tiles, queries and W1' arrive by TMA (or as the converters'
+      // proxy-fenced stores): the waits on their barriers order them for the MMAs.  The TMEM
+      // this call overwrites was released before barriers the caller has waited and fenced:
+      // D1 buffer n % 3 by the epilogue (H of sub-tile n-3, read by the D3 MMAs issued just
+      // before), the S buffer of chunk ci by the softmax for chunk ci-2, before it published
+      // that chunk's probabilities.
       auto issue_mma1 = [&](int n) -> bool {
-        const int ci = n / SUBS, sub = n % SUBS;
+        const int ci = n >> 1, hh = n & 1;
         wk.advance_to(ci);
-        const int u = wk.u;
         const int st = ci % STAGES;
-        if (sub == 0) {
+        if (hh == 0) {
           if (!wait_all(&bar.a_full[st], (ci / STAGES) & 1)) return false;
+          const int u = wk.u;
           if (u != m_cur_u) {
             if (m_cur_u >= 0 && leader) mma_commit(&bar.q_empty[m_unit_i & 1]);
             ++m_unit_i;
@@ -417,92 +458,76 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
               if (!wait_all(&bar.w1_ready, m_seg_i & 1)) return false;
             }
           }
-          // The S buffer of chunk ci was last read by the softmax for chunk ci-2, before it
-          // published that chunk's probabilities, which this warp has waited for already.
-          const int sb = ci & 1;
-          tc_fence_after();
-          const uint64_t dA = dA0 + (uint64_t)((st * Lay::A_STAGE) >> 4);
-          const uint64_t dQ = dQ0 + (uint64_t)(((m_unit_i & 1) * Lay::Q_BUF) >> 4);
-          const uint32_t ts = t_s + sb * 16;
-          const int b0 = n & 1;
-          const uint64_t dB = dA0 + (uint64_t)((st * Lay::A_STAGE + sub * 8192) >> 4);
-          const uint32_t td = t_d1 + b0 * 128;
-          if (leader) {
-            // three independent accumulation chains (scores, hidden half 0, hidden half 1)
-            // interleaved step by step, so one chain's accumulator latency hides behind the
-            // others
+        }
+        const int bf = n % NBUF;
+        const uint32_t td = t_d1 + bf * 128;
+        const uint64_t dA = dA0 + (uint64_t)((st * Lay::A_STAGE) >> 4);
+        const uint64_t dW = dW0 + (uint64_t)((hh * Lay::W_HALF) >> 4);
+        if (leader) {
+          if (hh == 0) {
+            const int sb = ci & 1;
+            const uint64_t dQ = dQ0 + (uint64_t)(((m_unit_i & 1) * Lay::Q_BUF) >> 4);
 #pragma unroll
             for (int kk = 0; kk < R / 16; ++kk) {
               const uint64_t ko = (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2);
               const uint32_t acc = kk > 0 ? 1u : 0u;
-              mma_ss(ts, dA + ko, dQ + (uint64_t)((kk >> 2) * 128 + (kk & 3) * 2), IDESC_S, acc);
-              mma_ts(td, t_w1 + kk * 8, dB + ko, IDESC_1, acc);
-              mma_ts(td + 64, t_w1 + (R / 2) + kk * 8, dB + ko, IDESC_1, acc);
+              mma_ss(t_s + sb * 16, dA + ko, dQ + (uint64_t)((kk >> 2) * 128 + (kk & 3) * 2), IDESC_S, acc);
+              mma_ss(td, dW + ko, dA + ko, IDESC_1, acc);
             }
             mma_commit(&bar.s_full[sb]);
-            mma_commit(&bar.d1_full[b0]);
-            if (sub == SUBS - 1) mma_commit(&bar.a_empty[st]);
-            if (n + 1 < NS && sub == SUBS - 1 && wk.next_starts_segment()) mma_commit(&bar.seg_done);
-          }
-          __syncwarp();
-          return true;
-        } else {
-          tc_fence_after();
-        }
-        const int b = n & 1;
-        const uint64_t dB = dA0 + (uint64_t)((st * Lay::A_STAGE + sub * 8192) >> 4);
-        const uint32_t td = t_d1 + b * 128;
-        if (leader) {
+            mma_commit(&bar.d1_full[bf]);
+          } else {
 #pragma unroll
-          for (int kk = 0; kk < R / 16; ++kk) {   // the two hidden halves interleaved
-            const uint64_t ko = (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2);
-            const uint32_t acc = kk > 0 ? 1u : 0u;
-            mma_ts(td, t_w1 + kk * 8, dB + ko, IDESC_1, acc);
-            mma_ts(td + 64, t_w1 + (R / 2) + kk * 8, dB + ko, IDESC_1, acc);
+            for (int kk = 0; kk < R / 16; ++kk) {
+              const uint64_t ko = (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2);
+              mma_ss(td, dW + ko, dA + ko, IDESC_1, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&bar.d1_full[bf]);
+            mma_commit(&bar.a_empty[st]);
+            if (n + 1 < NS && wk.next_starts_segment())
+              mma_commit(&bar.seg_done);   // the last MMA that reads this W1' has been issued
           }
-          mma_commit(&bar.d1_full[b]);
-          if (sub == SUBS - 1) mma_commit(&bar.a_empty[st]);
-          if (n + 1 < NS && sub == SUBS - 1 && wk.next_starts_segment())
-            mma_commit(&bar.seg_done);   // the last MMA that reads this W1' has been issued
         }
         __syncwarp();
         return true;
       };
 
-      bool ok = issue_mma1(0);
-      if (ok && NS > 1) ok = issue_mma1(1);
+      bool ok = true;
+      for (int n = 0; ok && n < NBUF && n < NS; ++n) ok = issue_mma1(n);
       for (int n = 0; ok && n < NS; ++n) {
-        const int ci = n / SUBS, sub = n % SUBS, b = n & 1, pb = ci & 1;
-        if (!wait_all(&bar.h_ready[b], (n >> 1) & 1)) break;
+        const int ci = n >> 1, hh = n & 1, pb = ci & 1, bf = n % NBUF;
+        if (!wait_all(&bar.h_ready[bf], (n / NBUF) & 1)) break;
         const int st = ci % STAGES;
         // One acquire covers the softmax's hand-offs: before it publishes the probabilities
         // of chunk ci it has waited for the chunk's residual rows and read out the D3 / D4
         // buffer of chunk ci-2.  Each wait costs this warp far more than a satisfied test
         // suggests (it shares its issue slots with busy epilogue and softmax warps).
-        if (sub == 0 && !wait_all(&bar.p_ready[pb], (ci >> 1) & 1)) break;
+        if (hh == 0 && !wait_all(&bar.p_ready[pb], (ci >> 1) & 1)) break;
         tc_fence_after();
-        const uint64_t dP = dP0 + (uint64_t)((pb * Lay::P_BUF + sub * 1024) >> 4);
-        const uint64_t dPR = dPR0 + (uint64_t)((pb * Lay::PR_BUF) >> 4);
-        const uint64_t dR = dR0 + (uint64_t)((st * Lay::RES_BUF) >> 4);
-        const uint32_t acc0 = sub > 0 ? 1u : 0u;
+        const uint64_t dP = dP0 + (uint64_t)((pb * Lay::P_BUF) >> 4);
         if (leader) {
+          // softmax-weighted hidden sums of this half: H (fp16 pairs, token pair j at
+          // column j of the buffer) times P, K = the chunk's tokens
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {          // the two hidden halves interleaved
+          for (int kk = 0; kk < C / 16; ++kk)
+            mma_ts(t_d3 + pb * 32 + hh * 16, t_d1 + bf * 128 + kk * 8, dP + (uint64_t)(kk * 16), IDESC_3,
+                   kk > 0 ? 1u : 0u);
+          if (hh == 0) {
+            // the chunk's weighted residual rows: 16 records = two 8-row groups of the
+            // MN-major tile per MMA
+            const uint64_t dPR = dPR0 + (uint64_t)((pb * Lay::PR_BUF) >> 4);
+            const uint64_t dR = dR0 + (uint64_t)((st * Lay::RES_BUF) >> 4);
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-              mma_ts(t_d3 + pb * 32 + hh * 16, t_d1 + b * 128 + hh * 64 + kk * 8, dP + (uint64_t)(kk * 16),
-                     IDESC_3, kk > 0 ? 1u : acc0);
-            // residual rows with the chunk's first sub-tile: 16 records = two 8-row groups
-            // of the MN-major tile
-            if (sub == 0 && kk < kResCap / 16)
+            for (int kk = 0; kk < kResCap / 16; ++kk)
               mma_ss(t_d4 + pb * 16, dR + (uint64_t)(kk * (2048 >> 4)), dPR + (uint64_t)(kk * 16), IDESC_4,
                      kk > 0 ? 1u : 0u);
+            mma_commit(&bar.r_empty[st]);
+          } else {
+            mma_commit(&bar.d3_full[pb]);
           }
-          if (sub == 0) mma_commit(&bar.r_empty[st]);
-          if (sub == SUBS - 1) mma_commit(&bar.d3_full[pb]);
         }
         __syncwarp();
-        if (n + 2 < NS) ok = issue_mma1(n + 2);
+        if (n + NBUF < NS) ok = issue_mma1(n + NBUF);
       }
       // every MMA this warp issued must finish before TMEM is released
       if (leader) {
@@ -584,117 +609,42 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __res
     }
   } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + 8) {
     // ============================================================ silu epilogue
-    // Warpgroup A (warps 4-7) takes the even sub-tiles, B (8-11) the odd ones, each doing
-    // both hidden halves, so one group's MUFU work overlaps the other's TMEM round trips.
-    // Group A also swaps W1' in TMEM when the (layer, KV head) changes.
-    const int grp_ab = (warp - kEpiWarp0) >> 2;  // 0 = A (even), 1 = B (odd)
+    // Warpgroup A (warps 4-7) takes hidden half 0 of every chunk, B (8-11) half 1, all C
+    // tokens each, so one group's MUFU work overlaps the other's TMEM round trips.
+    const int grp_ab = (warp - kEpiWarp0) >> 2;  // hidden half of this group
     const int wl = warp & 3;
-    const int row = wl * 32 + lane;              // hidden unit inside a half
     const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
-    const int b = grp_ab;                        // D1 buffer of this group's sub-tiles
-    int cur_seg = -1, seg_i = -1;
-    bool ok = true;
-    TileWalk wk;
-    wk.init(x0, g.k, g.B);
-    for (int n = grp_ab; ok && n < NS; n += 2) {
-      wk.advance_to(n / SUBS);
-      if (grp_ab == 0) {
-        // perform every W1' swap that falls at or before sub-tile n
-        const int u = wk.u;
-        const int seg = wk.seg;
-        if (seg != cur_seg) {
-          ++seg_i;
-          if (seg_i > 0) {
-            // the previous segment's last MMA reading W1' must be complete
-            ok = __all_sync(0xffffffffu, mbar_wait(&bar.seg_done, (seg_i - 1) & 1, abort_flag, err, ERR_TIMEOUT));
-            if (!ok) break;
-            tc_fence_after();
-          }
-          const Unit un = unit_of(g, u);
-          const int l = g.layer0 + un.li;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const uint4* src = reinterpret_cast<const uint4*>(
-                w1f + (((size_t)l * g.Hkv + un.hkv) * kHid + hh * 128 + row) * R);
-#pragma unroll
-            for (int half = 0; half < R / 64; ++half) {
-              uint32_t w[32];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const uint4 q = __ldg(src + half * 8 + i);
-                w[4 * i] = q.x; w[4 * i + 1] = q.y; w[4 * i + 2] = q.z; w[4 * i + 3] = q.w;
-              }
-              tmem_st32(tmem + lane_off + Lay::T_W1 + hh * (R / 2) + half * 32, w);
-            }
-          }
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bar.w1_ready);
-          cur_seg = seg;
-        }
-      }
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.d1_full[b], (n >> 1) & 1, abort_flag, err, ERR_TIMEOUT))) {
-        ok = false;
+    for (int n = grp_ab; n < NS; n += 2) {
+      const int bf = n % NBUF;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.d1_full[bf], (n / NBUF) & 1, abort_flag, err, ERR_TIMEOUT)))
         break;
-      }
       tc_fence_after();
+      // 64 tokens at a time: their fp32 pre-activations (64 columns) in, their H (fp16
+      // pairs, 32 columns) out over the first half of the columns already read, so H of
+      // token pair (2j, 2j+1) lands in column j of the buffer
+      const uint32_t dcol = tmem + lane_off + Lay::T_D1 + bf * 128;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const uint32_t dcol = tmem + lane_off + Lay::T_D1 + (b * 2 + hh) * 64;
+      for (int q = 0; q < C / 64; ++q) {
         uint32_t h[32];
         {
           uint32_t v[32];
-          tmem_ld32(dcol, v);
+          tmem_ld32(dcol + q * 64, v);
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 16; ++c)
             h[c] = silu_half2_of_halfx(pack_f16x2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])));
-          tmem_ld32(dcol + 32, v);
+          tmem_ld32(dcol + q * 64 + 32, v);
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 16; ++c)
             h[16 + c] = silu_half2_of_halfx(pack_f16x2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])));
         }
-        tmem_st32(dcol, h);
+        tmem_st32(dcol + q * 32, h);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bar.h_ready[b]);
-      if (grp_ab == 0 && n + 1 < NS && (n + 1) % SUBS == 0 && wk.next_starts_segment()) {
-        // a segment that starts at group B's sub-tile n+1 needs W1' before B can go on
-        const int u1 = wk.u + 1;
-        const int seg1 = wk.seg + 1;
-        {
-          ++seg_i;
-          ok = __all_sync(0xffffffffu, mbar_wait(&bar.seg_done, (seg_i - 1) & 1, abort_flag, err, ERR_TIMEOUT));
-          if (!ok) break;
-          tc_fence_after();
-          const Unit un = unit_of(g, u1);
-          const int l = g.layer0 + un.li;
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const uint4* src = reinterpret_cast<const uint4*>(
-                w1f + (((size_t)l * g.Hkv + un.hkv) * kHid + hh * 128 + row) * R);
-#pragma unroll
-            for (int half = 0; half < R / 64; ++half) {
-              uint32_t w[32];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const uint4 q = __ldg(src + half * 8 + i);
-                w[4 * i] = q.x; w[4 * i + 1] = q.y; w[4 * i + 2] = q.z; w[4 * i + 3] = q.w;
-              }
-              tmem_st32(tmem + lane_off + Lay::T_W1 + hh * (R / 2) + half * 32, w);
-            }
-          }
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&bar.w1_ready);
-          cur_seg = seg1;
-        }
-      }
+      if (lane == 0) mbar_arrive(&bar.h_ready[bf]);
     }
   } else if (warp >= kSoftWarp0) {
     // ============================================================ softmax + accumulation
@@ -903,7 +853,9 @@ cudaError_t launch_tc(const Geom& g, const CacheBuffers& cb, const Scratch& sc, 
   using Lay = TcLayout<R, C, I8>;
   const int NG = g.L / g.G;
   const uint64_t rows = (uint64_t)g.B * NG * g.Hkv * g.nL * C;
-  CUtensorMap tmA, tmQ, tmRes;
+  CUtensorMap tmW, tmA, tmQ, tmRes;
+  // W1'/2 of every (layer, KV head): [L][Hkv][256][R] 16-bit, boxes of 64 x 128 rows
+  if (!make_map(&tmW, w1f, R, (uint64_t)g.L * g.Hkv * kHid, 128)) return cudaErrorInvalidValue;
   if (!make_map(&tmQ, sc.qt_tc, R, (uint64_t)g.U * 16, 16)) return cudaErrorInvalidValue;
   if (I8) {   // int8 rows arrive by plain bulk copies; the tile maps are not used
     tmA = tmQ;
@@ -917,8 +869,7 @@ cudaError_t launch_tc(const Geom& g, const CacheBuffers& cb, const Scratch& sc, 
   auto k = attend_tc_kernel<R, C, GQ, I8>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
   if (e != cudaSuccess) return e;
-  k<<<g.P, kThreadsTC, Lay::SMEM, s>>>(g, cb, sc, static_cast<const __nv_bfloat16*>(w1f), tmA, tmQ,
-                                        tmRes);
+  k<<<g.P, kThreadsTC, Lay::SMEM, s>>>(g, cb, sc, tmW, tmA, tmQ, tmRes);
   return cudaGetLastError();
 }
 
