@@ -494,40 +494,48 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
 
       bool ok = true;
       for (int n = 0; ok && n < NBUF && n < NS; ++n) ok = issue_mma1(n);
-      for (int n = 0; ok && n < NS; ++n) {
-        const int ci = n >> 1, hh = n & 1, pb = ci & 1, bf = n % NBUF;
-        if (!wait_all(&bar.h_ready[bf], (n / NBUF) & 1)) break;
-        const int st = ci % STAGES;
-        // One acquire covers the softmax's hand-offs: before it publishes the probabilities
-        // of chunk ci it has waited for the chunk's residual rows and read out the D3 / D4
-        // buffer of chunk ci-2.  Each wait costs this warp far more than a satisfied test
-        // suggests (it shares its issue slots with busy epilogue and softmax warps).
-        if (hh == 0 && !wait_all(&bar.p_ready[pb], (ci >> 1) & 1)) break;
-        tc_fence_after();
+      // Per chunk: the weighted sums of both hidden halves (and the residual rows) back to
+      // back, their commit, and only then the next pre-activations.  A commit waits for
+      // every MMA this thread issued before it, so D1 work queued between the two halves
+      // would hold back the softmax's fold of the chunk, and with it the probabilities of
+      // the next chunk.
+      for (int ci = 0; ok && ci < NCH; ++ci) {
+        const int pb = ci & 1, st = ci % STAGES;
         const uint64_t dP = dP0 + (uint64_t)((pb * Lay::P_BUF) >> 4);
-        if (leader) {
-          // softmax-weighted hidden sums of this half: H (fp16 pairs, token pair j at
-          // column j of the buffer) times P, K = the chunk's tokens
 #pragma unroll
-          for (int kk = 0; kk < C / 16; ++kk)
-            mma_ts(t_d3 + pb * 32 + hh * 16, t_d1 + bf * 128 + kk * 8, dP + (uint64_t)(kk * 16), IDESC_3,
-                   kk > 0 ? 1u : 0u);
-          if (hh == 0) {
-            // the chunk's weighted residual rows: 16 records = two 8-row groups of the
-            // MN-major tile per MMA
-            const uint64_t dPR = dPR0 + (uint64_t)((pb * Lay::PR_BUF) >> 4);
-            const uint64_t dR = dR0 + (uint64_t)((st * Lay::RES_BUF) >> 4);
+        for (int hh = 0; hh < 2; ++hh) {
+          const int n = 2 * ci + hh, bf = n % NBUF;
+          if (!wait_all(&bar.h_ready[bf], (n / NBUF) & 1)) { ok = false; break; }
+          // One acquire covers the softmax's hand-offs: before it publishes the
+          // probabilities of chunk ci it has waited for the chunk's residual rows and read
+          // out the D3 / D4 buffer of chunk ci-2.
+          if (hh == 0 && !wait_all(&bar.p_ready[pb], (ci >> 1) & 1)) { ok = false; break; }
+          tc_fence_after();
+          if (leader) {
+            // softmax-weighted hidden sums of this half: H (fp16 pairs, token pair j at
+            // column j of the buffer) times P, K = the chunk's tokens
 #pragma unroll
-            for (int kk = 0; kk < kResCap / 16; ++kk)
-              mma_ss(t_d4 + pb * 16, dR + (uint64_t)(kk * (2048 >> 4)), dPR + (uint64_t)(kk * 16), IDESC_4,
+            for (int kk = 0; kk < C / 16; ++kk)
+              mma_ts(t_d3 + pb * 32 + hh * 16, t_d1 + bf * 128 + kk * 8, dP + (uint64_t)(kk * 16), IDESC_3,
                      kk > 0 ? 1u : 0u);
-            mma_commit(&bar.r_empty[st]);
-          } else {
-            mma_commit(&bar.d3_full[pb]);
+            if (hh == 0) {
+              // the chunk's weighted residual rows: 16 records = two 8-row groups of the
+              // MN-major tile per MMA
+              const uint64_t dPR = dPR0 + (uint64_t)((pb * Lay::PR_BUF) >> 4);
+              const uint64_t dR = dR0 + (uint64_t)((st * Lay::RES_BUF) >> 4);
+#pragma unroll
+              for (int kk = 0; kk < kResCap / 16; ++kk)
+                mma_ss(t_d4 + pb * 16, dR + (uint64_t)(kk * (2048 >> 4)), dPR + (uint64_t)(kk * 16), IDESC_4,
+                       kk > 0 ? 1u : 0u);
+              mma_commit(&bar.r_empty[st]);
+            } else {
+              mma_commit(&bar.d3_full[pb]);
+            }
           }
+          __syncwarp();
         }
-        __syncwarp();
-        if (n + NBUF < NS) ok = issue_mma1(n + NBUF);
+        // the next pre-activations into the two buffers just read
+        for (int n = 2 * ci + NBUF; ok && n < 2 * ci + NBUF + 2 && n < NS; ++n) ok = issue_mma1(n);
       }
       // every MMA this warp issued must finish before TMEM is released
       if (leader) {
