@@ -319,13 +319,16 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
 
 // ---------------------------------------------------------------------------- fast path
 // The same computation for the common shapes (bf16, d = 128, r in {64, 128}, g in {4, 8},
-// at most kRankMax chunks), arranged so that every thread issues all of its global loads
-// before it uses any of them: the kernel above spends most of its time waiting on one
-// 16-byte load after another.  Basis and summary rows are split across threads, the raw
-// tail is staged block by block in shared memory with cooperative 16-byte loads (rows
-// padded by 16 bytes against bank conflicts), and the selected ids are placed with a
-// ballot scan instead of a serial count.
+// at most kRankMax chunks).  The chunk selection (projection, scores, top-k) and the raw
+// tail's partial softmax do not depend on each other, so each runs in its own half of a
+// 512-thread CTA with its own named barrier; only the queries are shared.  Every thread
+// issues all of its global loads before it uses any of them, basis and summary rows are
+// split across threads, the raw tail is staged in 64-token blocks through a two-buffer
+// cp.async ring (rows padded by 16 bytes against bank conflicts), and the selected ids
+// are placed with a ballot scan.
 constexpr int kFastTB = 64;               // tail tokens per staged block
+constexpr int kFastHalf = 256;            // threads per half of the fast kernel
+constexpr int kFastThreads = 2 * kFastHalf;
 
 // 16-byte asynchronous copy global -> shared (zero-filled when !valid); completes at the
 // next cp.async.wait_group.
@@ -336,12 +339,18 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, boo
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+// barrier among the 256 threads of one half (ids 1 and 2; 0 is __syncthreads)
+__device__ __forceinline__ void half_sync(int id) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kFastHalf) : "memory");
+}
 constexpr int kRowPad = 8;                // bf16 elements of padding per staged tail row
 
 template <int R, int GQ>
 struct FastSmem {
   static constexpr int D = 128;
   static constexpr int KROW = D + kRowPad;
+  static constexpr size_t TBUF = (size_t)kFastTB * KROW * 2 + (size_t)kFastTB * D * 2;   // K + V block
   static constexpr size_t bytes(int nC) {
     return (size_t)nC * 8                      // keys
            + (size_t)GQ * D * 4                // qs
@@ -349,8 +358,8 @@ struct FastSmem {
            + (size_t)R * 4                     // qsum
            + (size_t)nC * 4                    // scores
            + (size_t)nC * 4                    // selected flags
-           + (size_t)kFastTB * KROW * 2        // tail K block
-           + (size_t)kFastTB * D * 2           // tail V block
+           + 256 * 4                           // radix histogram
+           + 2 * TBUF                          // two tail blocks
            + (size_t)GQ * kFastTB * 4          // logits / probabilities
            + (size_t)4 * GQ * D * 4            // P.V partial sums of the 4 token quarters
            + (size_t)3 * GQ * 4 + 64;          // mrun, lrun, alpha, warp totals
@@ -358,7 +367,7 @@ struct FastSmem {
 };
 
 template <int R, int GQ>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kFastThreads)
 select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __restrict__ q,
                    float* __restrict__ scores_out, int32_t* __restrict__ sel_out, int tc_q_mode,
                    int do_tail) {
@@ -371,7 +380,9 @@ select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
   const int grp = l / g.G;
   const int NG = g.L / g.G;
   const int nC = g.nC;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
+  const bool tail_half = tid >= kFastHalf;
+  const int ht = tid & (kFastHalf - 1), lane = ht & 31, warp = ht >> 5;   // within the half
 
   unsigned long long* keys = reinterpret_cast<unsigned long long*>(smem_raw);   // [nC]
   float* qs = reinterpret_cast<float*>(keys + nC);                               // [GQ][D]
@@ -379,9 +390,9 @@ select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
   float* qsum = qt + GQ * R;                                                     // [R]
   float* sc_s = qsum + R;                                                        // [nC]
   int* selv = reinterpret_cast<int*>(sc_s + nC);                                 // [nC]
-  __nv_bfloat16* kblk = reinterpret_cast<__nv_bfloat16*>(selv + nC);            // [TB][KROW]
-  __nv_bfloat16* vblk = kblk + kFastTB * SM::KROW;                               // [TB][D]
-  float* lg = reinterpret_cast<float*>(vblk + kFastTB * D);                      // [GQ][TB]
+  int* hist = selv + nC;                                                         // [256]
+  unsigned char* tbuf = reinterpret_cast<unsigned char*>(hist + 256);            // 2 x (K, V) blocks
+  float* lg = reinterpret_cast<float*>(tbuf + 2 * SM::TBUF);                     // [GQ][TB]
   float* pv = lg + GQ * kFastTB;                                                 // [4][GQ][D]
   float* mrun = pv + 4 * GQ * D;                                                 // [GQ]
   float* lrun = mrun + GQ;
@@ -389,8 +400,6 @@ select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
   int* wtot = reinterpret_cast<int*>(alpha + GQ);                                // [8]
   __shared__ int radix_state[2];
 
-  // the raw tail's first block goes to shared memory asynchronously right away; it lands
-  // while the queries are projected and the chunks scored and selected
   int tl = do_tail ? cb.tail_len[un.b] : 0;
   if (tl < 0 || tl > g.T) {
     if (tid == 0) atomicOr(sc.err, ERR_TAIL_LEN);
@@ -399,249 +408,248 @@ select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
   const size_t toff = (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (size_t)g.T * D;
   const __nv_bfloat16* tk = reinterpret_cast<const __nv_bfloat16*>(cb.tail_k) + toff;
   const __nv_bfloat16* tv = reinterpret_cast<const __nv_bfloat16*>(cb.tail_v) + toff;
-  if (do_tail) {
-    const int nb0 = min(kFastTB, tl);
+  // tail block b -> buffer b % 2: 16 x 16-byte pieces per row, 4 + 4 copies per thread of
+  // the tail half; rows past the tail are zero-filled
+  auto stage_block = [&](int blk) {
+    __nv_bfloat16* kb = reinterpret_cast<__nv_bfloat16*>(tbuf + (blk & 1) * SM::TBUF);
+    __nv_bfloat16* vb = kb + kFastTB * SM::KROW;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const int it = tid + k * kThreads, t = it >> 4, e = it & 15;
-      const bool in = t < nb0;
-      cp_async16(kblk + t * SM::KROW + e * 8, in ? tk + (size_t)t * D + e * 8 : tk, in);
-      cp_async16(vblk + t * D + e * 8, in ? tv + (size_t)t * D + e * 8 : tv, in);
+      const int it = ht + k * kFastHalf, t = it >> 4, e = it & 15;
+      const int tt = blk * kFastTB + t;
+      const bool in = tt < tl;
+      cp_async16(kb + t * SM::KROW + e * 8, in ? tk + (size_t)tt * D + e * 8 : tk, in);
+      cp_async16(vb + t * D + e * 8, in ? tv + (size_t)tt * D + e * 8 : tv, in);
     }
     cp_async_commit();
+  };
+  // the tail's first two blocks go to shared memory right away
+  if (tail_half && do_tail) {
+    stage_block(0);
+    stage_block(1);
   }
 
   // --- the unit's queries (GQ x 128 bf16: one 16-byte load per thread for GQ <= 16)
   const size_t qoff = ((size_t)(un.li * g.B + un.b) * g.Hq + (size_t)un.hkv * GQ) * D;
-  if (tid < GQ * D / 8) {
+  if (!tail_half && ht < GQ * D / 8) {
     float v[8];
-    Vec8<__nv_bfloat16>::load(q + qoff + tid * 8, v);
+    Vec8<__nv_bfloat16>::load(q + qoff + ht * 8, v);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) qs[tid * 8 + i] = v[i];
+    for (int i = 0; i < 8; ++i) qs[ht * 8 + i] = v[i];
   }
   __syncthreads();
 
-  // --- qt_j = B_l q_j: each basis row split over PARTS threads, all loads issued first
-  {
-    constexpr int PARTS = kThreads / R;          // 2 for r = 128, 4 for r = 64
-    constexpr int SEG = D / PARTS;               // elements per thread
-    const int i = tid / PARTS, part = tid % PARTS;
-    const __nv_bfloat16* row = reinterpret_cast<const __nv_bfloat16*>(cb.basis) +
-                               (((size_t)l * g.Hkv + un.hkv) * R + i) * D + part * SEG;
-    uint4 w[SEG / 8];
+  if (!tail_half) {
+    // ============================================================ chunk selection
+    // --- qt_j = B_l q_j: each basis row split over PARTS threads, all loads issued first
+    {
+      constexpr int PARTS = kFastHalf / R;         // 2 for r = 128, 4 for r = 64
+      constexpr int SEG = D / PARTS;               // elements per thread
+      const int i = ht / PARTS, part = ht % PARTS;
+      const __nv_bfloat16* row = reinterpret_cast<const __nv_bfloat16*>(cb.basis) +
+                                 (((size_t)l * g.Hkv + un.hkv) * R + i) * D + part * SEG;
+      uint4 w[SEG / 8];
 #pragma unroll
-    for (int e = 0; e < SEG / 8; ++e) w[e] = __ldg(reinterpret_cast<const uint4*>(row) + e);
-    float a[GQ];
+      for (int e = 0; e < SEG / 8; ++e) w[e] = __ldg(reinterpret_cast<const uint4*>(row) + e);
+      float a[GQ];
 #pragma unroll
-    for (int j = 0; j < GQ; ++j) a[j] = 0.f;
+      for (int j = 0; j < GQ; ++j) a[j] = 0.f;
 #pragma unroll
-    for (int e = 0; e < SEG / 8; ++e) {
-      const uint32_t ww[4] = {w[e].x, w[e].y, w[e].z, w[e].w};
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const float v0 = __uint_as_float(ww[h] << 16), v1 = __uint_as_float(ww[h] & 0xffff0000u);
-        const int col = part * SEG + e * 8 + 2 * h;
-#pragma unroll
-        for (int j = 0; j < GQ; ++j) a[j] = fmaf(v1, qs[j * D + col + 1], fmaf(v0, qs[j * D + col], a[j]));
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < GQ; ++j) {
-#pragma unroll
-      for (int o = 1; o < PARTS; o <<= 1) a[j] += __shfl_xor_sync(0xffffffffu, a[j], o);
-    }
-    if (part == 0) {
-#pragma unroll
-      for (int j = 0; j < GQ; ++j) qt[j * R + i] = a[j];
-    }
-  }
-  __syncthreads();
-  for (int i = tid; i < R; i += kThreads) {
-    float s = 0.f;
-#pragma unroll
-    for (int j = 0; j < GQ; ++j) s += qt[j * R + i];
-    qsum[i] = s;
-  }
-  for (int i = tid; i < GQ * R; i += kThreads) sc.qt[(size_t)u * GQ * R + i] = qt[i] * g.qk_scale_log2;
-  if (tc_q_mode) {
-    for (int i = tid; i < 16 * R; i += kThreads) {
-      const int j = i / R;
-      const float v = j < GQ ? qt[i] * g.qk_scale_log2 : 0.f;
-      if (tc_q_mode == 1)
-        reinterpret_cast<__nv_bfloat16*>(sc.qt_tc)[(size_t)u * 16 * R + i] = __float2bfloat16_rn(v);
-      else
-        reinterpret_cast<__half*>(sc.qt_tc)[(size_t)u * 16 * R + i] = __float2half_rn(v);
-    }
-  }
-  __syncthreads();
-
-  // --- chunk scores: one thread per chunk, the whole summary row loaded at once
-  const int16_t* slot = cb.slot ? cb.slot + (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * nC : nullptr;
-  const __nv_bfloat16* summ = reinterpret_cast<const __nv_bfloat16*>(cb.summary) +
-                              (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * (size_t)g.nL * R;
-  const float inv_sqrt_d = rsqrtf((float)D);
-  for (int c = tid; c < nC; c += kThreads) {
-    const int sl = slot ? (int)slot[c] : c;
-    float s = -INFINITY;
-    if (sl >= 0 && sl < g.nL) {
-      const uint4* row = reinterpret_cast<const uint4*>(summ + (size_t)sl * R);
-      uint4 w[R / 8];
-#pragma unroll
-      for (int e = 0; e < R / 8; ++e) w[e] = __ldg(row + e);
-      float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-      for (int e = 0; e < R / 8; ++e) {
+      for (int e = 0; e < SEG / 8; ++e) {
         const uint32_t ww[4] = {w[e].x, w[e].y, w[e].z, w[e].w};
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
-          a0 = fmaf(__uint_as_float(ww[h] << 16), qsum[e * 8 + 2 * h], a0);
-          a1 = fmaf(__uint_as_float(ww[h] & 0xffff0000u), qsum[e * 8 + 2 * h + 1], a1);
+          const float v0 = __uint_as_float(ww[h] << 16), v1 = __uint_as_float(ww[h] & 0xffff0000u);
+          const int col = part * SEG + e * 8 + 2 * h;
+#pragma unroll
+          for (int j = 0; j < GQ; ++j) a[j] = fmaf(v1, qs[j * D + col + 1], fmaf(v0, qs[j * D + col], a[j]));
         }
       }
-      s = (a0 + a1) * inv_sqrt_d;
-    } else if (sl >= g.nL) {
-      atomicOr(sc.err, ERR_SLOT);
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) {
+#pragma unroll
+        for (int o = 1; o < PARTS; o <<= 1) a[j] += __shfl_xor_sync(0xffffffffu, a[j], o);
+      }
+      if (part == 0) {
+#pragma unroll
+        for (int j = 0; j < GQ; ++j) qt[j * R + i] = a[j];
+      }
     }
-    sc_s[c] = s;
-    keys[c] = ((unsigned long long)(~float_order(s)) << 32) | (unsigned)c;
-  }
-  __syncthreads();
-  if (scores_out) {
-    float* so = scores_out + ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * nC;
-    for (int c = tid; c < nC; c += kThreads) so[c] = sc_s[c];
-  }
+    half_sync(1);
+    for (int i = ht; i < R; i += kFastHalf) {
+      float s = 0.f;
+#pragma unroll
+      for (int j = 0; j < GQ; ++j) s += qt[j * R + i];
+      qsum[i] = s;
+    }
+    for (int i = ht; i < GQ * R; i += kFastHalf) sc.qt[(size_t)u * GQ * R + i] = qt[i] * g.qk_scale_log2;
+    if (tc_q_mode) {
+      for (int i = ht; i < 16 * R; i += kFastHalf) {
+        const int j = i / R;
+        const float v = j < GQ ? qt[i] * g.qk_scale_log2 : 0.f;
+        if (tc_q_mode == 1)
+          reinterpret_cast<__nv_bfloat16*>(sc.qt_tc)[(size_t)u * 16 * R + i] = __float2bfloat16_rn(v);
+        else
+          reinterpret_cast<__half*>(sc.qt_tc)[(size_t)u * 16 * R + i] = __float2half_rn(v);
+      }
+    }
+    half_sync(1);
 
-  // --- top-k: radix select on the 32-bit order key (ascending = descending score), 8 bits
-  // a pass, finds the k-th smallest key T and how many keys equal to T are still to take;
-  // those go to the lowest ids.  hist reuses the logit buffer (free until the tail).
-  int* hist = reinterpret_cast<int*>(lg);
-  uint32_t prefix = 0;
-  int kk = g.k;
+    // --- chunk scores: one thread per chunk, the whole summary row loaded at once
+    const int16_t* slot = cb.slot ? cb.slot + (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * nC : nullptr;
+    const __nv_bfloat16* summ = reinterpret_cast<const __nv_bfloat16*>(cb.summary) +
+                                (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * (size_t)g.nL * R;
+    const float inv_sqrt_d = rsqrtf((float)D);
+    for (int c = ht; c < nC; c += kFastHalf) {
+      const int sl = slot ? (int)slot[c] : c;
+      float s = -INFINITY;
+      if (sl >= 0 && sl < g.nL) {
+        const uint4* row = reinterpret_cast<const uint4*>(summ + (size_t)sl * R);
+        uint4 w[R / 8];
+#pragma unroll
+        for (int e = 0; e < R / 8; ++e) w[e] = __ldg(row + e);
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int e = 0; e < R / 8; ++e) {
+          const uint32_t ww[4] = {w[e].x, w[e].y, w[e].z, w[e].w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            a0 = fmaf(__uint_as_float(ww[h] << 16), qsum[e * 8 + 2 * h], a0);
+            a1 = fmaf(__uint_as_float(ww[h] & 0xffff0000u), qsum[e * 8 + 2 * h + 1], a1);
+          }
+        }
+        s = (a0 + a1) * inv_sqrt_d;
+      } else if (sl >= g.nL) {
+        atomicOr(sc.err, ERR_SLOT);
+      }
+      sc_s[c] = s;
+      keys[c] = ((unsigned long long)(~float_order(s)) << 32) | (unsigned)c;
+    }
+    half_sync(1);
+    if (scores_out) {
+      float* so = scores_out + ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * nC;
+      for (int c = ht; c < nC; c += kFastHalf) so[c] = sc_s[c];
+    }
+
+    // --- top-k: radix select on the 32-bit order key (ascending = descending score), 8 bits
+    // a pass, finds the k-th smallest key T and how many keys equal to T are still to take;
+    // those go to the lowest ids.
+    uint32_t prefix = 0;
+    int kk = g.k;
 #pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    hist[tid] = 0;
-    __syncthreads();
-    for (int c = tid; c < nC; c += kThreads) {
-      const uint32_t k32 = (uint32_t)(keys[c] >> 32);
-      if (shift == 24 || (k32 >> (shift + 8)) == (prefix >> (shift + 8))) atomicAdd(&hist[(k32 >> shift) & 255], 1);
-    }
-    __syncthreads();
-    const int hv = hist[tid];
-    int v = hv;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      hist[ht] = 0;
+      half_sync(1);
+      for (int c = ht; c < nC; c += kFastHalf) {
+        const uint32_t k32 = (uint32_t)(keys[c] >> 32);
+        if (shift == 24 || (k32 >> (shift + 8)) == (prefix >> (shift + 8))) atomicAdd(&hist[(k32 >> shift) & 255], 1);
+      }
+      half_sync(1);
+      const int hv = hist[ht];
+      int v = hv;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int nv = __shfl_up_sync(0xffffffffu, v, o);
-      if (lane >= o) v += nv;
-    }
-    if (lane == 31) wtot[warp] = v;
-    __syncthreads();
-    int woff = 0;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int nv = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += nv;
+      }
+      if (lane == 31) wtot[warp] = v;
+      half_sync(1);
+      int woff = 0;
 #pragma unroll
-    for (int w2 = 0; w2 < kThreads / 32; ++w2) woff += w2 < warp ? wtot[w2] : 0;
-    const int incl = v + woff, excl = incl - hv;
-    if (excl < kk && incl >= kk) {
-      radix_state[0] = tid;
-      radix_state[1] = excl;
+      for (int w2 = 0; w2 < kFastHalf / 32; ++w2) woff += w2 < warp ? wtot[w2] : 0;
+      const int incl = v + woff, excl = incl - hv;
+      if (excl < kk && incl >= kk) {
+        radix_state[0] = ht;
+        radix_state[1] = excl;
+      }
+      half_sync(1);
+      prefix |= (uint32_t)radix_state[0] << shift;
+      kk -= radix_state[1];
+      half_sync(1);   // hist and wtot are rewritten by the next pass
     }
-    __syncthreads();
-    prefix |= (uint32_t)radix_state[0] << shift;
-    kk -= radix_state[1];
-    __syncthreads();   // hist and wtot are rewritten by the next pass
-  }
-  // selected: key below T, or equal to T and among the kk lowest such ids
-  {
-    int eqrun = 0;
-    for (int base = 0; base < nC; base += kThreads) {
-      const int c = base + tid;
-      const uint32_t k32 = c < nC ? (uint32_t)(keys[c] >> 32) : 0xffffffffu;
-      const bool feq = c < nC && k32 == prefix;
-      const unsigned beq = __ballot_sync(0xffffffffu, feq);
-      if (lane == 0) wtot[warp] = __popc(beq);
-      __syncthreads();
+    // selected: key below T, or equal to T and among the kk lowest such ids
+    {
+      int eqrun = 0;
+      for (int base = 0; base < nC; base += kFastHalf) {
+        const int c = base + ht;
+        const uint32_t k32 = c < nC ? (uint32_t)(keys[c] >> 32) : 0xffffffffu;
+        const bool feq = c < nC && k32 == prefix;
+        const unsigned beq = __ballot_sync(0xffffffffu, feq);
+        if (lane == 0) wtot[warp] = __popc(beq);
+        half_sync(1);
+        int woff = 0, btot = 0;
+#pragma unroll
+        for (int w2 = 0; w2 < kFastHalf / 32; ++w2) {
+          const int t2 = wtot[w2];
+          woff += w2 < warp ? t2 : 0;
+          btot += t2;
+        }
+        const int eqrank = eqrun + woff + __popc(beq & ((1u << lane) - 1u));
+        if (c < nC) selv[c] = (k32 < prefix || (feq && eqrank < kk)) ? 1 : 0;
+        eqrun += btot;
+        half_sync(1);
+      }
+    }
+    int32_t* sel_slot = sc.sel_slot + (size_t)u * g.k;
+    int32_t* sel_id = sc.sel_id + (size_t)u * g.k;
+    int32_t* sel_user = sel_out ? sel_out + ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * g.k : nullptr;
+    int run = 0;
+    for (int base = 0; base < nC; base += kFastHalf) {
+      const int c = base + ht;
+      const int f = c < nC ? selv[c] : 0;
+      const unsigned bal = __ballot_sync(0xffffffffu, f);
+      if (lane == 0) wtot[warp] = __popc(bal);
+      half_sync(1);
       int woff = 0, btot = 0;
 #pragma unroll
-      for (int w2 = 0; w2 < kThreads / 32; ++w2) {
+      for (int w2 = 0; w2 < kFastHalf / 32; ++w2) {
         const int t2 = wtot[w2];
         woff += w2 < warp ? t2 : 0;
         btot += t2;
       }
-      const int eqrank = eqrun + woff + __popc(beq & ((1u << lane) - 1u));
-      if (c < nC) selv[c] = (k32 < prefix || (feq && eqrank < kk)) ? 1 : 0;
-      eqrun += btot;
-      __syncthreads();
-    }
-  }
-  int32_t* sel_slot = sc.sel_slot + (size_t)u * g.k;
-  int32_t* sel_id = sc.sel_id + (size_t)u * g.k;
-  int32_t* sel_user = sel_out ? sel_out + ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * g.k : nullptr;
-  int run = 0;
-  for (int base = 0; base < nC; base += kThreads) {
-    const int c = base + tid;
-    const int f = c < nC ? selv[c] : 0;
-    const unsigned bal = __ballot_sync(0xffffffffu, f);
-    if (lane == 0) wtot[warp] = __popc(bal);
-    __syncthreads();
-    int woff = 0, btot = 0;
-#pragma unroll
-    for (int w2 = 0; w2 < kThreads / 32; ++w2) {
-      const int t2 = wtot[w2];
-      woff += w2 < warp ? t2 : 0;
-      btot += t2;
-    }
-    if (f) {
-      const int pos = run + woff + __popc(bal & ((1u << lane) - 1u));
-      int sl = slot ? (int)slot[c] : c;
-      if (sl < 0 || sl >= g.nL) {
-        atomicOr(sc.err, ERR_SELECT);
-        sl = 0;
+      if (f) {
+        const int pos = run + woff + __popc(bal & ((1u << lane) - 1u));
+        int sl = slot ? (int)slot[c] : c;
+        if (sl < 0 || sl >= g.nL) {
+          atomicOr(sc.err, ERR_SELECT);
+          sl = 0;
+        }
+        if (pos < g.k) {
+          sel_slot[pos] = sl;
+          sel_id[pos] = c;
+          if (sel_user) sel_user[pos] = c;
+        }
       }
-      if (pos < g.k) {
-        sel_slot[pos] = sl;
-        sel_id[pos] = c;
-        if (sel_user) sel_user[pos] = c;
-      }
+      run += btot;
+      half_sync(1);   // wtot is rewritten by the next round
     }
-    run += btot;
-    __syncthreads();   // wtot is rewritten by the next round
+    return;
   }
   if (!do_tail) return;
 
-  // --- raw tail: partial softmax over its tokens, staged in blocks of kFastTB tokens
-  constexpr int NACC = GQ * D / 2 / kThreads;   // (head, dim pair) sums per thread
+  // ============================================================ raw tail
+  // partial softmax over its tokens, block by block from the two-buffer ring
+  constexpr int NACC = GQ * D / 2 / kFastHalf;   // (head, dim pair) sums per thread
   float accr[NACC][2];
 #pragma unroll
   for (int n = 0; n < NACC; ++n) accr[n][0] = accr[n][1] = 0.f;
-  if (tid < GQ) {
-    mrun[tid] = -INFINITY;
-    lrun[tid] = 0.f;
+  if (ht < GQ) {
+    mrun[ht] = -INFINITY;
+    lrun[ht] = 0.f;
   }
-  __syncthreads();
-  cp_async_wait_all();   // the first block (zero rows past the tail when it is short)
-  for (int t0 = 0; t0 < tl; t0 += kFastTB) {
+  const int nblk = (tl + kFastTB - 1) / kFastTB;
+  for (int bi = 0; bi < nblk; ++bi) {
+    const int t0 = bi * kFastTB;
     const int nb = min(kFastTB, tl - t0);
-    // stage the block's key and value rows: 16 x 16 bytes per row, 4 + 4 loads per thread
-    // (the first block is already in place)
-    if (t0 > 0) {
-      uint4 kv[8];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int it = tid + k * kThreads, t = it >> 4, e = it & 15;
-        const bool in = t < nb;
-        kv[k] = in ? __ldg(reinterpret_cast<const uint4*>(tk + (size_t)(t0 + t) * D) + e) : make_uint4(0, 0, 0, 0);
-        kv[4 + k] = in ? __ldg(reinterpret_cast<const uint4*>(tv + (size_t)(t0 + t) * D) + e) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int it = tid + k * kThreads, t = it >> 4, e = it & 15;
-        *reinterpret_cast<uint4*>(kblk + t * SM::KROW + e * 8) = kv[k];
-        *reinterpret_cast<uint4*>(vblk + t * D + e * 8) = kv[4 + k];
-      }
-    }
-    __syncthreads();
+    // block bi's copies (and, when it exists, block bi+1's may still be in flight)
+    if (bi + 1 < nblk) cp_async_wait_one(); else cp_async_wait_all();
+    half_sync(2);
+    const __nv_bfloat16* kblk = reinterpret_cast<const __nv_bfloat16*>(tbuf + (bi & 1) * SM::TBUF);
+    const __nv_bfloat16* vblk = kblk + kFastTB * SM::KROW;
     // logits: thread (token, GQ/4 heads)
     {
       constexpr int JPT = GQ / 4;
-      const int t = tid & (kFastTB - 1), jb = tid / kFastTB;
+      const int t = ht & (kFastTB - 1), jb = ht / kFastTB;
       float a[JPT];
 #pragma unroll
       for (int jj = 0; jj < JPT; ++jj) a[jj] = 0.f;
@@ -664,7 +672,7 @@ select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
       for (int jj = 0; jj < JPT; ++jj)
         lg[(jb * JPT + jj) * kFastTB + t] = t < nb ? a[jj] * g.qk_scale_log2 : -INFINITY;
     }
-    __syncthreads();
+    half_sync(2);
     // online softmax update: one warp per head
     if (warp < GQ) {
       const int j = warp;
@@ -681,10 +689,10 @@ select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
         mrun[j] = mnew;
       }
     }
-    __syncthreads();
+    half_sync(2);
     // P.V over the block: thread (dim pair, quarter of the tokens), all heads
     {
-      const int dp = tid & 63, tq = tid >> 6;
+      const int dp = ht & 63, tq = ht >> 6;
       float sacc[GQ][2];
 #pragma unroll
       for (int j = 0; j < GQ; ++j) sacc[j][0] = sacc[j][1] = 0.f;
@@ -705,10 +713,10 @@ select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
         pv[(tq * GQ + j) * D + 2 * dp + 1] = sacc[j][1];
       }
     }
-    __syncthreads();
+    half_sync(2);
 #pragma unroll
     for (int n = 0; n < NACC; ++n) {
-      const int it = tid + n * kThreads, j = it >> 6, dp = it & 63;
+      const int it = ht + n * kFastHalf, j = it >> 6, dp = it & 63;
       float s0 = 0.f, s1 = 0.f;
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
@@ -718,16 +726,18 @@ select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
       accr[n][0] = accr[n][0] * alpha[j] + s0;
       accr[n][1] = accr[n][1] * alpha[j] + s1;
     }
-    __syncthreads();   // the next block reuses the staging buffers
+    half_sync(2);   // buffer bi % 2, the logits and the partial sums are free again
+    if (bi + 2 < nblk) stage_block(bi + 2);
   }
+  cp_async_wait_all();
   float* rec = sc.tail_part + (size_t)u * g.tail_stride;
-  if (tid < GQ) {
-    rec[tid] = mrun[tid];
-    rec[GQ + tid] = lrun[tid];
+  if (ht < GQ) {
+    rec[ht] = mrun[ht];
+    rec[GQ + ht] = lrun[ht];
   }
 #pragma unroll
   for (int n = 0; n < NACC; ++n) {
-    const int it = tid + n * kThreads, j = it >> 6, dp = it & 63;
+    const int it = ht + n * kFastHalf, j = it >> 6, dp = it & 63;
     rec[2 * GQ + j * D + 2 * dp] = accr[n][0];
     rec[2 * GQ + j * D + 2 * dp + 1] = accr[n][1];
   }
@@ -755,8 +765,8 @@ cudaError_t launch_select_fast(const Geom& g, const CacheBuffers& cb, const Scra
   auto k = select_fast_kernel<R, GQ>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<g.U, kThreads, smem, s>>>(g, cb, sc, static_cast<const __nv_bfloat16*>(q), scores_out, sel_out,
-                                tc_q_mode, tail ? 1 : 0);
+  k<<<g.U, kFastThreads, smem, s>>>(g, cb, sc, static_cast<const __nv_bfloat16*>(q), scores_out, sel_out,
+                                    tc_q_mode, tail ? 1 : 0);
   return cudaGetLastError();
 }
 
