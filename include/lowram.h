@@ -278,6 +278,59 @@ lowram_status lowram_decode_attn_static(const lowram_config* cfg, const lowram_c
                                         int32_t layer0, int32_t n_layers, const void* q,
                                         void* out, int32_t* sel, lowram_stream stream);
 
+/* ---------------------------------------------------------------- prefill-side encoder
+ *
+ * lowram_encode: dense keys and values -> the compressed arrays lowram_cache_create takes
+ * (no eviction: pass slot = NULL there), with a GIVEN basis and predictor (no fitting).
+ * Steps, per sequence b, layer group, KV head and chunk of C tokens:
+ *   1. coefficients a_t = (1/G) sum_{l in group} k_{l,t} . B_l^T, the least-squares fit of
+ *      the group's keys on its stacked basis when every B_l has orthonormal rows
+ *      ("LowRAM Compresses KV Cache Asymmetrically", section "Cross-Layer Low-Rank Key
+ *      Compression"; the caller must pass such a basis -- for another one the result is
+ *      the average of the per-layer projections, not the least-squares fit);
+ *   2. storage: bf16 (STORE_NATIVE), or int8 with a per-row fp16 scale = max|a| / 127
+ *      rounded to fp16 and codes round-half-even(a / scale) clamped to +-127 (STORE_INT8;
+ *      same section, "Composition with Quantization and Eviction");
+ *   3. summary: the mean of the chunk's stored (dequantised) coefficient rows, bf16;
+ *   4. per layer: vhat_t = W2 silu(W1 khat_t) with khat_t the key rebuilt from the STORED
+ *      coefficients, delta_t = v_t - vhat_t ("Core Mechanism: Predict Values and Keep
+ *      Difficult Residuals");
+ *   5. residual flags: the n_resid tokens of each (b, l, KV head) with the largest
+ *      |delta_t|_2 (float32), ties to the lower token index;
+ *   6. records: unit by unit in the order (b, l, KV head), chunk by chunk, ascending token
+ *      offset; unit u's records are [u * n_resid, (u + 1) * n_resid).
+ *
+ * Arguments (DEVICE pointers, 16-byte aligned, row-major):
+ *   keys, values [B][L][Hkv][N][d] bf16;  basis [L][Hkv][r][d], w1 [L][Hkv][h][d],
+ *   w2 [L][Hkv][d][h] bf16 (the same arrays a cache is then created with);
+ *   dst->coeff [B][L/G][Hkv][N][r] bf16 or int8, dst->coeff_scale [B][L/G][Hkv][N] fp16
+ *   (STORE_INT8, else NULL), dst->summary [B][L/G][Hkv][nC][r] bf16,
+ *   dst->res_ptr [B][L][Hkv][nC+1] int32, dst->res_pos [B*L*Hkv*n_resid] uint16,
+ *   dst->res_val [B*L*Hkv*n_resid][d] bf16 or int8, dst->res_scale [B*L*Hkv*n_resid] fp16
+ *   (STORE_INT8, else NULL);  workspace: at least lowram_encode_workspace_bytes(cfg) bytes.
+ *   The caller owns every buffer.  cfg->n_live must equal n_ctx / chunk; top_k, tail_cap
+ *   and n_q_heads are not used.
+ * Supported shapes: dtype BF16, head_dim 128, mlp_hidden 256, rank 64 or 128, chunk 64 or
+ * 128, 0 <= n_resid <= n_ctx, B*L*Hkv*n_resid < 2^31; LOWRAM_EUNSUPPORTED otherwise.
+ * Stream-ordered on `stream`, no allocation, no host synchronisation. */
+typedef struct {
+  void* coeff;
+  void* coeff_scale;
+  void* summary;
+  int32_t* res_ptr;
+  uint16_t* res_pos;
+  void* res_val;
+  void* res_scale;
+} lowram_encode_dst;
+
+/* Workspace bytes lowram_encode needs for cfg (0 if cfg is invalid).  Host only. */
+uint64_t lowram_encode_workspace_bytes(const lowram_config* cfg);
+
+lowram_status lowram_encode(const lowram_config* cfg, int32_t n_resid, const void* keys,
+                            const void* values, const void* basis, const void* w1,
+                            const void* w2, const lowram_encode_dst* dst, void* workspace,
+                            uint64_t workspace_bytes, lowram_stream stream);
+
 const char* lowram_status_string(lowram_status status);
 const char* lowram_last_error_string(void);
 

@@ -25,6 +25,7 @@ __all__ = [
     "lowram_decode_attn_host", "lowram_cache_bytes", "lowram_cache_validate",
     "lowram_cache_set_stage_events", "lowram_cache_last_launches", "lowram_cache_last_path",
     "LowramCache", "config_struct", "lowram_decode_attn_static", "lowram_dense_decode_attn",
+    "lowram_encode",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblowram.so")
@@ -49,6 +50,11 @@ class LowramSrcC(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in (
         "coeff", "coeff_scale", "basis", "w1", "w2", "summary", "slot", "res_ptr", "res_pos",
         "res_val", "res_scale", "tail_k", "tail_v", "tail_len")] + [("n_records", ctypes.c_int64)]
+
+
+class LowramEncodeDstC(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "coeff", "coeff_scale", "summary", "res_ptr", "res_pos", "res_val", "res_scale")]
 
 
 class LowramBytesC(ctypes.Structure):
@@ -88,6 +94,9 @@ def lib() -> ctypes.CDLL:
         "lowram_decode_attn_static": (I32, [ctypes.POINTER(LowramConfigC), ctypes.POINTER(LowramSrcC),
                                             I32, I32, P, P, P, P]),
         "lowram_dense_decode_attn": (I32, [I32, I32, I32, I32, I32, I64, P, P, P, P, P]),
+        "lowram_encode_workspace_bytes": (U64, [ctypes.POINTER(LowramConfigC)]),
+        "lowram_encode": (I32, [ctypes.POINTER(LowramConfigC), I32, P, P, P, P, P,
+                                ctypes.POINTER(LowramEncodeDstC), P, U64, P]),
         "lowram_status_string": (ctypes.c_char_p, [I32]),
         "lowram_last_error_string": (ctypes.c_char_p, []),
     }
@@ -273,6 +282,42 @@ def lowram_cache_last_launches(handle: int) -> int:
 
 def lowram_cache_last_path(handle: int) -> int:
     return int(lib().lowram_cache_last_path(handle))
+
+
+def lowram_encode(cfg, n_resid: int, keys, values, basis, w1, w2, stream=None) -> dict:
+    """Encode dense keys/values [B][L][Hkv][N][d] (bf16, CUDA) with the given basis, w1, w2
+    (bf16, CUDA; layouts of ``lowram.h``) into the compressed storage arrays.  Allocates the
+    outputs and the workspace with torch on the keys' device and returns the arrays by their
+    ``lowram_cache_src`` names (no ``slot``: nothing is evicted)."""
+    import torch
+    c = config_struct(cfg)
+    c.n_live = c.n_ctx // c.chunk
+    B, L, G, H, N, C = c.batch, c.n_layers, c.group, c.n_kv_heads, c.n_ctx, c.chunk
+    r, d = c.rank, c.head_dim
+    int8 = c.store == 1
+    dev = keys.device
+    n = B * L * H * int(n_resid)
+    out = {
+        "coeff": torch.empty(B, L // G, H, N, r, dtype=torch.int8 if int8 else torch.bfloat16, device=dev),
+        "coeff_scale": torch.empty(B, L // G, H, N, dtype=torch.float16, device=dev) if int8 else None,
+        "summary": torch.empty(B, L // G, H, N // C, r, dtype=torch.bfloat16, device=dev),
+        "res_ptr": torch.empty(B, L, H, N // C + 1, dtype=torch.int32, device=dev),
+        "res_pos": torch.empty(n, dtype=torch.int16, device=dev),
+        "res_val": torch.empty(n, d, dtype=torch.int8 if int8 else torch.bfloat16, device=dev),
+        "res_scale": torch.empty(n, dtype=torch.float16, device=dev) if int8 else None,
+    }
+    ws_bytes = int(lib().lowram_encode_workspace_bytes(ctypes.byref(c)))
+    if ws_bytes == 0:
+        raise LowramError(1, "lowram_encode_workspace_bytes", "invalid config for the encoder")
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    dst = LowramEncodeDstC()
+    for k in LowramEncodeDstC._fields_:
+        setattr(dst, k[0], _ptr(out[k[0]]) if (out[k[0]] is not None and out[k[0]].numel()) else None)
+    _check(lib().lowram_encode(ctypes.byref(c), int(n_resid), _ptr(keys), _ptr(values), _ptr(basis),
+                               _ptr(w1), _ptr(w2), ctypes.byref(dst), _ptr(ws), ws_bytes, _stream(stream)),
+           "lowram_encode")
+    out["_workspace"] = ws        # kept alive until the stream has used it
+    return out
 
 
 class LowramCache:

@@ -168,6 +168,71 @@ const char* lowram_status_string(lowram_status s) {
 
 const char* lowram_last_error_string(void) { return g_last_error.c_str(); }
 
+// ------------------------------------------------------------------------------ encoder
+
+namespace {
+
+lowram_status encode_geom(const lowram_config* cfg, Geom* g) {
+  if (!cfg) return inval("config is NULL");
+  // top_k, n_q_heads and tail_cap play no part in encoding: check the rest
+  lowram_config cc = *cfg;
+  cc.top_k = 1;
+  cc.n_q_heads = cc.n_kv_heads;
+  cc.tail_cap = 0;
+  const lowram_config* c = &cc;
+  lowram_status st = check_config(c);
+  if (st != LOWRAM_OK) return st;
+  const int nC = c->n_ctx / c->chunk;
+  if (c->n_live != nC) return inval("the encoder evicts nothing: n_live must equal n_ctx / chunk");
+  if (c->dtype != LOWRAM_BF16 || c->head_dim != 128 || c->mlp_hidden != 256 || !(c->rank == 64 || c->rank == 128) ||
+      !(c->chunk == 64 || c->chunk == 128)) {
+    g_last_error = "the encoder takes bf16, head_dim 128, mlp_hidden 256, rank 64 or 128, chunk 64 or 128";
+    return LOWRAM_EUNSUPPORTED;
+  }
+  *g = Geom{};
+  g->B = c->batch; g->L = c->n_layers; g->G = c->group; g->Hkv = c->n_kv_heads; g->Hq = c->n_q_heads;
+  g->g = c->n_q_heads / c->n_kv_heads; g->d = c->head_dim; g->r = c->rank; g->h = c->mlp_hidden;
+  g->N = c->n_ctx; g->C = c->chunk; g->nC = nC; g->nL = nC; g->k = c->top_k; g->T = c->tail_cap;
+  g->layer0 = 0; g->n_layers = c->n_layers;
+  return LOWRAM_OK;
+}
+
+}  // namespace
+
+uint64_t lowram_encode_workspace_bytes(const lowram_config* cfg) {
+  Geom g;
+  if (encode_geom(cfg, &g) != LOWRAM_OK) return 0;
+  return encode_workspace_bytes(g);
+}
+
+lowram_status lowram_encode(const lowram_config* cfg, int32_t n_resid, const void* keys, const void* values,
+                            const void* basis, const void* w1, const void* w2, const lowram_encode_dst* dst,
+                            void* workspace, uint64_t workspace_bytes, lowram_stream stream) {
+  Geom g;
+  lowram_status st = encode_geom(cfg, &g);
+  if (st != LOWRAM_OK) return st;
+  if (n_resid < 0 || n_resid > g.N) return inval("n_resid must lie in [0, n_ctx]");
+  const long long units = (long long)g.B * g.L * g.Hkv;
+  if (units * n_resid >= (1LL << 31)) return inval("B * L * Hkv * n_resid must be below 2^31");
+  if (!dst) return inval("NULL destination");
+  const void* req[] = {keys, values, basis, w1, w2, dst->coeff, dst->summary, dst->res_ptr, workspace};
+  for (const void* p : req)
+    if (!p || !aligned16(p)) return inval("a required pointer is NULL or not 16-byte aligned");
+  const bool i8 = cfg->store == LOWRAM_STORE_INT8;
+  if (i8 && (!dst->coeff_scale || !aligned16(dst->coeff_scale)))
+    return inval("int8 store needs a 16-byte aligned coeff_scale");
+  if (n_resid > 0) {
+    if (!dst->res_pos || !aligned16(dst->res_pos) || !dst->res_val || !aligned16(dst->res_val))
+      return inval("residual arrays missing or misaligned");
+    if (i8 && (!dst->res_scale || !aligned16(dst->res_scale))) return inval("int8 store needs res_scale");
+  }
+  if (workspace_bytes < encode_workspace_bytes(g)) return inval("workspace smaller than lowram_encode_workspace_bytes");
+  cudaError_t e = launch_encode(g, cfg->store, n_resid, keys, values, basis, w1, w2, *dst, workspace,
+                                reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "encode");
+  return LOWRAM_OK;
+}
+
 lowram_status lowram_cache_create(const lowram_config* cfg, const lowram_cache_src* src,
                                   lowram_cache** out, lowram_stream stream) {
   lowram_status st = check_config(cfg);

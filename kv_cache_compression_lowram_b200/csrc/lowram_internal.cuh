@@ -152,6 +152,13 @@ cudaError_t launch_combine(const Geom& g, const CacheBuffers& cb, const Scratch&
 // [h][r] scaled by 1/2 for tensor cores).
 cudaError_t launch_fold(const Geom& g, const CacheBuffers& cb, int dtype, int store,
                         float* w1f_t, void* w1f_tc, cudaStream_t s);
+// Prefill-side encoder (dense K, V -> compressed arrays); bf16, d = 128, h = 256,
+// r in {64, 128}, C in {64, 128}.  The workspace holds the fp32 W1' fold, the residual
+// norms and the flags.
+size_t encode_workspace_bytes(const Geom& g);
+cudaError_t launch_encode(const Geom& g, int store, int n_res, const void* keys, const void* values,
+                          const void* basis, const void* w1, const void* w2, const lowram_encode_dst& dst,
+                          void* workspace, cudaStream_t s);
 // Device-side table checks.
 cudaError_t launch_validate(const Geom& g, const CacheBuffers& cb, uint32_t* err,
                             cudaStream_t s);

@@ -191,6 +191,7 @@ def _gen(device, *keys: int) -> torch.Generator:
 
 # tensor tags for seeding
 _T_COEFF, _T_BASIS, _T_W1, _T_W2, _T_EPS, _T_EVICT, _T_TAILA, _T_TAILK, _T_TAILV, _T_Q = range(10)
+_T_DKA, _T_DKN, _T_DV = 10, 11, 12
 
 
 # --------------------------------------------------------------------------- container
@@ -403,6 +404,36 @@ def make_weights(cfg: LowramConfig, identity_basis: bool = False):
             w2[l, hk] = torch.randn(d, h, generator=_gen("cpu", cfg.seed, _T_W2, l, hk),
                                     dtype=torch.float64) / math.sqrt(h)
     return basis, w1, w2
+
+
+def make_dense_kv(cfg: LowramConfig, device="cpu"):
+    """Dense prefill keys and values [B][L][Hkv][N][d] (bf16) for the encoder.
+
+    Keys follow the cache's law: K_l = A B_l + N(0, 0.01^2) with A (coefficient law, shared
+    by the layers of a group) and B_l from ``make_weights``; values are N(0, 0.1^2) with a
+    seeded 5 % of tokens scaled by 4 (so that residual norms spread out).  Returns (K, V).
+    """
+    B, L, G, Hkv, N, d, r = (cfg.batch, cfg.n_layers, cfg.group, cfg.n_kv_heads, cfg.n_ctx,
+                             cfg.head_dim, cfg.rank)
+    basis, _, _ = make_weights(cfg)
+    K = torch.empty(B, L, Hkv, N, d, dtype=torch.bfloat16, device=device)
+    V = torch.empty(B, L, Hkv, N, d, dtype=torch.bfloat16, device=device)
+    bdev = basis.to(device=device, dtype=torch.float32)
+    for b in range(B):
+        for grp in range(L // G):
+            for h in range(Hkv):
+                a = _coeff_law(N, r, _gen(device, cfg.seed, _T_DKA, b, grp, h), device).float()
+                for li in range(G):
+                    l = grp * G + li
+                    noise = torch.randn(N, d, generator=_gen(device, cfg.seed, _T_DKN, b, l, h),
+                                        device=device) * 0.01
+                    K[b, l, h] = (a @ bdev[l, h] + noise).to(torch.bfloat16)
+        for l in range(L):
+            gen = _gen(device, cfg.seed, _T_DV, b, l)
+            v = torch.randn(Hkv, N, d, generator=gen, device=device) * 0.1
+            big = torch.rand(Hkv, N, generator=gen, device=device) < 0.05
+            V[b, l] = torch.where(big.unsqueeze(-1), 4.0 * v, v).to(torch.bfloat16)
+    return K, V
 
 
 def make_cache(cfg: LowramConfig, device="cpu", tail_len=None) -> SynthCache:

@@ -92,14 +92,19 @@ def flag_worst(norms: np.ndarray, n_res: int) -> np.ndarray:
 def encode(cfg: dict, keys: np.ndarray, values: np.ndarray, basis: np.ndarray,
            w1: np.ndarray, w2: np.ndarray, n_res: int,
            tail_k: Optional[np.ndarray] = None, tail_v: Optional[np.ndarray] = None,
-           tail_len: Optional[np.ndarray] = None) -> dict:
+           tail_len: Optional[np.ndarray] = None, given: Optional[tuple] = None) -> dict:
     """Encode dense keys/values [B][L][Hkv][N][d] (float64) with the given basis [L][Hkv][r][d],
     predictor w1 [L][Hkv][h][d], w2 [L][Hkv][d][h] (float64) into the storage layout of
     ``lowram.h`` (no eviction: every chunk live).  Returns the dict ``OracleCache`` reads,
     with bf16 arrays as uint16 bit patterns (storage dtype bf16; int8 + fp16 scales when
     cfg["store"] == "int8").  The tail arrays are passed through (zero-length tails if
     omitted).  Also returns, under "extra", the float64 intermediates the tests compare:
-    coefficients before storage, residual norms and flags."""
+    coefficients before storage, residual norms and flags.
+
+    ``given`` = (codes, scales) replaces the result of steps 1-2 with given stored
+    coefficients (bf16 bit patterns and None, or int8 codes and fp16 scales, layout of
+    ``coeff`` / ``coeff_scale``), so that steps 3-6 can be checked on exactly the stored
+    values another implementation produced."""
     B, L, Hkv, N, d = keys.shape
     G, C = cfg["group"], cfg["chunk"]
     r = basis.shape[2]
@@ -117,15 +122,20 @@ def encode(cfg: dict, keys: np.ndarray, values: np.ndarray, basis: np.ndarray,
             for h in range(Hkv):
                 a = lstsq_coefficients(keys[b, ls, h], basis[ls, h])       # step 1
                 coeff_full[b, grp, h] = a
-                if int8:                                                    # step 2
+                if given is not None:
+                    q = given[0][b, grp, h]
+                    s = given[1][b, grp, h] if int8 else None
+                elif int8:                                                  # step 2
                     q, s = quantize_rows_int8(a)
+                else:
+                    q, s = round_bf16_bits(a), None
+                if int8:
                     coeff_store[b, grp, h] = q
                     coeff_scale[b, grp, h] = s
                     deq = q.astype(np.float64) * s.astype(np.float64)[:, None]
                 else:
-                    bits = round_bf16_bits(a)
-                    coeff_store[b, grp, h] = bits
-                    deq = _bits_f64(bits)
+                    coeff_store[b, grp, h] = q
+                    deq = _bits_f64(q)
                 stored[b, grp, h] = deq
                 summary[b, grp, h] = round_bf16_bits(deq.reshape(nC, C, r).mean(axis=1))   # step 3
 

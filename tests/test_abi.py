@@ -91,3 +91,27 @@ def test_status_strings():
     lib = K.lib()
     for s in range(7):
         assert lib.lowram_status_string(s)
+
+
+def test_encode_host_checks():
+    """Workspace size and the argument checks that return before any CUDA call."""
+    cfg = S.MISTRAL_GROUP
+    c = K.config_struct(cfg)
+    c.n_live = c.n_ctx // c.chunk
+    al = lambda x: (x + 255) // 256 * 256
+    units = cfg.batch * cfg.n_layers * cfg.n_kv_heads
+    want = (al(cfg.n_layers * cfg.n_kv_heads * cfg.rank * cfg.mlp_hidden * 4) + al(units * cfg.n_ctx * 4)
+            + al(units * cfg.n_ctx))
+    assert K.lib().lowram_encode_workspace_bytes(ctypes.byref(c)) == want
+    f32 = K.config_struct(S.TINY_F32)
+    assert K.lib().lowram_encode_workspace_bytes(ctypes.byref(f32)) == 0
+    dst = K.LowramEncodeDstC()
+    st = K.lib().lowram_encode(ctypes.byref(f32), 1, None, None, None, None, None, ctypes.byref(dst),
+                               None, 0, None)
+    assert st == 4   # LOWRAM_EUNSUPPORTED
+    st = K.lib().lowram_encode(ctypes.byref(c), -1, None, None, None, None, None, ctypes.byref(dst),
+                               None, 0, None)
+    assert st == 1   # LOWRAM_EINVAL
+    st = K.lib().lowram_encode(ctypes.byref(c), 4, None, None, None, None, None, ctypes.byref(dst),
+                               None, 0, None)
+    assert st == 1

@@ -212,3 +212,17 @@ def test_planted_mistake_high_index_ties_fails_flags(monkeypatch):
     ref[order.numpy()] = True
     assert not np.array_equal(wrong(norms, 2), ref)
     np.testing.assert_array_equal(E.flag_worst(norms, 2), ref)
+
+
+@pytest.mark.parametrize("store", ["native", "int8"])
+def test_given_stored_coefficients_reproduce_steps_3_to_6(store):
+    """Feeding the encoder's own stored coefficients back reproduces every later output."""
+    cfg = dict(CFG, store=store)
+    rng = np.random.default_rng(11)
+    basis, w1, w2 = _weights(rng, cfg)
+    _, K, V = _planted(rng, cfg, basis, noise=0.02)
+    a = E.encode(cfg, K, V, basis, w1, w2, 32)
+    b = E.encode(cfg, K, V, basis, w1, w2, 32, given=(a["coeff"], a["coeff_scale"]))
+    for k in ("coeff", "summary", "res_ptr", "res_pos", "res_val"):
+        np.testing.assert_array_equal(a[k], b[k])
+    np.testing.assert_array_equal(a["extra"]["flags"], b["extra"]["flags"])
