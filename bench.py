@@ -49,6 +49,8 @@ def parse():
                     help="also run the batch sweep 1,4,16,32,64 (extra JSON lines)")
     ap.add_argument("--dense", action="store_true",
                     help="only the uncompressed bf16 dense-KV baseline at its largest batch")
+    ap.add_argument("--encode", action="store_true",
+                    help="only the prefill-side encoder (dense K, V -> compressed cache) of the workload")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -443,6 +445,103 @@ def run_dense(args, ws, rank, local, cfg_name=DEFAULT_CONFIG):
     return line
 
 
+ENC_METRIC = "prefill tokens/s encoded (dense K,V -> compressed cache, all layers and KV heads)"
+
+
+def encode_flops(cfg) -> float:
+    """Arithmetic of one encode call: the group projections (2 G d r per token and group),
+    and the predictor, evaluated twice (residual norms, then the flagged tokens' records),
+    2 * 2 h (r + d) per token and layer."""
+    pos = cfg.batch * cfg.n_kv_heads * cfg.n_ctx
+    proj = pos * cfg.n_groups * cfg.group * cfg.head_dim * cfg.rank * 2
+    pred = pos * cfg.n_layers * 2 * 2 * cfg.mlp_hidden * (cfg.rank + cfg.head_dim)
+    return float(proj + pred)
+
+
+def encode_oracle_rate(cfg, Kd, Vd, weights, budget_s: float = 20.0):
+    """The encoder oracle on (b, group, KV head) slices until the budget is spent; returns
+    (prefill tokens/s scaled to the whole workload, sample description, threads)."""
+    import dataclasses as dc
+    import oracle.encode as E
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = 1
+    G = cfg.group
+    sub = dc.asdict(cfg.replace(name="enc_slice", batch=1, n_layers=G, n_kv_heads=1))
+    f64 = lambda t: t.float().double().cpu().numpy()
+    basis, w1, w2 = weights
+    done, t0 = 0, time.perf_counter()
+    slices = [(b, grp, h) for b in range(cfg.batch) for grp in range(cfg.n_groups) for h in range(cfg.n_kv_heads)]
+    rng = np.random.default_rng(0)
+    for i in rng.permutation(len(slices)):
+        b, grp, h = slices[i]
+        ls = slice(grp * G, (grp + 1) * G)
+        E.encode(sub, f64(Kd[b:b + 1, ls, h:h + 1]), f64(Vd[b:b + 1, ls, h:h + 1]), f64(basis[ls, h:h + 1]),
+                 f64(w1[ls, h:h + 1]), f64(w2[ls, h:h + 1]), cfg.n_resid)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    # a slice is 1 / (groups * KV heads) of a sequence's encode
+    tokens = done * cfg.n_ctx / (cfg.n_groups * cfg.n_kv_heads)
+    return tokens / dt, f"{done} of {len(slices)} (b, group, KV head) slices, {dt:.1f} s", threads
+
+
+def run_encode(args, ws, rank, local):
+    """The prefill-side encoder on the workload's dense keys and values (resident in HBM)."""
+    import kv_cache_compression_lowram_b200 as K
+    cfg = replica_config(S.CONFIGS[args.config], rank).replace(evict_frac=0.0)
+    dev = torch.device("cuda", local)
+    Kd, Vd = S.make_dense_kv(cfg, device=dev)
+    weights = [t.to(torch.bfloat16) for t in S.make_weights(cfg)]
+    wd = [t.to(dev).contiguous() for t in weights]
+    out = K.lowram_encode(cfg, cfg.n_resid, Kd, Vd, *wd)
+    for _ in range(max(0, args.warmup - 1)):
+        K.lowram_encode(cfg, cfg.n_resid, Kd, Vd, *wd, out=out)
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 10))
+    clocks = ClockSampler(local)
+    barrier(ws)
+    clocks.start()
+    time.sleep(0.3)
+    stream = torch.cuda.current_stream()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        K.lowram_encode(cfg, cfg.n_resid, Kd, Vd, *wd, out=out)
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    value, ms_total = aggregate_rate(cfg.batch * cfg.n_ctx * steps, start.elapsed_time(end), ws)
+    ms_step = ms_total / steps
+    flops = encode_flops(cfg)
+    # CUDA-core fp32 peak: 148 SMs x 128 FMA lanes x 2 flops x the maximum SM clock
+    peak = 148 * 128 * 2 * ((clk or {}).get("sm_max_mhz") or 1965.0) * 1e6 / 1e12
+    achieved = flops / (ms_step / 1e3) / 1e12
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        rate, sample, threads = encode_oracle_rate(cfg, Kd, Vd, weights)
+        cpu = {"value": round(rate, 2), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": sample}
+    return {
+        "metric": ENC_METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "impl": "encoder",
+        "config": {"workload": cfg.name, "batch": cfg.batch, "n_layers": cfg.n_layers, "n_ctx": cfg.n_ctx,
+                   "kv_heads": cfg.n_kv_heads, "rank": cfg.rank, "chunk": cfg.chunk, "store": cfg.store,
+                   "n_resid": cfg.n_resid, "dense_kv_gb": round(Kd.numel() * 4 / 1e9, 2),
+                   "l2": "inputs larger than L2"},
+        "roofline": {"bound": "alu", "kernel": "encode (all kernels of the call)", "achieved": round(achieved, 2),
+                     "peak": round(peak, 1), "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": None, "flops_per_call": flops},
+        "cpu_baseline": cpu, "e2e": None, "gpu_launches": steps * 5, "clocks": clk,
+    }
+
+
 def run_reference(args, ws, rank):
     """The oracle (fp64 numpy, host cores) on the same workload, bounded samples per step."""
     if rank != 0:
@@ -483,11 +582,13 @@ def main():
         line = run_reference(args, ws, rank)
     elif args.dense:
         line = run_dense(args, ws, rank, local)
+    elif args.encode:
+        line = run_encode(args, ws, rank, local)
     else:
         line = run_lowram(args, ws, rank, local)
     if rank == 0 and line is not None:
         print(json.dumps(line), flush=True)
-    if args.sweep and args.impl == "lowram" and not args.dense:
+    if args.sweep and args.impl == "lowram" and not args.dense and not args.encode:
         import gc
         for b in (1, 4, 16, 32, 64):
             args.config = f"llama8b_32k_bf16_b{b}"

@@ -284,14 +284,17 @@ def lowram_cache_last_path(handle: int) -> int:
     return int(lib().lowram_cache_last_path(handle))
 
 
-def lowram_encode(cfg, n_resid: int, keys, values, basis, w1, w2, stream=None) -> dict:
+def lowram_encode(cfg, n_resid: int, keys, values, basis, w1, w2, stream=None, out=None) -> dict:
     """Encode dense keys/values [B][L][Hkv][N][d] (bf16, CUDA) with the given basis, w1, w2
     (bf16, CUDA; layouts of ``lowram.h``) into the compressed storage arrays.  Allocates the
-    outputs and the workspace with torch on the keys' device and returns the arrays by their
+    outputs and the workspace with torch on the keys' device (or reuses ``out``, the dict a
+    previous call with the same shapes returned) and returns the arrays by their
     ``lowram_cache_src`` names (no ``slot``: nothing is evicted)."""
     import torch
     c = config_struct(cfg)
     c.n_live = c.n_ctx // c.chunk
+    if out is not None:
+        return _encode_into(c, int(n_resid), keys, values, basis, w1, w2, out, stream)
     B, L, G, H, N, C = c.batch, c.n_layers, c.group, c.n_kv_heads, c.n_ctx, c.chunk
     r, d = c.rank, c.head_dim
     int8 = c.store == 1
@@ -309,14 +312,20 @@ def lowram_encode(cfg, n_resid: int, keys, values, basis, w1, w2, stream=None) -
     ws_bytes = int(lib().lowram_encode_workspace_bytes(ctypes.byref(c)))
     if ws_bytes == 0:
         raise LowramError(1, "lowram_encode_workspace_bytes", "invalid config for the encoder")
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    out["_workspace"] = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    return _encode_into(c, int(n_resid), keys, values, basis, w1, w2, out, stream)
+
+
+def _encode_into(c, n_resid, keys, values, basis, w1, w2, out, stream):
+    ws = out["_workspace"]
     dst = LowramEncodeDstC()
     for k in LowramEncodeDstC._fields_:
-        setattr(dst, k[0], _ptr(out[k[0]]) if (out[k[0]] is not None and out[k[0]].numel()) else None)
-    _check(lib().lowram_encode(ctypes.byref(c), int(n_resid), _ptr(keys), _ptr(values), _ptr(basis),
-                               _ptr(w1), _ptr(w2), ctypes.byref(dst), _ptr(ws), ws_bytes, _stream(stream)),
+        t = out[k[0]]
+        setattr(dst, k[0], _ptr(t) if (t is not None and t.numel()) else None)
+    _check(lib().lowram_encode(ctypes.byref(c), n_resid, _ptr(keys), _ptr(values), _ptr(basis),
+                               _ptr(w1), _ptr(w2), ctypes.byref(dst), _ptr(ws), int(ws.numel()),
+                               _stream(stream)),
            "lowram_encode")
-    out["_workspace"] = ws        # kept alive until the stream has used it
     return out
 
 
