@@ -15,12 +15,17 @@
 //                       the flagged tokens
 //   enc_select_kernel   per (b, layer, KV head): the n_resid largest norms (ties to the
 //                       lower token) by a radix select, flags and the CSR offsets
-// All CUDA-core fp32 arithmetic from bf16 inputs (register-tiled, operands staged in shared
-// memory); the tensor-core form of the two contractions is future work.
+// enc_resid_kernel is the CUDA-core fp32 form (any store); enc_resid_tc_kernel the tcgen05
+// form of the same pass for bf16 stores (D1 = W1'/2 . A^T, silu into shared memory as fp16,
+// Vhat = W2 . H with W2 in fp16, fp32 accumulators in TMEM).
+#include <algorithm>
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include "lowram_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace lowram {
 namespace {
@@ -461,36 +466,346 @@ enc_select_kernel(int N, int C, int n_res, const float* __restrict__ norms, uint
   }
 }
 
+// ------------------------------------------------------------- tensor-core residuals
+// One persistent CTA per SM walks a contiguous range of tiles (unit, chunk), units ordered
+// (layer, KV head, sequence) so that W1' and W2 are reloaded only when the (layer, KV head)
+// changes.  Per tile, in order (every step waits for the previous one):
+//   TMA: the chunk's stored coefficient tile (C rows x R, 128-byte swizzle, K-major)
+//   MMA: D1_hh = (W1'_hh / 2) . A^T for hidden halves hh = 0, 1 (SS, M=128, N=C, K=R)
+//   warps 0-3 / 4-7: H_hh = silu(2 D1_hh) = u + u tanh(u) as fp16, written to shared memory
+//        MN-major (hidden rows, token-contiguous, 128-byte swizzle) -- half 0 over the A tile
+//   MMA: D2 = W2 . H (SS, M=128 value dims, N=C, K=256; W2 in fp16, K-major)
+//   warps: delta = V - D2 per (dim, token); norms (pass 1) or the flagged rows (pass 2)
+// TMEM columns: D1 half 0 [0, C), half 1 [C, 2C), D2 [2C, 3C).
+template <int R, int C>
+struct EncTcLayout {
+  static constexpr int KSLABS = R / 64;
+  static constexpr int W1_HALF = KSLABS * 16384;          // 128 hidden rows x R, bf16
+  static constexpr int W2_BYTES = 4 * 16384;              // 128 dims x 256 hidden, fp16
+  static constexpr int H_HALF = (C / 64) * 16384;         // 128 hidden rows x C tokens, fp16
+  static constexpr int A_BYTES = KSLABS * 16384;
+  static constexpr int OFF_W1 = 0;
+  static constexpr int OFF_W2 = OFF_W1 + 2 * W1_HALF;
+  static constexpr int OFF_AH = OFF_W2 + W2_BYTES;        // the A tile, then H half 0
+  static constexpr int OFF_H1 = OFF_AH + (A_BYTES > H_HALF ? A_BYTES : H_HALF);
+  static constexpr int OFF_MISC = OFF_H1 + H_HALF;
+  static constexpr int MISC_BYTES = 64 + 4 * C * 4 + 2 * C * 4;
+  static constexpr int SMEM = OFF_MISC + MISC_BYTES + 1024;
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+struct EncTcMisc {
+  uint64_t bar_w, bar_in, bar_mma;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int R, int C, bool EMIT>
+__global__ void __launch_bounds__(kEncThreads, 1)
+enc_resid_tc_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant__ CUtensorMap tmW1,
+                    const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmA,
+                    const __nv_bfloat16* __restrict__ values, float* __restrict__ norms,
+                    const uint8_t* __restrict__ flags, const int32_t* __restrict__ res_ptr,
+                    uint16_t* __restrict__ res_pos, __nv_bfloat16* __restrict__ res_val, uint32_t* err) {
+  using namespace tc;
+  using Lay = EncTcLayout<R, C>;
+  extern __shared__ unsigned char enc_smem_dyn[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(enc_smem_dyn) + 1023) & ~uintptr_t(1023));
+  EncTcMisc* misc = reinterpret_cast<EncTcMisc*>(smem + Lay::OFF_MISC);
+  float* part = reinterpret_cast<float*>(smem + Lay::OFF_MISC + 64);   // [4][C]
+  int* fl = reinterpret_cast<int*>(part + 4 * C);                       // [C]
+  int* pfx = fl + C;                                                    // [C]
+  volatile int* abort_flag = &misc->abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nC = N / C, NG = L / G;
+  const long long total = (long long)B * L * Hkv * nC;
+  const long long x0 = total * blockIdx.x / gridDim.x, x1 = total * (blockIdx.x + 1) / gridDim.x;
+
+  if (tid == 0) {
+    mbar_init(&misc->bar_w, 1);
+    mbar_init(&misc->bar_in, 1);
+    mbar_init(&misc->bar_mma, 1);
+    misc->abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == 0) {
+    tmem_alloc(&misc->tmem_base, 512);
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc->tmem_base;
+  const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+  const uint64_t dW1 = smem_desc(smem_u32(smem + Lay::OFF_W1), 16, 1024, 2);
+  const uint64_t dW2 = smem_desc(smem_u32(smem + Lay::OFF_W2), 16, 1024, 2);
+  const uint64_t dA = smem_desc(smem_u32(smem + Lay::OFF_AH), 16, 1024, 2);
+  const uint64_t dH0 = smem_desc(smem_u32(smem + Lay::OFF_AH), 16384, 1024, 2);   // MN-major
+  const uint64_t dH1 = smem_desc(smem_u32(smem + Lay::OFF_H1), 16384, 1024, 2);
+  constexpr uint32_t IDESC_1 = idesc_f16(128, C, 1, 1);         // W1' (bf16) x A (bf16)
+  constexpr uint32_t IDESC_2 = idesc_f16(128, C, 0, 0, 0, 1);   // W2 (f16) x H (f16, MN-major)
+  uint32_t ph_w = 0, ph_in = 0, ph_mma = 0;
+  int cur_seg = -1;
+  bool ok = true;
+  const int hh = warp >> 2;                 // epilogue 1: hidden half; epilogue 2: token half
+  const int row = 32 * (warp & 3) + lane;   // TMEM lane: hidden unit in the half / value dim
+
+  for (long long x = x0; ok && x < x1; ++x) {
+    const int u = (int)(x / nC), c = (int)(x % nC);
+    const int b = u % B, seg = u / B, hkv = seg % Hkv, l = seg / Hkv, grp = l / G;
+    const size_t unit = ((size_t)b * L + l) * Hkv + hkv;
+    if (seg != cur_seg) {   // W1' halves and W2 of this (layer, KV head)
+      if (tid == 0) {
+        mbar_expect_tx(&misc->bar_w, (uint32_t)(2 * Lay::W1_HALF + Lay::W2_BYTES));
+        for (int h2 = 0; h2 < 2; ++h2)
+          for (int ks = 0; ks < Lay::KSLABS; ++ks)
+            tma_load_2d(smem + Lay::OFF_W1 + h2 * Lay::W1_HALF + ks * 16384, &tmW1, &misc->bar_w, ks * 64,
+                        seg * 256 + h2 * 128);
+        for (int j = 0; j < 4; ++j)
+          tma_load_2d(smem + Lay::OFF_W2 + j * 16384, &tmW2, &misc->bar_w, j * 64, seg * 128);
+      }
+      ok = mbar_wait(&misc->bar_w, ph_w, abort_flag, err, ERR_TIMEOUT);
+      ph_w ^= 1;
+      cur_seg = seg;
+      if (!ok) break;
+    }
+    const long long arow = (((long long)b * NG + grp) * Hkv + hkv) * N + (long long)c * C;
+    if (tid == 0) {
+      mbar_expect_tx(&misc->bar_in, (uint32_t)(Lay::KSLABS * C * 128));
+      for (int ks = 0; ks < Lay::KSLABS; ++ks)
+        tma_load_2d(smem + Lay::OFF_AH + ks * 16384, &tmA, &misc->bar_in, ks * 64, (int)arow);
+    }
+    if (EMIT)
+      for (int t = tid; t < C; t += kEncThreads) fl[t] = flags[unit * N + (size_t)c * C + t];
+    // this thread's values for the residual epilogue (dim `row`, tokens hh*C/2 .. +C/2),
+    // requested now so that they arrive during the MMAs
+    uint32_t vv[C / 4];
+    {
+      const unsigned short* vrow = reinterpret_cast<const unsigned short*>(values) +
+                                   (unit * N + (size_t)c * C + hh * (C / 2)) * kEncD + row;
+#pragma unroll
+      for (int j = 0; j < C / 4; ++j)
+        vv[j] = (uint32_t)__ldg(vrow + (size_t)(2 * j) * kEncD) | ((uint32_t)__ldg(vrow + (size_t)(2 * j + 1) * kEncD) << 16);
+    }
+    ok = mbar_wait(&misc->bar_in, ph_in, abort_flag, err, ERR_TIMEOUT);
+    ph_in ^= 1;
+    if (!ok) break;
+    // D1 of both hidden halves
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+        for (int kk = 0; kk < R / 16; ++kk) {
+          const uint64_t ko = (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2);
+          mma_ss(tmem + h2 * C, dW1 + (uint64_t)((h2 * Lay::W1_HALF) >> 4) + ko, dA + ko, IDESC_1, kk > 0 ? 1u : 0u);
+        }
+      mma_commit(&misc->bar_mma);
+    }
+    ok = mbar_wait(&misc->bar_mma, ph_mma, abort_flag, err, ERR_TIMEOUT);
+    ph_mma ^= 1;
+    if (!ok) break;
+    tc_fence_after();
+    // silu -> H_hh (fp16) in shared memory, MN-major: hidden row `row`, 8 tokens per 16 bytes
+    {
+      unsigned char* hrow = smem + (hh == 0 ? Lay::OFF_AH : Lay::OFF_H1) + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+      for (int q = 0; q < C / 32; ++q) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + hh * C + q * 32, v);
+        tmem_wait_ld();
+        uint32_t h[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          h[j] = silu_half2_of_halfx(pack_f16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])));
+        unsigned char* blk = hrow + (q >> 1) * 16384;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int c16 = (q & 1) * 4 + k;
+          *reinterpret_cast<uint4*>(blk + ((c16 ^ (row & 7)) << 4)) = make_uint4(h[4 * k], h[4 * k + 1], h[4 * k + 2], h[4 * k + 3]);
+        }
+      }
+    }
+    tc_fence_before();
+    fence_proxy_async_smem();
+    __syncthreads();
+    // D2 = W2 . H over both hidden halves
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int slab = h2 * 2 + (kk >> 2);
+          mma_ss(tmem + 2 * C, dW2 + (uint64_t)((slab * 16384 + (kk & 3) * 32) >> 4),
+                 (h2 == 0 ? dH0 : dH1) + (uint64_t)((kk * 2048) >> 4), IDESC_2, (h2 | kk) ? 1u : 0u);
+        }
+      mma_commit(&misc->bar_mma);
+    }
+    if (EMIT && tid < C) {   // rank of each token among the chunk's flagged tokens
+      int s = 0;
+      for (int t = 0; t < tid; ++t) s += fl[t];
+      pfx[tid] = s;
+    }
+    ok = mbar_wait(&misc->bar_mma, ph_mma, abort_flag, err, ERR_TIMEOUT);
+    ph_mma ^= 1;
+    __syncthreads();   // pfx
+    if (!ok) break;
+    tc_fence_after();
+    // delta = V - Vhat for dim `row`, tokens hh*C/2 .. +C/2
+    const size_t rbase = EMIT ? (size_t)res_ptr[unit * (nC + 1) + c] : 0;
+#pragma unroll
+    for (int q = 0; q < C / 64; ++q) {
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_off + 2 * C + hh * (C / 2) + q * 32, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int t = hh * (C / 2) + q * 32 + j;
+        const uint32_t w = vv[(q * 32 + j) >> 1];
+        const float vt = __uint_as_float(((j & 1) ? (w >> 16) : (w & 0xffffu)) << 16);
+        const float d = vt - __uint_as_float(v[j]);
+        if (!EMIT) {
+          float ss = d * d;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+          if (lane == 0) part[(warp & 3) * C + t] = ss;
+        } else if (fl[t]) {
+          const size_t rec = rbase + pfx[t];
+          res_val[rec * kEncD + row] = __float2bfloat16_rn(d);
+          if (row == 0) res_pos[rec] = (uint16_t)t;
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (!EMIT)
+      for (int t = tid; t < C; t += kEncThreads)
+        norms[unit * N + (size_t)c * C + t] = sqrtf(part[t] + part[C + t] + part[2 * C + t] + part[3 * C + t]);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// 2-D tensor map over a row-major [rows][inner] 16-bit array, boxes of 64 x box_rows elements
+// in the 128-byte swizzle layout.
+bool enc_make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return false;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+__global__ void to_half_kernel(const __nv_bfloat16* __restrict__ src, __half* __restrict__ dst, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    dst[i] = __float2half_rn(__bfloat162float(src[i]));
+}
+
+// Workspace pieces (256-byte aligned, in this order).
+struct EncWs {
+  float* w1f_t;            // [L][Hkv][r][h] fp32 W1'
+  __nv_bfloat16* w1f_tc;   // [L][Hkv][h][r] bf16 W1'/2 (tensor-core path)
+  __half* w2h;             // [L][Hkv][d][h] fp16 W2 (tensor-core path)
+  float* norms;            // [units][N]
+  uint8_t* flags;          // [units][N]
+  uint32_t* err;           // device error word of the tensor-core kernels
+};
+
+EncWs carve(const Geom& g, void* workspace, size_t* bytes) {
+  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  const size_t units = (size_t)g.B * g.L * g.Hkv, lh = (size_t)g.L * g.Hkv;
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    unsigned char* p = static_cast<unsigned char*>(workspace) + off;
+    off += al(n);
+    return p;
+  };
+  EncWs w;
+  w.w1f_t = reinterpret_cast<float*>(take(lh * g.r * g.h * 4));
+  w.w1f_tc = reinterpret_cast<__nv_bfloat16*>(take(lh * g.h * g.r * 2));
+  w.w2h = reinterpret_cast<__half*>(take(lh * g.d * g.h * 2));
+  w.norms = reinterpret_cast<float*>(take(units * g.N * 4));
+  w.flags = take(units * g.N);
+  w.err = reinterpret_cast<uint32_t*>(take(4));
+  if (bytes) *bytes = off;
+  return w;
+}
+
 template <int R, int C, bool I8>
 cudaError_t launch_encode_t(const Geom& g, int n_res, const void* keys, const void* values,
-                            const void* basis, const void* w2, const lowram_encode_dst& dst,
-                            const float* w1f_t, float* norms, uint8_t* flags, cudaStream_t s) {
+                            const void* basis, const void* w2, const lowram_encode_dst& dst, const EncWs& w,
+                            cudaStream_t s) {
   const int NG = g.L / g.G, nC = g.N / C;
+  const size_t units = (size_t)g.B * g.L * g.Hkv;
   dim3 gc(nC, g.Hkv, g.B * NG), gr(nC, g.Hkv, g.B * g.L);
   enc_coeff_kernel<R, C, I8><<<gc, kEncThreads, 0, s>>>(
       g.L, g.G, g.Hkv, g.N, static_cast<const __nv_bfloat16*>(keys), static_cast<const __nv_bfloat16*>(basis),
       dst.coeff, static_cast<__half*>(dst.coeff_scale), static_cast<__nv_bfloat16*>(dst.summary));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (!I8) {   // tensor cores
+    using Lay = EncTcLayout<R, C>;
+    CUtensorMap tmW1, tmW2, tmA;
+    const uint64_t lh = (uint64_t)g.L * g.Hkv;
+    if (!enc_make_map(&tmW1, w.w1f_tc, R, lh * kEncH, 128) || !enc_make_map(&tmW2, w.w2h, kEncH, lh * kEncD, 128) ||
+        !enc_make_map(&tmA, dst.coeff, R, (uint64_t)g.B * NG * g.Hkv * g.N, C))
+      return cudaErrorInvalidValue;
+    to_half_kernel<<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w2), w.w2h, (size_t)lh * kEncD * kEncH);
+    if ((e = cudaMemsetAsync(w.err, 0, 4, s)) != cudaSuccess) return e;
+    int n_sm = 0;
+    if ((e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, 0)) != cudaSuccess) return e;
+    const unsigned grid = (unsigned)std::min<size_t>((size_t)n_sm, units * nC);
+    auto k1 = enc_resid_tc_kernel<R, C, false>;
+    auto k2 = enc_resid_tc_kernel<R, C, true>;
+    if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM)) != cudaSuccess) return e;
+    k1<<<grid, kEncThreads, Lay::SMEM, s>>>(g.B, g.L, g.G, g.Hkv, g.N, tmW1, tmW2, tmA,
+                                            static_cast<const __nv_bfloat16*>(values), w.norms, nullptr, nullptr,
+                                            nullptr, nullptr, w.err);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    enc_select_kernel<<<(unsigned)units, kSelThreads, (size_t)nC * sizeof(int), s>>>(g.N, C, n_res, w.norms,
+                                                                                     w.flags, dst.res_ptr);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (n_res > 0)
+      k2<<<grid, kEncThreads, Lay::SMEM, s>>>(g.B, g.L, g.G, g.Hkv, g.N, tmW1, tmW2, tmA,
+                                              static_cast<const __nv_bfloat16*>(values), w.norms, w.flags,
+                                              dst.res_ptr, dst.res_pos, static_cast<__nv_bfloat16*>(dst.res_val),
+                                              w.err);
+    return cudaGetLastError();
+  }
   const size_t smem = ResidSmem<R, C>::bytes();
   auto k1 = enc_resid_kernel<R, C, I8, false>;
   auto k2 = enc_resid_kernel<R, C, I8, true>;
   if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
   if ((e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess) return e;
   k1<<<gr, kEncThreads, smem, s>>>(g.L, g.G, g.Hkv, g.N, n_res, dst.coeff, static_cast<const __half*>(dst.coeff_scale),
-                                   w1f_t, static_cast<const __nv_bfloat16*>(w2),
-                                   static_cast<const __nv_bfloat16*>(values), norms, nullptr, nullptr, nullptr,
+                                   w.w1f_t, static_cast<const __nv_bfloat16*>(w2),
+                                   static_cast<const __nv_bfloat16*>(values), w.norms, nullptr, nullptr, nullptr,
                                    nullptr, nullptr);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const size_t units = (size_t)g.B * g.L * g.Hkv;
-  enc_select_kernel<<<(unsigned)units, kSelThreads, (size_t)nC * sizeof(int), s>>>(g.N, C, n_res, norms, flags,
+  enc_select_kernel<<<(unsigned)units, kSelThreads, (size_t)nC * sizeof(int), s>>>(g.N, C, n_res, w.norms, w.flags,
                                                                                    dst.res_ptr);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (n_res > 0)
     k2<<<gr, kEncThreads, smem, s>>>(g.L, g.G, g.Hkv, g.N, n_res, dst.coeff,
-                                     static_cast<const __half*>(dst.coeff_scale), w1f_t,
+                                     static_cast<const __half*>(dst.coeff_scale), w.w1f_t,
                                      static_cast<const __nv_bfloat16*>(w2), static_cast<const __nv_bfloat16*>(values),
-                                     norms, flags, dst.res_ptr, dst.res_pos, dst.res_val,
+                                     w.norms, w.flags, dst.res_ptr, dst.res_pos, dst.res_val,
                                      static_cast<__half*>(dst.res_scale));
   return cudaGetLastError();
 }
@@ -498,30 +813,25 @@ cudaError_t launch_encode_t(const Geom& g, int n_res, const void* keys, const vo
 }  // namespace
 
 size_t encode_workspace_bytes(const Geom& g) {
-  const size_t units = (size_t)g.B * g.L * g.Hkv;
-  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
-  return al((size_t)g.L * g.Hkv * g.r * g.h * 4) + al(units * g.N * 4) + al(units * g.N);
+  size_t bytes = 0;
+  carve(g, nullptr, &bytes);
+  return bytes;
 }
 
 cudaError_t launch_encode(const Geom& g, int store, int n_res, const void* keys, const void* values,
                           const void* basis, const void* w1, const void* w2, const lowram_encode_dst& dst,
                           void* workspace, cudaStream_t s) {
-  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
-  const size_t units = (size_t)g.B * g.L * g.Hkv;
-  unsigned char* ws = static_cast<unsigned char*>(workspace);
-  float* w1f_t = reinterpret_cast<float*>(ws);
-  float* norms = reinterpret_cast<float*>(ws + al((size_t)g.L * g.Hkv * g.r * g.h * 4));
-  uint8_t* flags = reinterpret_cast<uint8_t*>(ws + al((size_t)g.L * g.Hkv * g.r * g.h * 4) + al(units * g.N * 4));
+  const EncWs w = carve(g, workspace, nullptr);
   CacheBuffers cb{};
   cb.w1 = w1;
   cb.basis = basis;
-  cudaError_t e = launch_fold(g, cb, LOWRAM_BF16, LOWRAM_STORE_NATIVE, w1f_t, nullptr, s);
+  cudaError_t e = launch_fold(g, cb, LOWRAM_BF16, LOWRAM_STORE_NATIVE, w.w1f_t, w.w1f_tc, s);
   if (e != cudaSuccess) return e;
   const bool i8 = store == LOWRAM_STORE_INT8;
-#define LOWRAM_ENC_CASE(RR, CC)                                                                      \
-  if (g.r == RR && g.C == CC)                                                                        \
-    return i8 ? launch_encode_t<RR, CC, true>(g, n_res, keys, values, basis, w2, dst, w1f_t, norms, flags, s) \
-              : launch_encode_t<RR, CC, false>(g, n_res, keys, values, basis, w2, dst, w1f_t, norms, flags, s);
+#define LOWRAM_ENC_CASE(RR, CC)                                                                    \
+  if (g.r == RR && g.C == CC)                                                                      \
+    return i8 ? launch_encode_t<RR, CC, true>(g, n_res, keys, values, basis, w2, dst, w, s)        \
+              : launch_encode_t<RR, CC, false>(g, n_res, keys, values, basis, w2, dst, w, s);
   LOWRAM_ENC_CASE(128, 128)
   LOWRAM_ENC_CASE(128, 64)
   LOWRAM_ENC_CASE(64, 128)

@@ -100,8 +100,10 @@ def test_encode_host_checks():
     c.n_live = c.n_ctx // c.chunk
     al = lambda x: (x + 255) // 256 * 256
     units = cfg.batch * cfg.n_layers * cfg.n_kv_heads
-    want = (al(cfg.n_layers * cfg.n_kv_heads * cfg.rank * cfg.mlp_hidden * 4) + al(units * cfg.n_ctx * 4)
-            + al(units * cfg.n_ctx))
+    lh = cfg.n_layers * cfg.n_kv_heads
+    want = (al(lh * cfg.rank * cfg.mlp_hidden * 4) + al(lh * cfg.mlp_hidden * cfg.rank * 2)
+            + al(lh * cfg.head_dim * cfg.mlp_hidden * 2) + al(units * cfg.n_ctx * 4) + al(units * cfg.n_ctx)
+            + al(4))
     assert K.lib().lowram_encode_workspace_bytes(ctypes.byref(c)) == want
     f32 = K.config_struct(S.TINY_F32)
     assert K.lib().lowram_encode_workspace_bytes(ctypes.byref(f32)) == 0

@@ -1,10 +1,12 @@
 """Parity of the CUDA encoder (through the C ABI) with the fp64 encoder oracle.
 
-Stored coefficients and summaries agree to one bf16 unit (the GPU accumulates in fp32,
-the oracle in fp64, and both round the result to bf16) or one int8 code; residual flags
-agree wherever the oracle's n_res-th and (n_res+1)-th norms are apart by more than 1e-4
-relative, and otherwise every token the GPU flags lies within that distance of the
-oracle's threshold; residual rows agree to the bf16 (int8) rounding of the stored rows.
+Stored coefficients agree to the tolerance the bf16-rounded basis implies (see
+_check_encode); summaries to one bf16 unit.  Residual norms: the tensor-core predictor
+(bf16 stores) rounds the hidden activations to fp16 (2^-11 relative) before the second
+GEMM, which moves a residual norm by a few 1e-4 of itself; so flags agree wherever the
+oracle's n_res-th and (n_res+1)-th norms are apart by more than 1e-3 relative, and
+otherwise every token on which the two sides differ lies within 1e-3 of the oracle's
+threshold.  Residual rows agree to their bf16 (int8) rounding.
 The encoded cache then decodes on the GPU in parity with the decode oracle.
 """
 
@@ -114,7 +116,7 @@ def _check_encode(cfg, g, o, og, n_res):
             continue
         thr = np.sort(norms[idx])[::-1][n_res - 1]
         diff = fg[idx] != fo[idx]
-        assert np.all(np.abs(norms[idx][diff] - thr) <= 1e-4 * thr), idx
+        assert np.all(np.abs(norms[idx][diff] - thr) <= 1e-3 * thr), idx
     # residual rows of tokens both sides flagged
     d = cfg.head_dim
     if n_res > 0:
