@@ -155,6 +155,8 @@ LLAMA_32K = _reg(LowramConfig(
 # Batch sweep of the 32K Llama shape.
 for _b in (1, 4, 16, 32, 64):
     _reg(LLAMA_32K.replace(name=f"llama8b_32k_bf16_b{_b}", batch=_b))
+# One sequence, 8 layers: a profiling case above L2 size but only ~1 GB of dense K, V.
+_reg(LLAMA_32K.replace(name="llama8b_32k_bf16_b1_l8", batch=1, n_layers=8))
 # Composition with int8 quantisation and 50 % chunk eviction at 64K context, batch 8.
 LLAMA_64K_INT8 = _reg(LowramConfig(
     name="llama8b_64k_int8_evict", batch=8, n_layers=32, group=4, n_kv_heads=8,
