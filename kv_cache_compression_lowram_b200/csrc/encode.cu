@@ -567,7 +567,7 @@ enc_resid_tc_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant__
       ok = mbar_wait(&misc->bar_w, ph_w, abort_flag, err, ERR_TIMEOUT);
       ph_w ^= 1;
       cur_seg = seg;
-      if (!ok) break;
+      if (!__syncthreads_and(ok)) break;
     }
     const long long arow = (((long long)b * NG + grp) * Hkv + hkv) * N + (long long)c * C;
     if (tid == 0) {
@@ -589,7 +589,7 @@ enc_resid_tc_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant__
     }
     ok = mbar_wait(&misc->bar_in, ph_in, abort_flag, err, ERR_TIMEOUT);
     ph_in ^= 1;
-    if (!ok) break;
+    if (!__syncthreads_and(ok)) break;
     // D1 of both hidden halves
     if (tid == 0) {
       tc_fence_after();
@@ -604,7 +604,7 @@ enc_resid_tc_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant__
     }
     ok = mbar_wait(&misc->bar_mma, ph_mma, abort_flag, err, ERR_TIMEOUT);
     ph_mma ^= 1;
-    if (!ok) break;
+    if (!__syncthreads_and(ok)) break;
     tc_fence_after();
     // silu -> H_hh (fp16) in shared memory, MN-major: hidden row `row`, 8 tokens per 16 bytes
     {
@@ -649,8 +649,7 @@ enc_resid_tc_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant__
     }
     ok = mbar_wait(&misc->bar_mma, ph_mma, abort_flag, err, ERR_TIMEOUT);
     ph_mma ^= 1;
-    __syncthreads();   // pfx
-    if (!ok) break;
+    if (!__syncthreads_and(ok)) break;   // (also publishes pfx)
     tc_fence_after();
     // delta = V - Vhat for dim `row`, tokens hh*C/2 .. +C/2
     const size_t rbase = EMIT ? (size_t)res_ptr[unit * (nC + 1) + c] : 0;
@@ -687,6 +686,192 @@ enc_resid_tc_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant__
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// ----------------------------------------------------------- tensor-core coefficients
+// Per (b, group, KV head, chunk) tile of 128 tokens: D = sum_{l in group} K_l . B_l^T (SS
+// MMAs, M = 128 tokens, N = R, K = d in steps of 16), the key and basis slabs of layer l+1
+// loaded by TMA while the MMAs of layer l run (two buffers).  Epilogue: thread = token row
+// (TMEM lane), so an int8 row scale is thread-local; the chunk summary sums the stored
+// rows through shared memory.  Persistent, one tile in flight.
+template <int R>
+struct EncCoeffLayout {
+  static constexpr int BUF = 2 * 16384 + 2 * R * 128;   // key slabs (128 rows) + basis slabs (R rows)
+  static constexpr int OFF_BUF = 0;
+  static constexpr int OFF_SUM = 2 * BUF;                // [128][R] fp32 stored rows
+  static constexpr int OFF_MISC = OFF_SUM + 128 * R * 4;
+  static constexpr int SMEM = OFF_MISC + 64 + 1024;
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+struct EncCoeffMisc {
+  uint64_t bar_in[2], bar_mma[2];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int R, bool I8>
+__global__ void __launch_bounds__(128, 1)
+enc_coeff_tc_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmB, void* __restrict__ coeff,
+                    __half* __restrict__ coeff_scale, __nv_bfloat16* __restrict__ summary, uint32_t* err) {
+  using namespace tc;
+  using Lay = EncCoeffLayout<R>;
+  constexpr int C = 128;
+  extern __shared__ unsigned char enc_smem_dyn[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(enc_smem_dyn) + 1023) & ~uintptr_t(1023));
+  EncCoeffMisc* misc = reinterpret_cast<EncCoeffMisc*>(smem + Lay::OFF_MISC);
+  float* rows = reinterpret_cast<float*>(smem + Lay::OFF_SUM);
+  volatile int* abort_flag = &misc->abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int nC = N / C, NG = L / G;
+  const long long total = (long long)B * NG * Hkv * nC;
+  const long long x0 = total * blockIdx.x / gridDim.x, x1 = total * (blockIdx.x + 1) / gridDim.x;
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&misc->bar_in[i], 1);
+      mbar_init(&misc->bar_mma[i], 1);
+    }
+    misc->abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == 0) {
+    tmem_alloc(&misc->tmem_base, 128 <= R ? 128 : 64);
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc->tmem_base;
+  constexpr uint32_t IDESC = idesc_f16(128, R, 1, 1);
+  uint32_t ph_in[2] = {0, 0}, ph_mma[2] = {0, 0};
+  int used[2] = {0, 0};   // MMAs were issued on buffer i and not yet waited for
+  bool ok = true;
+  // job j of the CTA: (tile, layer in group); buffer j % 2
+  auto issue_load = [&](long long x, int li, int buf) {
+    const int c = (int)(x % nC);
+    const long long y = x / nC;
+    const int hkv = (int)(y % Hkv), grp = (int)((y / Hkv) % NG), b = (int)(y / ((long long)Hkv * NG));
+    const int l = grp * G + li;
+    unsigned char* bb = smem + Lay::OFF_BUF + buf * Lay::BUF;
+    mbar_expect_tx(&misc->bar_in[buf], (uint32_t)(2 * 16384 + 2 * R * 128));
+    const int krow = (int)((((long long)b * L + l) * Hkv + hkv) * N + (long long)c * C);
+    for (int ks = 0; ks < 2; ++ks) {
+      tma_load_2d(bb + ks * 16384, &tmK, &misc->bar_in[buf], ks * 64, krow);
+      tma_load_2d(bb + 2 * 16384 + ks * R * 128, &tmB, &misc->bar_in[buf], ks * 64, (l * Hkv + hkv) * R);
+    }
+  };
+  const long long jobs = (x1 - x0) * G;
+  if (tid == 0 && jobs > 0) issue_load(x0, 0, 0);
+  for (long long j = 0; ok && j < jobs; ++j) {
+    const long long x = x0 + j / G;
+    const int li = (int)(j % G), buf = (int)(j & 1);
+    if (tid == 0) {
+      // the next job's slabs go to the other buffer once the MMAs that read it are done
+      if (j + 1 < jobs) {
+        const int nb = buf ^ 1;
+        if (used[nb]) {
+          ok = mbar_wait(&misc->bar_mma[nb], ph_mma[nb], abort_flag, err, ERR_TIMEOUT);
+          ph_mma[nb] ^= 1;
+          used[nb] = 0;
+        }
+        if (ok) issue_load(x0 + (j + 1) / G, (int)((j + 1) % G), nb);
+      }
+      if (ok) ok = mbar_wait(&misc->bar_in[buf], ph_in[buf], abort_flag, err, ERR_TIMEOUT);
+      ph_in[buf] ^= 1;
+      if (ok) {
+        tc_fence_after();
+        const unsigned char* bb = smem + Lay::OFF_BUF + buf * Lay::BUF;
+        const uint64_t dK = smem_desc(smem_u32(bb), 16, 1024, 2);
+        const uint64_t dB = smem_desc(smem_u32(bb + 2 * 16384), 16, 1024, 2);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int ks = kk >> 2;
+          mma_ss(tmem, dK + (uint64_t)((ks * 16384 + (kk & 3) * 32) >> 4),
+                 dB + (uint64_t)((ks * R * 128 + (kk & 3) * 32) >> 4), IDESC, (li > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&misc->bar_mma[buf]);
+        used[buf] = 1;
+      }
+    }
+    if (!__syncthreads_and(ok)) break;   // every thread leaves at the same point
+    if (li != G - 1) continue;
+    // the tile is complete: its last MMAs, then the epilogue
+    if (tid == 0) {
+      ok = mbar_wait(&misc->bar_mma[buf], ph_mma[buf], abort_flag, err, ERR_TIMEOUT);
+      ph_mma[buf] ^= 1;
+      used[buf] = 0;
+    }
+    if (!__syncthreads_and(ok)) break;
+    tc_fence_after();
+    const int c = (int)(x % nC);
+    const long long y = x / nC;
+    const int hkv = (int)(y % Hkv), grp = (int)((y / Hkv) % NG), b = (int)(y / ((long long)Hkv * NG));
+    const size_t row0 = (((size_t)b * NG + grp) * Hkv + hkv) * N + (size_t)c * C;
+    const int t = tid;   // token row of the tile = TMEM lane
+    const float inv_g = 1.f / (float)G;
+    float amax = 0.f;
+    if (I8) {   // the row's largest |a| first
+#pragma unroll
+      for (int q = 0; q < R / 32; ++q) {
+        uint32_t v[32];
+        tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + q * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k) amax = fmaxf(amax, fabsf(__uint_as_float(v[k]) * inv_g));
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < R / 32; ++q) {
+      uint32_t v[32];
+      tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + q * 32, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int k8 = 0; k8 < 4; ++k8) {
+        float x8[8], deq[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) x8[k] = __uint_as_float(v[k8 * 8 + k]) * inv_g;
+        const int col = q * 32 + k8 * 8;
+        if (I8) {
+          __half sh;
+          uint2 codes;
+          quantize8(x8, amax, &sh, &codes, deq);
+          *reinterpret_cast<uint2*>(static_cast<int8_t*>(coeff) + (row0 + t) * R + col) = codes;
+          if (col == 0) coeff_scale[row0 + t] = sh;
+        } else {
+          const uint4 p = pack_bf16x8(x8);
+          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(coeff) + (row0 + t) * R + col) = p;
+          const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            deq[2 * h] = __uint_as_float(pw[h] << 16);
+            deq[2 * h + 1] = __uint_as_float(pw[h] & 0xffff0000u);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) rows[t * R + ((col + k + t) % R)] = deq[k];   // rotated: no bank conflicts
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    for (int rr = tid; rr < R; rr += 128) {
+      float sum = 0.f;
+      for (int t2 = 0; t2 < C; ++t2) sum += rows[t2 * R + ((rr + t2) % R)];
+      summary[((((size_t)b * NG + grp) * Hkv + hkv) * nC + c) * R + rr] = __float2bfloat16_rn(sum / (float)C);
+    }
+    __syncthreads();
+  }
+  // let every copy and MMA this CTA started finish before shared memory and TMEM go away
+  if (tid == 0) {
+    volatile int never = 0;
+    for (int i = 0; i < 2; ++i)
+      if (used[i]) mbar_wait(&misc->bar_mma[i], ph_mma[i], &never, err, ERR_TIMEOUT);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128 <= R ? 128 : 64);
   }
 }
 
@@ -753,11 +938,28 @@ cudaError_t launch_encode_t(const Geom& g, int n_res, const void* keys, const vo
   const int NG = g.L / g.G, nC = g.N / C;
   const size_t units = (size_t)g.B * g.L * g.Hkv;
   dim3 gc(nC, g.Hkv, g.B * NG), gr(nC, g.Hkv, g.B * g.L);
-  enc_coeff_kernel<R, C, I8><<<gc, kEncThreads, 0, s>>>(
-      g.L, g.G, g.Hkv, g.N, static_cast<const __nv_bfloat16*>(keys), static_cast<const __nv_bfloat16*>(basis),
-      dst.coeff, static_cast<__half*>(dst.coeff_scale), static_cast<__nv_bfloat16*>(dst.summary));
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaError_t e;
+  int n_sm = 0;
+  if ((e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, 0)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(w.err, 0, 4, s)) != cudaSuccess) return e;
+  if (C == 128) {   // coefficients on tensor cores
+    using CL = EncCoeffLayout<R>;
+    CUtensorMap tmK, tmB;
+    if (!enc_make_map(&tmK, keys, kEncD, (uint64_t)g.B * g.L * g.Hkv * g.N, 128) ||
+        !enc_make_map(&tmB, basis, kEncD, (uint64_t)g.L * g.Hkv * R, R))
+      return cudaErrorInvalidValue;
+    auto kc = enc_coeff_tc_kernel<R, I8>;
+    if ((e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, CL::SMEM)) != cudaSuccess) return e;
+    const unsigned cgrid = (unsigned)std::min<size_t>((size_t)n_sm, (size_t)g.B * NG * g.Hkv * nC);
+    kc<<<cgrid, 128, CL::SMEM, s>>>(g.B, g.L, g.G, g.Hkv, g.N, tmK, tmB, dst.coeff,
+                                    static_cast<__half*>(dst.coeff_scale), static_cast<__nv_bfloat16*>(dst.summary),
+                                    w.err);
+  } else {
+    enc_coeff_kernel<R, C, I8><<<gc, kEncThreads, 0, s>>>(
+        g.L, g.G, g.Hkv, g.N, static_cast<const __nv_bfloat16*>(keys), static_cast<const __nv_bfloat16*>(basis),
+        dst.coeff, static_cast<__half*>(dst.coeff_scale), static_cast<__nv_bfloat16*>(dst.summary));
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (!I8) {   // tensor cores
     using Lay = EncTcLayout<R, C>;
     CUtensorMap tmW1, tmW2, tmA;
@@ -766,9 +968,6 @@ cudaError_t launch_encode_t(const Geom& g, int n_res, const void* keys, const vo
         !enc_make_map(&tmA, dst.coeff, R, (uint64_t)g.B * NG * g.Hkv * g.N, C))
       return cudaErrorInvalidValue;
     to_half_kernel<<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w2), w.w2h, (size_t)lh * kEncD * kEncH);
-    if ((e = cudaMemsetAsync(w.err, 0, 4, s)) != cudaSuccess) return e;
-    int n_sm = 0;
-    if ((e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, 0)) != cudaSuccess) return e;
     const unsigned grid = (unsigned)std::min<size_t>((size_t)n_sm, units * nC);
     auto k1 = enc_resid_tc_kernel<R, C, false>;
     auto k2 = enc_resid_tc_kernel<R, C, true>;
