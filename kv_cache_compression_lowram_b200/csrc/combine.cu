@@ -221,25 +221,57 @@ combine_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, __nv_bfloat16* __restri
   }
 }
 
-// W1'[i][rr] = sum_dd W1[i][dd] * B_l[rr][dd] for every (layer, KV head).
+// W1'[i][rr] = sum_dd W1[i][dd] * B_l[rr][dd] for every (layer, KV head).  A block computes a
+// 32 (hidden) x 64 (rank) tile of one (layer, KV head) with both operands staged through
+// shared memory 32 columns of d at a time; thread (ty, tx) accumulates hidden rows 2ty, 2ty+1
+// and ranks 4tx .. 4tx+3.
 template <typename T>
-__global__ void fold_kernel(Geom g, const T* __restrict__ w1, const T* __restrict__ basis,
-                            float* __restrict__ w1f_t, __nv_bfloat16* __restrict__ w1f_bf16,
-                            __half* __restrict__ w1f_f16) {
-  const size_t n = (size_t)g.L * g.Hkv * g.h * g.r;
-  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < n;
-       idx += (size_t)gridDim.x * blockDim.x) {
-    const int rr = (int)(idx % g.r);
-    const int i = (int)((idx / g.r) % g.h);
-    const size_t lh = idx / ((size_t)g.r * g.h);
-    const T* wr = w1 + (lh * g.h + i) * g.d;
-    const T* br = basis + (lh * g.r + rr) * g.d;
-    float a = 0.f;
-    for (int dd = 0; dd < g.d; ++dd) a = fmaf(to_f(wr[dd]), to_f(br[dd]), a);
-    if (w1f_t) w1f_t[(lh * g.r + rr) * g.h + i] = a;
-    // tensor-core copy holds W1'/2: the MMA then yields u = x/2 and silu(x) = u + u*tanh(u)
-    if (w1f_bf16) w1f_bf16[idx] = __float2bfloat16_rn(0.5f * a);
-    if (w1f_f16) w1f_f16[idx] = __float2half_rn(0.5f * a);
+__global__ void __launch_bounds__(256)
+fold_tiled_kernel(Geom g, const T* __restrict__ w1, const T* __restrict__ basis, float* __restrict__ w1f_t,
+                  __nv_bfloat16* __restrict__ w1f_bf16, __half* __restrict__ w1f_f16) {
+  constexpr int TI = 32, TR = 64, TK = 32;
+  __shared__ float ws[TI][TK + 1];
+  __shared__ float bs[TR][TK + 1];
+  const int i0 = blockIdx.x * TI, r0 = blockIdx.y * TR;
+  const size_t lh = blockIdx.z;
+  const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+  float acc[2][4] = {};
+  for (int k0 = 0; k0 < g.d; k0 += TK) {
+    for (int p = tid; p < TI * TK; p += 256) {
+      const int i = p / TK, k = p % TK;
+      ws[i][k] = (i0 + i < g.h && k0 + k < g.d) ? to_f(w1[(lh * g.h + i0 + i) * g.d + k0 + k]) : 0.f;
+    }
+    for (int p = tid; p < TR * TK; p += 256) {
+      const int rr = p / TK, k = p % TK;
+      bs[rr][k] = (r0 + rr < g.r && k0 + k < g.d) ? to_f(basis[(lh * g.r + r0 + rr) * g.d + k0 + k]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int k = 0; k < TK; ++k) {
+      const float a0 = ws[2 * ty][k], a1 = ws[2 * ty + 1][k];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float bv = bs[4 * tx + j][k];
+        acc[0][j] = fmaf(a0, bv, acc[0][j]);
+        acc[1][j] = fmaf(a1, bv, acc[1][j]);
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int ii = 0; ii < 2; ++ii) {
+    const int i = i0 + 2 * ty + ii;
+    if (i >= g.h) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int rr = r0 + 4 * tx + j;
+      if (rr >= g.r) continue;
+      const float a = acc[ii][j];
+      if (w1f_t) w1f_t[(lh * g.r + rr) * g.h + i] = a;
+      // tensor-core copy holds W1'/2: the MMA then yields u = x/2 and silu(x) = u + u*tanh(u)
+      if (w1f_bf16) w1f_bf16[(lh * g.h + i) * g.r + rr] = __float2bfloat16_rn(0.5f * a);
+      if (w1f_f16) w1f_f16[(lh * g.h + i) * g.r + rr] = __float2half_rn(0.5f * a);
+    }
   }
 }
 
@@ -319,18 +351,15 @@ cudaError_t launch_combine(const Geom& g, const CacheBuffers& cb, const Scratch&
 
 cudaError_t launch_fold(const Geom& g, const CacheBuffers& cb, int dtype, int store,
                         float* w1f_t, void* w1f_tc, cudaStream_t s) {
-  const size_t n = (size_t)g.L * g.Hkv * g.h * g.r;
-  const int blocks = (int)((n + 255) / 256 < 65535 * 8 ? (n + 255) / 256 : 65535 * 8);
+  const dim3 grid((g.h + 31) / 32, (g.r + 63) / 64, g.L * g.Hkv);
   if (dtype == LOWRAM_F32) {
-    fold_kernel<float><<<blocks, 256, 0, s>>>(g, static_cast<const float*>(cb.w1),
-                                              static_cast<const float*>(cb.basis), w1f_t,
-                                              nullptr, nullptr);
+    fold_tiled_kernel<float><<<grid, 256, 0, s>>>(g, static_cast<const float*>(cb.w1),
+                                                  static_cast<const float*>(cb.basis), w1f_t, nullptr, nullptr);
   } else {
     __nv_bfloat16* bf = store == LOWRAM_STORE_INT8 ? nullptr : static_cast<__nv_bfloat16*>(w1f_tc);
     __half* hf = store == LOWRAM_STORE_INT8 ? static_cast<__half*>(w1f_tc) : nullptr;
-    fold_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
-        g, static_cast<const __nv_bfloat16*>(cb.w1), static_cast<const __nv_bfloat16*>(cb.basis),
-        w1f_t, bf, hf);
+    fold_tiled_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+        g, static_cast<const __nv_bfloat16*>(cb.w1), static_cast<const __nv_bfloat16*>(cb.basis), w1f_t, bf, hf);
   }
   return cudaGetLastError();
 }
