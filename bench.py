@@ -442,7 +442,8 @@ def run_dense(args, ws, rank, local, cfg_name=DEFAULT_CONFIG):
         "config": {"workload": f"dense_bf16_{cfg.name}_b{B}", "batch": B, "n_layers": cfg.n_layers,
                    "tokens": S_, "kv_heads": cfg.n_kv_heads, "q_heads": cfg.n_q_heads,
                    "head_dim": cfg.head_dim, "dense_cache_gb": round(k.numel() * 4 / 1e9, 2)},
-        "roofline": {"bound": "hbm", "kernel": "dense_kernel", "achieved": round(achieved, 1),
+        "roofline": {"bound": "hbm",
+                     "kernel": "dense_tc_kernel" if cfg.head_dim == 128 else "dense_kernel", "achieved": round(achieved, 1),
                      "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
                      "peak_kind": peak_kind},
         "gpu_launches": steps, "clocks": clk,

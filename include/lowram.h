@@ -242,7 +242,11 @@ int32_t lowram_cache_last_path(const lowram_cache* cache);
  * sequence ("LowRAM Compresses KV Cache Asymmetrically", section "Core Mechanism").
  *   k, v [B][L][Hkv][S][d] bf16, DEVICE, 16-byte aligned;
  *   q, out [L][B][Hq][d] bf16, DEVICE.  All L layers in one call, stream-ordered.
- * Needs head_dim % 8 == 0, head_dim <= 256, Hq/Hkv <= 16; returns EINVAL otherwise. */
+ * Needs head_dim % 8 == 0, head_dim <= 256, Hq/Hkv <= 16; returns EINVAL otherwise.
+ * d = 128 with Hq/Hkv in {1, 2, 4, 8, 16} and a 16-byte aligned q runs on tcgen05 tensor
+ * cores (probabilities rounded to bf16 for the P.V product, fp32 accumulation); other
+ * shapes on CUDA cores (fp32 throughout).  The tensor-core kernel's waits are bounded: if
+ * one runs out (it does not in normal operation) that unit's outputs are written as NaN. */
 lowram_status lowram_dense_decode_attn(int32_t batch, int32_t n_layers, int32_t n_kv_heads,
                                        int32_t n_q_heads, int32_t head_dim, int64_t seq_len,
                                        const void* k, const void* v, const void* q, void* out,
