@@ -221,7 +221,8 @@ lowram_status lowram_cache_bytes(const lowram_cache* cache, lowram_bytes* out);
 /* Device-side consistency check of the index tables (slot map, CSR offsets, record
  * positions, tail lengths) and of the error word left by earlier kernels.  Synchronises
  * `stream`.  Returns ECORRUPT if a table is inconsistent, ETIMEOUT if an earlier kernel
- * reported a bounded wait that ran out, OK otherwise; the error word is cleared. */
+ * reported a bounded wait that ran out, EINVAL if an earlier lowram_cache_append found a
+ * full tail (and dropped that token), OK otherwise; the error word is cleared. */
 lowram_status lowram_cache_validate(lowram_cache* cache, lowram_stream stream);
 
 /* Optional timing hook: when events != NULL, lowram_decode_attn records events[0] before
@@ -235,6 +236,46 @@ int32_t lowram_cache_last_launches(const lowram_cache* cache);
 
 /* Which path the last lowram_decode_attn call on this cache ran (a lowram_path value). */
 int32_t lowram_cache_last_path(const lowram_cache* cache);
+
+/* ------------------------------------------------------------- decode-loop upkeep
+ *
+ * Tokens generated after prefill stay uncompressed in the raw tail (rit.work
+ * "lowram-kv-cache-compression": generated tokens are kept raw).  When every sequence's
+ * tail holds at least one chunk, lowram_cache_repack compresses the oldest chunk of the
+ * tail with the cache's basis and predictor.  The pages name no moment for this; the
+ * library's reading: one chunk of C tokens at a time, encoded by the steps of
+ * lowram_encode below, appended after the existing chunks. */
+
+/* The arrays the cache owns, as a read-only view (DEVICE pointers, layouts of
+ * lowram_cache_src; slot is NULL when nothing is evicted), and its current config.  Valid
+ * until the next lowram_cache_repack or lowram_cache_destroy.  Host only. */
+lowram_status lowram_cache_view(const lowram_cache* cache, lowram_config* cfg, lowram_cache_src* src);
+
+/* Append one decode step's key and value to every (layer, sequence, KV head) tail:
+ *   k_new, v_new [L][B][Hkv][d], the tail's element type (dt; bf16 with STORE_INT8),
+ *   DEVICE, 16-byte aligned.
+ * Writes tail[b][l][h][tail_len[b]] and then adds 1 to tail_len[b].  A sequence whose tail
+ * is full (tail_len[b] == T) is left unchanged and its token dropped; the error word
+ * records it and lowram_cache_validate then returns LOWRAM_EINVAL.  Needs
+ * head_dim * element size to be a multiple of 16 (EUNSUPPORTED otherwise).
+ * Stream-ordered: two small kernels, no allocation, no host synchronisation. */
+lowram_status lowram_cache_append(lowram_cache* cache, const void* k_new, const void* v_new,
+                                  lowram_stream stream);
+
+/* Re-pack the oldest C tail tokens of every (sequence, layer, KV head) into one new chunk.
+ * The new chunk is encoded as lowram_encode encodes a context of C tokens (steps 1-6 below,
+ * with n_resid residual records per (b, l, KV head) for this chunk, 0 <= n_resid <= C),
+ * appended after the existing chunks (slot nL when the cache evicts: a new live chunk),
+ * and the tail shifts down by C (tail_len[b] -= C).  Afterwards n_ctx grows by C and
+ * n_live by 1; residual records are re-laid in unit order (b, l, KV head), a unit's old
+ * records first.
+ * Requires every tail_len[b] >= C (EINVAL otherwise), tail_cap >= chunk, and the shapes
+ * lowram_encode supports (EUNSUPPORTED otherwise).
+ * SYNCHRONOUS and allocating: it reads the tail lengths to the host, allocates the arrays
+ * of the longer cache (device memory peaks at about twice the cache), copies the old arrays
+ * into them, frees the old ones and returns after the stream has finished.  On any error
+ * the cache is left as it was.  Meant to run once every C decode steps. */
+lowram_status lowram_cache_repack(lowram_cache* cache, int32_t n_resid, lowram_stream stream);
 
 /* Dense decode attention over an UNCOMPRESSED bf16 KV cache, the baseline a compressed cache
  * is compared with: every cached token is attended, o_j = softmax_t(q_j . k_t / sqrt(d)) v_t

@@ -25,6 +25,7 @@ __all__ = [
     "lowram_decode_attn_host", "lowram_cache_bytes", "lowram_cache_validate",
     "lowram_cache_set_stage_events", "lowram_cache_last_launches", "lowram_cache_last_path",
     "LowramCache", "config_struct", "lowram_decode_attn_static", "lowram_dense_decode_attn",
+    "lowram_cache_view", "lowram_cache_append", "lowram_cache_repack",
     "lowram_encode",
 ]
 
@@ -91,6 +92,9 @@ def lib() -> ctypes.CDLL:
         "lowram_cache_set_stage_events": (I32, [P, P]),
         "lowram_cache_last_launches": (I32, [P]),
         "lowram_cache_last_path": (I32, [P]),
+        "lowram_cache_view": (I32, [P, ctypes.POINTER(LowramConfigC), ctypes.POINTER(LowramSrcC)]),
+        "lowram_cache_append": (I32, [P, P, P, P]),
+        "lowram_cache_repack": (I32, [P, I32, P]),
         "lowram_decode_attn_static": (I32, [ctypes.POINTER(LowramConfigC), ctypes.POINTER(LowramSrcC),
                                             I32, I32, P, P, P, P]),
         "lowram_dense_decode_attn": (I32, [I32, I32, I32, I32, I32, I64, P, P, P, P, P]),
@@ -257,9 +261,10 @@ def lowram_cache_bytes(handle: int) -> dict:
 
 
 def lowram_cache_validate(handle: int, stream=None) -> int:
-    """Returns the lowram_status (0 = consistent, 5 = corrupt tables, 6 = a wait timed out)."""
+    """Returns the lowram_status (0 = consistent, 1 = an append found a full tail, 5 = corrupt
+    tables, 6 = a wait timed out)."""
     st = int(lib().lowram_cache_validate(handle, _stream(stream)))
-    if st not in (0, 5, 6):
+    if st not in (0, 1, 5, 6):
         _check(st, "lowram_cache_validate")
     return st
 
@@ -282,6 +287,67 @@ def lowram_cache_last_launches(handle: int) -> int:
 
 def lowram_cache_last_path(handle: int) -> int:
     return int(lib().lowram_cache_last_path(handle))
+
+
+def lowram_cache_append(handle: int, k_new, v_new, stream=None) -> None:
+    """Append one decode step's k, v [L][B][Hkv][d] (the tail's dtype, CUDA) to every tail."""
+    _check(lib().lowram_cache_append(handle, _ptr(k_new), _ptr(v_new), _stream(stream)),
+           "lowram_cache_append")
+
+
+def lowram_cache_repack(handle: int, n_resid: int, stream=None) -> None:
+    """Compress the oldest chunk of every tail into a new chunk (synchronous; see lowram.h)."""
+    _check(lib().lowram_cache_repack(handle, int(n_resid), _stream(stream)), "lowram_cache_repack")
+
+
+class _DeviceArray:
+    """A device pointer with a shape, for torch.as_tensor (CUDA array interface, no copy)."""
+
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = {"shape": tuple(int(x) for x in shape), "typestr": typestr,
+                                         "data": (int(ptr), False), "version": 3, "strides": None}
+
+
+def lowram_cache_view(handle: int):
+    """(config dict, arrays dict): the cache's current config and torch tensors aliasing the
+    device arrays it owns (read-only use; valid until the next re-pack or destroy)."""
+    import torch
+    c, src = LowramConfigC(), LowramSrcC()
+    _check(lib().lowram_cache_view(handle, ctypes.byref(c), ctypes.byref(src)), "lowram_cache_view")
+    cfg = {n: int(getattr(c, n)) for n, _ in LowramConfigC._fields_}
+    B, L, G, H, d, r = c.batch, c.n_layers, c.group, c.n_kv_heads, c.head_dim, c.rank
+    h, C, T, nL, nC = c.mlp_hidden, c.chunk, c.tail_cap, c.n_live, c.n_ctx // c.chunk
+    R = int(src.n_records)
+    int8 = c.store == 1
+    dt = torch.float32 if c.dtype == 0 else torch.bfloat16
+    tail_dt = torch.bfloat16 if int8 else dt
+    codes = {torch.int8: "|i1", torch.int16: "<i2", torch.int32: "<i4", torch.float16: "<f2",
+             torch.float32: "<f4"}
+
+    def wrap(ptr, shape, dtype):
+        if not ptr:
+            return None
+        base = torch.int16 if dtype == torch.bfloat16 else dtype
+        t = torch.as_tensor(_DeviceArray(ptr, shape, codes[base]), device="cuda")
+        return t.view(torch.bfloat16) if dtype == torch.bfloat16 else t
+
+    arrays = {
+        "coeff": wrap(src.coeff, (B, L // G, H, nL * C, r), torch.int8 if int8 else dt),
+        "coeff_scale": wrap(src.coeff_scale, (B, L // G, H, nL * C), torch.float16) if int8 else None,
+        "basis": wrap(src.basis, (L, H, r, d), dt),
+        "w1": wrap(src.w1, (L, H, h, d), dt),
+        "w2": wrap(src.w2, (L, H, d, h), dt),
+        "summary": wrap(src.summary, (B, L // G, H, nL, r), dt),
+        "slot": wrap(src.slot, (B, L // G, H, nC), torch.int16),
+        "res_ptr": wrap(src.res_ptr, (B, L, H, nL + 1), torch.int32),
+        "res_pos": wrap(src.res_pos, (R,), torch.int16) if R else torch.empty(0, dtype=torch.int16, device="cuda"),
+        "res_val": wrap(src.res_val, (R, d), torch.int8 if int8 else dt),
+        "res_scale": wrap(src.res_scale, (R,), torch.float16) if (int8 and R) else None,
+        "tail_k": wrap(src.tail_k, (B, L, H, T, d), tail_dt),
+        "tail_v": wrap(src.tail_v, (B, L, H, T, d), tail_dt),
+        "tail_len": wrap(src.tail_len, (B,), torch.int32),
+    }
+    return cfg, arrays
 
 
 def lowram_encode(cfg, n_resid: int, keys, values, basis, w1, w2, stream=None, out=None) -> dict:
@@ -374,6 +440,23 @@ class LowramCache:
                           dtype=torch.int32, device=q.device)
         lowram_select_chunks(self.handle, layer0, n_layers, q, scores, sel, stream)
         return scores, sel
+
+    def append(self, k_new, v_new, stream=None) -> None:
+        """Append one decode step's k, v [L][B][Hkv][d] to every sequence's raw tail."""
+        lowram_cache_append(self.handle, k_new, v_new, stream)
+
+    def repack(self, n_resid: int, stream=None) -> None:
+        """Compress the oldest chunk of every tail (synchronous); the config grows by a chunk."""
+        lowram_cache_repack(self.handle, n_resid, stream)
+        cfg, _ = lowram_cache_view(self.handle)
+        if isinstance(self.cfg, dict):
+            self.cfg = dict(self.cfg, n_ctx=cfg["n_ctx"], n_live=cfg["n_live"])
+        else:
+            self.cfg = cfg
+
+    def view(self):
+        """(config dict, arrays dict) of the cache's own device arrays (see lowram_cache_view)."""
+        return lowram_cache_view(self.handle)
 
     def bytes(self) -> dict:
         return lowram_cache_bytes(self.handle)

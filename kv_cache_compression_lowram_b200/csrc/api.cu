@@ -3,8 +3,10 @@
 #include <cstdio>
 #include <cstring>
 #include <string>
+#include <vector>
 
 #include "lowram_internal.cuh"
+#include "upkeep.cuh"
 
 using namespace lowram;
 
@@ -373,6 +375,224 @@ lowram_status lowram_cache_bytes(const lowram_cache* c, lowram_bytes* out) {
   return LOWRAM_OK;
 }
 
+lowram_status lowram_cache_view(const lowram_cache* c, lowram_config* cfg, lowram_cache_src* src) {
+  if (!c || !cfg || !src) return inval("NULL cache or output");
+  *cfg = c->cfg;
+  src->coeff = c->cb.coeff; src->coeff_scale = c->cb.coeff_scale; src->basis = c->cb.basis;
+  src->w1 = c->cb.w1; src->w2 = c->cb.w2; src->summary = c->cb.summary; src->slot = c->cb.slot;
+  src->res_ptr = c->cb.res_ptr; src->res_pos = c->cb.res_pos; src->res_val = c->cb.res_val;
+  src->res_scale = c->cb.res_scale; src->tail_k = c->cb.tail_k; src->tail_v = c->cb.tail_v;
+  src->tail_len = c->cb.tail_len; src->n_records = c->cb.n_records;
+  return LOWRAM_OK;
+}
+
+lowram_status lowram_cache_append(lowram_cache* c, const void* k_new, const void* v_new, lowram_stream stream) {
+  if (!c) return inval("NULL cache");
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new))
+    return inval("k_new / v_new NULL or not 16-byte aligned");
+  if (c->cfg.tail_cap < 1) return inval("the cache has no tail (tail_cap = 0)");
+  const size_t eb = c->cfg.store == LOWRAM_STORE_INT8 ? 2 : c->s_dt;
+  const size_t row = (size_t)c->cfg.head_dim * eb;
+  if (row % 16) {
+    g_last_error = "append moves 16-byte pieces: head_dim * element size must be a multiple of 16";
+    return LOWRAM_EUNSUPPORTED;
+  }
+  cudaError_t e = launch_append(c->cfg.batch, c->cfg.n_layers, c->cfg.n_kv_heads, c->cfg.tail_cap, (int)row, k_new,
+                                v_new, const_cast<void*>(c->cb.tail_k), const_cast<void*>(c->cb.tail_v),
+                                const_cast<int32_t*>(c->cb.tail_len), c->sc.err, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "append");
+  return LOWRAM_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+// Device allocations of one re-pack; whatever is not handed to the cache is freed on exit.
+struct RepackMem {
+  std::vector<void*> ptrs;
+  ~RepackMem() {
+    for (void* p : ptrs) cudaFree(p);
+  }
+  template <typename P>
+  lowram_status get(P** out, size_t bytes) {
+    void* p = nullptr;
+    cudaError_t e = cudaMalloc(&p, bytes ? bytes : 16);
+    if (e != cudaSuccess) {
+      g_last_error = std::string("cudaMalloc: ") + cudaGetErrorString(e);
+      return LOWRAM_ENOMEM;
+    }
+    ptrs.push_back(p);
+    *out = static_cast<P*>(p);
+    return LOWRAM_OK;
+  }
+  void release(const void* p) {   // the cache owns it from now on
+    for (auto& q : ptrs)
+      if (q == p) q = nullptr;
+  }
+};
+
+// new_p replaces old_p among the cache's allocations (old_p is freed); an array the cache
+// did not hold before (no records at create time) is added.
+void swap_owned(lowram_cache* c, const void* old_p, void* new_p) {
+  if (old_p)
+    for (int i = 0; i < c->n_owned; ++i)
+      if (c->owned[i] == old_p) {
+        cudaFree(c->owned[i]);
+        c->owned[i] = new_p;
+        return;
+      }
+  c->owned[c->n_owned++] = new_p;
+}
+
+}  // namespace
+
+extern "C" {
+
+lowram_status lowram_cache_repack(lowram_cache* c, int32_t n_resid, lowram_stream stream) {
+  if (!c) return inval("NULL cache");
+  const lowram_config f = c->cfg;
+  const int C = f.chunk, T = f.tail_cap;
+  if (n_resid < 0 || n_resid > C) return inval("n_resid must lie in [0, chunk]");
+  if (T < C) return inval("the tail cannot hold a chunk (tail_cap < chunk)");
+  if (c->nC + 1 > kMaxChunks || (long long)f.n_ctx + C >= (1LL << 31)) return inval("the cache is at its chunk limit");
+  // the new chunk is encoded by the encoder kernels: their shapes
+  lowram_config ec = f;
+  ec.n_ctx = C;
+  ec.n_live = 1;
+  Geom ge;
+  lowram_status st = encode_geom(&ec, &ge);
+  if (st != LOWRAM_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t B = f.batch, L = f.n_layers, H = f.n_kv_heads, d = f.head_dim, r = f.rank;
+  const size_t NG = c->NG, nC = c->nC, nL = c->nL, U = B * L * H;
+  const bool i8 = f.store == LOWRAM_STORE_INT8;
+  const size_t sa = i8 ? 1 : 2, tail_row = d * 2, n_new = U * (size_t)n_resid;
+  if ((long long)c->cb.n_records + (long long)n_new + kResPad >= (1LL << 31)) return inval("too many residual records");
+
+  // 1. every tail must hold a chunk
+  std::vector<int32_t> tl(B);
+  cudaError_t e = cudaMemcpyAsync(tl.data(), c->cb.tail_len, B * 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "read tail lengths");
+  for (size_t b = 0; b < B; ++b)
+    if (tl[b] < C || tl[b] > T) return inval("every sequence's tail must hold at least one chunk");
+
+  RepackMem m;
+  // 2. the oldest C tail tokens as dense [B][L][Hkv][C][d] keys and values
+  const void* keys = c->cb.tail_k;
+  const void* vals = c->cb.tail_v;
+  if (T != C) {
+    void *kg = nullptr, *vg = nullptr;
+    if ((st = m.get(&kg, U * C * tail_row)) != LOWRAM_OK || (st = m.get(&vg, U * C * tail_row)) != LOWRAM_OK) return st;
+    e = cudaMemcpy2DAsync(kg, C * tail_row, c->cb.tail_k, (size_t)T * tail_row, C * tail_row, U, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(vg, C * tail_row, c->cb.tail_v, (size_t)T * tail_row, C * tail_row, U, cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "gather the tail's oldest chunk");
+    keys = kg;
+    vals = vg;
+  }
+  // 3. encode it
+  lowram_encode_dst dst{};
+  void* ws = nullptr;
+  uint32_t* err = nullptr;
+  const size_t ws_bytes = encode_workspace_bytes(ge);
+  if ((st = m.get(&dst.coeff, B * NG * H * C * r * sa)) != LOWRAM_OK ||
+      (st = m.get(&dst.summary, B * NG * H * r * 2)) != LOWRAM_OK ||
+      (st = m.get(&dst.res_ptr, U * 2 * 4)) != LOWRAM_OK || (st = m.get(&dst.res_pos, n_new * 2)) != LOWRAM_OK ||
+      (st = m.get(&dst.res_val, n_new * d * sa)) != LOWRAM_OK || (st = m.get(&ws, ws_bytes)) != LOWRAM_OK ||
+      (st = m.get(&err, 16)) != LOWRAM_OK)
+    return st;
+  if (i8 && ((st = m.get(&dst.coeff_scale, B * NG * H * C * 2)) != LOWRAM_OK ||
+             (st = m.get(&dst.res_scale, n_new * 2)) != LOWRAM_OK))
+    return st;
+  if ((e = cudaMemsetAsync(err, 0, 16, s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  e = launch_encode(ge, f.store, n_resid, keys, vals, c->cb.basis, c->cb.w1, c->cb.w2, dst, ws, s);
+  if (e != cudaSuccess) return cuda_fail(e, "encode the new chunk");
+
+  // 4. the arrays of the longer cache: old rows, then the new chunk's, per (b, group, KV head)
+  void *coeff = nullptr, *cscale = nullptr, *summ = nullptr;
+  int16_t* slot = nullptr;
+  int32_t* rptr = nullptr;
+  long long* base = nullptr;
+  if ((st = m.get(&coeff, B * NG * H * (nL + 1) * C * r * sa)) != LOWRAM_OK ||
+      (st = m.get(&summ, B * NG * H * (nL + 1) * r * 2)) != LOWRAM_OK ||
+      (st = m.get(&rptr, U * (nL + 2) * 4)) != LOWRAM_OK || (st = m.get(&base, (U + 1) * 8)) != LOWRAM_OK)
+    return st;
+  if (i8 && (st = m.get(&cscale, B * NG * H * (nL + 1) * C * 2)) != LOWRAM_OK) return st;
+  if (c->cb.slot && (st = m.get(&slot, B * NG * H * (nC + 1) * 2)) != LOWRAM_OK) return st;
+  auto rows2d = [&](void* to, const void* from_old, const void* from_new, size_t old_w, size_t new_w) {
+    cudaError_t x = cudaMemcpy2DAsync(to, old_w + new_w, from_old, old_w, old_w, B * NG * H, cudaMemcpyDeviceToDevice, s);
+    if (x == cudaSuccess && from_new)
+      x = cudaMemcpy2DAsync(static_cast<unsigned char*>(to) + old_w, old_w + new_w, from_new, new_w, new_w, B * NG * H,
+                            cudaMemcpyDeviceToDevice, s);
+    return x;
+  };
+  e = rows2d(coeff, c->cb.coeff, dst.coeff, nL * C * r * sa, C * r * sa);
+  if (e == cudaSuccess && i8) e = rows2d(cscale, c->cb.coeff_scale, dst.coeff_scale, nL * C * 2, C * 2);
+  if (e == cudaSuccess) e = rows2d(summ, c->cb.summary, dst.summary, nL * r * 2, r * 2);
+  if (e == cudaSuccess && slot) {
+    e = rows2d(slot, c->cb.slot, nullptr, nC * 2, 2);
+    if (e == cudaSuccess) e = launch_repack_slot((long long)(B * NG * H), (int)nC, (int)nL, slot, s);
+  }
+  if (e == cudaSuccess) e = launch_repack_scan((int)U, (int)nL, c->cb.res_ptr, dst.res_ptr, base, err, s);
+  long long total = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&total, base + U, 8, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "re-lay the chunk arrays");
+  if (total < 0 || total + kResPad >= (1LL << 31)) return inval("re-packed record count out of range");
+  uint16_t* rpos = nullptr;
+  void* rval = nullptr;
+  __half* rscale = nullptr;
+  if ((st = m.get(&rpos, (size_t)total * 2)) != LOWRAM_OK ||
+      (st = m.get(&rval, ((size_t)total + kResPad) * d * sa)) != LOWRAM_OK)
+    return st;
+  if (i8 && (st = m.get(&rscale, (size_t)total * 2)) != LOWRAM_OK) return st;
+  e = launch_repack_records((int)U, (int)nL, (int)(d * sa), c->cb.n_records, (long long)n_new, c->cb.res_ptr,
+                            c->cb.res_pos, c->cb.res_val, c->cb.res_scale, dst.res_ptr, dst.res_pos, dst.res_val,
+                            static_cast<const __half*>(dst.res_scale), base, rptr, rpos, rval, rscale, err, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(static_cast<unsigned char*>(rval) + (size_t)total * d * sa, 0, kResPad * d * sa, s);
+  uint32_t word = 0, enc_word = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&word, err, 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&enc_word, encode_error_word(ge, ws), 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  word |= enc_word;
+  if (e != cudaSuccess) return cuda_fail(e, "re-lay the residual records");
+  if (word & ERR_RES_PTR) {
+    g_last_error = "the cache's CSR offsets are inconsistent: nothing re-packed";
+    return LOWRAM_ECORRUPT;
+  }
+  if (word & ERR_TIMEOUT) {
+    g_last_error = "the encoder gave up a bounded wait: nothing re-packed";
+    return LOWRAM_ETIMEOUT;
+  }
+  if (c->n_owned + 4 > (int)(sizeof(c->owned) / sizeof(c->owned[0]))) return inval("internal: too many owned allocations");
+  // 5. the tail drops its oldest chunk (the last step: the cache is unchanged until here)
+  e = launch_tail_shift((int)B, (int)L, (int)H, T, C, (int)tail_row, const_cast<void*>(c->cb.tail_k),
+                        const_cast<void*>(c->cb.tail_v), const_cast<int32_t*>(c->cb.tail_len), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "shift the tail");
+  // 6. the cache takes the new arrays
+  auto take = [&](const void* old_p, void* new_p) {
+    m.release(new_p);
+    swap_owned(c, old_p, new_p);
+  };
+  take(c->cb.coeff, coeff); c->cb.coeff = coeff;
+  if (i8) { take(c->cb.coeff_scale, cscale); c->cb.coeff_scale = static_cast<const __half*>(cscale); }
+  take(c->cb.summary, summ); c->cb.summary = summ;
+  if (slot) { take(c->cb.slot, slot); c->cb.slot = slot; }
+  take(c->cb.res_ptr, rptr); c->cb.res_ptr = rptr;
+  take(c->cb.res_pos, rpos); c->cb.res_pos = rpos;
+  take(c->cb.res_val, rval); c->cb.res_val = rval;
+  if (i8) { take(c->cb.res_scale, rscale); c->cb.res_scale = rscale; }
+  c->cb.n_records = total;
+  c->cfg.n_ctx += C;
+  c->cfg.n_live += 1;
+  c->nC += 1;
+  c->nL += 1;
+  return LOWRAM_OK;
+}
+
 lowram_status lowram_cache_set_stage_events(lowram_cache* c, void* const* events) {
   if (!c) return inval("NULL cache");
   if (!events) {
@@ -500,6 +720,10 @@ lowram_status lowram_cache_validate(lowram_cache* c, lowram_stream stream) {
   if (word & ERR_TIMEOUT) {
     g_last_error = "a kernel gave up a bounded wait";
     return LOWRAM_ETIMEOUT;
+  }
+  if (word & ERR_TAIL_FULL) {
+    g_last_error = "an append found a full tail: that sequence's token was dropped";
+    return LOWRAM_EINVAL;
   }
   return LOWRAM_OK;
 }

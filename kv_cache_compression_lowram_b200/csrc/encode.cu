@@ -25,6 +25,7 @@
 #include <cuda_fp16.h>
 
 #include "lowram_internal.cuh"
+#include "upkeep.cuh"
 #include "tc_ptx.cuh"
 
 namespace lowram {
@@ -1015,6 +1016,11 @@ size_t encode_workspace_bytes(const Geom& g) {
   size_t bytes = 0;
   carve(g, nullptr, &bytes);
   return bytes;
+}
+
+uint32_t* encode_error_word(const Geom& g, void* workspace) {
+  size_t bytes = 0;
+  return carve(g, workspace, &bytes).err;
 }
 
 cudaError_t launch_encode(const Geom& g, int store, int n_res, const void* keys, const void* values,

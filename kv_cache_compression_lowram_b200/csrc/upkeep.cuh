@@ -1,0 +1,31 @@
+// Internal declarations of the decode-loop upkeep of a cache (repack.cu): tail append,
+// residual-record re-layout and tail shift after a re-pack.  Not part of the C ABI.
+#pragma once
+
+#include "lowram_internal.cuh"
+
+namespace lowram {
+
+// Error-word bit of the upkeep kernels (next to the ERR_* bits of lowram_internal.cuh).
+constexpr uint32_t ERR_TAIL_FULL = 1u << 6;   // an append found a full tail: token dropped
+
+// The error word inside an encoder workspace (encode.cu): bounded-wait timeouts of the
+// encoder's tensor-core kernels.
+uint32_t* encode_error_word(const Geom& g, void* workspace);
+
+// row_bytes: bytes of one tail row / record row, a multiple of 16.
+cudaError_t launch_append(int B, int L, int Hkv, int T, int row_bytes, const void* k_new, const void* v_new,
+                          void* tail_k, void* tail_v, int32_t* tail_len, uint32_t* err, cudaStream_t s);
+cudaError_t launch_repack_scan(int U, int nL, const int32_t* old_ptr, const int32_t* new_ptr, long long* base,
+                               uint32_t* err, cudaStream_t s);
+cudaError_t launch_repack_records(int U, int nL, int row_bytes, long long n_old, long long n_new_total,
+                                  const int32_t* old_ptr, const uint16_t* old_pos, const void* old_val,
+                                  const __half* old_scale, const int32_t* new_ptr, const uint16_t* new_pos,
+                                  const void* new_val, const __half* new_scale, const long long* base,
+                                  int32_t* out_ptr, uint16_t* out_pos, void* out_val, __half* out_scale,
+                                  uint32_t* err, cudaStream_t s);
+cudaError_t launch_repack_slot(long long rows, int nC, int nL, int16_t* slot, cudaStream_t s);
+cudaError_t launch_tail_shift(int B, int L, int Hkv, int T, int C, int row_bytes, void* tail_k, void* tail_v,
+                              int32_t* tail_len, cudaStream_t s);
+
+}  // namespace lowram

@@ -117,3 +117,12 @@ def test_encode_host_checks():
     st = K.lib().lowram_encode(ctypes.byref(c), 4, None, None, None, None, None, ctypes.byref(dst),
                                None, 0, None)
     assert st == 1
+
+
+def test_upkeep_host_checks():
+    """Cache view, append and re-pack reject a NULL cache before touching the device."""
+    lib = K.lib()
+    cfg, src = K.LowramConfigC(), K.LowramSrcC()
+    assert lib.lowram_cache_view(None, ctypes.byref(cfg), ctypes.byref(src)) == 1
+    assert lib.lowram_cache_append(None, None, None, None) == 1
+    assert lib.lowram_cache_repack(None, 4, None) == 1
