@@ -51,6 +51,8 @@ def parse():
                     help="only the uncompressed bf16 dense-KV baseline at its largest batch")
     ap.add_argument("--encode", action="store_true",
                     help="only the prefill-side encoder (dense K, V -> compressed cache) of the workload")
+    ap.add_argument("--repack", action="store_true",
+                    help="only the decode-loop upkeep: C tail appends and one chunk re-pack per step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -558,6 +560,137 @@ def run_encode(args, ws, rank, local):
     }
 
 
+REPACK_METRIC = "chunk re-packs/s (the oldest C tail tokens of every sequence, layer and KV head -> one compressed chunk)"
+
+
+def repack_oracle_rate(cfg, n_res: int, budget_s: float = 20.0):
+    """The re-pack oracle on one-sequence, one-layer-group slices of the workload (all KV
+    heads) until the budget is spent; returns (re-packs/s scaled to the whole workload by the
+    unit count, sample description, threads)."""
+    import oracle.repack as RP
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = 1
+    sub = cfg.replace(name=cfg.name + "_slice", batch=1, n_layers=cfg.group)
+    npc = S.cache_to_numpy(S.make_cache(sub, device="cuda" if torch.cuda.is_available() else "cpu",
+                                        tail_len=[cfg.chunk]))
+    done, t0 = 0, time.perf_counter()
+    while True:
+        RP.repack(npc, n_res)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    share = (sub.batch * sub.n_layers) / (cfg.batch * cfg.n_layers)
+    return done * share / dt, f"{done} re-packs of a (1 sequence, {cfg.group} layers, {cfg.n_kv_heads} KV heads) slice, {dt:.1f} s", threads
+
+
+def run_repack(args, ws, rank, local):
+    """Decode-loop upkeep on the workload: one step = C appends of a decode token to every
+    tail and one re-pack of the full tails into a new chunk (the cache grows a chunk per step)."""
+    import kv_cache_compression_lowram_b200 as K
+    cfg = replica_config(S.CONFIGS[args.config], rank)
+    C, T = cfg.chunk, cfg.tail_cap
+    assert T >= C, "the workload's tail cannot hold a chunk"
+    dev = torch.device("cuda", local)
+    n_res = max(1, int(round(cfg.resid_frac * C)))
+    cache = S.make_cache(cfg, device=dev, tail_len=[C] * cfg.batch)
+    lc = K.LowramCache.from_synth(cache)
+    del cache
+    torch.cuda.synchronize()
+    shape = (cfg.n_layers, cfg.batch, cfg.n_kv_heads, cfg.head_dim)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(cfg.seed + 31 + rank)
+    kv_dev = [((torch.randn(shape, generator=gen, device=dev) * 0.3).to(torch.bfloat16),
+               (torch.randn(shape, generator=gen, device=dev) * 0.1).to(torch.bfloat16)) for _ in range(C)]
+    kv_host = [(k.cpu().pin_memory(), v.cpu().pin_memory()) for k, v in kv_dev[:8]]
+    stream = torch.cuda.current_stream()
+
+    def upkeep_bytes():
+        b = lc.bytes()
+        return b["coeff"] + b["summary"] + b["residual"] + b["index"]
+
+    def step(host: bool):
+        lc.repack(n_res)
+        for i in range(C):
+            if host:   # end to end: the step's k, v arrive from pinned host memory
+                k, v = kv_host[i % len(kv_host)]
+                kd, vd = kv_dev[i]
+                kd.copy_(k, non_blocking=True)
+                vd.copy_(v, non_blocking=True)
+                lc.append(kd, vd)
+            else:
+                lc.append(*kv_dev[i])
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 10))
+    clocks = ClockSampler(local)
+    barrier(ws)
+    clocks.start()
+    time.sleep(0.3)
+    rp_ms, ap_ms, moved = [], [], []
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    t_all = time.perf_counter()
+    for _ in range(steps):
+        before = upkeep_bytes()
+        ev[0].record(stream)
+        lc.repack(n_res)                         # synchronous
+        ev[1].record(stream)
+        for i in range(C):
+            lc.append(*kv_dev[i])
+        ev[2].record(stream)
+        torch.cuda.synchronize()
+        after = upkeep_bytes()
+        rp_ms.append(ev[0].elapsed_time(ev[1]))
+        ap_ms.append(ev[1].elapsed_time(ev[2]))
+        U = cfg.batch * cfg.n_layers * cfg.n_kv_heads
+        # the re-laid arrays read and written once, the tail's oldest chunk read by the encoder
+        moved.append(before + after + 2 * U * C * cfg.head_dim * 2)
+    wall_ms = (time.perf_counter() - t_all) * 1e3
+    clk = clocks.stop()
+    ms_step = max_over_ranks(sum(rp_ms) / steps + sum(ap_ms) / steps, ws)
+    value = _reduce(1.0, ws, "sum") / (ms_step / 1e3)
+    ms_repack = sum(rp_ms) / steps
+    achieved = (sum(moved) / steps) / (ms_repack / 1e3) / 1e9
+    peak, peak_kind = peaks()
+    # end to end: the appended tokens come from pinned host memory, timed on the host
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    for _ in range(3):
+        step(True)
+    torch.cuda.synchronize()
+    e2e_ms = (time.perf_counter() - t0) * 1e3 / 3
+    h2d = C * 2 * cfg.n_layers * cfg.batch * cfg.n_kv_heads * cfg.head_dim * 2
+    d2h = cfg.batch * 4 + 8 + 8        # tail lengths, the record total, two error words
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        rate, sample, threads = repack_oracle_rate(cfg, n_res)
+        cpu = {"value": round(rate, 4), "unit": "re-packs/s", "cores": threads, "kind": "oracle", "sample": sample}
+    cfg_now, _ = lc.view()
+    lc.close()
+    return {
+        "metric": REPACK_METRIC, "value": round(value, 2), "unit": "re-packs/s", "n_gpus": ws, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "upkeep",
+        "config": {"workload": cfg.name, "batch": cfg.batch, "n_layers": cfg.n_layers, "n_ctx_start": cfg.n_ctx,
+                   "n_ctx_end": cfg_now["n_ctx"], "chunk": C, "n_resid_per_chunk": n_res, "store": cfg.store,
+                   "step": f"1 re-pack + {C} appends", "l2": "inputs larger than L2"},
+        "ms_per_repack": round(ms_repack, 3), "us_per_append": round(1e3 * sum(ap_ms) / steps / C, 2),
+        "repack_us_per_decode_step": round(1e3 * ms_repack / C, 2), "wall_ms_timed_region": round(wall_ms, 1),
+        "roofline": {"bound": "hbm", "kernel": "re-pack (whole synchronous call: encoder, copies, allocation)",
+                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": None, "bytes_per_repack": int(sum(moved) / steps), "peak_kind": peak_kind},
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(1e3 / e2e_ms, 2), "unit": "re-packs/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": steps * (2 * C + 12), "clocks": clk,
+    }
+
+
 def run_reference(args, ws, rank):
     """The oracle (fp64 numpy, host cores) on the same workload, bounded samples per step."""
     if rank != 0:
@@ -600,11 +733,13 @@ def main():
         line = run_dense(args, ws, rank, local)
     elif args.encode:
         line = run_encode(args, ws, rank, local)
+    elif args.repack:
+        line = run_repack(args, ws, rank, local)
     else:
         line = run_lowram(args, ws, rank, local)
     if rank == 0 and line is not None:
         print(json.dumps(line), flush=True)
-    if args.sweep and args.impl == "lowram" and not args.dense and not args.encode:
+    if args.sweep and args.impl == "lowram" and not (args.dense or args.encode or args.repack):
         import gc
         for b in (1, 4, 16, 32, 64):
             args.config = f"llama8b_32k_bf16_b{b}"
