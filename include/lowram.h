@@ -246,10 +246,16 @@ int32_t lowram_cache_last_path(const lowram_cache* cache);
  * library's reading: one chunk of C tokens at a time, encoded by the steps of
  * lowram_encode below, appended after the existing chunks. */
 
-/* The arrays the cache owns, as a read-only view (DEVICE pointers, layouts of
- * lowram_cache_src; slot is NULL when nothing is evicted), and its current config.  Valid
- * until the next lowram_cache_repack or lowram_cache_destroy.  Host only. */
-lowram_status lowram_cache_view(const lowram_cache* cache, lowram_config* cfg, lowram_cache_src* src);
+/* The arrays the cache owns, as a read-only view (DEVICE pointers; slot is NULL when
+ * nothing is evicted), and its current config.  Layouts are those of lowram_cache_src except
+ * that each (b, group, KV head) / (b, l, KV head) keeps room for *spare_chunks more chunks:
+ * unit strides of (nL + S) * C coefficient rows (and scales), nL + S summaries, nL + S + 1
+ * CSR offsets and nC + S slot entries, S = *spare_chunks (0 until a re-pack adds room).
+ * After a re-pack the records of each unit are followed by spare record rows, so n_records
+ * counts allocated rows, not live records.  Valid until the next lowram_cache_repack or
+ * lowram_cache_destroy.  Host only. */
+lowram_status lowram_cache_view(const lowram_cache* cache, lowram_config* cfg, lowram_cache_src* src,
+                                int32_t* spare_chunks);
 
 /* Append one decode step's key and value to every (layer, sequence, KV head) tail:
  *   k_new, v_new [L][B][Hkv][d], the tail's element type (dt; bf16 with STORE_INT8),
@@ -271,10 +277,14 @@ lowram_status lowram_cache_append(lowram_cache* cache, const void* k_new, const 
  * records first.
  * Requires every tail_len[b] >= C (EINVAL otherwise), tail_cap >= chunk, and the shapes
  * lowram_encode supports (EUNSUPPORTED otherwise).
- * SYNCHRONOUS and allocating: it reads the tail lengths to the host, allocates the arrays
- * of the longer cache (device memory peaks at about twice the cache), copies the old arrays
- * into them, frees the old ones and returns after the stream has finished.  On any error
- * the cache is left as it was.  Meant to run once every C decode steps. */
+ * SYNCHRONOUS: it reads the tail lengths to the host and returns after the stream has
+ * finished.  When the cache has room for one more chunk per unit (and for the new records
+ * after each unit's last ones), the new chunk is written in place; otherwise the arrays are
+ * re-laid into new allocations with room for max(4, nL / 16) more chunks per unit and as
+ * many spare records per unit as this call keeps per chunk (device memory peaks at about
+ * twice the cache during that copy; the old arrays are freed).  A cache created from
+ * caller arrays gets its room at its first re-pack.  On any error the cache is left as it
+ * was.  Meant to run once every C decode steps. */
 lowram_status lowram_cache_repack(lowram_cache* cache, int32_t n_resid, lowram_stream stream);
 
 /* Dense decode attention over an UNCOMPRESSED bf16 KV cache, the baseline a compressed cache

@@ -92,7 +92,8 @@ def lib() -> ctypes.CDLL:
         "lowram_cache_set_stage_events": (I32, [P, P]),
         "lowram_cache_last_launches": (I32, [P]),
         "lowram_cache_last_path": (I32, [P]),
-        "lowram_cache_view": (I32, [P, ctypes.POINTER(LowramConfigC), ctypes.POINTER(LowramSrcC)]),
+        "lowram_cache_view": (I32, [P, ctypes.POINTER(LowramConfigC), ctypes.POINTER(LowramSrcC),
+                                    ctypes.POINTER(I32)]),
         "lowram_cache_append": (I32, [P, P, P, P]),
         "lowram_cache_repack": (I32, [P, I32, P]),
         "lowram_decode_attn_static": (I32, [ctypes.POINTER(LowramConfigC), ctypes.POINTER(LowramSrcC),
@@ -310,11 +311,15 @@ class _DeviceArray:
 
 def lowram_cache_view(handle: int):
     """(config dict, arrays dict): the cache's current config and torch tensors aliasing the
-    device arrays it owns (read-only use; valid until the next re-pack or destroy)."""
+    device arrays it owns (read-only use; valid until the next re-pack or destroy).  The
+    chunk arrays are strided views of their live part (the cache keeps room for more chunks
+    after a re-pack: ``cfg["spare_chunks"]``); records may have spare rows between units."""
     import torch
-    c, src = LowramConfigC(), LowramSrcC()
-    _check(lib().lowram_cache_view(handle, ctypes.byref(c), ctypes.byref(src)), "lowram_cache_view")
+    c, src, spare = LowramConfigC(), LowramSrcC(), ctypes.c_int32()
+    _check(lib().lowram_cache_view(handle, ctypes.byref(c), ctypes.byref(src), ctypes.byref(spare)),
+           "lowram_cache_view")
     cfg = {n: int(getattr(c, n)) for n, _ in LowramConfigC._fields_}
+    cfg["spare_chunks"] = S_ = int(spare.value)
     B, L, G, H, d, r = c.batch, c.n_layers, c.group, c.n_kv_heads, c.head_dim, c.rank
     h, C, T, nL, nC = c.mlp_hidden, c.chunk, c.tail_cap, c.n_live, c.n_ctx // c.chunk
     R = int(src.n_records)
@@ -331,15 +336,19 @@ def lowram_cache_view(handle: int):
         t = torch.as_tensor(_DeviceArray(ptr, shape, codes[base]), device="cuda")
         return t.view(torch.bfloat16) if dtype == torch.bfloat16 else t
 
+    def live(t, n):   # the first n entries along the unit's axis
+        return None if t is None else t[:, :, :, :n]
+
     arrays = {
-        "coeff": wrap(src.coeff, (B, L // G, H, nL * C, r), torch.int8 if int8 else dt),
-        "coeff_scale": wrap(src.coeff_scale, (B, L // G, H, nL * C), torch.float16) if int8 else None,
+        "coeff": live(wrap(src.coeff, (B, L // G, H, (nL + S_) * C, r), torch.int8 if int8 else dt), nL * C),
+        "coeff_scale": live(wrap(src.coeff_scale, (B, L // G, H, (nL + S_) * C), torch.float16), nL * C)
+        if int8 else None,
         "basis": wrap(src.basis, (L, H, r, d), dt),
         "w1": wrap(src.w1, (L, H, h, d), dt),
         "w2": wrap(src.w2, (L, H, d, h), dt),
-        "summary": wrap(src.summary, (B, L // G, H, nL, r), dt),
-        "slot": wrap(src.slot, (B, L // G, H, nC), torch.int16),
-        "res_ptr": wrap(src.res_ptr, (B, L, H, nL + 1), torch.int32),
+        "summary": live(wrap(src.summary, (B, L // G, H, nL + S_, r), dt), nL),
+        "slot": live(wrap(src.slot, (B, L // G, H, nC + S_), torch.int16), nC),
+        "res_ptr": live(wrap(src.res_ptr, (B, L, H, nL + S_ + 1), torch.int32), nL + 1),
         "res_pos": wrap(src.res_pos, (R,), torch.int16) if R else torch.empty(0, dtype=torch.int16, device="cuda"),
         "res_val": wrap(src.res_val, (R, d), torch.int8 if int8 else dt),
         "res_scale": wrap(src.res_scale, (R,), torch.float16) if (int8 and R) else None,

@@ -1,4 +1,5 @@
 // C ABI of the LowRAM decode library: cache object, argument checks, launches.
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -13,6 +14,11 @@ using namespace lowram;
 struct lowram_cache {
   lowram_config cfg;
   int nC, nL, NG, g, device, n_sm;
+  int nLs, nCs;                // per-unit capacity (strides) in live slots / chunk ids
+  bool canonical;              // records laid out unit by unit in unit order, with slack
+  bool last_repack_in_place;
+  void* up_mem;                // re-pack scratch (encoder inputs, outputs and workspace), kept
+  size_t up_bytes;
   size_t s_dt;                 // bytes of one dt element
   void* owned[48];             // every device allocation the cache owns
   int n_owned;
@@ -98,6 +104,7 @@ Geom make_geom(const lowram_cache* c, int layer0, int n_layers, bool tc) {
   g.B = f.batch; g.L = f.n_layers; g.G = f.group; g.Hkv = f.n_kv_heads; g.Hq = f.n_q_heads;
   g.g = f.n_q_heads / f.n_kv_heads; g.d = f.head_dim; g.r = f.rank; g.h = f.mlp_hidden;
   g.N = f.n_ctx; g.C = f.chunk; g.nC = c->nC; g.nL = c->nL; g.k = f.top_k; g.T = f.tail_cap;
+  g.nLs = c->nLs; g.nCs = c->nCs;
   g.layer0 = layer0; g.n_layers = n_layers;
   g.U = n_layers * g.Hkv * g.B;
   const long long total = (long long)g.U * g.k;
@@ -195,6 +202,7 @@ lowram_status encode_geom(const lowram_config* cfg, Geom* g) {
   g->B = c->batch; g->L = c->n_layers; g->G = c->group; g->Hkv = c->n_kv_heads; g->Hq = c->n_q_heads;
   g->g = c->n_q_heads / c->n_kv_heads; g->d = c->head_dim; g->r = c->rank; g->h = c->mlp_hidden;
   g->N = c->n_ctx; g->C = c->chunk; g->nC = nC; g->nL = nC; g->k = c->top_k; g->T = c->tail_cap;
+  g->nLs = nC; g->nCs = nC;
   g->layer0 = 0; g->n_layers = c->n_layers;
   return LOWRAM_OK;
 }
@@ -268,6 +276,8 @@ lowram_status lowram_cache_create(const lowram_config* cfg, const lowram_cache_s
   std::memset(c, 0, sizeof(*c));
   c->cfg = *cfg;
   c->nC = nC; c->nL = cfg->n_live; c->NG = cfg->n_layers / cfg->group;
+  c->nLs = c->nL; c->nCs = nC; c->canonical = false; c->last_repack_in_place = false;
+  c->up_mem = nullptr; c->up_bytes = 0;
   c->g = cfg->n_q_heads / cfg->n_kv_heads;
   c->device = dev; c->n_sm = n_sm;
   c->s_dt = cfg->dtype == LOWRAM_F32 ? 4 : 2;
@@ -366,6 +376,7 @@ void lowram_cache_destroy(lowram_cache* c) {
   if (!c) return;
   cudaDeviceSynchronize();
   for (int i = 0; i < c->n_owned; ++i) cudaFree(c->owned[i]);
+  if (c->up_mem) cudaFree(c->up_mem);
   delete c;
 }
 
@@ -375,8 +386,10 @@ lowram_status lowram_cache_bytes(const lowram_cache* c, lowram_bytes* out) {
   return LOWRAM_OK;
 }
 
-lowram_status lowram_cache_view(const lowram_cache* c, lowram_config* cfg, lowram_cache_src* src) {
-  if (!c || !cfg || !src) return inval("NULL cache or output");
+lowram_status lowram_cache_view(const lowram_cache* c, lowram_config* cfg, lowram_cache_src* src,
+                                int32_t* spare_chunks) {
+  if (!c || !cfg || !src || !spare_chunks) return inval("NULL cache or output");
+  *spare_chunks = c->nLs - c->nL;
   *cfg = c->cfg;
   src->coeff = c->cb.coeff; src->coeff_scale = c->cb.coeff_scale; src->basis = c->cb.basis;
   src->w1 = c->cb.w1; src->w2 = c->cb.w2; src->summary = c->cb.summary; src->slot = c->cb.slot;
@@ -445,6 +458,38 @@ void swap_owned(lowram_cache* c, const void* old_p, void* new_p) {
   c->owned[c->n_owned++] = new_p;
 }
 
+// The re-pack scratch, carved from one allocation (256-byte aligned pieces): the error
+// words, the gathered tail chunk (when T > C), the encoder's outputs and its workspace.
+struct UpScratch {
+  uint32_t* err;
+  void* kg;
+  void* vg;
+  lowram_encode_dst dst;
+  void* ws;
+};
+
+size_t carve_up(void* base, size_t gather, size_t coeff, size_t cscale, size_t summ, size_t rptr, size_t rpos,
+                size_t rval, size_t rscale, size_t ws, UpScratch* o) {
+  size_t off = 0;
+  auto take = [&](size_t n) -> void* {
+    void* p = base ? static_cast<unsigned char*>(base) + off : nullptr;
+    off += (n + 255) & ~size_t(255);
+    return n ? p : nullptr;
+  };
+  o->err = static_cast<uint32_t*>(take(16));
+  o->kg = take(gather);
+  o->vg = take(gather);
+  o->dst.coeff = take(coeff);
+  o->dst.coeff_scale = take(cscale);
+  o->dst.summary = take(summ);
+  o->dst.res_ptr = static_cast<int32_t*>(take(rptr));
+  o->dst.res_pos = static_cast<uint16_t*>(take(rpos));
+  o->dst.res_val = take(rval);
+  o->dst.res_scale = take(rscale);
+  o->ws = take(ws);
+  return off;
+}
+
 }  // namespace
 
 extern "C" {
@@ -466,25 +511,53 @@ lowram_status lowram_cache_repack(lowram_cache* c, int32_t n_resid, lowram_strea
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t B = f.batch, L = f.n_layers, H = f.n_kv_heads, d = f.head_dim, r = f.rank;
   const size_t NG = c->NG, nC = c->nC, nL = c->nL, U = B * L * H;
+  const size_t nLs = c->nLs, nCs = c->nCs;
   const bool i8 = f.store == LOWRAM_STORE_INT8;
   const size_t sa = i8 ? 1 : 2, tail_row = d * 2, n_new = U * (size_t)n_resid;
-  if ((long long)c->cb.n_records + (long long)n_new + kResPad >= (1LL << 31)) return inval("too many residual records");
 
-  // 1. every tail must hold a chunk
+  RepackMem m;
+  // scratch kept by the cache between re-packs (grown when this call needs more)
+  UpScratch up;
+  auto carve = [&](void* base) {
+    return carve_up(base, T != C ? U * C * tail_row : 0, B * NG * H * C * r * sa, i8 ? B * NG * H * C * 2 : 0,
+                    B * NG * H * r * 2, U * 2 * 4, n_new * 2, n_new * d * sa, i8 ? n_new * 2 : 0,
+                    encode_workspace_bytes(ge), &up);
+  };
+  const size_t up_need = carve(nullptr);
+  if (up_need > c->up_bytes) {
+    if (c->up_mem) cudaFree(c->up_mem);
+    c->up_mem = nullptr;
+    c->up_bytes = 0;
+    cudaError_t ea = cudaMalloc(&c->up_mem, up_need);
+    if (ea != cudaSuccess) {
+      c->up_mem = nullptr;
+      g_last_error = std::string("cudaMalloc: ") + cudaGetErrorString(ea);
+      return LOWRAM_ENOMEM;
+    }
+    c->up_bytes = up_need;
+  }
+  carve(c->up_mem);
+  uint32_t* err = up.err;
+  cudaError_t e = cudaMemsetAsync(err, 0, 16, s);
+  // 1. every tail must hold a chunk; room for the chunk in place?
+  const bool room_slots = c->canonical && nL + 1 <= nLs && nC + 1 <= nCs;
+  if (e == cudaSuccess && room_slots)
+    e = launch_repack_room((int)U, (int)nL, (int)nLs, n_resid, c->cb.res_ptr, c->cb.n_records, err + 1, s);
   std::vector<int32_t> tl(B);
-  cudaError_t e = cudaMemcpyAsync(tl.data(), c->cb.tail_len, B * 4, cudaMemcpyDeviceToHost, s);
+  uint32_t no_room = 0;
+  if (e == cudaSuccess) e = cudaMemcpyAsync(tl.data(), c->cb.tail_len, B * 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&no_room, err + 1, 4, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "read tail lengths");
   for (size_t b = 0; b < B; ++b)
     if (tl[b] < C || tl[b] > T) return inval("every sequence's tail must hold at least one chunk");
+  const bool in_place = room_slots && !no_room;
 
-  RepackMem m;
   // 2. the oldest C tail tokens as dense [B][L][Hkv][C][d] keys and values
   const void* keys = c->cb.tail_k;
   const void* vals = c->cb.tail_v;
   if (T != C) {
-    void *kg = nullptr, *vg = nullptr;
-    if ((st = m.get(&kg, U * C * tail_row)) != LOWRAM_OK || (st = m.get(&vg, U * C * tail_row)) != LOWRAM_OK) return st;
+    void *kg = up.kg, *vg = up.vg;
     e = cudaMemcpy2DAsync(kg, C * tail_row, c->cb.tail_k, (size_t)T * tail_row, C * tail_row, U, cudaMemcpyDeviceToDevice, s);
     if (e == cudaSuccess)
       e = cudaMemcpy2DAsync(vg, C * tail_row, c->cb.tail_v, (size_t)T * tail_row, C * tail_row, U, cudaMemcpyDeviceToDevice, s);
@@ -493,71 +566,92 @@ lowram_status lowram_cache_repack(lowram_cache* c, int32_t n_resid, lowram_strea
     vals = vg;
   }
   // 3. encode it
-  lowram_encode_dst dst{};
-  void* ws = nullptr;
-  uint32_t* err = nullptr;
-  const size_t ws_bytes = encode_workspace_bytes(ge);
-  if ((st = m.get(&dst.coeff, B * NG * H * C * r * sa)) != LOWRAM_OK ||
-      (st = m.get(&dst.summary, B * NG * H * r * 2)) != LOWRAM_OK ||
-      (st = m.get(&dst.res_ptr, U * 2 * 4)) != LOWRAM_OK || (st = m.get(&dst.res_pos, n_new * 2)) != LOWRAM_OK ||
-      (st = m.get(&dst.res_val, n_new * d * sa)) != LOWRAM_OK || (st = m.get(&ws, ws_bytes)) != LOWRAM_OK ||
-      (st = m.get(&err, 16)) != LOWRAM_OK)
-    return st;
-  if (i8 && ((st = m.get(&dst.coeff_scale, B * NG * H * C * 2)) != LOWRAM_OK ||
-             (st = m.get(&dst.res_scale, n_new * 2)) != LOWRAM_OK))
-    return st;
-  if ((e = cudaMemsetAsync(err, 0, 16, s)) != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  const lowram_encode_dst dst = up.dst;
+  void* ws = up.ws;
   e = launch_encode(ge, f.store, n_resid, keys, vals, c->cb.basis, c->cb.w1, c->cb.w2, dst, ws, s);
   if (e != cudaSuccess) return cuda_fail(e, "encode the new chunk");
 
-  // 4. the arrays of the longer cache: old rows, then the new chunk's, per (b, group, KV head)
-  void *coeff = nullptr, *cscale = nullptr, *summ = nullptr;
+  // 2-D copy of B*NG*H rows: `width` bytes from `from` (pitch spitch) to `to` (pitch dpitch)
+  auto rows2d = [&](void* to, size_t dpitch, const void* from, size_t spitch, size_t width) {
+    return cudaMemcpy2DAsync(to, dpitch, from, spitch, width, B * NG * H, cudaMemcpyDeviceToDevice, s);
+  };
+  auto at = [](const void* p, size_t off) { return static_cast<unsigned char*>(const_cast<void*>(p)) + off; };
+  long long total = c->cb.n_records;
+  void *coeff = nullptr, *cscale = nullptr, *summ = nullptr, *rval = nullptr;
   int16_t* slot = nullptr;
   int32_t* rptr = nullptr;
-  long long* base = nullptr;
-  if ((st = m.get(&coeff, B * NG * H * (nL + 1) * C * r * sa)) != LOWRAM_OK ||
-      (st = m.get(&summ, B * NG * H * (nL + 1) * r * 2)) != LOWRAM_OK ||
-      (st = m.get(&rptr, U * (nL + 2) * 4)) != LOWRAM_OK || (st = m.get(&base, (U + 1) * 8)) != LOWRAM_OK)
-    return st;
-  if (i8 && (st = m.get(&cscale, B * NG * H * (nL + 1) * C * 2)) != LOWRAM_OK) return st;
-  if (c->cb.slot && (st = m.get(&slot, B * NG * H * (nC + 1) * 2)) != LOWRAM_OK) return st;
-  auto rows2d = [&](void* to, const void* from_old, const void* from_new, size_t old_w, size_t new_w) {
-    cudaError_t x = cudaMemcpy2DAsync(to, old_w + new_w, from_old, old_w, old_w, B * NG * H, cudaMemcpyDeviceToDevice, s);
-    if (x == cudaSuccess && from_new)
-      x = cudaMemcpy2DAsync(static_cast<unsigned char*>(to) + old_w, old_w + new_w, from_new, new_w, new_w, B * NG * H,
-                            cudaMemcpyDeviceToDevice, s);
-    return x;
-  };
-  e = rows2d(coeff, c->cb.coeff, dst.coeff, nL * C * r * sa, C * r * sa);
-  if (e == cudaSuccess && i8) e = rows2d(cscale, c->cb.coeff_scale, dst.coeff_scale, nL * C * 2, C * 2);
-  if (e == cudaSuccess) e = rows2d(summ, c->cb.summary, dst.summary, nL * r * 2, r * 2);
-  if (e == cudaSuccess && slot) {
-    e = rows2d(slot, c->cb.slot, nullptr, nC * 2, 2);
-    if (e == cudaSuccess) e = launch_repack_slot((long long)(B * NG * H), (int)nC, (int)nL, slot, s);
-  }
-  if (e == cudaSuccess) e = launch_repack_scan((int)U, (int)nL, c->cb.res_ptr, dst.res_ptr, base, err, s);
-  long long total = 0;
-  if (e == cudaSuccess) e = cudaMemcpyAsync(&total, base + U, 8, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return cuda_fail(e, "re-lay the chunk arrays");
-  if (total < 0 || total + kResPad >= (1LL << 31)) return inval("re-packed record count out of range");
   uint16_t* rpos = nullptr;
-  void* rval = nullptr;
   __half* rscale = nullptr;
-  if ((st = m.get(&rpos, (size_t)total * 2)) != LOWRAM_OK ||
-      (st = m.get(&rval, ((size_t)total + kResPad) * d * sa)) != LOWRAM_OK)
-    return st;
-  if (i8 && (st = m.get(&rscale, (size_t)total * 2)) != LOWRAM_OK) return st;
-  e = launch_repack_records((int)U, (int)nL, (int)(d * sa), c->cb.n_records, (long long)n_new, c->cb.res_ptr,
-                            c->cb.res_pos, c->cb.res_val, c->cb.res_scale, dst.res_ptr, dst.res_pos, dst.res_val,
-                            static_cast<const __half*>(dst.res_scale), base, rptr, rpos, rval, rscale, err, s);
-  if (e == cudaSuccess) e = cudaMemsetAsync(static_cast<unsigned char*>(rval) + (size_t)total * d * sa, 0, kResPad * d * sa, s);
+  size_t nLs2 = nLs, nCs2 = nCs;
+  if (in_place) {
+    // 4a. the new chunk into slot nL of every unit; records after each unit's last ones
+    e = rows2d(at(c->cb.coeff, nL * C * r * sa), nLs * C * r * sa, dst.coeff, C * r * sa, C * r * sa);
+    if (e == cudaSuccess && i8)
+      e = rows2d(at(c->cb.coeff_scale, nL * C * 2), nLs * C * 2, dst.coeff_scale, C * 2, C * 2);
+    if (e == cudaSuccess) e = rows2d(at(c->cb.summary, nL * r * 2), nLs * r * 2, dst.summary, r * 2, r * 2);
+    if (e == cudaSuccess && c->cb.slot)
+      e = launch_repack_slot((long long)(B * NG * H), (int)nCs, (int)nC, (int)nL, const_cast<int16_t*>(c->cb.slot), s);
+    if (e == cudaSuccess)
+      e = launch_repack_append_records((int)U, (int)nL, (int)nLs, (int)(d * sa), c->cb.n_records, (long long)n_new,
+                                       dst.res_ptr, dst.res_pos, dst.res_val, static_cast<const __half*>(dst.res_scale),
+                                       const_cast<int32_t*>(c->cb.res_ptr), const_cast<uint16_t*>(c->cb.res_pos),
+                                       const_cast<void*>(c->cb.res_val), const_cast<__half*>(c->cb.res_scale), err, s);
+    if (e != cudaSuccess) return cuda_fail(e, "write the new chunk in place");
+  } else {
+    // 4b. arrays of the longer cache with spare capacity: old rows, then the new chunk's,
+    // per (b, group, KV head); spare chunks and spare records per unit for later re-packs
+    const size_t spare = std::max<size_t>(kSpareChunksMin, (nL + 1) / kSpareChunksDiv);
+    nLs2 = nL + 1 + spare;
+    nCs2 = nC + 1 + spare;
+    if (nCs2 > (size_t)kMaxChunks) nCs2 = nC + 1, nLs2 = nL + 1;   // no room to spare
+    const size_t spare_rec = (nLs2 - nL - 1) * (size_t)n_resid;
+    long long* base = nullptr;
+    if ((st = m.get(&coeff, B * NG * H * nLs2 * C * r * sa)) != LOWRAM_OK ||
+        (st = m.get(&summ, B * NG * H * nLs2 * r * 2)) != LOWRAM_OK ||
+        (st = m.get(&rptr, U * (nLs2 + 1) * 4)) != LOWRAM_OK || (st = m.get(&base, (U + 1) * 8)) != LOWRAM_OK)
+      return st;
+    if (i8 && (st = m.get(&cscale, B * NG * H * nLs2 * C * 2)) != LOWRAM_OK) return st;
+    if (c->cb.slot && (st = m.get(&slot, B * NG * H * nCs2 * 2)) != LOWRAM_OK) return st;
+    e = rows2d(coeff, nLs2 * C * r * sa, c->cb.coeff, nLs * C * r * sa, nL * C * r * sa);
+    if (e == cudaSuccess) e = rows2d(at(coeff, nL * C * r * sa), nLs2 * C * r * sa, dst.coeff, C * r * sa, C * r * sa);
+    if (e == cudaSuccess && i8) {
+      e = rows2d(cscale, nLs2 * C * 2, c->cb.coeff_scale, nLs * C * 2, nL * C * 2);
+      if (e == cudaSuccess) e = rows2d(at(cscale, nL * C * 2), nLs2 * C * 2, dst.coeff_scale, C * 2, C * 2);
+    }
+    if (e == cudaSuccess) e = rows2d(summ, nLs2 * r * 2, c->cb.summary, nLs * r * 2, nL * r * 2);
+    if (e == cudaSuccess) e = rows2d(at(summ, nL * r * 2), nLs2 * r * 2, dst.summary, r * 2, r * 2);
+    if (e == cudaSuccess && slot) {
+      e = rows2d(slot, nCs2 * 2, c->cb.slot, nCs * 2, nC * 2);
+      if (e == cudaSuccess) e = launch_repack_slot((long long)(B * NG * H), (int)nCs2, (int)nC, (int)nL, slot, s);
+    }
+    if (e == cudaSuccess)
+      e = launch_repack_scan((int)U, (int)nL, (int)nLs, (long long)spare_rec, c->cb.res_ptr, dst.res_ptr, base, err, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(&total, base + U, 8, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "re-lay the chunk arrays");
+    if (total < 0 || total + kResPad >= (1LL << 31)) return inval("re-packed record count out of range");
+    if ((st = m.get(&rpos, (size_t)total * 2)) != LOWRAM_OK ||
+        (st = m.get(&rval, ((size_t)total + kResPad) * d * sa)) != LOWRAM_OK)
+      return st;
+    if (i8 && (st = m.get(&rscale, (size_t)total * 2)) != LOWRAM_OK) return st;
+    // spare record rows are zero: the tensor-core kernel reads a fixed box of rows from a
+    // chunk's first record and multiplies the rows past the chunk's records by zero
+    e = cudaMemsetAsync(rval, 0, ((size_t)total + kResPad) * d * sa, s);
+    if (e == cudaSuccess)
+      e = launch_repack_records((int)U, (int)nL, (int)nLs, (int)nLs2, (int)(d * sa), c->cb.n_records, (long long)n_new,
+                                c->cb.res_ptr, c->cb.res_pos, c->cb.res_val, c->cb.res_scale, dst.res_ptr, dst.res_pos,
+                                dst.res_val, static_cast<const __half*>(dst.res_scale), base, rptr, rpos, rval, rscale,
+                                err, s);
+    if (e != cudaSuccess) return cuda_fail(e, "re-lay the residual records");
+  }
   uint32_t word = 0, enc_word = 0;
-  if (e == cudaSuccess) e = cudaMemcpyAsync(&word, err, 4, cudaMemcpyDeviceToHost, s);
+  e = cudaMemcpyAsync(&word, err, 4, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaMemcpyAsync(&enc_word, encode_error_word(ge, ws), 4, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  word |= enc_word;
   if (e != cudaSuccess) return cuda_fail(e, "re-lay the residual records");
+  word |= enc_word;
+  // In place, only rows past the live ones were written so far: an error leaves the cache
+  // as it was (its counts are unchanged).
   if (word & ERR_RES_PTR) {
     g_last_error = "the cache's CSR offsets are inconsistent: nothing re-packed";
     return LOWRAM_ECORRUPT;
@@ -566,30 +660,37 @@ lowram_status lowram_cache_repack(lowram_cache* c, int32_t n_resid, lowram_strea
     g_last_error = "the encoder gave up a bounded wait: nothing re-packed";
     return LOWRAM_ETIMEOUT;
   }
-  if (c->n_owned + 4 > (int)(sizeof(c->owned) / sizeof(c->owned[0]))) return inval("internal: too many owned allocations");
+  if (!in_place && c->n_owned + 4 > (int)(sizeof(c->owned) / sizeof(c->owned[0])))
+    return inval("internal: too many owned allocations");
   // 5. the tail drops its oldest chunk (the last step: the cache is unchanged until here)
   e = launch_tail_shift((int)B, (int)L, (int)H, T, C, (int)tail_row, const_cast<void*>(c->cb.tail_k),
                         const_cast<void*>(c->cb.tail_v), const_cast<int32_t*>(c->cb.tail_len), s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "shift the tail");
-  // 6. the cache takes the new arrays
-  auto take = [&](const void* old_p, void* new_p) {
-    m.release(new_p);
-    swap_owned(c, old_p, new_p);
-  };
-  take(c->cb.coeff, coeff); c->cb.coeff = coeff;
-  if (i8) { take(c->cb.coeff_scale, cscale); c->cb.coeff_scale = static_cast<const __half*>(cscale); }
-  take(c->cb.summary, summ); c->cb.summary = summ;
-  if (slot) { take(c->cb.slot, slot); c->cb.slot = slot; }
-  take(c->cb.res_ptr, rptr); c->cb.res_ptr = rptr;
-  take(c->cb.res_pos, rpos); c->cb.res_pos = rpos;
-  take(c->cb.res_val, rval); c->cb.res_val = rval;
-  if (i8) { take(c->cb.res_scale, rscale); c->cb.res_scale = rscale; }
-  c->cb.n_records = total;
+  // 6. the new counts (and, after a re-lay, the new arrays)
+  if (!in_place) {
+    auto take = [&](const void* old_p, void* new_p) {
+      m.release(new_p);
+      swap_owned(c, old_p, new_p);
+    };
+    take(c->cb.coeff, coeff); c->cb.coeff = coeff;
+    if (i8) { take(c->cb.coeff_scale, cscale); c->cb.coeff_scale = static_cast<const __half*>(cscale); }
+    take(c->cb.summary, summ); c->cb.summary = summ;
+    if (slot) { take(c->cb.slot, slot); c->cb.slot = slot; }
+    take(c->cb.res_ptr, rptr); c->cb.res_ptr = rptr;
+    take(c->cb.res_pos, rpos); c->cb.res_pos = rpos;
+    take(c->cb.res_val, rval); c->cb.res_val = rval;
+    if (i8) { take(c->cb.res_scale, rscale); c->cb.res_scale = rscale; }
+    c->cb.n_records = total;
+    c->nLs = (int)nLs2;
+    c->nCs = (int)nCs2;
+    c->canonical = true;
+  }
   c->cfg.n_ctx += C;
   c->cfg.n_live += 1;
   c->nC += 1;
   c->nL += 1;
+  c->last_repack_in_place = in_place;
   return LOWRAM_OK;
 }
 

@@ -75,11 +75,11 @@ attend_simt_kernel(Geom g, CacheBuffers cb, Scratch sc, const float* __restrict_
     const int l = g.layer0 + un.li;
     const int grp = l / g.G;
     const int slot = sc.sel_slot[x];
-    const size_t row0 = ((((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * g.nL + slot) * g.C;
+    const size_t row0 = ((((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * g.nLs + slot) * g.C;
     const T* coeff = reinterpret_cast<const T*>(cb.coeff);
     const int8_t* coeff8 = reinterpret_cast<const int8_t*>(cb.coeff);
     const float* w1 = w1f_t + ((size_t)l * g.Hkv + un.hkv) * g.r * g.h;
-    const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nL + 1);
+    const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nLs + 1);
     const int rec0 = rptr[slot], rec1 = rptr[slot + 1];
 
     for (int t0 = 0; t0 < g.C; t0 += kTB) {

@@ -312,7 +312,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
         const int l = g.layer0 + un.li;
         const int grp = l / g.G;
         const int slot = sc.sel_slot[x];
-        const int row0 = (int)(((((long long)un.b * NG + grp) * g.Hkv + un.hkv) * g.nL + slot) * C);
+        const int row0 = (int)(((((long long)un.b * NG + grp) * g.Hkv + un.hkv) * g.nLs + slot) * C);
         if (leader) {
           if (I8) {
             unsigned char* dst = smem + Lay::OFF_SA + s2 * Lay::SA_SLOT;
@@ -350,7 +350,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
           __syncwarp();
           w1_issued = seg_i + 1;
         }
-        const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nL + 1);
+        const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nLs + 1);
         const int r0 = rptr[slot], r1 = rptr[slot + 1];
         const int nres = min(r1 - r0, kResCap);
         const int my_pos = lane < nres ? (int)cb.res_pos[r0 + lane] : C;
@@ -860,7 +860,7 @@ cudaError_t launch_tc(const Geom& g, const CacheBuffers& cb, const Scratch& sc, 
                       cudaStream_t s) {
   using Lay = TcLayout<R, C, I8>;
   const int NG = g.L / g.G;
-  const uint64_t rows = (uint64_t)g.B * NG * g.Hkv * g.nL * C;
+  const uint64_t rows = (uint64_t)g.B * NG * g.Hkv * g.nLs * C;
   CUtensorMap tmW, tmA, tmQ, tmRes;
   // W1'/2 of every (layer, KV head): [L][Hkv][256][R] 16-bit, boxes of 64 x 128 rows
   if (!make_map(&tmW, w1f, R, (uint64_t)g.L * g.Hkv * kHid, 128)) return cudaErrorInvalidValue;
@@ -891,7 +891,7 @@ bool attend_tc_supported(const Geom& g, int dtype, int store) {
   if (store != LOWRAM_STORE_NATIVE && !(store == LOWRAM_STORE_INT8 && g.C == 128)) return false;
   if (g.d != kDh || g.h != kHid || !(g.g == 4 || g.g == 8)) return false;
   if (!(g.r == 64 || g.r == 128) || !(g.C == 64 || g.C == 128)) return false;
-  const uint64_t rows = (uint64_t)g.B * (g.L / g.G) * g.Hkv * g.nL * g.C;
+  const uint64_t rows = (uint64_t)g.B * (g.L / g.G) * g.Hkv * g.nLs * g.C;
   if (rows >= (1ull << 31) || (uint64_t)g.U * 16 >= (1ull << 31)) return false;
   return encode_fn() != nullptr;
 }

@@ -281,7 +281,7 @@ __global__ void validate_kernel(Geom g, CacheBuffers cb, uint32_t* err) {
   const int n_units = g.B * g.L * g.Hkv;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx < n_slot_rows && cb.slot) {
-    const int16_t* s = cb.slot + (size_t)idx * g.nC;
+    const int16_t* s = cb.slot + (size_t)idx * g.nCs;
     int next = 0;
     bool bad = false;
     for (int c = 0; c < g.nC; ++c) {
@@ -294,7 +294,7 @@ __global__ void validate_kernel(Geom g, CacheBuffers cb, uint32_t* err) {
     if (bad) atomicOr(err, ERR_SLOT);
   }
   if (idx < n_units) {
-    const int32_t* p = cb.res_ptr + (size_t)idx * (g.nL + 1);
+    const int32_t* p = cb.res_ptr + (size_t)idx * (g.nLs + 1);
     bool bad_ptr = false, bad_pos = false;
     for (int s = 0; s <= g.nL; ++s) {
       if (p[s] < 0 || p[s] > cb.n_records) bad_ptr = true;

@@ -31,6 +31,8 @@ constexpr int kResPad = 32;        // zero rows kept after a cache's residual ro
 // Geometry shared by every kernel of one decode call.
 struct Geom {
   int B, L, G, Hkv, Hq, g, d, r, h, N, C, nC, nL, k, T;
+  int nLs, nCs;        // per-unit strides of the chunk arrays: live slots (coefficient rows /
+                       // C, summaries, CSR offsets - 1) and chunk ids (slot map); >= nL, nC
   int layer0, n_layers;
   int U;               // units in this call: n_layers * Hkv * B
   int P;               // CTAs of the chunk-attention kernel (tile partition)

@@ -46,24 +46,26 @@ __global__ void append_count_kernel(int B, int T, int32_t* __restrict__ tail_len
   if (b < B && tail_len[b] >= 0 && tail_len[b] < T) tail_len[b] += 1;
 }
 
-// Record bases of the re-packed cache: unit u (order (b, l, KV head)) gets its old records
-// [old_ptr[u][0], old_ptr[u][nL]) and its new chunk's [new_ptr[u][0], new_ptr[u][1]);
-// base[u] is the exclusive prefix sum of the two counts, base[U] the total.  One block.
+// Record bases of the re-laid cache: unit u (order (b, l, KV head)) gets its old records
+// [old_ptr[u][0], old_ptr[u][nL]), its new chunk's [new_ptr[u][0], new_ptr[u][1]) and
+// spare_rec spare rows; base[u] is the exclusive prefix sum of those counts, base[U] the
+// total.  old_ptr rows have nLs + 1 entries.  One block.
 __global__ void __launch_bounds__(1024)
-repack_scan_kernel(int U, int nL, const int32_t* __restrict__ old_ptr, const int32_t* __restrict__ new_ptr,
-                   long long* __restrict__ base, uint32_t* __restrict__ err) {
+repack_scan_kernel(int U, int nL, int nLs, long long spare_rec, const int32_t* __restrict__ old_ptr,
+                   const int32_t* __restrict__ new_ptr, long long* __restrict__ base, uint32_t* __restrict__ err) {
   __shared__ long long part[1024];
   const int tid = threadIdx.x;
   const int per = (U + blockDim.x - 1) / blockDim.x;
   const int u0 = min(U, tid * per), u1 = min(U, u0 + per);
   auto count = [&](int u) -> long long {
-    const long long o = (long long)old_ptr[(size_t)u * (nL + 1) + nL] - old_ptr[(size_t)u * (nL + 1)];
+    const int32_t* op = old_ptr + (size_t)u * (nLs + 1);
+    const long long o = (long long)op[nL] - op[0];
     const long long n = (long long)new_ptr[2 * (size_t)u + 1] - new_ptr[2 * (size_t)u];
     if (o < 0 || n < 0) {
       atomicOr(err, ERR_RES_PTR);
-      return 0;
+      return spare_rec;
     }
-    return o + n;
+    return o + n + spare_rec;
   };
   long long s = 0;
   for (int u = u0; u < u1; ++u) s += count(u);
@@ -83,10 +85,22 @@ repack_scan_kernel(int U, int nL, const int32_t* __restrict__ old_ptr, const int
   if (tid == blockDim.x - 1) base[U] = part[tid];
 }
 
-// One CTA per unit: its old records, then its new chunk's, to [base[u], base[u+1]); the
-// unit's CSR row of nL+2 offsets.  Record rows are row16 pieces of 16 bytes.
+// Room check of an in-place re-pack: unit u's records end before the next unit's region
+// starts (the array's end for the last unit), so n_res more fit after them.
+__global__ void repack_room_kernel(int U, int nL, int nLs, int n_res, const int32_t* __restrict__ res_ptr,
+                                   long long n_records, uint32_t* __restrict__ flag) {
+  const int u = blockIdx.x * blockDim.x + threadIdx.x;
+  if (u >= U) return;
+  const long long start = res_ptr[(size_t)u * (nLs + 1) + nL];
+  const long long end = u + 1 < U ? (long long)res_ptr[(size_t)(u + 1) * (nLs + 1)] : n_records;
+  if (start < 0 || start + n_res > end) atomicOr(flag, 1u);
+}
+
+// One CTA per unit: its old records, then its new chunk's, to base[u] onwards; the first
+// nL + 2 offsets of the unit's CSR row (rows of nLs_new + 1).  Record rows are row16 pieces
+// of 16 bytes.
 __global__ void __launch_bounds__(kCopyThreads)
-repack_records_kernel(int nL, int row16, long long n_old, long long n_new_total,
+repack_records_kernel(int nL, int nLs_old, int nLs_new, int row16, long long n_old, long long n_new_total,
                       const int32_t* __restrict__ old_ptr, const uint16_t* __restrict__ old_pos,
                       const uint4* __restrict__ old_val, const __half* __restrict__ old_scale,
                       const int32_t* __restrict__ new_ptr, const uint16_t* __restrict__ new_pos,
@@ -95,14 +109,14 @@ repack_records_kernel(int nL, int row16, long long n_old, long long n_new_total,
                       uint16_t* __restrict__ out_pos, uint4* __restrict__ out_val,
                       __half* __restrict__ out_scale, uint32_t* __restrict__ err) {
   const int u = blockIdx.x;
-  const int32_t* op = old_ptr + (size_t)u * (nL + 1);
+  const int32_t* op = old_ptr + (size_t)u * (nLs_old + 1);
   const long long o0 = op[0], no = (long long)op[nL] - o0;
   const long long e0 = new_ptr[2 * (size_t)u], ne = (long long)new_ptr[2 * (size_t)u + 1] - e0;
   const long long b0 = base[u];
   const bool ok_old = no >= 0 && o0 >= 0 && o0 + no <= n_old;
   const bool ok_new = ne >= 0 && e0 >= 0 && e0 + ne <= n_new_total;
   if ((!ok_old || !ok_new) && threadIdx.x == 0) atomicOr(err, ERR_RES_PTR);
-  int32_t* orow = out_ptr + (size_t)u * (nL + 2);
+  int32_t* orow = out_ptr + (size_t)u * (nLs_new + 1);
   for (int c = threadIdx.x; c <= nL; c += blockDim.x) orow[c] = (int32_t)(b0 + (ok_old ? op[c] - o0 : 0));
   if (threadIdx.x == 0) orow[nL + 1] = (int32_t)(b0 + (ok_old ? no : 0) + (ok_new ? ne : 0));
   if (ok_old) {
@@ -124,10 +138,34 @@ repack_records_kernel(int nL, int row16, long long n_old, long long n_new_total,
   }
 }
 
-// The new chunk's slot under eviction: slot[.][nC] = nL (one thread per row of nC+1).
-__global__ void repack_slot_kernel(long long rows, int nC, int nL, int16_t* __restrict__ slot) {
+// In-place re-pack, one CTA per unit: the new chunk's records go right after the unit's
+// last ones (the room check has passed) and the unit's CSR row gains offset nL + 1.
+__global__ void __launch_bounds__(kCopyThreads)
+repack_append_records_kernel(int nL, int nLs, int row16, long long n_records, long long n_new_total,
+                             const int32_t* __restrict__ new_ptr, const uint16_t* __restrict__ new_pos,
+                             const uint4* __restrict__ new_val, const __half* __restrict__ new_scale,
+                             int32_t* __restrict__ res_ptr, uint16_t* __restrict__ res_pos,
+                             uint4* __restrict__ res_val, __half* __restrict__ res_scale, uint32_t* __restrict__ err) {
+  const int u = blockIdx.x;
+  int32_t* row = res_ptr + (size_t)u * (nLs + 1);
+  const long long d0 = row[nL];
+  const long long e0 = new_ptr[2 * (size_t)u], ne = (long long)new_ptr[2 * (size_t)u + 1] - e0;
+  if (ne < 0 || e0 < 0 || e0 + ne > n_new_total || d0 < 0 || d0 + ne > n_records) {
+    if (threadIdx.x == 0) atomicOr(err, ERR_RES_PTR);
+    return;
+  }
+  for (long long i = threadIdx.x; i < ne * row16; i += blockDim.x) res_val[d0 * row16 + i] = new_val[e0 * row16 + i];
+  for (long long i = threadIdx.x; i < ne; i += blockDim.x) {
+    res_pos[d0 + i] = new_pos[e0 + i];
+    if (res_scale) res_scale[d0 + i] = new_scale[e0 + i];
+  }
+  if (threadIdx.x == 0) row[nL + 1] = (int32_t)(d0 + ne);
+}
+
+// The new chunk's slot under eviction: entry nC of every slot row (rows of nCs) is nL.
+__global__ void repack_slot_kernel(long long rows, int nCs, int nC, int nL, int16_t* __restrict__ slot) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < rows) slot[i * (nC + 1) + nC] = (int16_t)nL;
+  if (i < rows) slot[i * nCs + nC] = (int16_t)nL;
 }
 
 // One CTA per (b, l, KV head): tail rows [C, len) move to [0, len - C), a block of C rows at
@@ -170,27 +208,44 @@ cudaError_t launch_append(int B, int L, int Hkv, int T, int row_bytes, const voi
   return cudaGetLastError();
 }
 
-cudaError_t launch_repack_scan(int U, int nL, const int32_t* old_ptr, const int32_t* new_ptr, long long* base,
-                               uint32_t* err, cudaStream_t s) {
-  repack_scan_kernel<<<1, 1024, 0, s>>>(U, nL, old_ptr, new_ptr, base, err);
+cudaError_t launch_repack_room(int U, int nL, int nLs, int n_res, const int32_t* res_ptr, long long n_records,
+                               uint32_t* flag, cudaStream_t s) {
+  repack_room_kernel<<<(U + 255) / 256, 256, 0, s>>>(U, nL, nLs, n_res, res_ptr, n_records, flag);
   return cudaGetLastError();
 }
 
-cudaError_t launch_repack_records(int U, int nL, int row_bytes, long long n_old, long long n_new_total,
-                                  const int32_t* old_ptr, const uint16_t* old_pos, const void* old_val,
-                                  const __half* old_scale, const int32_t* new_ptr, const uint16_t* new_pos,
-                                  const void* new_val, const __half* new_scale, const long long* base,
-                                  int32_t* out_ptr, uint16_t* out_pos, void* out_val, __half* out_scale,
-                                  uint32_t* err, cudaStream_t s) {
+cudaError_t launch_repack_scan(int U, int nL, int nLs, long long spare_rec, const int32_t* old_ptr,
+                               const int32_t* new_ptr, long long* base, uint32_t* err, cudaStream_t s) {
+  repack_scan_kernel<<<1, 1024, 0, s>>>(U, nL, nLs, spare_rec, old_ptr, new_ptr, base, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_repack_records(int U, int nL, int nLs_old, int nLs_new, int row_bytes, long long n_old,
+                                  long long n_new_total, const int32_t* old_ptr, const uint16_t* old_pos,
+                                  const void* old_val, const __half* old_scale, const int32_t* new_ptr,
+                                  const uint16_t* new_pos, const void* new_val, const __half* new_scale,
+                                  const long long* base, int32_t* out_ptr, uint16_t* out_pos, void* out_val,
+                                  __half* out_scale, uint32_t* err, cudaStream_t s) {
   repack_records_kernel<<<U, kCopyThreads, 0, s>>>(
-      nL, row_bytes / 16, n_old, n_new_total, old_ptr, old_pos, static_cast<const uint4*>(old_val), old_scale,
-      new_ptr, new_pos, static_cast<const uint4*>(new_val), new_scale, base, out_ptr, out_pos,
+      nL, nLs_old, nLs_new, row_bytes / 16, n_old, n_new_total, old_ptr, old_pos, static_cast<const uint4*>(old_val),
+      old_scale, new_ptr, new_pos, static_cast<const uint4*>(new_val), new_scale, base, out_ptr, out_pos,
       static_cast<uint4*>(out_val), out_scale, err);
   return cudaGetLastError();
 }
 
-cudaError_t launch_repack_slot(long long rows, int nC, int nL, int16_t* slot, cudaStream_t s) {
-  repack_slot_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(rows, nC, nL, slot);
+cudaError_t launch_repack_append_records(int U, int nL, int nLs, int row_bytes, long long n_records,
+                                         long long n_new_total, const int32_t* new_ptr, const uint16_t* new_pos,
+                                         const void* new_val, const __half* new_scale, int32_t* res_ptr,
+                                         uint16_t* res_pos, void* res_val, __half* res_scale, uint32_t* err,
+                                         cudaStream_t s) {
+  repack_append_records_kernel<<<U, kCopyThreads, 0, s>>>(
+      nL, nLs, row_bytes / 16, n_records, n_new_total, new_ptr, new_pos, static_cast<const uint4*>(new_val),
+      new_scale, res_ptr, res_pos, static_cast<uint4*>(res_val), res_scale, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_repack_slot(long long rows, int nCs, int nC, int nL, int16_t* slot, cudaStream_t s) {
+  repack_slot_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(rows, nCs, nC, nL, slot);
   return cudaGetLastError();
 }
 

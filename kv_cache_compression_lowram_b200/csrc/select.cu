@@ -178,9 +178,9 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
   __syncthreads();
 
   // --- chunk scores over live chunks: one thread per chunk
-  const int16_t* slot = cb.slot ? cb.slot + (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * g.nC : nullptr;
+  const int16_t* slot = cb.slot ? cb.slot + (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * g.nCs : nullptr;
   const T* summ = reinterpret_cast<const T*>(cb.summary) +
-                  (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * (size_t)g.nL * g.r;
+                  (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * (size_t)g.nLs * g.r;
   const float inv_sqrt_d = rsqrtf((float)g.d);
   for (int c = tid; c < g.nC; c += blockDim.x) {
     const int sl = slot ? (int)slot[c] : c;
@@ -496,9 +496,9 @@ select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
     half_sync(1);
 
     // --- chunk scores: one thread per chunk, the whole summary row loaded at once
-    const int16_t* slot = cb.slot ? cb.slot + (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * nC : nullptr;
+    const int16_t* slot = cb.slot ? cb.slot + (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * g.nCs : nullptr;
     const __nv_bfloat16* summ = reinterpret_cast<const __nv_bfloat16*>(cb.summary) +
-                                (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * (size_t)g.nL * R;
+                                (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * (size_t)g.nLs * R;
     const float inv_sqrt_d = rsqrtf((float)D);
     for (int c = ht; c < nC; c += kFastHalf) {
       const int sl = slot ? (int)slot[c] : c;

@@ -99,6 +99,7 @@ extern "C" lowram_status lowram_decode_attn_static(const lowram_config* cfg,
   g.B = cfg->batch; g.L = cfg->n_layers; g.G = cfg->group; g.Hkv = cfg->n_kv_heads;
   g.Hq = cfg->n_q_heads; g.g = g.Hq / g.Hkv; g.d = cfg->head_dim; g.r = cfg->rank;
   g.h = cfg->mlp_hidden; g.N = cfg->n_ctx; g.C = cfg->chunk; g.nC = nC; g.nL = cfg->n_live;
+  g.nLs = g.nL; g.nCs = g.nC;
   g.k = cfg->top_k; g.T = cfg->tail_cap; g.layer0 = layer0; g.n_layers = n_layers;
   g.U = n_layers * g.Hkv * g.B;
   const long long total = (long long)g.U * g.k;

@@ -123,6 +123,7 @@ def test_upkeep_host_checks():
     """Cache view, append and re-pack reject a NULL cache before touching the device."""
     lib = K.lib()
     cfg, src = K.LowramConfigC(), K.LowramSrcC()
-    assert lib.lowram_cache_view(None, ctypes.byref(cfg), ctypes.byref(src)) == 1
+    spare = ctypes.c_int32()
+    assert lib.lowram_cache_view(None, ctypes.byref(cfg), ctypes.byref(src), ctypes.byref(spare)) == 1
     assert lib.lowram_cache_append(None, None, None, None) == 1
     assert lib.lowram_cache_repack(None, 4, None) == 1

@@ -52,6 +52,96 @@ def _unit_records(npc, cfg, u_slots):
     return out
 
 
+def _check_layout(rp, arrays, n_live_records, spare_records):
+    """Units in unit order, each unit's records followed by its spare rows, inside the array."""
+    assert rp[0, 0] == 0
+    assert np.all(rp[:-1, -1] + spare_records == rp[1:, 0])
+    assert rp[-1, -1] + spare_records == arrays["res_pos"].shape[0]
+    assert int((rp[:, -1] - rp[:, 0]).sum()) == n_live_records
+
+
+def _new_chunk(arrays, cfg, s, n_res):
+    """The arrays of live slot s (a re-packed chunk) in the encoder's output form."""
+    B, L, H, C = cfg.batch, cfg.n_layers, cfg.n_kv_heads, cfg.chunk
+    U = B * L * H
+    int8 = cfg.store == "int8"
+    rp = arrays["res_ptr"].cpu().numpy().astype(np.int64).reshape(U, -1)
+    idx = torch.as_tensor(np.concatenate([np.arange(rp[u, s], rp[u, s + 1]) for u in range(U)]), device=DEV)
+    assert np.all(rp[:, s + 1] - rp[:, s] == n_res)
+    return {
+        "coeff": arrays["coeff"][:, :, :, s * C:(s + 1) * C].contiguous(),
+        "coeff_scale": arrays["coeff_scale"][:, :, :, s * C:(s + 1) * C].contiguous() if int8 else None,
+        "summary": arrays["summary"][:, :, :, s:s + 1].contiguous(),
+        "res_ptr": torch.tensor(np.stack([np.arange(U) * n_res, np.arange(1, U + 1) * n_res], -1)
+                                .reshape(B, L, H, 2), dtype=torch.int32),
+        "res_pos": arrays["res_pos"][idx], "res_val": arrays["res_val"][idx],
+        "res_scale": arrays["res_scale"][idx] if int8 else None,
+    }
+
+
+def _codes(g, int8):
+    if int8:
+        return (g["coeff"].cpu().numpy(), g["coeff_scale"].cpu().numpy())
+    return (g["coeff"].cpu().view(torch.int16).numpy().view(np.uint16), None)
+
+
+def _decode_check(lc, cfg2, arrays):
+    got = _np_arrays(arrays, cfg2)
+    gpu_cache = S.SynthCache(cfg=cfg2, **{n: (t.clone() if t is not None else None) for n, t in arrays.items()})
+    gpu_cache.slot = torch.as_tensor(got["slot"], device=DEV)
+    q = S.make_queries(gpu_cache).to(DEV)
+    out, sel = lc.decode(q, sel=True)
+    scores, _ = lc.select(q)
+    torch.cuda.synchronize()
+    check(cfg2, O.OracleCache(got), q, out, sel, scores=scores)
+
+
+@pytest.mark.parametrize("store,evict", [("native", 0.0), ("int8", 0.5)])
+def test_repeated_repacks_in_place_and_relaid(store, evict):
+    """Six re-packs from one long tail: the first re-lays the cache with room for 4 more
+    chunks, the next four write in place, the sixth re-lays again.  Every new chunk is the
+    encoder's work on its tail segment; old chunks stay bit for bit; the cache decodes in
+    parity after an in-place re-pack and at the end."""
+    import oracle.encode as E
+    C = 128
+    cfg = S.LLAMA_32K.replace(name="repack6", batch=2, n_layers=4, n_kv_heads=2, n_ctx=512, top_k=2,
+                              tail_cap=6 * C, store=store, evict_frac=evict)
+    n_res = 16
+    cache = S.make_cache(cfg, tail_len=[6 * C, 6 * C])
+    npc = S.cache_to_numpy(cache)
+    lc = K.LowramCache.from_synth(cache.to(DEV))
+    nL0 = cfg.n_live
+    spares = []
+    for i in range(6):
+        lc.repack(n_res)
+        cfg2d, arrays = lc.view()
+        spares.append(cfg2d["spare_chunks"])
+        if i == 2:
+            cfg2 = cfg.replace(n_ctx=cfg.n_ctx + 3 * C)
+            _decode_check(lc, cfg2, arrays)
+    assert spares == [4, 3, 2, 1, 0, 4]
+    cfg2d, arrays = lc.view()
+    cfg2 = cfg.replace(n_ctx=cfg.n_ctx + 6 * C)
+    assert cfg2d["n_live"] == nL0 + 6 and arrays["tail_len"].cpu().tolist() == [0, 0]
+    int8 = store == "int8"
+    assert np.array_equal(S._np_storage(arrays["coeff"][:, :, :, :nL0 * C]), npc["coeff"])
+    assert np.array_equal(S._np_storage(arrays["summary"][:, :, :, :nL0]), npc["summary"])
+    U = cfg.batch * cfg.n_layers * cfg.n_kv_heads
+    rp = arrays["res_ptr"].cpu().numpy().astype(np.int64).reshape(U, -1)
+    _check_layout(rp, arrays, npc["res_pos"].shape[0] + 6 * U * n_res, 4 * n_res)
+    cfg_c = cfg.replace(name="repack_chunk", n_ctx=C, evict_frac=0.0)
+    f64 = O._bf16_bits_to_f64
+    for i in range(6):
+        g_new = _new_chunk(arrays, cfg, nL0 + i, n_res)
+        seg = slice(i * C, (i + 1) * C)
+        args = (dataclasses.asdict(cfg_c), f64(npc["tail_k"][:, :, :, seg]), f64(npc["tail_v"][:, :, :, seg]),
+                f64(npc["basis"]), f64(npc["w1"]), f64(npc["w2"]), n_res)
+        _check_encode(cfg_c, g_new, E.encode(*args), E.encode(*args, given=_codes(g_new, int8)), n_res)
+    assert lc.validate() == 0
+    _decode_check(lc, cfg2, arrays)
+    lc.close()
+
+
 def test_append_matches_oracle():
     cfg = S.MISTRAL_GROUP.replace(name="append", batch=3, n_ctx=1024)
     cache = S.make_cache(cfg, tail_len=[5, cfg.tail_cap, 0])
@@ -139,12 +229,12 @@ def test_repack_matches_oracle(case):
     assert np.array_equal(got["slot"], ref["slot"])
     old_g, old_o = _unit_records(got, cfg2, range(nL)), _unit_records(npc, cfg, range(nL))
     assert old_g == old_o
-    # CSR: units back to back in unit order, as the oracle lays them
-    assert rp[0, 0] == 0 and np.array_equal(rp[1:, 0], rp[:-1, -1])
-    assert rp[-1, -1] == arrays["res_pos"].shape[0] == npc["res_pos"].shape[0] + U * n_res
-    # where the flags agree, the whole re-packed record layout equals the oracle's
-    if np.array_equal(got["res_pos"], ref_g["res_pos"]):
-        assert np.array_equal(got["res_ptr"], ref_g["res_ptr"])
+    _check_layout(rp, arrays, npc["res_pos"].shape[0] + U * n_res, cfg2d["spare_chunks"] * n_res)
+    # where the flags agree, each unit's records are laid as the oracle lays them
+    rp_o = ref_g["res_ptr"].astype(np.int64).reshape(U, nL + 2)
+    live_pos = np.concatenate([got["res_pos"][rp[u, 0]:rp[u, -1]] for u in range(U)])
+    if np.array_equal(live_pos, ref_g["res_pos"]):
+        assert np.array_equal(rp - rp[:, :1], rp_o - rp_o[:, :1])
     # the tail: shifted by C, lengths down by C
     assert list(got["tail_len"]) == list(ref["tail_len"]) == [extra[0], extra[1]]
     for name in ("tail_k", "tail_v"):
