@@ -122,14 +122,21 @@ combine_kernel(Geom g, CacheBuffers cb, Scratch sc, T* __restrict__ out) {
   }
 }
 
-// The same merge for bf16 with d = 128, h = 256, g in {4, 8}, arranged so that no thread
-// waits on one load after another: each W2 row is split over two threads whose 16 x 16-byte
-// loads are all issued on entry (they land while the partials are merged), and the
-// partial records are read as float4.
+// The same merge for bf16 with d = 128, h = 256, g in {4, 8}, arranged as one round trip to
+// memory: every thread issues all its loads on entry -- its half of one W2 row (16 x 16
+// bytes) and, for each of its float4 slices of the weighted sums, the slice of every piece
+// record with that head's running max and sum -- then derives the merge weights of its
+// head itself (max over the pieces, 2^(m_r - M)), so the only barrier is the one before
+// the second predictor layer reads the merged hidden sums.  Up to kFastRec pieces per unit
+// (a unit's k chunk tiles touch at most two CTAs at the bench sizes; more take the generic kernel).
+constexpr int kFastRec = 2;
+
 template <int GQ>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 combine_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, __nv_bfloat16* __restrict__ out) {
   constexpr int D = 128, H = 256;
+  constexpr int NH = GQ * H / 4 / kThreads;          // float4 slices of the hidden sums per thread
+  constexpr int ND = (GQ * D / 4 + kThreads - 1) / kThreads;
   extern __shared__ __align__(16) float sm[];
   const int u = blockIdx.x;
   const Unit un = unit_of(g, u);
@@ -147,54 +154,109 @@ combine_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, __nv_bfloat16* __restri
   const int c0 = cta_of_tile(total, g.P, (long long)u * g.k);
   const int c1 = cta_of_tile(total, g.P, (long long)(u + 1) * g.k - 1);
   const int nrec = c1 - c0 + 1;
-  if (nrec > g.max_rec) {  // cannot happen with a consistent tile partition
+  if (nrec > g.max_rec || nrec > kFastRec) {  // cannot happen with a consistent tile partition
     if (tid == 0) atomicOr(sc.err, ERR_SELECT);
     return;
   }
   float* accH = sm;                 // [GQ][H]
   float* accD = accH + GQ * H;      // [GQ][D]
   float* lsum = accD + GQ * D;      // [GQ]
-  float* wts = lsum + GQ;           // [nrec + 1][GQ]  (last row: tail)
   const float* trec = sc.tail_part + (size_t)u * g.tail_stride;
   const float* rec0 = sc.part + (size_t)(u + c0) * g.rec_stride;
+  // merge weights of head j over the pieces (and the tail): w_r = 2^(m_r - M)
+  auto weights = [&](int j, const float (&m)[kFastRec], float mt, float (&wr)[kFastRec], float& wt) {
+    float M = mt;
+#pragma unroll
+    for (int r = 0; r < kFastRec; ++r)
+      if (r < nrec) M = fmaxf(M, m[r]);
+#pragma unroll
+    for (int r = 0; r < kFastRec; ++r) wr[r] = (r < nrec && m[r] != -INFINITY) ? exp2f(m[r] - M) : 0.f;
+    wt = mt == -INFINITY ? 0.f : exp2f(mt - M);
+  };
+  // hidden sums: loads first
+  float4 vh[NH][kFastRec];
+  float mh[NH][kFastRec];
+#pragma unroll
+  for (int q = 0; q < NH; ++q) {
+    const int i4 = tid + q * kThreads, j = (i4 * 4) / H;
+#pragma unroll
+    for (int r = 0; r < kFastRec; ++r) {
+      const float* rec = rec0 + (size_t)r * g.rec_stride;
+      if (r < nrec) {
+        mh[q][r] = rec[j];
+        vh[q][r] = *reinterpret_cast<const float4*>(rec + 2 * GQ + i4 * 4);
+      }
+    }
+  }
+  // residual / tail sums: loads first
+  float4 vd[ND][kFastRec], vt[ND];
+  float md[ND][kFastRec], mtd[ND];
+#pragma unroll
+  for (int q = 0; q < ND; ++q) {
+    const int i4 = tid + q * kThreads;
+    if (i4 < GQ * D / 4) {
+      const int j = (i4 * 4) / D;
+      mtd[q] = trec[j];
+      vt[q] = *reinterpret_cast<const float4*>(trec + 2 * GQ + i4 * 4);
+#pragma unroll
+      for (int r = 0; r < kFastRec; ++r) {
+        const float* rec = rec0 + (size_t)r * g.rec_stride;
+        if (r < nrec) {
+          md[q][r] = rec[j];
+          vd[q][r] = *reinterpret_cast<const float4*>(rec + 2 * GQ + GQ * H + i4 * 4);
+        }
+      }
+    }
+  }
+  // the softmax denominators
   if (tid < GQ) {
     const int j = tid;
-    float M = trec[j];
-    for (int r = 0; r < nrec; ++r) M = fmaxf(M, rec0[(size_t)r * g.rec_stride + j]);
-    float L = 0.f;
-    for (int r = 0; r < nrec; ++r) {
+    float m[kFastRec], sr[kFastRec], wr[kFastRec], wt;
+#pragma unroll
+    for (int r = 0; r < kFastRec; ++r) {
       const float* rec = rec0 + (size_t)r * g.rec_stride;
-      const float wr = rec[j] == -INFINITY ? 0.f : exp2f(rec[j] - M);
-      wts[r * GQ + j] = wr;
-      L += wr * rec[GQ + j];
+      m[r] = r < nrec ? rec[j] : -INFINITY;
+      sr[r] = r < nrec ? rec[GQ + j] : 0.f;
     }
-    const float wt = trec[j] == -INFINITY ? 0.f : exp2f(trec[j] - M);
-    wts[nrec * GQ + j] = wt;
-    lsum[j] = L + wt * trec[GQ + j];
+    const float mt = trec[j], st = trec[GQ + j];
+    weights(j, m, mt, wr, wt);
+    float L = wt * st;
+#pragma unroll
+    for (int r = 0; r < kFastRec; ++r) L = fmaf(wr[r], sr[r], L);
+    lsum[j] = L;
   }
-  __syncthreads();
-  // weighted hidden sums and residual/tail sums, four floats per thread and record
-  for (int i4 = tid; i4 < GQ * H / 4; i4 += kThreads) {
-    const int j = (i4 * 4) / H;
+#pragma unroll
+  for (int q = 0; q < NH; ++q) {
+    const int i4 = tid + q * kThreads, j = (i4 * 4) / H;
+    float wr[kFastRec], wt;
+    weights(j, mh[q], trec[j], wr, wt);
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int r = 0; r < nrec; ++r) {
-      const float4 v = *reinterpret_cast<const float4*>(rec0 + (size_t)r * g.rec_stride + 2 * GQ + i4 * 4);
-      const float wr = wts[r * GQ + j];
-      a.x = fmaf(wr, v.x, a.x); a.y = fmaf(wr, v.y, a.y); a.z = fmaf(wr, v.z, a.z); a.w = fmaf(wr, v.w, a.w);
+#pragma unroll
+    for (int r = 0; r < kFastRec; ++r) {
+      if (r < nrec) {
+        a.x = fmaf(wr[r], vh[q][r].x, a.x); a.y = fmaf(wr[r], vh[q][r].y, a.y);
+        a.z = fmaf(wr[r], vh[q][r].z, a.z); a.w = fmaf(wr[r], vh[q][r].w, a.w);
+      }
     }
     *reinterpret_cast<float4*>(accH + i4 * 4) = a;
   }
-  for (int i4 = tid; i4 < GQ * D / 4; i4 += kThreads) {
-    const int j = (i4 * 4) / D;
-    const float wt = wts[nrec * GQ + j];
-    const float4 tv = *reinterpret_cast<const float4*>(trec + 2 * GQ + i4 * 4);
-    float4 a = make_float4(wt * tv.x, wt * tv.y, wt * tv.z, wt * tv.w);
-    for (int r = 0; r < nrec; ++r) {
-      const float4 v = *reinterpret_cast<const float4*>(rec0 + (size_t)r * g.rec_stride + 2 * GQ + GQ * H + i4 * 4);
-      const float wr = wts[r * GQ + j];
-      a.x = fmaf(wr, v.x, a.x); a.y = fmaf(wr, v.y, a.y); a.z = fmaf(wr, v.z, a.z); a.w = fmaf(wr, v.w, a.w);
+#pragma unroll
+  for (int q = 0; q < ND; ++q) {
+    const int i4 = tid + q * kThreads;
+    if (i4 < GQ * D / 4) {
+      const int j = (i4 * 4) / D;
+      float wr[kFastRec], wt;
+      weights(j, md[q], mtd[q], wr, wt);
+      float4 a = make_float4(wt * vt[q].x, wt * vt[q].y, wt * vt[q].z, wt * vt[q].w);
+#pragma unroll
+      for (int r = 0; r < kFastRec; ++r) {
+        if (r < nrec) {
+          a.x = fmaf(wr[r], vd[q][r].x, a.x); a.y = fmaf(wr[r], vd[q][r].y, a.y);
+          a.z = fmaf(wr[r], vd[q][r].z, a.z); a.w = fmaf(wr[r], vd[q][r].w, a.w);
+        }
+      }
+      *reinterpret_cast<float4*>(accD + i4 * 4) = a;
     }
-    *reinterpret_cast<float4*>(accD + i4 * 4) = a;
   }
   __syncthreads();
   // second predictor layer: this thread's half row against every head's hidden sums
@@ -335,7 +397,7 @@ cudaError_t launch_combine(const Geom& g, const CacheBuffers& cb, const Scratch&
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<g.U, kThreads, smem, s>>>(g, cb, sc, static_cast<float*>(out));
-  } else if (g.d == 128 && g.h == 256 && (g.g == 4 || g.g == 8)) {
+  } else if (g.d == 128 && g.h == 256 && (g.g == 4 || g.g == 8) && g.max_rec <= kFastRec) {
     auto k = g.g == 4 ? combine_fast_kernel<4> : combine_fast_kernel<8>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
