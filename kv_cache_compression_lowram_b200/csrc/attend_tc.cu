@@ -116,6 +116,8 @@ struct Bars {
   uint64_t w1_ready;   // W1' of the next (layer, KV head) is in shared memory
   uint64_t seg_done;   // every MMA that read the previous W1' is complete
   uint64_t drain;
+  uint64_t h_free[3];  // the weighted sums of the H in a D1 buffer are complete (bf16 split issue)
+  uint64_t drain2;
 };
 
 struct Misc {
@@ -237,7 +239,9 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
     for (int i = 0; i < NBUF; ++i) {
       mbar_init(&bar.d1_full[i], 1);
       mbar_init(&bar.h_ready[i], 4);      // the 4 warps of the sub-tile's epilogue group
+      mbar_init(&bar.h_free[i], 1);
     }
+    mbar_init(&bar.drain2, 1);
     mbar_init(&bar.w1_ready, 1);          // TMA
     mbar_init(&bar.seg_done, 1);
     mbar_init(&bar.drain, 1);
@@ -493,12 +497,92 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
       };
 
       bool ok = true;
-      for (int n = 0; ok && n < NBUF && n < NS; ++n) ok = issue_mma1(n);
-      // Per chunk: the weighted sums of both hidden halves (and the residual rows) back to
-      // back, their commit, and only then the next pre-activations.  A commit waits for
-      // every MMA this thread issued before it, so D1 work queued between the two halves
-      // would hold back the softmax's fold of the chunk, and with it the probabilities of
-      // the next chunk.
+      if (!I8) {
+        // bf16 store: this warp issues only the pre-activations and the scores, as far ahead
+        // as the D1 buffers allow; warp 2 issues the weighted sums as the silu groups finish.
+        // D1 buffer n % 3 is reused once the weighted sums of sub-tile n-3 are complete; the
+        // scores of chunk ci overwrite those of chunk ci-2 once the softmax has published
+        // that chunk's probabilities.
+        for (int n = 0; ok && n < NS; ++n) {
+          const int ci = n >> 1;
+          if (n >= NBUF) ok = wait_all(&bar.h_free[n % NBUF], ((n / NBUF) - 1) & 1);
+          if (ok && (n & 1) == 0 && ci >= 2) ok = wait_all(&bar.p_ready[ci & 1], ((ci - 2) >> 1) & 1);
+          if (ok) {
+            tc_fence_after();
+            ok = issue_mma1(n);
+          }
+        }
+      } else {
+        for (int n = 0; ok && n < NBUF && n < NS; ++n) ok = issue_mma1(n);
+        // Per chunk: the weighted sums of both hidden halves (and the residual rows) back to
+        // back, their commit, and only then the next pre-activations.  A commit waits for
+        // every MMA this thread issued before it, so D1 work queued between the two halves
+        // would hold back the softmax's fold of the chunk, and with it the probabilities of
+        // the next chunk.
+        for (int ci = 0; ok && ci < NCH; ++ci) {
+          const int pb = ci & 1, st = ci % STAGES;
+          const uint64_t dP = dP0 + (uint64_t)((pb * Lay::P_BUF) >> 4);
+  #pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int n = 2 * ci + hh, bf = n % NBUF;
+            if (!wait_all(&bar.h_ready[bf], (n / NBUF) & 1)) { ok = false; break; }
+            // One acquire covers the softmax's hand-offs: before it publishes the
+            // probabilities of chunk ci it has waited for the chunk's residual rows and read
+            // out the D3 / D4 buffer of chunk ci-2.
+            if (hh == 0 && !wait_all(&bar.p_ready[pb], (ci >> 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+            if (leader) {
+              // softmax-weighted hidden sums of this half: H (fp16 pairs, token pair j at
+              // column j of the buffer) times P, K = the chunk's tokens
+  #pragma unroll
+              for (int kk = 0; kk < C / 16; ++kk)
+                mma_ts(t_d3 + pb * 32 + hh * 16, t_d1 + bf * 128 + kk * 8, dP + (uint64_t)(kk * 16), IDESC_3,
+                       kk > 0 ? 1u : 0u);
+              if (hh == 0) {
+                // the chunk's weighted residual rows: 16 records = two 8-row groups of the
+                // MN-major tile per MMA
+                const uint64_t dPR = dPR0 + (uint64_t)((pb * Lay::PR_BUF) >> 4);
+                const uint64_t dR = dR0 + (uint64_t)((st * Lay::RES_BUF) >> 4);
+  #pragma unroll
+                for (int kk = 0; kk < kResCap / 16; ++kk)
+                  mma_ss(t_d4 + pb * 16, dR + (uint64_t)(kk * (2048 >> 4)), dPR + (uint64_t)(kk * 16), IDESC_4,
+                         kk > 0 ? 1u : 0u);
+                mma_commit(&bar.r_empty[st]);
+              } else {
+                mma_commit(&bar.d3_full[pb]);
+              }
+            }
+            __syncwarp();
+          }
+          // the next pre-activations into the two buffers just read
+          for (int n = 2 * ci + NBUF; ok && n < 2 * ci + NBUF + 2 && n < NS; ++n) ok = issue_mma1(n);
+        }
+      }
+      // every MMA this warp issued must finish before TMEM is released
+      if (leader) {
+        mma_commit(&bar.drain);
+        volatile int never = 0;
+        mbar_wait(&bar.drain, 0, &never, err, ERR_TIMEOUT);
+      }
+      __syncwarp();
+    }
+  } else if (!I8 && warp == 2) {
+    // ============================================================ weighted-sum issuer (bf16)
+    // Per chunk: the weighted hidden sums of each half as soon as its silu group has written
+    // H (and, for half 0, the softmax its probabilities), the residual rows' sum with half
+    // 0; a commit per half frees its D1 buffer for the pre-activation warp, and the commit
+    // after half 1 hands the chunk to the softmax.  Issued apart from the pre-activations,
+    // so waiting for an epilogue group never holds back the next D1 MMAs.
+    const bool leader = elect_one();
+    if (NS > 0) {
+      const uint64_t dP0 = smem_desc(sP, 128, Lay::P_SBO, 0);       // probabilities
+      const uint64_t dR0 = smem_desc(sRes, Lay::RES_SLAB, 1024, 2); // residual rows, MN-major
+      const uint64_t dPR0 = smem_desc(sPR, 128, Lay::PR_SBO, 0);    // probabilities at records
+      const uint32_t t_d1 = tmem + Lay::T_D1, t_d3 = tmem + Lay::T_D3, t_d4 = tmem + Lay::T_D4;
+      auto wait_all = [&](uint64_t* b, uint32_t par) -> bool {
+        return __all_sync(0xffffffffu, mbar_wait(b, par, abort_flag, err, ERR_TIMEOUT));
+      };
+      bool ok = true;
       for (int ci = 0; ok && ci < NCH; ++ci) {
         const int pb = ci & 1, st = ci % STAGES;
         const uint64_t dP = dP0 + (uint64_t)((pb * Lay::P_BUF) >> 4);
@@ -506,21 +590,14 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
         for (int hh = 0; hh < 2; ++hh) {
           const int n = 2 * ci + hh, bf = n % NBUF;
           if (!wait_all(&bar.h_ready[bf], (n / NBUF) & 1)) { ok = false; break; }
-          // One acquire covers the softmax's hand-offs: before it publishes the
-          // probabilities of chunk ci it has waited for the chunk's residual rows and read
-          // out the D3 / D4 buffer of chunk ci-2.
           if (hh == 0 && !wait_all(&bar.p_ready[pb], (ci >> 1) & 1)) { ok = false; break; }
           tc_fence_after();
           if (leader) {
-            // softmax-weighted hidden sums of this half: H (fp16 pairs, token pair j at
-            // column j of the buffer) times P, K = the chunk's tokens
 #pragma unroll
             for (int kk = 0; kk < C / 16; ++kk)
               mma_ts(t_d3 + pb * 32 + hh * 16, t_d1 + bf * 128 + kk * 8, dP + (uint64_t)(kk * 16), IDESC_3,
                      kk > 0 ? 1u : 0u);
             if (hh == 0) {
-              // the chunk's weighted residual rows: 16 records = two 8-row groups of the
-              // MN-major tile per MMA
               const uint64_t dPR = dPR0 + (uint64_t)((pb * Lay::PR_BUF) >> 4);
               const uint64_t dR = dR0 + (uint64_t)((st * Lay::RES_BUF) >> 4);
 #pragma unroll
@@ -528,20 +605,18 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
                 mma_ss(t_d4 + pb * 16, dR + (uint64_t)(kk * (2048 >> 4)), dPR + (uint64_t)(kk * 16), IDESC_4,
                        kk > 0 ? 1u : 0u);
               mma_commit(&bar.r_empty[st]);
-            } else {
-              mma_commit(&bar.d3_full[pb]);
             }
+            mma_commit(&bar.h_free[bf]);
+            if (hh == 1) mma_commit(&bar.d3_full[pb]);
           }
           __syncwarp();
         }
-        // the next pre-activations into the two buffers just read
-        for (int n = 2 * ci + NBUF; ok && n < 2 * ci + NBUF + 2 && n < NS; ++n) ok = issue_mma1(n);
       }
       // every MMA this warp issued must finish before TMEM is released
       if (leader) {
-        mma_commit(&bar.drain);
+        mma_commit(&bar.drain2);
         volatile int never = 0;
-        mbar_wait(&bar.drain, 0, &never, err, ERR_TIMEOUT);
+        mbar_wait(&bar.drain2, 0, &never, err, ERR_TIMEOUT);
       }
       __syncwarp();
     }
