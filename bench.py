@@ -51,6 +51,8 @@ def parse():
                     help="only the uncompressed bf16 dense-KV baseline at its largest batch")
     ap.add_argument("--encode", action="store_true",
                     help="only the prefill-side encoder (dense K, V -> compressed cache) of the workload")
+    ap.add_argument("--dense-batch", type=int, default=0,
+                    help="with --dense: this batch instead of the largest that fits (profiling)")
     ap.add_argument("--repack", action="store_true",
                     help="only the decode-loop upkeep: C tail appends and one chunk re-pack per step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -404,6 +406,8 @@ def run_dense(args, ws, rank, local, cfg_name=DEFAULT_CONFIG):
     per_seq = 2 * cfg.n_layers * cfg.n_kv_heads * S_ * cfg.head_dim * 2
     free, _ = torch.cuda.mem_get_info(dev)
     B = max(1, int((free - 6e9) // per_seq))
+    if getattr(args, "dense_batch", 0) > 0:
+        B = min(B, args.dense_batch)
     gen = torch.Generator(device=dev)
     gen.manual_seed(cfg.seed + 17 + rank)
     k = torch.empty(B, cfg.n_layers, cfg.n_kv_heads, S_, cfg.head_dim, dtype=torch.bfloat16, device=dev)
