@@ -308,11 +308,14 @@ def run_lowram(args, ws, rank, local):
     used_path = {1: "simt", 2: "tc"}.get(lc.last_path, "?")
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    queries_step = cfg.batch * cfg.n_layers
     clocks = ClockSampler(local)
     barrier(ws)
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)
+    # (1) eager calls with the library's stage events: per-kernel launch durations for the
+    # roofline (the events sit between the kernels, so this pass is a little slower)
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     start.record(stream)
@@ -321,13 +324,46 @@ def run_lowram(args, ws, rank, local):
         K.lowram_decode_attn(lc.handle, 0, cfg.n_layers, q, out, sel, path)
     end.record(stream)
     torch.cuda.synchronize()
+    K.lowram_cache_set_stage_events(lc.handle, None)
+    eager_ms_total = start.elapsed_time(end)
+    stage_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(3)]
+    # (2) the timed steps: the same call captured once in a CUDA graph and replayed (the
+    # library launches only on the caller's stream, with no synchronisation and no
+    # allocation); if capture is not possible the eager pass is the measurement
+    graph_ms, graph_err = None, None
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            K.lowram_decode_attn(lc.handle, 0, cfg.n_layers, q, out, sel, path)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+    except Exception as exc:
+        g = None
+        graph_err = str(exc).splitlines()[0][:200] if str(exc) else type(exc).__name__
+    # every rank takes the same collective steps, whether or not its capture worked
+    barrier(ws)
+    torch.cuda.synchronize()
+    if g is not None:
+        gs, ge = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        gs.record(stream)
+        for _ in range(args.steps):
+            g.replay()
+        ge.record(stream)
+        torch.cuda.synchronize()
+        graph_ms = gs.elapsed_time(ge)
+        del g
     barrier(ws)
     clk = clocks.stop()
-    K.lowram_cache_set_stage_events(lc.handle, None)
-    queries_step = cfg.batch * cfg.n_layers
-    value, ms_total = aggregate_rate(queries_step * args.steps, start.elapsed_time(end), ws)
+    eager_value, eager_total = aggregate_rate(queries_step * args.steps, eager_ms_total, ws)
+    gval, gtotal = aggregate_rate(queries_step * args.steps, graph_ms if graph_ms is not None else 1e30, ws)
+    graph_ok = graph_ms is not None and gtotal < 1e29
+    value, ms_total = (gval, gtotal) if graph_ok else (eager_value, eager_total)
     ms_step = ms_total / args.steps
-    stage_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j in range(3)]
+    timing = {"timed": "cuda graph replays" if graph_ok else "eager calls",
+              "eager_ms_per_step": round(eager_total / args.steps, 4), "eager_value": round(eager_value, 1)}
+    if not graph_ok:
+        timing["graph_unavailable"] = graph_err or "capture failed on another rank"
 
     # end to end through the host entry point: pinned q in, pinned out back, every step
     q_h = q.cpu().pin_memory()
@@ -387,6 +423,7 @@ def run_lowram(args, ws, rank, local):
                 "h2d_bytes_per_step": qbytes, "d2h_bytes_per_step": qbytes},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
+        "timing": timing,
     }
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         rate, sample, threads = oracle_rate(cfg, cache, q)
