@@ -210,7 +210,11 @@ lowram_status lowram_select_chunks(lowram_cache* cache, int32_t layer0, int32_t 
 
 /* Same as lowram_decode_attn with HOST buffers q_host/out_host/sel_host (sel may be NULL):
  * copies q to the device, decodes, copies the results back and synchronises `stream`.
- * Pinned host memory makes the copies asynchronous; pageable memory works too. */
+ * Pinned host memory makes the copies asynchronous; pageable memory works too.  The decode
+ * runs on device buffers the cache owns, so the first call for a layer range captures it
+ * into a CUDA graph (on a stream of the cache's own) and later calls replay the graph; a
+ * re-pack drops it, stage events (lowram_cache_set_stage_events) bypass it, and if capture
+ * fails the calls stay eager. */
 lowram_status lowram_decode_attn_host(lowram_cache* cache, int32_t layer0, int32_t n_layers,
                                       const void* q_host, void* out_host, int32_t* sel_host,
                                       lowram_stream stream);

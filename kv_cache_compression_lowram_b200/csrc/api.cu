@@ -19,6 +19,12 @@ struct lowram_cache {
   bool last_repack_in_place;
   void* up_mem;                // re-pack scratch (encoder inputs, outputs and workspace), kept
   size_t up_bytes;
+  // lowram_decode_attn_host replays its decode (on the staging buffers) from a CUDA graph
+  // captured at its first call for a layer range; a re-pack or destroy drops it
+  cudaStream_t cap_stream;
+  cudaGraphExec_t host_exec;
+  int hg_layer0, hg_n, hg_sel;
+  bool hg_off;                 // capture failed once: eager calls from then on
   size_t s_dt;                 // bytes of one dt element
   void* owned[48];             // every device allocation the cache owns
   int n_owned;
@@ -278,6 +284,7 @@ lowram_status lowram_cache_create(const lowram_config* cfg, const lowram_cache_s
   c->nC = nC; c->nL = cfg->n_live; c->NG = cfg->n_layers / cfg->group;
   c->nLs = c->nL; c->nCs = nC; c->canonical = false; c->last_repack_in_place = false;
   c->up_mem = nullptr; c->up_bytes = 0;
+  c->cap_stream = nullptr; c->host_exec = nullptr; c->hg_off = false;
   c->g = cfg->n_q_heads / cfg->n_kv_heads;
   c->device = dev; c->n_sm = n_sm;
   c->s_dt = cfg->dtype == LOWRAM_F32 ? 4 : 2;
@@ -377,6 +384,8 @@ void lowram_cache_destroy(lowram_cache* c) {
   cudaDeviceSynchronize();
   for (int i = 0; i < c->n_owned; ++i) cudaFree(c->owned[i]);
   if (c->up_mem) cudaFree(c->up_mem);
+  if (c->host_exec) cudaGraphExecDestroy(c->host_exec);
+  if (c->cap_stream) cudaStreamDestroy(c->cap_stream);
   delete c;
 }
 
@@ -691,6 +700,10 @@ lowram_status lowram_cache_repack(lowram_cache* c, int32_t n_resid, lowram_strea
   c->nC += 1;
   c->nL += 1;
   c->last_repack_in_place = in_place;
+  if (c->host_exec) {   // its kernels' geometry and pointers are those of the shorter cache
+    cudaGraphExecDestroy(c->host_exec);
+    c->host_exec = nullptr;
+  }
   return LOWRAM_OK;
 }
 
@@ -783,9 +796,45 @@ lowram_status lowram_decode_attn_host(lowram_cache* c, int32_t layer0, int32_t n
   const size_t sbytes = (size_t)n_layers * c->cfg.batch * c->cfg.n_kv_heads * c->cfg.top_k * 4;
   cudaError_t e = cudaMemcpyAsync(c->q_stage, q_host, qbytes, cudaMemcpyHostToDevice, s);
   if (e != cudaSuccess) return cuda_fail(e, "copy q to the device");
-  st = lowram_decode_attn(c, layer0, n_layers, c->q_stage, c->out_stage,
-                          sel_host ? c->sel_stage : nullptr, LOWRAM_PATH_AUTO, stream);
-  if (st != LOWRAM_OK) return st;
+  int32_t* sel_dev = sel_host ? c->sel_stage : nullptr;
+  bool replayed = false;
+  if (!c->ev_on && !c->hg_off) {
+    const bool same = c->host_exec && c->hg_layer0 == layer0 && c->hg_n == n_layers && c->hg_sel == (sel_dev != nullptr);
+    if (!same) {
+      if (c->host_exec) cudaGraphExecDestroy(c->host_exec);
+      c->host_exec = nullptr;
+      // capture on a stream of the cache's own (the legacy default stream cannot be captured)
+      cudaGraph_t graph = nullptr;
+      bool ok = c->cap_stream || cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking) == cudaSuccess;
+      ok = ok && cudaStreamBeginCapture(c->cap_stream, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+      if (ok) {
+        const lowram_status sc = lowram_decode_attn(c, layer0, n_layers, c->q_stage, c->out_stage, sel_dev,
+                                                    LOWRAM_PATH_AUTO, reinterpret_cast<lowram_stream>(c->cap_stream));
+        const cudaError_t ec = cudaStreamEndCapture(c->cap_stream, &graph);
+        ok = sc == LOWRAM_OK && ec == cudaSuccess && graph &&
+             cudaGraphInstantiate(&c->host_exec, graph, 0) == cudaSuccess;
+        if (graph) cudaGraphDestroy(graph);
+      }
+      if (ok) {
+        c->hg_layer0 = layer0;
+        c->hg_n = n_layers;
+        c->hg_sel = sel_dev != nullptr;
+      } else {
+        c->host_exec = nullptr;
+        c->hg_off = true;
+        cudaGetLastError();   // clear a capture error; the eager call below reports its own
+      }
+    }
+    if (c->host_exec) {
+      e = cudaGraphLaunch(c->host_exec, s);
+      if (e != cudaSuccess) return cuda_fail(e, "decode graph launch");
+      replayed = true;
+    }
+  }
+  if (!replayed) {
+    st = lowram_decode_attn(c, layer0, n_layers, c->q_stage, c->out_stage, sel_dev, LOWRAM_PATH_AUTO, stream);
+    if (st != LOWRAM_OK) return st;
+  }
   e = cudaMemcpyAsync(out_host, c->out_stage, qbytes, cudaMemcpyDeviceToHost, s);
   if (e != cudaSuccess) return cuda_fail(e, "copy out to the host");
   if (sel_host) {

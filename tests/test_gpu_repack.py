@@ -296,3 +296,25 @@ def test_decode_loop_append_repack_decode():
     assert lc.validate() == 0
     check(cfg2, O.OracleCache(got), q, out, sel)
     lc.close()
+
+
+def test_host_entry_graph_follows_the_repack():
+    """lowram_decode_attn_host replays a captured decode; after a re-pack it must decode the
+    longer cache (the captured graph is dropped), matching the device entry point."""
+    cfg = S.LLAMA_32K.replace(name="host_graph", batch=2, n_layers=4, n_kv_heads=2, n_ctx=512, top_k=2)
+    cache = S.make_cache(cfg, tail_len=[cfg.chunk, cfg.chunk])
+    lc = K.LowramCache.from_synth(cache.to(DEV))
+    q = S.make_queries(cache).to(DEV)
+    q_h = q.cpu().pin_memory()
+    out_h = torch.empty_like(q_h).pin_memory()
+    for step in range(2):
+        out_d = lc.decode(q)
+        torch.cuda.synchronize()
+        for _ in range(3):   # the first call captures, the others replay
+            out_h.zero_()
+            K.lowram_decode_attn_host(lc.handle, 0, cfg.n_layers, q_h, out_h)
+            assert torch.equal(out_h, out_d.cpu())
+        if step == 0:
+            lc.repack(16)
+    assert lc.view()[0]["n_ctx"] == cfg.n_ctx + cfg.chunk
+    lc.close()
