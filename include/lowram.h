@@ -219,7 +219,9 @@ lowram_status lowram_decode_attn_host(lowram_cache* cache, int32_t layer0, int32
                                       const void* q_host, void* out_host, int32_t* sel_host,
                                       lowram_stream stream);
 
-/* Byte accounting of a created cache (host only, no device access). */
+/* Byte accounting of a created cache (host only, no device access): the live arrays.  Room a
+ * re-pack keeps for later chunks (lowram_cache_view's spare_chunks, and the spare record
+ * rows after each unit's records) is allocated in addition and not counted here. */
 lowram_status lowram_cache_bytes(const lowram_cache* cache, lowram_bytes* out);
 
 /* Device-side consistency check of the index tables (slot map, CSR offsets, record
@@ -256,8 +258,10 @@ int32_t lowram_cache_last_path(const lowram_cache* cache);
  * unit strides of (nL + S) * C coefficient rows (and scales), nL + S summaries, nL + S + 1
  * CSR offsets and nC + S slot entries, S = *spare_chunks (0 until a re-pack adds room).
  * After a re-pack the records of each unit are followed by spare record rows, so n_records
- * counts allocated rows, not live records.  Valid until the next lowram_cache_repack or
- * lowram_cache_destroy.  Host only. */
+ * counts allocated rows, not live records.  While *spare_chunks is 0 the view is exactly a
+ * lowram_cache_src (lowram_decode_attn_static and lowram_cache_create accept it); with
+ * spare room the chunk arrays are strided and those entry points do not.  Valid until the
+ * next lowram_cache_repack or lowram_cache_destroy.  Host only. */
 lowram_status lowram_cache_view(const lowram_cache* cache, lowram_config* cfg, lowram_cache_src* src,
                                 int32_t* spare_chunks);
 
