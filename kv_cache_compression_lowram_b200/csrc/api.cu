@@ -19,6 +19,7 @@ struct lowram_cache {
   bool last_repack_in_place;
   void* up_mem;                // re-pack scratch (encoder inputs, outputs and workspace), kept
   size_t up_bytes;
+  bool up_w2h_ready;           // the re-pack scratch's encoder workspace holds W2 in fp16
   // lowram_decode_attn_host replays its decode (on the staging buffers) from a CUDA graph
   // captured at its first call for a layer range; a re-pack or destroy drops it
   cudaStream_t cap_stream;
@@ -283,7 +284,7 @@ lowram_status lowram_cache_create(const lowram_config* cfg, const lowram_cache_s
   c->cfg = *cfg;
   c->nC = nC; c->nL = cfg->n_live; c->NG = cfg->n_layers / cfg->group;
   c->nLs = c->nL; c->nCs = nC; c->canonical = false; c->last_repack_in_place = false;
-  c->up_mem = nullptr; c->up_bytes = 0;
+  c->up_mem = nullptr; c->up_bytes = 0; c->up_w2h_ready = false;
   c->cap_stream = nullptr; c->host_exec = nullptr; c->hg_off = false;
   c->g = cfg->n_q_heads / cfg->n_kv_heads;
   c->device = dev; c->n_sm = n_sm;
@@ -468,7 +469,8 @@ void swap_owned(lowram_cache* c, const void* old_p, void* new_p) {
 }
 
 // The re-pack scratch, carved from one allocation (256-byte aligned pieces): the error
-// words, the gathered tail chunk (when T > C), the encoder's outputs and its workspace.
+// words, the encoder's workspace, the gathered tail chunk (when T > C) and the encoder's
+// outputs.
 struct UpScratch {
   uint32_t* err;
   void* kg;
@@ -486,6 +488,7 @@ size_t carve_up(void* base, size_t gather, size_t coeff, size_t cscale, size_t s
     return n ? p : nullptr;
   };
   o->err = static_cast<uint32_t*>(take(16));
+  o->ws = take(ws);   // at a fixed offset: the fp16 W2 it keeps between re-packs stays put
   o->kg = take(gather);
   o->vg = take(gather);
   o->dst.coeff = take(coeff);
@@ -495,7 +498,6 @@ size_t carve_up(void* base, size_t gather, size_t coeff, size_t cscale, size_t s
   o->dst.res_pos = static_cast<uint16_t*>(take(rpos));
   o->dst.res_val = take(rval);
   o->dst.res_scale = take(rscale);
-  o->ws = take(ws);
   return off;
 }
 
@@ -537,6 +539,7 @@ lowram_status lowram_cache_repack(lowram_cache* c, int32_t n_resid, lowram_strea
     if (c->up_mem) cudaFree(c->up_mem);
     c->up_mem = nullptr;
     c->up_bytes = 0;
+    c->up_w2h_ready = false;
     cudaError_t ea = cudaMalloc(&c->up_mem, up_need);
     if (ea != cudaSuccess) {
       c->up_mem = nullptr;
@@ -577,8 +580,12 @@ lowram_status lowram_cache_repack(lowram_cache* c, int32_t n_resid, lowram_strea
   // 3. encode it
   const lowram_encode_dst dst = up.dst;
   void* ws = up.ws;
-  e = launch_encode(ge, f.store, n_resid, keys, vals, c->cb.basis, c->cb.w1, c->cb.w2, dst, ws, s);
+  // the cache's own folds of W1 (the encoder would compute the same), and W2 in fp16 kept
+  // in the scratch from the previous re-pack
+  e = launch_encode(ge, f.store, n_resid, keys, vals, c->cb.basis, c->cb.w1, c->cb.w2, dst, ws, s, c->w1f_t,
+                    i8 ? nullptr : c->w1f_tc, c->up_w2h_ready);
   if (e != cudaSuccess) return cuda_fail(e, "encode the new chunk");
+  c->up_w2h_ready = true;
 
   // 2-D copy of B*NG*H rows: `width` bytes from `from` (pitch spitch) to `to` (pitch dpitch)
   auto rows2d = [&](void* to, size_t dpitch, const void* from, size_t spitch, size_t width) {

@@ -935,7 +935,7 @@ EncWs carve(const Geom& g, void* workspace, size_t* bytes) {
 template <int R, int C, bool I8>
 cudaError_t launch_encode_t(const Geom& g, int n_res, const void* keys, const void* values,
                             const void* basis, const void* w2, const lowram_encode_dst& dst, const EncWs& w,
-                            cudaStream_t s) {
+                            bool w2h_ready, cudaStream_t s) {
   const int NG = g.L / g.G, nC = g.N / C;
   const size_t units = (size_t)g.B * g.L * g.Hkv;
   dim3 gc(nC, g.Hkv, g.B * NG), gr(nC, g.Hkv, g.B * g.L);
@@ -968,7 +968,8 @@ cudaError_t launch_encode_t(const Geom& g, int n_res, const void* keys, const vo
     if (!enc_make_map(&tmW1, w.w1f_tc, R, lh * kEncH, 128) || !enc_make_map(&tmW2, w.w2h, kEncH, lh * kEncD, 128) ||
         !enc_make_map(&tmA, dst.coeff, R, (uint64_t)g.B * NG * g.Hkv * g.N, C))
       return cudaErrorInvalidValue;
-    to_half_kernel<<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w2), w.w2h, (size_t)lh * kEncD * kEncH);
+    if (!w2h_ready)
+      to_half_kernel<<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w2), w.w2h, (size_t)lh * kEncD * kEncH);
     const unsigned grid = (unsigned)std::min<size_t>((size_t)n_sm, units * nC);
     auto k1 = enc_resid_tc_kernel<R, C, false>;
     auto k2 = enc_resid_tc_kernel<R, C, true>;
@@ -1026,17 +1027,29 @@ uint32_t* encode_error_word(const Geom& g, void* workspace) {
 cudaError_t launch_encode(const Geom& g, int store, int n_res, const void* keys, const void* values,
                           const void* basis, const void* w1, const void* w2, const lowram_encode_dst& dst,
                           void* workspace, cudaStream_t s) {
-  const EncWs w = carve(g, workspace, nullptr);
-  CacheBuffers cb{};
-  cb.w1 = w1;
-  cb.basis = basis;
-  cudaError_t e = launch_fold(g, cb, LOWRAM_BF16, LOWRAM_STORE_NATIVE, w.w1f_t, w.w1f_tc, s);
-  if (e != cudaSuccess) return e;
+  return launch_encode(g, store, n_res, keys, values, basis, w1, w2, dst, workspace, s, nullptr, nullptr, false);
+}
+
+cudaError_t launch_encode(const Geom& g, int store, int n_res, const void* keys, const void* values,
+                          const void* basis, const void* w1, const void* w2, const lowram_encode_dst& dst,
+                          void* workspace, cudaStream_t s, const float* w1f_t, const void* w1f_tc,
+                          bool w2h_ready) {
+  EncWs w = carve(g, workspace, nullptr);
   const bool i8 = store == LOWRAM_STORE_INT8;
-#define LOWRAM_ENC_CASE(RR, CC)                                                                    \
-  if (g.r == RR && g.C == CC)                                                                      \
-    return i8 ? launch_encode_t<RR, CC, true>(g, n_res, keys, values, basis, w2, dst, w, s)        \
-              : launch_encode_t<RR, CC, false>(g, n_res, keys, values, basis, w2, dst, w, s);
+  if (w1f_t && (i8 || w1f_tc)) {   // the caller's folds (the int8 path reads only the fp32 one)
+    w.w1f_t = const_cast<float*>(w1f_t);
+    if (!i8) w.w1f_tc = static_cast<__nv_bfloat16*>(const_cast<void*>(w1f_tc));
+  } else {
+    CacheBuffers cb{};
+    cb.w1 = w1;
+    cb.basis = basis;
+    cudaError_t e = launch_fold(g, cb, LOWRAM_BF16, LOWRAM_STORE_NATIVE, w.w1f_t, w.w1f_tc, s);
+    if (e != cudaSuccess) return e;
+  }
+#define LOWRAM_ENC_CASE(RR, CC)                                                                          \
+  if (g.r == RR && g.C == CC)                                                                            \
+    return i8 ? launch_encode_t<RR, CC, true>(g, n_res, keys, values, basis, w2, dst, w, w2h_ready, s)   \
+              : launch_encode_t<RR, CC, false>(g, n_res, keys, values, basis, w2, dst, w, w2h_ready, s);
   LOWRAM_ENC_CASE(128, 128)
   LOWRAM_ENC_CASE(128, 64)
   LOWRAM_ENC_CASE(64, 128)

@@ -13,6 +13,15 @@ constexpr uint32_t ERR_TAIL_FULL = 1u << 6;   // an append found a full tail: to
 // encoder's tensor-core kernels.
 uint32_t* encode_error_word(const Geom& g, void* workspace);
 
+// launch_encode with the folds a cache already holds: w1f_t the fp32 W1' = W1 B_l^T
+// [L][Hkv][r][h], w1f_tc its bf16 halves [L][Hkv][h][r] (native stores; unused for int8),
+// so the encoder does not fold again; w2h_ready: the workspace already holds the fp16 copy
+// of W2 from an earlier call with the same weights.
+cudaError_t launch_encode(const Geom& g, int store, int n_res, const void* keys, const void* values,
+                          const void* basis, const void* w1, const void* w2, const lowram_encode_dst& dst,
+                          void* workspace, cudaStream_t s, const float* w1f_t, const void* w1f_tc,
+                          bool w2h_ready);
+
 // A re-pack that cannot write the new chunk in place re-lays the cache with room for this
 // many more chunks per unit (and as many records per unit as this re-pack keeps per chunk):
 // max(kSpareChunksMin, live chunks / kSpareChunksDiv).

@@ -99,21 +99,23 @@ def _decode_check(lc, cfg2, arrays):
 @pytest.mark.parametrize("store,evict", [("native", 0.0), ("int8", 0.5)])
 def test_repeated_repacks_in_place_and_relaid(store, evict):
     """Six re-packs from one long tail: the first re-lays the cache with room for 4 more
-    chunks, the next four write in place, the sixth re-lays again.  Every new chunk is the
-    encoder's work on its tail segment; old chunks stay bit for bit; the cache decodes in
-    parity after an in-place re-pack and at the end."""
+    chunks, the next four write in place, the sixth re-lays again; the residual count per
+    chunk changes from call to call (the re-pack scratch, with the encoder's kept copy of
+    W2, is laid out again each time).  Every new chunk is the encoder's work on its tail
+    segment; old chunks stay bit for bit; the cache decodes in parity after an in-place
+    re-pack and at the end."""
     import oracle.encode as E
     C = 128
     cfg = S.LLAMA_32K.replace(name="repack6", batch=2, n_layers=4, n_kv_heads=2, n_ctx=512, top_k=2,
                               tail_cap=6 * C, store=store, evict_frac=evict)
-    n_res = 16
+    n_res_seq = [16, 8, 16, 8, 8, 16]
     cache = S.make_cache(cfg, tail_len=[6 * C, 6 * C])
     npc = S.cache_to_numpy(cache)
     lc = K.LowramCache.from_synth(cache.to(DEV))
     nL0 = cfg.n_live
     spares = []
     for i in range(6):
-        lc.repack(n_res)
+        lc.repack(n_res_seq[i])
         cfg2d, arrays = lc.view()
         spares.append(cfg2d["spare_chunks"])
         if i == 2:
@@ -128,10 +130,11 @@ def test_repeated_repacks_in_place_and_relaid(store, evict):
     assert np.array_equal(S._np_storage(arrays["summary"][:, :, :, :nL0]), npc["summary"])
     U = cfg.batch * cfg.n_layers * cfg.n_kv_heads
     rp = arrays["res_ptr"].cpu().numpy().astype(np.int64).reshape(U, -1)
-    _check_layout(rp, arrays, npc["res_pos"].shape[0] + 6 * U * n_res, 4 * n_res)
+    _check_layout(rp, arrays, npc["res_pos"].shape[0] + U * sum(n_res_seq), 4 * n_res_seq[-1])
     cfg_c = cfg.replace(name="repack_chunk", n_ctx=C, evict_frac=0.0)
     f64 = O._bf16_bits_to_f64
     for i in range(6):
+        n_res = n_res_seq[i]
         g_new = _new_chunk(arrays, cfg, nL0 + i, n_res)
         seg = slice(i * C, (i + 1) * C)
         args = (dataclasses.asdict(cfg_c), f64(npc["tail_k"][:, :, :, seg]), f64(npc["tail_v"][:, :, :, seg]),
