@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 import lowram_synth as S  # noqa: E402
 
 METRIC = "decode-attn queries/s over compressed KV at 32K ctx; achieved % of HBM roofline"
+NOMINAL_HBM_GBS = 8000.0   # the metric's roofline denominator (B200 HBM3e, nominal)
 DEFAULT_CONFIG = "llama8b_32k_bf16"
 
 
@@ -207,52 +208,55 @@ class ClockSampler:
 # ------------------------------------------------------------------- byte accounting
 
 def algorithmic_bytes(cfg, cache_host: dict, sel: np.ndarray, layer0: int, n_layers: int) -> dict:
-    """Bytes the method must move for one decode call, from the call's actual selection.
+    """Bytes the method must move for one decode call, counted per unit (sequence, layer, KV
+    head) by the hot path's byte formula, from the call's actual selection.
 
-    Per unit: the coefficient rows (+ int8 scales) of its selected chunks, the residual
-    records of those chunks (values, positions, int8 scales) and their CSR offsets, the raw
-    tail (actual lengths), q and out.  Once per (sequence, layer group, KV head): the chunk
-    summaries and the slot map; coefficient rows of a chunk selected by several layers of
-    one group are counted once.  Once per (layer, KV head): basis, folded W1' and W2.
+    Per unit: the chunk summaries it scores (n_live rows of r) and, with eviction, its slot
+    map; the coefficient rows of its k selected chunks (+ int8 row scales); the residual
+    records of those chunks (values, positions, int8 scales) and k+1 CSR offsets; its raw
+    tail (actual length); q and out.  Once per (layer, KV head): the basis, the folded W1'
+    (h x r, what the kernels read in place of W1) and W2.  "attend" is the chunk-attention
+    kernel's share: coefficient rows, records, offsets and W1'.  "unique_coeff" is for
+    reference only: the coefficient bytes if rows that several layers of one group select
+    were read once per group (the rows are shared by the group's layers).
     """
     B, Hkv, g, d, r, h = cfg.batch, cfg.n_kv_heads, cfg.q_per_kv, cfg.head_dim, cfg.rank, cfg.mlp_hidden
     C, k, T = cfg.chunk, cfg.top_k, cfg.tail_cap
     s = 4 if cfg.dtype == "f32" else 2
     i8 = cfg.store == "int8"
     sa = 1 if i8 else s
+    row_bytes = C * (r * sa + (2 if i8 else 0))
     res_ptr = cache_host["res_ptr"]
     slot = cache_host["slot"]
     tail_len = cache_host["tail_len"]
     coeff = 0
     resid = 0
-    ptrs = 0
     groups_seen = {}
     for li in range(n_layers):
         l = layer0 + li
         grp = l // cfg.group
         for b in range(B):
             for hk in range(Hkv):
-                key = (b, grp, hk)
-                chosen = groups_seen.setdefault(key, set())
+                chosen = groups_seen.setdefault((b, grp, hk), set())
                 for c in sel[li, b, hk]:
                     sl = int(slot[b, grp, hk, c])
                     chosen.add(sl)
                     n = int(res_ptr[b, l, hk, sl + 1] - res_ptr[b, l, hk, sl])
                     resid += n * (d * sa + 2 + (2 if i8 else 0))
-                ptrs += (k + 1) * 4
-    for key, chosen in groups_seen.items():
-        coeff += len(chosen) * C * (r * sa + (2 if i8 else 0))
+                coeff += k * row_bytes
     n_units = n_layers * B * Hkv
-    summaries = len(groups_seen) * cfg.n_live * r * s
-    slotmap = len(groups_seen) * cfg.n_chunks * 2 if cfg.n_live < cfg.n_chunks else 0
+    ptrs = n_units * (k + 1) * 4
+    unique_coeff = sum(len(ch) for ch in groups_seen.values()) * row_bytes
+    summaries = n_units * cfg.n_live * r * s
+    slotmap = n_units * cfg.n_chunks * 2 if cfg.n_live < cfg.n_chunks else 0
     tail = sum(2 * int(tail_len[b]) * d * (2 if i8 else s) for b in range(B)) * n_layers * Hkv
     qo = 2 * n_units * g * d * s
-    weights = n_layers * Hkv * (r * d * s + h * r * (2 if s == 2 else 4) + d * h * s)
     w1f = n_layers * Hkv * h * r * (2 if s == 2 else 4)
+    weights = n_layers * Hkv * (r * d * s + d * h * s) + w1f
     total = coeff + resid + ptrs + summaries + slotmap + tail + qo + weights
     attend = coeff + resid + ptrs + w1f
     return {"total": total, "attend": attend, "coeff": coeff, "residual": resid,
-            "summary": summaries, "tail": tail, "weights": weights}
+            "summary": summaries, "tail": tail, "weights": weights, "unique_coeff": unique_coeff}
 
 
 # ---------------------------------------------------------------------- CPU oracle leg
@@ -414,8 +418,12 @@ def run_lowram(args, ws, rank, local):
                      "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": ab["attend"],
                      "launch_ms": round(attend_ms, 4)},
+        # the metric's own roofline: the whole call's algorithmic bytes per step over the
+        # timed ms_per_step, against the nominal 8 TB/s and against the measured copy peak
         "call_roofline": {"algorithmic_bytes": ab["total"], "achieved_gbs": round(call_gbs, 1),
-                          "frac": round(call_gbs / peak, 4),
+                          "frac_of_8000_gbs": round(call_gbs / NOMINAL_HBM_GBS, 4),
+                          "frac_of_measured": round(call_gbs / peak, 4),
+                          "unique_coeff_bytes": ab["unique_coeff"],
                           "stage_ms": {"select_tail": round(stage_ms[0], 4),
                                        "attend": round(stage_ms[1], 4),
                                        "combine": round(stage_ms[2], 4)}},

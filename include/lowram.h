@@ -159,11 +159,17 @@ typedef struct {
                            int8 stores, 4 for F32) plus the same raw tail */
 } lowram_bytes;
 
-/* Execution path chosen by lowram_decode_attn. */
+/* Execution path of lowram_decode_attn.  There is one product path per shape: AUTO takes the
+ * tcgen05 kernel for every BF16 shape it serves and the CUDA-core kernel for the rest (every
+ * LOWRAM_F32 cache, and BF16 shapes the tensor-core kernel does not serve).  SIMT and TC only
+ * pin that choice.  SIMT on a cache AUTO would serve on tensor cores is a DIAGNOSTIC: a
+ * second, independent implementation (fp32 arithmetic, about 100x slower) that tests use to
+ * cross-check the tensor-core kernel; it is not a second backend to deploy. */
 typedef enum {
-  LOWRAM_PATH_AUTO = 0,  /* tensor-core path when the shapes allow it, else CUDA cores */
-  LOWRAM_PATH_SIMT = 1,  /* CUDA-core path (any shapes; the only path for LOWRAM_F32) */
-  LOWRAM_PATH_TC = 2     /* tcgen05 tensor-core path; LOWRAM_EUNSUPPORTED if shapes don't fit */
+  LOWRAM_PATH_AUTO = 0,  /* the product path: tensor cores when the shapes allow, else CUDA cores */
+  LOWRAM_PATH_SIMT = 1,  /* CUDA-core kernel (any shapes; the only one for LOWRAM_F32; for BF16
+                            shapes the tensor cores serve, a diagnostic cross-check) */
+  LOWRAM_PATH_TC = 2     /* tcgen05 tensor-core kernel; LOWRAM_EUNSUPPORTED if shapes don't fit */
 } lowram_path;
 
 /* Dense KV-cache bytes M_KV * B = 2 * L * Hkv * d * N * s * B ("LowRAM Compresses KV Cache
@@ -393,6 +399,31 @@ lowram_status lowram_encode(const lowram_config* cfg, int32_t n_resid, const voi
                             const void* values, const void* basis, const void* w1,
                             const void* w2, const lowram_encode_dst* dst, void* workspace,
                             uint64_t workspace_bytes, lowram_stream stream);
+
+/* ------------------------------------------------------------------- test hooks
+ *
+ * For tests of the failure paths only; a deployment never calls these.  They make a failure
+ * happen on the host side (an allocation reported as failed) or make a bounded wait in a
+ * kernel run out early; neither faults, traps or hangs the GPU.  The pages have no
+ * counterpart. */
+
+/* Limit, in SM clock cycles, of the main-loop waits of the tensor-core chunk-attention kernel
+ * in later lowram_decode_attn calls on this cache; cycles <= 0 restores the default (about
+ * one second).  A wait that runs out raises the kernel's error word and abort flag: every
+ * warp of that CTA stops, the CTA waits (with the default limit) for the copies and MMAs it
+ * has already issued, frees its tensor memory and returns, so the context stays usable.  The
+ * call's outputs are then meaningless and lowram_cache_validate returns LOWRAM_ETIMEOUT.  A
+ * limit of a few cycles makes the first wait that is not already satisfied run out.
+ * Drops the graph lowram_decode_attn_host keeps.  EINVAL for a NULL cache. */
+lowram_status lowram_debug_set_wait_limit(lowram_cache* cache, int64_t cycles);
+
+/* Inject one allocation failure: the next `after` device allocations made by
+ * lowram_cache_create or lowram_cache_repack succeed and the one after them fails as if
+ * cudaMalloc had run out of memory (those calls then return LOWRAM_ENOMEM, leaving no
+ * allocation behind; a failed re-pack leaves the cache as it was).  One-shot: the hook is
+ * off again after the failure.  after < 0 switches it off.  Process-wide; not meant for
+ * concurrent use. */
+void lowram_debug_fail_alloc(int32_t after);
 
 const char* lowram_status_string(lowram_status status);
 const char* lowram_last_error_string(void);

@@ -102,6 +102,8 @@ def lib() -> ctypes.CDLL:
         "lowram_encode_workspace_bytes": (U64, [ctypes.POINTER(LowramConfigC)]),
         "lowram_encode": (I32, [ctypes.POINTER(LowramConfigC), I32, P, P, P, P, P,
                                 ctypes.POINTER(LowramEncodeDstC), P, U64, P]),
+        "lowram_debug_set_wait_limit": (I32, [P, I64]),
+        "lowram_debug_fail_alloc": (None, [I32]),
         "lowram_status_string": (ctypes.c_char_p, [I32]),
         "lowram_last_error_string": (ctypes.c_char_p, []),
     }
@@ -288,6 +290,16 @@ def lowram_cache_last_launches(handle: int) -> int:
 
 def lowram_cache_last_path(handle: int) -> int:
     return int(lib().lowram_cache_last_path(handle))
+
+
+def lowram_debug_set_wait_limit(handle: int, cycles: int) -> None:
+    """Test hook: limit of the tensor-core kernel's main-loop waits (cycles <= 0: default)."""
+    _check(lib().lowram_debug_set_wait_limit(handle, int(cycles)), "lowram_debug_set_wait_limit")
+
+
+def lowram_debug_fail_alloc(after: int) -> None:
+    """Test hook: the device allocation after the next ``after`` ones fails (-1: off)."""
+    lib().lowram_debug_fail_alloc(int(after))
 
 
 def lowram_cache_append(handle: int, k_new, v_new, stream=None) -> None:

@@ -1,5 +1,6 @@
 // C ABI of the LowRAM decode library: cache object, argument checks, launches.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -40,6 +41,7 @@ struct lowram_cache {
   cudaEvent_t ev[4];
   bool ev_on;
   int last_launches, last_path;
+  long long wait_limit;        // main-loop wait limit of the tensor-core kernel (test hook)
 };
 
 namespace {
@@ -76,6 +78,10 @@ lowram_status check_config(const lowram_config* c) {
   if (c->head_dim > kMaxD || c->rank > kMaxR || c->mlp_hidden > kMaxH)
     return inval("head_dim/rank/mlp_hidden above the supported maximum (256/512/1024)");
   if (nC > kMaxChunks) return inval("more than 8192 chunks");
+  // the kernels index coefficient rows with 32-bit integers
+  if ((uint64_t)c->batch * (uint64_t)(c->n_layers / c->group) * (uint64_t)c->n_kv_heads * (uint64_t)c->n_live *
+          (uint64_t)c->chunk >= (1ull << 31))
+    return inval("coefficient rows batch * (n_layers / group) * n_kv_heads * n_live * chunk must stay below 2^31");
   if (c->tail_cap > kMaxTail) return inval("tail_cap exceeds 4096");
   if (c->dtype != LOWRAM_F32 && c->dtype != LOWRAM_BF16) return inval("unknown dtype");
   if (c->store != LOWRAM_STORE_NATIVE && c->store != LOWRAM_STORE_INT8) return inval("unknown store");
@@ -121,7 +127,26 @@ Geom make_geom(const lowram_cache* c, int layer0, int n_layers, bool tc) {
   g.tail_stride = (2 * g.g + g.g * g.d + 3) & ~3;
   g.max_rec = max_records_per_unit(total, g.P, g.k);
   g.qk_scale_log2 = 1.4426950408889634f / sqrtf((float)g.d);
+  g.wait_cycles = c->wait_limit;
   return g;
+}
+
+// Test hook (lowram_debug_fail_alloc): allocations still to succeed before one fails, or -1.
+std::atomic<int> g_fail_after{-1};
+
+// Every device allocation of the library goes through here.
+cudaError_t device_malloc(void** p, size_t bytes) {
+  int n = g_fail_after.load();
+  while (n >= 0) {
+    if (g_fail_after.compare_exchange_weak(n, n - 1)) {
+      if (n == 0) {   // the injected failure (the hook is now off again: the counter is -1)
+        *p = nullptr;
+        return cudaErrorMemoryAllocation;
+      }
+      break;
+    }
+  }
+  return cudaMalloc(p, bytes);
 }
 
 template <typename P>
@@ -132,7 +157,7 @@ lowram_status alloc(lowram_cache* c, P** out, size_t bytes) {
     g_last_error = "internal: too many owned allocations";
     return LOWRAM_ENOMEM;
   }
-  cudaError_t e = cudaMalloc(&p, bytes);
+  cudaError_t e = device_malloc(&p, bytes);
   if (e != cudaSuccess) {
     g_last_error = std::string("cudaMalloc: ") + cudaGetErrorString(e);
     return LOWRAM_ENOMEM;
@@ -211,6 +236,7 @@ lowram_status encode_geom(const lowram_config* cfg, Geom* g) {
   g->N = c->n_ctx; g->C = c->chunk; g->nC = nC; g->nL = nC; g->k = c->top_k; g->T = c->tail_cap;
   g->nLs = nC; g->nCs = nC;
   g->layer0 = 0; g->n_layers = c->n_layers;
+  g->wait_cycles = kDefaultWaitCycles;
   return LOWRAM_OK;
 }
 
@@ -289,6 +315,7 @@ lowram_status lowram_cache_create(const lowram_config* cfg, const lowram_cache_s
   c->g = cfg->n_q_heads / cfg->n_kv_heads;
   c->device = dev; c->n_sm = n_sm;
   c->s_dt = cfg->dtype == LOWRAM_F32 ? 4 : 2;
+  c->wait_limit = kDefaultWaitCycles;
 
   const size_t B = cfg->batch, L = cfg->n_layers, H = cfg->n_kv_heads, d = cfg->head_dim;
   const size_t r = cfg->rank, h = cfg->mlp_hidden, C = cfg->chunk, T = cfg->tail_cap;
@@ -440,7 +467,7 @@ struct RepackMem {
   template <typename P>
   lowram_status get(P** out, size_t bytes) {
     void* p = nullptr;
-    cudaError_t e = cudaMalloc(&p, bytes ? bytes : 16);
+    cudaError_t e = device_malloc(&p, bytes ? bytes : 16);
     if (e != cudaSuccess) {
       g_last_error = std::string("cudaMalloc: ") + cudaGetErrorString(e);
       return LOWRAM_ENOMEM;
@@ -532,7 +559,7 @@ lowram_status lowram_cache_repack(lowram_cache* c, int32_t n_resid, lowram_strea
   auto carve = [&](void* base) {
     return carve_up(base, T != C ? U * C * tail_row : 0, B * NG * H * C * r * sa, i8 ? B * NG * H * C * 2 : 0,
                     B * NG * H * r * 2, U * 2 * 4, n_new * 2, n_new * d * sa, i8 ? n_new * 2 : 0,
-                    encode_workspace_bytes(ge), &up);
+                    encode_workspace_bytes(ge, true), &up);
   };
   const size_t up_need = carve(nullptr);
   if (up_need > c->up_bytes) {
@@ -540,7 +567,7 @@ lowram_status lowram_cache_repack(lowram_cache* c, int32_t n_resid, lowram_strea
     c->up_mem = nullptr;
     c->up_bytes = 0;
     c->up_w2h_ready = false;
-    cudaError_t ea = cudaMalloc(&c->up_mem, up_need);
+    cudaError_t ea = device_malloc(&c->up_mem, up_need);
     if (ea != cudaSuccess) {
       c->up_mem = nullptr;
       g_last_error = std::string("cudaMalloc: ") + cudaGetErrorString(ea);
@@ -662,7 +689,7 @@ lowram_status lowram_cache_repack(lowram_cache* c, int32_t n_resid, lowram_strea
   }
   uint32_t word = 0, enc_word = 0;
   e = cudaMemcpyAsync(&word, err, 4, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(&enc_word, encode_error_word(ge, ws), 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&enc_word, encode_error_word(ge, ws, true), 4, cudaMemcpyDeviceToHost, s);
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "re-lay the residual records");
   word |= enc_word;
@@ -733,7 +760,8 @@ int32_t lowram_cache_last_path(const lowram_cache* c) { return c ? c->last_path 
 
 static lowram_status check_layers(const lowram_cache* c, int32_t layer0, int32_t n_layers) {
   if (!c) return inval("NULL cache");
-  if (layer0 < 0 || n_layers < 1 || layer0 + n_layers > c->cfg.n_layers)
+  // written so that no sum can overflow: layer0 >= 0 first, then n_layers against the rest
+  if (layer0 < 0 || n_layers < 1 || layer0 >= c->cfg.n_layers || n_layers > c->cfg.n_layers - layer0)
     return inval("layer range outside the cache");
   return LOWRAM_OK;
 }
@@ -781,7 +809,7 @@ lowram_status lowram_decode_attn(lowram_cache* c, int32_t layer0, int32_t n_laye
   if (tc)
     e = launch_attend_tc(g, c->cb, c->sc, c->cfg.store, c->w1f_tc, c->n_sm, s);
   else
-    e = launch_attend_simt(g, c->cb, c->sc, c->cfg.dtype, c->cfg.store, c->w1f_t, s);
+    e = launch_attend_simt(g, c->cb, c->sc, c->cfg.dtype, c->cfg.store, c->w1f_t, 0, s);
   if (e != cudaSuccess) return cuda_fail(e, "chunk attention kernel");
   if (c->ev_on && (e = cudaEventRecord(c->ev[2], s)) != cudaSuccess) return cuda_fail(e, "event");
   e = launch_combine(g, c->cb, c->sc, c->cfg.dtype, out, s);
@@ -884,5 +912,17 @@ lowram_status lowram_cache_validate(lowram_cache* c, lowram_stream stream) {
   }
   return LOWRAM_OK;
 }
+
+lowram_status lowram_debug_set_wait_limit(lowram_cache* c, int64_t cycles) {
+  if (!c) return inval("NULL cache");
+  c->wait_limit = cycles > 0 ? (long long)cycles : kDefaultWaitCycles;
+  if (c->host_exec) {   // the captured graph holds the old limit
+    cudaGraphExecDestroy(c->host_exec);
+    c->host_exec = nullptr;
+  }
+  return LOWRAM_OK;
+}
+
+void lowram_debug_fail_alloc(int32_t after) { g_fail_after.store(after < 0 ? -1 : after); }
 
 }  // extern "C"

@@ -28,7 +28,7 @@ __device__ __forceinline__ float silu_f(float x) { return x / (1.f + __expf(-x))
 
 template <typename T, bool INT8>
 __global__ void __launch_bounds__(kThreads)
-attend_simt_kernel(Geom g, CacheBuffers cb, Scratch sc, const float* __restrict__ w1f_t) {
+attend_simt_kernel(Geom g, CacheBuffers cb, Scratch sc, const float* __restrict__ w1f_t, int w1f_layer0) {
   extern __shared__ __align__(16) float sm[];
   const int rp = g.r + 1;                       // padded row (bank-conflict free)
   float* a_s = sm;                              // [kTB][rp]
@@ -78,9 +78,17 @@ attend_simt_kernel(Geom g, CacheBuffers cb, Scratch sc, const float* __restrict_
     const size_t row0 = ((((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * g.nLs + slot) * g.C;
     const T* coeff = reinterpret_cast<const T*>(cb.coeff);
     const int8_t* coeff8 = reinterpret_cast<const int8_t*>(cb.coeff);
-    const float* w1 = w1f_t + ((size_t)l * g.Hkv + un.hkv) * g.r * g.h;
+    const float* w1 = w1f_t + ((size_t)(l - w1f_layer0) * g.Hkv + un.hkv) * g.r * g.h;
     const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nLs + 1);
-    const int rec0 = rptr[slot], rec1 = rptr[slot + 1];
+    // a record range outside [0, n_records] (a corrupt CSR table; the caller's own arrays on
+    // the allocation-free path are never validated) is clamped and reported, so no record
+    // read leaves the arrays
+    int rec0 = rptr[slot], rec1 = rptr[slot + 1];
+    if (rec0 < 0 || rec1 < rec0 || (long long)rec1 > cb.n_records) {
+      if (tid == 0) atomicOr(sc.err, ERR_RES_PTR);
+      rec0 = (int)max(0ll, min((long long)rec0, (long long)cb.n_records));
+      rec1 = (int)max((long long)rec0, min((long long)rec1, (long long)cb.n_records));
+    }
 
     for (int t0 = 0; t0 < g.C; t0 += kTB) {
       const int nb = min(kTB, g.C - t0);
@@ -179,7 +187,8 @@ size_t simt_smem_bytes(const Geom& g) {
 }  // namespace
 
 cudaError_t launch_attend_simt(const Geom& g, const CacheBuffers& cb, const Scratch& sc,
-                               int dtype, int store, const float* w1f_t, cudaStream_t s) {
+                               int dtype, int store, const float* w1f_t, int w1f_layer0,
+                               cudaStream_t s) {
   const size_t smem = simt_smem_bytes(g);
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   cudaError_t e;
@@ -187,17 +196,17 @@ cudaError_t launch_attend_simt(const Geom& g, const CacheBuffers& cb, const Scra
     auto k = attend_simt_kernel<float, false>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<g.P, kThreads, smem, s>>>(g, cb, sc, w1f_t);
+    k<<<g.P, kThreads, smem, s>>>(g, cb, sc, w1f_t, w1f_layer0);
   } else if (store == LOWRAM_STORE_INT8) {
     auto k = attend_simt_kernel<__nv_bfloat16, true>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<g.P, kThreads, smem, s>>>(g, cb, sc, w1f_t);
+    k<<<g.P, kThreads, smem, s>>>(g, cb, sc, w1f_t, w1f_layer0);
   } else {
     auto k = attend_simt_kernel<__nv_bfloat16, false>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k<<<g.P, kThreads, smem, s>>>(g, cb, sc, w1f_t);
+    k<<<g.P, kThreads, smem, s>>>(g, cb, sc, w1f_t, w1f_layer0);
   }
   return cudaGetLastError();
 }

@@ -214,6 +214,8 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
   const int NS = NCH * SUBS;
   const int NG = g.L / g.G;
   uint32_t* err = sc.err;
+  // limit of the main-loop waits (the drain waits at an abort keep the full kWaitCycles)
+  const long long wlim = g.wait_cycles;
 
   // ------------------------------------------------------------------ set-up
   if (tid == 0) {
@@ -291,7 +293,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
           prev_u = u;
           const int qb = unit_i & 1;
           if (unit_i >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar.q_empty[qb], ((unit_i >> 1) - 1) & 1,
-                                                                abort_flag, err, ERR_TIMEOUT)))
+                                                                abort_flag, err, ERR_TIMEOUT, wlim)))
             break;
           if (leader) {
             mbar_expect_tx(&bar.q_full[qb], 16 * R * 2);
@@ -306,10 +308,10 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
         const uint32_t par = ((ci / STAGES) - 1) & 1;
         if (I8) {   // the int8 tile goes to the staging ring; the converters fill stage st
           if (ci >= 2 && !__all_sync(0xffffffffu, mbar_wait(&bar.stg_empty[s2], ((ci >> 1) - 1) & 1, abort_flag,
-                                                            err, ERR_TIMEOUT)))
+                                                            err, ERR_TIMEOUT, wlim)))
             break;
         } else if (ci >= STAGES &&
-                   !__all_sync(0xffffffffu, mbar_wait(&bar.a_empty[st], par, abort_flag, err, ERR_TIMEOUT))) {
+                   !__all_sync(0xffffffffu, mbar_wait(&bar.a_empty[st], par, abort_flag, err, ERR_TIMEOUT, wlim))) {
           break;
         }
         const Unit un = unit_of(g, u);
@@ -339,7 +341,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
           ++seg_i;
           prev_seg = wk.seg;
           if (seg_i > 0 && !__all_sync(0xffffffffu, mbar_wait(&bar.seg_done, (seg_i - 1) & 1, abort_flag, err,
-                                                              ERR_TIMEOUT)))
+                                                              ERR_TIMEOUT, wlim)))
             break;
           if (leader) {
             mbar_expect_tx(&bar.w1_ready, (uint32_t)(2 * Lay::W_HALF));
@@ -355,14 +357,19 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
           w1_issued = seg_i + 1;
         }
         const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nLs + 1);
-        const int r0 = rptr[slot], r1 = rptr[slot + 1];
+        int r0 = rptr[slot], r1 = rptr[slot + 1];
+        if (r0 < 0 || r1 < r0 || (long long)r1 > cb.n_records) {   // corrupt CSR offsets: clamp, report
+          if (lane == 0) atomicOr(err, ERR_RES_PTR);
+          r0 = (int)max(0ll, min((long long)r0, (long long)cb.n_records));
+          r1 = (int)max((long long)r0, min((long long)r1, (long long)cb.n_records));
+        }
         const int nres = min(r1 - r0, kResCap);
         const int my_pos = lane < nres ? (int)cb.res_pos[r0 + lane] : C;
         const __half my_rs = (I8 && lane < nres) ? cb.res_scale[r0 + lane] : __ushort_as_half((unsigned short)0);
-        if (ci >= STAGES && !__all_sync(0xffffffffu, mbar_wait(&bar.r_empty[st], par, abort_flag, err, ERR_TIMEOUT)))
+        if (ci >= STAGES && !__all_sync(0xffffffffu, mbar_wait(&bar.r_empty[st], par, abort_flag, err, ERR_TIMEOUT, wlim)))
           break;
         if (I8 && ci >= 2 &&
-            !__all_sync(0xffffffffu, mbar_wait(&bar.rstg_empty[s2], ((ci >> 1) - 1) & 1, abort_flag, err, ERR_TIMEOUT)))
+            !__all_sync(0xffffffffu, mbar_wait(&bar.rstg_empty[s2], ((ci >> 1) - 1) & 1, abort_flag, err, ERR_TIMEOUT, wlim)))
           break;
         if (I8) misc->stage_rs[st][lane] = my_rs;
         // record range and token -> record map for the softmax warps (published by the
@@ -433,7 +440,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
       TileWalk wk;
       wk.init(x0, g.k, g.B);
       auto wait_all = [&](uint64_t* b, uint32_t par) -> bool {
-        return __all_sync(0xffffffffu, mbar_wait(b, par, abort_flag, err, ERR_TIMEOUT));
+        return __all_sync(0xffffffffu, mbar_wait(b, par, abort_flag, err, ERR_TIMEOUT, wlim));
       };
       // Pre-activations of sub-tile n (hidden half hh = n % 2 of chunk n / 2) into D1 buffer
       // n % 3; hidden half 0 also carries the chunk's scores (two accumulation chains
@@ -580,7 +587,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
       const uint64_t dPR0 = smem_desc(sPR, 128, Lay::PR_SBO, 0);    // probabilities at records
       const uint32_t t_d1 = tmem + Lay::T_D1, t_d3 = tmem + Lay::T_D3, t_d4 = tmem + Lay::T_D4;
       auto wait_all = [&](uint64_t* b, uint32_t par) -> bool {
-        return __all_sync(0xffffffffu, mbar_wait(b, par, abort_flag, err, ERR_TIMEOUT));
+        return __all_sync(0xffffffffu, mbar_wait(b, par, abort_flag, err, ERR_TIMEOUT, wlim));
       };
       bool ok = true;
       for (int ci = 0; ok && ci < NCH; ++ci) {
@@ -631,9 +638,9 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
     bool ok = true;
     for (int ci = 0; ok && ci < NCH; ++ci) {
       const int st = ci % STAGES, s2 = ci & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&bar.stg_full[s2], (ci >> 1) & 1, abort_flag, err, ERR_TIMEOUT));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar.stg_full[s2], (ci >> 1) & 1, abort_flag, err, ERR_TIMEOUT, wlim));
       if (ok && ci >= STAGES)
-        ok = __all_sync(0xffffffffu, mbar_wait(&bar.a_empty[st], ((ci / STAGES) - 1) & 1, abort_flag, err, ERR_TIMEOUT));
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar.a_empty[st], ((ci / STAGES) - 1) & 1, abort_flag, err, ERR_TIMEOUT, wlim));
       if (!ok) break;
       {
         const unsigned char* src = smem + Lay::OFF_SA + s2 * Lay::SA_SLOT;
@@ -661,9 +668,9 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
         mbar_arrive(&bar.stg_empty[s2]);
         mbar_arrive(&bar.a_full[st]);
       }
-      ok = __all_sync(0xffffffffu, mbar_wait(&bar.rstg_full[s2], (ci >> 1) & 1, abort_flag, err, ERR_TIMEOUT));
+      ok = __all_sync(0xffffffffu, mbar_wait(&bar.rstg_full[s2], (ci >> 1) & 1, abort_flag, err, ERR_TIMEOUT, wlim));
       if (ok && ci >= STAGES)
-        ok = __all_sync(0xffffffffu, mbar_wait(&bar.r_empty[st], ((ci / STAGES) - 1) & 1, abort_flag, err, ERR_TIMEOUT));
+        ok = __all_sync(0xffffffffu, mbar_wait(&bar.r_empty[st], ((ci / STAGES) - 1) & 1, abort_flag, err, ERR_TIMEOUT, wlim));
       if (!ok) break;
       {
         const unsigned char* src = smem + Lay::OFF_SR + s2 * Lay::SR_SLOT;
@@ -699,7 +706,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
     const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
     for (int n = grp_ab; n < NS; n += 2) {
       const int bf = n % NBUF;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bar.d1_full[bf], (n / NBUF) & 1, abort_flag, err, ERR_TIMEOUT)))
+      if (!__all_sync(0xffffffffu, mbar_wait(&bar.d1_full[bf], (n / NBUF) & 1, abort_flag, err, ERR_TIMEOUT, wlim)))
         break;
       tc_fence_after();
       // 64 tokens at a time: their fp32 pre-activations (64 columns) in, their H (fp16
@@ -755,7 +762,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
     // fold D3 / D4 of chunk c (sums relative to the running max after c) into the totals
     auto fold = [&](int c) {
       const int pb = c & 1;
-      live = __all_sync(0xffffffffu, live && mbar_wait(&bar.d3_full[pb], (c >> 1) & 1, abort_flag, err, ERR_TIMEOUT));
+      live = __all_sync(0xffffffffu, live && mbar_wait(&bar.d3_full[pb], (c >> 1) & 1, abort_flag, err, ERR_TIMEOUT, wlim));
       if (!live) return;
       tc_fence_after();
       uint32_t v0[16], v1[16], v4[16];
@@ -800,8 +807,8 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
         cur_u = u;
       }
       const int st = ci % STAGES, sb = ci & 1, pb = ci & 1;
-      live = __all_sync(0xffffffffu, live && mbar_wait(&bar.r_full[st], (ci / STAGES) & 1, abort_flag, err, ERR_TIMEOUT) &&
-                                         mbar_wait(&bar.s_full[sb], (ci >> 1) & 1, abort_flag, err, ERR_TIMEOUT));
+      live = __all_sync(0xffffffffu, live && mbar_wait(&bar.r_full[st], (ci / STAGES) & 1, abort_flag, err, ERR_TIMEOUT, wlim) &&
+                                         mbar_wait(&bar.s_full[sb], (ci >> 1) & 1, abort_flag, err, ERR_TIMEOUT, wlim));
       uint32_t sv[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) sv[j] = 0u;

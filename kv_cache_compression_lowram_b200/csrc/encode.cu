@@ -912,7 +912,9 @@ struct EncWs {
   uint32_t* err;           // device error word of the tensor-core kernels
 };
 
-EncWs carve(const Geom& g, void* workspace, size_t* bytes) {
+// With folds_given the caller supplies both W1' folds, so their regions are left out (the
+// pointers stay null until launch_encode points them at the caller's arrays).
+EncWs carve(const Geom& g, void* workspace, size_t* bytes, bool folds_given) {
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
   const size_t units = (size_t)g.B * g.L * g.Hkv, lh = (size_t)g.L * g.Hkv;
   size_t off = 0;
@@ -922,8 +924,8 @@ EncWs carve(const Geom& g, void* workspace, size_t* bytes) {
     return p;
   };
   EncWs w;
-  w.w1f_t = reinterpret_cast<float*>(take(lh * g.r * g.h * 4));
-  w.w1f_tc = reinterpret_cast<__nv_bfloat16*>(take(lh * g.h * g.r * 2));
+  w.w1f_t = folds_given ? nullptr : reinterpret_cast<float*>(take(lh * g.r * g.h * 4));
+  w.w1f_tc = folds_given ? nullptr : reinterpret_cast<__nv_bfloat16*>(take(lh * g.h * g.r * 2));
   w.w2h = reinterpret_cast<__half*>(take(lh * g.d * g.h * 2));
   w.norms = reinterpret_cast<float*>(take(units * g.N * 4));
   w.flags = take(units * g.N);
@@ -1013,15 +1015,15 @@ cudaError_t launch_encode_t(const Geom& g, int n_res, const void* keys, const vo
 
 }  // namespace
 
-size_t encode_workspace_bytes(const Geom& g) {
+size_t encode_workspace_bytes(const Geom& g, bool folds_given) {
   size_t bytes = 0;
-  carve(g, nullptr, &bytes);
+  carve(g, nullptr, &bytes, folds_given);
   return bytes;
 }
 
-uint32_t* encode_error_word(const Geom& g, void* workspace) {
+uint32_t* encode_error_word(const Geom& g, void* workspace, bool folds_given) {
   size_t bytes = 0;
-  return carve(g, workspace, &bytes).err;
+  return carve(g, workspace, &bytes, folds_given).err;
 }
 
 cudaError_t launch_encode(const Geom& g, int store, int n_res, const void* keys, const void* values,
@@ -1034,9 +1036,10 @@ cudaError_t launch_encode(const Geom& g, int store, int n_res, const void* keys,
                           const void* basis, const void* w1, const void* w2, const lowram_encode_dst& dst,
                           void* workspace, cudaStream_t s, const float* w1f_t, const void* w1f_tc,
                           bool w2h_ready) {
-  EncWs w = carve(g, workspace, nullptr);
   const bool i8 = store == LOWRAM_STORE_INT8;
-  if (w1f_t && (i8 || w1f_tc)) {   // the caller's folds (the int8 path reads only the fp32 one)
+  const bool folds_given = w1f_t && (i8 || w1f_tc);
+  EncWs w = carve(g, workspace, nullptr, folds_given);
+  if (folds_given) {   // the caller's folds (the int8 path reads only the fp32 one)
     w.w1f_t = const_cast<float*>(w1f_t);
     if (!i8) w.w1f_tc = static_cast<__nv_bfloat16*>(const_cast<void*>(w1f_tc));
   } else {

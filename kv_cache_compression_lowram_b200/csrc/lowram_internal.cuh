@@ -40,7 +40,11 @@ struct Geom {
   int tail_stride;     // floats per tail partial record
   int max_rec;         // upper bound of chunk records per unit (CTAs a unit's tiles touch)
   float qk_scale_log2; // log2(e) / sqrt(d)
+  long long wait_cycles;  // limit of the tensor-core kernel's main-loop waits (SM cycles)
 };
+
+// Default limit of a bounded wait inside a kernel: about one second of SM clock.
+constexpr long long kDefaultWaitCycles = 2000000000LL;
 
 // Unit u enumerates (layer, KV head, sequence) with the sequence fastest, so the units
 // that share one layer's weights are adjacent.
@@ -139,9 +143,11 @@ __device__ __forceinline__ float warp_max(float v) {
 cudaError_t launch_select(const Geom& g, const CacheBuffers& cb, const Scratch& sc,
                           int dtype, const void* q, float* scores_out, int32_t* sel_out,
                           int tc_q_mode, bool tail, cudaStream_t s);
-// Steps 3-5 on CUDA cores over the selected chunks.
+// Steps 3-5 on CUDA cores over the selected chunks.  w1f_t holds the fp32 W1' of layers
+// [w1f_layer0, ...): layer l's fold is at (l - w1f_layer0) * Hkv * r * h.
 cudaError_t launch_attend_simt(const Geom& g, const CacheBuffers& cb, const Scratch& sc,
-                               int dtype, int store, const float* w1f_t, cudaStream_t s);
+                               int dtype, int store, const float* w1f_t, int w1f_layer0,
+                               cudaStream_t s);
 // Steps 3-5 on tcgen05 tensor cores.  Returns cudaErrorNotSupported for shapes it
 // does not handle.
 cudaError_t launch_attend_tc(const Geom& g, const CacheBuffers& cb, const Scratch& sc,
@@ -156,8 +162,9 @@ cudaError_t launch_fold(const Geom& g, const CacheBuffers& cb, int dtype, int st
                         float* w1f_t, void* w1f_tc, cudaStream_t s);
 // Prefill-side encoder (dense K, V -> compressed arrays); bf16, d = 128, h = 256,
 // r in {64, 128}, C in {64, 128}.  The workspace holds the fp32 W1' fold, the residual
-// norms and the flags.
-size_t encode_workspace_bytes(const Geom& g);
+// norms and the flags; with folds_given (the caller passes both W1' folds, as the re-pack
+// does) the fold regions are left out.
+size_t encode_workspace_bytes(const Geom& g, bool folds_given = false);
 cudaError_t launch_encode(const Geom& g, int store, int n_res, const void* keys, const void* values,
                           const void* basis, const void* w1, const void* w2, const lowram_encode_dst& dst,
                           void* workspace, cudaStream_t s);

@@ -74,7 +74,7 @@ extern "C" lowram_status lowram_decode_attn_static(const lowram_config* cfg,
   lowram_status st = lowram_config_bytes(cfg, src ? src->n_records : 0, 0, &nb);  // shape checks
   if (st != LOWRAM_OK) return st;
   if (!src || !q || !out) return fail_inval("NULL src, q or out");
-  if (layer0 < 0 || n_layers < 1 || layer0 + n_layers > cfg->n_layers)
+  if (layer0 < 0 || n_layers < 1 || layer0 >= cfg->n_layers || n_layers > cfg->n_layers - layer0)
     return fail_inval("layer range outside the cache");
   const bool i8 = cfg->store == LOWRAM_STORE_INT8;
   const int nC = cfg->n_ctx / cfg->chunk;
@@ -108,6 +108,7 @@ extern "C" lowram_status lowram_decode_attn_static(const lowram_config* cfg,
   g.tail_stride = (2 * g.g + g.g * g.d + 3) & ~3;
   g.max_rec = max_records_per_unit(total, g.P, g.k);
   g.qk_scale_log2 = 1.4426950408889634f / sqrtf((float)g.d);
+  g.wait_cycles = kDefaultWaitCycles;
 
   // carve the static array: error word, folded W1' of the requested layers, projected
   // queries, selection, split partials, tail partials
@@ -162,13 +163,11 @@ extern "C" lowram_status lowram_decode_attn_static(const lowram_config* cfg,
   float* w1f = reinterpret_cast<float*>(sb + o_w1f);
   e = launch_fold(gf, cbf, cfg->dtype, cfg->store, w1f, nullptr, s);
   if (e != cudaSuccess) return fail_cuda(e, "fold kernel");
-  // the chunk kernel indexes W1' by absolute layer; it only reads layers >= layer0
-  const float* w1f_abs = reinterpret_cast<const float*>(
-      reinterpret_cast<uintptr_t>(w1f) - (uintptr_t)layer0 * g.Hkv * g.r * g.h * sizeof(float));
 
   e = launch_select(g, cb, sc, cfg->dtype, q, nullptr, sel, 0, true, s);
   if (e != cudaSuccess) return fail_cuda(e, "select kernel");
-  e = launch_attend_simt(g, cb, sc, cfg->dtype, cfg->store, w1f_abs, s);
+  // w1f holds layers [layer0, layer0 + n_layers): the kernel indexes it from layer0
+  e = launch_attend_simt(g, cb, sc, cfg->dtype, cfg->store, w1f, layer0, s);
   if (e != cudaSuccess) return fail_cuda(e, "chunk attention kernel");
   e = launch_combine(g, cb, sc, cfg->dtype, out, s);
   if (e != cudaSuccess) return fail_cuda(e, "combine kernel");

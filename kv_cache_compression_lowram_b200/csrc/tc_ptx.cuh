@@ -42,15 +42,16 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait for the phase with the given parity to complete.  Returns false (and raises the
-// CTA's abort flag and the device error word) if it does not within kWaitCycles, or as
-// soon as another thread has raised the abort flag.
+// CTA's abort flag and the device error word) if it does not within `limit` cycles
+// (kWaitCycles unless the caller gives less), or as soon as another thread has raised the
+// abort flag.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* err, uint32_t err_bit) {
+                                          uint32_t* err, uint32_t err_bit, long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       atomicOr(err, err_bit);
       return false;

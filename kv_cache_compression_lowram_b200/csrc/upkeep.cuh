@@ -11,7 +11,7 @@ constexpr uint32_t ERR_TAIL_FULL = 1u << 6;   // an append found a full tail: to
 
 // The error word inside an encoder workspace (encode.cu): bounded-wait timeouts of the
 // encoder's tensor-core kernels.
-uint32_t* encode_error_word(const Geom& g, void* workspace);
+uint32_t* encode_error_word(const Geom& g, void* workspace, bool folds_given = false);
 
 // launch_encode with the folds a cache already holds: w1f_t the fp32 W1' = W1 B_l^T
 // [L][Hkv][r][h], w1f_tc its bf16 halves [L][Hkv][h][r] (native stores; unused for int8),

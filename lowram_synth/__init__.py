@@ -586,6 +586,42 @@ def make_queries(cache: SynthCache, layer0: int = 0, n_layers: Optional[int] = N
     return out.to(cfg.torch_dtype)
 
 
+def select_sequences(cache: SynthCache, seqs, device="cpu") -> SynthCache:
+    """The cache of sequences ``seqs`` alone (in that order), on ``device``.
+
+    Every per-sequence array keeps only those sequences; the residual records of each kept
+    sequence (a contiguous range: records are laid out sequence by sequence) are gathered
+    and the CSR offsets rebased.  Used to check a large batch against the oracle on a few
+    sequences without copying the whole cache to the host.
+    """
+    seqs = [int(b) for b in seqs]
+    idx = torch.as_tensor(seqs, device=cache.coeff.device)
+    rp = cache.res_ptr.to(torch.int64)
+    spans = [(int(rp[b].min()), int(rp[b].max())) for b in seqs]
+    rec_idx = torch.cat([torch.arange(a, e, device=cache.res_pos.device) for a, e in spans]) \
+        if spans else torch.empty(0, dtype=torch.int64, device=cache.res_pos.device)
+    new_rp = []
+    base = 0
+    for b, (a, e) in zip(seqs, spans):
+        new_rp.append(rp[b] - a + base)
+        base += e - a
+    res_ptr = torch.stack(new_rp).to(torch.int32)
+
+    def rows(t):
+        return None if t is None else t.index_select(0, idx).to(device)
+
+    def recs(t):
+        return None if t is None else t.index_select(0, rec_idx).to(device)
+
+    return SynthCache(
+        cfg=cache.cfg.replace(name=cache.cfg.name + "_seqs", batch=len(seqs)),
+        coeff=rows(cache.coeff), coeff_scale=rows(cache.coeff_scale), basis=cache.basis.to(device),
+        w1=cache.w1.to(device), w2=cache.w2.to(device), summary=rows(cache.summary),
+        slot=rows(cache.slot), res_ptr=res_ptr.to(device), res_pos=recs(cache.res_pos),
+        res_val=recs(cache.res_val), res_scale=recs(cache.res_scale), tail_k=rows(cache.tail_k),
+        tail_v=rows(cache.tail_v), tail_len=rows(cache.tail_len))
+
+
 # ------------------------------------------------------------------------ numpy export
 
 def _np_storage(t: Optional[torch.Tensor]):

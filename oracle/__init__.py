@@ -20,7 +20,7 @@ Every function cites the passage it follows.  Page names used below:
   context split into fragments, the ones that fit the current query chosen; tokens
   generated after prefill kept uncompressed.
 
-Readings where the pages are silent (each is listed with its reason in the design doc):
+Readings where the pages are silent (each a reading this library takes, not a page's rule):
 the chunk summary is the mean of the chunk's coefficient rows, so the chunk's mean key at
 layer l is abar_c . B_l, and a chunk's score is sum_j q_j . kbar_c / sqrt(d); selection is
 per (b, l, KV head) and ties go to the lower chunk id; the predictor is

@@ -8,7 +8,7 @@ Pages (names as in ``oracle/__init__.py``): [Rit] keeps the tokens generated aft
 uncompressed (the raw tail); [Abstract] and [Asym] compress a context with a given basis
 and predictor (coefficients on the group basis, Vhat = f(K), residuals kept for the worst
 tokens).  The pages name no moment at which new tokens join the compressed store; this
-library's reading (listed with its reason in the design doc): once every sequence's tail holds
+library's reading (no page fixes it; it is the plainest one): once every sequence's tail holds
 at least C tokens, the oldest C tail tokens of every (sequence, layer, KV head) are encoded
 by the encoder's steps (``oracle.encode``) as one new chunk, appended after the existing
 chunks (a new live chunk when the cache evicts), and removed from the tail.

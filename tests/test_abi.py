@@ -64,6 +64,7 @@ def test_bad_configs_rejected_on_host():
         dict(rank=10_000),
         dict(dtype="f32", store="int8"),
         dict(batch=0),
+        dict(batch=70_000),          # coefficient rows above 2^31 (32-bit row indices)
     ]
     for kw in bad:
         cfg = S.LLAMA_32K.replace(**kw)
@@ -127,3 +128,12 @@ def test_upkeep_host_checks():
     assert lib.lowram_cache_view(None, ctypes.byref(cfg), ctypes.byref(src), ctypes.byref(spare)) == 1
     assert lib.lowram_cache_append(None, None, None, None) == 1
     assert lib.lowram_cache_repack(None, 4, None) == 1
+
+
+def test_test_hooks_host_side():
+    """The failure-path hooks: NULL caches are rejected and the allocation hook can be armed
+    and disarmed without a device (it only counts allocations)."""
+    lib = K.lib()
+    assert lib.lowram_debug_set_wait_limit(None, 5) == 1
+    K.lowram_debug_fail_alloc(3)
+    K.lowram_debug_fail_alloc(-1)

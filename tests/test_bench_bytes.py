@@ -1,9 +1,10 @@
 """The roofline numerator of bench.py (algorithmic bytes of one decode call) against the
-per-unit byte count written out here: per unit, the coefficient rows of its k selected chunks,
-their residual records (row + position) and k+1 CSR offsets, its raw tail, q and out; per
-(sequence, layer group, KV head), the chunk summaries (coefficient space, r per chunk); per
-(layer, KV head), the basis, the folded W1' and W2.  Coefficient rows of a chunk chosen by
-several layers of one group are read once.  CPU only."""
+per-unit byte count written out here: per unit, the chunk summaries it scores (coefficient
+space, r per chunk), the coefficient rows of its k selected chunks, their residual records
+(row + position) and k+1 CSR offsets, its raw tail, q and out; per (layer, KV head), the
+basis, the folded W1' and W2.  Every unit's rows count, also when several layers of one group
+select the same chunk (the formula counts per unit); the once-per-group count is reported
+beside it.  CPU only."""
 
 import numpy as np
 
@@ -33,9 +34,9 @@ def _expected(cfg, counts, sel, tail_len, shared_rows):
             for hk in range(H):
                 per_unit += sum(int(counts[b, l, hk, c]) for c in sel[l, b, hk]) * (d * s + 2)
                 per_unit += (k + 1) * 4 + 2 * int(tail_len[b]) * d * s + 2 * g * d * s
-    groups = B * (L // cfg.group) * H
-    rows = groups * (k if shared_rows else cfg.group * k) * C * r * s
-    summaries = groups * cfg.n_live * r * s
+    units = B * L * H
+    rows = units * k * C * r * s
+    summaries = units * cfg.n_live * r * s
     weights = L * H * (r * d + h * r + d * h) * s
     return per_unit + rows + summaries + weights
 
@@ -51,16 +52,18 @@ def test_disjoint_selections_match_the_per_unit_count():
     assert ab["total"] == _expected(cfg, counts, sel, host["tail_len"], shared_rows=False)
 
 
-def test_rows_chosen_by_a_whole_group_count_once():
+def test_rows_chosen_by_a_whole_group_count_per_unit():
     cfg = CFG
     host, counts = _host(cfg, seed=1)
     k, L, B, H = cfg.top_k, cfg.n_layers, cfg.batch, cfg.n_kv_heads
     sel = np.broadcast_to(np.arange(k), (L, B, H, k)).copy()
     ab = bench.algorithmic_bytes(cfg, host, sel, 0, L)
     assert ab["total"] == _expected(cfg, counts, sel, host["tail_len"], shared_rows=True)
-    # the attend kernel's share: rows, records and offsets, and the folded W1' it reads
     groups = B * (L // cfg.group) * H
-    rows = groups * k * cfg.chunk * cfg.rank * 2
+    assert ab["unique_coeff"] == groups * k * cfg.chunk * cfg.rank * 2
+    assert ab["coeff"] == cfg.group * ab["unique_coeff"]
+    # the attend kernel's share: rows, records and offsets, and the folded W1' it reads
+    rows = L * B * H * k * cfg.chunk * cfg.rank * 2
     recs = sum(int(counts[b, l, hk, c]) for l in range(L) for b in range(B) for hk in range(H)
                for c in sel[l, b, hk]) * (cfg.head_dim * 2 + 2)
     ptrs = L * B * H * (k + 1) * 4

@@ -1,12 +1,12 @@
 """Parity of the CUDA encoder (through the C ABI) with the fp64 encoder oracle.
 
-Stored coefficients agree to the tolerance the bf16-rounded basis implies (see
-_check_encode); summaries to one bf16 unit.  Residual norms: the tensor-core predictor
-(bf16 stores) rounds the hidden activations to fp16 (2^-11 relative) before the second
-GEMM, which moves a residual norm by a few 1e-4 of itself; so flags agree wherever the
-oracle's n_res-th and (n_res+1)-th norms are apart by more than 1e-3 relative, and
-otherwise every token on which the two sides differ lies within 1e-3 of the oracle's
-threshold.  Residual rows agree to their bf16 (int8) rounding.
+Stored coefficients agree to the tolerance the bf16-rounded basis implies, with no
+systematic bias (see _check_encode); summaries to one bf16 unit.  Residual norms: each
+token's norm, read back from the kernel's workspace, must lie within NORM_RTOL of the
+oracle's (the roundings behind that bound are listed at NORM_RTOL).  Flags then agree except
+on tokens whose norm is within the two tokens' bounds of the oracle's threshold, the only
+ones a norm error of that size can move across it.  Residual rows agree to their bf16
+(int8) rounding.
 The encoded cache then decodes on the GPU in parity with the decode oracle.
 """
 
@@ -40,6 +40,33 @@ def _gpu_codes(g, cfg):
     if cfg.store == "int8":
         return (g["coeff"].cpu().numpy(), g["coeff_scale"].cpu().numpy())
     return (g["coeff"].cpu().view(torch.int16).numpy().view(np.uint16), None)
+
+
+# Residual norms: the kernels fold W1' = W1 B_l^T once and round it (bf16 for the tensor-core
+# predictor: unit roundoff 2^-9), and the tensor-core predictor also rounds u = pre/2 and H
+# to fp16 (2^-11) around the hardware tanh.  Each pre-activation is then off by a sum of 128
+# independent roundings, and a residual norm by a sum over 128 dimensions of those, so the
+# relative norm error concentrates far below the 2^-9 of a single rounding: a numpy model of
+# exactly these roundings on the 32K workload's weights puts it at 8e-5 (median) and 5.8e-4
+# (largest of 8192 tokens), with the W1' rounding alone at 5.8e-4 and the fp16 H alone at
+# 1.2e-4.  The CUDA-core predictor (int8 stores) keeps everything in fp32.  The bound
+# asserted token by token, where the kernel's norms can be read back:
+NORM_RTOL = 1e-3
+NORM_ATOL = 1e-6
+
+
+def _gpu_norms(g, cfg):
+    """The kernel's residual norms [B][L][Hkv][N] (fp32), read from the workspace that
+    ``lowram_encode`` was given (pieces 256-byte aligned: fp32 W1', bf16 W1'/2, fp16 W2,
+    norms, flags, error word)."""
+    al = lambda x: (x + 255) // 256 * 256
+    lh = cfg.n_layers * cfg.n_kv_heads
+    units = cfg.batch * lh
+    off = al(lh * cfg.rank * cfg.mlp_hidden * 4) + al(lh * cfg.mlp_hidden * cfg.rank * 2) \
+        + al(lh * cfg.head_dim * cfg.mlp_hidden * 2)
+    ws = g["_workspace"]
+    n = ws[off:off + units * cfg.n_ctx * 4].view(torch.float32)
+    return n.view(cfg.batch, cfg.n_layers, cfg.n_kv_heads, cfg.n_ctx).double().cpu().numpy()
 
 
 def _encode_both(cfg, n_res, device_kv="cpu"):
@@ -80,8 +107,10 @@ def _flags_from_records(g, cfg):
     return flags, rec_tok
 
 
-def _check_encode(cfg, g, o, og, n_res):
-    """o: the oracle's encode; og: the oracle's steps 3-6 on the GPU's stored coefficients."""
+def _check_encode(cfg, g, o, og, n_res, norms_gpu=None):
+    """o: the oracle's encode; og: the oracle's steps 3-6 on the GPU's stored coefficients;
+    norms_gpu: the kernel's residual norms [B][L][Hkv][N] when they can be read back (the
+    re-pack keeps its workspace inside the cache)."""
     int8 = cfg.store == "int8"
     # coefficients.  The GPU projects, (1/G) sum_l k_l B_l^T; the oracle solves the normal
     # equations of the stored (bf16-rounded) basis, whose rows are orthonormal only to about
@@ -95,6 +124,13 @@ def _check_encode(cfg, g, o, og, n_res):
         assert np.all(np.abs(ag - ao) <= 2 ** -6 * rowmax + unit + 1e-9)
     else:
         assert np.all(np.abs(ag - ao) <= 2 ** -6 * rowmax + 2 ** -7 * np.abs(ao) + 1e-9)
+    # no systematic bias: rounding to nearest and the basis' departure from orthonormality
+    # both scatter around zero, so the mean signed difference stays far below one unit of
+    # the storage rounding (2^-8 relative for bf16), which a biased rounding would reach
+    scale = np.abs(ao).mean()
+    assert abs(float((ag - ao).mean())) <= 2 ** -11 * scale
+    for idx in np.ndindex(*ag.shape[:3]):
+        assert abs(float((ag[idx] - ao[idx]).mean())) <= 2 ** -9 * np.abs(ao[idx]).mean() + 1e-12, idx
     o = og   # from here on, everything is a function of the stored coefficients
     # summaries: fp32 vs fp64 sums of the same stored rows, rounded to bf16
     sg = g["summary"].double().cpu().numpy()
@@ -110,13 +146,18 @@ def _check_encode(cfg, g, o, og, n_res):
     fg, rec_tok = _flags_from_records(g, cfg)
     fo = o["extra"]["flags"]
     norms = o["extra"]["norms"]
+    bound = NORM_RTOL * norms + NORM_ATOL
+    if norms_gpu is not None:
+        assert np.all(np.abs(norms_gpu - norms) <= bound), float((np.abs(norms_gpu - norms) / norms).max())
     for idx in np.ndindex(*fo.shape[:3]):
         if np.array_equal(fg[idx], fo[idx]) or n_res in (0, cfg.n_ctx):
             assert np.array_equal(fg[idx], fo[idx])
             continue
-        thr = np.sort(norms[idx])[::-1][n_res - 1]
+        order = np.lexsort((np.arange(cfg.n_ctx), -norms[idx]))
+        t_thr = order[n_res - 1]
+        thr = norms[idx][t_thr]
         diff = fg[idx] != fo[idx]
-        assert np.all(np.abs(norms[idx][diff] - thr) <= 1e-3 * thr), idx
+        assert np.all(np.abs(norms[idx][diff] - thr) <= bound[idx][diff] + bound[idx][t_thr]), idx
     # residual rows of tokens both sides flagged
     d = cfg.head_dim
     if n_res > 0:
@@ -159,14 +200,14 @@ def test_encode_matches_oracle(name, kw, store):
     cfg = S.CONFIGS[name].replace(name="enc_" + name, store=store, evict_frac=0.0, **kw)
     n_res = cfg.n_resid
     g, o, og = _encode_both(cfg, n_res)
-    _check_encode(cfg, g, o, og, n_res)
+    _check_encode(cfg, g, o, og, n_res, norms_gpu=_gpu_norms(g, cfg))
 
 
 @pytest.mark.parametrize("n_res", [0, 1, 512])
 def test_encode_residual_count_edges(n_res):
     cfg = S.MISTRAL_GROUP.replace(name="enc_edges", n_layers=2, n_kv_heads=1, n_ctx=512)
     g, o, og = _encode_both(cfg, n_res)
-    _check_encode(cfg, g, o, og, n_res)
+    _check_encode(cfg, g, o, og, n_res, norms_gpu=_gpu_norms(g, cfg))
 
 
 def _as_cache(cfg, g, weights):
@@ -216,6 +257,7 @@ def test_encode_full_size_sampled_units():
     weights = _weights_bf16(cfg)
     g = K.lowram_encode(cfg, cfg.n_resid, Kd, Vd, *(t.to(DEV).contiguous() for t in weights))
     torch.cuda.synchronize()
+    norms_full = _gpu_norms(g, cfg)
     G = cfg.group
     for (b, grp, h) in [(1, 3, 5), (3, 7, 0)]:
         sub = cfg.replace(name="enc_slice", batch=1, n_layers=G, n_kv_heads=1)
@@ -237,4 +279,5 @@ def test_encode_full_size_sampled_units():
             "res_scale": None,
         }
         og = E.encode(*args, given=_gpu_codes(gs, sub))
-        _check_encode(sub, gs, o, og, n_res)
+        ng = norms_full[b:b + 1, ls, h:h + 1]
+        _check_encode(sub, gs, o, og, n_res, norms_gpu=ng)

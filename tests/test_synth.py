@@ -115,3 +115,17 @@ def test_queries_target_chunks():
     assert q.dtype == torch.bfloat16
     q2 = S.make_queries(c, layer0=1, n_layers=1)
     assert torch.equal(q2[0], q[1])
+
+
+def test_select_sequences_keeps_the_oracle_result_of_those_sequences():
+    """Slicing a batch down to a few sequences (used to check large batches on sampled
+    sequences) changes nothing about those sequences' decode results."""
+    import oracle as O
+    cfg = S.MISTRAL_GROUP.replace(name="m3", batch=3, n_ctx=1024, top_k=4)
+    cache = S.make_cache(cfg, tail_len=[64, 10, 33])
+    q = S.make_queries(cache)
+    sub = S.select_sequences(cache, [2, 0])
+    assert sub.cfg.batch == 2 and sub.n_records == int(sub.res_ptr.max())
+    full = O.decode(O.OracleCache(S.cache_to_numpy(cache)), q.double().numpy())["out"]
+    part = O.decode(O.OracleCache(S.cache_to_numpy(sub)), q[:, [2, 0]].double().numpy())["out"]
+    assert np.array_equal(full[:, [2, 0]], part)

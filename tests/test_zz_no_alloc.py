@@ -5,8 +5,9 @@ all device memory for its own pool, a runtime that forbids allocation after star
 thread capturing a CUDA graph in a mode that rejects allocation calls.  They call
 lowram_decode_attn_static, which reads the compressed cache straight from their arrays and
 keeps all scratch in a static device array inside the library.  Its results must match
-lowram_decode_attn on the same cache, on two calls in a row, because the static array keeps
-whatever the previous call left in it.
+lowram_decode_attn on the same cache and the fp64 oracle, on two calls in a row, because the
+static array keeps whatever the previous call left in it, and the calls must leave free device
+memory where it was.
 
 This file is collected last so that a run stopping at the first failure has already run
 every other test.
@@ -17,6 +18,8 @@ import torch
 
 import kv_cache_compression_lowram_b200 as K
 import lowram_synth as S
+import oracle as O
+from parity_utils import check
 
 pytestmark = pytest.mark.gpu
 
@@ -47,13 +50,23 @@ def test_static_entry_point_matches_regular_one(name, kw, layer0, n_layers, tol)
     ref, ref_sel = lc.decode(q, sel=True, layer0=layer0, path=K.PATH_SIMT)
     torch.cuda.synchronize()
     lc.close()
-    for _ in range(2):
-        out = torch.full_like(q, float("nan"))
-        sel = torch.full_like(ref_sel, -1)
-        K.lowram_decode_attn_static(cfg, cache, layer0, n_layers, q, out, sel)
+    outs = [torch.full_like(q, float("nan")) for _ in range(3)]
+    sels = [torch.full_like(ref_sel, -1) for _ in range(3)]
+    # the first call on this device sets up the static array's address (it may also be
+    # where the driver loads the module that holds the array); then free device memory must
+    # not move across two more calls: they allocate nothing
+    K.lowram_decode_attn_static(cfg, cache, layer0, n_layers, q, outs[2], sels[2])
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for i in range(2):
+        K.lowram_decode_attn_static(cfg, cache, layer0, n_layers, q, outs[i], sels[i])
         torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    for out, sel in zip(outs[:2], sels[:2]):
         assert torch.equal(sel, ref_sel)
         assert _vector_error(cfg, out, ref) <= tol
+        # and against the fp64 oracle, under the same parity rules as the regular path
+        check(cfg, O.OracleCache(S.cache_to_numpy(cache)), q, out, sel, layer0=layer0)
 
 
 def test_static_entry_point_rejects_calls_above_its_scratch():
