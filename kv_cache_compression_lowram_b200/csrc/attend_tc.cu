@@ -192,7 +192,9 @@ __device__ __forceinline__ void i8x4_scaled_f16(uint32_t w, __half2 scale, uint3
   hi = *reinterpret_cast<const uint32_t*>(&x23);
 }
 
-template <int R, int C, int GQ, bool I8>
+// TW: the main-loop waits take the call's limit (the test hook that exercises the abort path);
+// otherwise every wait has the compile-time default and compiles to the plain bounded wait.
+template <int R, int C, int GQ, bool I8, bool TW>
 __global__ void __launch_bounds__(kThreadsTC, 1)
 attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CUtensorMap tmW,
                  const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmQ,
@@ -215,7 +217,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
   const int NG = g.L / g.G;
   uint32_t* err = sc.err;
   // limit of the main-loop waits (the drain waits at an abort keep the full kWaitCycles)
-  const long long wlim = g.wait_cycles;
+  const long long wlim = TW ? g.wait_cycles : kWaitCycles;
 
   // ------------------------------------------------------------------ set-up
   if (tid == 0) {
@@ -937,9 +939,9 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
   return r == CUDA_SUCCESS;
 }
 
-template <int R, int C, int GQ, bool I8>
-cudaError_t launch_tc(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const void* w1f,
-                      cudaStream_t s) {
+template <int R, int C, int GQ, bool I8, bool TW>
+cudaError_t launch_tc_t(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const void* w1f,
+                        cudaStream_t s) {
   using Lay = TcLayout<R, C, I8>;
   const int NG = g.L / g.G;
   const uint64_t rows = (uint64_t)g.B * NG * g.Hkv * g.nLs * C;
@@ -956,11 +958,18 @@ cudaError_t launch_tc(const Geom& g, const CacheBuffers& cb, const Scratch& sc, 
     if (!make_map(&tmRes, cb.res_val, kDh, (uint64_t)cb.n_records + kResPad, kResCap))
       return cudaErrorInvalidValue;
   }
-  auto k = attend_tc_kernel<R, C, GQ, I8>;
+  auto k = attend_tc_kernel<R, C, GQ, I8, TW>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
   if (e != cudaSuccess) return e;
   k<<<g.P, kThreadsTC, Lay::SMEM, s>>>(g, cb, sc, tmW, tmA, tmQ, tmRes);
   return cudaGetLastError();
+}
+
+template <int R, int C, int GQ, bool I8>
+cudaError_t launch_tc(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const void* w1f,
+                      cudaStream_t s) {
+  if (g.wait_cycles < kDefaultWaitCycles) return launch_tc_t<R, C, GQ, I8, true>(g, cb, sc, w1f, s);
+  return launch_tc_t<R, C, GQ, I8, false>(g, cb, sc, w1f, s);
 }
 
 }  // namespace

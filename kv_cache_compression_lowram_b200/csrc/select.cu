@@ -319,16 +319,16 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
 
 // ---------------------------------------------------------------------------- fast path
 // The same computation for the common shapes (bf16, d = 128, r in {64, 128}, g in {4, 8},
-// at most kRankMax chunks).  The chunk selection (projection, scores, top-k) and the raw
-// tail's partial softmax do not depend on each other, so each runs in its own half of a
-// 512-thread CTA with its own named barrier; only the queries are shared.  Every thread
-// issues all of its global loads before it uses any of them, basis and summary rows are
-// split across threads, the raw tail is staged in 64-token blocks through a two-buffer
-// cp.async ring (rows padded by 16 bytes against bank conflicts), and the selected ids
-// are placed with a ballot scan.
-constexpr int kFastTB = 64;               // tail tokens per staged block
-constexpr int kFastHalf = 256;            // threads per half of the fast kernel
-constexpr int kFastThreads = 2 * kFastHalf;
+// at most 1024 chunks), one CTA of 8 warps per unit.  The chunk selection and the raw tail's
+// partial softmax do not depend on each other: warps 0-3 project the queries, score the
+// chunks and select, warps 4-7 run the tail, each group with its own named barrier.  The
+// top-k needs no barrier at all: one warp holds every chunk's order key (nC / 32 per lane)
+// and finds the k-th largest by a bitwise binary search with warp-wide counts, then takes
+// the keys equal to it in ascending chunk id.  The tail's value rows are staged into shared
+// memory by cp.async at entry, so their latency hides under the logits.  Shared memory and
+// registers stay small (several units per SM), so a whole call runs in about one wave.
+constexpr int kSelThreads = 256;     // warps 0-3: selection; warps 4-7: raw tail
+constexpr int kSelTB = 128;          // tail tokens per block (one per tail thread)
 
 // 16-byte asynchronous copy global -> shared (zero-filled when !valid); completes at the
 // next cp.async.wait_group.
@@ -339,276 +339,234 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, boo
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-// barrier among the 256 threads of one half (ids 1 and 2; 0 is __syncthreads)
-__device__ __forceinline__ void half_sync(int id) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(kFastHalf) : "memory");
-}
-constexpr int kRowPad = 8;                // bf16 elements of padding per staged tail row
+__device__ __forceinline__ void bar_named(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
-template <int R, int GQ>
-struct FastSmem {
-  static constexpr int D = 128;
-  static constexpr int KROW = D + kRowPad;
-  static constexpr size_t TBUF = (size_t)kFastTB * KROW * 2 + (size_t)kFastTB * D * 2;   // K + V block
-  static constexpr size_t bytes(int nC) {
-    return (size_t)nC * 8                      // keys
-           + (size_t)GQ * D * 4                // qs
-           + (size_t)GQ * R * 4                // qt
-           + (size_t)R * 4                     // qsum
-           + (size_t)nC * 4                    // scores
-           + (size_t)nC * 4                    // selected flags
-           + 256 * 4                           // radix histogram
-           + 2 * TBUF                          // two tail blocks
-           + (size_t)GQ * kFastTB * 4          // logits / probabilities
-           + (size_t)4 * GQ * D * 4            // P.V partial sums of the 4 token quarters
-           + (size_t)3 * GQ * 4 + 64;          // mrun, lrun, alpha, warp totals
+// Exclusive prefix sum over the lanes of a warp.
+__device__ __forceinline__ int warp_excl_scan(int v) {
+  const int lane = threadIdx.x & 31;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
+  return x - v;
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& w, float (&v)[8]) {
+  const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(ww[i] << 16);
+    v[2 * i + 1] = __uint_as_float(ww[i] & 0xffff0000u);
+  }
+}
+
+template <int R, int GQ, int NPL>
+struct SelSmem {
+  float qs[GQ][128];              // the unit's queries
+  float qsum[R];                  // sum_j B_l q_j
+  float score[NPL * 32];          // chunk scores (ids >= nC unused)
+  float p[kSelTB][GQ];            // tail probabilities of the current block, token-major
+  float red_max[4][GQ];           // per tail warp: block maxima, then block sums
+  float red_sum[4][GQ];
+  float pv[GQ][128];              // the second token half's P.V sums
+  __align__(16) __nv_bfloat16 v[kSelTB][128];   // the block's tail values
 };
 
-template <int R, int GQ>
-__global__ void __launch_bounds__(kFastThreads)
-select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __restrict__ q,
+template <int R, int GQ, int NPL>
+__global__ void __launch_bounds__(kSelThreads, GQ <= 4 ? 3 : 2)
+select_warp_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __restrict__ q,
                    float* __restrict__ scores_out, int32_t* __restrict__ sel_out, int tc_q_mode,
                    int do_tail) {
   constexpr int D = 128;
-  using SM = FastSmem<R, GQ>;
+  using SM = SelSmem<R, GQ, NPL>;
   extern __shared__ __align__(16) unsigned char smem_raw[];
+  SM& sm = *reinterpret_cast<SM*>(smem_raw);
   const int u = blockIdx.x;
   const Unit un = unit_of(g, u);
   const int l = g.layer0 + un.li;
   const int grp = l / g.G;
   const int NG = g.L / g.G;
   const int nC = g.nC;
-  const int tid = threadIdx.x;
-  const bool tail_half = tid >= kFastHalf;
-  const int ht = tid & (kFastHalf - 1), lane = ht & 31, warp = ht >> 5;   // within the half
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  unsigned long long* keys = reinterpret_cast<unsigned long long*>(smem_raw);   // [nC]
-  float* qs = reinterpret_cast<float*>(keys + nC);                               // [GQ][D]
-  float* qt = qs + GQ * D;                                                       // [GQ][R]
-  float* qsum = qt + GQ * R;                                                     // [R]
-  float* sc_s = qsum + R;                                                        // [nC]
-  int* selv = reinterpret_cast<int*>(sc_s + nC);                                 // [nC]
-  int* hist = selv + nC;                                                         // [256]
-  unsigned char* tbuf = reinterpret_cast<unsigned char*>(hist + 256);            // 2 x (K, V) blocks
-  float* lg = reinterpret_cast<float*>(tbuf + 2 * SM::TBUF);                     // [GQ][TB]
-  float* pv = lg + GQ * kFastTB;                                                 // [4][GQ][D]
-  float* mrun = pv + 4 * GQ * D;                                                 // [GQ]
-  float* lrun = mrun + GQ;
-  float* alpha = lrun + GQ;
-  int* wtot = reinterpret_cast<int*>(alpha + GQ);                                // [8]
-  __shared__ int radix_state[2];
-
-  int tl = do_tail ? cb.tail_len[un.b] : 0;
-  if (tl < 0 || tl > g.T) {
-    if (tid == 0) atomicOr(sc.err, ERR_TAIL_LEN);
-    tl = tl < 0 ? 0 : g.T;
-  }
+  // tail set-up first: its value rows start streaming into shared memory right away
+  int tl = 0;
   const size_t toff = (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (size_t)g.T * D;
   const __nv_bfloat16* tk = reinterpret_cast<const __nv_bfloat16*>(cb.tail_k) + toff;
   const __nv_bfloat16* tv = reinterpret_cast<const __nv_bfloat16*>(cb.tail_v) + toff;
-  // tail block b -> buffer b % 2: 16 x 16-byte pieces per row, 4 + 4 copies per thread of
-  // the tail half; rows past the tail are zero-filled
-  auto stage_block = [&](int blk) {
-    __nv_bfloat16* kb = reinterpret_cast<__nv_bfloat16*>(tbuf + (blk & 1) * SM::TBUF);
-    __nv_bfloat16* vb = kb + kFastTB * SM::KROW;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int it = ht + k * kFastHalf, t = it >> 4, e = it & 15;
-      const int tt = blk * kFastTB + t;
-      const bool in = tt < tl;
-      cp_async16(kb + t * SM::KROW + e * 8, in ? tk + (size_t)tt * D + e * 8 : tk, in);
-      cp_async16(vb + t * D + e * 8, in ? tv + (size_t)tt * D + e * 8 : tv, in);
+  const int tt = tid - 128;   // tail thread index (warps 4-7)
+  auto stage_v = [&](int t0) {   // rows t0 .. t0+127 (zero past the tail)
+#pragma unroll 4
+    for (int k = 0; k < 16; ++k) {
+      const int it = tt + k * 128, t = it >> 4, e = it & 15;
+      const bool in = t0 + t < tl;
+      cp_async16(&sm.v[t][e * 8], in ? tv + (size_t)(t0 + t) * D + e * 8 : tv, in);
     }
     cp_async_commit();
   };
-  // the tail's first two blocks go to shared memory right away
-  if (tail_half && do_tail) {
-    stage_block(0);
-    stage_block(1);
+  if (warp >= 4 && do_tail) {
+    tl = cb.tail_len[un.b];
+    if (tl < 0 || tl > g.T) {
+      if (tt == 0) atomicOr(sc.err, ERR_TAIL_LEN);
+      tl = tl < 0 ? 0 : g.T;
+    }
+    if (tl > 0) stage_v(0);
   }
 
-  // --- the unit's queries (GQ x 128 bf16: one 16-byte load per thread for GQ <= 16)
+  // the unit's queries (GQ x 128 bf16, 16 bytes per thread)
   const size_t qoff = ((size_t)(un.li * g.B + un.b) * g.Hq + (size_t)un.hkv * GQ) * D;
-  if (!tail_half && ht < GQ * D / 8) {
+  if (tid < GQ * D / 8) {
     float v[8];
-    Vec8<__nv_bfloat16>::load(q + qoff + ht * 8, v);
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(q + qoff) + tid), v);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) qs[ht * 8 + i] = v[i];
+    for (int i = 0; i < 8; ++i) (&sm.qs[0][0])[tid * 8 + i] = v[i];
   }
   __syncthreads();
 
-  if (!tail_half) {
+  if (warp < 4) {
     // ============================================================ chunk selection
-    // --- qt_j = B_l q_j: each basis row split over PARTS threads, all loads issued first
+    const int st = tid;   // 0..127
+    // --- qt_j = B_l q_j: PARTS threads per basis row
     {
-      constexpr int PARTS = kFastHalf / R;         // 2 for r = 128, 4 for r = 64
-      constexpr int SEG = D / PARTS;               // elements per thread
-      const int i = ht / PARTS, part = ht % PARTS;
-      const __nv_bfloat16* row = reinterpret_cast<const __nv_bfloat16*>(cb.basis) +
-                                 (((size_t)l * g.Hkv + un.hkv) * R + i) * D + part * SEG;
-      uint4 w[SEG / 8];
-#pragma unroll
-      for (int e = 0; e < SEG / 8; ++e) w[e] = __ldg(reinterpret_cast<const uint4*>(row) + e);
+      constexpr int PARTS = 128 / R;
+      constexpr int SEG = D / PARTS;
+      const int i = st / PARTS, part = st % PARTS;
+      const uint4* row = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(cb.basis) +
+                                                        (((size_t)l * g.Hkv + un.hkv) * R + i) * D + part * SEG);
       float a[GQ];
 #pragma unroll
       for (int j = 0; j < GQ; ++j) a[j] = 0.f;
 #pragma unroll
-      for (int e = 0; e < SEG / 8; ++e) {
-        const uint32_t ww[4] = {w[e].x, w[e].y, w[e].z, w[e].w};
+      for (int h8 = 0; h8 < SEG / 32; ++h8) {   // 32 elements (4 loads) at a time
+        uint4 w[4];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const float v0 = __uint_as_float(ww[h] << 16), v1 = __uint_as_float(ww[h] & 0xffff0000u);
-          const int col = part * SEG + e * 8 + 2 * h;
+        for (int e = 0; e < 4; ++e) w[e] = __ldg(row + h8 * 4 + e);
 #pragma unroll
-          for (int j = 0; j < GQ; ++j) a[j] = fmaf(v1, qs[j * D + col + 1], fmaf(v0, qs[j * D + col], a[j]));
+        for (int e = 0; e < 4; ++e) {
+          float v[8];
+          bf16x8_to_f32(w[e], v);
+          const int col = part * SEG + (h8 * 4 + e) * 8;
+#pragma unroll
+          for (int j = 0; j < GQ; ++j) {
+            const float4 q0 = *reinterpret_cast<const float4*>(&sm.qs[j][col]);
+            const float4 q1 = *reinterpret_cast<const float4*>(&sm.qs[j][col + 4]);
+            a[j] = fmaf(v[0], q0.x, fmaf(v[1], q0.y, fmaf(v[2], q0.z, fmaf(v[3], q0.w, a[j]))));
+            a[j] = fmaf(v[4], q1.x, fmaf(v[5], q1.y, fmaf(v[6], q1.z, fmaf(v[7], q1.w, a[j]))));
+          }
         }
       }
+      if (PARTS == 2) {
 #pragma unroll
-      for (int j = 0; j < GQ; ++j) {
-#pragma unroll
-        for (int o = 1; o < PARTS; o <<= 1) a[j] += __shfl_xor_sync(0xffffffffu, a[j], o);
+        for (int j = 0; j < GQ; ++j) a[j] += __shfl_xor_sync(0xffffffffu, a[j], 1);
       }
       if (part == 0) {
+        float s = 0.f;
 #pragma unroll
-        for (int j = 0; j < GQ; ++j) qt[j * R + i] = a[j];
+        for (int j = 0; j < GQ; ++j) s += a[j];
+        sm.qsum[i] = s;
+#pragma unroll
+        for (int j = 0; j < GQ; ++j) {
+          const float v = a[j] * g.qk_scale_log2;
+          sc.qt[((size_t)u * GQ + j) * R + i] = v;
+          // rows >= GQ of the 16-row copy stay zero (cleared when the scratch is created)
+          if (tc_q_mode == 1)
+            reinterpret_cast<__nv_bfloat16*>(sc.qt_tc)[((size_t)u * 16 + j) * R + i] = __float2bfloat16_rn(v);
+          else if (tc_q_mode == 2)
+            reinterpret_cast<__half*>(sc.qt_tc)[((size_t)u * 16 + j) * R + i] = __float2half_rn(v);
+        }
       }
     }
-    half_sync(1);
-    for (int i = ht; i < R; i += kFastHalf) {
-      float s = 0.f;
-#pragma unroll
-      for (int j = 0; j < GQ; ++j) s += qt[j * R + i];
-      qsum[i] = s;
-    }
-    for (int i = ht; i < GQ * R; i += kFastHalf) sc.qt[(size_t)u * GQ * R + i] = qt[i] * g.qk_scale_log2;
-    if (tc_q_mode) {
-      for (int i = ht; i < 16 * R; i += kFastHalf) {
-        const int j = i / R;
-        const float v = j < GQ ? qt[i] * g.qk_scale_log2 : 0.f;
-        if (tc_q_mode == 1)
-          reinterpret_cast<__nv_bfloat16*>(sc.qt_tc)[(size_t)u * 16 * R + i] = __float2bfloat16_rn(v);
-        else
-          reinterpret_cast<__half*>(sc.qt_tc)[(size_t)u * 16 * R + i] = __float2half_rn(v);
-      }
-    }
-    half_sync(1);
+    bar_named(1, 128);
 
-    // --- chunk scores: one thread per chunk, the whole summary row loaded at once
+    // --- chunk scores: chunk ids st, st + 128, ...; the whole summary row loaded at once
     const int16_t* slot = cb.slot ? cb.slot + (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * g.nCs : nullptr;
     const __nv_bfloat16* summ = reinterpret_cast<const __nv_bfloat16*>(cb.summary) +
                                 (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * (size_t)g.nLs * R;
     const float inv_sqrt_d = rsqrtf((float)D);
-    for (int c = ht; c < nC; c += kFastHalf) {
-      const int sl = slot ? (int)slot[c] : c;
-      float s = -INFINITY;
-      if (sl >= 0 && sl < g.nL) {
-        const uint4* row = reinterpret_cast<const uint4*>(summ + (size_t)sl * R);
-        uint4 w[R / 8];
-#pragma unroll
-        for (int e = 0; e < R / 8; ++e) w[e] = __ldg(row + e);
-        float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-        for (int e = 0; e < R / 8; ++e) {
-          const uint32_t ww[4] = {w[e].x, w[e].y, w[e].z, w[e].w};
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            a0 = fmaf(__uint_as_float(ww[h] << 16), qsum[e * 8 + 2 * h], a0);
-            a1 = fmaf(__uint_as_float(ww[h] & 0xffff0000u), qsum[e * 8 + 2 * h + 1], a1);
-          }
-        }
-        s = (a0 + a1) * inv_sqrt_d;
-      } else if (sl >= g.nL) {
-        atomicOr(sc.err, ERR_SLOT);
-      }
-      sc_s[c] = s;
-      keys[c] = ((unsigned long long)(~float_order(s)) << 32) | (unsigned)c;
-    }
-    half_sync(1);
-    if (scores_out) {
-      float* so = scores_out + ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * nC;
-      for (int c = ht; c < nC; c += kFastHalf) so[c] = sc_s[c];
-    }
-
-    // --- top-k: radix select on the 32-bit order key (ascending = descending score), 8 bits
-    // a pass, finds the k-th smallest key T and how many keys equal to T are still to take;
-    // those go to the lowest ids.
-    uint32_t prefix = 0;
-    int kk = g.k;
+    float* so = scores_out ? scores_out + ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * nC : nullptr;
 #pragma unroll 1
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      hist[ht] = 0;
-      half_sync(1);
-      for (int c = ht; c < nC; c += kFastHalf) {
-        const uint32_t k32 = (uint32_t)(keys[c] >> 32);
-        if (shift == 24 || (k32 >> (shift + 8)) == (prefix >> (shift + 8))) atomicAdd(&hist[(k32 >> shift) & 255], 1);
-      }
-      half_sync(1);
-      const int hv = hist[ht];
-      int v = hv;
+    for (int c = st; c < NPL * 32; c += 128) {
+      float s = -INFINITY;
+      if (c < nC) {
+        const int sl = slot ? (int)slot[c] : c;
+        if (sl >= 0 && sl < g.nL) {
+          const uint4* row = reinterpret_cast<const uint4*>(summ + (size_t)sl * R);
+          float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int nv = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += nv;
-      }
-      if (lane == 31) wtot[warp] = v;
-      half_sync(1);
-      int woff = 0;
+          for (int h8 = 0; h8 < R / 64; ++h8) {   // 64 ranks (8 loads) at a time
+            uint4 w[8];
 #pragma unroll
-      for (int w2 = 0; w2 < kFastHalf / 32; ++w2) woff += w2 < warp ? wtot[w2] : 0;
-      const int incl = v + woff, excl = incl - hv;
-      if (excl < kk && incl >= kk) {
-        radix_state[0] = ht;
-        radix_state[1] = excl;
-      }
-      half_sync(1);
-      prefix |= (uint32_t)radix_state[0] << shift;
-      kk -= radix_state[1];
-      half_sync(1);   // hist and wtot are rewritten by the next pass
-    }
-    // selected: key below T, or equal to T and among the kk lowest such ids
-    {
-      int eqrun = 0;
-      for (int base = 0; base < nC; base += kFastHalf) {
-        const int c = base + ht;
-        const uint32_t k32 = c < nC ? (uint32_t)(keys[c] >> 32) : 0xffffffffu;
-        const bool feq = c < nC && k32 == prefix;
-        const unsigned beq = __ballot_sync(0xffffffffu, feq);
-        if (lane == 0) wtot[warp] = __popc(beq);
-        half_sync(1);
-        int woff = 0, btot = 0;
+            for (int e = 0; e < 8; ++e) w[e] = __ldg(row + h8 * 8 + e);
 #pragma unroll
-        for (int w2 = 0; w2 < kFastHalf / 32; ++w2) {
-          const int t2 = wtot[w2];
-          woff += w2 < warp ? t2 : 0;
-          btot += t2;
+            for (int e = 0; e < 8; ++e) {
+              float v[8];
+              bf16x8_to_f32(w[e], v);
+              const int col = (h8 * 8 + e) * 8;
+              const float4 q0 = *reinterpret_cast<const float4*>(&sm.qsum[col]);
+              const float4 q1 = *reinterpret_cast<const float4*>(&sm.qsum[col + 4]);
+              a0 = fmaf(v[0], q0.x, fmaf(v[2], q0.z, fmaf(v[4], q1.x, fmaf(v[6], q1.z, a0))));
+              a1 = fmaf(v[1], q0.y, fmaf(v[3], q0.w, fmaf(v[5], q1.y, fmaf(v[7], q1.w, a1))));
+            }
+          }
+          s = (a0 + a1) * inv_sqrt_d;
+        } else if (sl >= g.nL) {
+          atomicOr(sc.err, ERR_SLOT);
         }
-        const int eqrank = eqrun + woff + __popc(beq & ((1u << lane) - 1u));
-        if (c < nC) selv[c] = (k32 < prefix || (feq && eqrank < kk)) ? 1 : 0;
-        eqrun += btot;
-        half_sync(1);
+        if (so) so[c] = s;
+      }
+      sm.score[c] = s;
+    }
+    bar_named(1, 128);
+    if (warp != 0) return;
+
+    // --- top-k (one warp): lane holds chunks lane*NPL .. lane*NPL + NPL-1; the order key
+    // of a score is monotone in the score, and ids >= nC get key 0 (below every chunk's)
+    uint32_t key[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; i += 4) {
+      const float4 f = *reinterpret_cast<const float4*>(&sm.score[lane * NPL + i]);
+      const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+      for (int x = 0; x < 4; ++x) key[i + x] = lane * NPL + i + x < nC ? float_order(fv[x]) : 0u;
+    }
+    // the k-th largest key: the largest T with #{key >= T} >= k, bit by bit from the top
+    uint32_t T = 0;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = T | (1u << bit);
+      int cnt = 0;
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) cnt += key[i] >= cand ? 1 : 0;
+      if (__reduce_add_sync(0xffffffffu, cnt) >= g.k) T = cand;
+    }
+    int gt = 0, eq = 0;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      gt += key[i] > T ? 1 : 0;
+      eq += key[i] == T ? 1 : 0;
+    }
+    const int need_eq = g.k - (int)__reduce_add_sync(0xffffffffu, gt);   // >= 1 keys equal to T, lowest ids
+    int eq_rank = warp_excl_scan(eq);
+    uint32_t take = 0;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      if (key[i] > T) {
+        take |= 1u << i;
+      } else if (key[i] == T) {
+        if (eq_rank < need_eq) take |= 1u << i;
+        ++eq_rank;
       }
     }
+    int pos = warp_excl_scan(__popc(take));
     int32_t* sel_slot = sc.sel_slot + (size_t)u * g.k;
     int32_t* sel_id = sc.sel_id + (size_t)u * g.k;
     int32_t* sel_user = sel_out ? sel_out + ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * g.k : nullptr;
-    int run = 0;
-    for (int base = 0; base < nC; base += kFastHalf) {
-      const int c = base + ht;
-      const int f = c < nC ? selv[c] : 0;
-      const unsigned bal = __ballot_sync(0xffffffffu, f);
-      if (lane == 0) wtot[warp] = __popc(bal);
-      half_sync(1);
-      int woff = 0, btot = 0;
 #pragma unroll
-      for (int w2 = 0; w2 < kFastHalf / 32; ++w2) {
-        const int t2 = wtot[w2];
-        woff += w2 < warp ? t2 : 0;
-        btot += t2;
-      }
-      if (f) {
-        const int pos = run + woff + __popc(bal & ((1u << lane) - 1u));
+    for (int i = 0; i < NPL; ++i) {
+      if (take & (1u << i)) {
+        const int c = lane * NPL + i;
         int sl = slot ? (int)slot[c] : c;
         if (sl < 0 || sl >= g.nL) {
           atomicOr(sc.err, ERR_SELECT);
@@ -619,127 +577,127 @@ select_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
           sel_id[pos] = c;
           if (sel_user) sel_user[pos] = c;
         }
+        ++pos;
       }
-      run += btot;
-      half_sync(1);   // wtot is rewritten by the next round
     }
     return;
   }
   if (!do_tail) return;
 
   // ============================================================ raw tail
-  // partial softmax over its tokens, block by block from the two-buffer ring
-  constexpr int NACC = GQ * D / 2 / kFastHalf;   // (head, dim pair) sums per thread
-  float accr[NACC][2];
+  // Blocks of 128 tokens: thread tt's logits are token t0 + tt's (all heads); its P.V share
+  // is dimension pair dp over one half th of the block's tokens.
+  const int tw = warp - 4;
+  const int dp = tt & 63, th = tt >> 6;
+  float m_run[GQ], l_run[GQ], acc[GQ][2];
 #pragma unroll
-  for (int n = 0; n < NACC; ++n) accr[n][0] = accr[n][1] = 0.f;
-  if (ht < GQ) {
-    mrun[ht] = -INFINITY;
-    lrun[ht] = 0.f;
+  for (int j = 0; j < GQ; ++j) {
+    m_run[j] = -INFINITY;
+    l_run[j] = 0.f;
+    acc[j][0] = acc[j][1] = 0.f;
   }
-  const int nblk = (tl + kFastTB - 1) / kFastTB;
-  for (int bi = 0; bi < nblk; ++bi) {
-    const int t0 = bi * kFastTB;
-    const int nb = min(kFastTB, tl - t0);
-    // block bi's copies (and, when it exists, block bi+1's may still be in flight)
-    if (bi + 1 < nblk) cp_async_wait_one(); else cp_async_wait_all();
-    half_sync(2);
-    const __nv_bfloat16* kblk = reinterpret_cast<const __nv_bfloat16*>(tbuf + (bi & 1) * SM::TBUF);
-    const __nv_bfloat16* vblk = kblk + kFastTB * SM::KROW;
-    // logits: thread (token, GQ/4 heads)
-    {
-      constexpr int JPT = GQ / 4;
-      const int t = ht & (kFastTB - 1), jb = ht / kFastTB;
-      float a[JPT];
+#pragma unroll 1
+  for (int t0 = 0; t0 < tl; t0 += kSelTB) {
+    const int nb = min(kSelTB, tl - t0);
+    float lg[GQ];
 #pragma unroll
-      for (int jj = 0; jj < JPT; ++jj) a[jj] = 0.f;
-      const uint4* krow = reinterpret_cast<const uint4*>(kblk + t * SM::KROW);
-#pragma unroll 4
-      for (int e = 0; e < D / 8; ++e) {
-        const uint4 w = krow[e];
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    for (int j = 0; j < GQ; ++j) lg[j] = -INFINITY;
+    if (tt < nb) {
+      const uint4* krow = reinterpret_cast<const uint4*>(tk + (size_t)(t0 + tt) * D);
+      float a[GQ];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const float v0 = __uint_as_float(ww[h] << 16), v1 = __uint_as_float(ww[h] & 0xffff0000u);
+      for (int j = 0; j < GQ; ++j) a[j] = 0.f;
 #pragma unroll
-          for (int jj = 0; jj < JPT; ++jj) {
-            const float* qq = qs + (jb * JPT + jj) * D + e * 8 + 2 * h;
-            a[jj] = fmaf(v1, qq[1], fmaf(v0, qq[0], a[jj]));
+      for (int h8 = 0; h8 < 4; ++h8) {   // 32 dims (4 loads) at a time: the running state stays in registers
+        uint4 w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) w[e] = __ldg(krow + h8 * 4 + e);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float v[8];
+          bf16x8_to_f32(w[e], v);
+          const int col = (h8 * 4 + e) * 8;
+#pragma unroll
+          for (int j = 0; j < GQ; ++j) {
+            const float4 q0 = *reinterpret_cast<const float4*>(&sm.qs[j][col]);
+            const float4 q1 = *reinterpret_cast<const float4*>(&sm.qs[j][col + 4]);
+            a[j] = fmaf(v[0], q0.x, fmaf(v[1], q0.y, fmaf(v[2], q0.z, fmaf(v[3], q0.w, a[j]))));
+            a[j] = fmaf(v[4], q1.x, fmaf(v[5], q1.y, fmaf(v[6], q1.z, fmaf(v[7], q1.w, a[j]))));
           }
         }
       }
 #pragma unroll
-      for (int jj = 0; jj < JPT; ++jj)
-        lg[(jb * JPT + jj) * kFastTB + t] = t < nb ? a[jj] * g.qk_scale_log2 : -INFINITY;
+      for (int j = 0; j < GQ; ++j) lg[j] = a[j] * g.qk_scale_log2;
     }
-    half_sync(2);
-    // online softmax update: one warp per head
-    if (warp < GQ) {
-      const int j = warp;
-      const float x0 = lg[j * kFastTB + lane], x1 = lg[j * kFastTB + 32 + lane];
-      const float mnew = fmaxf(mrun[j], warp_max(fmaxf(x0, x1)));
-      const float p0 = exp2f(x0 - mnew), p1 = exp2f(x1 - mnew);
-      lg[j * kFastTB + lane] = p0;
-      lg[j * kFastTB + 32 + lane] = p1;
-      const float ssum = warp_sum(p0 + p1);
-      if (lane == 0) {
-        const float a = exp2f(mrun[j] - mnew);   // 0 while mrun = -inf
-        alpha[j] = a;
-        lrun[j] = lrun[j] * a + ssum;
-        mrun[j] = mnew;
+#pragma unroll
+    for (int j = 0; j < GQ; ++j) {
+      const float mx = warp_max(lg[j]);
+      if (lane == 0) sm.red_max[tw][j] = mx;
+    }
+    bar_named(2, 128);
+    float alpha[GQ];
+#pragma unroll
+    for (int j = 0; j < GQ; ++j) {
+      const float mb = fmaxf(fmaxf(sm.red_max[0][j], sm.red_max[1][j]), fmaxf(sm.red_max[2][j], sm.red_max[3][j]));
+      const float mn = fmaxf(m_run[j], mb);   // finite: the block has at least one token
+      alpha[j] = exp2f(m_run[j] - mn);        // 0 while m_run = -inf
+      const float p = exp2f(lg[j] - mn);      // 0 past the tail
+      sm.p[tt][j] = p;
+      const float ps = warp_sum(p);
+      if (lane == 0) sm.red_sum[tw][j] = ps;
+      m_run[j] = mn;
+    }
+    cp_async_wait_all();   // this thread's copies of the block's value rows (the barrier shares them)
+    bar_named(2, 128);
+#pragma unroll
+    for (int j = 0; j < GQ; ++j) {
+      l_run[j] = l_run[j] * alpha[j] + (sm.red_sum[0][j] + sm.red_sum[1][j]) + (sm.red_sum[2][j] + sm.red_sum[3][j]);
+      acc[j][0] *= alpha[j];
+      acc[j][1] *= alpha[j];
+    }
+    const int tb = th * (kSelTB / 2), te = min(tb + kSelTB / 2, nb);
+#pragma unroll 4
+    for (int t = tb; t < te; ++t) {
+      const uint32_t w = *reinterpret_cast<const uint32_t*>(&sm.v[t][2 * dp]);
+      const float v0 = __uint_as_float(w << 16), v1 = __uint_as_float(w & 0xffff0000u);
+#pragma unroll
+      for (int j = 0; j < GQ; j += 4) {
+        const float4 pj = *reinterpret_cast<const float4*>(&sm.p[t][j]);
+        acc[j][0] = fmaf(pj.x, v0, acc[j][0]);
+        acc[j][1] = fmaf(pj.x, v1, acc[j][1]);
+        acc[j + 1][0] = fmaf(pj.y, v0, acc[j + 1][0]);
+        acc[j + 1][1] = fmaf(pj.y, v1, acc[j + 1][1]);
+        acc[j + 2][0] = fmaf(pj.z, v0, acc[j + 2][0]);
+        acc[j + 2][1] = fmaf(pj.z, v1, acc[j + 2][1]);
+        acc[j + 3][0] = fmaf(pj.w, v0, acc[j + 3][0]);
+        acc[j + 3][1] = fmaf(pj.w, v1, acc[j + 3][1]);
       }
     }
-    half_sync(2);
-    // P.V over the block: thread (dim pair, quarter of the tokens), all heads
-    {
-      const int dp = ht & 63, tq = ht >> 6;
-      float sacc[GQ][2];
-#pragma unroll
-      for (int j = 0; j < GQ; ++j) sacc[j][0] = sacc[j][1] = 0.f;
-      const int tb = tq * (kFastTB / 4), te = min(tb + kFastTB / 4, nb);
-      for (int t = tb; t < te; ++t) {
-        const uint32_t w = reinterpret_cast<const uint32_t*>(vblk + t * D)[dp];
-        const float v0 = __uint_as_float(w << 16), v1 = __uint_as_float(w & 0xffff0000u);
-#pragma unroll
-        for (int j = 0; j < GQ; ++j) {
-          const float pj = lg[j * kFastTB + t];
-          sacc[j][0] = fmaf(pj, v0, sacc[j][0]);
-          sacc[j][1] = fmaf(pj, v1, sacc[j][1]);
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < GQ; ++j) {
-        pv[(tq * GQ + j) * D + 2 * dp] = sacc[j][0];
-        pv[(tq * GQ + j) * D + 2 * dp + 1] = sacc[j][1];
-      }
+    if (t0 + kSelTB < tl) {   // the next block's value rows, once every thread is done with these
+      bar_named(2, 128);
+      stage_v(t0 + kSelTB);
     }
-    half_sync(2);
-#pragma unroll
-    for (int n = 0; n < NACC; ++n) {
-      const int it = ht + n * kFastHalf, j = it >> 6, dp = it & 63;
-      float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        s0 += pv[(q4 * GQ + j) * D + 2 * dp];
-        s1 += pv[(q4 * GQ + j) * D + 2 * dp + 1];
-      }
-      accr[n][0] = accr[n][0] * alpha[j] + s0;
-      accr[n][1] = accr[n][1] * alpha[j] + s1;
-    }
-    half_sync(2);   // buffer bi % 2, the logits and the partial sums are free again
-    if (bi + 2 < nblk) stage_block(bi + 2);
   }
-  cp_async_wait_all();
+  // the two token halves' sums, then the tail record (log2-domain max, sum, sums per head)
+  if (th == 1) {
+#pragma unroll
+    for (int j = 0; j < GQ; ++j) {
+      sm.pv[j][2 * dp] = acc[j][0];
+      sm.pv[j][2 * dp + 1] = acc[j][1];
+    }
+  }
+  bar_named(2, 128);
   float* rec = sc.tail_part + (size_t)u * g.tail_stride;
-  if (ht < GQ) {
-    rec[ht] = mrun[ht];
-    rec[GQ + ht] = lrun[ht];
-  }
+  if (th == 0) {
 #pragma unroll
-  for (int n = 0; n < NACC; ++n) {
-    const int it = ht + n * kFastHalf, j = it >> 6, dp = it & 63;
-    rec[2 * GQ + j * D + 2 * dp] = accr[n][0];
-    rec[2 * GQ + j * D + 2 * dp + 1] = accr[n][1];
+    for (int j = 0; j < GQ; ++j) {
+      rec[2 * GQ + j * D + 2 * dp] = acc[j][0] + sm.pv[j][2 * dp];
+      rec[2 * GQ + j * D + 2 * dp + 1] = acc[j][1] + sm.pv[j][2 * dp + 1];
+    }
+  }
+  if (tt < GQ) {
+    rec[tt] = m_run[tt];
+    rec[GQ + tt] = l_run[tt];
   }
 }
 
@@ -757,17 +715,24 @@ size_t select_smem_bytes(const Geom& g) {
 
 namespace {
 
+template <int R, int GQ, int NPL>
+cudaError_t launch_select_warp(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const void* q,
+                               float* scores_out, int32_t* sel_out, int tc_q_mode, bool tail, cudaStream_t s) {
+  using SM = SelSmem<R, GQ, NPL>;
+  auto k = select_warp_kernel<R, GQ, NPL>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SM));
+  if (e != cudaSuccess) return e;
+  k<<<g.U, kSelThreads, sizeof(SM), s>>>(g, cb, sc, static_cast<const __nv_bfloat16*>(q), scores_out, sel_out,
+                                         tc_q_mode, tail ? 1 : 0);
+  return cudaGetLastError();
+}
+
 template <int R, int GQ>
 cudaError_t launch_select_fast(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const void* q,
-                               float* scores_out, int32_t* sel_out, int tc_q_mode, bool tail,
-                               cudaStream_t s) {
-  const size_t smem = FastSmem<R, GQ>::bytes(g.nC);
-  auto k = select_fast_kernel<R, GQ>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  k<<<g.U, kFastThreads, smem, s>>>(g, cb, sc, static_cast<const __nv_bfloat16*>(q), scores_out, sel_out,
-                                    tc_q_mode, tail ? 1 : 0);
-  return cudaGetLastError();
+                               float* scores_out, int32_t* sel_out, int tc_q_mode, bool tail, cudaStream_t s) {
+  if (g.nC <= 256) return launch_select_warp<R, GQ, 8>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s);
+  if (g.nC <= 512) return launch_select_warp<R, GQ, 16>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s);
+  return launch_select_warp<R, GQ, 32>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s);
 }
 
 }  // namespace

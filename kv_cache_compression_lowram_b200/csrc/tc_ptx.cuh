@@ -41,17 +41,47 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of the same phase (no hardware suspend).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// A wait with a shortened limit (the test hook that exercises the abort path).  try_wait may
+// suspend the thread in hardware for a while before it reports "not yet", long enough to
+// hide a short limit, so this polls with test_wait, which never suspends.  Kept out of line:
+// the hot path's waits carry only the branch to it.
+static __device__ __noinline__ bool mbar_wait_short(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                             uint32_t* err, uint32_t err_bit, long long limit) {
+  const long long t0 = clock64();
+  while (!mbar_test_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > limit) {
+      *abort_flag = 1;
+      atomicOr(err, err_bit);
+      return false;
+    }
+  }
+  return true;
+}
 // Wait for the phase with the given parity to complete.  Returns false (and raises the
 // CTA's abort flag and the device error word) if it does not within `limit` cycles
 // (kWaitCycles unless the caller gives less), or as soon as another thread has raised the
 // abort flag.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           uint32_t* err, uint32_t err_bit, long long limit = kWaitCycles) {
+  if (limit < kWaitCycles) return mbar_wait_short(bar, parity, abort_flag, err, err_bit, limit);
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
-    if (clock64() - t0 > limit) {
+    if (clock64() - t0 > kWaitCycles) {
       *abort_flag = 1;
       atomicOr(err, err_bit);
       return false;
