@@ -622,6 +622,46 @@ def select_sequences(cache: SynthCache, seqs, device="cpu") -> SynthCache:
         tail_v=rows(cache.tail_v), tail_len=rows(cache.tail_len))
 
 
+def shard_chunks(cache: SynthCache, c_lo: int, c_hi: int, keep_tail: bool) -> SynthCache:
+    """The cache of chunk ids [c_lo, c_hi) of every unit, as a cache of its own (local ids).
+
+    Every unit keeps those chunks' coefficient rows, scales and summaries and the residual
+    records of those chunks (gathered unit by unit, CSR offsets rebased).  The raw tail is
+    kept (keep_tail) or emptied (tail_len = 0, arrays kept).  Caches with evicted chunks are
+    not split (their live chunks per range differ between units).  Used to build the shards
+    of a context-sharded decode from one generated cache.
+    """
+    cfg = cache.cfg
+    assert cfg.n_live == cfg.n_chunks, "no eviction in a split cache"
+    assert 0 <= c_lo < c_hi <= cfg.n_chunks
+    C = cfg.chunk
+    n = c_hi - c_lo
+    dev = cache.coeff.device
+    rp = cache.res_ptr.to(torch.int64)
+    lo, hi = rp[..., c_lo], rp[..., c_hi]                      # [B][L][Hkv]
+    counts = (hi - lo).reshape(-1)
+    starts = lo.reshape(-1)
+    idx = torch.cat([torch.arange(int(a), int(a) + int(c), device=dev) for a, c in zip(starts.tolist(), counts.tolist())]) \
+        if counts.numel() else torch.empty(0, dtype=torch.int64, device=dev)
+    base = (torch.cumsum(counts, 0) - counts).reshape(lo.shape)
+    res_ptr = (rp[..., c_lo:c_hi + 1] - lo.unsqueeze(-1) + base.unsqueeze(-1)).to(torch.int32)
+
+    def recs(t):
+        return None if t is None else t.index_select(0, idx).contiguous()
+
+    tl = cache.tail_len.clone() if keep_tail else torch.zeros_like(cache.tail_len)
+    B, NG, H = cfg.batch, cfg.n_groups, cfg.n_kv_heads
+    return SynthCache(
+        cfg=cfg.replace(name=f"{cfg.name}_c{c_lo}_{c_hi}", n_ctx=n * C),
+        coeff=cache.coeff[:, :, :, c_lo * C:c_hi * C].contiguous(),
+        coeff_scale=None if cache.coeff_scale is None else cache.coeff_scale[:, :, :, c_lo * C:c_hi * C].contiguous(),
+        basis=cache.basis, w1=cache.w1, w2=cache.w2,
+        summary=cache.summary[:, :, :, c_lo:c_hi].contiguous(),
+        slot=torch.arange(n, dtype=torch.int16, device=dev).expand(B, NG, H, n).contiguous(),
+        res_ptr=res_ptr, res_pos=recs(cache.res_pos), res_val=recs(cache.res_val),
+        res_scale=recs(cache.res_scale), tail_k=cache.tail_k, tail_v=cache.tail_v, tail_len=tl)
+
+
 # ------------------------------------------------------------------------ numpy export
 
 def _np_storage(t: Optional[torch.Tensor]):
