@@ -347,6 +347,62 @@ lowram_status lowram_decode_attn_static(const lowram_config* cfg, const lowram_c
                                         int32_t layer0, int32_t n_layers, const void* q,
                                         void* out, int32_t* sel, lowram_stream stream);
 
+/* ------------------------------------------------------------- context-sharded decode
+ *
+ * One sequence's context split by chunk over P shards, usually one per GPU, so that a context
+ * too long for one GPU's memory (or bandwidth) is decoded by several ("LowRAM Compresses KV
+ * Cache Asymmetrically", section "Why Peak Throughput Can Improve by 5x": decode is bound by
+ * moving the KV cache, also between GPUs).  Shard s is an ordinary cache created from the
+ * chunk ids [off_s, off_s + nC_s) of every (sequence, layer group, KV head): its coefficient
+ * rows, scales, summaries and those chunks' residual records, its chunk ids local (global id =
+ * off_s + local id); every shard holds the same weights, and only the shard with the newest
+ * tokens has a non-empty raw tail (tail_len = 0 elsewhere).  Each shard needs nC_s >= top_k
+ * live chunks.  One decode step:
+ *   1. every shard: lowram_shard_candidates -> its own top k as (score, global chunk id);
+ *   2. the caller gathers every shard's candidates on every shard, in ascending off_s order
+ *      (an all-gather; the library itself does not communicate);
+ *   3. every shard: lowram_shard_partial -> the k best of all candidates by (descending score,
+ *      ascending global id) -- exactly the unsharded selection, since a chunk among the k
+ *      best overall has fewer than k better chunks in its own shard -- then attention of each
+ *      query head over the selected chunks the shard holds plus its raw tail, unnormalised;
+ *   4. the caller gathers the shards' partials; lowram_merge_partials gives the output:
+ *      o_j = sum_s w_s y_{s,j} / sum_s w_s l_{s,j},  w_s = 2^(m_{s,j} - max_s m_{s,j}).
+ * The result equals lowram_decode_attn on the whole cache up to floating-point regrouping.
+ * Shapes: those the tensor-core path serves (EUNSUPPORTED otherwise). */
+
+/* Phase 1 on one shard for layers [layer0, layer0 + n_layers):
+ *   q          [n_layers][B][Hq][d] dt, DEVICE (the same queries on every shard);
+ *   cand_score [n_layers][B][Hkv][k] fp32, DEVICE: the scores of the shard's own k best chunks;
+ *   cand_id    [n_layers][B][Hkv][k] int32, DEVICE: their global ids (chunk_offset + local id),
+ *              ascending.
+ * Also leaves in the cache's scratch what phase 2 needs (the projected queries and the raw
+ * tail's partial softmax): lowram_shard_partial must be the next call on this cache that
+ * writes its scratch (no decode, selection or re-pack in between).  Stream-ordered, no
+ * allocation, no host synchronisation.  EINVAL for a bad range, NULL pointer or negative
+ * offset. */
+lowram_status lowram_shard_candidates(lowram_cache* shard, int32_t layer0, int32_t n_layers, const void* q,
+                                      int32_t chunk_offset, float* cand_score, int32_t* cand_id,
+                                      lowram_stream stream);
+
+/* Phase 2 on one shard, after every shard's candidates were gathered:
+ *   cand_score / cand_id [n_shards][n_layers][B][Hkv][k] (shards in ascending chunk_offset);
+ *   partial [n_layers][B][Hq][d + 2] fp32, DEVICE: per query head j, m_j (the largest logit
+ *           in log2 units: q.k / sqrt(d) * log2(e)), l_j = sum_t 2^(logit_t - m_j) and
+ *           y_j[d] = sum_t 2^(logit_t - m_j) v_t over the shard's selected tokens and tail
+ *           (m_j = -inf, l_j = 0, y_j = 0 when the shard holds none of them);
+ *   sel     [n_layers][B][Hkv][k] int32, DEVICE, may be NULL: the global selection, ascending.
+ * EINVAL unless it follows lowram_shard_candidates for the same layers on this cache, or when
+ * n_shards < 1 or n_shards * top_k > 1024.  Stream-ordered, no allocation or synchronisation. */
+lowram_status lowram_shard_partial(lowram_cache* shard, int32_t layer0, int32_t n_layers, int32_t chunk_offset,
+                                   int32_t n_shards, const float* cand_score, const int32_t* cand_id,
+                                   float* partial, int32_t* sel, lowram_stream stream);
+
+/* Merge of the shards' partial records: partials [n_parts][n_rows][head_dim + 2] fp32 (rows
+ * laid out as lowram_shard_partial writes them), out [n_rows][head_dim] in out_dtype
+ * (LOWRAM_F32 or LOWRAM_BF16), DEVICE.  EINVAL for bad sizes.  Stream-ordered. */
+lowram_status lowram_merge_partials(int32_t n_parts, int64_t n_rows, int32_t head_dim, const float* partials,
+                                    int32_t out_dtype, void* out, lowram_stream stream);
+
 /* ---------------------------------------------------------------- prefill-side encoder
  *
  * lowram_encode: dense keys and values -> the compressed arrays lowram_cache_create takes

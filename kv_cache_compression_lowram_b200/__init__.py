@@ -102,6 +102,9 @@ def lib() -> ctypes.CDLL:
         "lowram_encode_workspace_bytes": (U64, [ctypes.POINTER(LowramConfigC)]),
         "lowram_encode": (I32, [ctypes.POINTER(LowramConfigC), I32, P, P, P, P, P,
                                 ctypes.POINTER(LowramEncodeDstC), P, U64, P]),
+        "lowram_shard_candidates": (I32, [P, I32, I32, P, I32, P, P, P]),
+        "lowram_shard_partial": (I32, [P, I32, I32, I32, I32, P, P, P, P, P]),
+        "lowram_merge_partials": (I32, [I32, I64, I32, P, I32, P, P]),
         "lowram_debug_set_wait_limit": (I32, [P, I64]),
         "lowram_debug_fail_alloc": (None, [I32]),
         "lowram_status_string": (ctypes.c_char_p, [I32]),
@@ -290,6 +293,30 @@ def lowram_cache_last_launches(handle: int) -> int:
 
 def lowram_cache_last_path(handle: int) -> int:
     return int(lib().lowram_cache_last_path(handle))
+
+
+def lowram_shard_candidates(handle: int, layer0: int, n_layers: int, q, chunk_offset: int, cand_score, cand_id,
+                            stream=None) -> None:
+    """Phase 1 of a context-sharded decode step on one shard (see lowram.h)."""
+    _check(lib().lowram_shard_candidates(handle, layer0, n_layers, _ptr(q), int(chunk_offset), _ptr(cand_score),
+                                         _ptr(cand_id), _stream(stream)), "lowram_shard_candidates")
+
+
+def lowram_shard_partial(handle: int, layer0: int, n_layers: int, chunk_offset: int, n_shards: int, cand_score,
+                         cand_id, partial, sel=None, stream=None) -> None:
+    """Phase 2 on one shard, from every shard's gathered candidates (see lowram.h)."""
+    _check(lib().lowram_shard_partial(handle, layer0, n_layers, int(chunk_offset), int(n_shards), _ptr(cand_score),
+                                      _ptr(cand_id), _ptr(partial), _ptr(sel), _stream(stream)),
+           "lowram_shard_partial")
+
+
+def lowram_merge_partials(partials, out, stream=None) -> None:
+    """partials [n_parts][n_rows][d + 2] fp32 -> out [n_rows][d] (fp32 or bf16), CUDA tensors."""
+    import torch
+    n_parts, n_rows, w = (int(x) for x in partials.shape)
+    dt = 0 if out.dtype == torch.float32 else 1
+    _check(lib().lowram_merge_partials(n_parts, n_rows, w - 2, _ptr(partials), dt, _ptr(out), _stream(stream)),
+           "lowram_merge_partials")
 
 
 def lowram_debug_set_wait_limit(handle: int, cycles: int) -> None:

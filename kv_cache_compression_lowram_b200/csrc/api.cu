@@ -42,6 +42,9 @@ struct lowram_cache {
   bool ev_on;
   int last_launches, last_path;
   long long wait_limit;        // main-loop wait limit of the tensor-core kernel (test hook)
+  // context-sharded decode: tile list of phase 2, and the layer range phase 1 prepared
+  int32_t *t_unit, *t_slot, *t_ptr, *t_total, *t_cnt;
+  int shard_l0, shard_n;
 };
 
 namespace {
@@ -394,7 +397,12 @@ lowram_status lowram_cache_create(const lowram_config* cfg, const lowram_cache_s
       (st = alloc(c, &c->sc.err, 16)) != LOWRAM_OK ||
       (st = alloc(c, &c->q_stage, L * B * cfg->n_q_heads * d * s)) != LOWRAM_OK ||
       (st = alloc(c, &c->out_stage, L * B * cfg->n_q_heads * d * s)) != LOWRAM_OK ||
-      (st = alloc(c, &c->sel_stage, Umax * k * 4)) != LOWRAM_OK) {
+      (st = alloc(c, &c->sel_stage, Umax * k * 4)) != LOWRAM_OK ||
+      (st = alloc(c, &c->t_unit, Umax * k * 4)) != LOWRAM_OK ||
+      (st = alloc(c, &c->t_slot, Umax * k * 4)) != LOWRAM_OK ||
+      (st = alloc(c, &c->t_ptr, (Umax + 1) * 4)) != LOWRAM_OK ||
+      (st = alloc(c, &c->t_total, 16)) != LOWRAM_OK ||
+      (st = alloc(c, &c->t_cnt, Umax * 4)) != LOWRAM_OK) {
     lowram_cache_destroy(c);
     return st;
   }
@@ -403,6 +411,8 @@ lowram_status lowram_cache_create(const lowram_config* cfg, const lowram_cache_s
   e = cudaMemsetAsync(c->sc.qt_tc, 0, Umax * 16 * r * 2, cs);
   if (e != cudaSuccess) { lowram_cache_destroy(c); return cuda_fail(e, "cudaMemsetAsync"); }
   c->last_path = -1;
+  c->shard_l0 = -1;
+  c->shard_n = 0;
   *out = c;
   return LOWRAM_OK;
 }
@@ -534,6 +544,7 @@ extern "C" {
 
 lowram_status lowram_cache_repack(lowram_cache* c, int32_t n_resid, lowram_stream stream) {
   if (!c) return inval("NULL cache");
+  c->shard_l0 = -1;
   const lowram_config f = c->cfg;
   const int C = f.chunk, T = f.tail_cap;
   if (n_resid < 0 || n_resid > C) return inval("n_resid must lie in [0, chunk]");
@@ -773,6 +784,7 @@ lowram_status lowram_select_chunks(lowram_cache* c, int32_t layer0, int32_t n_la
   if (st != LOWRAM_OK) return st;
   if (!q) return inval("NULL q");
   Geom g = make_geom(c, layer0, n_layers, false);
+  c->shard_l0 = -1;   // the scratch phase 1 of a sharded decode left is overwritten
   cudaError_t e = launch_select(g, c->cb, c->sc, c->cfg.dtype, q, scores, sel, 0, false,
                                 reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "select kernel");
@@ -800,6 +812,7 @@ lowram_status lowram_decode_attn(lowram_cache* c, int32_t layer0, int32_t n_laye
     tc = tc_able;
   }
   Geom g = make_geom(c, layer0, n_layers, tc);
+  c->shard_l0 = -1;   // the scratch phase 1 of a sharded decode left is overwritten
   cudaError_t e;
   if (c->ev_on && (e = cudaEventRecord(c->ev[0], s)) != cudaSuccess) return cuda_fail(e, "event");
   const int tc_q_mode = tc ? (c->cfg.store == LOWRAM_STORE_INT8 ? 2 : 1) : 0;
@@ -910,6 +923,77 @@ lowram_status lowram_cache_validate(lowram_cache* c, lowram_stream stream) {
     g_last_error = "an append found a full tail: that sequence's token was dropped";
     return LOWRAM_EINVAL;
   }
+  return LOWRAM_OK;
+}
+
+// ------------------------------------------------------------- context-sharded decode
+
+lowram_status lowram_shard_candidates(lowram_cache* c, int32_t layer0, int32_t n_layers, const void* q,
+                                      int32_t chunk_offset, float* cand_score, int32_t* cand_id,
+                                      lowram_stream stream) {
+  lowram_status st = check_layers(c, layer0, n_layers);
+  if (st != LOWRAM_OK) return st;
+  if (!q || !cand_score || !cand_id) return inval("NULL q or candidate output");
+  if (chunk_offset < 0) return inval("chunk_offset must be >= 0");
+  Geom g = make_geom(c, layer0, n_layers, true);
+  if (!attend_tc_supported(g, c->cfg.dtype, c->cfg.store)) {
+    g_last_error = "context-sharded decode runs on the tensor-core kernel's shapes only";
+    return LOWRAM_EUNSUPPORTED;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int tc_q_mode = c->cfg.store == LOWRAM_STORE_INT8 ? 2 : 1;
+  cudaError_t e = launch_select(g, c->cb, c->sc, c->cfg.dtype, q, nullptr, nullptr, tc_q_mode, true, s,
+                                SelCand{cand_score, cand_id, chunk_offset});
+  if (e != cudaSuccess) return cuda_fail(e, "select kernel");
+  c->shard_l0 = layer0;
+  c->shard_n = n_layers;
+  c->last_launches = 1;
+  return LOWRAM_OK;
+}
+
+lowram_status lowram_shard_partial(lowram_cache* c, int32_t layer0, int32_t n_layers, int32_t chunk_offset,
+                                   int32_t n_shards, const float* cand_score, const int32_t* cand_id,
+                                   float* partial, int32_t* sel, lowram_stream stream) {
+  lowram_status st = check_layers(c, layer0, n_layers);
+  if (st != LOWRAM_OK) return st;
+  if (!cand_score || !cand_id || !partial) return inval("NULL candidates or partial output");
+  if (chunk_offset < 0) return inval("chunk_offset must be >= 0");
+  if (n_shards < 1 || (long long)n_shards * c->cfg.top_k > 1024)
+    return inval("n_shards must be >= 1 with n_shards * top_k <= 1024");
+  if (layer0 != c->shard_l0 || n_layers != c->shard_n)
+    return inval("lowram_shard_partial must follow lowram_shard_candidates for the same layers on this cache");
+  Geom g = make_geom(c, layer0, n_layers, true);
+  if (!attend_tc_supported(g, c->cfg.dtype, c->cfg.store)) {
+    g_last_error = "context-sharded decode runs on the tensor-core kernel's shapes only";
+    return LOWRAM_EUNSUPPORTED;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  Scratch sc = c->sc;
+  sc.tile_unit = c->t_unit;
+  sc.tile_slot = c->t_slot;
+  sc.tile_ptr = c->t_ptr;
+  sc.tile_total = c->t_total;
+  sc.unit_ntile = c->t_cnt;
+  cudaError_t e = launch_shard_select(g, c->cb, sc, cand_score, cand_id, n_shards, chunk_offset, sel, s);
+  if (e != cudaSuccess) return cuda_fail(e, "shard selection kernels");
+  e = launch_attend_tc(g, c->cb, sc, c->cfg.store, c->w1f_tc, c->n_sm, s);
+  if (e != cudaSuccess) return cuda_fail(e, "chunk attention kernel");
+  e = launch_combine_partial(g, c->cb, sc, c->cfg.dtype, partial, s);
+  if (e != cudaSuccess) return cuda_fail(e, "partial combine kernel");
+  c->last_launches = 4;
+  c->last_path = LOWRAM_PATH_TC;
+  return LOWRAM_OK;
+}
+
+lowram_status lowram_merge_partials(int32_t n_parts, int64_t n_rows, int32_t head_dim, const float* partials,
+                                    int32_t out_dtype, void* out, lowram_stream stream) {
+  if (n_parts < 1 || n_rows < 0 || n_rows >= (1LL << 31) || head_dim < 1 || head_dim > kMaxD)
+    return inval("n_parts >= 1, 0 <= n_rows < 2^31 and 1 <= head_dim <= 256 are required");
+  if (out_dtype != LOWRAM_F32 && out_dtype != LOWRAM_BF16) return inval("unknown output dtype");
+  if (n_rows > 0 && (!partials || !out)) return inval("NULL partials or out");
+  cudaError_t e = launch_merge_partials(n_parts, n_rows, head_dim, partials, out_dtype, out,
+                                        reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "merge kernel");
   return LOWRAM_OK;
 }
 

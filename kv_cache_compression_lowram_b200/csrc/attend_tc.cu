@@ -160,7 +160,43 @@ struct TileWalk {
     }
   }
   __device__ __forceinline__ bool next_starts_segment() const { return rem + 1 == k && ub + 1 == B; }
+  __device__ __forceinline__ bool first_of_unit() const { return rem == 0; }
 };
+
+// The same walk over an explicit tile list (context-sharded decode: a unit holds any number
+// of the call's tiles, 0 .. k): tile x belongs to unit tu[x].  The next tile's unit is read
+// one step ahead, so its latency hides under the current tile's work.
+struct TileWalkList {
+  const int32_t* tu;
+  long long x0, x1;
+  int ci, u, seg, B, nu;
+  bool first;
+  __device__ __forceinline__ void init(long long x0_, long long x1_, const int32_t* tu_, int B_) {
+    tu = tu_;
+    x0 = x0_;
+    x1 = x1_;
+    B = B_;
+    ci = 0;
+    u = x0 < x1 ? __ldg(tu + x0) : 0;
+    first = x0 == 0 || (x0 < x1 && __ldg(tu + x0 - 1) != u);
+    seg = u / B;
+    nu = x0 + 1 < x1 ? __ldg(tu + x0 + 1) : -1;
+  }
+  __device__ __forceinline__ void advance_to(int target) {
+    while (ci < target) {
+      ++ci;
+      first = nu != u;
+      u = nu;
+      seg = u / B;
+      nu = x0 + ci + 1 < x1 ? __ldg(tu + x0 + ci + 1) : -1;
+    }
+  }
+  // only asked while a next tile exists in this CTA's range
+  __device__ __forceinline__ bool next_starts_segment() const { return nu / B != seg; }
+  __device__ __forceinline__ bool first_of_unit() const { return first; }
+};
+template <bool CT> struct WalkOf { using type = TileWalk; };
+template <> struct WalkOf<true> { using type = TileWalkList; };
 
 // Offset of element (row j, column k) in a K-major operand tile without swizzle: 8 x 16-byte
 // core matrices, K-adjacent ones 128 bytes apart, 8-row groups sbo bytes apart.
@@ -194,7 +230,9 @@ __device__ __forceinline__ void i8x4_scaled_f16(uint32_t w, __half2 scale, uint3
 
 // TW: the main-loop waits take the call's limit (the test hook that exercises the abort path);
 // otherwise every wait has the compile-time default and compiles to the plain bounded wait.
-template <int R, int C, int GQ, bool I8, bool TW>
+// CT: the tiles come as an explicit list (sc.tile_unit / sc.tile_slot, sc.tile_total of them)
+// instead of k per unit.
+template <int R, int C, int GQ, bool I8, bool TW, bool CT>
 __global__ void __launch_bounds__(kThreadsTC, 1)
 attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CUtensorMap tmW,
                  const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmQ,
@@ -209,7 +247,9 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
   volatile int* abort_flag = &misc->abort_flag;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const long long total = (long long)g.U * g.k;
+  using Walk = typename WalkOf<CT>::type;
+  const long long total = CT ? (long long)*sc.tile_total : (long long)g.U * g.k;
+  const int32_t* tslot = CT ? sc.tile_slot : sc.sel_slot;   // storage slot of tile x
   const long long x0 = tile_begin(total, g.P, blockIdx.x);
   const long long x1 = tile_begin(total, g.P, blockIdx.x + 1);
   const int NCH = (int)(x1 - x0);
@@ -218,6 +258,10 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
   uint32_t* err = sc.err;
   // limit of the main-loop waits (the drain waits at an abort keep the full kWaitCycles)
   const long long wlim = TW ? g.wait_cycles : kWaitCycles;
+  auto init_walk = [&](Walk& w, long long a, long long b) {
+    if constexpr (CT) w.init(a, b, sc.tile_unit, g.B);
+    else w.init(a, g.k, g.B);
+  };
 
   // ------------------------------------------------------------------ set-up
   if (tid == 0) {
@@ -284,8 +328,8 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
     if (NCH > 0) {
       int unit_i = -1, prev_u = -1, issued_a = 0, issued_r = 0, q_issued = 0;
       int seg_i = -1, prev_seg = -1, w1_issued = 0;
-      TileWalk wk;
-      wk.init(x0, g.k, g.B);
+      Walk wk;
+      init_walk(wk, x0, x1);
       for (int ci = 0; ci < NCH; ++ci) {
         const long long x = x0 + ci;
         wk.advance_to(ci);
@@ -319,7 +363,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
         const Unit un = unit_of(g, u);
         const int l = g.layer0 + un.li;
         const int grp = l / g.G;
-        const int slot = sc.sel_slot[x];
+        const int slot = tslot[x];
         const int row0 = (int)(((((long long)un.b * NG + grp) * g.Hkv + un.hkv) * g.nLs + slot) * C);
         if (leader) {
           if (I8) {
@@ -439,8 +483,8 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
       const uint64_t dPR0 = smem_desc(sPR, 128, Lay::PR_SBO, 0);    // probabilities at records
       const uint32_t t_d1 = tmem + Lay::T_D1;
       const uint32_t t_s = tmem + Lay::T_S, t_d3 = tmem + Lay::T_D3, t_d4 = tmem + Lay::T_D4;
-      TileWalk wk;
-      wk.init(x0, g.k, g.B);
+      Walk wk;
+      init_walk(wk, x0, x1);
       auto wait_all = [&](uint64_t* b, uint32_t par) -> bool {
         return __all_sync(0xffffffffu, mbar_wait(b, par, abort_flag, err, ERR_TIMEOUT, wlim));
       };
@@ -796,8 +840,8 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
         accH1[j] = 0.f;
       }
     };
-    TileWalk wk;
-    wk.init(x0, g.k, g.B);
+    Walk wk;
+    init_walk(wk, x0, x1);
     for (int ci = 0; ci < NCH; ++ci) {
       wk.advance_to(ci);
       const int u = wk.u;
@@ -893,7 +937,7 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
       // fold the previous chunk's D3 / D4 when it belongs to this unit (its MMAs ran
       // meanwhile); it is relative to the max after chunk ci-1, so the running sums are
       // rescaled by that chunk's factor first
-      if (ci >= 1 && wk.rem != 0) fold(ci - 1);
+      if (ci >= 1 && !wk.first_of_unit()) fold(ci - 1);
 #pragma unroll
       for (int j = 0; j < GQ; ++j) al_prev[j] = al[j];
     }
@@ -939,7 +983,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
   return r == CUDA_SUCCESS;
 }
 
-template <int R, int C, int GQ, bool I8, bool TW>
+template <int R, int C, int GQ, bool I8, bool TW, bool CT>
 cudaError_t launch_tc_t(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const void* w1f,
                         cudaStream_t s) {
   using Lay = TcLayout<R, C, I8>;
@@ -958,7 +1002,7 @@ cudaError_t launch_tc_t(const Geom& g, const CacheBuffers& cb, const Scratch& sc
     if (!make_map(&tmRes, cb.res_val, kDh, (uint64_t)cb.n_records + kResPad, kResCap))
       return cudaErrorInvalidValue;
   }
-  auto k = attend_tc_kernel<R, C, GQ, I8, TW>;
+  auto k = attend_tc_kernel<R, C, GQ, I8, TW, CT>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
   if (e != cudaSuccess) return e;
   k<<<g.P, kThreadsTC, Lay::SMEM, s>>>(g, cb, sc, tmW, tmA, tmQ, tmRes);
@@ -968,8 +1012,9 @@ cudaError_t launch_tc_t(const Geom& g, const CacheBuffers& cb, const Scratch& sc
 template <int R, int C, int GQ, bool I8>
 cudaError_t launch_tc(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const void* w1f,
                       cudaStream_t s) {
-  if (g.wait_cycles < kDefaultWaitCycles) return launch_tc_t<R, C, GQ, I8, true>(g, cb, sc, w1f, s);
-  return launch_tc_t<R, C, GQ, I8, false>(g, cb, sc, w1f, s);
+  if (sc.tile_total) return launch_tc_t<R, C, GQ, I8, false, true>(g, cb, sc, w1f, s);
+  if (g.wait_cycles < kDefaultWaitCycles) return launch_tc_t<R, C, GQ, I8, true, false>(g, cb, sc, w1f, s);
+  return launch_tc_t<R, C, GQ, I8, false, false>(g, cb, sc, w1f, s);
 }
 
 }  // namespace

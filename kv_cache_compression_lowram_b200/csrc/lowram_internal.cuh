@@ -106,6 +106,14 @@ struct Scratch {
   float* part;        // chunk partial records
   float* tail_part;   // [U][tail_stride]
   uint32_t* err;      // device error word
+  // Explicit tile list (context-sharded decode; tile_total == nullptr otherwise): tile x of
+  // the call is chunk slot tile_slot[x] of unit tile_unit[x], units in ascending order; unit
+  // u's tiles are [tile_ptr[u], tile_ptr[u + 1]); *tile_total tiles in all.
+  int32_t* tile_unit;
+  int32_t* tile_slot;
+  int32_t* tile_ptr;
+  int32_t* tile_total;
+  int32_t* unit_ntile; // [U] tiles of each unit (written by the shard selection)
 };
 
 // ---------------------------------------------------------------- element conversions
@@ -138,11 +146,19 @@ __device__ __forceinline__ float warp_max(float v) {
 
 // ----------------------------------------------------------------------- launchers
 
+// Optional output of the selection for context-sharded decode: the selected chunks' scores
+// and ids + offset (the shard's first global chunk id), [n_layers][B][Hkv][k] like sel.
+struct SelCand {
+  float* score;
+  int32_t* id;
+  int offset;
+};
+
 // Steps 1-2 (+ the raw tail's partial softmax): one CTA per unit.
 // tc_q_mode: 0 = no 16-bit copy of qt, 1 = bf16 copy, 2 = fp16 copy.
 cudaError_t launch_select(const Geom& g, const CacheBuffers& cb, const Scratch& sc,
                           int dtype, const void* q, float* scores_out, int32_t* sel_out,
-                          int tc_q_mode, bool tail, cudaStream_t s);
+                          int tc_q_mode, bool tail, cudaStream_t s, SelCand cand = SelCand{nullptr, nullptr, 0});
 // Steps 3-5 on CUDA cores over the selected chunks.  w1f_t holds the fp32 W1' of layers
 // [w1f_layer0, ...): layer l's fold is at (l - w1f_layer0) * Hkv * r * h.
 cudaError_t launch_attend_simt(const Geom& g, const CacheBuffers& cb, const Scratch& sc,
@@ -168,6 +184,15 @@ size_t encode_workspace_bytes(const Geom& g, bool folds_given = false);
 cudaError_t launch_encode(const Geom& g, int store, int n_res, const void* keys, const void* values,
                           const void* basis, const void* w1, const void* w2, const lowram_encode_dst& dst,
                           void* workspace, cudaStream_t s);
+// Context-sharded decode, phase 2 (shard.cu): the global selection from every shard's
+// candidates and the shard's tile list (sc.tile_*), the shard's unnormalised partial per query
+// head ([n_layers][B][Hq][d + 2]: m in log2 units, l, y), and the merge of the shards' partials.
+cudaError_t launch_shard_select(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const float* cand_score,
+                                const int32_t* cand_id, int n_shards, int offset, int32_t* sel_out, cudaStream_t s);
+cudaError_t launch_combine_partial(const Geom& g, const CacheBuffers& cb, const Scratch& sc, int dtype,
+                                   float* partial, cudaStream_t s);
+cudaError_t launch_merge_partials(int n_parts, long long n_rows, int d, const float* parts, int out_dtype, void* out,
+                                  cudaStream_t s);
 // Device-side table checks.
 cudaError_t launch_validate(const Geom& g, const CacheBuffers& cb, uint32_t* err,
                             cudaStream_t s);

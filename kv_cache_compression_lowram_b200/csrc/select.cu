@@ -95,7 +95,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
               float* __restrict__ scores_out, int32_t* __restrict__ sel_out, int tc_q_mode,
-              int do_tail) {
+              int do_tail, SelCand cand) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int u = blockIdx.x;
   const Unit un = unit_of(g, u);
@@ -204,6 +204,7 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
   int32_t* sel_slot = sc.sel_slot + (size_t)u * g.k;
   int32_t* sel_id = sc.sel_id + (size_t)u * g.k;
   int32_t* sel_user = sel_out ? sel_out + ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * g.k : nullptr;
+  const size_t ui = ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv);   // the caller's unit index
   if (rank_topk) {
     // rank of each key among all keys (keys are distinct: the id is in the low bits)
     for (int c = tid; c < g.nC; c += blockDim.x) {
@@ -227,6 +228,10 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
       sel_slot[pos] = sl;
       sel_id[pos] = c;
       if (sel_user) sel_user[pos] = c;
+      if (cand.score) {
+        cand.score[ui * g.k + pos] = sc_s[c];
+        cand.id[ui * g.k + pos] = c + cand.offset;
+      }
     }
   } else {
     bitonic_sort(keys, nCp);
@@ -245,6 +250,10 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
       sel_slot[i] = sl;
       sel_id[i] = id;
       if (sel_user) sel_user[i] = id;
+      if (cand.score) {
+        cand.score[ui * g.k + i] = sc_s[id];
+        cand.id[ui * g.k + i] = id + cand.offset;
+      }
     }
   }
   if (!do_tail) return;
@@ -378,7 +387,7 @@ template <int R, int GQ, int NPL>
 __global__ void __launch_bounds__(kSelThreads, GQ <= 4 ? 3 : 2)
 select_warp_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __restrict__ q,
                    float* __restrict__ scores_out, int32_t* __restrict__ sel_out, int tc_q_mode,
-                   int do_tail) {
+                   int do_tail, SelCand cand) {
   constexpr int D = 128;
   using SM = SelSmem<R, GQ, NPL>;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -535,11 +544,11 @@ select_warp_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
     uint32_t T = 0;
 #pragma unroll 1
     for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = T | (1u << bit);
+      const uint32_t trial = T | (1u << bit);
       int cnt = 0;
 #pragma unroll
-      for (int i = 0; i < NPL; ++i) cnt += key[i] >= cand ? 1 : 0;
-      if (__reduce_add_sync(0xffffffffu, cnt) >= g.k) T = cand;
+      for (int i = 0; i < NPL; ++i) cnt += key[i] >= trial ? 1 : 0;
+      if (__reduce_add_sync(0xffffffffu, cnt) >= g.k) T = trial;
     }
     int gt = 0, eq = 0;
 #pragma unroll
@@ -576,6 +585,11 @@ select_warp_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
           sel_slot[pos] = sl;
           sel_id[pos] = c;
           if (sel_user) sel_user[pos] = c;
+          if (cand.score) {
+            const size_t ui = ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * g.k + pos;
+            cand.score[ui] = sm.score[c];
+            cand.id[ui] = c + cand.offset;
+          }
         }
         ++pos;
       }
@@ -717,32 +731,34 @@ namespace {
 
 template <int R, int GQ, int NPL>
 cudaError_t launch_select_warp(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const void* q,
-                               float* scores_out, int32_t* sel_out, int tc_q_mode, bool tail, cudaStream_t s) {
+                               float* scores_out, int32_t* sel_out, int tc_q_mode, bool tail, cudaStream_t s,
+                               SelCand cand) {
   using SM = SelSmem<R, GQ, NPL>;
   auto k = select_warp_kernel<R, GQ, NPL>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SM));
   if (e != cudaSuccess) return e;
   k<<<g.U, kSelThreads, sizeof(SM), s>>>(g, cb, sc, static_cast<const __nv_bfloat16*>(q), scores_out, sel_out,
-                                         tc_q_mode, tail ? 1 : 0);
+                                         tc_q_mode, tail ? 1 : 0, cand);
   return cudaGetLastError();
 }
 
 template <int R, int GQ>
 cudaError_t launch_select_fast(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const void* q,
-                               float* scores_out, int32_t* sel_out, int tc_q_mode, bool tail, cudaStream_t s) {
-  if (g.nC <= 256) return launch_select_warp<R, GQ, 8>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s);
-  if (g.nC <= 512) return launch_select_warp<R, GQ, 16>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s);
-  return launch_select_warp<R, GQ, 32>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s);
+                               float* scores_out, int32_t* sel_out, int tc_q_mode, bool tail, cudaStream_t s,
+                               SelCand cand) {
+  if (g.nC <= 256) return launch_select_warp<R, GQ, 8>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s, cand);
+  if (g.nC <= 512) return launch_select_warp<R, GQ, 16>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s, cand);
+  return launch_select_warp<R, GQ, 32>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s, cand);
 }
 
 }  // namespace
 
 cudaError_t launch_select(const Geom& g, const CacheBuffers& cb, const Scratch& sc, int dtype,
                           const void* q, float* scores_out, int32_t* sel_out, int tc_q_mode,
-                          bool tail, cudaStream_t s) {
+                          bool tail, cudaStream_t s, SelCand cand) {
   if (dtype == LOWRAM_BF16 && g.d == 128 && g.nC <= kRankMax && (reinterpret_cast<uintptr_t>(q) & 15) == 0) {
 #define LOWRAM_SELECT_FAST(RR, GG) \
-    if (g.r == RR && g.g == GG) return launch_select_fast<RR, GG>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s);
+    if (g.r == RR && g.g == GG) return launch_select_fast<RR, GG>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s, cand);
     LOWRAM_SELECT_FAST(128, 4)
     LOWRAM_SELECT_FAST(128, 8)
     LOWRAM_SELECT_FAST(64, 4)
@@ -756,13 +772,13 @@ cudaError_t launch_select(const Geom& g, const CacheBuffers& cb, const Scratch& 
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<g.U, kThreads, smem, s>>>(g, cb, sc, static_cast<const float*>(q), scores_out, sel_out,
-                                  tc_q_mode, tail ? 1 : 0);
+                                  tc_q_mode, tail ? 1 : 0, cand);
   } else {
     auto k = select_kernel<__nv_bfloat16>;
     cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<g.U, kThreads, smem, s>>>(g, cb, sc, static_cast<const __nv_bfloat16*>(q), scores_out,
-                                  sel_out, tc_q_mode, tail ? 1 : 0);
+                                  sel_out, tc_q_mode, tail ? 1 : 0, cand);
   }
   return cudaGetLastError();
 }

@@ -131,7 +131,7 @@ extern "C" lowram_status lowram_decode_attn_static(const lowram_config* cfg,
   unsigned char* sb = static_cast<unsigned char*>(base);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
 
-  Scratch sc;
+  Scratch sc{};
   sc.err = reinterpret_cast<uint32_t*>(sb + o_err);
   sc.qt = reinterpret_cast<float*>(sb + o_qt);
   sc.qt_tc = nullptr;
