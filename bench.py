@@ -56,6 +56,9 @@ def parse():
                     help="with --dense: this batch instead of the largest that fits (profiling)")
     ap.add_argument("--repack", action="store_true",
                     help="only the decode-loop upkeep: C tail appends and one chunk re-pack per step")
+    ap.add_argument("--shards", type=int, default=0,
+                    help="context-sharded decode of the workload over this many chunk shards: one shard "
+                         "per rank under torchrun (NCCL gathers), else every shard on this one GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -790,6 +793,77 @@ def run_reference(args, ws, rank):
     }
 
 
+SHARD_METRIC = "context-sharded decode-attn queries/s (one sequence's chunks split over shards)"
+
+
+def run_shards(args, ws, rank, local):
+    """Context-sharded decode of the workload: its chunks split into P equal contiguous ranges.
+
+    Under torchrun (P = world size) each rank holds one shard and the protocol's two gathers
+    are NCCL all-gathers; on one GPU the P shards run one after another on the same device and
+    the gathers are device copies (torch.stack), so the time is that of P shards' kernels in
+    sequence, not a multi-GPU time.  One step = phase 1 on every shard, gather, phase 2,
+    gather, merge.  Timed with CUDA events, max over ranks."""
+    import kv_cache_compression_lowram_b200 as K
+    from kv_cache_compression_lowram_b200.sharded import ShardDecoder, all_gather
+    cfg = S.CONFIGS[args.config]
+    P = args.shards if ws == 1 else ws
+    if ws > 1 and args.shards not in (0, ws):
+        raise SystemExit("--shards must equal the world size under torchrun")
+    nC = cfg.n_chunks
+    bounds = [nC * s // P for s in range(P + 1)]
+    dev = torch.device("cuda", local)
+    cache = S.make_cache(cfg, device=dev)            # the same seeded cache on every rank
+    q = S.make_queries(cache)
+    mine = range(P) if ws == 1 else [rank]
+    decs = {}
+    for s_ in mine:
+        sh = S.shard_chunks(cache, bounds[s_], bounds[s_ + 1], keep_tail=(s_ == P - 1))
+        decs[s_] = ShardDecoder(K.LowramCache.from_synth(sh), bounds[s_], P)
+        del sh
+    del cache
+    torch.cuda.empty_cache()
+    gather = all_gather() if ws > 1 else None
+
+    def step():
+        if ws > 1:
+            return decs[rank].decode(q, gather=gather)[0]
+        cands = [decs[s_].candidates(q) for s_ in range(P)]
+        cs_all = torch.stack([c[0] for c in cands])
+        ci_all = torch.stack([c[1] for c in cands])
+        parts = torch.stack([decs[s_].partial(cs_all, ci_all)[0] for s_ in range(P)])
+        return decs[0].merge(parts)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    clocks = ClockSampler(local)
+    barrier(ws)
+    clocks.start()
+    time.sleep(0.3)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    queries = cfg.batch * cfg.n_layers * args.steps
+    value, ms_total = aggregate_rate(queries / ws, start.elapsed_time(end), ws)
+    for d in decs.values():
+        d.cache.close()
+    return {
+        "metric": SHARD_METRIC, "value": round(value, 1), "unit": "queries/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_total / args.steps, 4), "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": cfg.dtype, "data": "synthetic", "impl": "lowram_sharded",
+        "config": {"workload": cfg.name, "shards": P, "chunk_bounds": bounds,
+                   "placement": "one shard per rank, NCCL all-gathers" if ws > 1 else
+                   "all shards on one GPU in sequence, gathers as device copies"},
+        "gpu_launches": (5 * P + 1) * args.steps if ws == 1 else 6 * args.steps, "clocks": clk,
+    }
+
+
 def main():
     args = parse()
     ws, rank, local = dist_init()
@@ -801,11 +875,13 @@ def main():
         line = run_encode(args, ws, rank, local)
     elif args.repack:
         line = run_repack(args, ws, rank, local)
+    elif args.shards:
+        line = run_shards(args, ws, rank, local)
     else:
         line = run_lowram(args, ws, rank, local)
     if rank == 0 and line is not None:
         print(json.dumps(line), flush=True)
-    if args.sweep and args.impl == "lowram" and not (args.dense or args.encode or args.repack):
+    if args.sweep and args.impl == "lowram" and not (args.dense or args.encode or args.repack or args.shards):
         import gc
         for b in (1, 4, 16, 32, 64):
             args.config = f"llama8b_32k_bf16_b{b}"

@@ -7,6 +7,7 @@
 // delta for the worst tokens), inside the attention of "OjaKV", section 3.
 // Also: the create-time fold W1' = W1 B_l^T and the device-side table check.
 #include "lowram_internal.cuh"
+#include "warp_mma.cuh"
 
 namespace lowram {
 namespace {
@@ -122,164 +123,180 @@ combine_kernel(Geom g, CacheBuffers cb, Scratch sc, T* __restrict__ out) {
   }
 }
 
-// The same merge for bf16 with d = 128, h = 256, g in {4, 8}, arranged as one round trip to
-// memory: every thread issues all its loads on entry -- its half of one W2 row (16 x 16
-// bytes) and, for each of its float4 slices of the weighted sums, the slice of every piece
-// record with that head's running max and sum -- then derives the merge weights of its
-// head itself (max over the pieces, 2^(m_r - M)), so the only barrier is the one before
-// the second predictor layer reads the merged hidden sums.  Up to kFastRec pieces per unit
-// (a unit's k chunk tiles touch at most two CTAs at the bench sizes; more take the generic kernel).
-constexpr int kFastRec = 2;
+// The same merge for bf16 with d = 128, h = 256, g in {4, 8}: one CTA for up to 16 / g units
+// of one (layer, KV head), so W2 is read once for all of them and its product with their 16
+// merged hidden-sum vectors runs as warp MMAs (mma.sync, fp32 accumulation; each fp32 sum is
+// split into bf16 hi + lo columns so the product keeps fp32-level accuracy).  W2 streams into
+// padded shared memory (rows 528 bytes apart: conflict-free ldmatrix) while the pieces are
+// merged.  Up to kCombPieces pieces per unit; more take the generic kernel.
+constexpr int kCombPieces = 8;
+constexpr int kCombThreads = 256;
 
 template <int GQ>
-__global__ void __launch_bounds__(kThreads, 2)
-combine_fast_kernel(Geom g, CacheBuffers cb, Scratch sc, __nv_bfloat16* __restrict__ out) {
-  constexpr int D = 128, H = 256;
-  constexpr int NH = GQ * H / 4 / kThreads;          // float4 slices of the hidden sums per thread
-  constexpr int ND = (GQ * D / 4 + kThreads - 1) / kThreads;
-  extern __shared__ __align__(16) float sm[];
-  const int u = blockIdx.x;
-  const Unit un = unit_of(g, u);
-  const int l = g.layer0 + un.li;
-  const int tid = threadIdx.x;
-  // this thread's half of W2 row dd, requested before anything else
-  const int dd = tid >> 1, half = tid & 1;
-  const uint4* wrow = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(cb.w2) +
-                                                     (((size_t)l * g.Hkv + un.hkv) * D + dd) * H + half * (H / 2));
-  uint4 w[H / 16];
-#pragma unroll
-  for (int e = 0; e < H / 16; ++e) w[e] = __ldg(wrow + e);
+struct CombSmem {
+  static constexpr int UB = 16 / GQ;          // units per CTA
+  static constexpr int NR = UB * GQ;          // (unit, head) rows: 16
+  static constexpr int WROW = 256 + 8;        // padded row, bf16 elements
+  static constexpr size_t W2 = 0;                                   // bf16 [128][WROW]
+  static constexpr size_t BM = W2 + 128 * WROW * 2;                 // bf16 [2 NR][WROW]: hi, lo rows
+  static constexpr size_t ACCD = BM + 2 * NR * WROW * 2;            // float [NR][128]
+  static constexpr size_t WT = ACCD + NR * 128 * 4;                 // float [NR][kCombPieces + 1]
+  static constexpr size_t LS = WT + NR * (kCombPieces + 1) * 4;     // float [NR]
+  static constexpr size_t PC = LS + NR * 4;                         // int [UB][2]: first piece, pieces
+  static constexpr size_t BYTES = PC + UB * 2 * 4;
+};
 
+__device__ __forceinline__ void cp_async16c(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gsrc)
+               : "memory");
+}
+
+template <int GQ>
+__global__ void __launch_bounds__(kCombThreads, 2)
+combine_mma_kernel(Geom g, CacheBuffers cb, Scratch sc, __nv_bfloat16* __restrict__ out) {
+  constexpr int D = 128, H = 256;
+  using SM = CombSmem<GQ>;
+  constexpr int UB = SM::UB, NR = SM::NR, WROW = SM::WROW;
+  extern __shared__ __align__(128) unsigned char smem[];
+  __nv_bfloat16* w2s = reinterpret_cast<__nv_bfloat16*>(smem + SM::W2);
+  __nv_bfloat16* bms = reinterpret_cast<__nv_bfloat16*>(smem + SM::BM);
+  float (*accd)[D] = reinterpret_cast<float (*)[D]>(smem + SM::ACCD);
+  float (*wt)[kCombPieces + 1] = reinterpret_cast<float (*)[kCombPieces + 1]>(smem + SM::WT);
+  float* ls = reinterpret_cast<float*>(smem + SM::LS);
+  int (*pc)[2] = reinterpret_cast<int (*)[2]>(smem + SM::PC);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nbb = (g.B + UB - 1) / UB;
+  const int pair = blockIdx.x / nbb;              // li * Hkv + hkv
+  const int b0 = (blockIdx.x % nbb) * UB;
+  const int nb = min(UB, g.B - b0);
+  const int li = pair / g.Hkv, hkv = pair % g.Hkv;
+  const int l = g.layer0 + li;
+  const int u0 = pair * g.B + b0;                 // units u0 .. u0 + nb - 1
+  // W2 of (l, hkv) into padded rows, asynchronously: 128 rows x 32 pieces of 16 bytes
+  const __nv_bfloat16* w2 = reinterpret_cast<const __nv_bfloat16*>(cb.w2) + ((size_t)l * g.Hkv + hkv) * D * H;
+#pragma unroll 4
+  for (int x = 0; x < D * H / 8 / kCombThreads; ++x) {
+    const int it = tid + x * kCombThreads, row = it >> 5, piece = it & 31;
+    cp_async16c(w2s + row * WROW + piece * 8, w2 + (size_t)row * H + piece * 8);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  // merge weights of every (unit, head) row: w_r = 2^(m_r - M) over the unit's pieces and tail
   const long long total = (long long)g.U * g.k;
-  const int c0 = cta_of_tile(total, g.P, (long long)u * g.k);
-  const int c1 = cta_of_tile(total, g.P, (long long)(u + 1) * g.k - 1);
-  const int nrec = c1 - c0 + 1;
-  if (nrec > g.max_rec || nrec > kFastRec) {  // cannot happen with a consistent tile partition
-    if (tid == 0) atomicOr(sc.err, ERR_SELECT);
-    return;
-  }
-  float* accH = sm;                 // [GQ][H]
-  float* accD = accH + GQ * H;      // [GQ][D]
-  float* lsum = accD + GQ * D;      // [GQ]
-  const float* trec = sc.tail_part + (size_t)u * g.tail_stride;
-  const float* rec0 = sc.part + (size_t)(u + c0) * g.rec_stride;
-  // merge weights of head j over the pieces (and the tail): w_r = 2^(m_r - M)
-  auto weights = [&](int j, const float (&m)[kFastRec], float mt, float (&wr)[kFastRec], float& wt) {
-    float M = mt;
-#pragma unroll
-    for (int r = 0; r < kFastRec; ++r)
-      if (r < nrec) M = fmaxf(M, m[r]);
-#pragma unroll
-    for (int r = 0; r < kFastRec; ++r) wr[r] = (r < nrec && m[r] != -INFINITY) ? exp2f(m[r] - M) : 0.f;
-    wt = mt == -INFINITY ? 0.f : exp2f(mt - M);
-  };
-  // hidden sums: loads first
-  float4 vh[NH][kFastRec];
-  float mh[NH][kFastRec];
-#pragma unroll
-  for (int q = 0; q < NH; ++q) {
-    const int i4 = tid + q * kThreads, j = (i4 * 4) / H;
-#pragma unroll
-    for (int r = 0; r < kFastRec; ++r) {
-      const float* rec = rec0 + (size_t)r * g.rec_stride;
-      if (r < nrec) {
-        mh[q][r] = rec[j];
-        vh[q][r] = *reinterpret_cast<const float4*>(rec + 2 * GQ + i4 * 4);
+  if (tid < NR) {
+    const int r = tid, bi = r / GQ, j = r % GQ;
+    float L = 0.f;
+    if (bi < nb) {
+      const int u = u0 + bi;
+      const int c0 = cta_of_tile(total, g.P, (long long)u * g.k);
+      const int nrec = cta_of_tile(total, g.P, (long long)(u + 1) * g.k - 1) - c0 + 1;
+      if (j == 0) {
+        pc[bi][0] = c0;
+        pc[bi][1] = nrec;
+        if (nrec > g.max_rec || nrec > kCombPieces) atomicOr(sc.err, ERR_SELECT);   // cannot happen
       }
-    }
-  }
-  // residual / tail sums: loads first
-  float4 vd[ND][kFastRec], vt[ND];
-  float md[ND][kFastRec], mtd[ND];
-#pragma unroll
-  for (int q = 0; q < ND; ++q) {
-    const int i4 = tid + q * kThreads;
-    if (i4 < GQ * D / 4) {
-      const int j = (i4 * 4) / D;
-      mtd[q] = trec[j];
-      vt[q] = *reinterpret_cast<const float4*>(trec + 2 * GQ + i4 * 4);
-#pragma unroll
-      for (int r = 0; r < kFastRec; ++r) {
-        const float* rec = rec0 + (size_t)r * g.rec_stride;
-        if (r < nrec) {
-          md[q][r] = rec[j];
-          vd[q][r] = *reinterpret_cast<const float4*>(rec + 2 * GQ + GQ * H + i4 * 4);
-        }
+      const int np = min(nrec, kCombPieces);
+      const float* trec = sc.tail_part + (size_t)u * g.tail_stride;
+      float M = trec[j];
+      for (int p = 0; p < np; ++p) M = fmaxf(M, sc.part[(size_t)(u + c0 + p) * g.rec_stride + j]);
+      for (int p = 0; p < np; ++p) {
+        const float* rec = sc.part + (size_t)(u + c0 + p) * g.rec_stride;
+        const float w = rec[j] == -INFINITY ? 0.f : exp2f(rec[j] - M);
+        wt[r][p] = w;
+        L = fmaf(w, rec[GQ + j], L);
       }
+      const float w_t = trec[j] == -INFINITY ? 0.f : exp2f(trec[j] - M);
+      wt[r][kCombPieces] = w_t;
+      L = fmaf(w_t, trec[GQ + j], L);
     }
-  }
-  // the softmax denominators
-  if (tid < GQ) {
-    const int j = tid;
-    float m[kFastRec], sr[kFastRec], wr[kFastRec], wt;
-#pragma unroll
-    for (int r = 0; r < kFastRec; ++r) {
-      const float* rec = rec0 + (size_t)r * g.rec_stride;
-      m[r] = r < nrec ? rec[j] : -INFINITY;
-      sr[r] = r < nrec ? rec[GQ + j] : 0.f;
-    }
-    const float mt = trec[j], st = trec[GQ + j];
-    weights(j, m, mt, wr, wt);
-    float L = wt * st;
-#pragma unroll
-    for (int r = 0; r < kFastRec; ++r) L = fmaf(wr[r], sr[r], L);
-    lsum[j] = L;
-  }
-#pragma unroll
-  for (int q = 0; q < NH; ++q) {
-    const int i4 = tid + q * kThreads, j = (i4 * 4) / H;
-    float wr[kFastRec], wt;
-    weights(j, mh[q], trec[j], wr, wt);
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int r = 0; r < kFastRec; ++r) {
-      if (r < nrec) {
-        a.x = fmaf(wr[r], vh[q][r].x, a.x); a.y = fmaf(wr[r], vh[q][r].y, a.y);
-        a.z = fmaf(wr[r], vh[q][r].z, a.z); a.w = fmaf(wr[r], vh[q][r].w, a.w);
-      }
-    }
-    *reinterpret_cast<float4*>(accH + i4 * 4) = a;
-  }
-#pragma unroll
-  for (int q = 0; q < ND; ++q) {
-    const int i4 = tid + q * kThreads;
-    if (i4 < GQ * D / 4) {
-      const int j = (i4 * 4) / D;
-      float wr[kFastRec], wt;
-      weights(j, md[q], mtd[q], wr, wt);
-      float4 a = make_float4(wt * vt[q].x, wt * vt[q].y, wt * vt[q].z, wt * vt[q].w);
-#pragma unroll
-      for (int r = 0; r < kFastRec; ++r) {
-        if (r < nrec) {
-          a.x = fmaf(wr[r], vd[q][r].x, a.x); a.y = fmaf(wr[r], vd[q][r].y, a.y);
-          a.z = fmaf(wr[r], vd[q][r].z, a.z); a.w = fmaf(wr[r], vd[q][r].w, a.w);
-        }
-      }
-      *reinterpret_cast<float4*>(accD + i4 * 4) = a;
-    }
+    ls[r] = L;
   }
   __syncthreads();
-  // second predictor layer: this thread's half row against every head's hidden sums
-  float a[GQ];
+  // merged hidden sums as bf16 hi / lo rows, merged residual + tail sums: thread = (row r,
+  // slice s of 16 hidden units and 8 dimensions)
+  {
+    const int r = tid >> 4, s = tid & 15, bi = r / GQ, j = r % GQ;
+    float hs[16], ds[8];
 #pragma unroll
-  for (int j = 0; j < GQ; ++j) a[j] = 0.f;
+    for (int x = 0; x < 16; ++x) hs[x] = 0.f;
 #pragma unroll
-  for (int e = 0; e < H / 16; ++e) {
-    const uint32_t ww[4] = {w[e].x, w[e].y, w[e].z, w[e].w};
+    for (int x = 0; x < 8; ++x) ds[x] = 0.f;
+    if (bi < nb) {
+      const int u = u0 + bi;
+      const int c0 = pc[bi][0], np = min(pc[bi][1], kCombPieces);
+      for (int p = 0; p < np; ++p) {
+        const float* rec = sc.part + (size_t)(u + c0 + p) * g.rec_stride;
+        const float w = wt[r][p];
+        const float4* hv = reinterpret_cast<const float4*>(rec + 2 * GQ + j * H + s * 16);
+        const float4* dv = reinterpret_cast<const float4*>(rec + 2 * GQ + GQ * H + j * D + s * 8);
 #pragma unroll
-    for (int h2 = 0; h2 < 4; ++h2) {
-      const float v0 = __uint_as_float(ww[h2] << 16), v1 = __uint_as_float(ww[h2] & 0xffff0000u);
-      const int m = half * (H / 2) + e * 8 + 2 * h2;
+        for (int x = 0; x < 4; ++x) {
+          const float4 v = hv[x];
+          hs[4 * x] = fmaf(w, v.x, hs[4 * x]);
+          hs[4 * x + 1] = fmaf(w, v.y, hs[4 * x + 1]);
+          hs[4 * x + 2] = fmaf(w, v.z, hs[4 * x + 2]);
+          hs[4 * x + 3] = fmaf(w, v.w, hs[4 * x + 3]);
+        }
 #pragma unroll
-      for (int j = 0; j < GQ; ++j) a[j] = fmaf(v1, accH[j * H + m + 1], fmaf(v0, accH[j * H + m], a[j]));
+        for (int x = 0; x < 2; ++x) {
+          const float4 v = dv[x];
+          ds[4 * x] = fmaf(w, v.x, ds[4 * x]);
+          ds[4 * x + 1] = fmaf(w, v.y, ds[4 * x + 1]);
+          ds[4 * x + 2] = fmaf(w, v.z, ds[4 * x + 2]);
+          ds[4 * x + 3] = fmaf(w, v.w, ds[4 * x + 3]);
+        }
+      }
+      const float w_t = wt[r][kCombPieces];
+      const float4* tv = reinterpret_cast<const float4*>(sc.tail_part + (size_t)u * g.tail_stride + 2 * GQ + j * D + s * 8);
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        const float4 v = tv[x];
+        ds[4 * x] = fmaf(w_t, v.x, ds[4 * x]);
+        ds[4 * x + 1] = fmaf(w_t, v.y, ds[4 * x + 1]);
+        ds[4 * x + 2] = fmaf(w_t, v.z, ds[4 * x + 2]);
+        ds[4 * x + 3] = fmaf(w_t, v.w, ds[4 * x + 3]);
+      }
+    }
+    __nv_bfloat16 hi[16], lo[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) wm::split_bf16(hs[x], hi[x], lo[x]);
+    *reinterpret_cast<uint4*>(bms + (2 * r) * WROW + s * 16) = *reinterpret_cast<const uint4*>(hi);
+    *reinterpret_cast<uint4*>(bms + (2 * r) * WROW + s * 16 + 8) = *reinterpret_cast<const uint4*>(hi + 8);
+    *reinterpret_cast<uint4*>(bms + (2 * r + 1) * WROW + s * 16) = *reinterpret_cast<const uint4*>(lo);
+    *reinterpret_cast<uint4*>(bms + (2 * r + 1) * WROW + s * 16 + 8) = *reinterpret_cast<const uint4*>(lo + 8);
+#pragma unroll
+    for (int x = 0; x < 8; ++x) accd[r][s * 8 + x] = ds[x];
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+  // y[d][n] = sum_h W2[d][h] Bm[n][h]: warp w takes dimensions 16w .. 16w+15, all 32 columns
+  float acc[4][4];
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int x = 0; x < 4; ++x) acc[nt][x] = 0.f;
+#pragma unroll 4
+  for (int ks = 0; ks < H / 16; ++ks) {
+    uint32_t a[4];
+    wm::ldsm_x4(a, w2s + (16 * warp + (lane & 15)) * WROW + ks * 16 + (lane >> 4) * 8);
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      uint32_t b[2];
+      wm::ldsm_x2(b, bms + (8 * nt + (lane & 7)) * WROW + ks * 16 + ((lane >> 3) & 1) * 8);
+      wm::mma_bf16(acc[nt], a, b);
     }
   }
+  // columns (c, c + 1) of n-tile nt are the hi and lo parts of row r = 4 nt + lane % 4
+  const int gq = lane >> 2;
 #pragma unroll
-  for (int j = 0; j < GQ; ++j) a[j] += __shfl_xor_sync(0xffffffffu, a[j], 1);
-  if (half == 0) {
-    __nv_bfloat16* o = out + ((size_t)(un.li * g.B + un.b) * g.Hq + (size_t)un.hkv * GQ) * D;
-#pragma unroll
-    for (int j = 0; j < GQ; ++j) o[(size_t)j * D + dd] = __float2bfloat16_rn((a[j] + accD[j * D + dd]) / lsum[j]);
+  for (int nt = 0; nt < 4; ++nt) {
+    const int r = 4 * nt + (lane & 3), bi = r / GQ, j = r % GQ;
+    if (bi < nb) {
+      __nv_bfloat16* o = out + ((size_t)(li * g.B + b0 + bi) * g.Hq + (size_t)hkv * GQ + j) * D;
+      const int d0 = 16 * warp + gq;
+      o[d0] = __float2bfloat16_rn((acc[nt][0] + acc[nt][1] + accd[r][d0]) / ls[r]);
+      o[d0 + 8] = __float2bfloat16_rn((acc[nt][2] + acc[nt][3] + accd[r][d0 + 8]) / ls[r]);
+    }
   }
 }
 
@@ -397,11 +414,14 @@ cudaError_t launch_combine(const Geom& g, const CacheBuffers& cb, const Scratch&
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     k<<<g.U, kThreads, smem, s>>>(g, cb, sc, static_cast<float*>(out));
-  } else if (g.d == 128 && g.h == 256 && (g.g == 4 || g.g == 8) && g.max_rec <= kFastRec) {
-    auto k = g.g == 4 ? combine_fast_kernel<4> : combine_fast_kernel<8>;
-    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  } else if (g.d == 128 && g.h == 256 && (g.g == 4 || g.g == 8) && g.max_rec <= kCombPieces) {
+    auto k = g.g == 4 ? combine_mma_kernel<4> : combine_mma_kernel<8>;
+    const size_t sm = g.g == 4 ? CombSmem<4>::BYTES : CombSmem<8>::BYTES;
+    const int ub = 16 / g.g;
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    k<<<g.U, kThreads, smem, s>>>(g, cb, sc, static_cast<__nv_bfloat16*>(out));
+    const unsigned grid = (unsigned)(g.n_layers * g.Hkv) * (unsigned)((g.B + ub - 1) / ub);
+    k<<<grid, kCombThreads, sm, s>>>(g, cb, sc, static_cast<__nv_bfloat16*>(out));
   } else {
     auto k = combine_kernel<__nv_bfloat16>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

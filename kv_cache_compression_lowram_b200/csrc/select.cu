@@ -15,6 +15,8 @@
 // and tail logit is one thread's dot product over 16-byte loads; top-k of up to 1024 chunks
 // is a rank count over the keys in shared memory (bitonic sort above that).
 #include "lowram_internal.cuh"
+#include "tc_ptx.cuh"
+#include "warp_mma.cuh"
 
 namespace lowram {
 namespace {
@@ -327,16 +329,18 @@ select_kernel(Geom g, CacheBuffers cb, Scratch sc, const T* __restrict__ q,
 }
 
 // ---------------------------------------------------------------------------- fast path
-// The same computation for the common shapes (bf16, d = 128, r in {64, 128}, g in {4, 8},
-// at most 1024 chunks), one CTA of 8 warps per unit.  The chunk selection and the raw tail's
-// partial softmax do not depend on each other: warps 0-3 project the queries, score the
-// chunks and select, warps 4-7 run the tail, each group with its own named barrier.  The
-// top-k needs no barrier at all: one warp holds every chunk's order key (nC / 32 per lane)
-// and finds the k-th largest by a bitwise binary search with warp-wide counts, then takes
-// the keys equal to it in ascending chunk id.  The tail's value rows are staged into shared
-// memory by cp.async at entry, so their latency hides under the logits.  Shared memory and
-// registers stay small (several units per SM), so a whole call runs in about one wave.
-constexpr int kSelThreads = 256;     // warps 0-3: selection; warps 4-7: raw tail
+// The same computation for the common shapes (bf16, d = 128, r in {64, 128}, g in {4, 8}, at
+// most 1024 chunks), as two CTAs of 4 warps per unit: the chunk selection and the raw tail's
+// partial softmax do not depend on each other.  Their small dense products run as warp MMAs
+// (mma.sync, bf16 in, fp32 accumulation) on rows staged into padded shared memory by cp.async:
+// the query projection B_l q_j (exact bf16 inputs), the chunk scores summary . qsum (qsum, an
+// fp32 vector, split into bf16 hi + lo columns: ~16 significant bits), the tail logits K q^T
+// and the tail sums P V (P split the same way).  The summary rows come in passes of 128
+// through two buffers, the second first holding the basis.  The top-k needs no block barrier:
+// one warp holds every chunk's order key (nC / 32 per lane) and finds the k-th largest by a
+// bitwise binary search with warp-wide counts, then takes the keys equal to it in ascending
+// chunk id.
+constexpr int kSplitThreads = 128;
 constexpr int kSelTB = 128;          // tail tokens per block (one per tail thread)
 
 // 16-byte asynchronous copy global -> shared (zero-filled when !valid); completes at the
@@ -348,7 +352,6 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, boo
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void bar_named(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
 // Exclusive prefix sum over the lanes of a warp.
 __device__ __forceinline__ int warp_excl_scan(int v) {
@@ -371,174 +374,201 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& w, float (&v)[8]) {
   }
 }
 
-template <int R, int GQ, int NPL>
-struct SelSmem {
-  float qs[GQ][128];              // the unit's queries
-  float qsum[R];                  // sum_j B_l q_j
-  float score[NPL * 32];          // chunk scores (ids >= nC unused)
-  float p[kSelTB][GQ];            // tail probabilities of the current block, token-major
-  float red_max[4][GQ];           // per tail warp: block maxima, then block sums
-  float red_sum[4][GQ];
-  float pv[GQ][128];              // the second token half's P.V sums
-  __align__(16) __nv_bfloat16 v[kSelTB][128];   // the block's tail values
+// dot(8 bf16, 8 consecutive floats of x)
+__device__ __forceinline__ float dot8(const uint4& w, const float* x, float a) {
+  float v[8];
+  bf16x8_to_f32(w, v);
+  const float4 q0 = *reinterpret_cast<const float4*>(x);
+  const float4 q1 = *reinterpret_cast<const float4*>(x + 4);
+  a = fmaf(v[0], q0.x, fmaf(v[1], q0.y, fmaf(v[2], q0.z, fmaf(v[3], q0.w, a))));
+  return fmaf(v[4], q1.x, fmaf(v[5], q1.y, fmaf(v[6], q1.z, fmaf(v[7], q1.w, a))));
+}
+
+// Shared-memory layout of the fast kernel (byte offsets).  Rows staged from global memory
+// (basis, summaries, tail keys and values) are 16-byte-chunk swizzled: chunk c of row r sits
+// at chunk (c & ~7) | ((c ^ r) & 7), so the 8 rows an ldmatrix reads start in 8 different bank
+// groups without padding.  The small operands built in the kernel are padded rows instead.
+template <int R, int GQ>
+struct MmaSmem {
+  static constexpr int PAD = 136;                         // padded small-operand row, bf16
+  static constexpr int PASS = 128;                        // summary rows per staged pass
+  static constexpr size_t QB = 0;                         // bf16 [8][PAD]: the unit's queries (rows >= GQ zero)
+  // selection CTA
+  static constexpr size_t QS = QB + 8 * PAD * 2;          // bf16 [8][PAD]: qsum hi, lo (rows >= 2 zero)
+  static constexpr size_t SCORE = QS + 8 * PAD * 2;       // float [1024]: chunk scores by slot, then by id
+  // tail CTA (over the selection CTA's QS / SCORE)
+  static constexpr size_t PB = QS;                        // bf16 [16][PAD]: probabilities hi / lo
+  static constexpr size_t MISC = PB + 16 * PAD * 2;       // float [2][4][GQ]: block maxima, sums
+  static constexpr size_t BUF0 = (SCORE + 1024 * 4 + 127) / 128 * 128;   // 32 KB of staged rows
+  static constexpr size_t BUF1 = BUF0 + 32768;                           // 32 KB of staged rows
+  static constexpr size_t BYTES = BUF1 + 32768;
+  static_assert(MISC + 2 * 4 * GQ * 4 <= BUF0, "tail scratch overlaps the staged rows");
 };
 
+// Byte offset of 16-byte chunk c of row r in a swizzled block of rows of row_bytes.
+__device__ __forceinline__ uint32_t swz(int r, int c, int row_bytes) {
+  return (uint32_t)(r * row_bytes + (((c & 7) ^ (r & 7)) | (c & ~7)) * 16);
+}
+
+// CTA 2u (or u without a tail) selects for unit u, CTA 2u + 1 runs u's raw tail.
 template <int R, int GQ, int NPL>
-__global__ void __launch_bounds__(kSelThreads, GQ <= 4 ? 3 : 2)
-select_warp_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __restrict__ q,
-                   float* __restrict__ scores_out, int32_t* __restrict__ sel_out, int tc_q_mode,
-                   int do_tail, SelCand cand) {
+__global__ void __launch_bounds__(kSplitThreads, 3)
+select_mma_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __restrict__ q,
+                  float* __restrict__ scores_out, int32_t* __restrict__ sel_out, int tc_q_mode,
+                  int do_tail, SelCand cand) {
   constexpr int D = 128;
-  using SM = SelSmem<R, GQ, NPL>;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  SM& sm = *reinterpret_cast<SM*>(smem_raw);
-  const int u = blockIdx.x;
+  using SM = MmaSmem<R, GQ>;
+  constexpr int PAD = SM::PAD;
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  __nv_bfloat16* qb = reinterpret_cast<__nv_bfloat16*>(smem_raw + SM::QB);
+  unsigned char* buf[2] = {smem_raw + SM::BUF0, smem_raw + SM::BUF1};
+  const int u = do_tail ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const bool tail_cta = do_tail && (blockIdx.x & 1);
   const Unit un = unit_of(g, u);
   const int l = g.layer0 + un.li;
   const int grp = l / g.G;
   const int NG = g.L / g.G;
   const int nC = g.nC;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-  // tail set-up first: its value rows start streaming into shared memory right away
-  int tl = 0;
-  const size_t toff = (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (size_t)g.T * D;
-  const __nv_bfloat16* tk = reinterpret_cast<const __nv_bfloat16*>(cb.tail_k) + toff;
-  const __nv_bfloat16* tv = reinterpret_cast<const __nv_bfloat16*>(cb.tail_v) + toff;
-  const int tt = tid - 128;   // tail thread index (warps 4-7)
-  auto stage_v = [&](int t0) {   // rows t0 .. t0+127 (zero past the tail)
-#pragma unroll 4
-    for (int k = 0; k < 16; ++k) {
-      const int it = tt + k * 128, t = it >> 4, e = it & 15;
-      const bool in = t0 + t < tl;
-      cp_async16(&sm.v[t][e * 8], in ? tv + (size_t)(t0 + t) * D + e * 8 : tv, in);
+  const int gq = lane >> 2, cq = (lane & 3) * 2;   // MMA fragment row / column base
+  const size_t qoff = ((size_t)(un.li * g.B + un.b) * g.Hq + (size_t)un.hkv * GQ) * D;
+  // rows of `rows` x `width` bf16 elements (width % 64 == 0) from global into swizzled rows
+  auto stage = [&](unsigned char* dst, const __nv_bfloat16* src, int rows, int width) {
+    const int pieces = width / 8;
+    for (int it = tid; it < rows * pieces; it += kSplitThreads) {
+      const int r = it / pieces, pc = it % pieces;
+      cp_async16(dst + swz(r, pc, width * 2), src + (size_t)r * width + pc * 8, true);
     }
     cp_async_commit();
   };
-  if (warp >= 4 && do_tail) {
-    tl = cb.tail_len[un.b];
-    if (tl < 0 || tl > g.T) {
-      if (tt == 0) atomicOr(sc.err, ERR_TAIL_LEN);
-      tl = tl < 0 ? 0 : g.T;
+  // the unit's queries as bf16 B-operand rows (exact: the queries are bf16)
+  auto load_q = [&]() {
+    for (int it = tid; it < 8 * 16; it += kSplitThreads) {
+      const int j = it >> 4, pc = it & 15;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (j < GQ) v = __ldg(reinterpret_cast<const uint4*>(q + qoff + (size_t)j * D) + pc);
+      *reinterpret_cast<uint4*>(qb + j * PAD + pc * 8) = v;
     }
-    if (tl > 0) stage_v(0);
-  }
+  };
 
-  // the unit's queries (GQ x 128 bf16, 16 bytes per thread)
-  const size_t qoff = ((size_t)(un.li * g.B + un.b) * g.Hq + (size_t)un.hkv * GQ) * D;
-  if (tid < GQ * D / 8) {
-    float v[8];
-    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(q + qoff) + tid), v);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) (&sm.qs[0][0])[tid * 8 + i] = v[i];
-  }
-  __syncthreads();
-
-  if (warp < 4) {
+  if (!tail_cta) {
     // ============================================================ chunk selection
-    const int st = tid;   // 0..127
-    // --- qt_j = B_l q_j: PARTS threads per basis row
-    {
-      constexpr int PARTS = 128 / R;
-      constexpr int SEG = D / PARTS;
-      const int i = st / PARTS, part = st % PARTS;
-      const uint4* row = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(cb.basis) +
-                                                        (((size_t)l * g.Hkv + un.hkv) * R + i) * D + part * SEG);
-      float a[GQ];
-#pragma unroll
-      for (int j = 0; j < GQ; ++j) a[j] = 0.f;
-#pragma unroll
-      for (int h8 = 0; h8 < SEG / 32; ++h8) {   // 32 elements (4 loads) at a time
-        uint4 w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) w[e] = __ldg(row + h8 * 4 + e);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float v[8];
-          bf16x8_to_f32(w[e], v);
-          const int col = part * SEG + (h8 * 4 + e) * 8;
-#pragma unroll
-          for (int j = 0; j < GQ; ++j) {
-            const float4 q0 = *reinterpret_cast<const float4*>(&sm.qs[j][col]);
-            const float4 q1 = *reinterpret_cast<const float4*>(&sm.qs[j][col + 4]);
-            a[j] = fmaf(v[0], q0.x, fmaf(v[1], q0.y, fmaf(v[2], q0.z, fmaf(v[3], q0.w, a[j]))));
-            a[j] = fmaf(v[4], q1.x, fmaf(v[5], q1.y, fmaf(v[6], q1.z, fmaf(v[7], q1.w, a[j]))));
-          }
-        }
-      }
-      if (PARTS == 2) {
-#pragma unroll
-        for (int j = 0; j < GQ; ++j) a[j] += __shfl_xor_sync(0xffffffffu, a[j], 1);
-      }
-      if (part == 0) {
-        float s = 0.f;
-#pragma unroll
-        for (int j = 0; j < GQ; ++j) s += a[j];
-        sm.qsum[i] = s;
-#pragma unroll
-        for (int j = 0; j < GQ; ++j) {
-          const float v = a[j] * g.qk_scale_log2;
-          sc.qt[((size_t)u * GQ + j) * R + i] = v;
-          // rows >= GQ of the 16-row copy stay zero (cleared when the scratch is created)
-          if (tc_q_mode == 1)
-            reinterpret_cast<__nv_bfloat16*>(sc.qt_tc)[((size_t)u * 16 + j) * R + i] = __float2bfloat16_rn(v);
-          else if (tc_q_mode == 2)
-            reinterpret_cast<__half*>(sc.qt_tc)[((size_t)u * 16 + j) * R + i] = __float2half_rn(v);
-        }
-      }
-    }
-    bar_named(1, 128);
-
-    // --- chunk scores: chunk ids st, st + 128, ...; the whole summary row loaded at once
-    const int16_t* slot = cb.slot ? cb.slot + (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * g.nCs : nullptr;
+    __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(smem_raw + SM::QS);
+    float* score = reinterpret_cast<float*>(smem_raw + SM::SCORE);
     const __nv_bfloat16* summ = reinterpret_cast<const __nv_bfloat16*>(cb.summary) +
                                 (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * (size_t)g.nLs * R;
+    const int n_pass = (g.nL + SM::PASS - 1) / SM::PASS;
+    auto stage_pass = [&](int p) {
+      stage(buf[p & 1], summ + (size_t)p * SM::PASS * R, min(SM::PASS, g.nL - p * SM::PASS), R);
+    };
+    // basis rows into buf[1], the first summary pass into buf[0]
+    stage(buf[1], reinterpret_cast<const __nv_bfloat16*>(cb.basis) + ((size_t)l * g.Hkv + un.hkv) * R * D, R, D);
+    stage_pass(0);
+    load_q();
+    for (int it = tid; it < 6 * PAD / 8; it += kSplitThreads)   // rows 2..7 of the qsum operand stay zero
+      *reinterpret_cast<uint4*>(qs + 2 * PAD + it * 8) = make_uint4(0, 0, 0, 0);
+    asm volatile("cp.async.wait_group 1;" ::: "memory");   // the basis
+    __syncthreads();
+    // --- qt[i][j] = sum_e B_l[i][e] q_j[e]: M = R basis rows, N = 8 (heads), K = 128; warp w
+    // takes row tiles w, w + 4, ...
+    for (int mt = warp; mt < R / 16; mt += 4) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        uint32_t a[4], b[2];
+        wm::ldsm_x4(a, buf[1] + swz(16 * mt + (lane & 15), 2 * ks + (lane >> 4), D * 2));
+        wm::ldsm_x2(b, qb + (lane & 7) * PAD + ks * 16 + ((lane >> 3) & 1) * 8);
+        wm::mma_bf16(acc, a, b);
+      }
+      // acc: (row i = 16 mt + gq [+ 8], heads cq, cq + 1)
+#pragma unroll
+      for (int h8 = 0; h8 < 2; ++h8) {
+        const int i = 16 * mt + gq + 8 * h8;
+        const float v0 = acc[2 * h8], v1 = acc[2 * h8 + 1];
+        float part = (cq < GQ ? v0 : 0.f) + (cq + 1 < GQ ? v1 : 0.f);
+        part += __shfl_xor_sync(0xffffffffu, part, 1);
+        part += __shfl_xor_sync(0xffffffffu, part, 2);
+        if ((lane & 3) == 0) {   // qsum[i] as bf16 hi / lo rows of the score operand
+          __nv_bfloat16 hi, lo;
+          wm::split_bf16(part, hi, lo);
+          qs[i] = hi;
+          qs[PAD + i] = lo;
+        }
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const int j = cq + x;
+          if (j < GQ) {
+            const float v = (x ? v1 : v0) * g.qk_scale_log2;
+            sc.qt[((size_t)u * GQ + j) * R + i] = v;
+            // rows >= GQ of the 16-row copy stay zero (cleared when the scratch is created)
+            if (tc_q_mode == 1)
+              reinterpret_cast<__nv_bfloat16*>(sc.qt_tc)[((size_t)u * 16 + j) * R + i] = __float2bfloat16_rn(v);
+            else if (tc_q_mode == 2)
+              reinterpret_cast<__half*>(sc.qt_tc)[((size_t)u * 16 + j) * R + i] = __float2half_rn(v);
+          }
+        }
+      }
+    }
+    __syncthreads();   // buf[1] (the basis) is free; qsum is complete
+    if (n_pass > 1) stage_pass(1);
+    // --- scores by live slot, pass by pass: S[c] = summary[c] . (qsum hi + qsum lo)
     const float inv_sqrt_d = rsqrtf((float)D);
+    for (int p = 0; p < n_pass; ++p) {
+      if (p + 1 < n_pass) asm volatile("cp.async.wait_group 1;" ::: "memory");
+      else asm volatile("cp.async.wait_group 0;" ::: "memory");
+      __syncthreads();
+      const int rows = min(SM::PASS, g.nL - p * SM::PASS);
+      const unsigned char* sb = buf[p & 1];
+      for (int mt = warp; mt * 16 < rows; mt += 4) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < R / 16; ++ks) {
+          uint32_t a[4], b[2];
+          // rows past the pass's last hold stale data: their results are not stored
+          wm::ldsm_x4(a, sb + swz(16 * mt + (lane & 15), 2 * ks + (lane >> 4), R * 2));
+          wm::ldsm_x2(b, qs + (lane & 7) * PAD + ks * 16 + ((lane >> 3) & 1) * 8);
+          wm::mma_bf16(acc, a, b);
+        }
+        if ((lane & 3) == 0) {   // columns 0, 1 = the hi and lo parts
+          const int r0 = p * SM::PASS + 16 * mt + gq;
+          if (16 * mt + gq < rows) score[r0] = (acc[0] + acc[1]) * inv_sqrt_d;
+          if (16 * mt + gq + 8 < rows) score[r0 + 8] = (acc[2] + acc[3]) * inv_sqrt_d;
+        }
+      }
+      __syncthreads();   // buf[p & 1] is free
+      if (p + 2 < n_pass) stage_pass(p + 2);
+    }
+    // scores by chunk id (evicted chunks -inf); written in place from the top, since slot <= id
+    const int16_t* slot = cb.slot ? cb.slot + (((size_t)un.b * NG + grp) * g.Hkv + un.hkv) * g.nCs : nullptr;
     float* so = scores_out ? scores_out + ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * nC : nullptr;
-#pragma unroll 1
-    for (int c = st; c < NPL * 32; c += 128) {
-      float s = -INFINITY;
+    float sv[NPL * 32 / kSplitThreads];
+#pragma unroll
+    for (int x = 0; x < NPL * 32 / kSplitThreads; ++x) {
+      const int c = tid + x * kSplitThreads;
+      float v = -INFINITY;
       if (c < nC) {
         const int sl = slot ? (int)slot[c] : c;
-        if (sl >= 0 && sl < g.nL) {
-          const uint4* row = reinterpret_cast<const uint4*>(summ + (size_t)sl * R);
-          float a0 = 0.f, a1 = 0.f;
-#pragma unroll
-          for (int h8 = 0; h8 < R / 64; ++h8) {   // 64 ranks (8 loads) at a time
-            uint4 w[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) w[e] = __ldg(row + h8 * 8 + e);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              float v[8];
-              bf16x8_to_f32(w[e], v);
-              const int col = (h8 * 8 + e) * 8;
-              const float4 q0 = *reinterpret_cast<const float4*>(&sm.qsum[col]);
-              const float4 q1 = *reinterpret_cast<const float4*>(&sm.qsum[col + 4]);
-              a0 = fmaf(v[0], q0.x, fmaf(v[2], q0.z, fmaf(v[4], q1.x, fmaf(v[6], q1.z, a0))));
-              a1 = fmaf(v[1], q0.y, fmaf(v[3], q0.w, fmaf(v[5], q1.y, fmaf(v[7], q1.w, a1))));
-            }
-          }
-          s = (a0 + a1) * inv_sqrt_d;
-        } else if (sl >= g.nL) {
-          atomicOr(sc.err, ERR_SLOT);
-        }
-        if (so) so[c] = s;
+        if (sl >= 0 && sl < g.nL) v = score[sl];
+        else if (sl >= g.nL) atomicOr(sc.err, ERR_SLOT);
+        if (so) so[c] = v;
       }
-      sm.score[c] = s;
+      sv[x] = v;
     }
-    bar_named(1, 128);
+    __syncthreads();
+#pragma unroll
+    for (int x = 0; x < NPL * 32 / kSplitThreads; ++x) score[tid + x * kSplitThreads] = sv[x];
+    __syncthreads();
     if (warp != 0) return;
 
     // --- top-k (one warp): lane holds chunks lane*NPL .. lane*NPL + NPL-1; the order key
     // of a score is monotone in the score, and ids >= nC get key 0 (below every chunk's)
     uint32_t key[NPL];
 #pragma unroll
-    for (int i = 0; i < NPL; i += 4) {
-      const float4 f = *reinterpret_cast<const float4*>(&sm.score[lane * NPL + i]);
+    for (int x = 0; x < NPL; x += 4) {
+      const float4 f = *reinterpret_cast<const float4*>(&score[lane * NPL + x]);
       const float fv[4] = {f.x, f.y, f.z, f.w};
 #pragma unroll
-      for (int x = 0; x < 4; ++x) key[i + x] = lane * NPL + i + x < nC ? float_order(fv[x]) : 0u;
+      for (int y = 0; y < 4; ++y) key[x + y] = lane * NPL + x + y < nC ? float_order(fv[y]) : 0u;
     }
     // the k-th largest key: the largest T with #{key >= T} >= k, bit by bit from the top
     uint32_t T = 0;
@@ -547,35 +577,36 @@ select_warp_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
       const uint32_t trial = T | (1u << bit);
       int cnt = 0;
 #pragma unroll
-      for (int i = 0; i < NPL; ++i) cnt += key[i] >= trial ? 1 : 0;
+      for (int x = 0; x < NPL; ++x) cnt += key[x] >= trial ? 1 : 0;
       if (__reduce_add_sync(0xffffffffu, cnt) >= g.k) T = trial;
     }
     int gt = 0, eq = 0;
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      gt += key[i] > T ? 1 : 0;
-      eq += key[i] == T ? 1 : 0;
+    for (int x = 0; x < NPL; ++x) {
+      gt += key[x] > T ? 1 : 0;
+      eq += key[x] == T ? 1 : 0;
     }
     const int need_eq = g.k - (int)__reduce_add_sync(0xffffffffu, gt);   // >= 1 keys equal to T, lowest ids
     int eq_rank = warp_excl_scan(eq);
     uint32_t take = 0;
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      if (key[i] > T) {
-        take |= 1u << i;
-      } else if (key[i] == T) {
-        if (eq_rank < need_eq) take |= 1u << i;
+    for (int x = 0; x < NPL; ++x) {
+      if (key[x] > T) {
+        take |= 1u << x;
+      } else if (key[x] == T) {
+        if (eq_rank < need_eq) take |= 1u << x;
         ++eq_rank;
       }
     }
     int pos = warp_excl_scan(__popc(take));
     int32_t* sel_slot = sc.sel_slot + (size_t)u * g.k;
     int32_t* sel_id = sc.sel_id + (size_t)u * g.k;
-    int32_t* sel_user = sel_out ? sel_out + ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * g.k : nullptr;
+    const size_t ui = (size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv;   // the caller's unit index
+    int32_t* sel_user = sel_out ? sel_out + ui * g.k : nullptr;
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      if (take & (1u << i)) {
-        const int c = lane * NPL + i;
+    for (int x = 0; x < NPL; ++x) {
+      if (take & (1u << x)) {
+        const int c = lane * NPL + x;
         int sl = slot ? (int)slot[c] : c;
         if (sl < 0 || sl >= g.nL) {
           atomicOr(sc.err, ERR_SELECT);
@@ -586,9 +617,8 @@ select_warp_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
           sel_id[pos] = c;
           if (sel_user) sel_user[pos] = c;
           if (cand.score) {
-            const size_t ui = ((size_t)(un.li * g.B + un.b) * g.Hkv + un.hkv) * g.k + pos;
-            cand.score[ui] = sm.score[c];
-            cand.id[ui] = c + cand.offset;
+            cand.score[ui * g.k + pos] = score[c];
+            cand.id[ui * g.k + pos] = c + cand.offset;
           }
         }
         ++pos;
@@ -596,122 +626,178 @@ select_warp_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __r
     }
     return;
   }
-  if (!do_tail) return;
 
   // ============================================================ raw tail
-  // Blocks of 128 tokens: thread tt's logits are token t0 + tt's (all heads); its P.V share
-  // is dimension pair dp over one half th of the block's tokens.
-  const int tw = warp - 4;
-  const int dp = tt & 63, th = tt >> 6;
-  float m_run[GQ], l_run[GQ], acc[GQ][2];
+  // Blocks of 128 tokens staged in shared memory: logits L = K q^T (M = tokens, N = heads),
+  // online softmax per head, then acc += P V with P as bf16 hi / lo rows (M = 16) and V read
+  // transposed (N = 128 dimensions, K = tokens); the accumulators stay in registers.
+  __nv_bfloat16* pb = reinterpret_cast<__nv_bfloat16*>(smem_raw + SM::PB);
+  float (*red)[4][GQ] = reinterpret_cast<float (*)[4][GQ]>(smem_raw + SM::MISC);
+  int tl = cb.tail_len[un.b];
+  if (tl < 0 || tl > g.T) {
+    if (tid == 0) atomicOr(sc.err, ERR_TAIL_LEN);
+    tl = tl < 0 ? 0 : g.T;
+  }
+  const size_t toff = (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (size_t)g.T * D;
+  const __nv_bfloat16* tk = reinterpret_cast<const __nv_bfloat16*>(cb.tail_k) + toff;
+  const __nv_bfloat16* tv = reinterpret_cast<const __nv_bfloat16*>(cb.tail_v) + toff;
+  auto stage_block = [&](int t0) {   // rows t0 .. t0+127 of K and V, zeros past the tail
+    for (int it = tid; it < 128 * 16; it += kSplitThreads) {
+      const int r = it >> 4, pc = it & 15;
+      const bool in = t0 + r < tl;
+      cp_async16(buf[0] + swz(r, pc, D * 2), in ? tk + (size_t)(t0 + r) * D + pc * 8 : tk, in);
+      cp_async16(buf[1] + swz(r, pc, D * 2), in ? tv + (size_t)(t0 + r) * D + pc * 8 : tv, in);
+    }
+    cp_async_commit();
+  };
+  if (tl > 0) stage_block(0);
+  load_q();
+  for (int it = tid; it < 16 * PAD / 8; it += kSplitThreads)   // P rows past the heads' stay zero
+    *reinterpret_cast<uint4*>(pb + it * 8) = make_uint4(0, 0, 0, 0);
+  float m_run[GQ], l_run[GQ];
 #pragma unroll
   for (int j = 0; j < GQ; ++j) {
     m_run[j] = -INFINITY;
     l_run[j] = 0.f;
-    acc[j][0] = acc[j][1] = 0.f;
   }
+  float acc[4][4];   // P V: warp w holds dimensions 32 w .. 32 w + 31 (n-tiles 4w .. 4w + 3)
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int x = 0; x < 4; ++x) acc[nt][x] = 0.f;
 #pragma unroll 1
   for (int t0 = 0; t0 < tl; t0 += kSelTB) {
     const int nb = min(kSelTB, tl - t0);
-    float lg[GQ];
+    cp_async_wait_all();
+    __syncthreads();
+    // logits of tokens 32 w .. 32 w + 31 (two m-tiles), heads cq, cq + 1
+    float lg[2][4];
 #pragma unroll
-    for (int j = 0; j < GQ; ++j) lg[j] = -INFINITY;
-    if (tt < nb) {
-      const uint4* krow = reinterpret_cast<const uint4*>(tk + (size_t)(t0 + tt) * D);
-      float a[GQ];
+    for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
-      for (int j = 0; j < GQ; ++j) a[j] = 0.f;
+      for (int x = 0; x < 4; ++x) lg[mt][x] = 0.f;
 #pragma unroll
-      for (int h8 = 0; h8 < 4; ++h8) {   // 32 dims (4 loads) at a time: the running state stays in registers
-        uint4 w[4];
+      for (int ks = 0; ks < D / 16; ++ks) {
+        uint32_t a[4], b[2];
+        wm::ldsm_x4(a, buf[0] + swz(32 * warp + 16 * mt + (lane & 15), 2 * ks + (lane >> 4), D * 2));
+        wm::ldsm_x2(b, qb + (lane & 7) * PAD + ks * 16 + ((lane >> 3) & 1) * 8);
+        wm::mma_bf16(lg[mt], a, b);
+      }
+    }
+    // per head (column): the block's max over this warp's tokens, then over the warps
+    float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) w[e] = __ldg(krow + h8 * 4 + e);
+    for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float v[8];
-          bf16x8_to_f32(w[e], v);
-          const int col = (h8 * 4 + e) * 8;
+      for (int x = 0; x < 4; ++x) {
+        const int t = 32 * warp + 16 * mt + gq + 8 * (x >> 1);
+        lg[mt][x] = t < nb ? lg[mt][x] * g.qk_scale_log2 : -INFINITY;
+        mx[x & 1] = fmaxf(mx[x & 1], lg[mt][x]);
+      }
 #pragma unroll
-          for (int j = 0; j < GQ; ++j) {
-            const float4 q0 = *reinterpret_cast<const float4*>(&sm.qs[j][col]);
-            const float4 q1 = *reinterpret_cast<const float4*>(&sm.qs[j][col + 4]);
-            a[j] = fmaf(v[0], q0.x, fmaf(v[1], q0.y, fmaf(v[2], q0.z, fmaf(v[3], q0.w, a[j]))));
-            a[j] = fmaf(v[4], q1.x, fmaf(v[5], q1.y, fmaf(v[6], q1.z, fmaf(v[7], q1.w, a[j]))));
-          }
+    for (int x = 0; x < 2; ++x) {
+      mx[x] = fmaxf(mx[x], __shfl_xor_sync(0xffffffffu, mx[x], 4));
+      mx[x] = fmaxf(mx[x], __shfl_xor_sync(0xffffffffu, mx[x], 8));
+      mx[x] = fmaxf(mx[x], __shfl_xor_sync(0xffffffffu, mx[x], 16));
+      if (gq == 0 && cq + x < GQ) red[0][warp][cq + x] = mx[x];
+    }
+    __syncthreads();
+    float mnew[2], ps[2] = {0.f, 0.f};
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const int j = cq + x;
+      const float mb = j < GQ ? fmaxf(fmaxf(red[0][0][j], red[0][1][j]), fmaxf(red[0][2][j], red[0][3][j])) : 0.f;
+      mnew[x] = j < GQ ? fmaxf(m_run[j], mb) : 0.f;
+    }
+    // probabilities as bf16 hi / lo rows of the A operand: rows 0 .. GQ-1 hi, GQ .. 2 GQ - 1 lo
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const int j = cq + (x & 1);
+        const int t = 32 * warp + 16 * mt + gq + 8 * (x >> 1);
+        if (j < GQ) {
+          const float pv = exp2f(lg[mt][x] - mnew[x & 1]);   // 0 past the tail
+          ps[x & 1] += pv;
+          __nv_bfloat16 hi, lo;
+          wm::split_bf16(pv, hi, lo);
+          pb[j * PAD + t] = hi;
+          pb[(GQ + j) * PAD + t] = lo;
         }
       }
 #pragma unroll
-      for (int j = 0; j < GQ; ++j) lg[j] = a[j] * g.qk_scale_log2;
+    for (int x = 0; x < 2; ++x) {
+      ps[x] += __shfl_xor_sync(0xffffffffu, ps[x], 4);
+      ps[x] += __shfl_xor_sync(0xffffffffu, ps[x], 8);
+      ps[x] += __shfl_xor_sync(0xffffffffu, ps[x], 16);
+      if (gq == 0 && cq + x < GQ) red[1][warp][cq + x] = ps[x];
     }
-#pragma unroll
-    for (int j = 0; j < GQ; ++j) {
-      const float mx = warp_max(lg[j]);
-      if (lane == 0) sm.red_max[tw][j] = mx;
-    }
-    bar_named(2, 128);
+    __syncthreads();
+    // rescale the running sums per head, then acc += P V over the block
     float alpha[GQ];
 #pragma unroll
     for (int j = 0; j < GQ; ++j) {
-      const float mb = fmaxf(fmaxf(sm.red_max[0][j], sm.red_max[1][j]), fmaxf(sm.red_max[2][j], sm.red_max[3][j]));
-      const float mn = fmaxf(m_run[j], mb);   // finite: the block has at least one token
-      alpha[j] = exp2f(m_run[j] - mn);        // 0 while m_run = -inf
-      const float p = exp2f(lg[j] - mn);      // 0 past the tail
-      sm.p[tt][j] = p;
-      const float ps = warp_sum(p);
-      if (lane == 0) sm.red_sum[tw][j] = ps;
+      const float mb = fmaxf(fmaxf(red[0][0][j], red[0][1][j]), fmaxf(red[0][2][j], red[0][3][j]));
+      const float mn = fmaxf(m_run[j], mb);
+      alpha[j] = exp2f(m_run[j] - mn);   // 0 while m_run = -inf
+      l_run[j] = l_run[j] * alpha[j] + (red[1][0][j] + red[1][1][j]) + (red[1][2][j] + red[1][3][j]);
       m_run[j] = mn;
     }
-    cp_async_wait_all();   // this thread's copies of the block's value rows (the barrier shares them)
-    bar_named(2, 128);
+    // accumulator rows: gq (c0, c1) and gq + 8 (c2, c3) of the 16 P rows; row r's head is r % GQ
+    // when r < 2 GQ (its hi or lo part), none otherwise
 #pragma unroll
-    for (int j = 0; j < GQ; ++j) {
-      l_run[j] = l_run[j] * alpha[j] + (sm.red_sum[0][j] + sm.red_sum[1][j]) + (sm.red_sum[2][j] + sm.red_sum[3][j]);
-      acc[j][0] *= alpha[j];
-      acc[j][1] *= alpha[j];
+    for (int nt = 0; nt < 4; ++nt) {
+      const float a0 = gq < 2 * GQ ? alpha[gq % GQ] : 0.f;
+      const float a1 = gq + 8 < 2 * GQ ? alpha[(gq + 8) % GQ] : 0.f;
+      acc[nt][0] *= a0;
+      acc[nt][1] *= a0;
+      acc[nt][2] *= a1;
+      acc[nt][3] *= a1;
     }
-    const int tb = th * (kSelTB / 2), te = min(tb + kSelTB / 2, nb);
-#pragma unroll 4
-    for (int t = tb; t < te; ++t) {
-      const uint32_t w = *reinterpret_cast<const uint32_t*>(&sm.v[t][2 * dp]);
-      const float v0 = __uint_as_float(w << 16), v1 = __uint_as_float(w & 0xffff0000u);
 #pragma unroll
-      for (int j = 0; j < GQ; j += 4) {
-        const float4 pj = *reinterpret_cast<const float4*>(&sm.p[t][j]);
-        acc[j][0] = fmaf(pj.x, v0, acc[j][0]);
-        acc[j][1] = fmaf(pj.x, v1, acc[j][1]);
-        acc[j + 1][0] = fmaf(pj.y, v0, acc[j + 1][0]);
-        acc[j + 1][1] = fmaf(pj.y, v1, acc[j + 1][1]);
-        acc[j + 2][0] = fmaf(pj.z, v0, acc[j + 2][0]);
-        acc[j + 2][1] = fmaf(pj.z, v1, acc[j + 2][1]);
-        acc[j + 3][0] = fmaf(pj.w, v0, acc[j + 3][0]);
-        acc[j + 3][1] = fmaf(pj.w, v1, acc[j + 3][1]);
+    for (int ks = 0; ks < kSelTB / 16; ++ks) {
+      uint32_t a[4];
+      wm::ldsm_x4(a, pb + (lane & 15) * PAD + ks * 16 + (lane >> 4) * 8);
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        uint32_t b[2];
+        // B = V[token][dim]: k = token rows, n = dims, read transposed
+        wm::ldsm_x2_t(b, buf[1] + swz(ks * 16 + (lane & 15), 4 * warp + nt, D * 2));
+        wm::mma_bf16(acc[nt], a, b);
       }
     }
-    if (t0 + kSelTB < tl) {   // the next block's value rows, once every thread is done with these
-      bar_named(2, 128);
-      stage_v(t0 + kSelTB);
+    if (t0 + kSelTB < tl) {   // every thread is done with this block's rows
+      __syncthreads();
+      stage_block(t0 + kSelTB);
     }
   }
-  // the two token halves' sums, then the tail record (log2-domain max, sum, sums per head)
-  if (th == 1) {
-#pragma unroll
-    for (int j = 0; j < GQ; ++j) {
-      sm.pv[j][2 * dp] = acc[j][0];
-      sm.pv[j][2 * dp + 1] = acc[j][1];
-    }
-  }
-  bar_named(2, 128);
+  // the tail record (log2-domain max, sum, sums per head): hi and lo rows of head j are rows j
+  // and GQ + j of the accumulator
   float* rec = sc.tail_part + (size_t)u * g.tail_stride;
-  if (th == 0) {
+  if (GQ == 8) {
+    // rows gq (hi) and gq + 8 (lo) of the same lane
 #pragma unroll
-    for (int j = 0; j < GQ; ++j) {
-      rec[2 * GQ + j * D + 2 * dp] = acc[j][0] + sm.pv[j][2 * dp];
-      rec[2 * GQ + j * D + 2 * dp + 1] = acc[j][1] + sm.pv[j][2 * dp + 1];
+    for (int nt = 0; nt < 4; ++nt) {
+      const int dd = 32 * warp + 8 * nt + cq;
+      rec[2 * GQ + gq * D + dd] = acc[nt][0] + acc[nt][2];
+      rec[2 * GQ + gq * D + dd + 1] = acc[nt][1] + acc[nt][3];
+    }
+  } else {
+    // GQ = 4: hi rows 0-3 in lanes 0-15, lo rows 4-7 in lanes 16-31 (c0, c1)
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const float o0 = acc[nt][0] + __shfl_xor_sync(0xffffffffu, acc[nt][0], 16);
+      const float o1 = acc[nt][1] + __shfl_xor_sync(0xffffffffu, acc[nt][1], 16);
+      if (gq < GQ) {
+        const int dd = 32 * warp + 8 * nt + cq;
+        rec[2 * GQ + gq * D + dd] = o0;
+        rec[2 * GQ + gq * D + dd + 1] = o1;
+      }
     }
   }
-  if (tt < GQ) {
-    rec[tt] = m_run[tt];
-    rec[GQ + tt] = l_run[tt];
+  if (tid < GQ) {
+    rec[tid] = m_run[tid];
+    rec[GQ + tid] = l_run[tid];
   }
 }
 
@@ -730,15 +816,17 @@ size_t select_smem_bytes(const Geom& g) {
 namespace {
 
 template <int R, int GQ, int NPL>
-cudaError_t launch_select_warp(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const void* q,
-                               float* scores_out, int32_t* sel_out, int tc_q_mode, bool tail, cudaStream_t s,
-                               SelCand cand) {
-  using SM = SelSmem<R, GQ, NPL>;
-  auto k = select_warp_kernel<R, GQ, NPL>;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SM));
+cudaError_t launch_select_split(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const void* q,
+                                float* scores_out, int32_t* sel_out, int tc_q_mode, bool tail, cudaStream_t s,
+                                SelCand cand) {
+  using SM = MmaSmem<R, GQ>;
+  const size_t smem = SM::BYTES;
+  auto k = select_mma_kernel<R, GQ, NPL>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  k<<<g.U, kSelThreads, sizeof(SM), s>>>(g, cb, sc, static_cast<const __nv_bfloat16*>(q), scores_out, sel_out,
-                                         tc_q_mode, tail ? 1 : 0, cand);
+  const unsigned grid = (unsigned)g.U * (tail ? 2u : 1u);
+  k<<<grid, kSplitThreads, smem, s>>>(g, cb, sc, static_cast<const __nv_bfloat16*>(q), scores_out, sel_out,
+                                       tc_q_mode, tail ? 1 : 0, cand);
   return cudaGetLastError();
 }
 
@@ -746,9 +834,9 @@ template <int R, int GQ>
 cudaError_t launch_select_fast(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const void* q,
                                float* scores_out, int32_t* sel_out, int tc_q_mode, bool tail, cudaStream_t s,
                                SelCand cand) {
-  if (g.nC <= 256) return launch_select_warp<R, GQ, 8>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s, cand);
-  if (g.nC <= 512) return launch_select_warp<R, GQ, 16>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s, cand);
-  return launch_select_warp<R, GQ, 32>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s, cand);
+  if (g.nC <= 256) return launch_select_split<R, GQ, 8>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s, cand);
+  if (g.nC <= 512) return launch_select_split<R, GQ, 16>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s, cand);
+  return launch_select_split<R, GQ, 32>(g, cb, sc, q, scores_out, sel_out, tc_q_mode, tail, s, cand);
 }
 
 }  // namespace
