@@ -307,6 +307,10 @@ attend_tc_kernel(Geom g, CacheBuffers cb, Scratch sc, const __grid_constant__ CU
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc->tmem_base;
+  // the set-up above overlaps the selection kernel's end (programmatic dependent launch);
+  // its outputs (projected queries, selected slots) are read only from here on
+  grid_dep_launch();
+  grid_dep_wait();
 
   const uint32_t sW = smem_u32(smem + Lay::OFF_W);
   const uint32_t sA = smem_u32(smem + Lay::OFF_A);
@@ -1005,8 +1009,18 @@ cudaError_t launch_tc_t(const Geom& g, const CacheBuffers& cb, const Scratch& sc
   auto k = attend_tc_kernel<R, C, GQ, I8, TW, CT>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM);
   if (e != cudaSuccess) return e;
-  k<<<g.P, kThreadsTC, Lay::SMEM, s>>>(g, cb, sc, tmW, tmA, tmQ, tmRes);
-  return cudaGetLastError();
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(g.P);
+  lc.blockDim = dim3(kThreadsTC);
+  lc.dynamicSmemBytes = Lay::SMEM;
+  lc.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  // the explicit tile list is read before the set-up: that launch waits for the list's kernel
+  lc.attrs = at;
+  lc.numAttrs = CT ? 0 : 1;
+  return cudaLaunchKernelEx(&lc, k, g, cb, sc, tmW, tmA, tmQ, tmRes);
 }
 
 template <int R, int C, int GQ, bool I8>

@@ -181,6 +181,9 @@ combine_mma_kernel(Geom g, CacheBuffers cb, Scratch sc, __nv_bfloat16* __restric
     cp_async16c(w2s + row * WROW + piece * 8, w2 + (size_t)row * H + piece * 8);
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
+  // W2 streams in while the chunk-attention kernel finishes (programmatic dependent launch);
+  // its partial records are read only after this
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // merge weights of every (unit, head) row: w_r = 2^(m_r - M) over the unit's pieces and tail
   const long long total = (long long)g.U * g.k;
   if (tid < NR) {
@@ -420,8 +423,18 @@ cudaError_t launch_combine(const Geom& g, const CacheBuffers& cb, const Scratch&
     const int ub = 16 / g.g;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
     if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)(g.n_layers * g.Hkv) * (unsigned)((g.B + ub - 1) / ub);
-    k<<<grid, kCombThreads, sm, s>>>(g, cb, sc, static_cast<__nv_bfloat16*>(out));
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3((unsigned)(g.n_layers * g.Hkv) * (unsigned)((g.B + ub - 1) / ub));
+    lc.blockDim = dim3(kCombThreads);
+    lc.dynamicSmemBytes = sm;
+    lc.stream = s;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = at;
+    lc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&lc, k, g, cb, sc, static_cast<__nv_bfloat16*>(out));
+    if (e != cudaSuccess) return e;
   } else {
     auto k = combine_kernel<__nv_bfloat16>;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

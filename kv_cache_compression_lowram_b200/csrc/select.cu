@@ -431,6 +431,7 @@ select_mma_kernel(Geom g, CacheBuffers cb, Scratch sc, const __nv_bfloat16* __re
   const int nC = g.nC;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, cq = (lane & 3) * 2;   // MMA fragment row / column base
+  tc::grid_dep_launch();   // the chunk-attention kernel may start its set-up as SMs free up
   const size_t qoff = ((size_t)(un.li * g.B + un.b) * g.Hq + (size_t)un.hkv * GQ) * D;
   // rows of `rows` x `width` bf16 elements (width % 64 == 0) from global into swizzled rows
   auto stage = [&](unsigned char* dst, const __nv_bfloat16* src, int rows, int width) {

@@ -271,6 +271,13 @@ __device__ __forceinline__ float tanh_mufu(float x) {
   return r;
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization
+// may start while the previous kernel in the stream still runs; grid_dep_wait() blocks until
+// that kernel has completed and its writes are visible (a no-op without the attribute), and
+// grid_dep_launch() lets the next such kernel start launching.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
+
 // One lane of a converged warp (the lowest), chosen with elect.sync.  Issuing tcgen05/TMA
 // work from an elected lane of a converged warp keeps the operands warp-uniform.
 __device__ __forceinline__ bool elect_one() {
