@@ -586,6 +586,45 @@ def make_queries(cache: SynthCache, layer0: int = 0, n_layers: Optional[int] = N
     return out.to(cfg.torch_dtype)
 
 
+def make_query_steps(cache: SynthCache, n_steps: int, rho: float, drift: float, layer0: int = 0,
+                     n_layers: Optional[int] = None, seed_offset: int = 0):
+    """Decode queries of n_steps consecutive steps, each [n_layers][B][Hq][d], whose selections
+    persist: per unit the query is z_t / sqrt(d) + beta (kbar_c1 / |kbar_c1| + kbar_c2 /
+    |kbar_c2|) as in ``make_queries``, with AR(1) noise z_t = rho z_{t-1} + sqrt(1 - rho^2) eps_t
+    and two target chunks that each jump to a random live chunk with probability ``drift`` per
+    step (else stay).  rho = 0, drift = 1 gives independent steps."""
+    cfg = cache.cfg
+    if n_layers is None:
+        n_layers = cfg.n_layers - layer0
+    dev = cache.summary.device
+    B, Hkv, g, d = cfg.batch, cfg.n_kv_heads, cfg.q_per_kv, cfg.head_dim
+    nL = cfg.n_live
+    summ = cache.summary.float()
+    basis = cache.basis.float()
+    gsel = _gen("cpu", cfg.seed, _T_Q, seed_offset, 11)
+    targets = torch.randint(0, nL, (n_layers, B, Hkv, 2), generator=gsel)
+    z = torch.randn(n_layers, B, cfg.n_q_heads, d, generator=_gen(dev, cfg.seed, _T_Q, seed_offset, 12, 0), device=dev)
+    steps = []
+    for t in range(n_steps):
+        if t > 0:
+            eps = torch.randn(z.shape, generator=_gen(dev, cfg.seed, _T_Q, seed_offset, 12, t), device=dev)
+            z = rho * z + math.sqrt(max(0.0, 1.0 - rho * rho)) * eps
+            jump = torch.rand(targets.shape, generator=gsel) < drift
+            targets = torch.where(jump, torch.randint(0, nL, targets.shape, generator=gsel), targets)
+        out = torch.empty(n_layers, B, cfg.n_q_heads, d, dtype=torch.float32, device=dev)
+        for li in range(n_layers):
+            l = layer0 + li
+            grp = l // cfg.group
+            for b in range(B):
+                for h in range(Hkv):
+                    kbar = summ[b, grp, h, targets[li, b, h].to(dev)] @ basis[l, h]      # [2][d]
+                    bias = (kbar / kbar.norm(dim=-1, keepdim=True).clamp_min(1e-30)).sum(0)
+                    j0 = h * g
+                    out[li, b, j0:j0 + g] = z[li, b, j0:j0 + g] / math.sqrt(d) + QUERY_BETA * bias
+        steps.append(out.to(cfg.torch_dtype))
+    return steps
+
+
 def select_sequences(cache: SynthCache, seqs, device="cpu") -> SynthCache:
     """The cache of sequences ``seqs`` alone (in that order), on ``device``.
 
