@@ -403,6 +403,52 @@ lowram_status lowram_shard_partial(lowram_cache* shard, int32_t layer0, int32_t 
 lowram_status lowram_merge_partials(int32_t n_parts, int64_t n_rows, int32_t head_dim, const float* partials,
                                     int32_t out_dtype, void* out, lowram_stream stream);
 
+/* ---------------------------------------------------------- reuse of rebuilt chunks
+ *
+ * Consecutive decode steps select mostly the same chunks; each step can reuse what an earlier
+ * one rebuilt (rit.work "lowram-kv-cache-compression", section "Значения предсказывают, ключи
+ * раскладывают по общему базису").  A store keeps, per (sequence, layer, KV head, chunk), the
+ * chunk's rebuilt values vhat_t = W2 silu(W1 khat_t) + delta_t (bf16, C x d = 32 KB at C = d =
+ * 128); a hit attends over them, scoring the keys from the stored coefficients as usual, and
+ * skips the predictor.  Policy (this library's; the pages give none): `capacity` entries filled
+ * first-in first-out; per decode call at most `fill_cap` of its misses are admitted, in unit
+ * order ((layer, KV head, sequence), sequence fastest), each unit's in ascending chunk id; hits
+ * are decided against the store as it was before the call.  The results equal those of
+ * lowram_decode_attn up to floating-point rounding (the stored values are rounded to bf16).
+ * Costs: a miss as lowram_decode_attn; a hit reads the chunk's coefficients and its stored
+ * values (2 x 32 KB) and runs no predictor; a fill rebuilds the chunk's values once more
+ * (tensor cores) and writes them.  Shapes: bf16 native stores, head_dim 128, mlp_hidden 256,
+ * rank 64 or 128, chunk 128, 4 or 8 query heads per KV head, top_k <= 32. */
+typedef struct lowram_reuse lowram_reuse; /* opaque; owns its device memory */
+typedef struct {
+  uint64_t hits, misses, fills;  /* cumulative chunk counts over the store's decode calls */
+} lowram_reuse_counts;
+
+/* A store for `cache` with `capacity` entries (capacity * 32 KB at C = d = 128, plus a table of
+ * 4 bytes per chunk slot of the cache), admitting at most fill_cap <= capacity misses per call.
+ * Stream-ordered.  EINVAL for bad sizes, EUNSUPPORTED for shapes without a reuse path, ENOMEM.
+ * The store is tied to the cache as it is now: after a lowram_cache_repack the store's calls
+ * return EINVAL (make a new one).  Destroy the store before the cache. */
+lowram_status lowram_reuse_create(lowram_cache* cache, int32_t capacity, int32_t fill_cap, lowram_reuse** out,
+                                  lowram_stream stream);
+void lowram_reuse_destroy(lowram_reuse* store); /* synchronises the device first; NULL is a no-op */
+
+/* lowram_decode_attn for layers [layer0, layer0 + n_layers) through the store (q, out, sel as
+ * there), updating it.  Stream-ordered, no allocation, no host synchronisation.  A store must
+ * not be used by two streams at the same time, nor its cache by another call in between the
+ * kernels of this one. */
+lowram_status lowram_decode_attn_reuse(lowram_reuse* store, int32_t layer0, int32_t n_layers, const void* q,
+                                       void* out, int32_t* sel, lowram_stream stream);
+
+/* The cumulative hit / miss / fill counts (synchronises `stream`). */
+lowram_status lowram_reuse_counts_get(lowram_reuse* store, lowram_reuse_counts* out, lowram_stream stream);
+
+/* Read-only DEVICE view of the store (valid until lowram_reuse_destroy): table [B][L][Hkv]
+ * [table_stride] int32 (the entry holding chunk slot s of (b, l, KV head), or -1), owner
+ * [capacity] int64 (the table index an entry serves, or -1) and entries [capacity][C][d] bf16. */
+lowram_status lowram_reuse_view(const lowram_reuse* store, const int32_t** table, const int64_t** owner,
+                                const void** entries, int64_t* table_stride);
+
 /* ---------------------------------------------------------------- prefill-side encoder
  *
  * lowram_encode: dense keys and values -> the compressed arrays lowram_cache_create takes

@@ -26,7 +26,8 @@ __all__ = [
     "lowram_cache_set_stage_events", "lowram_cache_last_launches", "lowram_cache_last_path",
     "LowramCache", "config_struct", "lowram_decode_attn_static", "lowram_dense_decode_attn",
     "lowram_cache_view", "lowram_cache_append", "lowram_cache_repack",
-    "lowram_encode",
+    "lowram_encode", "LowramReuse", "lowram_reuse_create", "lowram_reuse_destroy",
+    "lowram_decode_attn_reuse", "lowram_reuse_counts_get", "lowram_reuse_view",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblowram.so")
@@ -67,6 +68,10 @@ class LowramBytesC(ctypes.Structure):
 _LIB = None
 
 
+class LowramReuseCountsC(ctypes.Structure):
+    _fields_ = [("hits", ctypes.c_uint64), ("misses", ctypes.c_uint64), ("fills", ctypes.c_uint64)]
+
+
 def lib() -> ctypes.CDLL:
     """The loaded library (raises if liblowram.so was not built)."""
     global _LIB
@@ -105,6 +110,12 @@ def lib() -> ctypes.CDLL:
         "lowram_shard_candidates": (I32, [P, I32, I32, P, I32, P, P, P]),
         "lowram_shard_partial": (I32, [P, I32, I32, I32, I32, P, P, P, P, P]),
         "lowram_merge_partials": (I32, [I32, I64, I32, P, I32, P, P]),
+        "lowram_reuse_create": (I32, [P, I32, I32, ctypes.POINTER(P), P]),
+        "lowram_reuse_destroy": (None, [P]),
+        "lowram_decode_attn_reuse": (I32, [P, I32, I32, P, P, P, P]),
+        "lowram_reuse_counts_get": (I32, [P, ctypes.POINTER(LowramReuseCountsC), P]),
+        "lowram_reuse_view": (I32, [P, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P),
+                                    ctypes.POINTER(I64)]),
         "lowram_debug_set_wait_limit": (I32, [P, I64]),
         "lowram_debug_fail_alloc": (None, [I32]),
         "lowram_status_string": (ctypes.c_char_p, [I32]),
@@ -317,6 +328,87 @@ def lowram_merge_partials(partials, out, stream=None) -> None:
     dt = 0 if out.dtype == torch.float32 else 1
     _check(lib().lowram_merge_partials(n_parts, n_rows, w - 2, _ptr(partials), dt, _ptr(out), _stream(stream)),
            "lowram_merge_partials")
+
+
+def lowram_reuse_create(handle: int, capacity: int, fill_cap: int, stream=None) -> int:
+    """A store of rebuilt chunk values for cache ``handle`` (see lowram.h); returns its handle."""
+    out = ctypes.c_void_p()
+    _check(lib().lowram_reuse_create(handle, int(capacity), int(fill_cap), ctypes.byref(out), _stream(stream)),
+           "lowram_reuse_create")
+    return int(out.value)
+
+
+def lowram_reuse_destroy(store: int) -> None:
+    lib().lowram_reuse_destroy(store)
+
+
+def lowram_decode_attn_reuse(store: int, layer0: int, n_layers: int, q, out, sel=None, stream=None) -> None:
+    """lowram_decode_attn through a reuse store (CUDA tensors as there)."""
+    _check(lib().lowram_decode_attn_reuse(store, layer0, n_layers, _ptr(q), _ptr(out), _ptr(sel), _stream(stream)),
+           "lowram_decode_attn_reuse")
+
+
+def lowram_reuse_counts_get(store: int, stream=None) -> dict:
+    c = LowramReuseCountsC()
+    _check(lib().lowram_reuse_counts_get(store, ctypes.byref(c), _stream(stream)), "lowram_reuse_counts_get")
+    return {"hits": int(c.hits), "misses": int(c.misses), "fills": int(c.fills)}
+
+
+def lowram_reuse_view(store: int, cfg, capacity: int) -> dict:
+    """Zero-copy torch views of the store's table, owner and entries (device memory it owns)."""
+    import torch
+    table, owner, entries = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_void_p()
+    stride = ctypes.c_int64()
+    _check(lib().lowram_reuse_view(store, ctypes.byref(table), ctypes.byref(owner), ctypes.byref(entries),
+                                   ctypes.byref(stride)), "lowram_reuse_view")
+    B, L, H = _get(cfg, "batch"), _get(cfg, "n_layers"), _get(cfg, "n_kv_heads")
+    C, d = _get(cfg, "chunk"), _get(cfg, "head_dim")
+
+    def wrap(ptr, shape, typestr):
+        return torch.as_tensor(_DeviceArray(ptr.value, shape, typestr), device="cuda")
+
+    return {"table": wrap(table, (B, L, H, int(stride.value)), "<i4"),
+            "owner": wrap(owner, (int(capacity),), "<i8"),
+            "entries": wrap(entries, (int(capacity), C, d), "<i2").view(torch.bfloat16)}
+
+
+class LowramReuse:
+    """Owning wrapper of a reuse store (destroy it before its cache)."""
+
+    def __init__(self, cache: "LowramCache", capacity: int, fill_cap: int, stream=None):
+        self.cache, self.capacity = cache, int(capacity)
+        self.handle = lowram_reuse_create(cache.handle, capacity, fill_cap, stream)
+
+    def decode(self, q, out=None, sel: bool = False, layer0: int = 0, n_layers: Optional[int] = None, stream=None):
+        import torch
+        if n_layers is None:
+            n_layers = int(q.shape[0])
+        if out is None:
+            out = torch.empty_like(q)
+        s = None
+        if sel:
+            c = self.cache.cfg
+            s = torch.empty(n_layers, _get(c, "batch"), _get(c, "n_kv_heads"), _get(c, "top_k"),
+                            dtype=torch.int32, device=q.device)
+        lowram_decode_attn_reuse(self.handle, layer0, n_layers, q, out, s, stream)
+        return (out, s) if sel else out
+
+    def counts(self, stream=None) -> dict:
+        return lowram_reuse_counts_get(self.handle, stream)
+
+    def view(self) -> dict:
+        return lowram_reuse_view(self.handle, self.cache.cfg, self.capacity)
+
+    def close(self) -> None:
+        if getattr(self, "handle", 0):
+            lowram_reuse_destroy(self.handle)
+            self.handle = 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def lowram_debug_set_wait_limit(handle: int, cycles: int) -> None:

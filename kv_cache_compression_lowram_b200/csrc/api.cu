@@ -9,6 +9,7 @@
 
 #include "lowram_internal.cuh"
 #include "upkeep.cuh"
+#include "reuse.cuh"
 
 using namespace lowram;
 
@@ -45,6 +46,16 @@ struct lowram_cache {
   // context-sharded decode: tile list of phase 2, and the layer range phase 1 prepared
   int32_t *t_unit, *t_slot, *t_ptr, *t_total, *t_cnt;
   int shard_l0, shard_n;
+  uint64_t generation;         // advanced by every re-pack (a reuse store is tied to one)
+};
+
+// A store of rebuilt chunk values tied to one cache (reuse.cu has the kernels).
+struct lowram_reuse {
+  lowram_cache* cache;
+  uint64_t generation;
+  ReuseDev d;
+  void* mem[12];
+  int n_mem;
 };
 
 namespace {
@@ -744,6 +755,7 @@ lowram_status lowram_cache_repack(lowram_cache* c, int32_t n_resid, lowram_strea
   c->cfg.n_live += 1;
   c->nC += 1;
   c->nL += 1;
+  c->generation += 1;
   c->last_repack_in_place = in_place;
   if (c->host_exec) {   // its kernels' geometry and pointers are those of the shorter cache
     cudaGraphExecDestroy(c->host_exec);
@@ -994,6 +1006,131 @@ lowram_status lowram_merge_partials(int32_t n_parts, int64_t n_rows, int32_t hea
   cudaError_t e = launch_merge_partials(n_parts, n_rows, head_dim, partials, out_dtype, out,
                                         reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "merge kernel");
+  return LOWRAM_OK;
+}
+
+// ------------------------------------------------------------- reuse of rebuilt chunks
+
+void lowram_reuse_destroy(lowram_reuse* r) {
+  if (!r) return;
+  cudaDeviceSynchronize();
+  for (int i = 0; i < r->n_mem; ++i) cudaFree(r->mem[i]);
+  delete r;
+}
+
+lowram_status lowram_reuse_create(lowram_cache* c, int32_t capacity, int32_t fill_cap, lowram_reuse** out,
+                                  lowram_stream stream) {
+  if (!c || !out) return inval("NULL cache or output");
+  *out = nullptr;
+  if (capacity < 1 || fill_cap < 0 || fill_cap > capacity) return inval("need capacity >= 1 and 0 <= fill_cap <= capacity");
+  Geom g = make_geom(c, 0, c->cfg.n_layers, true);
+  if (!reuse_supported(g, c->cfg.dtype, c->cfg.store) || c->cfg.top_k > 32) {
+    g_last_error = "the reuse store takes bf16 native stores, head_dim 128, mlp_hidden 256, rank 64 or 128, "
+                   "chunk 128, 4 or 8 query heads per KV head and top_k <= 32";
+    return LOWRAM_EUNSUPPORTED;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  lowram_reuse* r = new lowram_reuse();
+  std::memset(r, 0, sizeof(*r));
+  r->cache = c;
+  r->generation = c->generation;
+  const size_t B = c->cfg.batch, L = c->cfg.n_layers, H = c->cfg.n_kv_heads, d = c->cfg.head_dim;
+  const size_t C = c->cfg.chunk, h = c->cfg.mlp_hidden, k = c->cfg.top_k, Umax = B * L * H;
+  const size_t table_n = Umax * (size_t)c->nLs;
+  const size_t tail_stride = (size_t)g.tail_stride;
+  struct Piece { void** p; size_t bytes; };
+  Piece pieces[] = {
+      {reinterpret_cast<void**>(&r->d.entries), (size_t)capacity * C * d * 2},
+      {reinterpret_cast<void**>(&r->d.table), table_n * 4},
+      {reinterpret_cast<void**>(&r->d.owner), (size_t)capacity * 8},
+      {reinterpret_cast<void**>(&r->d.ring), 16},
+      {reinterpret_cast<void**>(&r->d.counters), 32},
+      {reinterpret_cast<void**>(&r->d.hit_entry), Umax * k * 4},
+      {reinterpret_cast<void**>(&r->d.hit_slot), Umax * k * 4},
+      {reinterpret_cast<void**>(&r->d.hit_n), Umax * 4},
+      {reinterpret_cast<void**>(&r->d.hit_part), Umax * tail_stride * 4},
+      {const_cast<void**>(reinterpret_cast<const void**>(&r->d.w2h)), L * H * d * h * 2},
+  };
+  for (Piece& pc : pieces) {
+    cudaError_t e = device_malloc(pc.p, pc.bytes ? pc.bytes : 16);
+    if (e != cudaSuccess) {
+      lowram_reuse_destroy(r);
+      g_last_error = std::string("cudaMalloc: ") + cudaGetErrorString(e);
+      return LOWRAM_ENOMEM;
+    }
+    r->mem[r->n_mem++] = *pc.p;
+  }
+  r->d.E = capacity;
+  r->d.fill_cap = fill_cap;
+  r->d.table_stride = c->nLs;
+  cudaError_t e = cudaMemsetAsync(r->d.table, 0xff, table_n * 4, s);   // -1: no entry
+  if (e == cudaSuccess) e = cudaMemsetAsync(r->d.owner, 0xff, (size_t)capacity * 8, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(r->d.ring, 0, 16, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(r->d.counters, 0, 32, s);
+  if (e == cudaSuccess) e = launch_to_half(static_cast<const __nv_bfloat16*>(c->cb.w2), const_cast<__half*>(r->d.w2h),
+                                           L * H * d * h, s);
+  if (e != cudaSuccess) {
+    lowram_reuse_destroy(r);
+    return cuda_fail(e, "initialise the reuse store");
+  }
+  *out = r;
+  return LOWRAM_OK;
+}
+
+lowram_status lowram_decode_attn_reuse(lowram_reuse* r, int32_t layer0, int32_t n_layers, const void* q, void* out,
+                                       int32_t* sel, lowram_stream stream) {
+  if (!r) return inval("NULL store");
+  lowram_cache* c = r->cache;
+  lowram_status st = check_layers(c, layer0, n_layers);
+  if (st != LOWRAM_OK) return st;
+  if (!q || !out) return inval("NULL q or out");
+  if (r->generation != c->generation) return inval("the cache was re-packed after the store was made: make a new one");
+  Geom g = make_geom(c, layer0, n_layers, true);
+  if (!attend_tc_supported(g, c->cfg.dtype, c->cfg.store) || !reuse_supported(g, c->cfg.dtype, c->cfg.store)) {
+    g_last_error = "these shapes have no reuse path";
+    return LOWRAM_EUNSUPPORTED;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  c->shard_l0 = -1;
+  cudaError_t e = launch_select(g, c->cb, c->sc, c->cfg.dtype, q, nullptr, sel, 1, true, s);
+  if (e != cudaSuccess) return cuda_fail(e, "select kernel");
+  Scratch sc = c->sc;
+  sc.tile_unit = c->t_unit;
+  sc.tile_slot = c->t_slot;
+  sc.tile_ptr = c->t_ptr;
+  sc.tile_total = c->t_total;
+  sc.unit_ntile = c->t_cnt;
+  if ((e = launch_reuse(g, c->cb, sc, r->d, c->w1f_tc, c->n_sm, s, 0)) != cudaSuccess) return cuda_fail(e, "reuse plan");
+  if ((e = launch_attend_tc(g, c->cb, sc, c->cfg.store, c->w1f_tc, c->n_sm, s)) != cudaSuccess)
+    return cuda_fail(e, "chunk attention kernel");
+  if ((e = launch_reuse(g, c->cb, sc, r->d, c->w1f_tc, c->n_sm, s, 1)) != cudaSuccess) return cuda_fail(e, "reuse hits");
+  if ((e = launch_combine_list(g, c->cb, sc, r->d.hit_part, out, s)) != cudaSuccess) return cuda_fail(e, "combine kernel");
+  if ((e = launch_reuse(g, c->cb, sc, r->d, c->w1f_tc, c->n_sm, s, 2)) != cudaSuccess) return cuda_fail(e, "reuse fills");
+  c->last_launches = 8;
+  c->last_path = LOWRAM_PATH_TC;
+  return LOWRAM_OK;
+}
+
+lowram_status lowram_reuse_counts_get(lowram_reuse* r, lowram_reuse_counts* out, lowram_stream stream) {
+  if (!r || !out) return inval("NULL store or output");
+  unsigned long long v[3];
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(v, r->d.counters, sizeof v, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "read the reuse counters");
+  out->hits = v[0];
+  out->misses = v[1];
+  out->fills = v[2];
+  return LOWRAM_OK;
+}
+
+lowram_status lowram_reuse_view(const lowram_reuse* r, const int32_t** table, const int64_t** owner,
+                                const void** entries, int64_t* table_stride) {
+  if (!r || !table || !owner || !entries || !table_stride) return inval("NULL store or output");
+  *table = r->d.table;
+  *owner = reinterpret_cast<const int64_t*>(r->d.owner);
+  *entries = r->d.entries;
+  *table_stride = r->d.table_stride;
   return LOWRAM_OK;
 }
 

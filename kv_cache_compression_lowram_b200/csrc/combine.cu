@@ -8,6 +8,7 @@
 // Also: the create-time fold W1' = W1 B_l^T and the device-side table check.
 #include "lowram_internal.cuh"
 #include "warp_mma.cuh"
+#include "reuse.cuh"
 
 namespace lowram {
 namespace {
@@ -132,7 +133,7 @@ combine_kernel(Geom g, CacheBuffers cb, Scratch sc, T* __restrict__ out) {
 constexpr int kCombPieces = 8;
 constexpr int kCombThreads = 256;
 
-template <int GQ>
+template <int GQ, bool LIST = false>
 struct CombSmem {
   static constexpr int UB = 16 / GQ;          // units per CTA
   static constexpr int NR = UB * GQ;          // (unit, head) rows: 16
@@ -140,8 +141,9 @@ struct CombSmem {
   static constexpr size_t W2 = 0;                                   // bf16 [128][WROW]
   static constexpr size_t BM = W2 + 128 * WROW * 2;                 // bf16 [2 NR][WROW]: hi, lo rows
   static constexpr size_t ACCD = BM + 2 * NR * WROW * 2;            // float [NR][128]
-  static constexpr size_t WT = ACCD + NR * 128 * 4;                 // float [NR][kCombPieces + 1]
-  static constexpr size_t LS = WT + NR * (kCombPieces + 1) * 4;     // float [NR]
+  static constexpr int MAXP = LIST ? 33 : kCombPieces;             // pieces per unit
+  static constexpr size_t WT = ACCD + NR * 128 * 4;                 // float [NR][MAXP + 2]
+  static constexpr size_t LS = WT + NR * (MAXP + 2) * 4;            // float [NR]
   static constexpr size_t PC = LS + NR * 4;                         // int [UB][2]: first piece, pieces
   static constexpr size_t BYTES = PC + UB * 2 * 4;
 };
@@ -152,17 +154,21 @@ __device__ __forceinline__ void cp_async16c(void* smem_dst, const void* gsrc) {
                : "memory");
 }
 
-template <int GQ>
+// LIST: the pieces come from an explicit tile list (sc.tile_ptr / sc.tile_total; units may
+// have any number of tiles, none included) and every unit has one extra record in the tail's
+// format (extra_rec, [U][tail_stride]), merged like the tail.
+template <int GQ, bool LIST>
 __global__ void __launch_bounds__(kCombThreads, 2)
-combine_mma_kernel(Geom g, CacheBuffers cb, Scratch sc, __nv_bfloat16* __restrict__ out) {
+combine_mma_kernel(Geom g, CacheBuffers cb, Scratch sc, const float* __restrict__ extra_rec,
+                   __nv_bfloat16* __restrict__ out) {
   constexpr int D = 128, H = 256;
-  using SM = CombSmem<GQ>;
-  constexpr int UB = SM::UB, NR = SM::NR, WROW = SM::WROW;
+  using SM = CombSmem<GQ, LIST>;
+  constexpr int UB = SM::UB, NR = SM::NR, WROW = SM::WROW, MAXP = SM::MAXP;
   extern __shared__ __align__(128) unsigned char smem[];
   __nv_bfloat16* w2s = reinterpret_cast<__nv_bfloat16*>(smem + SM::W2);
   __nv_bfloat16* bms = reinterpret_cast<__nv_bfloat16*>(smem + SM::BM);
   float (*accd)[D] = reinterpret_cast<float (*)[D]>(smem + SM::ACCD);
-  float (*wt)[kCombPieces + 1] = reinterpret_cast<float (*)[kCombPieces + 1]>(smem + SM::WT);
+  float (*wt)[MAXP + 2] = reinterpret_cast<float (*)[MAXP + 2]>(smem + SM::WT);
   float* ls = reinterpret_cast<float*>(smem + SM::LS);
   int (*pc)[2] = reinterpret_cast<int (*)[2]>(smem + SM::PC);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -185,22 +191,33 @@ combine_mma_kernel(Geom g, CacheBuffers cb, Scratch sc, __nv_bfloat16* __restric
   // its partial records are read only after this
   asm volatile("griddepcontrol.wait;" ::: "memory");
   // merge weights of every (unit, head) row: w_r = 2^(m_r - M) over the unit's pieces and tail
-  const long long total = (long long)g.U * g.k;
+  const long long total = LIST ? (long long)*sc.tile_total : (long long)g.U * g.k;
   if (tid < NR) {
     const int r = tid, bi = r / GQ, j = r % GQ;
     float L = 0.f;
     if (bi < nb) {
       const int u = u0 + bi;
-      const int c0 = cta_of_tile(total, g.P, (long long)u * g.k);
-      const int nrec = cta_of_tile(total, g.P, (long long)(u + 1) * g.k - 1) - c0 + 1;
+      int c0 = 0, nrec = 0;
+      if (LIST) {
+        const int p0 = sc.tile_ptr[u], p1 = sc.tile_ptr[u + 1];
+        if (p1 > p0) {
+          c0 = cta_of_tile(total, g.P, p0);
+          nrec = cta_of_tile(total, g.P, p1 - 1) - c0 + 1;
+        }
+      } else {
+        c0 = cta_of_tile(total, g.P, (long long)u * g.k);
+        nrec = cta_of_tile(total, g.P, (long long)(u + 1) * g.k - 1) - c0 + 1;
+      }
       if (j == 0) {
         pc[bi][0] = c0;
         pc[bi][1] = nrec;
-        if (nrec > g.max_rec || nrec > kCombPieces) atomicOr(sc.err, ERR_SELECT);   // cannot happen
+        if (nrec > MAXP || (!LIST && nrec > g.max_rec)) atomicOr(sc.err, ERR_SELECT);   // cannot happen
       }
-      const int np = min(nrec, kCombPieces);
+      const int np = min(nrec, MAXP);
       const float* trec = sc.tail_part + (size_t)u * g.tail_stride;
+      const float* xrec = LIST ? extra_rec + (size_t)u * g.tail_stride : trec;
       float M = trec[j];
+      if (LIST) M = fmaxf(M, xrec[j]);
       for (int p = 0; p < np; ++p) M = fmaxf(M, sc.part[(size_t)(u + c0 + p) * g.rec_stride + j]);
       for (int p = 0; p < np; ++p) {
         const float* rec = sc.part + (size_t)(u + c0 + p) * g.rec_stride;
@@ -209,8 +226,13 @@ combine_mma_kernel(Geom g, CacheBuffers cb, Scratch sc, __nv_bfloat16* __restric
         L = fmaf(w, rec[GQ + j], L);
       }
       const float w_t = trec[j] == -INFINITY ? 0.f : exp2f(trec[j] - M);
-      wt[r][kCombPieces] = w_t;
+      wt[r][MAXP] = w_t;
       L = fmaf(w_t, trec[GQ + j], L);
+      if (LIST) {
+        const float w_x = xrec[j] == -INFINITY ? 0.f : exp2f(xrec[j] - M);
+        wt[r][MAXP + 1] = w_x;
+        L = fmaf(w_x, xrec[GQ + j], L);
+      }
     }
     ls[r] = L;
   }
@@ -226,7 +248,7 @@ combine_mma_kernel(Geom g, CacheBuffers cb, Scratch sc, __nv_bfloat16* __restric
     for (int x = 0; x < 8; ++x) ds[x] = 0.f;
     if (bi < nb) {
       const int u = u0 + bi;
-      const int c0 = pc[bi][0], np = min(pc[bi][1], kCombPieces);
+      const int c0 = pc[bi][0], np = min(pc[bi][1], MAXP);
       for (int p = 0; p < np; ++p) {
         const float* rec = sc.part + (size_t)(u + c0 + p) * g.rec_stride;
         const float w = wt[r][p];
@@ -249,15 +271,19 @@ combine_mma_kernel(Geom g, CacheBuffers cb, Scratch sc, __nv_bfloat16* __restric
           ds[4 * x + 3] = fmaf(w, v.w, ds[4 * x + 3]);
         }
       }
-      const float w_t = wt[r][kCombPieces];
-      const float4* tv = reinterpret_cast<const float4*>(sc.tail_part + (size_t)u * g.tail_stride + 2 * GQ + j * D + s * 8);
 #pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        const float4 v = tv[x];
-        ds[4 * x] = fmaf(w_t, v.x, ds[4 * x]);
-        ds[4 * x + 1] = fmaf(w_t, v.y, ds[4 * x + 1]);
-        ds[4 * x + 2] = fmaf(w_t, v.z, ds[4 * x + 2]);
-        ds[4 * x + 3] = fmaf(w_t, v.w, ds[4 * x + 3]);
+      for (int xr = 0; xr < (LIST ? 2 : 1); ++xr) {   // the tail, then the extra record
+        const float w_t = wt[r][MAXP + xr];
+        const float* base = xr ? extra_rec : sc.tail_part;
+        const float4* tv = reinterpret_cast<const float4*>(base + (size_t)u * g.tail_stride + 2 * GQ + j * D + s * 8);
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          const float4 v = tv[x];
+          ds[4 * x] = fmaf(w_t, v.x, ds[4 * x]);
+          ds[4 * x + 1] = fmaf(w_t, v.y, ds[4 * x + 1]);
+          ds[4 * x + 2] = fmaf(w_t, v.z, ds[4 * x + 2]);
+          ds[4 * x + 3] = fmaf(w_t, v.w, ds[4 * x + 3]);
+        }
       }
     }
     __nv_bfloat16 hi[16], lo[16];
@@ -418,7 +444,7 @@ cudaError_t launch_combine(const Geom& g, const CacheBuffers& cb, const Scratch&
     if (e != cudaSuccess) return e;
     k<<<g.U, kThreads, smem, s>>>(g, cb, sc, static_cast<float*>(out));
   } else if (g.d == 128 && g.h == 256 && (g.g == 4 || g.g == 8) && g.max_rec <= kCombPieces) {
-    auto k = g.g == 4 ? combine_mma_kernel<4> : combine_mma_kernel<8>;
+    auto k = g.g == 4 ? combine_mma_kernel<4, false> : combine_mma_kernel<8, false>;
     const size_t sm = g.g == 4 ? CombSmem<4>::BYTES : CombSmem<8>::BYTES;
     const int ub = 16 / g.g;
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
@@ -433,7 +459,7 @@ cudaError_t launch_combine(const Geom& g, const CacheBuffers& cb, const Scratch&
     at[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = at;
     lc.numAttrs = 1;
-    e = cudaLaunchKernelEx(&lc, k, g, cb, sc, static_cast<__nv_bfloat16*>(out));
+    e = cudaLaunchKernelEx(&lc, k, g, cb, sc, static_cast<const float*>(nullptr), static_cast<__nv_bfloat16*>(out));
     if (e != cudaSuccess) return e;
   } else {
     auto k = combine_kernel<__nv_bfloat16>;
@@ -441,6 +467,19 @@ cudaError_t launch_combine(const Geom& g, const CacheBuffers& cb, const Scratch&
     if (e != cudaSuccess) return e;
     k<<<g.U, kThreads, smem, s>>>(g, cb, sc, static_cast<__nv_bfloat16*>(out));
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_list(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const float* extra_rec,
+                                void* out, cudaStream_t s) {
+  if (g.d != 128 || g.h != 256 || !(g.g == 4 || g.g == 8) || g.k > 32) return cudaErrorNotSupported;
+  auto k = g.g == 4 ? combine_mma_kernel<4, true> : combine_mma_kernel<8, true>;
+  const size_t sm = g.g == 4 ? CombSmem<4, true>::BYTES : CombSmem<8, true>::BYTES;
+  const int ub = 16 / g.g;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)(g.n_layers * g.Hkv) * (unsigned)((g.B + ub - 1) / ub);
+  k<<<grid, kCombThreads, sm, s>>>(g, cb, sc, extra_rec, static_cast<__nv_bfloat16*>(out));
   return cudaGetLastError();
 }
 

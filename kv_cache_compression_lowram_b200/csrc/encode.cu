@@ -1015,6 +1015,11 @@ cudaError_t launch_encode_t(const Geom& g, int n_res, const void* keys, const vo
 
 }  // namespace
 
+cudaError_t launch_to_half(const __nv_bfloat16* src, __half* dst, size_t n, cudaStream_t s) {
+  to_half_kernel<<<1184, 256, 0, s>>>(src, dst, n);
+  return cudaGetLastError();
+}
+
 size_t encode_workspace_bytes(const Geom& g, bool folds_given) {
   size_t bytes = 0;
   carve(g, nullptr, &bytes, folds_given);

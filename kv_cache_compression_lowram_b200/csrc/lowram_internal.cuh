@@ -62,8 +62,12 @@ __host__ __device__ inline Unit unit_of(const Geom& g, int u) {
 
 // Tiles (unit, i-th selected chunk) are split over P CTAs in contiguous ranges;
 // CTA c owns tiles [tile_begin(c), tile_begin(c+1)).  The partial record of the piece
-// (unit u, CTA c) is record u + c.
+// (unit u, CTA c) is record u + c.  With fewer tiles than CTAs (an explicit tile list is
+// counted on the device, after the grid is sized) CTA c takes tile c alone and the empty
+// CTAs are the last ones, so the CTAs holding one unit's tiles are consecutive and every one
+// of them writes that unit's record.
 __host__ __device__ inline long long tile_begin(long long total, int P, int c) {
+  if (total < P) return c < total ? c : total;
   return (total * (long long)c) / P;
 }
 // Every CTA owns at least floor(total/P) >= 1 tiles, so the k tiles of one unit touch at
@@ -75,6 +79,7 @@ __host__ __device__ inline int max_records_per_unit(long long total, int P, int 
 }
 // The CTA whose range holds tile x.
 __host__ __device__ inline int cta_of_tile(long long total, int P, long long x) {
+  if (total < P) return (int)x;
   // largest c with floor(c*total/P) <= x  <=>  c = ceil((x+1)*P/total) - 1
   long long num = (x + 1) * (long long)P;
   return (int)((num + total - 1) / total) - 1;

@@ -17,6 +17,7 @@
 #include <climits>
 
 #include "lowram_internal.cuh"
+#include "reuse.cuh"
 
 namespace lowram {
 namespace {
@@ -294,6 +295,11 @@ cudaError_t launch_shard_select(const Geom& g, const CacheBuffers& cb, const Scr
     return cudaErrorInvalidValue;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  shard_scan_kernel<<<1, kScanThreads, 0, s>>>(g.U, g.k, sc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_scan(const Geom& g, const Scratch& sc, cudaStream_t s) {
   shard_scan_kernel<<<1, kScanThreads, 0, s>>>(g.U, g.k, sc);
   return cudaGetLastError();
 }

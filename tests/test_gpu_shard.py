@@ -80,6 +80,34 @@ def test_two_shards_of_the_32k_workload_sampled():
     check(cfg, O.OracleCache(S.cache_to_numpy(cache)), q, out, sel, units=sample_units(cfg, cfg.n_layers, 64, seed=7))
 
 
+def test_shards_reused_across_steps():
+    """The same shard decoders over consecutive steps with different queries: every step must
+    match the unsharded decode (a shard's tile list is shorter than the grid here, so this
+    also checks that no stale piece record of an earlier step is merged)."""
+    cfg = S.MISTRAL_GROUP.replace(name="shard_steps", batch=2)
+    cache = S.make_cache(cfg, device=DEV, tail_len=[64, 9])
+    bounds = [0, 16, 32, 48, 64]
+    decs = []
+    for s, (lo, hi) in enumerate(zip(bounds[:-1], bounds[1:])):
+        sh = S.shard_chunks(cache, lo, hi, keep_tail=(s == len(bounds) - 2))
+        decs.append(ShardDecoder(K.LowramCache.from_synth(sh), lo, len(bounds) - 1))
+    lc = K.LowramCache.from_synth(cache)
+    for t, q in enumerate(S.make_query_steps(cache, 3, 0.0, 1.0)):
+        cands = [d.candidates(q) for d in decs]
+        cs_all = torch.stack([c[0] for c in cands])
+        ci_all = torch.stack([c[1] for c in cands])
+        parts = [d.partial(cs_all, ci_all) for d in decs]
+        out = decs[0].merge(torch.stack([p[0] for p in parts]))
+        ref, ref_sel = lc.decode(q, sel=True)
+        torch.cuda.synchronize()
+        assert torch.equal(parts[0][1], ref_sel), t
+        err = ((out.float() - ref.float()).norm(dim=-1) / ref.float().norm(dim=-1)).max().item()
+        assert err <= 1e-2, (t, err)
+    for d in decs:
+        d.cache.close()
+    lc.close()
+
+
 def test_phase_two_requires_phase_one():
     cfg = S.MISTRAL_GROUP
     cache = S.make_cache(cfg).to(DEV)
