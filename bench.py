@@ -59,6 +59,11 @@ def parse():
     ap.add_argument("--shards", type=int, default=0,
                     help="context-sharded decode of the workload over this many chunk shards: one shard "
                          "per rank under torchrun (NCCL gathers), else every shard on this one GPU")
+    ap.add_argument("--reuse", action="store_true",
+                    help="decode steps whose selections persist, through a store of rebuilt chunks, at "
+                         "several drift rates (one JSON line each) next to the plain decode of the same steps")
+    ap.add_argument("--reuse-drift", type=float, action="append", default=None,
+                    help="with --reuse: this drift rate only (repeatable)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
 
@@ -864,6 +869,85 @@ def run_shards(args, ws, rank, local):
     }
 
 
+REUSE_METRIC = "decode-attn queries/s over compressed KV at 32K ctx, consecutive steps through a reuse store"
+REUSE_DRIFTS = (0.0, 0.02, 0.1, 1.0)
+
+
+def run_reuse(args, ws, rank, local):
+    """Consecutive decode steps of the workload (``make_query_steps``: AR(1) query noise, rho =
+    0.9, and per unit two target chunks that jump with probability ``drift`` per step) through
+    a reuse store (capacity 2 U k entries, fill cap U k), at several drift rates, one JSON
+    line each.  Each line also times the plain decode of the same steps; both eager calls
+    timed with CUDA events (the queries change every step), inputs resident in HBM.  The
+    store is warmed by the warm-up steps of the same sequence.  Per replica, no collective."""
+    import kv_cache_compression_lowram_b200 as K
+    cfg = replica_config(S.CONFIGS[args.config], rank)
+    dev = torch.device("cuda", local)
+    cache = S.make_cache(cfg, device=dev)
+    lc = K.LowramCache.from_synth(cache)
+    U = cfg.n_layers * cfg.batch * cfg.n_kv_heads
+    cap, fill_cap = 2 * U * cfg.top_k, U * cfg.top_k
+    stream = torch.cuda.current_stream()
+    out = torch.empty(cfg.n_layers, cfg.batch, cfg.n_q_heads, cfg.head_dim, dtype=cfg.torch_dtype, device=dev)
+    sel = torch.empty(cfg.n_layers, cfg.batch, cfg.n_kv_heads, cfg.top_k, dtype=torch.int32, device=dev)
+    lines = []
+    for di, drift in enumerate(REUSE_DRIFTS):
+        if args.reuse_drift and drift not in args.reuse_drift:
+            continue
+        steps = S.make_query_steps(cache, args.warmup + args.steps, 0.9, drift, seed_offset=100 + di)
+        store = K.LowramReuse(lc, cap, fill_cap)
+        for q in steps[:args.warmup]:
+            K.lowram_decode_attn_reuse(store.handle, 0, cfg.n_layers, q, out, sel)
+        torch.cuda.synchronize()
+        c0 = store.counts()
+        clocks = ClockSampler(local)
+        barrier(ws)
+        torch.cuda.synchronize()
+        clocks.start()
+        time.sleep(0.3)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for q in steps[args.warmup:]:
+            K.lowram_decode_attn_reuse(store.handle, 0, cfg.n_layers, q, out, sel)
+        b.record(stream)
+        torch.cuda.synchronize()
+        reuse_ms = a.elapsed_time(b)
+        launches = lc.last_launches
+        c1 = store.counts()
+        # the plain decode of the same steps
+        for q in steps[:args.warmup]:
+            K.lowram_decode_attn(lc.handle, 0, cfg.n_layers, q, out, sel)
+        barrier(ws)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for q in steps[args.warmup:]:
+            K.lowram_decode_attn(lc.handle, 0, cfg.n_layers, q, out, sel)
+        b.record(stream)
+        torch.cuda.synchronize()
+        plain_ms = a.elapsed_time(b)
+        clk = clocks.stop()
+        store.close()
+        del steps
+        queries = cfg.batch * cfg.n_layers * args.steps
+        value, ms_total = aggregate_rate(queries, reuse_ms, ws)
+        pvalue, pms_total = aggregate_rate(queries, plain_ms, ws)
+        hits, misses, fills = (c1[x] - c0[x] for x in ("hits", "misses", "fills"))
+        lines.append({
+            "metric": REUSE_METRIC, "value": round(value, 1), "unit": "queries/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_total / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": cfg.dtype,
+            "data": "synthetic (seeded temporal query recipe)", "impl": "lowram_reuse",
+            "config": {"workload": cfg.name, "rho": 0.9, "drift": drift, "capacity": cap, "fill_cap": fill_cap,
+                       "store_bytes": cap * cfg.chunk * cfg.head_dim * 2, "parallelism": f"replicas x{ws}"},
+            "hit_rate": round(hits / max(1, hits + misses), 4), "fills_per_step": round(fills / args.steps, 1),
+            "plain": {"value": round(pvalue, 1), "ms_per_step": round(pms_total / args.steps, 4)},
+            "speedup_vs_plain": round(pms_total / ms_total, 4),
+            "gpu_launches": launches * args.steps, "clocks": clk,
+        })
+    lc.close()
+    return lines
+
+
 def main():
     args = parse()
     ws, rank, local = dist_init()
@@ -877,11 +961,17 @@ def main():
         line = run_repack(args, ws, rank, local)
     elif args.shards:
         line = run_shards(args, ws, rank, local)
+    elif args.reuse:
+        for ln in run_reuse(args, ws, rank, local):
+            if rank == 0:
+                print(json.dumps(ln), flush=True)
+        line = None
     else:
         line = run_lowram(args, ws, rank, local)
     if rank == 0 and line is not None:
         print(json.dumps(line), flush=True)
-    if args.sweep and args.impl == "lowram" and not (args.dense or args.encode or args.repack or args.shards):
+    if args.sweep and args.impl == "lowram" and not (args.dense or args.encode or args.repack or args.shards
+                                                      or args.reuse):
         import gc
         for b in (1, 4, 16, 32, 64):
             args.config = f"llama8b_32k_bf16_b{b}"

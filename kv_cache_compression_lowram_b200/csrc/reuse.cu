@@ -61,6 +61,7 @@ reuse_plan_kernel(Geom g, Scratch sc, ReuseDev st) {
     n_miss += __popc(bm);
   }
   if (lane == 0) {
+    if (u == 0) st.ring[1] = st.ring[0];   // the commit kernel's view of the ring position
     st.hit_n[u] = n_hit;
     sc.unit_ntile[u] = n_miss;
     atomicAdd(st.counters + 0, (unsigned long long)n_hit);
@@ -232,10 +233,14 @@ reuse_hit_kernel(Geom g, CacheBuffers cb, Scratch sc, ReuseDev st) {
       l_run[j] = l_run[j] * alpha[j] + (red[1][0][j] + red[1][1][j]) + (red[1][2][j] + red[1][3][j]);
       m_run[j] = mn;
     }
+    float a0 = 0.f, a1 = 0.f;   // the factors of accumulator rows gq and gq + 8 (selected
+#pragma unroll                 // without a dynamic index, which would put alpha in memory)
+    for (int j = 0; j < GQ; ++j) {
+      if (gq < 2 * GQ && gq % GQ == j) a0 = alpha[j];
+      if (gq + 8 < 2 * GQ && (gq + 8) % GQ == j) a1 = alpha[j];
+    }
 #pragma unroll
     for (int nt = 0; nt < 4; ++nt) {
-      const float a0 = gq < 2 * GQ ? alpha[gq % GQ] : 0.f;
-      const float a1 = gq + 8 < 2 * GQ ? alpha[(gq + 8) % GQ] : 0.f;
       acc[nt][0] *= a0;
       acc[nt][1] *= a0;
       acc[nt][2] *= a1;
@@ -273,10 +278,12 @@ reuse_hit_kernel(Geom g, CacheBuffers cb, Scratch sc, ReuseDev st) {
       }
     }
   }
-  if (tid < GQ) {
-    rec[tid] = m_run[tid];
-    rec[GQ + tid] = l_run[tid];
-  }
+#pragma unroll
+  for (int j = 0; j < GQ; ++j)
+    if (tid == j) {
+      rec[j] = m_run[j];
+      rec[GQ + j] = l_run[j];
+    }
 }
 
 // ------------------------------------------------------------------------------- fills
@@ -284,7 +291,13 @@ reuse_hit_kernel(Geom g, CacheBuffers cb, Scratch sc, ReuseDev st) {
 // (ring + x) mod E.  Per tile, like the encoder's predictor pass: the coefficient tile by TMA,
 // D1_hh = (W1'_hh / 2) A^T (SS, M = 128 hidden rows, N = C tokens), H = silu(2 D1) as fp16 in
 // shared memory (MN-major), D2 = W2 H (SS, M = 128 value dims, N = C), then vhat = D2 plus the
-// chunk's residual rows, written to the entry as bf16 [C][d].
+// chunk's residual rows, assembled as bf16 [C][d] in shared memory and written to the entry
+// by one bulk copy.  Latency hiding within the CTA: the residual rows are staged by cp.async
+// while the MMAs run; the next tile's coefficient tile (and W1', W2 at a new (layer, KV head))
+// are requested as soon as the current tile's MMAs are done, i.e. during its epilogue; the
+// next tile's unit, slot and record range are read one tile ahead.
+constexpr int kFillResStage = 32;   // residual rows of a chunk staged in shared memory
+
 template <int R>
 struct FillLayout {
   static constexpr int KSLABS = R / 64;
@@ -295,9 +308,11 @@ struct FillLayout {
   static constexpr int OFF_W1 = 0;
   static constexpr int OFF_W2 = OFF_W1 + 2 * W1_HALF;
   static constexpr int OFF_AH = OFF_W2 + W2_BYTES;           // the A tile, then H half 0
-  static constexpr int OFF_H1 = OFF_AH + (A_BYTES > H_HALF ? A_BYTES : H_HALF);
-  static constexpr int OFF_MISC = OFF_H1 + H_HALF;
+  static constexpr int OFF_H1 = OFF_AH + (A_BYTES > H_HALF ? A_BYTES : H_HALF);   // H half 1, then vhat
+  static constexpr int OFF_RES = OFF_H1 + H_HALF;            // bf16 [kFillResStage][d]
+  static constexpr int OFF_MISC = OFF_RES + kFillResStage * kD * 2;
   static constexpr int SMEM = OFF_MISC + 64 + kC * 4 + 1024;
+  static_assert(kC * kD * 2 <= H_HALF, "vhat tile fits the H half-1 buffer");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
@@ -315,12 +330,15 @@ reuse_fill_kernel(Geom g, CacheBuffers cb, Scratch sc, ReuseDev st, const __grid
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_w + 3);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* tok_rec = reinterpret_cast<int*>(smem + Lay::OFF_MISC + 64);   // [C]: token -> record, or -1
+  const __nv_bfloat16* res_s = reinterpret_cast<const __nv_bfloat16*>(smem + Lay::OFF_RES);
+  __nv_bfloat16* out_s = reinterpret_cast<__nv_bfloat16*>(smem + Lay::OFF_H1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int NG = g.L / g.G;
   const long long n_fill = min((long long)*sc.tile_total, (long long)st.fill_cap);
   const long long x0 = n_fill * blockIdx.x / gridDim.x, x1 = n_fill * (blockIdx.x + 1) / gridDim.x;
   const int ring = *st.ring;
   uint32_t* err = sc.err;
+  const __nv_bfloat16* rv = reinterpret_cast<const __nv_bfloat16*>(cb.res_val);
   if (tid == 0) {
     mbar_init(bar_w, 1);
     mbar_init(bar_in, 1);
@@ -344,51 +362,89 @@ reuse_fill_kernel(Geom g, CacheBuffers cb, Scratch sc, ReuseDev st, const __grid
   constexpr uint32_t IDESC_1 = idesc_f16(128, kC, 1, 1);         // W1'/2 (bf16) x A (bf16)
   constexpr uint32_t IDESC_2 = idesc_f16(128, kC, 0, 0, 0, 1);   // W2 (f16) x H (f16, MN-major)
   uint32_t ph_w = 0, ph_in = 0, ph_mma = 0;
+  bool w_pending = false, a_pending = false;   // copies requested and not yet waited for
+  bool m_pending = false;                      // MMAs committed and not yet waited for
   int cur_seg = -1;
   bool ok = true;
   const int hh = warp >> 2;                 // silu: hidden half; epilogue: token half
   const int row = 32 * (warp & 3) + lane;   // TMEM lane: hidden unit in the half / value dim
-  for (long long x = x0; ok && x < x1; ++x) {
-    const int u = sc.tile_unit[x], slot = sc.tile_slot[x];
-    const Unit un = unit_of(g, u);
+
+  // tile x's unit, slot, (layer, KV head) and record range
+  struct TileRef {
+    int u, slot, seg, r0, r1;
+    long long arow;
+  };
+  auto tile_ref = [&](long long x) {
+    TileRef t;
+    t.u = sc.tile_unit[x];
+    t.slot = sc.tile_slot[x];
+    const Unit un = unit_of(g, t.u);
     const int l = g.layer0 + un.li, grp = l / g.G;
-    const int seg = l * g.Hkv + un.hkv;
-    const int e = (int)((ring + x) % st.E);
-    if (seg != cur_seg) {   // W1' halves and W2 of this (layer, KV head)
-      if (tid == 0) {
-        mbar_expect_tx(bar_w, (uint32_t)(2 * Lay::W1_HALF + Lay::W2_BYTES));
-        for (int h2 = 0; h2 < 2; ++h2)
-          for (int ks = 0; ks < Lay::KSLABS; ++ks)
-            tma_load_2d(smem + Lay::OFF_W1 + h2 * Lay::W1_HALF + ks * 16384, &tmW1, bar_w, ks * 64,
-                        seg * kH + h2 * 128);
-        for (int j = 0; j < 4; ++j) tma_load_2d(smem + Lay::OFF_W2 + j * 16384, &tmW2, bar_w, j * 64, seg * kD);
-      }
-      ok = mbar_wait(bar_w, ph_w, abort_flag, err, ERR_TIMEOUT);
-      ph_w ^= 1;
-      cur_seg = seg;
-      if (!__syncthreads_and(ok)) break;
-    }
-    const long long arow = ((((long long)un.b * NG + grp) * g.Hkv + un.hkv) * g.nLs + slot) * kC;
-    if (tid == 0) {
-      mbar_expect_tx(bar_in, (uint32_t)(Lay::KSLABS * kC * 128));
-      for (int ks = 0; ks < Lay::KSLABS; ++ks) tma_load_2d(smem + Lay::OFF_AH + ks * 16384, &tmA, bar_in, ks * 64, (int)arow);
-    }
-    // the chunk's residual records: token -> record index
+    t.seg = l * g.Hkv + un.hkv;
+    t.arow = ((((long long)un.b * NG + grp) * g.Hkv + un.hkv) * g.nLs + t.slot) * kC;
     const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nLs + 1);
-    int r0 = rptr[slot], r1 = rptr[slot + 1];
+    t.r0 = rptr[t.slot];
+    t.r1 = rptr[t.slot + 1];
+    return t;
+  };
+  // tid 0, once no MMA reads the buffers: the copies of tile t (W1', W2 only at a new pair)
+  auto issue_loads = [&](const TileRef& t, int seg_now) {
+    if (t.seg != seg_now) {
+      mbar_expect_tx(bar_w, (uint32_t)(2 * Lay::W1_HALF + Lay::W2_BYTES));
+      for (int h2 = 0; h2 < 2; ++h2)
+        for (int ks = 0; ks < Lay::KSLABS; ++ks)
+          tma_load_2d(smem + Lay::OFF_W1 + h2 * Lay::W1_HALF + ks * 16384, &tmW1, bar_w, ks * 64, t.seg * kH + h2 * 128);
+      for (int j = 0; j < 4; ++j) tma_load_2d(smem + Lay::OFF_W2 + j * 16384, &tmW2, bar_w, j * 64, t.seg * kD);
+    }
+    mbar_expect_tx(bar_in, (uint32_t)(Lay::KSLABS * kC * 128));
+    for (int ks = 0; ks < Lay::KSLABS; ++ks)
+      tma_load_2d(smem + Lay::OFF_AH + ks * 16384, &tmA, bar_in, ks * 64, (int)t.arow);
+  };
+
+  TileRef cur{};
+  if (x0 < x1) {
+    cur = tile_ref(x0);
+    if (tid == 0) issue_loads(cur, -1);
+  }
+  for (long long x = x0; ok && x < x1; ++x) {
+    // this tile's copies were issued (before the loop, or during the last tile's epilogue)
+    const bool new_seg = cur.seg != cur_seg;
+    w_pending = w_pending || new_seg;
+    a_pending = true;
+    cur_seg = cur.seg;
+    int r0 = cur.r0, r1 = cur.r1;
     if (r0 < 0 || r1 < r0 || (long long)r1 > (long long)cb.n_records) {
       if (tid == 0) atomicOr(err, ERR_RES_PTR);
       r0 = r1 = 0;
     }
+    // residual rows r0 .. r0 + 31 into shared memory (cp.async), and the token -> record map
+    const int nst = min(r1 - r0, kFillResStage);
+    for (int i = tid; i < nst * (kD / 8); i += 256) {
+      const int rr = i / (kD / 8), c = i % (kD / 8);
+      cp16(smem + Lay::OFF_RES + (rr * kD + c * 8) * 2, rv + (size_t)(r0 + rr) * kD + c * 8);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
     for (int t = tid; t < kC; t += 256) tok_rec[t] = -1;
     __syncthreads();
     for (int i = r0 + tid; i < r1; i += 256) {
       const int pos = cb.res_pos[i];
       if (pos < kC) tok_rec[pos] = i;
     }
+    // the next tile's reference, read now so that it is in registers at the epilogue
+    TileRef nxt{};
+    if (x + 1 < x1) nxt = tile_ref(x + 1);
+    // (a phase flips only once every thread has passed its wait, so that the drain below
+    // waits for the phase a failed wait was on)
+    if (new_seg) {
+      ok = mbar_wait(bar_w, ph_w, abort_flag, err, ERR_TIMEOUT);
+      if (!__syncthreads_and(ok)) break;
+      ph_w ^= 1;
+      w_pending = false;
+    }
     ok = mbar_wait(bar_in, ph_in, abort_flag, err, ERR_TIMEOUT);
-    ph_in ^= 1;
     if (!__syncthreads_and(ok)) break;
+    ph_in ^= 1;
+    a_pending = false;
     if (tid == 0) {
       tc_fence_after();
 #pragma unroll
@@ -399,10 +455,13 @@ reuse_fill_kernel(Geom g, CacheBuffers cb, Scratch sc, ReuseDev st, const __grid
           mma_ss(tmem + h2 * kC, dW1 + (uint64_t)((h2 * Lay::W1_HALF) >> 4) + ko, dA + ko, IDESC_1, kk > 0 ? 1u : 0u);
         }
       mma_commit(bar_mma);
+      bulk_wait_read_all();   // the last tile's vhat (in the H half-1 buffer) has been copied out
     }
+    m_pending = true;
     ok = mbar_wait(bar_mma, ph_mma, abort_flag, err, ERR_TIMEOUT);
-    ph_mma ^= 1;
     if (!__syncthreads_and(ok)) break;
+    ph_mma ^= 1;
+    m_pending = false;
     tc_fence_after();
     {   // silu -> H_hh (fp16) in shared memory, MN-major: hidden row `row`, 8 tokens per 16 bytes
       unsigned char* hrow = smem + (hh == 0 ? Lay::OFF_AH : Lay::OFF_H1) + (row >> 3) * 1024 + (row & 7) * 128;
@@ -439,13 +498,16 @@ reuse_fill_kernel(Geom g, CacheBuffers cb, Scratch sc, ReuseDev st, const __grid
         }
       mma_commit(bar_mma);
     }
+    m_pending = true;
     ok = mbar_wait(bar_mma, ph_mma, abort_flag, err, ERR_TIMEOUT);
-    ph_mma ^= 1;
+    asm volatile("cp.async.wait_group 0;" ::: "memory");   // this thread's residual rows
     if (!__syncthreads_and(ok)) break;
+    ph_mma ^= 1;
+    m_pending = false;
     tc_fence_after();
-    // vhat[t][row] = D2[row][t] + delta_t[row] for tokens hh * 64 .. + 63
-    __nv_bfloat16* dst = st.entries + (size_t)e * kC * kD;
-    const __nv_bfloat16* rv = reinterpret_cast<const __nv_bfloat16*>(cb.res_val);
+    // every MMA of this tile is done: the next tile's copies go out now
+    if (tid == 0 && x + 1 < x1) issue_loads(nxt, cur_seg);
+    // vhat[t][row] = D2[row][t] + delta_t[row] for tokens hh * 64 .. + 63, into shared memory
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       uint32_t v[32];
@@ -455,14 +517,33 @@ reuse_fill_kernel(Geom g, CacheBuffers cb, Scratch sc, ReuseDev st, const __grid
       for (int j = 0; j < 32; ++j) {
         const int t = hh * 64 + q * 32 + j;
         float val = __uint_as_float(v[j]);
-        const int ri = tok_rec[t];
-        if (ri >= 0) val += __bfloat162float(rv[(size_t)ri * kD + row]);
-        dst[(size_t)t * kD + row] = __float2bfloat16_rn(val);
+        const int ri = tok_rec[t];   // the same for the whole warp
+        if (ri >= 0) {
+          const int si = ri - r0;
+          val += __bfloat162float(si < kFillResStage ? res_s[si * kD + row] : rv[(size_t)ri * kD + row]);
+        }
+        out_s[t * kD + row] = __float2bfloat16_rn(val);
       }
     }
     tc_fence_before();
-    __syncthreads();   // H / A buffers and tok_rec are reused by the next tile
+    fence_proxy_async_smem();
+    __syncthreads();   // vhat complete; tok_rec and the staged rows are free again
+    if (tid == 0) {
+      bulk_store(st.entries + (size_t)((ring + x) % st.E) * kC * kD, out_s, (uint32_t)(kC * kD * 2));
+      bulk_commit();
+    }
+    cur = nxt;
   }
+  if (tid == 0) {
+    bulk_wait_all();
+    if (!ok) {   // a wait gave up: let the copies this CTA started land before it exits
+      volatile int never = 0;
+      if (w_pending) mbar_wait(bar_w, ph_w, &never, err, ERR_TIMEOUT);
+      if (a_pending) mbar_wait(bar_in, ph_in, &never, err, ERR_TIMEOUT);
+      if (m_pending) mbar_wait(bar_mma, ph_mma, &never, err, ERR_TIMEOUT);   // TMEM is freed below
+    }
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
@@ -472,12 +553,20 @@ reuse_fill_kernel(Geom g, CacheBuffers cb, Scratch sc, ReuseDev st, const __grid
 
 // ------------------------------------------------------------------------------ commit
 // The table after the fills: entry (ring + x) mod E now holds tile x of the miss list; its
-// previous chunk leaves the table.  Then the ring and the fill counter advance.
+// previous chunk leaves the table.  Then the ring and the fill counter advance.  One thread
+// per fill: the call's fills have distinct chunks and distinct entries, and no chunk they
+// evict is one of them (an evicted chunk was in the table, so it was a hit, not a miss).
+// The ring position comes from ring[1] (copied by the plan kernel), so the thread that
+// advances ring[0] races with no reader.
 __global__ void __launch_bounds__(256)
 reuse_commit_kernel(Geom g, Scratch sc, ReuseDev st) {
   const long long n_fill = min((long long)*sc.tile_total, (long long)st.fill_cap);
-  const int ring = *st.ring;
-  for (long long x = threadIdx.x; x < n_fill; x += blockDim.x) {
+  const int ring = st.ring[1];
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    st.ring[0] = (int)((ring + n_fill) % st.E);
+    st.counters[2] += (unsigned long long)n_fill;
+  }
+  for (long long x = (long long)blockIdx.x * blockDim.x + threadIdx.x; x < n_fill; x += (long long)gridDim.x * blockDim.x) {
     const int u = sc.tile_unit[x], slot = sc.tile_slot[x];
     const Unit un = unit_of(g, u);
     const int l = g.layer0 + un.li;
@@ -487,11 +576,6 @@ reuse_commit_kernel(Geom g, Scratch sc, ReuseDev st) {
     if (old >= 0 && st.table[old] == e) st.table[old] = -1;
     st.owner[e] = key;
     st.table[key] = e;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    *st.ring = (int)((ring + n_fill) % st.E);
-    st.counters[2] += (unsigned long long)n_fill;
   }
 }
 
@@ -548,7 +632,7 @@ cudaError_t run_reuse(const Geom& g, const CacheBuffers& cb, const Scratch& sc, 
   if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM)) != cudaSuccess) return e;
   k<<<n_sm, 256, Lay::SMEM, s>>>(g, cb, sc, st, tmW1, tmW2, tmA);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  reuse_commit_kernel<<<1, 256, 0, s>>>(g, sc, st);
+  reuse_commit_kernel<<<(unsigned)std::min<long long>(((long long)g.U * g.k + 255) / 256, 4LL * n_sm), 256, 0, s>>>(g, sc, st);
   return cudaGetLastError();
 }
 

@@ -10,7 +10,7 @@ struct ReuseDev {
   __nv_bfloat16* entries;        // [E][C][d]: rebuilt values of one (unit, chunk) each
   int32_t* table;                // [B][L][Hkv][table_stride]: entry of each chunk slot, or -1
   long long* owner;              // [E]: table index an entry serves, or -1
-  int32_t* ring;                 // [1]: next entry to fill
+  int32_t* ring;                 // [2]: next entry to fill; [1] its copy taken by the plan kernel
   unsigned long long* counters;  // [3]: hits, misses, fills (cumulative)
   int32_t* hit_entry;            // [U][k] per call: the unit's hit entries ...
   int32_t* hit_slot;             // [U][k] ... and their chunk slots

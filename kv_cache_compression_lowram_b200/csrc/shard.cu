@@ -173,17 +173,22 @@ shard_scan_kernel(int U, int k, Scratch sc) {
   }
   int base = part[tid] - sum;
   for (int u = u0; u < u1; ++u) {
-    const int cnt = sc.unit_ntile[u];
     sc.tile_ptr[u] = base;
-    for (int i = 0; i < cnt; ++i) {
-      sc.tile_unit[base + i] = u;
-      sc.tile_slot[base + i] = sc.sel_slot[(size_t)u * k + i];
-    }
-    base += cnt;
+    base += sc.unit_ntile[u];
   }
   if (tid == kScanThreads - 1) {
     sc.tile_ptr[U] = part[tid];
     *sc.tile_total = part[tid];
+  }
+  __syncthreads();   // the offsets above are visible to the whole block
+  // the list itself: one warp per unit, one lane per tile (coalesced)
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int u = warp; u < U; u += kScanThreads / 32) {
+    const int b0 = sc.tile_ptr[u], cnt = sc.tile_ptr[u + 1] - b0;
+    for (int i = lane; i < cnt; i += 32) {
+      sc.tile_unit[b0 + i] = u;
+      sc.tile_slot[b0 + i] = sc.sel_slot[(size_t)u * k + i];
+    }
   }
 }
 
