@@ -126,8 +126,13 @@ def aggregate_rate(queries_per_rank: float, ms_total: float, ws: int):
 # The figure stands only while the kernel's sources are the captured ones, so it carries
 # their hash.
 ATTEND_TC_SOURCES = ("attend_tc.cu", "tc_ptx.cuh", "lowram_internal.cuh")
+# The int8 + eviction workload's figure: 78.39 MB on its 128-unit case
+#   ncu --set full --clock-control none -k regex:attend_tc -s 3 -c 1 -o prof_i8 \
+#       python bench.py --config llama8b_64k_int8_evict_b2_l8 --steps 3 --warmup 3 --no-cpu-baseline
+# scaled by its 2048 units (x16).
 MEASURED_TRAFFIC = {
     "llama8b_32k_bf16": {"bytes": 1378693120, "sources_sha1": "f5c84f105739c204a47aa2fa824ea9b7ae0c0d33"},
+    "llama8b_64k_int8_evict": {"bytes": 1254232064, "sources_sha1": "44abd08d2b474f45a6bc2b362f1604ef429b0fe0"},
 }
 
 

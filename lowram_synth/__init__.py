@@ -162,6 +162,8 @@ LLAMA_64K_INT8 = _reg(LowramConfig(
     name="llama8b_64k_int8_evict", batch=8, n_layers=32, group=4, n_kv_heads=8,
     n_q_heads=32, head_dim=128, rank=128, mlp_hidden=256, n_ctx=65536, chunk=128, top_k=32,
     tail_cap=128, resid_frac=0.125, dtype="bf16", store="int8", evict_frac=0.5, seed=4000))
+# Its small profiling case (2 sequences, 8 layers: 0.13 GB of int8 coefficients).
+_reg(LLAMA_64K_INT8.replace(name="llama8b_64k_int8_evict_b2_l8", batch=2, n_layers=8))
 
 
 def get_config(name: str) -> LowramConfig:
