@@ -937,6 +937,17 @@ def run_reuse(args, ws, rank, local):
         value, ms_total = aggregate_rate(queries, reuse_ms, ws)
         pvalue, pms_total = aggregate_rate(queries, plain_ms, ws)
         hits, misses, fills = (c1[x] - c0[x] for x in ("hits", "misses", "fills"))
+        # work per step by kind of chunk: a hit reads the coefficient tile and the stored
+        # values and runs no predictor; a miss reads the tile and its residual records; a
+        # fill reads them once more and writes the entry
+        tile_b = cfg.chunk * cfg.rank * 2
+        rec_b = round(cfg.resid_frac * cfg.chunk) * (cfg.head_dim * 2 + 2)
+        entry_b = cfg.chunk * cfg.head_dim * 2
+        work = {"silu_saved": round(hits / args.steps) * cfg.chunk * cfg.mlp_hidden,
+                "hit_bytes": round(hits / args.steps) * (tile_b + entry_b),
+                "miss_bytes": round(misses / args.steps) * (tile_b + rec_b),
+                "fill_bytes": round(fills / args.steps) * (tile_b + rec_b + entry_b),
+                "plain_bytes": round((hits + misses) / args.steps) * (tile_b + rec_b)}
         lines.append({
             "metric": REUSE_METRIC, "value": round(value, 1), "unit": "queries/s", "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_total / args.steps, 4),
@@ -945,6 +956,7 @@ def run_reuse(args, ws, rank, local):
             "config": {"workload": cfg.name, "rho": 0.9, "drift": drift, "capacity": cap, "fill_cap": fill_cap,
                        "store_bytes": cap * cfg.chunk * cfg.head_dim * 2, "parallelism": f"replicas x{ws}"},
             "hit_rate": round(hits / max(1, hits + misses), 4), "fills_per_step": round(fills / args.steps, 1),
+            "work_per_step": work,
             "plain": {"value": round(pvalue, 1), "ms_per_step": round(pms_total / args.steps, 4)},
             "speedup_vs_plain": round(pms_total / ms_total, 4),
             "gpu_launches": launches * args.steps, "clocks": clk,

@@ -424,15 +424,7 @@ reuse_fill_kernel(Geom g, CacheBuffers cb, Scratch sc, ReuseDev st, const __grid
       cp16(smem + Lay::OFF_RES + (rr * kD + c * 8) * 2, rv + (size_t)(r0 + rr) * kD + c * 8);
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
-    for (int t = tid; t < kC; t += 256) tok_rec[t] = -1;
-    __syncthreads();
-    for (int i = r0 + tid; i < r1; i += 256) {
-      const int pos = cb.res_pos[i];
-      if (pos < kC) tok_rec[pos] = i;
-    }
-    // the next tile's reference, read now so that it is in registers at the epilogue
-    TileRef nxt{};
-    if (x + 1 < x1) nxt = tile_ref(x + 1);
+    for (int t = tid; t < kC; t += 256) tok_rec[t] = -1;   // filled once the MMAs are issued
     // (a phase flips only once every thread has passed its wait, so that the drain below
     // waits for the phase a failed wait was on)
     if (new_seg) {
@@ -457,6 +449,14 @@ reuse_fill_kernel(Geom g, CacheBuffers cb, Scratch sc, ReuseDev st, const __grid
       mma_commit(bar_mma);
       bulk_wait_read_all();   // the last tile's vhat (in the H half-1 buffer) has been copied out
     }
+    // while the pre-activations run: the token -> record map (the barrier above ordered the
+    // reset) and the next tile's reference (both dependent global loads)
+    for (int i = r0 + tid; i < r1; i += 256) {
+      const int pos = cb.res_pos[i];
+      if (pos < kC) tok_rec[pos] = i;
+    }
+    TileRef nxt{};
+    if (x + 1 < x1) nxt = tile_ref(x + 1);
     m_pending = true;
     ok = mbar_wait(bar_mma, ph_mma, abort_flag, err, ERR_TIMEOUT);
     if (!__syncthreads_and(ok)) break;
