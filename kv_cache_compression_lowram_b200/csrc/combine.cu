@@ -144,7 +144,8 @@ struct CombSmem {
   static constexpr int MAXP = LIST ? 33 : kCombPieces;             // pieces per unit
   static constexpr size_t WT = ACCD + NR * 128 * 4;                 // float [NR][MAXP + 2]
   static constexpr size_t LS = WT + NR * (MAXP + 2) * 4;            // float [NR]
-  static constexpr size_t PC = LS + NR * 4;                         // int [UB][2]: first piece, pieces
+  static constexpr size_t MS = LS + NR * 4;                         // float [NR]: merged max
+  static constexpr size_t PC = MS + NR * 4;                         // int [UB][2]: first piece, pieces
   static constexpr size_t BYTES = PC + UB * 2 * 4;
 };
 
@@ -155,12 +156,14 @@ __device__ __forceinline__ void cp_async16c(void* smem_dst, const void* gsrc) {
 }
 
 // LIST: the pieces come from an explicit tile list (sc.tile_ptr / sc.tile_total; units may
-// have any number of tiles, none included) and every unit has one extra record in the tail's
-// format (extra_rec, [U][tail_stride]), merged like the tail.
-template <int GQ, bool LIST>
+// have any number of tiles, none included) and, when extra_rec is given, every unit has one
+// extra record in the tail's format (extra_rec, [U][tail_stride]), merged like the tail.
+// PART: the output is left unnormalised, one fp32 row [m (log2 units), l, y[0..d)] per
+// (layer, sequence, query head) in `part` (a context shard's partial), instead of bf16 o.
+template <int GQ, bool LIST, bool PART = false>
 __global__ void __launch_bounds__(kCombThreads, 2)
 combine_mma_kernel(Geom g, CacheBuffers cb, Scratch sc, const float* __restrict__ extra_rec,
-                   __nv_bfloat16* __restrict__ out) {
+                   __nv_bfloat16* __restrict__ out, float* __restrict__ part) {
   constexpr int D = 128, H = 256;
   using SM = CombSmem<GQ, LIST>;
   constexpr int UB = SM::UB, NR = SM::NR, WROW = SM::WROW, MAXP = SM::MAXP;
@@ -170,6 +173,8 @@ combine_mma_kernel(Geom g, CacheBuffers cb, Scratch sc, const float* __restrict_
   float (*accd)[D] = reinterpret_cast<float (*)[D]>(smem + SM::ACCD);
   float (*wt)[MAXP + 2] = reinterpret_cast<float (*)[MAXP + 2]>(smem + SM::WT);
   float* ls = reinterpret_cast<float*>(smem + SM::LS);
+  float* ms = reinterpret_cast<float*>(smem + SM::MS);
+  const bool has_x = LIST && extra_rec != nullptr;
   int (*pc)[2] = reinterpret_cast<int (*)[2]>(smem + SM::PC);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nbb = (g.B + UB - 1) / UB;
@@ -215,9 +220,9 @@ combine_mma_kernel(Geom g, CacheBuffers cb, Scratch sc, const float* __restrict_
       }
       const int np = min(nrec, MAXP);
       const float* trec = sc.tail_part + (size_t)u * g.tail_stride;
-      const float* xrec = LIST ? extra_rec + (size_t)u * g.tail_stride : trec;
+      const float* xrec = has_x ? extra_rec + (size_t)u * g.tail_stride : trec;
       float M = trec[j];
-      if (LIST) M = fmaxf(M, xrec[j]);
+      if (has_x) M = fmaxf(M, xrec[j]);
       for (int p = 0; p < np; ++p) M = fmaxf(M, sc.part[(size_t)(u + c0 + p) * g.rec_stride + j]);
       for (int p = 0; p < np; ++p) {
         const float* rec = sc.part + (size_t)(u + c0 + p) * g.rec_stride;
@@ -228,11 +233,12 @@ combine_mma_kernel(Geom g, CacheBuffers cb, Scratch sc, const float* __restrict_
       const float w_t = trec[j] == -INFINITY ? 0.f : exp2f(trec[j] - M);
       wt[r][MAXP] = w_t;
       L = fmaf(w_t, trec[GQ + j], L);
-      if (LIST) {
+      if (has_x) {
         const float w_x = xrec[j] == -INFINITY ? 0.f : exp2f(xrec[j] - M);
         wt[r][MAXP + 1] = w_x;
         L = fmaf(w_x, xrec[GQ + j], L);
       }
+      ms[r] = M;
     }
     ls[r] = L;
   }
@@ -273,6 +279,7 @@ combine_mma_kernel(Geom g, CacheBuffers cb, Scratch sc, const float* __restrict_
       }
 #pragma unroll
       for (int xr = 0; xr < (LIST ? 2 : 1); ++xr) {   // the tail, then the extra record
+        if (xr == 1 && !has_x) break;
         const float w_t = wt[r][MAXP + xr];
         const float* base = xr ? extra_rec : sc.tail_part;
         const float4* tv = reinterpret_cast<const float4*>(base + (size_t)u * g.tail_stride + 2 * GQ + j * D + s * 8);
@@ -321,10 +328,21 @@ combine_mma_kernel(Geom g, CacheBuffers cb, Scratch sc, const float* __restrict_
   for (int nt = 0; nt < 4; ++nt) {
     const int r = 4 * nt + (lane & 3), bi = r / GQ, j = r % GQ;
     if (bi < nb) {
-      __nv_bfloat16* o = out + ((size_t)(li * g.B + b0 + bi) * g.Hq + (size_t)hkv * GQ + j) * D;
+      const size_t orow = (size_t)(li * g.B + b0 + bi) * g.Hq + (size_t)hkv * GQ + j;
       const int d0 = 16 * warp + gq;
-      o[d0] = __float2bfloat16_rn((acc[nt][0] + acc[nt][1] + accd[r][d0]) / ls[r]);
-      o[d0 + 8] = __float2bfloat16_rn((acc[nt][2] + acc[nt][3] + accd[r][d0 + 8]) / ls[r]);
+      if (PART) {
+        float* pr = part + orow * (D + 2);
+        pr[2 + d0] = acc[nt][0] + acc[nt][1] + accd[r][d0];
+        pr[2 + d0 + 8] = acc[nt][2] + acc[nt][3] + accd[r][d0 + 8];
+        if (warp == 0 && gq == 0) {
+          pr[0] = ms[r];
+          pr[1] = ls[r];
+        }
+      } else {
+        __nv_bfloat16* o = out + orow * D;
+        o[d0] = __float2bfloat16_rn((acc[nt][0] + acc[nt][1] + accd[r][d0]) / ls[r]);
+        o[d0 + 8] = __float2bfloat16_rn((acc[nt][2] + acc[nt][3] + accd[r][d0 + 8]) / ls[r]);
+      }
     }
   }
 }
@@ -459,7 +477,8 @@ cudaError_t launch_combine(const Geom& g, const CacheBuffers& cb, const Scratch&
     at[0].val.programmaticStreamSerializationAllowed = 1;
     lc.attrs = at;
     lc.numAttrs = 1;
-    e = cudaLaunchKernelEx(&lc, k, g, cb, sc, static_cast<const float*>(nullptr), static_cast<__nv_bfloat16*>(out));
+    e = cudaLaunchKernelEx(&lc, k, g, cb, sc, static_cast<const float*>(nullptr), static_cast<__nv_bfloat16*>(out),
+                           static_cast<float*>(nullptr));
     if (e != cudaSuccess) return e;
   } else {
     auto k = combine_kernel<__nv_bfloat16>;
@@ -479,7 +498,20 @@ cudaError_t launch_combine_list(const Geom& g, const CacheBuffers& cb, const Scr
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)(g.n_layers * g.Hkv) * (unsigned)((g.B + ub - 1) / ub);
-  k<<<grid, kCombThreads, sm, s>>>(g, cb, sc, extra_rec, static_cast<__nv_bfloat16*>(out));
+  k<<<grid, kCombThreads, sm, s>>>(g, cb, sc, extra_rec, static_cast<__nv_bfloat16*>(out), static_cast<float*>(nullptr));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_partial_fast(const Geom& g, const CacheBuffers& cb, const Scratch& sc, float* partial,
+                                        cudaStream_t s) {
+  if (g.d != 128 || g.h != 256 || !(g.g == 4 || g.g == 8) || g.k > 32) return cudaErrorNotSupported;
+  auto k = g.g == 4 ? combine_mma_kernel<4, true, true> : combine_mma_kernel<8, true, true>;
+  const size_t sm = g.g == 4 ? CombSmem<4, true>::BYTES : CombSmem<8, true>::BYTES;
+  const int ub = 16 / g.g;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = (unsigned)(g.n_layers * g.Hkv) * (unsigned)((g.B + ub - 1) / ub);
+  k<<<grid, kCombThreads, sm, s>>>(g, cb, sc, nullptr, nullptr, partial);
   return cudaGetLastError();
 }
 

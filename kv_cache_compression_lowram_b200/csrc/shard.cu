@@ -311,6 +311,9 @@ cudaError_t launch_tile_scan(const Geom& g, const Scratch& sc, cudaStream_t s) {
 
 cudaError_t launch_combine_partial(const Geom& g, const CacheBuffers& cb, const Scratch& sc, int dtype,
                                    float* partial, cudaStream_t s) {
+  // bf16, d = 128, h = 256, g in {4, 8}, k <= 32: the warp-MMA combine writes the partials
+  if (dtype != LOWRAM_F32 && g.d == 128 && g.h == 256 && (g.g == 4 || g.g == 8) && g.k <= 32)
+    return launch_combine_partial_fast(g, cb, sc, partial, s);
   const int max_pieces = g.k < g.P ? g.k : g.P;
   const size_t smem = sizeof(float) * ((size_t)g.g * g.h + (size_t)g.g * g.d + (size_t)(max_pieces + 1) * g.g + 2 * g.g);
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
