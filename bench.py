@@ -120,9 +120,10 @@ def aggregate_rate(queries_per_rank: float, ms_total: float, ws: int):
 
 # DRAM traffic of the tensor-core attend kernel per launch (dram__bytes_read.sum +
 # dram__bytes_write.sum from one ncu capture:
-#   ncu --set full --clock-control none -k regex:attend_tc -s 1 -c 1 -o prof \
+#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum \
+#       --clock-control none -k regex:attend_tc -s 1 -c 1 --csv --log-file dram_b1.csv \
 #       python bench.py --config llama8b_32k_bf16_b1 --steps 1 --warmup 1 --no-cpu-baseline
-# 344.84 MB on that 256-unit case, scaled by the units of the named workload: 1024, x4).
+# 343.92 MB on that 256-unit case, scaled by the units of the named workload: 1024, x4).
 # The figure stands only while the kernel's sources are the captured ones, so it carries
 # their hash.
 ATTEND_TC_SOURCES = ("attend_tc.cu", "tc_ptx.cuh", "lowram_internal.cuh")
@@ -131,7 +132,7 @@ ATTEND_TC_SOURCES = ("attend_tc.cu", "tc_ptx.cuh", "lowram_internal.cuh")
 #       python bench.py --config llama8b_64k_int8_evict_b2_l8 --steps 3 --warmup 3 --no-cpu-baseline
 # scaled by its 2048 units (x16).
 MEASURED_TRAFFIC = {
-    "llama8b_32k_bf16": {"bytes": 1378693120, "sources_sha1": "f5c84f105739c204a47aa2fa824ea9b7ae0c0d33"},
+    "llama8b_32k_bf16": {"bytes": 1375687680, "sources_sha1": "44abd08d2b474f45a6bc2b362f1604ef429b0fe0"},
     "llama8b_64k_int8_evict": {"bytes": 1254232064, "sources_sha1": "44abd08d2b474f45a6bc2b362f1604ef429b0fe0"},
 }
 

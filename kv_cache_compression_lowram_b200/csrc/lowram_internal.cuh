@@ -194,9 +194,6 @@ cudaError_t launch_encode(const Geom& g, int store, int n_res, const void* keys,
 // head ([n_layers][B][Hq][d + 2]: m in log2 units, l, y), and the merge of the shards' partials.
 cudaError_t launch_shard_select(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const float* cand_score,
                                 const int32_t* cand_id, int n_shards, int offset, int32_t* sel_out, cudaStream_t s);
-// The same on the warp-MMA combine (bf16, d = 128, h = 256, g in {4, 8}, k <= 32).
-cudaError_t launch_combine_partial_fast(const Geom& g, const CacheBuffers& cb, const Scratch& sc, float* partial,
-                                        cudaStream_t s);
 cudaError_t launch_combine_partial(const Geom& g, const CacheBuffers& cb, const Scratch& sc, int dtype,
                                    float* partial, cudaStream_t s);
 cudaError_t launch_merge_partials(int n_parts, long long n_rows, int d, const float* parts, int out_dtype, void* out,

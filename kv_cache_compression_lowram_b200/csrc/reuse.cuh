@@ -32,6 +32,11 @@ cudaError_t launch_reuse(const Geom& g, const CacheBuffers& cb, const Scratch& s
 cudaError_t launch_tile_scan(const Geom& g, const Scratch& sc, cudaStream_t s);
 // Combine over an explicit tile list plus one extra record per unit in the tail's format
 // (the reuse store's hits), normalised (combine.cu).
+// Per unit the pieces of the tile list and the tail merged, W2 applied, left unnormalised:
+// rows [m (log2 units), l, y[0..d)] per (layer, sequence, query head) (a context shard's
+// partial), on the warp-MMA combine (bf16, d = 128, h = 256, g in {4, 8}, k <= 32); combine.cu.
+cudaError_t launch_combine_partial_fast(const Geom& g, const CacheBuffers& cb, const Scratch& sc, float* partial,
+                                        cudaStream_t s);
 cudaError_t launch_combine_list(const Geom& g, const CacheBuffers& cb, const Scratch& sc, const float* extra_rec,
                                 void* out, cudaStream_t s);
 
