@@ -659,6 +659,7 @@ enc_resid_tc_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant__
       uint32_t v[32];
       tmem_ld32(tmem + lane_off + 2 * C + hh * (C / 2) + q * 32, v);
       tmem_wait_ld();
+      float ss[32];   // pass 1: this lane's d^2 for the 32 tokens of the slice
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const int t = hh * (C / 2) + q * 32 + j;
@@ -666,15 +667,29 @@ enc_resid_tc_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant__
         const float vt = __uint_as_float(((j & 1) ? (w >> 16) : (w & 0xffffu)) << 16);
         const float d = vt - __uint_as_float(v[j]);
         if (!EMIT) {
-          float ss = d * d;
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-          if (lane == 0) part[(warp & 3) * C + t] = ss;
+          ss[j] = d * d;
         } else if (fl[t]) {
           const size_t rec = rbase + pfx[t];
           res_val[rec * kEncD + row] = __float2bfloat16_rn(d);
           if (row == 0) res_pos[rec] = (uint16_t)t;
         }
+      }
+      if (!EMIT) {
+        // sums over the warp's 32 dims for 32 tokens with 31 shuffles (a transposing
+        // butterfly: at distance o a lane keeps the half of its partial sums whose token
+        // index has bit o equal to its own, adds the partner's, and passes the other half),
+        // after which lane L holds token L's sum
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+          const bool up = (lane & o) != 0;
+#pragma unroll
+          for (int i = 0; i < o; ++i) {
+            const float keep = up ? ss[i + o] : ss[i];
+            const float give = up ? ss[i] : ss[i + o];
+            ss[i] = keep + __shfl_xor_sync(0xffffffffu, give, o);
+          }
+        }
+        part[(warp & 3) * C + hh * (C / 2) + q * 32 + lane] = ss[0];
       }
     }
     tc_fence_before();
