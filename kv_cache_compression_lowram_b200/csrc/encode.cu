@@ -705,6 +705,303 @@ enc_resid_tc_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant__
   }
 }
 
+// ------------------------------------------- tensor-core residuals, C = 128, tokens as M
+// The same pass with the chunk's 128 tokens as the MMAs' M dimension, so that every
+// per-token step of the epilogue (the token's values row against its rebuilt row, the norm
+// of the difference, the record) is local to one thread:
+//   D1^T = A . (W1'/2)^T (SS, M = 128 tokens, N = 128 per hidden half, K = R)
+//   H^T  = silu(2 D1^T) as fp16 pairs, written over the first 128 of the tile's TMEM columns
+//          (thread = token: its 256 hidden units)
+//   D2^T = H^T . W2^T    (TS: A = H from TMEM, B = W2 in fp16, K-major; M = 128 tokens,
+//          N = 128 value dims, K = 256), into the tile's columns 128..255
+// Two tiles in flight: tile i of the CTA's range uses TMEM columns [256 (i%2), +256) and
+// coefficient stage i%2; warps 0-3 take the even tiles, 4-7 the odd ones; warp 8 issues the
+// copies and the MMAs, the next tile's pre-activations before this tile's second GEMM.
+constexpr int kEnc2Threads = 288;
+
+template <int R>
+struct EncTc2Layout {
+  static constexpr int KSLABS = R / 64;
+  static constexpr int W1_HALF = KSLABS * 16384;          // 128 hidden rows x R, bf16
+  static constexpr int W2_BYTES = 4 * 16384;              // 128 dims x 256 hidden, fp16
+  static constexpr int A_BYTES = KSLABS * 16384;          // 128 tokens x R, bf16
+  static constexpr int OFF_W1 = 0;
+  static constexpr int OFF_W2 = OFF_W1 + 2 * W1_HALF;
+  static constexpr int OFF_A = OFF_W2 + W2_BYTES;         // two stages
+  static constexpr int OFF_MISC = OFF_A + 2 * A_BYTES;
+  static constexpr int SMEM = OFF_MISC + 256 + 1024;
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+struct EncTc2Misc {
+  uint64_t w_full, drain, a_full[2], a_empty[2], d1_full[2], h_ready[2], d2_full[2], slot_free[2];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int R, bool EMIT>
+__global__ void __launch_bounds__(kEnc2Threads, 1)
+enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant__ CUtensorMap tmW1,
+                     const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmA,
+                     const __nv_bfloat16* __restrict__ values, float* __restrict__ norms,
+                     const uint8_t* __restrict__ flags, const int32_t* __restrict__ res_ptr,
+                     uint16_t* __restrict__ res_pos, __nv_bfloat16* __restrict__ res_val, uint32_t* err) {
+  using namespace tc;
+  constexpr int C = 128;
+  using Lay = EncTc2Layout<R>;
+  extern __shared__ unsigned char enc2_smem_dyn[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(enc2_smem_dyn) + 1023) & ~uintptr_t(1023));
+  EncTc2Misc* misc = reinterpret_cast<EncTc2Misc*>(smem + Lay::OFF_MISC);
+  volatile int* abort_flag = &misc->abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nC = N / C, NG = L / G;
+  const long long total = (long long)B * L * Hkv * nC;
+  const long long x0 = total * blockIdx.x / gridDim.x, x1 = total * (blockIdx.x + 1) / gridDim.x;
+  const long long n = x1 - x0;
+
+  if (tid == 0) {
+    mbar_init(&misc->w_full, 1);
+    mbar_init(&misc->drain, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&misc->a_full[s], 1);
+      mbar_init(&misc->a_empty[s], 1);
+      mbar_init(&misc->d1_full[s], 1);
+      mbar_init(&misc->h_ready[s], 4);     // the 4 warps of the tile's group
+      mbar_init(&misc->d2_full[s], 1);
+      mbar_init(&misc->slot_free[s], 4);
+    }
+    misc->abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == 8) {
+    tmem_alloc(&misc->tmem_base, 512);
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc->tmem_base;
+
+  if (warp == 8) {
+    // ============================================================ copies and MMAs
+    const bool leader = elect_one();
+    const uint64_t dW1 = smem_desc(smem_u32(smem + Lay::OFF_W1), 16, 1024, 2);
+    const uint64_t dW2 = smem_desc(smem_u32(smem + Lay::OFF_W2), 16, 1024, 2);
+    const uint64_t dA0 = smem_desc(smem_u32(smem + Lay::OFF_A), 16, 1024, 2);
+    constexpr uint32_t IDESC_1 = idesc_f16(128, 128, 1, 1);   // A (bf16) x W1'/2 (bf16), both K-major
+    constexpr uint32_t IDESC_2 = idesc_f16(128, 128, 0, 0);   // H (TMEM, fp16) x W2 (fp16, K-major)
+    auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, par, abort_flag, err, ERR_TIMEOUT));
+    };
+    auto seg_of = [&](long long i) { return (int)((x0 + i) / nC / B); };
+    auto issue_a = [&](long long i) {   // tile i's coefficient tile into stage i % 2
+      const long long x = x0 + i;
+      const int u = (int)(x / nC), c = (int)(x % nC);
+      const int b = u % B, seg = u / B, hkv = seg % Hkv, l = seg / Hkv, grp = l / G;
+      const long long arow = (((long long)b * NG + grp) * Hkv + hkv) * N + (long long)c * C;
+      if (leader) {
+        mbar_expect_tx(&misc->a_full[i & 1], (uint32_t)Lay::A_BYTES);
+        for (int ks = 0; ks < Lay::KSLABS; ++ks)
+          tma_load_2d(smem + Lay::OFF_A + (i & 1) * Lay::A_BYTES + ks * 16384, &tmA, &misc->a_full[i & 1], ks * 64,
+                      (int)arow);
+      }
+      __syncwarp();
+    };
+    uint32_t ph_w = 0, ph_drain = 0;
+    long long a_waited = 0, a_issued = 0;   // coefficient copies consumed / issued
+    bool ok = true, w_pending = false;
+    auto load_w = [&](int seg) -> bool {   // W1' halves and W2 of this (layer, KV head)
+      w_pending = true;
+      if (leader) {
+        mbar_expect_tx(&misc->w_full, (uint32_t)(2 * Lay::W1_HALF + Lay::W2_BYTES));
+        for (int h2 = 0; h2 < 2; ++h2)
+          for (int ks = 0; ks < Lay::KSLABS; ++ks)
+            tma_load_2d(smem + Lay::OFF_W1 + h2 * Lay::W1_HALF + ks * 16384, &tmW1, &misc->w_full, ks * 64,
+                        seg * 256 + h2 * 128);
+        for (int j = 0; j < 4; ++j) tma_load_2d(smem + Lay::OFF_W2 + j * 16384, &tmW2, &misc->w_full, j * 64, seg * 128);
+      }
+      __syncwarp();
+      if (!wait_all(&misc->w_full, ph_w)) return false;
+      ph_w ^= 1;
+      w_pending = false;
+      return true;
+    };
+    auto issue_d1 = [&](long long i) -> bool {
+      const int s = (int)(i & 1);
+      if (!wait_all(&misc->a_full[s], (uint32_t)((i >> 1) & 1))) return false;
+      a_waited = i + 1;
+      if (i >= 2 && !wait_all(&misc->slot_free[s], (uint32_t)(((i >> 1) - 1) & 1))) return false;
+      if (leader) {
+        tc_fence_after();
+        const uint64_t dA = dA0 + (uint64_t)((s * Lay::A_BYTES) >> 4);
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+          for (int kk = 0; kk < R / 16; ++kk) {
+            const uint64_t ko = (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2);
+            mma_ss(tmem + 256 * s + h2 * 128, dA + ko, dW1 + (uint64_t)((h2 * Lay::W1_HALF) >> 4) + ko, IDESC_1,
+                   kk > 0 ? 1u : 0u);
+          }
+        mma_commit(&misc->d1_full[s]);
+        mma_commit(&misc->a_empty[s]);
+      }
+      __syncwarp();
+      return true;
+    };
+    auto issue_d2 = [&](long long i) -> bool {
+      const int s = (int)(i & 1);
+      if (!wait_all(&misc->h_ready[s], (uint32_t)((i >> 1) & 1))) return false;
+      if (leader) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk)
+          mma_ts(tmem + 256 * s + 128, tmem + 256 * s + kk * 8,
+                 dW2 + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), IDESC_2, kk > 0 ? 1u : 0u);
+        mma_commit(&misc->d2_full[s]);
+      }
+      __syncwarp();
+      return true;
+    };
+    auto drain_mmas = [&](volatile int* flag) -> bool {   // every MMA issued so far is complete
+      if (leader) mma_commit(&misc->drain);
+      __syncwarp();
+      const bool r = __all_sync(0xffffffffu, mbar_wait(&misc->drain, ph_drain, flag, err, ERR_TIMEOUT));
+      ph_drain ^= 1;
+      return r;
+    };
+    if (n > 0) {
+      issue_a(0);
+      a_issued = 1;
+      if (n > 1) {
+        issue_a(1);
+        a_issued = 2;
+      }
+      int cur_seg = seg_of(0);
+      ok = load_w(cur_seg) && issue_d1(0);
+      for (long long i = 0; ok && i < n; ++i) {
+        const bool has_next = i + 1 < n;
+        const bool same = has_next && seg_of(i + 1) == cur_seg;
+        if (same && !(ok = issue_d1(i + 1))) break;   // the next tile's pre-activations first
+        if (!(ok = issue_d2(i))) break;
+        if (has_next && !same) {   // a new (layer, KV head): W1', W2 reloaded once no MMA reads them
+          if (!(ok = drain_mmas(abort_flag))) break;
+          cur_seg = seg_of(i + 1);
+          if (!(ok = load_w(cur_seg) && issue_d1(i + 1))) break;
+        }
+        // tile i's stage is free once its pre-activations are done: tile i + 2 goes there
+        if (i + 2 < n) {
+          if (!(ok = wait_all(&misc->a_empty[i & 1], (uint32_t)((i >> 1) & 1)))) break;
+          issue_a(i + 2);
+          a_issued = i + 3;
+        }
+      }
+      // before the CTA's TMEM and shared memory go: every MMA and copy it started is done
+      volatile int never = 0;
+      drain_mmas(&never);
+      if (!ok && leader) {
+        for (long long i = a_waited; i < a_issued; ++i)
+          mbar_wait(&misc->a_full[i & 1], (uint32_t)((i >> 1) & 1), &never, err, ERR_TIMEOUT);
+        if (w_pending) mbar_wait(&misc->w_full, ph_w, &never, err, ERR_TIMEOUT);   // a W1' / W2 copy in flight
+      }
+    }
+  } else {
+    // ============================================================ silu and epilogue
+    const int grp_t = warp >> 2;                       // tiles i with i % 2 == grp_t
+    const int wq = warp & 3;
+    const int t = 32 * wq + lane;                      // this thread's token (TMEM lane)
+    const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (long long i = grp_t; i < n; i += 2) {
+      const long long x = x0 + i;
+      const int s = (int)(i & 1);
+      const uint32_t par = (uint32_t)((i >> 1) & 1);
+      const int u = (int)(x / nC), c = (int)(x % nC);
+      const int b = u % B, seg = u / B, hkv = seg % Hkv, l = seg / Hkv;
+      const size_t unit = ((size_t)b * L + l) * Hkv + hkv;
+      const size_t tok = unit * N + (size_t)c * C;   // the chunk's first token
+      // the token's values row for the epilogue, requested now
+      uint4 vrow[kEncD / 8];
+      const uint4* vp = reinterpret_cast<const uint4*>(values + (tok + t) * kEncD);
+#pragma unroll
+      for (int j = 0; j < kEncD / 8; ++j) vrow[j] = __ldg(vp + j);
+      int flagged = 0, rank = 0;
+      size_t rbase = 0;
+      if (EMIT) {   // the token's rank among the chunk's flagged tokens: one ballot per warp
+        unsigned below = 0;
+#pragma unroll
+        for (int w4 = 0; w4 < 4; ++w4) {
+          const unsigned bw = __ballot_sync(0xffffffffu, flags[tok + 32 * w4 + lane] != 0);
+          if (w4 < wq) below += __popc(bw);
+          if (w4 == wq) {
+            flagged = (bw >> lane) & 1u;
+            below += __popc(bw & lt_mask);
+          }
+        }
+        rank = (int)below;
+        rbase = (size_t)res_ptr[unit * (nC + 1) + c];
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(&misc->d1_full[s], par, abort_flag, err, ERR_TIMEOUT))) break;
+      tc_fence_after();
+      // H = silu(2 D1) for this token's 256 hidden units, as fp16 pairs over columns 0..127
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + 256 * s + 32 * q, v);
+        tmem_wait_ld();
+        uint32_t h[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          h[j] = silu_half2_of_halfx(pack_f16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])));
+        tmem_st16(tmem + lane_off + 256 * s + 16 * q, h);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&misc->h_ready[s]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&misc->d2_full[s], par, abort_flag, err, ERR_TIMEOUT))) break;
+      tc_fence_after();
+      // delta = V - Vhat for this token's 128 dims: its norm (pass 1) or its record (pass 2)
+      float ss = 0.f;
+#pragma unroll
+      for (int q = 0; q < kEncD / 32; ++q) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_off + 256 * s + 128 + 32 * q, v);
+        tmem_wait_ld();
+        uint32_t o[16];
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const uint4 w4 = vrow[(32 * q + j) >> 3];
+          const uint32_t w = ((j >> 1) & 3) == 0 ? w4.x : ((j >> 1) & 3) == 1 ? w4.y : ((j >> 1) & 3) == 2 ? w4.z : w4.w;
+          const float d0 = __uint_as_float(w << 16) - __uint_as_float(v[j]);
+          const float d1 = __uint_as_float(w & 0xffff0000u) - __uint_as_float(v[j + 1]);
+          if (!EMIT) {
+            ss = fmaf(d0, d0, ss);
+            ss = fmaf(d1, d1, ss);
+          } else {
+            const __nv_bfloat162 p = __floats2bfloat162_rn(d0, d1);
+            o[j >> 1] = *reinterpret_cast<const uint32_t*>(&p);
+          }
+        }
+        if (EMIT && flagged) {
+          uint4* dst = reinterpret_cast<uint4*>(res_val + (rbase + rank) * kEncD + 32 * q);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&misc->slot_free[s]);
+      if (!EMIT) norms[tok + t] = sqrtf(ss);
+      if (EMIT && flagged) res_pos[rbase + rank] = (uint16_t)t;
+    }
+  }
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 // ----------------------------------------------------------- tensor-core coefficients
 // Per (b, group, KV head, chunk) tile of 128 tokens: D = sum_{l in group} K_l . B_l^T (SS
 // MMAs, M = 128 tokens, N = R, K = d in steps of 16), the key and basis slabs of layer l+1
@@ -988,6 +1285,26 @@ cudaError_t launch_encode_t(const Geom& g, int n_res, const void* keys, const vo
     if (!w2h_ready)
       to_half_kernel<<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w2), w.w2h, (size_t)lh * kEncD * kEncH);
     const unsigned grid = (unsigned)std::min<size_t>((size_t)n_sm, units * nC);
+    if (C == 128) {   // tokens as the MMAs' M dimension, two tiles in flight
+      using Lay2 = EncTc2Layout<R>;
+      auto t1 = enc_resid_tc2_kernel<R, false>;
+      auto t2 = enc_resid_tc2_kernel<R, true>;
+      if ((e = cudaFuncSetAttribute(t1, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay2::SMEM)) != cudaSuccess) return e;
+      if ((e = cudaFuncSetAttribute(t2, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay2::SMEM)) != cudaSuccess) return e;
+      t1<<<grid, kEnc2Threads, Lay2::SMEM, s>>>(g.B, g.L, g.G, g.Hkv, g.N, tmW1, tmW2, tmA,
+                                               static_cast<const __nv_bfloat16*>(values), w.norms, nullptr, nullptr,
+                                               nullptr, nullptr, w.err);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      enc_select_kernel<<<(unsigned)units, kSelThreads, (size_t)nC * sizeof(int), s>>>(g.N, C, n_res, w.norms,
+                                                                                       w.flags, dst.res_ptr);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      if (n_res > 0)
+        t2<<<grid, kEnc2Threads, Lay2::SMEM, s>>>(g.B, g.L, g.G, g.Hkv, g.N, tmW1, tmW2, tmA,
+                                                 static_cast<const __nv_bfloat16*>(values), w.norms, w.flags,
+                                                 dst.res_ptr, dst.res_pos, static_cast<__nv_bfloat16*>(dst.res_val),
+                                                 w.err);
+      return cudaGetLastError();
+    }
     auto k1 = enc_resid_tc_kernel<R, C, false>;
     auto k2 = enc_resid_tc_kernel<R, C, true>;
     if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM)) != cudaSuccess) return e;
