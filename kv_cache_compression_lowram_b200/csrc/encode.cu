@@ -943,16 +943,23 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
       if (!__all_sync(0xffffffffu, mbar_wait(&misc->d1_full[s], par, abort_flag, err, ERR_TIMEOUT))) break;
       tc_fence_after();
       // H = silu(2 D1) for this token's 256 hidden units, as fp16 pairs over columns 0..127
+      // (64 columns per TMEM round trip; the writes of a pair of chunks land on columns both
+      // chunks have already been read from)
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        uint32_t v[32];
+      for (int q = 0; q < 8; q += 2) {
+        uint32_t v[32], v2[32];
         tmem_ld32(tmem + lane_off + 256 * s + 32 * q, v);
+        tmem_ld32(tmem + lane_off + 256 * s + 32 * q + 32, v2);
         tmem_wait_ld();
         uint32_t h[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           h[j] = silu_half2_of_halfx(pack_f16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])));
         tmem_st16(tmem + lane_off + 256 * s + 16 * q, h);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          h[j] = silu_half2_of_halfx(pack_f16x2(__uint_as_float(v2[2 * j]), __uint_as_float(v2[2 * j + 1])));
+        tmem_st16(tmem + lane_off + 256 * s + 16 * q + 16, h);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -962,11 +969,14 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
       tc_fence_after();
       // delta = V - Vhat for this token's 128 dims: its norm (pass 1) or its record (pass 2)
       float ss = 0.f;
+      uint32_t vd[kEncD];   // the token's rebuilt row, all of it in one TMEM round trip
+#pragma unroll
+      for (int q = 0; q < kEncD / 32; ++q)
+        tmem_ld32(tmem + lane_off + 256 * s + 128 + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(vd + 32 * q));
+      tmem_wait_ld();
 #pragma unroll
       for (int q = 0; q < kEncD / 32; ++q) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + 256 * s + 128 + 32 * q, v);
-        tmem_wait_ld();
+        const uint32_t* v = vd + 32 * q;
         uint32_t o[16];
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
