@@ -1256,6 +1256,282 @@ EncWs carve(const Geom& g, void* workspace, size_t* bytes, bool folds_given) {
   return w;
 }
 
+// -------------------------------------- tensor-core coefficients, bases resident (G <= 4)
+// The same projection with the group's G bases kept in shared memory for as long as the
+// tiles share their (group, KV head), a ring of KST key stages fed ahead of the MMAs, and two
+// TMEM accumulators, so that a tile's epilogue (warps 0-3: thread = token row; its stored
+// row, and the chunk summary as butterfly sums over the warp plus shared-memory atomics over
+// the four warps) overlaps the next tile's MMAs (issued by warp 4).
+template <int R>
+struct EncCoeff2Layout {
+  static constexpr int KST = 3;
+  static constexpr int K_BYTES = 2 * 16384;   // 128 tokens x 128 dims, two 64-dim slabs
+  static constexpr int B_BYTES = 2 * R * 128;  // R basis rows x 128 dims, two slabs
+  static constexpr int OFF_B = 0;              // bases of the group's layers (up to 4)
+  static constexpr int OFF_K = OFF_B + 4 * B_BYTES;
+  static constexpr int OFF_RED = OFF_K + KST * K_BYTES;   // float [R]: the summary's sums
+  static constexpr int OFF_MISC = OFF_RED + R * 4;
+  static constexpr int SMEM = OFF_MISC + 192 + 1024;
+  static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+struct EncCoeff2Misc {
+  uint64_t b_full, drain, k_full[4], k_empty[4], d_full[2], acc_free[2];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// every thread of the 128-thread named barrier `id` learns whether all of them passed `p`
+__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred a, b;\n\t"
+      "setp.ne.u32 a, %1, 0;\n\t"
+      "bar.red.and.pred b, %2, %3, a;\n\t"
+      "selp.u32 %0, 1, 0, b;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)p), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
+template <int R, bool I8>
+__global__ void __launch_bounds__(160, 1)
+enc_coeff_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmB, void* __restrict__ coeff,
+                     __half* __restrict__ coeff_scale, __nv_bfloat16* __restrict__ summary, uint32_t* err) {
+  using namespace tc;
+  using Lay = EncCoeff2Layout<R>;
+  constexpr int C = 128, KST = Lay::KST;
+  extern __shared__ unsigned char encc2_smem_dyn[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(encc2_smem_dyn) + 1023) & ~uintptr_t(1023));
+  EncCoeff2Misc* misc = reinterpret_cast<EncCoeff2Misc*>(smem + Lay::OFF_MISC);
+  float* red = reinterpret_cast<float*>(smem + Lay::OFF_RED);
+  volatile int* abort_flag = &misc->abort_flag;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nC = N / C, NG = L / G;
+  const long long total = (long long)B * NG * Hkv * nC;
+  const long long x0 = total * blockIdx.x / gridDim.x, x1 = total * (blockIdx.x + 1) / gridDim.x;
+  const long long ntile = x1 - x0;
+  if (tid == 0) {
+    mbar_init(&misc->b_full, 1);
+    mbar_init(&misc->drain, 1);
+    for (int s = 0; s < KST; ++s) {
+      mbar_init(&misc->k_full[s], 1);
+      mbar_init(&misc->k_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&misc->d_full[s], 1);
+      mbar_init(&misc->acc_free[s], 4);
+    }
+    misc->abort_flag = 0;
+    mbar_init_fence();
+  }
+  for (int r = tid; r < R; r += blockDim.x) red[r] = 0.f;
+  if (warp == 4) {
+    tmem_alloc(&misc->tmem_base, 2 * R);
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc->tmem_base;
+  // tile x -> (b, group, KV head, chunk), chunk fastest
+  auto tile_of = [&](long long x, int& b, int& grp, int& hkv, int& c) {
+    c = (int)(x % nC);
+    const long long y = x / nC;
+    hkv = (int)(y % Hkv);
+    grp = (int)((y / Hkv) % NG);
+    b = (int)(y / ((long long)Hkv * NG));
+  };
+
+  if (warp == 4) {
+    // ============================================================ copies and MMAs
+    const bool leader = elect_one();
+    constexpr uint32_t IDESC = idesc_f16(128, R, 1, 1);   // keys (bf16) x basis (bf16), both K-major
+    const long long jobs = ntile * G;                     // job j: tile j / G, layer j % G
+    auto wait_all = [&](uint64_t* bar, uint32_t par, volatile int* flag) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, par, flag, err, ERR_TIMEOUT));
+    };
+    auto issue_k = [&](long long j) {
+      int b, grp, hkv, c;
+      tile_of(x0 + j / G, b, grp, hkv, c);
+      const int l = grp * G + (int)(j % G);
+      const int st = (int)(j % KST);
+      const int krow = (int)((((long long)b * L + l) * Hkv + hkv) * N + (long long)c * C);
+      if (leader) {
+        mbar_expect_tx(&misc->k_full[st], (uint32_t)Lay::K_BYTES);
+        for (int ks = 0; ks < 2; ++ks)
+          tma_load_2d(smem + Lay::OFF_K + st * Lay::K_BYTES + ks * 16384, &tmK, &misc->k_full[st], ks * 64, krow);
+      }
+      __syncwarp();
+    };
+    uint32_t ph_b = 0, ph_d = 0;
+    bool ok = true, b_pending = false;
+    long long k_issued = 0, k_waited = 0;
+    auto load_b = [&](long long i) -> bool {   // the bases of tile i's group layers and KV head
+      int b, grp, hkv, c;
+      tile_of(x0 + i, b, grp, hkv, c);
+      b_pending = true;
+      if (leader) {
+        mbar_expect_tx(&misc->b_full, (uint32_t)(G * Lay::B_BYTES));
+        for (int li = 0; li < G; ++li)
+          for (int ks = 0; ks < 2; ++ks)
+            tma_load_2d(smem + Lay::OFF_B + li * Lay::B_BYTES + ks * R * 128, &tmB, &misc->b_full, ks * 64,
+                        ((grp * G + li) * Hkv + hkv) * R);
+      }
+      __syncwarp();
+      if (!wait_all(&misc->b_full, ph_b, abort_flag)) return false;
+      ph_b ^= 1;
+      b_pending = false;
+      return true;
+    };
+    auto bseg = [&](long long i) {
+      int b, grp, hkv, c;
+      tile_of(x0 + i, b, grp, hkv, c);
+      return grp * Hkv + hkv;
+    };
+    auto drain = [&](volatile int* flag) -> bool {
+      if (leader) mma_commit(&misc->drain);
+      __syncwarp();
+      const bool r = wait_all(&misc->drain, ph_d, flag);
+      ph_d ^= 1;
+      return r;
+    };
+    if (jobs > 0) {
+      for (long long j = 0; j < KST && j < jobs; ++j) issue_k(j);
+      k_issued = jobs < KST ? jobs : KST;
+      int cur_b = bseg(0);
+      ok = load_b(0);
+      for (long long j = 0; ok && j < jobs; ++j) {
+        const long long i = j / G;
+        const int li = (int)(j % G), st = (int)(j % KST), acc = (int)(i & 1);
+        if (li == 0 && i > 0 && bseg(i) != cur_b) {   // a new (group, KV head): its bases
+          if (!(ok = drain(abort_flag))) break;
+          cur_b = bseg(i);
+          if (!(ok = load_b(i))) break;
+        }
+        if (!(ok = wait_all(&misc->k_full[st], (uint32_t)((j / KST) & 1), abort_flag))) break;
+        k_waited = j + 1;
+        if (li == 0 && i >= 2 && !(ok = wait_all(&misc->acc_free[acc], (uint32_t)(((i >> 1) - 1) & 1), abort_flag)))
+          break;
+        if (leader) {
+          tc_fence_after();
+          const uint64_t dK = smem_desc(smem_u32(smem + Lay::OFF_K + st * Lay::K_BYTES), 16, 1024, 2);
+          const uint64_t dB = smem_desc(smem_u32(smem + Lay::OFF_B + li * Lay::B_BYTES), 16, 1024, 2);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const int ks = kk >> 2;
+            mma_ss(tmem + acc * R, dK + (uint64_t)((ks * 16384 + (kk & 3) * 32) >> 4),
+                   dB + (uint64_t)((ks * R * 128 + (kk & 3) * 32) >> 4), IDESC, (li > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&misc->k_empty[st]);
+          if (li == G - 1) mma_commit(&misc->d_full[acc]);
+        }
+        __syncwarp();
+        // the stage of job j - 1 (its MMAs are done or nearly so) takes job j - 1 + KST
+        const long long jr = j - 1 + KST;
+        if (j >= 1 && jr < jobs) {
+          const long long jp = j - 1;
+          if (!(ok = wait_all(&misc->k_empty[jp % KST], (uint32_t)((jp / KST) & 1), abort_flag))) break;
+          issue_k(jr);
+          k_issued = jr + 1;
+        }
+      }
+      volatile int never = 0;
+      drain(&never);   // every MMA done before TMEM goes
+      if (!ok && leader) {
+        for (long long j = k_waited; j < k_issued; ++j)
+          mbar_wait(&misc->k_full[j % KST], (uint32_t)((j / KST) & 1), &never, err, ERR_TIMEOUT);
+        if (b_pending) mbar_wait(&misc->b_full, ph_b, &never, err, ERR_TIMEOUT);
+      }
+    }
+  } else {
+    // ============================================================ epilogue (thread = token)
+    const int t = tid;
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const float inv_g = 1.f / (float)G;
+    for (long long i = 0; i < ntile; ++i) {
+      const int acc = (int)(i & 1);
+      bool ok = mbar_wait(&misc->d_full[acc], (uint32_t)((i >> 1) & 1), abort_flag, err, ERR_TIMEOUT);
+      if (!named_bar_and(1, 128, ok)) break;   // the four warps leave together
+      tc_fence_after();
+      int b, grp, hkv, c;
+      tile_of(x0 + i, b, grp, hkv, c);
+      const size_t row0 = (((size_t)b * NG + grp) * Hkv + hkv) * N + (size_t)c * C;
+      const uint32_t tacc = tmem + lane_off + acc * R;
+      float amax = 0.f;
+      if (I8) {   // the row's largest |a| first
+#pragma unroll
+        for (int q = 0; q < R / 32; ++q) {
+          uint32_t v[32];
+          tmem_ld32(tacc + q * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) amax = fmaxf(amax, fabsf(__uint_as_float(v[k]) * inv_g));
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < R / 32; ++q) {
+        uint32_t v[32];
+        tmem_ld32(tacc + q * 32, v);
+        tmem_wait_ld();
+        float dq[32];   // the stored (dequantised) values of columns 32q .. 32q + 31
+#pragma unroll
+        for (int k8 = 0; k8 < 4; ++k8) {
+          float x8[8];
+#pragma unroll
+          for (int k = 0; k < 8; ++k) x8[k] = __uint_as_float(v[k8 * 8 + k]) * inv_g;
+          const int col = q * 32 + k8 * 8;
+          if (I8) {
+            __half sh;
+            uint2 codes;
+            quantize8(x8, amax, &sh, &codes, dq + k8 * 8);
+            *reinterpret_cast<uint2*>(static_cast<int8_t*>(coeff) + (row0 + t) * R + col) = codes;
+            if (col == 0) coeff_scale[row0 + t] = sh;
+          } else {
+            const uint4 p = pack_bf16x8(x8);
+            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(coeff) + (row0 + t) * R + col) = p;
+            const uint32_t pw[4] = {p.x, p.y, p.z, p.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              dq[k8 * 8 + 2 * h] = __uint_as_float(pw[h] << 16);
+              dq[k8 * 8 + 2 * h + 1] = __uint_as_float(pw[h] & 0xffff0000u);
+            }
+          }
+        }
+        // sums over the warp's 32 tokens (transposing butterfly: lane L ends with column
+        // 32q + L), then over the four warps in shared memory
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+          const bool up = (lane & o) != 0;
+#pragma unroll
+          for (int k = 0; k < o; ++k) {
+            const float keep = up ? dq[k + o] : dq[k];
+            const float give = up ? dq[k] : dq[k + o];
+            dq[k] = keep + __shfl_xor_sync(0xffffffffu, give, o);
+          }
+        }
+        atomicAdd(red + q * 32 + lane, dq[0]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&misc->acc_free[acc]);
+      named_bar_sync(1, 128);   // every warp's sums are in
+      for (int r = t; r < R; r += 128) {
+        summary[((((size_t)b * NG + grp) * Hkv + hkv) * nC + c) * R + r] = __float2bfloat16_rn(red[r] / (float)C);
+        red[r] = 0.f;
+      }
+      named_bar_sync(1, 128);   // the sums are reset before the next tile adds to them
+    }
+  }
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * R);
+  }
+}
+
 template <int R, int C, bool I8>
 cudaError_t launch_encode_t(const Geom& g, int n_res, const void* keys, const void* values,
                             const void* basis, const void* w2, const lowram_encode_dst& dst, const EncWs& w,
@@ -1273,12 +1549,23 @@ cudaError_t launch_encode_t(const Geom& g, int n_res, const void* keys, const vo
     if (!enc_make_map(&tmK, keys, kEncD, (uint64_t)g.B * g.L * g.Hkv * g.N, 128) ||
         !enc_make_map(&tmB, basis, kEncD, (uint64_t)g.L * g.Hkv * R, R))
       return cudaErrorInvalidValue;
-    auto kc = enc_coeff_tc_kernel<R, I8>;
-    if ((e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, CL::SMEM)) != cudaSuccess) return e;
     const unsigned cgrid = (unsigned)std::min<size_t>((size_t)n_sm, (size_t)g.B * NG * g.Hkv * nC);
-    kc<<<cgrid, 128, CL::SMEM, s>>>(g.B, g.L, g.G, g.Hkv, g.N, tmK, tmB, dst.coeff,
-                                    static_cast<__half*>(dst.coeff_scale), static_cast<__nv_bfloat16*>(dst.summary),
-                                    w.err);
+    if (g.G <= 4) {   // the group's bases resident, keys streamed, two accumulators
+      using CL2 = EncCoeff2Layout<R>;
+      auto kc = enc_coeff_tc2_kernel<R, I8>;
+      if ((e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, CL2::SMEM)) != cudaSuccess)
+        return e;
+      kc<<<cgrid, 160, CL2::SMEM, s>>>(g.B, g.L, g.G, g.Hkv, g.N, tmK, tmB, dst.coeff,
+                                       static_cast<__half*>(dst.coeff_scale),
+                                       static_cast<__nv_bfloat16*>(dst.summary), w.err);
+    } else {
+      auto kc = enc_coeff_tc_kernel<R, I8>;
+      if ((e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, CL::SMEM)) != cudaSuccess)
+        return e;
+      kc<<<cgrid, 128, CL::SMEM, s>>>(g.B, g.L, g.G, g.Hkv, g.N, tmK, tmB, dst.coeff,
+                                      static_cast<__half*>(dst.coeff_scale),
+                                      static_cast<__nv_bfloat16*>(dst.summary), w.err);
+    }
   } else {
     enc_coeff_kernel<R, C, I8><<<gc, kEncThreads, 0, s>>>(
         g.L, g.G, g.Hkv, g.N, static_cast<const __nv_bfloat16*>(keys), static_cast<const __nv_bfloat16*>(basis),
