@@ -919,11 +919,6 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
       const int b = u % B, seg = u / B, hkv = seg % Hkv, l = seg / Hkv;
       const size_t unit = ((size_t)b * L + l) * Hkv + hkv;
       const size_t tok = unit * N + (size_t)c * C;   // the chunk's first token
-      // the token's values row for the epilogue, requested now
-      uint4 vrow[kEncD / 8];
-      const uint4* vp = reinterpret_cast<const uint4*>(values + (tok + t) * kEncD);
-#pragma unroll
-      for (int j = 0; j < kEncD / 8; ++j) vrow[j] = __ldg(vp + j);
       int flagged = 0, rank = 0;
       size_t rbase = 0;
       if (EMIT) {   // the token's rank among the chunk's flagged tokens: one ballot per warp
@@ -940,6 +935,11 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
         rank = (int)below;
         rbase = (size_t)res_ptr[unit * (nC + 1) + c];
       }
+      // the token's values row for the epilogue, requested now (pass 2: flagged tokens only)
+      uint4 vrow[kEncD / 8];
+      const uint4* vp = reinterpret_cast<const uint4*>(values + (tok + t) * kEncD);
+#pragma unroll
+      for (int j = 0; j < kEncD / 8; ++j) vrow[j] = (!EMIT || flagged) ? __ldg(vp + j) : make_uint4(0, 0, 0, 0);
       if (!__all_sync(0xffffffffu, mbar_wait(&misc->d1_full[s], par, abort_flag, err, ERR_TIMEOUT))) break;
       tc_fence_after();
       // H = silu(2 D1) for this token's 256 hidden units, as fp16 pairs over columns 0..127
