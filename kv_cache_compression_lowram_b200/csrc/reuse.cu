@@ -286,266 +286,286 @@ reuse_hit_kernel(Geom g, CacheBuffers cb, Scratch sc, ReuseDev st) {
     }
 }
 
-// ------------------------------------------------------------------------------- fills
+// -------------------------------------------------------------------------------- fills
 // Persistent CTAs over the first n_fill tiles of the miss list; tile x goes to entry
-// (ring + x) mod E.  Per tile, like the encoder's predictor pass: the coefficient tile by TMA,
-// D1_hh = (W1'_hh / 2) A^T (SS, M = 128 hidden rows, N = C tokens), H = silu(2 D1) as fp16 in
-// shared memory (MN-major), D2 = W2 H (SS, M = 128 value dims, N = C), then vhat = D2 plus the
-// chunk's residual rows, assembled as bf16 [C][d] in shared memory and written to the entry
-// by one bulk copy.  Latency hiding within the CTA: the residual rows are staged by cp.async
-// while the MMAs run; the next tile's coefficient tile (and W1', W2 at a new (layer, KV head))
-// are requested as soon as the current tile's MMAs are done, i.e. during its epilogue; the
-// next tile's unit, slot and record range are read one tile ahead.
-constexpr int kFillResStage = 32;   // residual rows of a chunk staged in shared memory
+// (ring + x) mod E.  Per tile, with the chunk's 128 tokens as the MMAs' M dimension:
+//   D1^T = A . (W1'/2)^T (SS, M = 128 tokens, N = 128 per hidden half, K = r)
+//   H^T  = silu(2 D1^T) as fp16 pairs over the first 128 of the tile's TMEM columns
+//   D2^T = H^T . W2^T    (TS: A = H from TMEM, B = W2 in fp16; N = 128 value dims, K = 256)
+// then each thread (one token) adds its residual row, if the token has one, and writes its
+// 256-byte row of the entry.  Two tiles in flight: tile i of the CTA's range uses TMEM
+// columns [256 (i%2), +256) and coefficient stage i%2; warps 0-3 take the even tiles, 4-7
+// the odd ones; warp 8 issues the copies and the MMAs.
+constexpr int kFillThreads = 288;
 
 template <int R>
 struct FillLayout {
   static constexpr int KSLABS = R / 64;
   static constexpr int W1_HALF = KSLABS * 16384;
   static constexpr int W2_BYTES = 4 * 16384;
-  static constexpr int H_HALF = 2 * 16384;                   // 128 hidden rows x 128 tokens, fp16
   static constexpr int A_BYTES = KSLABS * 16384;
   static constexpr int OFF_W1 = 0;
   static constexpr int OFF_W2 = OFF_W1 + 2 * W1_HALF;
-  static constexpr int OFF_AH = OFF_W2 + W2_BYTES;           // the A tile, then H half 0
-  static constexpr int OFF_H1 = OFF_AH + (A_BYTES > H_HALF ? A_BYTES : H_HALF);   // H half 1, then vhat
-  static constexpr int OFF_RES = OFF_H1 + H_HALF;            // bf16 [kFillResStage][d]
-  static constexpr int OFF_MISC = OFF_RES + kFillResStage * kD * 2;
-  static constexpr int SMEM = OFF_MISC + 64 + kC * 4 + 1024;
-  static_assert(kC * kD * 2 <= H_HALF, "vhat tile fits the H half-1 buffer");
+  static constexpr int OFF_A = OFF_W2 + W2_BYTES;   // two stages
+  static constexpr int OFF_MISC = OFF_A + 2 * A_BYTES;
+  static constexpr int SMEM = OFF_MISC + 256 + 1024;
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
+struct FillMisc {
+  uint64_t w_full, drain, a_full[2], a_empty[2], d1_full[2], h_ready[2], d2_full[2], slot_free[2];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
 template <int R>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kFillThreads, 1)
 reuse_fill_kernel(Geom g, CacheBuffers cb, Scratch sc, ReuseDev st, const __grid_constant__ CUtensorMap tmW1,
                   const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmA) {
   using Lay = FillLayout<R>;
   extern __shared__ unsigned char fill_smem_dyn[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(fill_smem_dyn) + 1023) & ~uintptr_t(1023));
-  uint64_t* bar_w = reinterpret_cast<uint64_t*>(smem + Lay::OFF_MISC);
-  uint64_t* bar_in = bar_w + 1;
-  uint64_t* bar_mma = bar_w + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_w + 3);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* tok_rec = reinterpret_cast<int*>(smem + Lay::OFF_MISC + 64);   // [C]: token -> record, or -1
-  const __nv_bfloat16* res_s = reinterpret_cast<const __nv_bfloat16*>(smem + Lay::OFF_RES);
-  __nv_bfloat16* out_s = reinterpret_cast<__nv_bfloat16*>(smem + Lay::OFF_H1);
+  FillMisc* misc = reinterpret_cast<FillMisc*>(smem + Lay::OFF_MISC);
+  volatile int* abort_flag = &misc->abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int NG = g.L / g.G;
   const long long n_fill = min((long long)*sc.tile_total, (long long)st.fill_cap);
   const long long x0 = n_fill * blockIdx.x / gridDim.x, x1 = n_fill * (blockIdx.x + 1) / gridDim.x;
+  const long long n = x1 - x0;
   const int ring = *st.ring;
   uint32_t* err = sc.err;
-  const __nv_bfloat16* rv = reinterpret_cast<const __nv_bfloat16*>(cb.res_val);
   if (tid == 0) {
-    mbar_init(bar_w, 1);
-    mbar_init(bar_in, 1);
-    mbar_init(bar_mma, 1);
-    *abort_flag = 0;
+    mbar_init(&misc->w_full, 1);
+    mbar_init(&misc->drain, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&misc->a_full[s], 1);
+      mbar_init(&misc->a_empty[s], 1);
+      mbar_init(&misc->d1_full[s], 1);
+      mbar_init(&misc->h_ready[s], 4);
+      mbar_init(&misc->d2_full[s], 1);
+      mbar_init(&misc->slot_free[s], 4);
+    }
+    misc->abort_flag = 0;
     mbar_init_fence();
   }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, 512);
+  if (warp == 8) {
+    tmem_alloc(&misc->tmem_base, 512);
     tc_fence_before();
   }
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-  const uint64_t dW1 = smem_desc(smem_u32(smem + Lay::OFF_W1), 16, 1024, 2);
-  const uint64_t dW2 = smem_desc(smem_u32(smem + Lay::OFF_W2), 16, 1024, 2);
-  const uint64_t dA = smem_desc(smem_u32(smem + Lay::OFF_AH), 16, 1024, 2);
-  const uint64_t dH0 = smem_desc(smem_u32(smem + Lay::OFF_AH), 16384, 1024, 2);   // MN-major
-  const uint64_t dH1 = smem_desc(smem_u32(smem + Lay::OFF_H1), 16384, 1024, 2);
-  constexpr uint32_t IDESC_1 = idesc_f16(128, kC, 1, 1);         // W1'/2 (bf16) x A (bf16)
-  constexpr uint32_t IDESC_2 = idesc_f16(128, kC, 0, 0, 0, 1);   // W2 (f16) x H (f16, MN-major)
-  uint32_t ph_w = 0, ph_in = 0, ph_mma = 0;
-  bool w_pending = false, a_pending = false;   // copies requested and not yet waited for
-  bool m_pending = false;                      // MMAs committed and not yet waited for
-  int cur_seg = -1;
-  bool ok = true;
-  const int hh = warp >> 2;                 // silu: hidden half; epilogue: token half
-  const int row = 32 * (warp & 3) + lane;   // TMEM lane: hidden unit in the half / value dim
+  const uint32_t tmem = misc->tmem_base;
 
-  // tile x's unit, slot, (layer, KV head) and record range
-  struct TileRef {
-    int u, slot, seg, r0, r1;
-    long long arow;
-  };
-  auto tile_ref = [&](long long x) {
-    TileRef t;
-    t.u = sc.tile_unit[x];
-    t.slot = sc.tile_slot[x];
-    const Unit un = unit_of(g, t.u);
-    const int l = g.layer0 + un.li, grp = l / g.G;
-    t.seg = l * g.Hkv + un.hkv;
-    t.arow = ((((long long)un.b * NG + grp) * g.Hkv + un.hkv) * g.nLs + t.slot) * kC;
-    const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nLs + 1);
-    t.r0 = rptr[t.slot];
-    t.r1 = rptr[t.slot + 1];
-    return t;
-  };
-  // tid 0, once no MMA reads the buffers: the copies of tile t (W1', W2 only at a new pair)
-  auto issue_loads = [&](const TileRef& t, int seg_now) {
-    if (t.seg != seg_now) {
-      mbar_expect_tx(bar_w, (uint32_t)(2 * Lay::W1_HALF + Lay::W2_BYTES));
-      for (int h2 = 0; h2 < 2; ++h2)
+  if (warp == 8) {
+    // ============================================================ copies and MMAs
+    const bool leader = elect_one();
+    const uint64_t dW1 = smem_desc(smem_u32(smem + Lay::OFF_W1), 16, 1024, 2);
+    const uint64_t dW2 = smem_desc(smem_u32(smem + Lay::OFF_W2), 16, 1024, 2);
+    const uint64_t dA0 = smem_desc(smem_u32(smem + Lay::OFF_A), 16, 1024, 2);
+    constexpr uint32_t IDESC_1 = idesc_f16(128, 128, 1, 1);   // A (bf16) x W1'/2 (bf16), both K-major
+    constexpr uint32_t IDESC_2 = idesc_f16(128, 128, 0, 0);   // H (TMEM, fp16) x W2 (fp16, K-major)
+    auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, par, abort_flag, err, ERR_TIMEOUT));
+    };
+    auto seg_of = [&](long long i) {
+      const Unit un = unit_of(g, sc.tile_unit[x0 + i]);
+      return (g.layer0 + un.li) * g.Hkv + un.hkv;
+    };
+    auto issue_a = [&](long long i) {   // tile i's coefficient tile into stage i % 2
+      const int u = sc.tile_unit[x0 + i], slot = sc.tile_slot[x0 + i];
+      const Unit un = unit_of(g, u);
+      const int grp = (g.layer0 + un.li) / g.G;
+      const long long arow = ((((long long)un.b * NG + grp) * g.Hkv + un.hkv) * g.nLs + slot) * kC;
+      if (leader) {
+        mbar_expect_tx(&misc->a_full[i & 1], (uint32_t)Lay::A_BYTES);
         for (int ks = 0; ks < Lay::KSLABS; ++ks)
-          tma_load_2d(smem + Lay::OFF_W1 + h2 * Lay::W1_HALF + ks * 16384, &tmW1, bar_w, ks * 64, t.seg * kH + h2 * 128);
-      for (int j = 0; j < 4; ++j) tma_load_2d(smem + Lay::OFF_W2 + j * 16384, &tmW2, bar_w, j * 64, t.seg * kD);
-    }
-    mbar_expect_tx(bar_in, (uint32_t)(Lay::KSLABS * kC * 128));
-    for (int ks = 0; ks < Lay::KSLABS; ++ks)
-      tma_load_2d(smem + Lay::OFF_AH + ks * 16384, &tmA, bar_in, ks * 64, (int)t.arow);
-  };
-
-  TileRef cur{};
-  if (x0 < x1) {
-    cur = tile_ref(x0);
-    if (tid == 0) issue_loads(cur, -1);
-  }
-  for (long long x = x0; ok && x < x1; ++x) {
-    // this tile's copies were issued (before the loop, or during the last tile's epilogue)
-    const bool new_seg = cur.seg != cur_seg;
-    w_pending = w_pending || new_seg;
-    a_pending = true;
-    cur_seg = cur.seg;
-    int r0 = cur.r0, r1 = cur.r1;
-    if (r0 < 0 || r1 < r0 || (long long)r1 > (long long)cb.n_records) {
-      if (tid == 0) atomicOr(err, ERR_RES_PTR);
-      r0 = r1 = 0;
-    }
-    // residual rows r0 .. r0 + 31 into shared memory (cp.async), and the token -> record map
-    const int nst = min(r1 - r0, kFillResStage);
-    for (int i = tid; i < nst * (kD / 8); i += 256) {
-      const int rr = i / (kD / 8), c = i % (kD / 8);
-      cp16(smem + Lay::OFF_RES + (rr * kD + c * 8) * 2, rv + (size_t)(r0 + rr) * kD + c * 8);
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    for (int t = tid; t < kC; t += 256) tok_rec[t] = -1;   // filled once the MMAs are issued
-    // (a phase flips only once every thread has passed its wait, so that the drain below
-    // waits for the phase a failed wait was on)
-    if (new_seg) {
-      ok = mbar_wait(bar_w, ph_w, abort_flag, err, ERR_TIMEOUT);
-      if (!__syncthreads_and(ok)) break;
+          tma_load_2d(smem + Lay::OFF_A + (i & 1) * Lay::A_BYTES + ks * 16384, &tmA, &misc->a_full[i & 1], ks * 64,
+                      (int)arow);
+      }
+      __syncwarp();
+    };
+    uint32_t ph_w = 0, ph_drain = 0;
+    long long a_waited = 0, a_issued = 0;
+    bool ok = true, w_pending = false;
+    auto load_w = [&](int seg) -> bool {   // W1' halves and W2 of this (layer, KV head)
+      w_pending = true;
+      if (leader) {
+        mbar_expect_tx(&misc->w_full, (uint32_t)(2 * Lay::W1_HALF + Lay::W2_BYTES));
+        for (int h2 = 0; h2 < 2; ++h2)
+          for (int ks = 0; ks < Lay::KSLABS; ++ks)
+            tma_load_2d(smem + Lay::OFF_W1 + h2 * Lay::W1_HALF + ks * 16384, &tmW1, &misc->w_full, ks * 64,
+                        seg * kH + h2 * 128);
+        for (int j = 0; j < 4; ++j) tma_load_2d(smem + Lay::OFF_W2 + j * 16384, &tmW2, &misc->w_full, j * 64, seg * kD);
+      }
+      __syncwarp();
+      if (!wait_all(&misc->w_full, ph_w)) return false;
       ph_w ^= 1;
       w_pending = false;
+      return true;
+    };
+    auto issue_d1 = [&](long long i) -> bool {
+      const int s = (int)(i & 1);
+      if (!wait_all(&misc->a_full[s], (uint32_t)((i >> 1) & 1))) return false;
+      a_waited = i + 1;
+      if (i >= 2 && !wait_all(&misc->slot_free[s], (uint32_t)(((i >> 1) - 1) & 1))) return false;
+      if (leader) {
+        tc_fence_after();
+        const uint64_t dA = dA0 + (uint64_t)((s * Lay::A_BYTES) >> 4);
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2)
+#pragma unroll
+          for (int kk = 0; kk < R / 16; ++kk) {
+            const uint64_t ko = (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2);
+            mma_ss(tmem + 256 * s + h2 * 128, dA + ko, dW1 + (uint64_t)((h2 * Lay::W1_HALF) >> 4) + ko, IDESC_1,
+                   kk > 0 ? 1u : 0u);
+          }
+        mma_commit(&misc->d1_full[s]);
+        mma_commit(&misc->a_empty[s]);
+      }
+      __syncwarp();
+      return true;
+    };
+    auto issue_d2 = [&](long long i) -> bool {
+      const int s = (int)(i & 1);
+      if (!wait_all(&misc->h_ready[s], (uint32_t)((i >> 1) & 1))) return false;
+      if (leader) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk)
+          mma_ts(tmem + 256 * s + 128, tmem + 256 * s + kk * 8,
+                 dW2 + (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), IDESC_2, kk > 0 ? 1u : 0u);
+        mma_commit(&misc->d2_full[s]);
+      }
+      __syncwarp();
+      return true;
+    };
+    auto drain_mmas = [&](volatile int* flag) -> bool {
+      if (leader) mma_commit(&misc->drain);
+      __syncwarp();
+      const bool r = __all_sync(0xffffffffu, mbar_wait(&misc->drain, ph_drain, flag, err, ERR_TIMEOUT));
+      ph_drain ^= 1;
+      return r;
+    };
+    if (n > 0) {
+      issue_a(0);
+      a_issued = 1;
+      if (n > 1) {
+        issue_a(1);
+        a_issued = 2;
+      }
+      int cur_seg = seg_of(0);
+      ok = load_w(cur_seg) && issue_d1(0);
+      for (long long i = 0; ok && i < n; ++i) {
+        const bool has_next = i + 1 < n;
+        const int next_seg = has_next ? seg_of(i + 1) : cur_seg;
+        const bool same = has_next && next_seg == cur_seg;
+        if (same && !(ok = issue_d1(i + 1))) break;
+        if (!(ok = issue_d2(i))) break;
+        if (has_next && !same) {
+          if (!(ok = drain_mmas(abort_flag))) break;
+          cur_seg = next_seg;
+          if (!(ok = load_w(cur_seg) && issue_d1(i + 1))) break;
+        }
+        if (i + 2 < n) {
+          if (!(ok = wait_all(&misc->a_empty[i & 1], (uint32_t)((i >> 1) & 1)))) break;
+          issue_a(i + 2);
+          a_issued = i + 3;
+        }
+      }
+      volatile int never = 0;
+      drain_mmas(&never);
+      if (!ok && leader) {
+        for (long long i = a_waited; i < a_issued; ++i)
+          mbar_wait(&misc->a_full[i & 1], (uint32_t)((i >> 1) & 1), &never, err, ERR_TIMEOUT);
+        if (w_pending) mbar_wait(&misc->w_full, ph_w, &never, err, ERR_TIMEOUT);
+      }
     }
-    ok = mbar_wait(bar_in, ph_in, abort_flag, err, ERR_TIMEOUT);
-    if (!__syncthreads_and(ok)) break;
-    ph_in ^= 1;
-    a_pending = false;
-    if (tid == 0) {
+  } else {
+    // ============================================================ silu and epilogue
+    const int grp_t = warp >> 2;
+    const int wq = warp & 3;
+    const int t = 32 * wq + lane;                      // this thread's token (TMEM lane)
+    const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
+    const __nv_bfloat16* rv = reinterpret_cast<const __nv_bfloat16*>(cb.res_val);
+    for (long long i = grp_t; i < n; i += 2) {
+      const long long x = x0 + i;
+      const int s = (int)(i & 1);
+      const uint32_t par = (uint32_t)((i >> 1) & 1);
+      const int u = sc.tile_unit[x], slot = sc.tile_slot[x];
+      const Unit un = unit_of(g, u);
+      const int l = g.layer0 + un.li;
+      // this token's residual record, if it has one (the chunk's few records scanned)
+      const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nLs + 1);
+      int r0 = rptr[slot], r1 = rptr[slot + 1];
+      if (r0 < 0 || r1 < r0 || (long long)r1 > (long long)cb.n_records) {
+        if (t == 0) atomicOr(err, ERR_RES_PTR);
+        r0 = r1 = 0;
+      }
+      int rec = -1;
+      for (int k = r0; k < r1; ++k)
+        if ((int)cb.res_pos[k] == t) rec = k;
+      uint4 drow[kD / 8];
+      const uint4* dp = reinterpret_cast<const uint4*>(rv + (size_t)(rec < 0 ? 0 : rec) * kD);
+#pragma unroll
+      for (int j = 0; j < kD / 8; ++j) drow[j] = rec >= 0 ? __ldg(dp + j) : make_uint4(0, 0, 0, 0);
+      if (!__all_sync(0xffffffffu, mbar_wait(&misc->d1_full[s], par, abort_flag, err, ERR_TIMEOUT))) break;
       tc_fence_after();
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2)
-#pragma unroll
-        for (int kk = 0; kk < R / 16; ++kk) {
-          const uint64_t ko = (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2);
-          mma_ss(tmem + h2 * kC, dW1 + (uint64_t)((h2 * Lay::W1_HALF) >> 4) + ko, dA + ko, IDESC_1, kk > 0 ? 1u : 0u);
-        }
-      mma_commit(bar_mma);
-      bulk_wait_read_all();   // the last tile's vhat (in the H half-1 buffer) has been copied out
-    }
-    // while the pre-activations run: the token -> record map (the barrier above ordered the
-    // reset) and the next tile's reference (both dependent global loads)
-    for (int i = r0 + tid; i < r1; i += 256) {
-      const int pos = cb.res_pos[i];
-      if (pos < kC) tok_rec[pos] = i;
-    }
-    TileRef nxt{};
-    if (x + 1 < x1) nxt = tile_ref(x + 1);
-    m_pending = true;
-    ok = mbar_wait(bar_mma, ph_mma, abort_flag, err, ERR_TIMEOUT);
-    if (!__syncthreads_and(ok)) break;
-    ph_mma ^= 1;
-    m_pending = false;
-    tc_fence_after();
-    {   // silu -> H_hh (fp16) in shared memory, MN-major: hidden row `row`, 8 tokens per 16 bytes
-      unsigned char* hrow = smem + (hh == 0 ? Lay::OFF_AH : Lay::OFF_H1) + (row >> 3) * 1024 + (row & 7) * 128;
-#pragma unroll
-      for (int q = 0; q < kC / 32; ++q) {
-        uint32_t v[32];
-        tmem_ld32(tmem + lane_off + hh * kC + q * 32, v);
+      for (int q = 0; q < 8; q += 2) {
+        uint32_t v[32], v2[32];
+        tmem_ld32(tmem + lane_off + 256 * s + 32 * q, v);
+        tmem_ld32(tmem + lane_off + 256 * s + 32 * q + 32, v2);
         tmem_wait_ld();
-        uint32_t hv[16];
+        uint32_t h[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-          hv[j] = silu_half2_of_halfx(pack_f16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])));
-        unsigned char* blk = hrow + (q >> 1) * 16384;
+          h[j] = silu_half2_of_halfx(pack_f16x2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])));
+        tmem_st16(tmem + lane_off + 256 * s + 16 * q, h);
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          const int c16 = (q & 1) * 4 + k4;
-          *reinterpret_cast<uint4*>(blk + ((c16 ^ (row & 7)) << 4)) =
-              make_uint4(hv[4 * k4], hv[4 * k4 + 1], hv[4 * k4 + 2], hv[4 * k4 + 3]);
-        }
+        for (int j = 0; j < 16; ++j)
+          h[j] = silu_half2_of_halfx(pack_f16x2(__uint_as_float(v2[2 * j]), __uint_as_float(v2[2 * j + 1])));
+        tmem_st16(tmem + lane_off + 256 * s + 16 * q + 16, h);
       }
-    }
-    tc_fence_before();
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {   // D2 = W2 . H over both hidden halves
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&misc->h_ready[s]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&misc->d2_full[s], par, abort_flag, err, ERR_TIMEOUT))) break;
       tc_fence_after();
+      // vhat[t] = D2[t] + delta (if the token has a record), as bf16, straight to the entry,
+      // 64 dims per TMEM round trip
+      uint4* dst = reinterpret_cast<uint4*>(st.entries + ((size_t)((ring + x) % st.E) * kC + t) * kD);
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2)
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const int slab = h2 * 2 + (kk >> 2);
-          mma_ss(tmem + 2 * kC, dW2 + (uint64_t)((slab * 16384 + (kk & 3) * 32) >> 4),
-                 (h2 == 0 ? dH0 : dH1) + (uint64_t)((kk * 2048) >> 4), IDESC_2, (h2 | kk) ? 1u : 0u);
+      for (int hv = 0; hv < 2; ++hv) {
+        uint32_t vd[64];
+        tmem_ld32(tmem + lane_off + 256 * s + 128 + 64 * hv, *reinterpret_cast<uint32_t(*)[32]>(vd));
+        tmem_ld32(tmem + lane_off + 256 * s + 128 + 64 * hv + 32, *reinterpret_cast<uint32_t(*)[32]>(vd + 32));
+        tmem_wait_ld();
+        if (hv == 1) {   // the tile's TMEM is free for its slot's next tile
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&misc->slot_free[s]);
         }
-      mma_commit(bar_mma);
-    }
-    m_pending = true;
-    ok = mbar_wait(bar_mma, ph_mma, abort_flag, err, ERR_TIMEOUT);
-    asm volatile("cp.async.wait_group 0;" ::: "memory");   // this thread's residual rows
-    if (!__syncthreads_and(ok)) break;
-    ph_mma ^= 1;
-    m_pending = false;
-    tc_fence_after();
-    // every MMA of this tile is done: the next tile's copies go out now
-    if (tid == 0 && x + 1 < x1) issue_loads(nxt, cur_seg);
-    // vhat[t][row] = D2[row][t] + delta_t[row] for tokens hh * 64 .. + 63, into shared memory
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      uint32_t v[32];
-      tmem_ld32(tmem + lane_off + 2 * kC + hh * 64 + q * 32, v);
-      tmem_wait_ld();
+        for (int j = 0; j < 8; ++j) {
+          const uint4 dr = drow[8 * hv + j];
+          const uint32_t dw[4] = {dr.x, dr.y, dr.z, dr.w};
+          uint32_t o[4];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int t = hh * 64 + q * 32 + j;
-        float val = __uint_as_float(v[j]);
-        const int ri = tok_rec[t];   // the same for the whole warp
-        if (ri >= 0) {
-          const int si = ri - r0;
-          val += __bfloat162float(si < kFillResStage ? res_s[si * kD + row] : rv[(size_t)ri * kD + row]);
+          for (int k = 0; k < 4; ++k) {
+            const float a = __uint_as_float(vd[8 * j + 2 * k]) + __uint_as_float(dw[k] << 16);
+            const float b = __uint_as_float(vd[8 * j + 2 * k + 1]) + __uint_as_float(dw[k] & 0xffff0000u);
+            const __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
+            o[k] = *reinterpret_cast<const uint32_t*>(&p);
+          }
+          dst[8 * hv + j] = make_uint4(o[0], o[1], o[2], o[3]);
         }
-        out_s[t * kD + row] = __float2bfloat16_rn(val);
       }
     }
-    tc_fence_before();
-    fence_proxy_async_smem();
-    __syncthreads();   // vhat complete; tok_rec and the staged rows are free again
-    if (tid == 0) {
-      bulk_store(st.entries + (size_t)((ring + x) % st.E) * kC * kD, out_s, (uint32_t)(kC * kD * 2));
-      bulk_commit();
-    }
-    cur = nxt;
   }
-  if (tid == 0) {
-    bulk_wait_all();
-    if (!ok) {   // a wait gave up: let the copies this CTA started land before it exits
-      volatile int never = 0;
-      if (w_pending) mbar_wait(bar_w, ph_w, &never, err, ERR_TIMEOUT);
-      if (a_pending) mbar_wait(bar_in, ph_in, &never, err, ERR_TIMEOUT);
-      if (m_pending) mbar_wait(bar_mma, ph_mma, &never, err, ERR_TIMEOUT);   // TMEM is freed below
-    }
-  }
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -630,7 +650,7 @@ cudaError_t run_reuse(const Geom& g, const CacheBuffers& cb, const Scratch& sc, 
     return cudaErrorInvalidValue;
   auto k = reuse_fill_kernel<R>;
   if ((e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::SMEM)) != cudaSuccess) return e;
-  k<<<n_sm, 256, Lay::SMEM, s>>>(g, cb, sc, st, tmW1, tmW2, tmA);
+  k<<<n_sm, kFillThreads, Lay::SMEM, s>>>(g, cb, sc, st, tmW1, tmW2, tmA);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   reuse_commit_kernel<<<(unsigned)std::min<long long>(((long long)g.U * g.k + 255) / 256, 4LL * n_sm), 256, 0, s>>>(g, sc, st);
   return cudaGetLastError();
