@@ -191,6 +191,8 @@ ENC_CASES = [
     ("llama8b_32k_bf16", dict(batch=1, n_layers=4, n_kv_heads=2, n_ctx=1024)),        # r 128, C 128
     ("llama8b_32k_bf16", dict(batch=2, n_layers=4, n_kv_heads=1, n_ctx=512, rank=64)),  # r 64, C 128
     ("llama8b_32k_bf16", dict(batch=1, n_layers=4, n_kv_heads=2, n_ctx=512, chunk=64)),  # r 128, C 64
+    ("llama8b_32k_bf16", dict(batch=2, n_layers=4, n_kv_heads=2, n_ctx=768, group=2)),   # G 2: two bases resident
+    ("llama8b_32k_bf16", dict(batch=1, n_layers=8, n_kv_heads=1, n_ctx=512, group=8)),   # G 8: the one-tile form
 ]
 
 
