@@ -591,10 +591,10 @@ def run_encode(args, ws, rank, local):
     value, ms_total = aggregate_rate(cfg.batch * cfg.n_ctx * steps, start.elapsed_time(end), ws)
     ms_step = ms_total / steps
     flops = encode_flops(cfg)
-    if cfg.store == "native":
-        # the predictor (89 % of the flops) runs on tcgen05 tensor cores in bf16/fp16: the
-        # measured sustained bf16 GEMM rate (a 54 ms call is a long step); fp16 runs at the
-        # same nominal rate
+    if cfg.store == "native" or cfg.chunk == 128:
+        # the projection and the predictor (all but a few % of the flops) run on tcgen05
+        # tensor cores in bf16 / fp16 (int8 stores: the stored rows dequantised to fp16 on
+        # chip): the measured sustained bf16 GEMM rate; fp16 runs at the same nominal rate
         bound, peak, peak_kind = "tensor", tensor_peak_sustained(), "measured (bf16, sustained)"
     else:
         # int8 stores: CUDA-core fp32 kernels; 148 SMs x 128 FMA lanes x 2 flops x the
@@ -610,7 +610,7 @@ def run_encode(args, ws, rank, local):
     return {
         "metric": ENC_METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": ws, "steps": steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.store == "native" else "f32",
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.store == "native" or cfg.chunk == 128 else "f32",
         "data": "synthetic", "impl": "encoder",
         "config": {"workload": cfg.name, "batch": cfg.batch, "n_layers": cfg.n_layers, "n_ctx": cfg.n_ctx,
                    "kv_heads": cfg.n_kv_heads, "rank": cfg.rank, "chunk": cfg.chunk, "store": cfg.store,

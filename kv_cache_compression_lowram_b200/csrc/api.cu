@@ -632,7 +632,7 @@ lowram_status lowram_cache_repack(lowram_cache* c, int32_t n_resid, lowram_strea
   // the cache's own folds of W1 (the encoder would compute the same), and W2 in fp16 kept
   // in the scratch from the previous re-pack
   e = launch_encode(ge, f.store, n_resid, keys, vals, c->cb.basis, c->cb.w1, c->cb.w2, dst, ws, s, c->w1f_t,
-                    i8 ? nullptr : c->w1f_tc, c->up_w2h_ready);
+                    c->w1f_tc, c->up_w2h_ready);
   if (e != cudaSuccess) return cuda_fail(e, "encode the new chunk");
   c->up_w2h_ready = true;
 

@@ -719,36 +719,44 @@ enc_resid_tc_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant__
 // copies and the MMAs, the next tile's pre-activations before this tile's second GEMM.
 constexpr int kEnc2Threads = 288;
 
-template <int R>
+template <int R, bool I8 = false>
 struct EncTc2Layout {
   static constexpr int KSLABS = R / 64;
-  static constexpr int W1_HALF = KSLABS * 16384;          // 128 hidden rows x R, bf16
+  static constexpr int W1_HALF = KSLABS * 16384;          // 128 hidden rows x R, 16-bit
   static constexpr int W2_BYTES = 4 * 16384;              // 128 dims x 256 hidden, fp16
-  static constexpr int A_BYTES = KSLABS * 16384;          // 128 tokens x R, bf16
+  static constexpr int A_BYTES = KSLABS * 16384;          // 128 tokens x R, 16-bit
+  static constexpr int SA_SLOT = 128 * R + 128 * 2;       // int8 store: the int8 tile + row scales
   static constexpr int OFF_W1 = 0;
   static constexpr int OFF_W2 = OFF_W1 + 2 * W1_HALF;
   static constexpr int OFF_A = OFF_W2 + W2_BYTES;         // two stages
-  static constexpr int OFF_MISC = OFF_A + 2 * A_BYTES;
+  static constexpr int OFF_SA = OFF_A + 2 * A_BYTES;      // int8 store: two staging slots
+  static constexpr int OFF_MISC = OFF_SA + (I8 ? 2 * SA_SLOT : 0);
   static constexpr int SMEM = OFF_MISC + 256 + 1024;
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
 struct EncTc2Misc {
-  uint64_t w_full, drain, a_full[2], a_empty[2], d1_full[2], h_ready[2], d2_full[2], slot_free[2];
+  uint64_t w_full, drain, a_full[2], a_empty[2], d1_full[2], h_ready[2], d2_full[2], slot_free[2], a_conv[2];
   uint32_t tmem_base;
   int abort_flag;
 };
 
-template <int R, bool EMIT>
+// I8 (int8 store): the stored int8 rows and their scales arrive by bulk copies into a staging
+// slot, and each thread of the tile's group writes its own token's row sigma_t a_t as fp16
+// (int8 times the fp16 scale is exact in fp32, rounded once) into the coefficient stage the
+// MMAs read; W1'/2 is then fp16 too, and the residual record is the int8 row with its scale.
+template <int R, bool EMIT, bool I8 = false>
 __global__ void __launch_bounds__(kEnc2Threads, 1)
 enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant__ CUtensorMap tmW1,
                      const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmA,
+                     const void* __restrict__ coeff, const __half* __restrict__ coeff_scale,
                      const __nv_bfloat16* __restrict__ values, float* __restrict__ norms,
                      const uint8_t* __restrict__ flags, const int32_t* __restrict__ res_ptr,
-                     uint16_t* __restrict__ res_pos, __nv_bfloat16* __restrict__ res_val, uint32_t* err) {
+                     uint16_t* __restrict__ res_pos, void* __restrict__ res_val, __half* __restrict__ res_scale,
+                     uint32_t* err) {
   using namespace tc;
   constexpr int C = 128;
-  using Lay = EncTc2Layout<R>;
+  using Lay = EncTc2Layout<R, I8>;
   extern __shared__ unsigned char enc2_smem_dyn[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(enc2_smem_dyn) + 1023) & ~uintptr_t(1023));
@@ -770,6 +778,7 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
       mbar_init(&misc->h_ready[s], 4);     // the 4 warps of the tile's group
       mbar_init(&misc->d2_full[s], 1);
       mbar_init(&misc->slot_free[s], 4);
+      mbar_init(&misc->a_conv[s], 4);      // the group's converted rows (int8 store)
     }
     misc->abort_flag = 0;
     mbar_init_fence();
@@ -788,22 +797,30 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
     const uint64_t dW1 = smem_desc(smem_u32(smem + Lay::OFF_W1), 16, 1024, 2);
     const uint64_t dW2 = smem_desc(smem_u32(smem + Lay::OFF_W2), 16, 1024, 2);
     const uint64_t dA0 = smem_desc(smem_u32(smem + Lay::OFF_A), 16, 1024, 2);
-    constexpr uint32_t IDESC_1 = idesc_f16(128, 128, 1, 1);   // A (bf16) x W1'/2 (bf16), both K-major
+    // A x W1'/2, both K-major: bf16, or fp16 for the int8 store
+    constexpr uint32_t IDESC_1 = I8 ? idesc_f16(128, 128, 0, 0) : idesc_f16(128, 128, 1, 1);
     constexpr uint32_t IDESC_2 = idesc_f16(128, 128, 0, 0);   // H (TMEM, fp16) x W2 (fp16, K-major)
     auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, par, abort_flag, err, ERR_TIMEOUT));
     };
     auto seg_of = [&](long long i) { return (int)((x0 + i) / nC / B); };
-    auto issue_a = [&](long long i) {   // tile i's coefficient tile into stage i % 2
+    auto issue_a = [&](long long i) {   // tile i's coefficient tile into stage (or staging slot) i % 2
       const long long x = x0 + i;
       const int u = (int)(x / nC), c = (int)(x % nC);
       const int b = u % B, seg = u / B, hkv = seg % Hkv, l = seg / Hkv, grp = l / G;
       const long long arow = (((long long)b * NG + grp) * Hkv + hkv) * N + (long long)c * C;
       if (leader) {
-        mbar_expect_tx(&misc->a_full[i & 1], (uint32_t)Lay::A_BYTES);
-        for (int ks = 0; ks < Lay::KSLABS; ++ks)
-          tma_load_2d(smem + Lay::OFF_A + (i & 1) * Lay::A_BYTES + ks * 16384, &tmA, &misc->a_full[i & 1], ks * 64,
-                      (int)arow);
+        if (I8) {
+          unsigned char* dst = smem + Lay::OFF_SA + (i & 1) * Lay::SA_SLOT;
+          mbar_expect_tx(&misc->a_full[i & 1], (uint32_t)Lay::SA_SLOT);
+          bulk_load(dst, static_cast<const int8_t*>(coeff) + arow * R, (uint32_t)(C * R), &misc->a_full[i & 1]);
+          bulk_load(dst + C * R, coeff_scale + arow, (uint32_t)(C * 2), &misc->a_full[i & 1]);
+        } else {
+          mbar_expect_tx(&misc->a_full[i & 1], (uint32_t)Lay::A_BYTES);
+          for (int ks = 0; ks < Lay::KSLABS; ++ks)
+            tma_load_2d(smem + Lay::OFF_A + (i & 1) * Lay::A_BYTES + ks * 16384, &tmA, &misc->a_full[i & 1],
+                        ks * 64, (int)arow);
+        }
       }
       __syncwarp();
     };
@@ -828,7 +845,9 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
     };
     auto issue_d1 = [&](long long i) -> bool {
       const int s = (int)(i & 1);
-      if (!wait_all(&misc->a_full[s], (uint32_t)((i >> 1) & 1))) return false;
+      // the tile in the stage: by TMA, or (int8 store) converted by its group from the staging
+      // slot, which the group waited for (so the copy has landed either way)
+      if (!wait_all(I8 ? &misc->a_conv[s] : &misc->a_full[s], (uint32_t)((i >> 1) & 1))) return false;
       a_waited = i + 1;
       if (i >= 2 && !wait_all(&misc->slot_free[s], (uint32_t)(((i >> 1) - 1) & 1))) return false;
       if (leader) {
@@ -935,11 +954,39 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
         rank = (int)below;
         rbase = (size_t)res_ptr[unit * (nC + 1) + c];
       }
-      // the token's values row for the epilogue, requested now (pass 2: flagged tokens only)
+      // the token's values row for the epilogue (pass 2: flagged tokens only), requested now;
+      // for an int8 record once the silu is done, so that it does not sit in registers
+      // through the conversion and the silu
       uint4 vrow[kEncD / 8];
       const uint4* vp = reinterpret_cast<const uint4*>(values + (tok + t) * kEncD);
+      if (!(EMIT && I8)) {
 #pragma unroll
-      for (int j = 0; j < kEncD / 8; ++j) vrow[j] = (!EMIT || flagged) ? __ldg(vp + j) : make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < kEncD / 8; ++j) vrow[j] = (!EMIT || flagged) ? __ldg(vp + j) : make_uint4(0, 0, 0, 0);
+      }
+      if (I8) {   // this token's stored row, sigma_t a_t as fp16, into the coefficient stage
+        if (!__all_sync(0xffffffffu, mbar_wait(&misc->a_full[s], par, abort_flag, err, ERR_TIMEOUT))) break;
+        const unsigned char* src = smem + Lay::OFF_SA + s * Lay::SA_SLOT;
+        const float sg = __half2float(reinterpret_cast<const __half*>(src + C * R)[t]);
+        unsigned char* arow_s = smem + Lay::OFF_A + s * Lay::A_BYTES + t * 128;
+#pragma unroll
+        for (int j = 0; j < R / 8; ++j) {   // 8 values = one 16-byte chunk of the swizzled row
+          const uint2 q = *reinterpret_cast<const uint2*>(src + t * R + 8 * j);
+          const uint32_t qw[2] = {q.x, q.y};
+          uint32_t o[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float x0f = (float)(int8_t)((qw[k >> 1] >> (16 * (k & 1))) & 0xffu) * sg;
+            const float x1f = (float)(int8_t)((qw[k >> 1] >> (16 * (k & 1) + 8)) & 0xffu) * sg;
+            const __half2 h2 = __floats2half2_rn(x0f, x1f);
+            o[k] = *reinterpret_cast<const uint32_t*>(&h2);
+          }
+          const int ks = j >> 3, jj = j & 7;
+          *reinterpret_cast<uint4*>(arow_s + ks * 16384 + ((jj ^ (t & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&misc->a_conv[s]);
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&misc->d1_full[s], par, abort_flag, err, ERR_TIMEOUT))) break;
       tc_fence_after();
       // H = silu(2 D1) for this token's 256 hidden units, as fp16 pairs over columns 0..127
@@ -965,37 +1012,79 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&misc->h_ready[s]);
+      if (EMIT && I8) {
+#pragma unroll
+        for (int j = 0; j < kEncD / 8; ++j) vrow[j] = flagged ? __ldg(vp + j) : make_uint4(0, 0, 0, 0);
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&misc->d2_full[s], par, abort_flag, err, ERR_TIMEOUT))) break;
       tc_fence_after();
       // delta = V - Vhat for this token's 128 dims: its norm (pass 1) or its record (pass 2)
       float ss = 0.f;
-      uint32_t vd[kEncD];   // the token's rebuilt row, all of it in one TMEM round trip
+      if constexpr (EMIT && I8) {
+        // the int8 record: a pass over the row for its scale, a second for its codes (64 dims
+        // per TMEM round trip, delta recomputed, so that the row never sits in registers whole)
+        float dmax = 0.f;
+        __half sh = __ushort_as_half((unsigned short)0);
+#pragma unroll 1
+        for (int pass = 0; pass < 2; ++pass)
+#pragma unroll 1
+          for (int hv = 0; hv < 2; ++hv) {
+            uint32_t vh[64];
+            tmem_ld32(tmem + lane_off + 256 * s + 128 + 64 * hv, *reinterpret_cast<uint32_t(*)[32]>(vh));
+            tmem_ld32(tmem + lane_off + 256 * s + 128 + 64 * hv + 32, *reinterpret_cast<uint32_t(*)[32]>(vh + 32));
+            tmem_wait_ld();
 #pragma unroll
-      for (int q = 0; q < kEncD / 32; ++q)
-        tmem_ld32(tmem + lane_off + 256 * s + 128 + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(vd + 32 * q));
-      tmem_wait_ld();
+            for (int k8 = 0; k8 < 8; ++k8) {
+              const uint4 w4 = vrow[8 * hv + k8];
+              const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
+              float x8[8];
 #pragma unroll
-      for (int q = 0; q < kEncD / 32; ++q) {
-        const uint32_t* v = vd + 32 * q;
-        uint32_t o[16];
+              for (int h = 0; h < 4; ++h) {
+                x8[2 * h] = __uint_as_float(ww[h] << 16) - __uint_as_float(vh[8 * k8 + 2 * h]);
+                x8[2 * h + 1] = __uint_as_float(ww[h] & 0xffff0000u) - __uint_as_float(vh[8 * k8 + 2 * h + 1]);
+              }
+              if (pass == 0) {
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const uint4 w4 = vrow[(32 * q + j) >> 3];
-          const uint32_t w = ((j >> 1) & 3) == 0 ? w4.x : ((j >> 1) & 3) == 1 ? w4.y : ((j >> 1) & 3) == 2 ? w4.z : w4.w;
-          const float d0 = __uint_as_float(w << 16) - __uint_as_float(v[j]);
-          const float d1 = __uint_as_float(w & 0xffff0000u) - __uint_as_float(v[j + 1]);
-          if (!EMIT) {
-            ss = fmaf(d0, d0, ss);
-            ss = fmaf(d1, d1, ss);
-          } else {
-            const __nv_bfloat162 p = __floats2bfloat162_rn(d0, d1);
-            o[j >> 1] = *reinterpret_cast<const uint32_t*>(&p);
+                for (int k = 0; k < 8; ++k) dmax = fmaxf(dmax, fabsf(x8[k]));
+              } else if (flagged) {
+                uint2 codes;
+                quantize8(x8, dmax, &sh, &codes, nullptr);
+                *reinterpret_cast<uint2*>(static_cast<int8_t*>(res_val) + (rbase + rank) * kEncD + 64 * hv + 8 * k8) =
+                    codes;
+              }
+            }
           }
-        }
-        if (EMIT && flagged) {
-          uint4* dst = reinterpret_cast<uint4*>(res_val + (rbase + rank) * kEncD + 32 * q);
+        if (flagged) res_scale[rbase + rank] = sh;
+      } else {
+        uint32_t vd[kEncD];   // the token's rebuilt row, all of it in one TMEM round trip
 #pragma unroll
-          for (int k = 0; k < 4; ++k) dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+        for (int q = 0; q < kEncD / 32; ++q)
+          tmem_ld32(tmem + lane_off + 256 * s + 128 + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(vd + 32 * q));
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < kEncD / 32; ++q) {
+          const uint32_t* v = vd + 32 * q;
+          uint32_t o[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const uint4 w4 = vrow[(32 * q + j) >> 3];
+            const uint32_t w = ((j >> 1) & 3) == 0 ? w4.x : ((j >> 1) & 3) == 1 ? w4.y : ((j >> 1) & 3) == 2 ? w4.z : w4.w;
+            const float d0 = __uint_as_float(w << 16) - __uint_as_float(v[j]);
+            const float d1 = __uint_as_float(w & 0xffff0000u) - __uint_as_float(v[j + 1]);
+            if (!EMIT) {
+              ss = fmaf(d0, d0, ss);
+              ss = fmaf(d1, d1, ss);
+            } else {
+              const __nv_bfloat162 p = __floats2bfloat162_rn(d0, d1);
+              o[j >> 1] = *reinterpret_cast<const uint32_t*>(&p);
+            }
+          }
+          if (EMIT && flagged) {
+            uint4* dst =
+                reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(res_val) + (rbase + rank) * kEncD + 32 * q);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+          }
         }
       }
       tc_fence_before();
@@ -1227,7 +1316,7 @@ __global__ void to_half_kernel(const __nv_bfloat16* __restrict__ src, __half* __
 // Workspace pieces (256-byte aligned, in this order).
 struct EncWs {
   float* w1f_t;            // [L][Hkv][r][h] fp32 W1'
-  __nv_bfloat16* w1f_tc;   // [L][Hkv][h][r] bf16 W1'/2 (tensor-core path)
+  __nv_bfloat16* w1f_tc;   // [L][Hkv][h][r] W1'/2 (tensor-core path): bf16, fp16 for the int8 store
   __half* w2h;             // [L][Hkv][d][h] fp16 W2 (tensor-core path)
   float* norms;            // [units][N]
   uint8_t* flags;          // [units][N]
@@ -1572,34 +1661,39 @@ cudaError_t launch_encode_t(const Geom& g, int n_res, const void* keys, const vo
         dst.coeff, static_cast<__half*>(dst.coeff_scale), static_cast<__nv_bfloat16*>(dst.summary));
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (!I8) {   // tensor cores
+  if (C == 128 || !I8) {   // tensor cores
     using Lay = EncTcLayout<R, C>;
     CUtensorMap tmW1, tmW2, tmA;
     const uint64_t lh = (uint64_t)g.L * g.Hkv;
-    if (!enc_make_map(&tmW1, w.w1f_tc, R, lh * kEncH, 128) || !enc_make_map(&tmW2, w.w2h, kEncH, lh * kEncD, 128) ||
-        !enc_make_map(&tmA, dst.coeff, R, (uint64_t)g.B * NG * g.Hkv * g.N, C))
+    if (!enc_make_map(&tmW1, w.w1f_tc, R, lh * kEncH, 128) || !enc_make_map(&tmW2, w.w2h, kEncH, lh * kEncD, 128))
+      return cudaErrorInvalidValue;
+    if (I8)   // the int8 tiles arrive by plain bulk copies
+      tmA = tmW1;
+    else if (!enc_make_map(&tmA, dst.coeff, R, (uint64_t)g.B * NG * g.Hkv * g.N, C))
       return cudaErrorInvalidValue;
     if (!w2h_ready)
       to_half_kernel<<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w2), w.w2h, (size_t)lh * kEncD * kEncH);
     const unsigned grid = (unsigned)std::min<size_t>((size_t)n_sm, units * nC);
     if (C == 128) {   // tokens as the MMAs' M dimension, two tiles in flight
-      using Lay2 = EncTc2Layout<R>;
-      auto t1 = enc_resid_tc2_kernel<R, false>;
-      auto t2 = enc_resid_tc2_kernel<R, true>;
+      using Lay2 = EncTc2Layout<R, I8>;
+      auto t1 = enc_resid_tc2_kernel<R, false, I8>;
+      auto t2 = enc_resid_tc2_kernel<R, true, I8>;
       if ((e = cudaFuncSetAttribute(t1, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay2::SMEM)) != cudaSuccess) return e;
       if ((e = cudaFuncSetAttribute(t2, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay2::SMEM)) != cudaSuccess) return e;
-      t1<<<grid, kEnc2Threads, Lay2::SMEM, s>>>(g.B, g.L, g.G, g.Hkv, g.N, tmW1, tmW2, tmA,
+      t1<<<grid, kEnc2Threads, Lay2::SMEM, s>>>(g.B, g.L, g.G, g.Hkv, g.N, tmW1, tmW2, tmA, dst.coeff,
+                                               static_cast<const __half*>(dst.coeff_scale),
                                                static_cast<const __nv_bfloat16*>(values), w.norms, nullptr, nullptr,
-                                               nullptr, nullptr, w.err);
+                                               nullptr, nullptr, nullptr, w.err);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
       enc_select_kernel<<<(unsigned)units, kSelThreads, (size_t)nC * sizeof(int), s>>>(g.N, C, n_res, w.norms,
                                                                                        w.flags, dst.res_ptr);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
       if (n_res > 0)
-        t2<<<grid, kEnc2Threads, Lay2::SMEM, s>>>(g.B, g.L, g.G, g.Hkv, g.N, tmW1, tmW2, tmA,
+        t2<<<grid, kEnc2Threads, Lay2::SMEM, s>>>(g.B, g.L, g.G, g.Hkv, g.N, tmW1, tmW2, tmA, dst.coeff,
+                                                 static_cast<const __half*>(dst.coeff_scale),
                                                  static_cast<const __nv_bfloat16*>(values), w.norms, w.flags,
-                                                 dst.res_ptr, dst.res_pos, static_cast<__nv_bfloat16*>(dst.res_val),
-                                                 w.err);
+                                                 dst.res_ptr, dst.res_pos, dst.res_val,
+                                                 static_cast<__half*>(dst.res_scale), w.err);
       return cudaGetLastError();
     }
     auto k1 = enc_resid_tc_kernel<R, C, false>;
@@ -1671,16 +1765,17 @@ cudaError_t launch_encode(const Geom& g, int store, int n_res, const void* keys,
                           void* workspace, cudaStream_t s, const float* w1f_t, const void* w1f_tc,
                           bool w2h_ready) {
   const bool i8 = store == LOWRAM_STORE_INT8;
-  const bool folds_given = w1f_t && (i8 || w1f_tc);
+  const bool folds_given = w1f_t && w1f_tc;
   EncWs w = carve(g, workspace, nullptr, folds_given);
-  if (folds_given) {   // the caller's folds (the int8 path reads only the fp32 one)
+  if (folds_given) {   // the caller's folds: fp32, and W1'/2 in bf16 (native) or fp16 (int8 store)
     w.w1f_t = const_cast<float*>(w1f_t);
-    if (!i8) w.w1f_tc = static_cast<__nv_bfloat16*>(const_cast<void*>(w1f_tc));
+    w.w1f_tc = static_cast<__nv_bfloat16*>(const_cast<void*>(w1f_tc));
   } else {
     CacheBuffers cb{};
     cb.w1 = w1;
     cb.basis = basis;
-    cudaError_t e = launch_fold(g, cb, LOWRAM_BF16, LOWRAM_STORE_NATIVE, w.w1f_t, w.w1f_tc, s);
+    cudaError_t e = launch_fold(g, cb, LOWRAM_BF16, i8 ? LOWRAM_STORE_INT8 : LOWRAM_STORE_NATIVE, w.w1f_t,
+                                w.w1f_tc, s);
     if (e != cudaSuccess) return e;
   }
 #define LOWRAM_ENC_CASE(RR, CC)                                                                          \

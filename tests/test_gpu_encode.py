@@ -49,8 +49,10 @@ def _gpu_codes(g, cfg):
 # relative norm error concentrates far below the 2^-9 of a single rounding: a numpy model of
 # exactly these roundings on the 32K workload's weights puts it at 8e-5 (median) and 5.8e-4
 # (largest of 8192 tokens), with the W1' rounding alone at 5.8e-4 and the fp16 H alone at
-# 1.2e-4.  The CUDA-core predictor (int8 stores) keeps everything in fp32.  The bound
-# asserted token by token, where the kernel's norms can be read back:
+# 1.2e-4.  For int8 stores with C = 128 the tensor-core predictor takes W1'/2 and the
+# dequantised rows sigma*a in fp16 (unit roundoff 2^-11, four times finer); with C = 64 the
+# CUDA-core predictor keeps everything in fp32.  The bound asserted token by token, where the
+# kernel's norms can be read back:
 NORM_RTOL = 1e-3
 NORM_ATOL = 1e-6
 
