@@ -74,6 +74,31 @@ __device__ __forceinline__ void quantize8(const float* x, float amax, __half* sc
   *scale_out = sh;
 }
 
+// The same encoding of 8 values of a row whose fp16 scale s (> 0 or 0) and reciprocal r are
+// known: round-half-even of x / s from a first guess rint(x r), corrected by the exact
+// remainder x - q s (an fma: q s has at most 19 significant bits and lies within s of x, so
+// the remainder is representable), a tie going to even.  One division per row instead of
+// one per value; the result is the rounding of the exact quotient.
+__device__ __forceinline__ float rne_quot(float x, float s, float r) {
+  float q = rintf(x * r);
+  const float rem = fmaf(-q, s, x);
+  const float h = 0.5f * s;
+  const bool odd = ((int)q & 1) != 0;
+  if (rem > h || (rem == h && odd)) q += 1.f;
+  else if (rem < -h || (rem == -h && odd)) q -= 1.f;
+  return q;
+}
+__device__ __forceinline__ uint2 quantize8_scaled(const float* x, float s, float r) {
+  uint32_t w[2] = {0u, 0u};
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    float q = s > 0.f ? rne_quot(x[j], s, r) : 0.f;
+    q = fminf(fmaxf(q, -127.f), 127.f);
+    w[j >> 2] |= ((uint32_t)(int)q & 0xffu) << (8 * (j & 3));
+  }
+  return make_uint2(w[0], w[1]);
+}
+
 // --------------------------------------------------------------------- coefficients
 // Thread (ty, tx): tokens ty*TM .. +TM, ranks tx*8 .. +8.  Per (layer, 32-wide slice of
 // d): the chunk's key slice and the basis slice go to shared memory transposed (k-major),
@@ -1012,9 +1037,19 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&misc->h_ready[s]);
-      if (EMIT && I8) {
+      // int8 record: a flagged token's values row goes to shared memory while the second GEMM
+      // runs -- into this tile's coefficient stage, which only this group writes (its next
+      // conversion comes after this epilogue) and whose pre-activations are done; row t,
+      // 16-byte chunk j at j ^ (t % 16) (R = 128: 128 rows of 256 bytes; R = 64 reads the
+      // row from global memory in the passes below)
+      constexpr bool kVStage = Lay::A_BYTES >= C * kEncD * 2;
+      unsigned char* vst = smem + Lay::OFF_A + s * Lay::A_BYTES + (kVStage ? t * kEncD * 2 : 0);
+      if (EMIT && I8 && kVStage && flagged) {
+        uint4 tmp[kEncD / 8];
 #pragma unroll
-        for (int j = 0; j < kEncD / 8; ++j) vrow[j] = flagged ? __ldg(vp + j) : make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < kEncD / 8; ++j) tmp[j] = __ldg(vp + j);
+#pragma unroll
+        for (int j = 0; j < kEncD / 8; ++j) *reinterpret_cast<uint4*>(vst + ((j ^ (t & 15)) << 4)) = tmp[j];
       }
       if (!__all_sync(0xffffffffu, mbar_wait(&misc->d2_full[s], par, abort_flag, err, ERR_TIMEOUT))) break;
       tc_fence_after();
@@ -1023,19 +1058,20 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
       if constexpr (EMIT && I8) {
         // the int8 record: a pass over the row for its scale, a second for its codes (64 dims
         // per TMEM round trip, delta recomputed, so that the row never sits in registers whole)
-        float dmax = 0.f;
+        float dmax = 0.f, sc = 0.f, rc = 0.f;
         __half sh = __ushort_as_half((unsigned short)0);
 #pragma unroll 1
         for (int pass = 0; pass < 2; ++pass)
 #pragma unroll 1
-          for (int hv = 0; hv < 2; ++hv) {
-            uint32_t vh[64];
-            tmem_ld32(tmem + lane_off + 256 * s + 128 + 64 * hv, *reinterpret_cast<uint32_t(*)[32]>(vh));
-            tmem_ld32(tmem + lane_off + 256 * s + 128 + 64 * hv + 32, *reinterpret_cast<uint32_t(*)[32]>(vh + 32));
+          for (int q = 0; q < kEncD / 32; ++q) {
+            uint32_t vh[32];   // (the load is warp-wide; only flagged lanes use it)
+            tmem_ld32(tmem + lane_off + 256 * s + 128 + 32 * q, vh);
             tmem_wait_ld();
+            if (!flagged) continue;
 #pragma unroll
-            for (int k8 = 0; k8 < 8; ++k8) {
-              const uint4 w4 = vrow[8 * hv + k8];
+            for (int k8 = 0; k8 < 4; ++k8) {
+              const int j = 4 * q + k8;   // 16-byte chunk of the values row
+              const uint4 w4 = kVStage ? *reinterpret_cast<const uint4*>(vst + ((j ^ (t & 15)) << 4)) : __ldg(vp + j);
               const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
               float x8[8];
 #pragma unroll
@@ -1046,12 +1082,15 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
               if (pass == 0) {
 #pragma unroll
                 for (int k = 0; k < 8; ++k) dmax = fmaxf(dmax, fabsf(x8[k]));
-              } else if (flagged) {
-                uint2 codes;
-                quantize8(x8, dmax, &sh, &codes, nullptr);
-                *reinterpret_cast<uint2*>(static_cast<int8_t*>(res_val) + (rbase + rank) * kEncD + 64 * hv + 8 * k8) =
-                    codes;
+              } else {
+                *reinterpret_cast<uint2*>(static_cast<int8_t*>(res_val) + (rbase + rank) * kEncD + 32 * q + 8 * k8) =
+                    quantize8_scaled(x8, sc, rc);
               }
+            }
+            if (pass == 0 && q == kEncD / 32 - 1) {   // the row's scale, once its max is known
+              sh = __float2half_rn(dmax / 127.f);
+              sc = __half2float(sh);
+              rc = sc > 0.f ? 1.f / sc : 0.f;
             }
           }
         if (flagged) res_scale[rbase + rank] = sh;
