@@ -88,12 +88,17 @@ __device__ __forceinline__ float rne_quot(float x, float s, float r) {
   else if (rem < -h || (rem == -h && odd)) q -= 1.f;
   return q;
 }
+// (x r is within 2^-22 relative of x / s, i.e. within 4e-5 for |x / s| <= 127.5, so its
+// nearest integer is the answer unless x r lies within 1e-4 of a half-integer; only then is
+// the exact remainder consulted.)
 __device__ __forceinline__ uint2 quantize8_scaled(const float* x, float s, float r) {
   uint32_t w[2] = {0u, 0u};
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    float q = s > 0.f ? rne_quot(x[j], s, r) : 0.f;
-    q = fminf(fmaxf(q, -127.f), 127.f);
+    const float y = x[j] * r;
+    float q = rintf(y);
+    if (fabsf(y - q) > 0.4999f) q = rne_quot(x[j], s, r);
+    q = s > 0.f ? fminf(fmaxf(q, -127.f), 127.f) : 0.f;
     w[j >> 2] |= ((uint32_t)(int)q & 0xffu) << (8 * (j & 3));
   }
   return make_uint2(w[0], w[1]);
