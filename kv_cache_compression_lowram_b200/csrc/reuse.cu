@@ -492,23 +492,7 @@ reuse_fill_kernel(Geom g, CacheBuffers cb, Scratch sc, ReuseDev st, const __grid
       const long long x = x0 + i;
       const int s = (int)(i & 1);
       const uint32_t par = (uint32_t)((i >> 1) & 1);
-      const int u = sc.tile_unit[x], slot = sc.tile_slot[x];
-      const Unit un = unit_of(g, u);
-      const int l = g.layer0 + un.li;
-      // this token's residual record, if it has one (the chunk's few records scanned)
-      const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nLs + 1);
-      int r0 = rptr[slot], r1 = rptr[slot + 1];
-      if (r0 < 0 || r1 < r0 || (long long)r1 > (long long)cb.n_records) {
-        if (t == 0) atomicOr(err, ERR_RES_PTR);
-        r0 = r1 = 0;
-      }
-      int rec = -1;
-      for (int k = r0; k < r1; ++k)
-        if ((int)cb.res_pos[k] == t) rec = k;
-      uint4 drow[kD / 8];
-      const uint4* dp = reinterpret_cast<const uint4*>(rv + (size_t)(rec < 0 ? 0 : rec) * kD);
-#pragma unroll
-      for (int j = 0; j < kD / 8; ++j) drow[j] = rec >= 0 ? __ldg(dp + j) : make_uint4(0, 0, 0, 0);
+      const int u = sc.tile_unit[x], slot = sc.tile_slot[x];   // (used after the silu)
       if (!__all_sync(0xffffffffu, mbar_wait(&misc->d1_full[s], par, abort_flag, err, ERR_TIMEOUT))) break;
       tc_fence_after();
 #pragma unroll
@@ -531,6 +515,23 @@ reuse_fill_kernel(Geom g, CacheBuffers cb, Scratch sc, ReuseDev st, const __grid
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&misc->h_ready[s]);
+      // while the second GEMM runs: this token's residual record, if it has one (the chunk's
+      // few records scanned), and its row
+      const Unit un = unit_of(g, u);
+      const int l = g.layer0 + un.li;
+      const int32_t* rptr = cb.res_ptr + (((size_t)un.b * g.L + l) * g.Hkv + un.hkv) * (g.nLs + 1);
+      int r0 = rptr[slot], r1 = rptr[slot + 1];
+      if (r0 < 0 || r1 < r0 || (long long)r1 > (long long)cb.n_records) {
+        if (t == 0) atomicOr(err, ERR_RES_PTR);
+        r0 = r1 = 0;
+      }
+      int rec = -1;
+      for (int k = r0; k < r1; ++k)
+        if ((int)cb.res_pos[k] == t) rec = k;
+      uint4 drow[kD / 8];
+      const uint4* dp = reinterpret_cast<const uint4*>(rv + (size_t)(rec < 0 ? 0 : rec) * kD);
+#pragma unroll
+      for (int j = 0; j < kD / 8; ++j) drow[j] = rec >= 0 ? __ldg(dp + j) : make_uint4(0, 0, 0, 0);
       if (!__all_sync(0xffffffffu, mbar_wait(&misc->d2_full[s], par, abort_flag, err, ERR_TIMEOUT))) break;
       tc_fence_after();
       // vhat[t] = D2[t] + delta (if the token has a record), as bf16, straight to the entry,
