@@ -262,6 +262,28 @@ def test_host_entry_point_matches_device_call():
     lc.close()
 
 
+def test_host_entry_point_pinned_and_pageable_across_steps():
+    """Consecutive steps through the host entry point, alternating a pinned buffer refilled in
+    place and a fresh pageable one: every call matches the device entry point."""
+    cfg = S.LLAMA_32K.replace(name="host_q", batch=2, n_layers=4, n_kv_heads=2, n_ctx=1024, top_k=4)
+    cache = S.make_cache(cfg, device=DEV)
+    steps = S.make_query_steps(cache, 3, 0.0, 1.0)
+    lc = K.LowramCache.from_synth(cache)
+    q_pin = steps[0].cpu().pin_memory()
+    out_h = torch.empty_like(q_pin).pin_memory()
+    for t, q in enumerate(steps):
+        ref = lc.decode(q)
+        torch.cuda.synchronize()
+        q_pin.copy_(q.cpu())                   # same pinned buffer, new contents
+        K.lowram_decode_attn_host(lc.handle, 0, cfg.n_layers, q_pin, out_h)
+        assert torch.equal(out_h, ref.cpu()), t
+        q_page = q.cpu().clone()               # pageable
+        out_p = torch.empty_like(q_page)
+        K.lowram_decode_attn_host(lc.handle, 0, cfg.n_layers, q_page, out_p)
+        assert torch.equal(out_p, ref.cpu()), t
+    lc.close()
+
+
 def test_validate_detects_corrupt_tables():
     cfg = S.MISTRAL_GROUP
     cache = S.make_cache(cfg)
