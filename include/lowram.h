@@ -424,10 +424,11 @@ typedef struct {
   uint64_t hits, misses, fills;  /* cumulative chunk counts over the store's decode calls */
 } lowram_reuse_counts;
 
-/* A store for `cache` with `capacity` entries (capacity * 32 KB at C = d = 128, plus a table of
- * 4 bytes per chunk slot of the cache), admitting at most fill_cap <= capacity misses per call.
- * Stream-ordered.  EINVAL for bad sizes, EUNSUPPORTED for shapes without a reuse path, ENOMEM.
- * The store is tied to the cache as it is now: after a lowram_cache_repack the store's calls
+/* A store for `cache` with `capacity` entries (1 <= capacity <= 2^30; capacity * 32 KB at C = d
+ * = 128, plus a table of 4 bytes per chunk slot of the cache), admitting at most
+ * fill_cap <= capacity misses per call.
+ * Stream-ordered.  EINVAL for bad sizes, EUNSUPPORTED for shapes without a reuse path, ENOMEM;
+ * *out is NULL after any error.  The store is tied to the cache as it is now: after a lowram_cache_repack the store's calls
  * return EINVAL (make a new one).  Destroy the store before the cache. */
 lowram_status lowram_reuse_create(lowram_cache* cache, int32_t capacity, int32_t fill_cap, lowram_reuse** out,
                                   lowram_stream stream);

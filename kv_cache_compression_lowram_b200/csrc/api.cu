@@ -1020,9 +1020,11 @@ void lowram_reuse_destroy(lowram_reuse* r) {
 
 lowram_status lowram_reuse_create(lowram_cache* c, int32_t capacity, int32_t fill_cap, lowram_reuse** out,
                                   lowram_stream stream) {
+  if (out) *out = nullptr;
   if (!c || !out) return inval("NULL cache or output");
-  *out = nullptr;
-  if (capacity < 1 || fill_cap < 0 || fill_cap > capacity) return inval("need capacity >= 1 and 0 <= fill_cap <= capacity");
+  // capacity <= 2^30 keeps the ring arithmetic (position + fill index < 2 * capacity) in int32
+  if (capacity < 1 || capacity > (1 << 30) || fill_cap < 0 || fill_cap > capacity)
+    return inval("need 1 <= capacity <= 2^30 and 0 <= fill_cap <= capacity");
   Geom g = make_geom(c, 0, c->cfg.n_layers, true);
   if (!reuse_supported(g, c->cfg.dtype, c->cfg.store) || c->cfg.top_k > 32) {
     g_last_error = "the reuse store takes bf16 native stores, head_dim 128, mlp_hidden 256, rank 64 or 128, "

@@ -137,3 +137,39 @@ def test_test_hooks_host_side():
     assert lib.lowram_debug_set_wait_limit(None, 5) == 1
     K.lowram_debug_fail_alloc(3)
     K.lowram_debug_fail_alloc(-1)
+
+
+def test_shard_and_merge_host_checks():
+    """Context-sharded decode: NULL caches and impossible merge shapes are rejected before any
+    CUDA call."""
+    lib = K.lib()
+    assert lib.lowram_shard_candidates(None, 0, 1, None, 0, None, None, None) == 1
+    assert lib.lowram_shard_partial(None, 0, 1, 0, 2, None, None, None, None, None) == 1
+    bad = [
+        (0, 4, 128, 1),      # no parts
+        (2, -1, 128, 1),     # negative row count
+        (2, 1 << 31, 128, 1),
+        (2, 4, 0, 1),        # head_dim outside 1..256
+        (2, 4, 257, 1),
+        (2, 4, 128, 7),      # unknown output dtype
+        (2, 4, 128, 1),      # rows but NULL buffers
+    ]
+    for n_parts, n_rows, d, dt in bad:
+        assert lib.lowram_merge_partials(n_parts, n_rows, d, None, dt, None, None) == 1, (n_parts, n_rows, d, dt)
+        assert lib.lowram_last_error_string()
+
+
+def test_reuse_host_checks():
+    """The reuse store's entry points reject NULL handles and outputs on the host; destroying
+    NULL is a no-op."""
+    lib = K.lib()
+    h = ctypes.c_void_p(1234)
+    assert lib.lowram_reuse_create(None, 16, 16, ctypes.byref(h), None) == 1
+    assert not h.value   # the output handle is cleared on every error
+    assert lib.lowram_decode_attn_reuse(None, 0, 1, None, None, None, None) == 1
+    counts = K.LowramReuseCountsC()
+    assert lib.lowram_reuse_counts_get(None, ctypes.byref(counts), None) == 1
+    t, o, e = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_void_p()
+    stride = ctypes.c_int64()
+    assert lib.lowram_reuse_view(None, ctypes.byref(t), ctypes.byref(o), ctypes.byref(e), ctypes.byref(stride)) == 1
+    lib.lowram_reuse_destroy(None)

@@ -176,7 +176,8 @@ def test_store_refuses_after_repack_and_unsupported_shapes():
     with pytest.raises(K.LowramError) as ei:
         K.LowramReuse(other, 16, 16)
     assert ei.value.status == 4
-    with pytest.raises(K.LowramError) as ei:
-        K.LowramReuse(other, 16, 17)
-    assert ei.value.status == 1
+    for cap, fill in ((16, 17), (0, 0), ((1 << 30) + 1, 1), (16, -1)):
+        with pytest.raises(K.LowramError) as ei:
+            K.LowramReuse(other, cap, fill)
+        assert ei.value.status == 1, (cap, fill)
     other.close()
