@@ -67,6 +67,9 @@ class ShardDecoder:
         return cs, ci
 
     def partial(self, cs_all, ci_all, layer0: int = 0):
+        if int(cs_all.shape[0]) != self.n_shards or tuple(ci_all.shape) != tuple(cs_all.shape):
+            raise ValueError(f"expected the candidates of {self.n_shards} shards, got {tuple(cs_all.shape)} "
+                             f"scores and {tuple(ci_all.shape)} ids")
         n = self._n
         part = torch.empty(n, self.B, self.Hq, self.d + 2, dtype=torch.float32, device=cs_all.device)
         sel = torch.empty(n, self.B, self.Hkv, self.k, dtype=torch.int32, device=cs_all.device)

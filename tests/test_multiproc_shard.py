@@ -10,6 +10,7 @@ import os
 import socket
 
 import numpy as np
+import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
@@ -108,3 +109,20 @@ def test_sharded_protocol_two_ranks_gloo():
         assert np.array_equal(sel, ref["sel"])
         err = np.abs(got - ref["out"]).max(axis=-1) / np.abs(ref["out"]).max(axis=-1)
         assert err.max() <= 1e-12
+
+
+def test_shard_decoder_checks_the_gathered_shard_count():
+    """Phase 2 is refused on the host when the gather returned another number of shards than
+    the decoder was built for (no library call is made)."""
+    from types import SimpleNamespace
+
+    from kv_cache_compression_lowram_b200.sharded import ShardDecoder
+
+    cfg = dict(batch=1, n_kv_heads=2, n_q_heads=8, head_dim=128, top_k=4, dtype="bf16")
+    dec = ShardDecoder(SimpleNamespace(cfg=cfg, handle=None), 0, 2)
+    dec._n = 1
+    cs = torch.zeros(3, 1, 1, 2, 4)
+    with pytest.raises(ValueError):
+        dec.partial(cs, torch.zeros(3, 1, 1, 2, 4, dtype=torch.int32))
+    with pytest.raises(ValueError):
+        dec.partial(cs[:2], torch.zeros(2, 1, 1, 2, 3, dtype=torch.int32))
