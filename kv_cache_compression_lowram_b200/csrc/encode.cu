@@ -960,6 +960,7 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
     const int t = 32 * wq + lane;                      // this thread's token (TMEM lane)
     const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
     const unsigned lt_mask = (1u << lane) - 1u;
+    constexpr bool kVStageI8 = I8 && Lay::A_BYTES >= C * kEncD * 2;   // values rows staged (R = 128)
     for (long long i = grp_t; i < n; i += 2) {
       const long long x = x0 + i;
       const int s = (int)(i & 1);
@@ -994,6 +995,12 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
         for (int j = 0; j < kEncD / 8; ++j) vrow[j] = (!EMIT || flagged) ? __ldg(vp + j) : make_uint4(0, 0, 0, 0);
       }
       if (I8) {   // this token's stored row, sigma_t a_t as fp16, into the coefficient stage
+        // pass 2 stages the flagged tokens' values rows in this stage (below), and a warp's
+        // rows there overlap other warps' coefficient rows: the group's previous tile must be
+        // done by all four warps (their slot_free arrivals) before any of them overwrites it
+        if (EMIT && kVStageI8 && i >= 2 &&
+            !__all_sync(0xffffffffu, mbar_wait(&misc->slot_free[s], par ^ 1u, abort_flag, err, ERR_TIMEOUT)))
+          break;
         if (!__all_sync(0xffffffffu, mbar_wait(&misc->a_full[s], par, abort_flag, err, ERR_TIMEOUT))) break;
         const unsigned char* src = smem + Lay::OFF_SA + s * Lay::SA_SLOT;
         const float sg = __half2float(reinterpret_cast<const __half*>(src + C * R)[t]);
@@ -1047,7 +1054,7 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
       // conversion comes after this epilogue) and whose pre-activations are done; row t,
       // 16-byte chunk j at j ^ (t % 16) (R = 128: 128 rows of 256 bytes; R = 64 reads the
       // row from global memory in the passes below)
-      constexpr bool kVStage = Lay::A_BYTES >= C * kEncD * 2;
+      constexpr bool kVStage = kVStageI8;
       unsigned char* vst = smem + Lay::OFF_A + s * Lay::A_BYTES + (kVStage ? t * kEncD * 2 : 0);
       if (EMIT && I8 && kVStage && flagged) {
         uint4 tmp[kEncD / 8];

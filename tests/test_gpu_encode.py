@@ -195,6 +195,9 @@ ENC_CASES = [
     ("llama8b_32k_bf16", dict(batch=1, n_layers=4, n_kv_heads=2, n_ctx=512, chunk=64)),  # r 128, C 64
     ("llama8b_32k_bf16", dict(batch=2, n_layers=4, n_kv_heads=2, n_ctx=768, group=2)),   # G 2: two bases resident
     ("llama8b_32k_bf16", dict(batch=1, n_layers=8, n_kv_heads=1, n_ctx=512, group=8)),   # G 8: the one-tile form
+    # 512 tiles over the 148 persistent CTAs: each tile group takes a second tile into the stage
+    # its first one used
+    ("llama8b_32k_bf16", dict(batch=2, n_layers=4, n_kv_heads=2, n_ctx=4096)),
 ]
 
 
@@ -203,6 +206,18 @@ ENC_CASES = [
 def test_encode_matches_oracle(name, kw, store):
     cfg = S.CONFIGS[name].replace(name="enc_" + name, store=store, evict_frac=0.0, **kw)
     n_res = cfg.n_resid
+    g, o, og = _encode_both(cfg, n_res)
+    _check_encode(cfg, g, o, og, n_res, norms_gpu=_gpu_norms(g, cfg))
+
+
+@pytest.mark.parametrize("n_res", [64, 128])
+def test_encode_int8_records_with_sparse_flags(n_res):
+    """int8 records from the tensor-core passes (r = C = 128) when few tokens are flagged: most
+    warps of a tile then have no flagged token and finish its records long before the others,
+    while the tile group's next tile (several per CTA here) is converted into the stage where
+    the others' values rows sit."""
+    cfg = S.CONFIGS["llama8b_32k_bf16"].replace(name="enc_sparse", store="int8", evict_frac=0.0, batch=2,
+                                                n_layers=4, n_kv_heads=2, n_ctx=4096)
     g, o, og = _encode_both(cfg, n_res)
     _check_encode(cfg, g, o, og, n_res, norms_gpu=_gpu_norms(g, cfg))
 
