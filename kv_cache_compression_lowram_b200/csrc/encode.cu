@@ -74,8 +74,8 @@ __device__ __forceinline__ void quantize8(const float* x, float amax, __half* sc
   *scale_out = sh;
 }
 
-// The same encoding of 8 values of a row whose fp16 scale s (> 0 or 0) and reciprocal r are
-// known: round-half-even of x / s from a first guess rint(x r), corrected by the exact
+// The same encoding for a row whose fp16 scale s (> 0 or 0) and reciprocal r are known:
+// round-half-even of x / s from a first guess rint(x r), corrected by the exact
 // remainder x - q s (an fma: q s has at most 19 significant bits and lies within s of x, so
 // the remainder is representable), a tie going to even.  One division per row instead of
 // one per value; the result is the rounding of the exact quotient.
@@ -90,18 +90,14 @@ __device__ __forceinline__ float rne_quot(float x, float s, float r) {
 }
 // (x r is within 2^-22 relative of x / s, i.e. within 4e-5 for |x / s| <= 127.5, so its
 // nearest integer is the answer unless x r lies within 1e-4 of a half-integer; only then is
-// the exact remainder consulted.)
-__device__ __forceinline__ uint2 quantize8_scaled(const float* x, float s, float r) {
-  uint32_t w[2] = {0u, 0u};
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const float y = x[j] * r;
-    float q = rintf(y);
-    if (fabsf(y - q) > 0.4999f) q = rne_quot(x[j], s, r);
-    q = s > 0.f ? fminf(fmaxf(q, -127.f), 127.f) : 0.f;
-    w[j >> 2] |= ((uint32_t)(int)q & 0xffu) << (8 * (j & 3));
-  }
-  return make_uint2(w[0], w[1]);
+// the exact remainder consulted.)  The code of one value of a row with scale s and r = 1 / s
+// (0 when s = 0), clamped to [-127, 127].
+__device__ __forceinline__ uint32_t code8_scaled(float x, float s, float r) {
+  const float y = x * r;
+  float q = rintf(y);
+  if (fabsf(y - q) > 0.4999f) q = rne_quot(x, s, r);
+  q = s > 0.f ? fminf(fmaxf(q, -127.f), 127.f) : 0.f;
+  return (uint32_t)(int)q & 0xffu;
 }
 
 // --------------------------------------------------------------------- coefficients
@@ -960,7 +956,6 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
     const int t = 32 * wq + lane;                      // this thread's token (TMEM lane)
     const uint32_t lane_off = (uint32_t)(32 * wq) << 16;
     const unsigned lt_mask = (1u << lane) - 1u;
-    constexpr bool kVStageI8 = I8 && Lay::A_BYTES >= C * kEncD * 2;   // values rows staged (R = 128)
     for (long long i = grp_t; i < n; i += 2) {
       const long long x = x0 + i;
       const int s = (int)(i & 1);
@@ -969,20 +964,18 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
       const int b = u % B, seg = u / B, hkv = seg % Hkv, l = seg / Hkv;
       const size_t unit = ((size_t)b * L + l) * Hkv + hkv;
       const size_t tok = unit * N + (size_t)c * C;   // the chunk's first token
-      int flagged = 0, rank = 0;
+      int flagged = 0, rank = 0, rank0 = 0;   // rank0: flagged tokens of the earlier warps
+      unsigned fb = 0;                        // this warp's flagged lanes
       size_t rbase = 0;
       if (EMIT) {   // the token's rank among the chunk's flagged tokens: one ballot per warp
-        unsigned below = 0;
 #pragma unroll
         for (int w4 = 0; w4 < 4; ++w4) {
           const unsigned bw = __ballot_sync(0xffffffffu, flags[tok + 32 * w4 + lane] != 0);
-          if (w4 < wq) below += __popc(bw);
-          if (w4 == wq) {
-            flagged = (bw >> lane) & 1u;
-            below += __popc(bw & lt_mask);
-          }
+          if (w4 < wq) rank0 += __popc(bw);
+          if (w4 == wq) fb = bw;
         }
-        rank = (int)below;
+        flagged = (fb >> lane) & 1u;
+        rank = rank0 + __popc(fb & lt_mask);
         rbase = (size_t)res_ptr[unit * (nC + 1) + c];
       }
       // the token's values row for the epilogue (pass 2: flagged tokens only), requested now;
@@ -995,10 +988,10 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
         for (int j = 0; j < kEncD / 8; ++j) vrow[j] = (!EMIT || flagged) ? __ldg(vp + j) : make_uint4(0, 0, 0, 0);
       }
       if (I8) {   // this token's stored row, sigma_t a_t as fp16, into the coefficient stage
-        // pass 2 stages the flagged tokens' values rows in this stage (below), and a warp's
-        // rows there overlap other warps' coefficient rows: the group's previous tile must be
-        // done by all four warps (their slot_free arrivals) before any of them overwrites it
-        if (EMIT && kVStageI8 && i >= 2 &&
+        // pass 2 stages the flagged tokens' rows in this stage (below), and a warp's slots
+        // there overlap other warps' coefficient rows (r = 128): the group's previous tile must
+        // be done by all four warps (their slot_free arrivals) before any of them overwrites it
+        if (EMIT && i >= 2 &&
             !__all_sync(0xffffffffu, mbar_wait(&misc->slot_free[s], par ^ 1u, abort_flag, err, ERR_TIMEOUT)))
           break;
         if (!__all_sync(0xffffffffu, mbar_wait(&misc->a_full[s], par, abort_flag, err, ERR_TIMEOUT))) break;
@@ -1049,63 +1042,90 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&misc->h_ready[s]);
-      // int8 record: a flagged token's values row goes to shared memory while the second GEMM
-      // runs -- into this tile's coefficient stage, which only this group writes (its next
-      // conversion comes after this epilogue) and whose pre-activations are done; row t,
-      // 16-byte chunk j at j ^ (t % 16) (R = 128: 128 rows of 256 bytes; R = 64 reads the
-      // row from global memory in the passes below)
-      constexpr bool kVStage = kVStageI8;
-      unsigned char* vst = smem + Lay::OFF_A + s * Lay::A_BYTES + (kVStage ? t * kEncD * 2 : 0);
-      if (EMIT && I8 && kVStage && flagged) {
-        uint4 tmp[kEncD / 8];
+      // int8 record (pass 2): each warp quantises its flagged tokens' rows together, four
+      // dims per lane, instead of each row by its own lane.  The warp's quarter of this tile's
+      // coefficient stage (free: the pre-activations are done, and the group's next conversion
+      // waits for this tile's slot_free) holds kNSlot row slots of 512 bytes; the flagged token
+      // of warp rank m < kNSlot copies its values row (bf16) into the upper half of slot m now,
+      // while the second GEMM runs, 16-byte piece j at (16 + j) ^ (m % 8).
+      constexpr int kQB = Lay::A_BYTES / 4, kNSlot = kQB / 512;
+      unsigned char* wbase = smem + Lay::OFF_A + s * Lay::A_BYTES + wq * kQB;
+      const int wrank = __popc(fb & lt_mask), kw = __popc(fb);
+      auto stage_v = [&](int m) {
+        unsigned char* slot = wbase + m * 512;
 #pragma unroll
-        for (int j = 0; j < kEncD / 8; ++j) tmp[j] = __ldg(vp + j);
-#pragma unroll
-        for (int j = 0; j < kEncD / 8; ++j) *reinterpret_cast<uint4*>(vst + ((j ^ (t & 15)) << 4)) = tmp[j];
+        for (int j = 0; j < kEncD / 8; ++j)
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(slot + (((16 + j) ^ (m & 7)) << 4))),
+                       "l"(vp + j)
+                       : "memory");
+        asm volatile("cp.async.commit_group;" ::: "memory");
+      };
+      if (EMIT && I8 && flagged && wrank < kNSlot) stage_v(wrank);
+      if (!__all_sync(0xffffffffu, mbar_wait(&misc->d2_full[s], par, abort_flag, err, ERR_TIMEOUT))) {
+        if (EMIT && I8) asm volatile("cp.async.wait_all;" ::: "memory");   // no copy outlives the CTA
+        break;
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(&misc->d2_full[s], par, abort_flag, err, ERR_TIMEOUT))) break;
       tc_fence_after();
       // delta = V - Vhat for this token's 128 dims: its norm (pass 1) or its record (pass 2)
       float ss = 0.f;
       if constexpr (EMIT && I8) {
-        // the int8 record: a pass over the row for its scale, a second for its codes (64 dims
-        // per TMEM round trip, delta recomputed, so that the row never sits in registers whole)
-        float dmax = 0.f, sc = 0.f, rc = 0.f;
-        __half sh = __ushort_as_half((unsigned short)0);
-#pragma unroll 1
-        for (int pass = 0; pass < 2; ++pass)
+        // per batch of up to kNSlot flagged tokens: each writes its delta row (fp32) into its
+        // slot, 16-byte piece p (dims 4p .. 4p + 3) at p ^ (m % 8) -- over the values row as it
+        // is consumed (dims 32q .. 32q + 31 land on pieces 8q .. 8q + 7, which hold values of
+        // dims below 32q only); then the warp takes the slots one by one: lane L the dims
+        // 4L .. 4L + 3, the row's largest |delta| by a butterfly, its fp16 scale s, the codes
+        // round-half-even of delta / s (code8_scaled), 128 bytes stored at once
+        for (int b0 = 0; b0 < kw; b0 += kNSlot) {
+          const bool mine = flagged && wrank >= b0 && wrank < b0 + kNSlot;
+          const int m = wrank - b0;
+          if (b0 > 0 && mine) stage_v(m);   // later batches (more than kNSlot flagged lanes)
+          asm volatile("cp.async.wait_all;" ::: "memory");
+          unsigned char* slot = wbase + (mine ? m : 0) * 512;
 #pragma unroll 1
           for (int q = 0; q < kEncD / 32; ++q) {
-            uint32_t vh[32];   // (the load is warp-wide; only flagged lanes use it)
+            uint32_t vh[32];   // (warp-wide load; only this batch's lanes use it)
             tmem_ld32(tmem + lane_off + 256 * s + 128 + 32 * q, vh);
             tmem_wait_ld();
-            if (!flagged) continue;
+            if (!mine) continue;
+            uint4 w4[4];   // values dims 32q .. 32q + 31, read before any delta of them is written
+#pragma unroll
+            for (int k8 = 0; k8 < 4; ++k8)
+              w4[k8] = *reinterpret_cast<const uint4*>(slot + (((16 + 4 * q + k8) ^ (m & 7)) << 4));
 #pragma unroll
             for (int k8 = 0; k8 < 4; ++k8) {
-              const int j = 4 * q + k8;   // 16-byte chunk of the values row
-              const uint4 w4 = kVStage ? *reinterpret_cast<const uint4*>(vst + ((j ^ (t & 15)) << 4)) : __ldg(vp + j);
-              const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
+              const uint32_t ww[4] = {w4[k8].x, w4[k8].y, w4[k8].z, w4[k8].w};
               float x8[8];
 #pragma unroll
               for (int h = 0; h < 4; ++h) {
                 x8[2 * h] = __uint_as_float(ww[h] << 16) - __uint_as_float(vh[8 * k8 + 2 * h]);
                 x8[2 * h + 1] = __uint_as_float(ww[h] & 0xffff0000u) - __uint_as_float(vh[8 * k8 + 2 * h + 1]);
               }
-              if (pass == 0) {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) dmax = fmaxf(dmax, fabsf(x8[k]));
-              } else {
-                *reinterpret_cast<uint2*>(static_cast<int8_t*>(res_val) + (rbase + rank) * kEncD + 32 * q + 8 * k8) =
-                    quantize8_scaled(x8, sc, rc);
-              }
-            }
-            if (pass == 0 && q == kEncD / 32 - 1) {   // the row's scale, once its max is known
-              sh = __float2half_rn(dmax / 127.f);
-              sc = __half2float(sh);
-              rc = sc > 0.f ? 1.f / sc : 0.f;
+              const int p0 = 8 * q + 2 * k8;   // pieces p0, p0 + 1
+              *reinterpret_cast<float4*>(slot + ((p0 ^ (m & 7)) << 4)) = make_float4(x8[0], x8[1], x8[2], x8[3]);
+              *reinterpret_cast<float4*>(slot + (((p0 + 1) ^ (m & 7)) << 4)) =
+                  make_float4(x8[4], x8[5], x8[6], x8[7]);
             }
           }
-        if (flagged) res_scale[rbase + rank] = sh;
+          __syncwarp();   // the batch's delta rows are visible to the whole warp
+          const int nb = min(kNSlot, kw - b0);
+#pragma unroll 1
+          for (int mm = 0; mm < nb; ++mm) {
+            const float4 xv = *reinterpret_cast<const float4*>(wbase + mm * 512 + ((lane ^ (mm & 7)) << 4));
+            const float x4[4] = {xv.x, xv.y, xv.z, xv.w};
+            float amax = fmaxf(fmaxf(fabsf(x4[0]), fabsf(x4[1])), fmaxf(fabsf(x4[2]), fabsf(x4[3])));
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            const __half sh = __float2half_rn(amax / 127.f);
+            const float sc = __half2float(sh), rc = sc > 0.f ? 1.f / sc : 0.f;
+            uint32_t code = 0u;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) code |= code8_scaled(x4[k], sc, rc) << (8 * k);
+            const size_t rec = rbase + (size_t)(rank0 + b0 + mm);
+            *reinterpret_cast<uint32_t*>(static_cast<int8_t*>(res_val) + rec * kEncD + 4 * lane) = code;
+            if (lane == 0) res_scale[rec] = sh;
+          }
+          __syncwarp();   // every slot read before the next batch overwrites it
+        }
       } else {
         uint32_t vd[kEncD];   // the token's rebuilt row, all of it in one TMEM round trip
 #pragma unroll
