@@ -381,6 +381,8 @@ class LowramReuse:
 
     def decode(self, q, out=None, sel: bool = False, layer0: int = 0, n_layers: Optional[int] = None, stream=None):
         import torch
+        if not getattr(self.cache, "handle", 0):   # the library would follow a freed cache
+            raise LowramError(1, "LowramReuse.decode", "the store's cache was closed")
         if n_layers is None:
             n_layers = int(q.shape[0])
         if out is None:

@@ -173,3 +173,14 @@ def test_reuse_host_checks():
     stride = ctypes.c_int64()
     assert lib.lowram_reuse_view(None, ctypes.byref(t), ctypes.byref(o), ctypes.byref(e), ctypes.byref(stride)) == 1
     lib.lowram_reuse_destroy(None)
+
+
+def test_reuse_wrapper_refuses_a_closed_cache():
+    """A store whose cache was closed is refused before the library follows the freed cache."""
+    from types import SimpleNamespace
+
+    store = K.LowramReuse.__new__(K.LowramReuse)
+    store.cache, store.capacity, store.handle = SimpleNamespace(cfg=None, handle=0), 16, 0
+    with pytest.raises(K.LowramError) as ei:
+        store.decode(None)
+    assert ei.value.status == 1
