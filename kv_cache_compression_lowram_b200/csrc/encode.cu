@@ -734,7 +734,8 @@ enc_resid_tc_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant__
 // ------------------------------------------- tensor-core residuals, C = 128, tokens as M
 // The same pass with the chunk's 128 tokens as the MMAs' M dimension, so that every
 // per-token step of the epilogue (the token's values row against its rebuilt row, the norm
-// of the difference, the record) is local to one thread:
+// of the difference, a bf16 record) is local to one thread (an int8 record's scale and codes
+// are computed by the token's warp together, four dims per lane):
 //   D1^T = A . (W1'/2)^T (SS, M = 128 tokens, N = 128 per hidden half, K = R)
 //   H^T  = silu(2 D1^T) as fp16 pairs, written over the first 128 of the tile's TMEM columns
 //          (thread = token: its 256 hidden units)
@@ -979,8 +980,8 @@ enc_resid_tc2_kernel(int B, int L, int G, int Hkv, int N, const __grid_constant_
         rbase = (size_t)res_ptr[unit * (nC + 1) + c];
       }
       // the token's values row for the epilogue (pass 2: flagged tokens only), requested now;
-      // for an int8 record once the silu is done, so that it does not sit in registers
-      // through the conversion and the silu
+      // for an int8 record copied into shared memory once the silu is done (below), so that
+      // it does not sit in registers through the conversion and the silu
       uint4 vrow[kEncD / 8];
       const uint4* vp = reinterpret_cast<const uint4*>(values + (tok + t) * kEncD);
       if (!(EMIT && I8)) {
